@@ -1,0 +1,356 @@
+/*
+ * e4b oracle: a plain, slow, obviously-correct CPU statement of the NF4
+ * Mixture-of-Experts expert path.  TEST INFRASTRUCTURE ONLY: the tests, the
+ * package smoke check and the CPU-baseline leg of the benchmark call it; the
+ * product path never does.  It shares no code, header, table or helper with the
+ * CUDA library.
+ *
+ * Sources (cited by page title and section):
+ *   [P4]  "experts4bit-qlora 0.1.0" source diff, file _vendor/experts.py,
+ *         class Experts4bit (__init__, from_float, _quantize_stack,
+ *         _dequantize_expert, forward).
+ *   [P5]  bitsandbytes pull request #1965 "Add Experts4bit for 4-bit
+ *         quantization of fused MoE experts", sections "What this adds" and
+ *         "Correctness & coverage".
+ *   [P1]  "experts4bit-qlora" 0.4.0 package description, section "Storage
+ *         modes: the support matrix".
+ *   [QLoRA] Dettmers et al. 2023, "QLoRA", appendix on the NormalFloat data
+ *         type (the 16 NF4 values; the pages only call get_4bit_type("nf4")).
+ *
+ * Precision.  Quantize takes its decisions in fp32 (the pages quantize fp32
+ * weights with fp32 absmax); dequantize multiplies in fp32 and rounds once to
+ * bf16 (round-to-nearest-even); routing weights, forward and input gradient
+ * are computed in fp64.  Readings where the pages are silent:
+ *   - codes are chosen by strict comparison with the fp32 midpoints of the
+ *     sorted codebook, so an exact tie goes to the smaller value;
+ *   - an all-zero block stores absmax 0 and the zero code;
+ *   - the FP4 codebook is OCP e2m1 {0,.5,1,1.5,2,3,4,6}/6 with the sign in
+ *     bit 3 (parity with bitsandbytes' own fp4 table is unpinned);
+ *   - routing selects top-k on the fp32 logits (descending, ties to the lower
+ *     expert index), weights are softmax over all experts, optionally divided
+ *     by their sum over the selected k.
+ * Build: gcc -O2 -fopenmp -ffp-contract=off -shared -fPIC (no fast-math).
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+#define ORC_OK 0
+#define ORC_ERR_ARG 1
+#define ORC_ERR_BLOCKSIZE 2
+
+/* ---- codebooks ---------------------------------------------------------- */
+
+/* NF4: the 16 NormalFloat values of [QLoRA], ascending, index 7 is zero.  The
+ * code of a value is its index. */
+static const float kNF4[16] = {
+    -1.0f, -0.6961928009986877f, -0.5250730514526367f, -0.39491748809814453f,
+    -0.28444138169288635f, -0.18477343022823334f, -0.09105003625154495f, 0.0f,
+    0.07958029955625534f, 0.16093020141124725f, 0.24611230194568634f,
+    0.33791524171829224f, 0.44070982933044434f, 0.5626170039176941f,
+    0.7229568362236023f, 1.0f};
+
+/* FP4 (e2m1, max-normalised): value of a 4-bit code = sign(bit 3) * e2m1(bits
+ * 2..0) / 6.  e2m1 magnitudes: 0, 0.5, 1, 1.5, 2, 3, 4, 6. */
+static float fp4_value(int code) {
+    static const double mag[8] = {0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0};
+    float m = (float)(mag[code & 7] / 6.0);
+    return (code & 8) ? -m : m;
+}
+
+/* Value of code q (0..15) under codebook cb (0 = NF4, 1 = FP4). */
+float e4bo_code_value(int cb, int q) {
+    if (cb == 0) return kNF4[q & 15];
+    return fp4_value(q & 15);
+}
+
+/* The 15 distinct codebook values in ascending order and the code of each.
+ * NF4: 16 distinct values, the code is the index.  FP4: -0 is dropped (it is
+ * never produced), so 15 values remain. */
+static int sorted_codebook(int cb, float *vals, int *codes) {
+    if (cb == 0) {
+        for (int i = 0; i < 16; ++i) { vals[i] = kNF4[i]; codes[i] = i; }
+        return 16;
+    }
+    int n = 0;
+    for (int m = 7; m >= 1; --m) { vals[n] = fp4_value(8 | m); codes[n] = 8 | m; ++n; }
+    vals[n] = 0.0f; codes[n] = 0; ++n;
+    for (int m = 1; m <= 7; ++m) { vals[n] = fp4_value(m); codes[n] = m; ++n; }
+    return n;
+}
+
+/* Copy the 16 code values (indexed by code) for a test to inspect. */
+void e4bo_codebook(int cb, float *out16) {
+    for (int q = 0; q < 16; ++q) out16[q] = e4bo_code_value(cb, q);
+}
+
+/* ---- bf16 round-to-nearest-even from the IEEE bit definition ------------- */
+
+uint16_t e4bo_f32_to_bf16(float f) {
+    uint32_t u;
+    memcpy(&u, &f, 4);
+    if ((u & 0x7f800000u) == 0x7f800000u) {           /* inf / nan */
+        if (u & 0x007fffffu) return (uint16_t)((u >> 16) | 0x40u); /* quiet nan */
+        return (uint16_t)(u >> 16);
+    }
+    uint32_t upper = u >> 16, lower = u & 0xffffu;
+    if (lower > 0x8000u || (lower == 0x8000u && (upper & 1u))) upper += 1u;
+    return (uint16_t)upper;
+}
+
+float e4bo_bf16_to_f32(uint16_t h) {
+    uint32_t u = (uint32_t)h << 16;
+    float f;
+    memcpy(&f, &u, 4);
+    return f;
+}
+
+/* ---- quantize ([P4] _quantize_stack; [P5] "What this adds") -------------- */
+
+/* w: fp32 [E, out, in] row-major.  packed: [E, out*in/2] bytes, element 2b in
+ * the high nibble of byte b.  absmax: [E, out*in/blocksize], block j of row o
+ * at o*in/blocksize + j.  in % blocksize must be 0 ([P4] __init__ raises
+ * otherwise).  Only blocksize 64 is part of the contract. */
+int e4bo_quantize(const float *w, int64_t E, int64_t out, int64_t in, int blocksize,
+                  int cb, uint8_t *packed, float *absmax) {
+    if (!w || !packed || !absmax || E < 0 || out < 0 || in < 0) return ORC_ERR_ARG;
+    if (cb != 0 && cb != 1) return ORC_ERR_ARG;
+    if (blocksize != 64) return ORC_ERR_BLOCKSIZE;
+    if (in % blocksize != 0) return ORC_ERR_BLOCKSIZE;
+    float vals[16];
+    int codes[16];
+    int nv = sorted_codebook(cb, vals, codes);
+    float mid[15];
+    for (int i = 0; i + 1 < nv; ++i) mid[i] = (vals[i] + vals[i + 1]) * 0.5f;
+    const int zero_code = (cb == 0) ? 7 : 0;
+    const int64_t nblocks = E * out * in / blocksize;
+#pragma omp parallel for schedule(static)
+    for (int64_t b = 0; b < nblocks; ++b) {
+        const float *src = w + b * blocksize;
+        float a = 0.0f;
+        for (int i = 0; i < blocksize; ++i) {
+            float m = fabsf(src[i]);
+            if (m > a) a = m;
+        }
+        absmax[b] = a;
+        uint8_t *dst = packed + b * (blocksize / 2);
+        for (int i = 0; i < blocksize; i += 2) {
+            int q[2];
+            for (int t = 0; t < 2; ++t) {
+                if (a == 0.0f) { q[t] = zero_code; continue; }
+                float n = src[i + t] / a;   /* IEEE fp32 division, correctly rounded */
+                int r = 0;
+                for (int m = 0; m < nv - 1; ++m) r += (mid[m] < n) ? 1 : 0;
+                q[t] = codes[r];
+            }
+            dst[i / 2] = (uint8_t)((q[0] << 4) | q[1]);
+        }
+    }
+    return ORC_OK;
+}
+
+/* ---- dequantize ([P4] _dequantize_expert) -------------------------------- */
+
+/* fp32 value of element i: code value * absmax, one fp32 rounding. */
+static inline float deq_one(const uint8_t *packed, const float *absmax, int64_t i,
+                            int blocksize, int cb) {
+    uint8_t byte = packed[i >> 1];
+    int q = (i & 1) ? (byte & 15) : (byte >> 4);
+    return e4bo_code_value(cb, q) * absmax[i / blocksize];
+}
+
+int e4bo_dequantize_f32(const uint8_t *packed, const float *absmax, int64_t n,
+                        int blocksize, int cb, float *out) {
+    if (!packed || !absmax || !out || n < 0 || n % blocksize) return ORC_ERR_ARG;
+#pragma omp parallel for schedule(static)
+    for (int64_t i = 0; i < n; ++i) out[i] = deq_one(packed, absmax, i, blocksize, cb);
+    return ORC_OK;
+}
+
+int e4bo_dequantize_bf16(const uint8_t *packed, const float *absmax, int64_t n,
+                         int blocksize, int cb, uint16_t *out) {
+    if (!packed || !absmax || !out || n < 0 || n % blocksize) return ORC_ERR_ARG;
+#pragma omp parallel for schedule(static)
+    for (int64_t i = 0; i < n; ++i)
+        out[i] = e4bo_f32_to_bf16(deq_one(packed, absmax, i, blocksize, cb));
+    return ORC_OK;
+}
+
+/* ---- routing ------------------------------------------------------------- */
+
+/* logits fp32 [T, E] -> idx [T, k] (descending logit, ties to lower index) and
+ * weights [T, k] = softmax over all E at the chosen experts, optionally divided
+ * by their sum over the k. */
+int e4bo_route(const float *logits, int64_t T, int E, int k, int renorm,
+               int32_t *idx, double *wts) {
+    if (!logits || !idx || !wts || T < 0 || E <= 0 || k <= 0 || k > E) return ORC_ERR_ARG;
+#pragma omp parallel for schedule(static)
+    for (int64_t t = 0; t < T; ++t) {
+        const float *l = logits + t * E;
+        int32_t *o = idx + t * k;
+        for (int j = 0; j < k; ++j) {
+            int best = -1;
+            for (int e = 0; e < E; ++e) {
+                int taken = 0;
+                for (int jj = 0; jj < j; ++jj) taken |= (o[jj] == e);
+                if (taken) continue;
+                if (best < 0 || l[e] > l[best]) best = e;   /* strict: ties keep lower index */
+            }
+            o[j] = best;
+        }
+        double mx = (double)l[o[0]];
+        double z = 0.0;
+        for (int e = 0; e < E; ++e) z += exp((double)l[e] - mx);
+        double s = 0.0;
+        for (int j = 0; j < k; ++j) {
+            wts[t * k + j] = exp((double)l[o[j]] - mx) / z;
+            s += wts[t * k + j];
+        }
+        if (renorm)
+            for (int j = 0; j < k; ++j) wts[t * k + j] /= s;
+    }
+    return ORC_OK;
+}
+
+/* ---- grouping ([P4] forward: expert mask, hit list, token gather) --------- */
+
+/* Stable counting sort of the pair ids p = t*k + j by expert: rows of expert e
+ * are [offsets[e], offsets[e+1]) and hold pair ids in ascending order. */
+int e4bo_permute(const int32_t *idx, int64_t T, int k, int E, int32_t *counts,
+                 int32_t *offsets, int32_t *perm) {
+    if (!idx || !counts || !offsets || !perm || T < 0 || k <= 0 || E <= 0) return ORC_ERR_ARG;
+    int64_t P = T * k;
+    for (int e = 0; e < E; ++e) counts[e] = 0;
+    for (int64_t p = 0; p < P; ++p) {
+        if (idx[p] < 0 || idx[p] >= E) return ORC_ERR_ARG;
+        counts[idx[p]]++;
+    }
+    offsets[0] = 0;
+    for (int e = 0; e < E; ++e) offsets[e + 1] = offsets[e] + counts[e];
+    int32_t *fill = (int32_t *)malloc(sizeof(int32_t) * (size_t)E);
+    if (!fill) return ORC_ERR_ARG;
+    for (int e = 0; e < E; ++e) fill[e] = offsets[e];
+    for (int64_t p = 0; p < P; ++p) perm[fill[idx[p]]++] = (int32_t)p;
+    free(fill);
+    return ORC_OK;
+}
+
+/* ---- forward ([P4] Experts4bit.forward) ---------------------------------- */
+
+static double silu(double g) { return g / (1.0 + exp(-g)); }
+
+/* For each token t in tokens[0..nt) (all tokens when tokens == NULL) and each
+ * slot j with expert e = idx[t,j]:
+ *   g = x_t W_gate,e^T,  u = x_t W_up,e^T   (W_gate = rows [0,I), W_up = rows
+ *   [I,2I) of gate_up, i.e. proj.chunk(2) with gate first),
+ *   h = silu(g) * u,
+ *   y_t += w_{t,j} * h W_down,e^T,  summed over j in slot order.
+ * x: [T,H] fp64, wgu: [E,2I,H] fp32 (dequantized), wd: [E,H,I] fp32,
+ * y: [nt,H] fp64 (row i belongs to tokens[i]). */
+int e4bo_forward(const double *x, int64_t T, int E, int H, int I, int k,
+                 const int32_t *idx, const double *wts, const float *wgu,
+                 const float *wd, const int64_t *tokens, int64_t nt, double *y) {
+    if (!x || !idx || !wts || !wgu || !wd || !y || T < 0 || E <= 0 || k <= 0) return ORC_ERR_ARG;
+    if (!tokens) nt = T;
+#pragma omp parallel
+    {
+        double *h = (double *)malloc(sizeof(double) * (size_t)I);
+#pragma omp for schedule(dynamic, 1)
+        for (int64_t i = 0; i < nt; ++i) {
+            int64_t t = tokens ? tokens[i] : i;
+            const double *xt = x + t * H;
+            double *yt = y + i * H;
+            for (int c = 0; c < H; ++c) yt[c] = 0.0;
+            for (int j = 0; j < k; ++j) {
+                int e = idx[t * k + j];
+                const float *Wg = wgu + (int64_t)e * 2 * I * H;
+                const float *Wu = Wg + (int64_t)I * H;
+                const float *Wd = wd + (int64_t)e * H * I;
+                for (int r = 0; r < I; ++r) {
+                    double g = 0.0, u = 0.0;
+                    for (int c = 0; c < H; ++c) {
+                        g += xt[c] * (double)Wg[(int64_t)r * H + c];
+                        u += xt[c] * (double)Wu[(int64_t)r * H + c];
+                    }
+                    h[r] = silu(g) * u;
+                }
+                double w = wts[t * k + j];
+                for (int c = 0; c < H; ++c) {
+                    double acc = 0.0;
+                    for (int r = 0; r < I; ++r) acc += h[r] * (double)Wd[(int64_t)c * I + r];
+                    yt[c] += w * acc;
+                }
+            }
+        }
+        free(h);
+    }
+    return ORC_OK;
+}
+
+/* ---- input gradient ([P5] "What this adds": recompute-in-backward) -------- */
+
+/* grad_x_t = sum_j dx_{t,j}, routing held constant:
+ *   dY   = w_{t,j} * grad_out_t
+ *   dh   = dY W_down,e                    (contract over H)
+ *   dG   = dh * u * s(g) * (1 + g (1 - s(g)))   with s the logistic function
+ *   dU   = dh * silu(g)
+ *   dx   = dG W_gate,e + dU W_up,e        (contract over 2I)
+ * with g, u recomputed from x and the dequantized weights (never saved). */
+int e4bo_dgrad(const double *x, const double *gout, int64_t T, int E, int H, int I, int k,
+               const int32_t *idx, const double *wts, const float *wgu, const float *wd,
+               const int64_t *tokens, int64_t nt, double *gx) {
+    if (!x || !gout || !idx || !wts || !wgu || !wd || !gx || T < 0 || E <= 0 || k <= 0) return ORC_ERR_ARG;
+    if (!tokens) nt = T;
+#pragma omp parallel
+    {
+        double *dG = (double *)malloc(sizeof(double) * (size_t)I);
+        double *dU = (double *)malloc(sizeof(double) * (size_t)I);
+#pragma omp for schedule(dynamic, 1)
+        for (int64_t i = 0; i < nt; ++i) {
+            int64_t t = tokens ? tokens[i] : i;
+            const double *xt = x + t * H;
+            const double *go = gout + t * H;
+            double *gt = gx + i * H;
+            for (int c = 0; c < H; ++c) gt[c] = 0.0;
+            for (int j = 0; j < k; ++j) {
+                int e = idx[t * k + j];
+                const float *Wg = wgu + (int64_t)e * 2 * I * H;
+                const float *Wu = Wg + (int64_t)I * H;
+                const float *Wd = wd + (int64_t)e * H * I;
+                double w = wts[t * k + j];
+                for (int r = 0; r < I; ++r) {
+                    double g = 0.0, u = 0.0, dh = 0.0;
+                    for (int c = 0; c < H; ++c) {
+                        g += xt[c] * (double)Wg[(int64_t)r * H + c];
+                        u += xt[c] * (double)Wu[(int64_t)r * H + c];
+                        dh += w * go[c] * (double)Wd[(int64_t)c * I + r];
+                    }
+                    double s = 1.0 / (1.0 + exp(-g));
+                    dG[r] = dh * u * s * (1.0 + g * (1.0 - s));
+                    dU[r] = dh * g * s;
+                }
+                for (int c = 0; c < H; ++c) {
+                    double acc = 0.0;
+                    for (int r = 0; r < I; ++r)
+                        acc += dG[r] * (double)Wg[(int64_t)r * H + c] + dU[r] * (double)Wu[(int64_t)r * H + c];
+                    gt[c] += acc;
+                }
+            }
+        }
+        free(dG);
+        free(dU);
+    }
+    return ORC_OK;
+}
+
+int e4bo_num_threads(void) {
+#ifdef _OPENMP
+    return omp_get_max_threads();
+#else
+    return 1;
+#endif
+}

@@ -1,0 +1,352 @@
+"""Pins for the CPU oracle: each test checks the oracle against something other
+than itself -- a published construction, a closed form, an invariant the pages
+state, a library routine, brute force, or finite differences.  CPU only."""
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from bit_quantized_mixture_nf4_b200 import workloads as wl
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden", "fidelity_bounds.txt")
+
+
+def golden():
+    out = {}
+    for line in open(GOLDEN):
+        line = line.strip()
+        if not line or line.startswith("#"):
+            continue
+        k, v = line.split()[:2]
+        out[k] = float(v)
+    return out
+
+
+# ---------------------------------------------------------------- codebooks
+
+def test_nf4_codebook_matches_normalfloat_construction():
+    """NF4 = quantiles of N(0,1) (QLoRA's NormalFloat): 8 positive values from
+    ppf(linspace(d, 1/2, 9)[:-1]), 7 negative from -ppf(linspace(d, 1/2, 8)[:-1]),
+    zero, normalised by the maximum; d = (1 - 1/30 + 1 - 1/32) / 2."""
+    from scipy.stats import norm
+    d = 0.5 * ((1 - 1 / 30) + (1 - 1 / 32))
+    pos = norm.ppf(np.linspace(d, 0.5, 9)[:-1])
+    neg = -norm.ppf(np.linspace(d, 0.5, 8)[:-1])
+    v = np.sort(np.concatenate([pos, [0.0], neg]))
+    v = v / v.max()
+    c = oracle.codebook(oracle.NF4).astype(np.float64)
+    assert np.all(np.diff(c) > 0)
+    assert c[0] == -1.0 and c[7] == 0.0 and c[15] == 1.0
+    np.testing.assert_allclose(c, v, atol=5e-7, rtol=0)
+
+
+def test_fp4_codebook_is_e2m1_over_six():
+    c = oracle.codebook(oracle.FP4).astype(np.float64)
+    mags = np.array([0, 0.5, 1, 1.5, 2, 3, 4, 6]) / 6.0
+    np.testing.assert_allclose(c[:8], mags, rtol=1e-7)
+    np.testing.assert_allclose(c[8:], -mags, rtol=1e-7)
+    assert np.signbit(c[8])   # code 0b1000 is -0 (never produced by quantize)
+
+
+# ----------------------------------------------------------- bf16 rounding
+
+def test_bf16_rounding_matches_torch():
+    rng = np.random.default_rng(0)
+    v = np.concatenate([
+        rng.standard_normal(20000).astype(np.float32) * 10.0 ** rng.integers(-30, 30, 20000),
+        # exact ties: low half exactly 0x8000 with even and odd upper halves
+        (np.arange(2000, dtype=np.uint32) << 16 | 0x8000).view(np.float32),
+        np.array([0.0, -0.0, np.inf, -np.inf, 3.4e38, 1e-45, -1e-45], np.float32),
+    ]).astype(np.float32)
+    v = v[np.isfinite(v) | np.isinf(v)]
+    ours = oracle.f32_to_bf16_bits(v)
+    ref = torch.from_numpy(v).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    assert np.array_equal(ours, ref)
+
+
+# ------------------------------------------------------ quantize / dequantize
+
+def _blocks(n_blocks, scale=0.02, seed=0):
+    rng = np.random.default_rng(seed)
+    s = scale * np.exp(rng.uniform(-3, 3, (n_blocks, 1)))
+    return (rng.standard_normal((n_blocks, 64)) * s).astype(np.float32)
+
+
+@pytest.mark.parametrize("cb,half_gap", [(oracle.NF4, (1.0 - 0.6961928009986877) / 2), (oracle.FP4, 1.0 / 6.0)])
+def test_roundtrip_error_bound(cb, half_gap):
+    """|w - deq| <= absmax * (largest codebook gap)/2 per element (plus fp32 rounding)."""
+    w = _blocks(4096, seed=1).reshape(8, 512, 64)
+    packed, absmax = oracle.quantize(w, cb)
+    deq = oracle.dequantize(packed, absmax, w.shape, cb, "f32")
+    a = absmax.reshape(8, 512, 1)
+    err = np.abs(w.astype(np.float64) - deq.astype(np.float64))
+    bound = a * half_gap * (1 + 1e-6) + np.abs(w) * 2.0 ** -23
+    assert np.all(err <= bound)
+    # bf16 output adds at most half a bf16 ulp of the value
+    deq16 = oracle.dequantize(packed, absmax, w.shape, cb, "bf16")
+    assert np.all(np.abs(deq16 - deq) <= np.abs(deq) * 2.0 ** -8)
+
+
+@pytest.mark.parametrize("cb", [oracle.NF4, oracle.FP4])
+def test_exact_reproduction_of_codebook_values_and_zeros(cb):
+    c = oracle.codebook(cb)
+    codes = list(range(16)) if cb == oracle.NF4 else [q for q in range(16) if q != 8]
+    rng = np.random.default_rng(2)
+    for a in (1.0, 0.02, 3.7e-3, 117.0):
+        a = np.float32(a)
+        vals = np.array([np.float32(c[q]) * a for q in codes], np.float32)
+        block = np.zeros(64, np.float32)
+        pos = rng.permutation(64)[: len(vals)]
+        block[pos] = vals
+        packed, absmax = oracle.quantize(block.reshape(1, 1, 64), cb)
+        assert absmax[0, 0] == a
+        deq = oracle.dequantize(packed, absmax, (1, 1, 64), cb, "f32").ravel()
+        assert np.array_equal(deq[pos], vals)
+        zero_code = 7 if cb == oracle.NF4 else 0
+        nib = np.stack([packed[0] >> 4, packed[0] & 15], 1).ravel()
+        assert np.array_equal(nib[pos], np.array(codes))
+        rest = np.setdiff1d(np.arange(64), pos)
+        assert np.all(nib[rest] == zero_code)
+        assert np.all(deq[rest] == 0) and not np.any(np.signbit(deq[rest]))
+
+
+@pytest.mark.parametrize("cb", [oracle.NF4, oracle.FP4])
+def test_all_zero_block(cb):
+    packed, absmax = oracle.quantize(np.zeros((2, 3, 64), np.float32), cb)
+    zero_byte = 0x77 if cb == oracle.NF4 else 0x00
+    assert np.all(packed == zero_byte) and np.all(absmax == 0)
+    assert np.all(oracle.dequantize(packed, absmax, (2, 3, 64), cb, "f32") == 0)
+
+
+def test_nibble_order_first_element_high():
+    """The first element of each pair goes to the high nibble."""
+    block = np.zeros((1, 1, 64), np.float32)
+    block[0, 0, 0] = 1.0      # +absmax -> NF4 code 15
+    block[0, 0, 3] = -1.0     # -absmax -> NF4 code 0
+    packed, absmax = oracle.quantize(block, oracle.NF4)
+    assert packed[0, 0] == 0xF7 and packed[0, 1] == 0x70
+
+
+@pytest.mark.parametrize("cb", [oracle.NF4, oracle.FP4])
+def test_idempotent(cb):
+    w = _blocks(2048, seed=3).reshape(4, 256, 128)
+    packed, absmax = oracle.quantize(w, cb)
+    deq = oracle.dequantize(packed, absmax, w.shape, cb, "f32")
+    p2, a2 = oracle.quantize(deq, cb)
+    assert np.array_equal(a2, absmax)
+    assert np.array_equal(p2, packed)
+
+
+@pytest.mark.parametrize("cb", [oracle.NF4, oracle.FP4])
+def test_tie_goes_to_smaller_value(cb):
+    c = oracle.codebook(cb)
+    vals = np.unique(c[[q for q in range(16) if not (cb == oracle.FP4 and q == 8)]])
+    mids = ((vals[:-1] + vals[1:]) * np.float32(0.5)).astype(np.float32)
+    block = np.zeros(64, np.float32)
+    block[0] = 1.0
+    block[1:1 + len(mids)] = mids
+    packed, absmax = oracle.quantize(block.reshape(1, 1, 64), cb)
+    deq = oracle.dequantize(packed, absmax, (1, 1, 64), cb, "f32").ravel()
+    assert np.array_equal(deq[1:1 + len(mids)], vals[:-1])
+
+
+def test_blocksize_validation():
+    """in_features must be a multiple of the block size (64)."""
+    with pytest.raises(oracle.OracleError) as ei:
+        oracle.quantize(np.zeros((1, 2, 96), np.float32))
+    assert ei.value.code == 2
+    with pytest.raises(oracle.OracleError):
+        oracle.quantize(np.zeros((1, 2, 64), np.float32), blocksize=32)
+
+
+def test_error_ordering_nf4_below_fp4():
+    """NF4 reconstructs ~Gaussian weights better than FP4."""
+    rng = np.random.default_rng(4)
+    w = (rng.standard_normal((4, 1024, 64)) * 0.02).astype(np.float32)
+    errs = {}
+    for cb in (oracle.NF4, oracle.FP4):
+        p, a = oracle.quantize(w, cb)
+        d = oracle.dequantize(p, a, w.shape, cb, "f32")
+        errs[cb] = np.sqrt(np.mean((d - w) ** 2) / np.mean(w ** 2))
+    assert errs[oracle.NF4] < errs[oracle.FP4]
+
+
+def test_nf4_dequant_mean_abs_error_bound():
+    g = golden()
+    rng = np.random.default_rng(5)
+    w = (rng.standard_normal((2, 512, 256)) * 0.02).astype(np.float32)
+    p, a = oracle.quantize(w)
+    d = oracle.dequantize(p, a, w.shape, oracle.NF4, "bf16")
+    assert np.mean(np.abs(d - w)) <= g["nf4_dequant_mean_abs_bound"]
+
+
+# -------------------------------------------------------------- routing
+
+def _logits(T, E, seed):
+    rng = np.random.default_rng(seed)
+    l = rng.standard_normal((T, E)).astype(np.float32)
+    l[::7, 3] = l[::7, 5]           # exact ties between experts 3 and 5
+    return l
+
+
+@pytest.mark.parametrize("E,k,renorm", [(8, 2, True), (64, 8, False), (128, 8, True), (32, 4, True)])
+def test_route_brute_force(E, k, renorm):
+    T = 97
+    l = _logits(T, E, E + k)
+    idx, w = oracle.route(l, k, renorm)
+    for t in range(T):
+        order = np.lexsort((np.arange(E), -l[t].astype(np.float64)))   # logit desc, index asc
+        assert np.array_equal(idx[t], order[:k])
+        ld = l[t].astype(np.float64)
+        z = np.exp(ld - ld.max()).sum()
+        sel = ld[idx[t]]
+        # softmax ratios are exp of logit differences
+        np.testing.assert_allclose(w[t] / w[t][0], np.exp(sel - sel[0]), rtol=1e-12)
+        if renorm:
+            assert abs(w[t].sum() - 1.0) < 1e-12
+        else:
+            np.testing.assert_allclose(w[t][0], 1.0 / z, rtol=1e-12)
+
+
+def test_permute_invariants():
+    T, E, k = 300, 16, 4
+    l = _logits(T, E, 7)
+    idx, _ = oracle.route(l, k, True)
+    counts, offsets, perm = oracle.permute(idx, E)
+    flat = idx.ravel()
+    assert np.array_equal(counts, np.bincount(flat, minlength=E))
+    assert offsets[0] == 0 and offsets[-1] == T * k and np.all(np.diff(offsets) >= 0)
+    assert np.array_equal(np.sort(perm), np.arange(T * k))
+    for e in range(E):
+        seg = perm[offsets[e]:offsets[e + 1]]
+        assert np.all(flat[seg] == e)
+        assert np.all(np.diff(seg) > 0)          # ascending pair id == ascending token
+
+
+# -------------------------------------------------------------- forward
+
+def _tiny_problem(E=4, H=64, I=64, T=8, k=2, seed=9, renorm=True):
+    rng = np.random.default_rng(seed)
+    x = torch.from_numpy(rng.standard_normal((T, H)).astype(np.float32)).to(torch.bfloat16).float().numpy()
+    gu = (rng.standard_normal((E, 2 * I, H)) * 0.05).astype(np.float32)
+    dn = (rng.standard_normal((E, H, I)) * 0.05).astype(np.float32)
+    pg, ag = oracle.quantize(gu)
+    pd, ad = oracle.quantize(dn)
+    wgu = oracle.dequantize(pg, ag, gu.shape)
+    wd = oracle.dequantize(pd, ad, dn.shape)
+    l = rng.standard_normal((T, E)).astype(np.float32)
+    idx, w = oracle.route(l, k, renorm)
+    return x, idx, w, wgu, wd, gu, dn
+
+
+def _dense_reference(x, idx, w, wgu, wd):
+    """Every expert on every token in fp64 (einsum), then masked by routing."""
+    E, I2, H = wgu.shape
+    I = I2 // 2
+    xd = x.astype(np.float64)
+    G = np.einsum("th,eih->eti", xd, wgu[:, :I].astype(np.float64))
+    U = np.einsum("th,eih->eti", xd, wgu[:, I:].astype(np.float64))
+    Hh = G / (1 + np.exp(-G)) * U
+    Y = np.einsum("eti,ehi->eth", Hh, wd.astype(np.float64))
+    T = x.shape[0]
+    gate = np.zeros((E, T))
+    for t in range(T):
+        for j in range(idx.shape[1]):
+            gate[idx[t, j], t] += w[t, j]
+    return np.einsum("et,eth->th", gate, Y)
+
+
+def test_forward_matches_dense_fp64_reference():
+    x, idx, w, wgu, wd, *_ = _tiny_problem(E=6, H=128, I=64, T=24, k=3)
+    y = oracle.forward(x, idx, w, wgu, wd)
+    ref = _dense_reference(x, idx, w, wgu, wd)
+    np.testing.assert_allclose(y, ref, rtol=1e-10, atol=1e-12 * np.abs(ref).max())
+    # same-weights tolerance on the pages is 1e-4; fp64 is far inside it
+    assert np.abs(y - ref).max() <= golden()["forward_same_weights_tolerance"] * np.abs(ref).max()
+    sub = np.array([5, 0, 17])
+    np.testing.assert_array_equal(oracle.forward(x, idx, w, wgu, wd, tokens=sub), y[sub])
+
+
+def test_forward_single_expert_is_dense_swiglu_mlp():
+    x, _, _, wgu, wd, *_ = _tiny_problem(E=1, H=64, I=128, T=5, k=1)
+    idx = np.zeros((5, 1), np.int32)
+    w = np.ones((5, 1))
+    y = oracle.forward(x, idx, w, wgu, wd)
+    xt = torch.from_numpy(x).double()
+    g = xt @ torch.from_numpy(wgu[0, :128]).double().t()
+    u = xt @ torch.from_numpy(wgu[0, 128:]).double().t()
+    ref = (torch.nn.functional.silu(g) * u) @ torch.from_numpy(wd[0]).double().t()
+    np.testing.assert_allclose(y, ref.numpy(), rtol=1e-10, atol=1e-13)
+
+
+@pytest.mark.parametrize("cb,key", [(oracle.NF4, "nf4_forward_relerr_cap"), (oracle.FP4, "fp4_forward_relerr_cap")])
+def test_forward_relerr_vs_true_weights_within_page_caps(cb, key):
+    """Forward with quantized weights vs the true fp32 weights stays under the
+    per-scheme ceilings the pages print, and NF4 < FP4."""
+    g = golden()
+    rng = np.random.default_rng(11)
+    E, H, I, T, k = 8, 256, 512, 64, 2
+    x = torch.from_numpy(rng.standard_normal((T, H)).astype(np.float32)).to(torch.bfloat16).float().numpy()
+    gu = (rng.standard_normal((E, 2 * I, H)) * 0.02).astype(np.float32)
+    dn = (rng.standard_normal((E, H, I)) * 0.02).astype(np.float32)
+    idx, w = oracle.route(rng.standard_normal((T, E)).astype(np.float32), k, True)
+    ref = oracle.forward(x, idx, w, gu, dn)
+    errs = {}
+    for c in (oracle.NF4, oracle.FP4):
+        pg, ag = oracle.quantize(gu, c)
+        pd, ad = oracle.quantize(dn, c)
+        y = oracle.forward(x, idx, w, oracle.dequantize(pg, ag, gu.shape, c), oracle.dequantize(pd, ad, dn.shape, c))
+        errs[c] = np.linalg.norm(y - ref) / np.linalg.norm(ref)
+    assert errs[cb] <= g[key]
+    assert errs[oracle.NF4] <= g["nf4_forward_relerr_true_weights_bound"]
+    assert errs[oracle.NF4] < errs[oracle.FP4]
+
+
+# -------------------------------------------------------------- dgrad
+
+def test_dgrad_matches_central_finite_differences():
+    x, idx, w, wgu, wd, *_ = _tiny_problem(E=4, H=64, I=64, T=8, k=2)
+    rng = np.random.default_rng(12)
+    go = rng.standard_normal(x.shape)
+    gx = oracle.dgrad(x, go, idx, w, wgu, wd)
+    eps = 1e-6
+    num = np.zeros_like(gx)
+    for t in range(x.shape[0]):
+        for c in range(x.shape[1]):
+            xp = x.astype(np.float64).copy()
+            xm = xp.copy()
+            xp[t, c] += eps
+            xm[t, c] -= eps
+            fp = (oracle.forward(xp, idx, w, wgu, wd, tokens=[t]) * go[t]).sum()
+            fm = (oracle.forward(xm, idx, w, wgu, wd, tokens=[t]) * go[t]).sum()
+            num[t, c] = (fp - fm) / (2 * eps)
+    np.testing.assert_allclose(gx, num, rtol=1e-6, atol=1e-6 * np.abs(num).max())
+
+
+def test_dgrad_adjoint_identity():
+    """<grad_out, J v> = <dgrad(grad_out), v> with J v by a central difference."""
+    x, idx, w, wgu, wd, *_ = _tiny_problem(E=5, H=128, I=64, T=16, k=3, seed=13)
+    rng = np.random.default_rng(14)
+    go = rng.standard_normal(x.shape)
+    v = rng.standard_normal(x.shape)
+    eps = 1e-5
+    xd = x.astype(np.float64)
+    jv = (oracle.forward(xd + eps * v, idx, w, wgu, wd) - oracle.forward(xd - eps * v, idx, w, wgu, wd)) / (2 * eps)
+    lhs = np.sum(go * jv)
+    rhs = np.sum(oracle.dgrad(x, go, idx, w, wgu, wd) * v)
+    assert abs(lhs - rhs) <= 1e-7 * abs(rhs) + 1e-9
+
+
+# ------------------------------------------------------ seeded workloads
+
+def test_zipf_router_hot_set():
+    """The Qwen3-shaped router bias puts about half the selections on ~6% of experts."""
+    w = wl.QWEN3
+    x = wl.activations(w)
+    l = wl.router_logits(w, x).numpy()
+    idx, _ = oracle.route(l, w.k, w.renorm)
+    c = np.sort(np.bincount(idx.ravel(), minlength=w.E))[::-1]
+    share = c[:8].sum() / c.sum()
+    assert 0.35 < share < 0.65
