@@ -1,0 +1,394 @@
+#!/usr/bin/env python
+"""Benchmark of the NF4 Mixture-of-Experts expert layer: forward + input
+gradient (recompute-in-backward) on the OLMoE-1B-7B-shaped layer (E=64, H=2048,
+I=1024, top-8 without renormalisation, T=4096 tokens per GPU), NF4 weights with
+blocksize-64 fp32 absmax, synthetic seeded inputs.
+
+One step = route (softmax/top-k from fp32 logits) + group + grouped gate_up GEMM
+with SwiGLU + grouped down GEMM with the weighted combine + dgrad (two grouped
+GEMMs with the weights re-dequantized in-kernel), all through the C ABI.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl e4b|reference]
+
+Prints one JSON line (rank 0).  Multi-GPU: one process per GPU under torchrun,
+each GPU runs its own batch (data parallel, no collective on the data path),
+value = tokens of all ranks / max-over-ranks device time.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "routed tokens/s, NF4 MoE layer fwd+dgrad"
+UNIT = "tokens/s"
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="e4b", choices=["e4b", "reference"])
+    ap.add_argument("--tokens", type=int, default=4096)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    return ap.parse_args()
+
+
+def dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        d = json.load(open(path))
+        return d["hbm_gbs"], d["bf16_tflops"], d.get("bf16_tflops_sustained"), "measured"
+    return 6650.0, 1590.0, 1400.0, "fallback"
+
+
+def kernel_source_hash():
+    h = hashlib.sha256()
+    for f in ("grouped_gemm.cu", "e4b_device.cuh", "e4b_internal.h"):
+        h.update(open(os.path.join(ROOT, "bit_quantized_mixture_nf4_b200", "csrc", f), "rb").read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(kernel: str, workload: str):
+    """DRAM bytes per launch from the committed ncu summary, if taken on the current kernel source."""
+    path = os.path.join(ROOT, "profiles", "dram_traffic.txt")
+    if not os.path.exists(path):
+        return None
+    src = kernel_source_hash()
+    for line in open(path):
+        f = line.split()
+        if len(f) >= 4 and not line.startswith("#") and f[0] == kernel and f[1] == workload and f[3] == src:
+            return float(f[2])
+    return None
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled while the timed region runs."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
+         "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+         "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.idx = gpu_index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.idx), f"--query-gpu={self.Q}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *a):
+        self.out = ""
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.out, _ = self.proc.communicate(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self):
+        rows = []
+        for line in (self.out or "").splitlines():
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                rows.append(dict(sm=float(f[1]), smax=float(f[2]), power=float(f[3]), hw=f[5], hwt=f[6], swt=f[7],
+                                 swp=f[8]))
+            except ValueError:
+                continue
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        loaded = [r for r in rows if r["power"] > 200] or rows
+        reasons = set()
+        for r in rows:
+            for key, name in (("hw", "hw_slowdown"), ("hwt", "hw_thermal_slowdown"), ("swt", "sw_thermal_slowdown"),
+                              ("swp", "sw_power_cap")):
+                if r[key].lower() == "active":
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(r["sm"] for r in loaded), "sm_max_mhz": max(r["smax"] for r in rows),
+                "reasons": sorted(reasons), "samples": len(rows)}
+
+
+# ------------------------------------------------------------------ CPU oracle
+
+def oracle_step(w, x, logits, go, packed, sample_tokens, dequant_cache):
+    """One oracle pass: route + group all tokens, dequantize the experts (from the
+    packed bytes), forward + input gradient of the sampled tokens.  Returns
+    (seconds for the whole-batch fixed part, seconds for the sampled tokens)."""
+    import numpy as np
+    import oracle
+    t0 = time.perf_counter()
+    idx, wts = oracle.route(logits, w.k, w.renorm)
+    oracle.permute(idx, w.E)
+    pg, ag, pd, ad = packed
+    wgu = oracle.dequantize(pg, ag, (w.E, 2 * w.I, w.H), w.codebook)
+    wd = oracle.dequantize(pd, ad, (w.E, w.H, w.I), w.codebook)
+    t1 = time.perf_counter()
+    toks = np.asarray(sample_tokens, np.int64)
+    oracle.forward(x, idx, wts, wgu, wd, tokens=toks)
+    oracle.dgrad(x, go, idx, wts, wgu, wd, tokens=toks)
+    t2 = time.perf_counter()
+    return t1 - t0, t2 - t1
+
+
+def oracle_inputs(w):
+    import oracle
+    from bit_quantized_mixture_nf4_b200 import workloads as wl
+    x = wl.activations(w)
+    gu, dn = wl.weights(w)
+    logits = wl.router_logits(w, x).numpy()
+    go = wl.grad_output(w).float().numpy()
+    packed = oracle.quantize(gu.numpy(), w.codebook) + oracle.quantize(dn.numpy(), w.codebook)
+    return x.float().numpy(), logits, go, packed
+
+
+def cpu_rate(w, target_s=12.0, inputs=None):
+    """Oracle throughput in routed tokens/s on a bounded sample, scaled to a full batch."""
+    import numpy as np
+    import oracle
+    x, logits, go, packed = inputs if inputs is not None else oracle_inputs(w)
+    nth = oracle.num_threads()
+    rng = np.random.default_rng(0)
+    cal = rng.choice(w.T, size=min(w.T, nth), replace=False)
+    fixed, tcal = oracle_step(w, x, logits, go, packed, cal, None)
+    per_tok = tcal / len(cal)
+    S = int(max(len(cal), min(w.T, (target_s - fixed) / max(per_tok, 1e-9))))
+    S = max(nth, (S // nth) * nth)
+    toks = rng.choice(w.T, size=min(S, w.T), replace=False)
+    fixed, ttok = oracle_step(w, x, logits, go, packed, toks, None)
+    step = fixed + ttok * w.T / len(toks)
+    return w.T / step, dict(cores=nth, sample=f"{len(toks)} of {w.T} tokens (fwd+dgrad), whole-batch routing, "
+                                               f"grouping and dequantization; step time extrapolated linearly in "
+                                               f"tokens", fixed_s=fixed, sample_s=ttok)
+
+
+def run_reference(args, w):
+    world, rank, _ = dist_env()
+    if rank != 0:
+        return
+    inputs = oracle_inputs(w)
+    import numpy as np
+    import oracle
+    nth = oracle.num_threads()
+    rng = np.random.default_rng(1)
+    S = max(nth, 2 * nth)
+    toks = rng.choice(w.T, size=min(S, w.T), replace=False)
+    for _ in range(args.warmup):
+        oracle_step(w, *inputs, toks, None)
+    steps = []
+    for _ in range(args.steps):
+        fixed, ttok = oracle_step(w, *inputs, toks, None)
+        steps.append(fixed + ttok * w.T / len(toks))
+    step = statistics.median(steps)
+    value = w.T / step
+    sample = (f"{len(toks)} of {w.T} tokens per step (fwd+dgrad), whole-batch routing, grouping and "
+              f"dequantization; step time extrapolated linearly in tokens")
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": step * 1e3, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": f"olmoe-shaped E={w.E} H={w.H} I={w.I} top{w.k} T={w.T} nf4 fwd+dgrad",
+                       "global_batch": w.T * world, "l2": "n/a (CPU)"},
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": nth, "kind": "oracle", "sample": sample},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# ------------------------------------------------------------------ GPU arm
+
+def run_e4b(args, w):
+    import torch
+    import bit_quantized_mixture_nf4_b200 as e4b
+    from bit_quantized_mixture_nf4_b200 import workloads as wl
+
+    world, rank, local = dist_env()
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+
+    # inputs: activations / logits / grad_out drawn on the host (seeded), weights on the device
+    x_h = wl.activations(w)
+    logits_h = wl.router_logits(w, x_h)
+    go_h = wl.grad_output(w)
+    gu, dn = wl.weights(w, device=dev)
+    pg, ag = e4b.e4b_quantize_nf4(gu, codebook=w.codebook)
+    pd, ad = e4b.e4b_quantize_nf4(dn, codebook=w.codebook)
+    del gu, dn
+    torch.cuda.empty_cache()
+    experts = e4b.make_experts(pg, pd, ag, ad)
+    desc = e4b.make_desc(w.E, w.H, w.I, w.k, w.renorm, w.codebook, 64, e4b.PATH_AUTO)
+    T, P = w.T, w.P
+    x = x_h.to(dev)
+    logits = logits_h.to(dev)
+    go = go_h.to(dev)
+    idx = torch.empty(T, w.k, dtype=torch.int32, device=dev)
+    wts = torch.empty(T, w.k, dtype=torch.float32, device=dev)
+    y = torch.empty(T, w.H, dtype=torch.bfloat16, device=dev)
+    gx = torch.empty(T, w.H, dtype=torch.bfloat16, device=dev)
+    saved = torch.empty(P, 2 * w.I, dtype=torch.bfloat16, device=dev)
+    ws = e4b.workspace(desc, T, dev)
+    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)   # > 126 MB L2
+    stream = torch.cuda.current_stream()
+
+    def step():
+        e4b.e4b_moe_forward(desc, experts, x, logits, idx, wts, y, saved_gu=saved, ws=ws, stream=stream)
+        e4b.e4b_moe_backward_dgrad(desc, experts, x, idx, wts, go, saved_gu=saved, grad_x=gx, ws=ws, stream=stream)
+
+    for _ in range(max(args.warmup, 3)):
+        step()
+    torch.cuda.synchronize()
+    if e4b.e4b_device_status() != e4b.E4B_OK:
+        raise RuntimeError("device status not ok after warm-up")
+
+    # ------------------------------------------------ device-timed region
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    e4b.e4b_timing_reset()
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    launches0 = e4b.e4b_launch_count()
+    with ClockSampler(local) as clk:
+        e4b.e4b_timing_enable(True)
+        for i in range(args.steps):
+            flush.zero_()                       # evict L2 between timed steps (not timed)
+            starts[i].record(stream)
+            step()
+            ends[i].record(stream)
+        torch.cuda.synchronize()
+        e4b.e4b_timing_enable(False)
+    launches = e4b.e4b_launch_count() - launches0
+    if world > 1:
+        torch.distributed.barrier()
+    step_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
+    total_ms = sum(step_ms)
+    if world > 1:
+        t = torch.tensor([total_ms], device=dev, dtype=torch.float64)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        total_ms = float(t.item())
+    ms_per_step = total_ms / args.steps
+    value = world * T / (ms_per_step / 1e3)
+
+    kernels = {}
+    for name in ("gemm_gateup", "gemm_down", "gemm_dgrad_down", "gemm_dgrad_gateup", "route", "group", "gather",
+                 "convert"):
+        ms, n = e4b.e4b_timing_get(name)
+        if n:
+            kernels[name] = {"launches": n, "avg_ms": ms / n}
+    flops = {"gemm_gateup": 4, "gemm_down": 2, "gemm_dgrad_down": 2, "gemm_dgrad_gateup": 4}
+    dom = max((k for k in flops if k in kernels), key=lambda k: kernels[k]["avg_ms"] * kernels[k]["launches"])
+    hbm, bf16_burst, bf16_sus, peak_src = peaks()
+    dom_flops = flops[dom] * w.H * w.I * P
+    achieved = dom_flops / (kernels[dom]["avg_ms"] / 1e3) / 1e12
+    wl_name = f"olmoe_T{T}"
+    traffic = recorded_traffic(dom, wl_name)
+
+    # ------------------------------------------------ end-to-end through host buffers
+    e2e = None
+    if not args.no_e2e:
+        x_p = x_h.pin_memory()
+        l_p = logits_h.pin_memory()
+        g_p = go_h.pin_memory()
+        y_p = torch.empty(T, w.H, dtype=torch.bfloat16).pin_memory()
+        gx_p = torch.empty(T, w.H, dtype=torch.bfloat16).pin_memory()
+
+        def e2e_step():
+            x.copy_(x_p, non_blocking=True)
+            logits.copy_(l_p, non_blocking=True)
+            go.copy_(g_p, non_blocking=True)
+            step()
+            y_p.copy_(y, non_blocking=True)
+            gx_p.copy_(gx, non_blocking=True)
+
+        for _ in range(2):
+            e2e_step()
+        torch.cuda.synchronize()
+        if world > 1:
+            torch.distributed.barrier()
+        es, ee = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        es.record(stream)
+        for _ in range(args.steps):
+            e2e_step()
+        ee.record(stream)
+        torch.cuda.synchronize()
+        e2e_ms = es.elapsed_time(ee) / args.steps
+        if world > 1:
+            t = torch.tensor([e2e_ms], device=dev, dtype=torch.float64)
+            torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+            e2e_ms = float(t.item())
+        h2d = x_p.numel() * 2 + l_p.numel() * 4 + g_p.numel() * 2
+        d2h = y_p.numel() * 2 + gx_p.numel() * 2
+        e2e = {"value": world * T / (e2e_ms / 1e3), "unit": UNIT, "h2d_bytes_per_step": h2d,
+               "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms}
+
+    if e4b.e4b_device_status() != e4b.E4B_OK:
+        raise RuntimeError("device status not ok after the timed region")
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        rate, info = cpu_rate(w)
+        cpu = {"value": rate, "unit": UNIT, "cores": info["cores"], "kind": "oracle", "sample": info["sample"]}
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": max(args.warmup, 3), "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": f"olmoe-shaped E={w.E} H={w.H} I={w.I} top{w.k} no-renorm T={T}/GPU, nf4 "
+                                   f"blocksize 64, fwd (routed from logits, g/u saved) + dgrad",
+                       "global_batch": T * world, "parallelism": f"dp{world} (independent batches)",
+                       "l2": "flushed between timed steps (256 MB write)", "routed_pairs_per_gpu": P},
+            "roofline": {"kernel": dom, "bound": "tensor", "achieved": achieved, "peak": bf16_burst,
+                         "unit": "TFLOP/s", "frac": achieved / bf16_burst, "traffic": traffic,
+                         "peak_kind": f"{peak_src} bf16 dense (burst)",
+                         "flops_per_launch": dom_flops, "avg_launch_ms": kernels[dom]["avg_ms"]},
+            "kernels": kernels,
+            "clocks": clk.summary(),
+            "gpu_launches": launches,
+            "e2e": e2e,
+            "cpu_baseline": cpu,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        torch.distributed.barrier()
+        torch.distributed.destroy_process_group()
+
+
+def main():
+    args = parse()
+    from bit_quantized_mixture_nf4_b200 import workloads as wl
+    w = wl.OLMOE.with_tokens(args.tokens)
+    if args.impl == "reference":
+        run_reference(args, w)
+    else:
+        run_e4b(args, w)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,232 @@
+"""e4b: NF4 / FP4 quantized Mixture-of-Experts expert kernels for NVIDIA B200.
+
+A thin ctypes binding over ``libe4b.so`` (the C ABI in ``include/e4b.h``).  The
+functions keep the C names and only marshal arguments: PyTorch tensors supply
+device memory and the current CUDA stream; every step of the computation runs
+in the library's sm_100a kernels.  There is no CPU fallback: the first call
+fails loudly when the library is missing, and a compute call without a CUDA
+device raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libe4b.so")
+
+E4B_OK, E4B_ERR_INVALID_ARG, E4B_ERR_BLOCKSIZE, E4B_ERR_UNSUPPORTED, E4B_ERR_WORKSPACE, E4B_ERR_CUDA, \
+    E4B_ERR_TIMEOUT = range(7)
+NF4, FP4 = 0, 1
+F32, BF16 = 0, 1
+PATH_AUTO, PATH_GROUPED, PATH_DECODE = 0, 1, 2
+
+EXPORTS = ("e4b_quantize_nf4", "e4b_dequantize_nf4", "e4b_moe_workspace_size", "e4b_moe_forward",
+           "e4b_moe_backward_dgrad", "e4b_device_status", "e4b_status_string", "e4b_launch_count",
+           "e4b_timing_enable", "e4b_timing_reset", "e4b_timing_get")
+# kernel kinds of e4b_timing_get
+KERNEL_KINDS = ("quantize", "dequantize", "route", "group", "gather", "convert", "gemm_gateup", "gemm_down",
+                "gemm_dgrad_down", "gemm_dgrad_gateup", "decode_gateup", "decode_down")
+
+
+class e4b_moe_desc(ctypes.Structure):
+    _fields_ = [("E", ctypes.c_int), ("H", ctypes.c_int), ("I", ctypes.c_int), ("top_k", ctypes.c_int),
+                ("renormalize", ctypes.c_int), ("codebook", ctypes.c_int), ("blocksize", ctypes.c_int),
+                ("path", ctypes.c_int)]
+
+
+class e4b_experts(ctypes.Structure):
+    _fields_ = [("gate_up", ctypes.c_void_p), ("down", ctypes.c_void_p), ("gate_up_absmax", ctypes.c_void_p),
+                ("down_absmax", ctypes.c_void_p)]
+
+
+class E4BError(RuntimeError):
+    def __init__(self, fn: str, status: int, msg: str):
+        super().__init__(f"{fn}: {msg} (status {status})")
+        self.status = status
+
+
+_lib = None
+
+
+def _load():
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"libe4b.so not built at {LIB_PATH}; run python -m bit_quantized_mixture_nf4_b200.build")
+    lib = ctypes.CDLL(LIB_PATH)
+    P, i64, i32, sz = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_size_t
+    lib.e4b_quantize_nf4.argtypes = [P, i64, i64, i64, i32, i32, P, P, P]
+    lib.e4b_dequantize_nf4.argtypes = [P, P, i64, i64, i64, i32, i32, i32, P, P]
+    lib.e4b_moe_workspace_size.argtypes = [ctypes.POINTER(e4b_moe_desc), i64]
+    lib.e4b_moe_workspace_size.restype = sz
+    lib.e4b_moe_forward.argtypes = [ctypes.POINTER(e4b_moe_desc), ctypes.POINTER(e4b_experts), P, i64, P, P, P, P,
+                                    P, P, P, P, sz, P]
+    lib.e4b_moe_backward_dgrad.argtypes = [ctypes.POINTER(e4b_moe_desc), ctypes.POINTER(e4b_experts), P, i64, P, P,
+                                           P, P, P, P, sz, P]
+    lib.e4b_device_status.argtypes = [P]
+    lib.e4b_status_string.argtypes = [i32]
+    lib.e4b_status_string.restype = ctypes.c_char_p
+    lib.e4b_launch_count.restype = ctypes.c_uint64
+    lib.e4b_timing_enable.argtypes = [i32]
+    lib.e4b_timing_enable.restype = None
+    lib.e4b_timing_reset.restype = None
+    lib.e4b_timing_get.argtypes = [i32, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_uint64)]
+    lib.e4b_timing_get.restype = ctypes.c_int
+    for f in ("e4b_quantize_nf4", "e4b_dequantize_nf4", "e4b_moe_forward", "e4b_moe_backward_dgrad",
+              "e4b_device_status"):
+        getattr(lib, f).restype = ctypes.c_int
+    _lib = lib
+    return lib
+
+
+def __getattr__(name):
+    if name == "lib":
+        return _load()
+    raise AttributeError(name)
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _check(fn: str, status: int):
+    if status != E4B_OK:
+        raise E4BError(fn, status, _load().e4b_status_string(status).decode())
+
+
+def _cuda(t: torch.Tensor, name: str, dtype=None):
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor (no CPU path)")
+    if dtype is not None and t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    return t
+
+
+def e4b_status_string(status: int) -> str:
+    return _load().e4b_status_string(status).decode()
+
+
+def e4b_launch_count() -> int:
+    return int(_load().e4b_launch_count())
+
+
+def e4b_timing_enable(on: bool = True):
+    _load().e4b_timing_enable(int(bool(on)))
+
+
+def e4b_timing_reset():
+    _load().e4b_timing_reset()
+
+
+def e4b_timing_get(kind) -> tuple:
+    """(total device ms, timed launches) of one kernel kind (index or name in KERNEL_KINDS)."""
+    if isinstance(kind, str):
+        kind = KERNEL_KINDS.index(kind)
+    ms, n = ctypes.c_double(), ctypes.c_uint64()
+    _check("e4b_timing_get", _load().e4b_timing_get(kind, ctypes.byref(ms), ctypes.byref(n)))
+    return ms.value, int(n.value)
+
+
+def e4b_device_status(stream=None) -> int:
+    return int(_load().e4b_device_status(_stream(stream)))
+
+
+def e4b_quantize_nf4(w: torch.Tensor, blocksize: int = 64, codebook: int = NF4, packed=None, absmax=None,
+                     stream=None):
+    """w: fp32 [E, out, in] on the GPU -> (packed uint8 [E, out*in/2], absmax fp32 [E, out*in/64])."""
+    _cuda(w, "w", torch.float32)
+    if w.dim() != 3:
+        raise ValueError("w must be a 3-D [E, out, in] stack")
+    E, o, i = w.shape
+    if packed is None:
+        packed = torch.empty(E, o * i // 2, dtype=torch.uint8, device=w.device)
+    if absmax is None:
+        absmax = torch.empty(E, o * i // max(blocksize, 1), dtype=torch.float32, device=w.device)
+    _check("e4b_quantize_nf4", _load().e4b_quantize_nf4(_ptr(w), E, o, i, blocksize, codebook, _ptr(packed), _ptr(absmax),
+                                                    _stream(stream)))
+    return packed, absmax
+
+
+def e4b_dequantize_nf4(packed: torch.Tensor, absmax: torch.Tensor, shape, blocksize: int = 64, codebook: int = NF4,
+                       out_dtype: int = BF16, out=None, stream=None):
+    """Packed + absmax -> [E, out, in] bf16 (out_dtype=BF16) or fp32 (F32)."""
+    _cuda(packed, "packed", torch.uint8)
+    _cuda(absmax, "absmax", torch.float32)
+    E, o, i = shape
+    if out is None:
+        out = torch.empty(E, o, i, dtype=torch.bfloat16 if out_dtype == BF16 else torch.float32, device=packed.device)
+    _check("e4b_dequantize_nf4", _load().e4b_dequantize_nf4(_ptr(packed), _ptr(absmax), E, o, i, blocksize, codebook,
+                                                        out_dtype, _ptr(out), _stream(stream)))
+    return out
+
+
+def make_desc(E, H, I, top_k, renormalize=True, codebook=NF4, blocksize=64, path=PATH_AUTO) -> e4b_moe_desc:
+    return e4b_moe_desc(E, H, I, top_k, int(bool(renormalize)), codebook, blocksize, path)
+
+
+def make_experts(gate_up, down, gate_up_absmax, down_absmax) -> e4b_experts:
+    for n, t in (("gate_up", gate_up), ("down", down)):
+        _cuda(t, n, torch.uint8)
+    for n, t in (("gate_up_absmax", gate_up_absmax), ("down_absmax", down_absmax)):
+        _cuda(t, n, torch.float32)
+    return e4b_experts(gate_up.data_ptr(), down.data_ptr(), gate_up_absmax.data_ptr(), down_absmax.data_ptr())
+
+
+def e4b_moe_workspace_size(desc: e4b_moe_desc, T: int) -> int:
+    return int(_load().e4b_moe_workspace_size(ctypes.byref(desc), T))
+
+
+def workspace(desc: e4b_moe_desc, T: int, device="cuda") -> torch.Tensor:
+    return torch.empty(max(e4b_moe_workspace_size(desc, T), 1), dtype=torch.uint8, device=device)
+
+
+def e4b_moe_forward(desc: e4b_moe_desc, experts: e4b_experts, x: torch.Tensor, router_logits=None, topk_idx=None,
+                    topk_w=None, y=None, saved_gu=None, offsets_out=None, perm_out=None, ws=None, stream=None):
+    """Expert-layer forward.  With router_logits the layer routes and fills
+    topk_idx / topk_w (allocated here when not given); without, they are inputs.
+    Returns (y, topk_idx, topk_w)."""
+    _cuda(x, "x", torch.bfloat16)
+    T = x.shape[0]
+    dev = x.device
+    if topk_idx is None:
+        topk_idx = torch.empty(T, desc.top_k, dtype=torch.int32, device=dev)
+    if topk_w is None:
+        topk_w = torch.empty(T, desc.top_k, dtype=torch.float32, device=dev)
+    if router_logits is not None:
+        _cuda(router_logits, "router_logits", torch.float32)
+    if y is None:
+        y = torch.empty(T, desc.H, dtype=torch.bfloat16, device=dev)
+    if ws is None:
+        ws = workspace(desc, T, dev)
+    _check("e4b_moe_forward", _load().e4b_moe_forward(
+        ctypes.byref(desc), ctypes.byref(experts), _ptr(x), T, _ptr(router_logits), _ptr(topk_idx), _ptr(topk_w),
+        _ptr(y), _ptr(saved_gu), _ptr(offsets_out), _ptr(perm_out), _ptr(ws), ws.numel(), _stream(stream)))
+    return y, topk_idx, topk_w
+
+
+def e4b_moe_backward_dgrad(desc: e4b_moe_desc, experts: e4b_experts, x, topk_idx, topk_w, grad_out, saved_gu=None,
+                           grad_x=None, ws=None, stream=None):
+    """Input gradient with routing held constant; returns grad_x bf16 [T, H]."""
+    _cuda(grad_out, "grad_out", torch.bfloat16)
+    T = grad_out.shape[0]
+    dev = grad_out.device
+    if grad_x is None:
+        grad_x = torch.empty(T, desc.H, dtype=torch.bfloat16, device=dev)
+    if ws is None:
+        ws = workspace(desc, T, dev)
+    _check("e4b_moe_backward_dgrad", _load().e4b_moe_backward_dgrad(
+        ctypes.byref(desc), ctypes.byref(experts), _ptr(x), T, _ptr(topk_idx), _ptr(topk_w), _ptr(grad_out),
+        _ptr(saved_gu), _ptr(grad_x), _ptr(ws), ws.numel(), _stream(stream)))
+    return grad_x

@@ -1,0 +1,400 @@
+// C ABI of the e4b library (declared in include/e4b.h): argument validation,
+// workspace layout and the launch sequence of each entry point.
+#include <atomic>
+#include <cstring>
+#include <mutex>
+#include <utility>
+#include <vector>
+
+#include "../../include/e4b.h"
+#include "e4b_internal.h"
+
+namespace e4b {
+
+static std::atomic<uint64_t> g_launches{0};
+void count_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
+
+// ------------------------------------------------------------ kernel timing
+struct TimingState {
+    std::mutex mu;
+    bool on = false;
+    std::vector<std::pair<cudaEvent_t, cudaEvent_t>> pending[KK_COUNT];
+    cudaEvent_t open[KK_COUNT] = {};
+    double total_ms[KK_COUNT] = {};
+    uint64_t count[KK_COUNT] = {};
+};
+static TimingState g_timing;
+
+static cudaEvent_t new_event() {
+    cudaEvent_t e = nullptr;
+    cudaEventCreate(&e);
+    return e;
+}
+
+void timing_begin(int kind, cudaStream_t st) {
+    std::lock_guard<std::mutex> lock(g_timing.mu);
+    if (!g_timing.on) return;
+    g_timing.open[kind] = new_event();
+    cudaEventRecord(g_timing.open[kind], st);
+}
+
+void timing_end(int kind, cudaStream_t st) {
+    std::lock_guard<std::mutex> lock(g_timing.mu);
+    if (!g_timing.on || !g_timing.open[kind]) return;
+    cudaEvent_t e = new_event();
+    cudaEventRecord(e, st);
+    g_timing.pending[kind].emplace_back(g_timing.open[kind], e);
+    g_timing.open[kind] = nullptr;
+}
+
+static void timing_collect() {
+    for (int k = 0; k < KK_COUNT; ++k) {
+        for (auto& pr : g_timing.pending[k]) {
+            float ms = 0.0f;
+            cudaEventSynchronize(pr.second);
+            if (cudaEventElapsedTime(&ms, pr.first, pr.second) == cudaSuccess) {
+                g_timing.total_ms[k] += ms;
+                g_timing.count[k] += 1;
+            }
+            cudaEventDestroy(pr.first);
+            cudaEventDestroy(pr.second);
+        }
+        g_timing.pending[k].clear();
+    }
+}
+
+int num_sms() {
+    static int cache[64] = {0};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+    if (!cache[dev]) {
+        int n = 0;
+        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+        cache[dev] = n > 0 ? n : 148;
+    }
+    return cache[dev];
+}
+
+// One status word per device, read and cleared by e4b_device_status.
+__device__ uint32_t g_device_status;
+
+uint32_t* device_status_ptr() {
+    static uint32_t* cache[64] = {nullptr};
+    static std::mutex mu;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+    std::lock_guard<std::mutex> lock(mu);
+    if (!cache[dev]) {
+        void* ptr = nullptr;
+        if (cudaGetSymbolAddress(&ptr, g_device_status) != cudaSuccess) return nullptr;
+        cache[dev] = static_cast<uint32_t*>(ptr);
+    }
+    return cache[dev];
+}
+
+// ------------------------------------------------------------ workspace layout
+struct WsLayout {
+    size_t chunk_counts, chunk_base, counts, offsets, tile_prefix, perm, a_perm, h, gu, dgu, acc32, dec_h, total;
+};
+
+static size_t align_up(size_t v) { return (v + 255) & ~size_t(255); }
+
+static WsLayout layout_for(const e4b_moe_desc* d, int64_t T) {
+    WsLayout L{};
+    const int64_t P = T * d->top_k;
+    const int64_t nch = (P + kChunkPairs - 1) / kChunkPairs;
+    size_t off = 0;
+    auto take = [&](size_t bytes) { size_t o = off; off = align_up(off + bytes); return o; };
+    L.chunk_counts = take((size_t)nch * d->E * 4);
+    L.chunk_base = take((size_t)nch * d->E * 4);
+    L.counts = take((size_t)d->E * 4);
+    L.offsets = take((size_t)(d->E + 1) * 4);
+    L.tile_prefix = take((size_t)(d->E + 1) * 4);
+    L.perm = take((size_t)P * 4);
+    L.a_perm = take((size_t)P * d->H * 2);
+    L.h = take((size_t)P * d->I * 2);
+    L.gu = take((size_t)P * 2 * d->I * 2);
+    L.dgu = take((size_t)P * 2 * d->I * 2);
+    L.acc32 = take((size_t)T * d->H * 4);
+    L.dec_h = take((size_t)P * d->I * 4);
+    L.total = off;
+    return L;
+}
+
+static e4b_status check_desc(const e4b_moe_desc* d) {
+    if (!d) return E4B_ERR_INVALID_ARG;
+    if (d->blocksize != 64) return E4B_ERR_BLOCKSIZE;
+    if (d->E < 1 || d->E > 256 || d->H <= 0 || d->I <= 0) return E4B_ERR_INVALID_ARG;
+    if (d->H % 64 || d->I % 64) return E4B_ERR_BLOCKSIZE;
+    if (d->top_k < 1 || d->top_k > 8 || d->top_k > d->E) return E4B_ERR_INVALID_ARG;
+    if (d->codebook != E4B_CODEBOOK_NF4 && d->codebook != E4B_CODEBOOK_FP4) return E4B_ERR_INVALID_ARG;
+    if (d->path < E4B_PATH_AUTO || d->path > E4B_PATH_DECODE) return E4B_ERR_INVALID_ARG;
+    return E4B_OK;
+}
+
+static e4b_status check_experts(const e4b_experts* w) {
+    if (!w || !w->gate_up || !w->down || !w->gate_up_absmax || !w->down_absmax) return E4B_ERR_INVALID_ARG;
+    return E4B_OK;
+}
+
+#define E4B_CUDA_TRY(expr)                              \
+    do {                                                \
+        if ((expr) != cudaSuccess) return E4B_ERR_CUDA; \
+    } while (0)
+
+static GemmParams base_params(const e4b_moe_desc* d, uint8_t* ws, const WsLayout& L, const float* topk_w,
+                              int64_t P) {
+    GemmParams p{};
+    p.E = d->E;
+    p.k_top = d->top_k;
+    p.offsets = reinterpret_cast<const int*>(ws + L.offsets);
+    p.tile_prefix = reinterpret_cast<const int*>(ws + L.tile_prefix);
+    p.perm = reinterpret_cast<const int*>(ws + L.perm);
+    p.topk_w = topk_w;
+    p.status = device_status_ptr();
+    (void)P;
+    return p;
+}
+
+static int max_m_tiles(int64_t P, int E) { return (int)((P + gemm_tile_rows() - 1) / gemm_tile_rows()) + E; }
+
+// gate_up GEMM + SwiGLU over the grouped rows in ws.a_perm.
+static e4b_status run_gateup(const e4b_moe_desc* d, const e4b_experts* w, uint8_t* ws, const WsLayout& L,
+                             const float* topk_w, int64_t P, __nv_bfloat16* h_out, __nv_bfloat16* gu_out,
+                             cudaStream_t st) {
+    GemmParams p = base_params(d, ws, L, topk_w, P);
+    p.K = d->H;
+    p.N = d->I;
+    p.n_tiles = (d->I + 127) / 128;
+    p.absmax = w->gate_up_absmax;
+    p.b_rows_per_expert = 2 * d->I;
+    p.b_rows_total = (int64_t)d->E * 2 * d->I;
+    p.b_blocks_per_row = d->H / 64;
+    p.up_offset = d->I;
+    p.out_bf16 = h_out;
+    p.gu = gu_out;
+    p.ld_out = d->I;
+    E4B_CUDA_TRY(launch_grouped_gemm(EPI_GATEUP, d->codebook, ws + L.a_perm, P, w->gate_up, p.b_rows_total, d->H / 2,
+                                     p, max_m_tiles(P, d->E), st));
+    return E4B_OK;
+}
+
+}  // namespace e4b
+
+using namespace e4b;
+
+extern "C" {
+
+const char* e4b_status_string(e4b_status s) {
+    switch (s) {
+        case E4B_OK: return "ok";
+        case E4B_ERR_INVALID_ARG: return "invalid argument";
+        case E4B_ERR_BLOCKSIZE: return "blocksize must be 64 and divide in_features";
+        case E4B_ERR_UNSUPPORTED: return "unsupported request";
+        case E4B_ERR_WORKSPACE: return "workspace missing or too small";
+        case E4B_ERR_CUDA: return "CUDA error";
+        case E4B_ERR_TIMEOUT: return "device wait timed out";
+    }
+    return "unknown status";
+}
+
+uint64_t e4b_launch_count(void) { return g_launches.load(); }
+
+void e4b_timing_enable(int on) {
+    std::lock_guard<std::mutex> lock(g_timing.mu);
+    timing_collect();
+    g_timing.on = on != 0;
+}
+
+void e4b_timing_reset(void) {
+    std::lock_guard<std::mutex> lock(g_timing.mu);
+    timing_collect();
+    for (int k = 0; k < KK_COUNT; ++k) {
+        g_timing.total_ms[k] = 0.0;
+        g_timing.count[k] = 0;
+    }
+}
+
+e4b_status e4b_timing_get(int kind, double* total_ms, uint64_t* launches) {
+    if (kind < 0 || kind >= KK_COUNT || !total_ms || !launches) return E4B_ERR_INVALID_ARG;
+    std::lock_guard<std::mutex> lock(g_timing.mu);
+    timing_collect();
+    *total_ms = g_timing.total_ms[kind];
+    *launches = g_timing.count[kind];
+    return E4B_OK;
+}
+
+e4b_status e4b_device_status(void* stream) {
+    if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return E4B_ERR_CUDA;
+    uint32_t* ptr = device_status_ptr();
+    if (!ptr) return E4B_ERR_CUDA;
+    uint32_t v = 0;
+    if (cudaMemcpy(&v, ptr, 4, cudaMemcpyDeviceToHost) != cudaSuccess) return E4B_ERR_CUDA;
+    if (v) {
+        const uint32_t zero = 0;
+        if (cudaMemcpy(ptr, &zero, 4, cudaMemcpyHostToDevice) != cudaSuccess) return E4B_ERR_CUDA;
+        return E4B_ERR_TIMEOUT;
+    }
+    return E4B_OK;
+}
+
+e4b_status e4b_quantize_nf4(const float* w, int64_t E, int64_t out, int64_t in, int blocksize, e4b_codebook cb,
+                            uint8_t* packed, float* absmax, void* stream) {
+    if (blocksize != 64) return E4B_ERR_BLOCKSIZE;
+    if (E < 0 || out < 0 || in < 0) return E4B_ERR_INVALID_ARG;
+    if (in % 64) return E4B_ERR_BLOCKSIZE;
+    if (cb != E4B_CODEBOOK_NF4 && cb != E4B_CODEBOOK_FP4) return E4B_ERR_INVALID_ARG;
+    const int64_t n = E * out * in;
+    if (n == 0) return E4B_OK;
+    if (!w || !packed || !absmax) return E4B_ERR_INVALID_ARG;
+    E4B_CUDA_TRY(launch_quantize(w, n / 64, cb, packed, absmax, static_cast<cudaStream_t>(stream)));
+    return E4B_OK;
+}
+
+e4b_status e4b_dequantize_nf4(const uint8_t* packed, const float* absmax, int64_t E, int64_t out, int64_t in,
+                              int blocksize, e4b_codebook cb, e4b_dtype out_dtype, void* w_out, void* stream) {
+    if (blocksize != 64) return E4B_ERR_BLOCKSIZE;
+    if (E < 0 || out < 0 || in < 0) return E4B_ERR_INVALID_ARG;
+    if (in % 64) return E4B_ERR_BLOCKSIZE;
+    if (cb != E4B_CODEBOOK_NF4 && cb != E4B_CODEBOOK_FP4) return E4B_ERR_INVALID_ARG;
+    if (out_dtype != E4B_F32 && out_dtype != E4B_BF16) return E4B_ERR_INVALID_ARG;
+    const int64_t n = E * out * in;
+    if (n == 0) return E4B_OK;
+    if (!packed || !absmax || !w_out) return E4B_ERR_INVALID_ARG;
+    E4B_CUDA_TRY(launch_dequantize(packed, absmax, n, cb, out_dtype == E4B_BF16, w_out,
+                                   static_cast<cudaStream_t>(stream)));
+    return E4B_OK;
+}
+
+size_t e4b_moe_workspace_size(const e4b_moe_desc* d, int64_t T) {
+    if (check_desc(d) != E4B_OK || T < 0) return 0;
+    return layout_for(d, T).total;
+}
+
+e4b_status e4b_moe_forward(const e4b_moe_desc* d, const e4b_experts* w, const void* x, int64_t T,
+                           const float* router_logits, int32_t* topk_idx, float* topk_w, void* y, void* saved_gu,
+                           int32_t* offsets_out, int32_t* perm_out, void* workspace, size_t ws_bytes,
+                           void* stream) {
+    e4b_status s = check_desc(d);
+    if (s != E4B_OK) return s;
+    if ((s = check_experts(w)) != E4B_OK) return s;
+    if (T < 0 || T * d->top_k > (int64_t)INT32_MAX) return E4B_ERR_INVALID_ARG;
+    if (T == 0) return E4B_OK;
+    if (!x || !topk_idx || !topk_w || !y) return E4B_ERR_INVALID_ARG;
+    const WsLayout L = layout_for(d, T);
+    if (!workspace || ws_bytes < L.total) return E4B_ERR_WORKSPACE;
+    const bool want_grouped_outputs = saved_gu || offsets_out || perm_out;
+    bool decode = (d->path == E4B_PATH_DECODE) || (d->path == E4B_PATH_AUTO && T <= 8 && !want_grouped_outputs);
+    if (d->path == E4B_PATH_DECODE && (T > 8 || want_grouped_outputs)) return E4B_ERR_UNSUPPORTED;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
+    const int64_t P = T * d->top_k;
+
+    if (router_logits)
+        E4B_CUDA_TRY(launch_route(router_logits, T, d->E, d->top_k, d->renormalize, topk_idx, topk_w, st));
+
+    if (decode) {
+        E4B_CUDA_TRY(launch_decode_forward(d->codebook, d->E, d->H, d->I, d->top_k, T,
+                                           static_cast<const __nv_bfloat16*>(x), topk_idx, topk_w, w->gate_up,
+                                           w->gate_up_absmax, w->down, w->down_absmax,
+                                           reinterpret_cast<float*>(ws + L.dec_h), static_cast<__nv_bfloat16*>(y),
+                                           st));
+        return E4B_OK;
+    }
+
+    int32_t* offsets = reinterpret_cast<int32_t*>(ws + L.offsets);
+    int32_t* perm = reinterpret_cast<int32_t*>(ws + L.perm);
+    E4B_CUDA_TRY(launch_group(topk_idx, P, d->E, gemm_tile_rows(), reinterpret_cast<int32_t*>(ws + L.chunk_counts),
+                              reinterpret_cast<int32_t*>(ws + L.chunk_base), reinterpret_cast<int32_t*>(ws + L.counts),
+                              offsets, reinterpret_cast<int32_t*>(ws + L.tile_prefix), perm, st));
+    E4B_CUDA_TRY(launch_gather_rows(static_cast<const __nv_bfloat16*>(x), perm, offsets + d->E, d->top_k, P, d->H,
+                                    reinterpret_cast<__nv_bfloat16*>(ws + L.a_perm), st));
+    float* acc = reinterpret_cast<float*>(ws + L.acc32);
+    E4B_CUDA_TRY(cudaMemsetAsync(acc, 0, (size_t)T * d->H * 4, st));
+    __nv_bfloat16* h = reinterpret_cast<__nv_bfloat16*>(ws + L.h);
+    if ((s = run_gateup(d, w, ws, L, topk_w, P, h, static_cast<__nv_bfloat16*>(saved_gu), st)) != E4B_OK) return s;
+
+    GemmParams p = base_params(d, ws, L, topk_w, P);
+    p.K = d->I;
+    p.N = d->H;
+    p.n_tiles = (d->H + 255) / 256;
+    p.absmax = w->down_absmax;
+    p.b_rows_per_expert = d->H;
+    p.b_rows_total = (int64_t)d->E * d->H;
+    p.b_blocks_per_row = d->I / 64;
+    p.out_f32 = acc;
+    p.ld_out = d->H;
+    E4B_CUDA_TRY(launch_grouped_gemm(EPI_DOWN, d->codebook, h, P, w->down, p.b_rows_total, d->I / 2, p,
+                                     max_m_tiles(P, d->E), st));
+    E4B_CUDA_TRY(launch_f32_to_bf16(acc, T * d->H, static_cast<__nv_bfloat16*>(y), st));
+    if (offsets_out) E4B_CUDA_TRY(cudaMemcpyAsync(offsets_out, offsets, (d->E + 1) * 4, cudaMemcpyDeviceToDevice, st));
+    if (perm_out) E4B_CUDA_TRY(cudaMemcpyAsync(perm_out, perm, P * 4, cudaMemcpyDeviceToDevice, st));
+    return E4B_OK;
+}
+
+e4b_status e4b_moe_backward_dgrad(const e4b_moe_desc* d, const e4b_experts* w, const void* x, int64_t T,
+                                  const int32_t* topk_idx, const float* topk_w, const void* grad_out,
+                                  const void* saved_gu, void* grad_x, void* workspace, size_t ws_bytes,
+                                  void* stream) {
+    e4b_status s = check_desc(d);
+    if (s != E4B_OK) return s;
+    if ((s = check_experts(w)) != E4B_OK) return s;
+    if (T < 0 || T * d->top_k > (int64_t)INT32_MAX) return E4B_ERR_INVALID_ARG;
+    if (T == 0) return E4B_OK;
+    if (!topk_idx || !topk_w || !grad_out || !grad_x || (!saved_gu && !x)) return E4B_ERR_INVALID_ARG;
+    const WsLayout L = layout_for(d, T);
+    if (!workspace || ws_bytes < L.total) return E4B_ERR_WORKSPACE;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
+    const int64_t P = T * d->top_k;
+    int32_t* perm = reinterpret_cast<int32_t*>(ws + L.perm);
+    E4B_CUDA_TRY(launch_group(topk_idx, P, d->E, gemm_tile_rows(), reinterpret_cast<int32_t*>(ws + L.chunk_counts),
+                              reinterpret_cast<int32_t*>(ws + L.chunk_base), reinterpret_cast<int32_t*>(ws + L.counts),
+                              reinterpret_cast<int32_t*>(ws + L.offsets), reinterpret_cast<int32_t*>(ws + L.tile_prefix),
+                              perm, st));
+    __nv_bfloat16* a_perm = reinterpret_cast<__nv_bfloat16*>(ws + L.a_perm);
+    const int32_t* nrows = reinterpret_cast<const int32_t*>(ws + L.offsets) + d->E;
+    const __nv_bfloat16* gu = static_cast<const __nv_bfloat16*>(saved_gu);
+    if (!gu) {   // recompute the gate/up pre-activations from x
+        E4B_CUDA_TRY(launch_gather_rows(static_cast<const __nv_bfloat16*>(x), perm, nrows, d->top_k, P, d->H, a_perm, st));
+        __nv_bfloat16* gu_ws = reinterpret_cast<__nv_bfloat16*>(ws + L.gu);
+        if ((s = run_gateup(d, w, ws, L, topk_w, P, reinterpret_cast<__nv_bfloat16*>(ws + L.h), gu_ws, st)) != E4B_OK)
+            return s;
+        gu = gu_ws;
+    }
+    E4B_CUDA_TRY(launch_gather_rows(static_cast<const __nv_bfloat16*>(grad_out), perm, nrows, d->top_k, P, d->H, a_perm, st));
+    float* acc = reinterpret_cast<float*>(ws + L.acc32);
+    E4B_CUDA_TRY(cudaMemsetAsync(acc, 0, (size_t)T * d->H * 4, st));
+    __nv_bfloat16* dgu = reinterpret_cast<__nv_bfloat16*>(ws + L.dgu);
+
+    GemmParams p = base_params(d, ws, L, topk_w, P);   // dh = w * grad_out W_down, then SwiGLU backward
+    p.K = d->H;
+    p.N = d->I;
+    p.n_tiles = (d->I + 255) / 256;
+    p.absmax = w->down_absmax;
+    p.b_rows_per_expert = d->H;
+    p.b_rows_total = (int64_t)d->E * d->H;
+    p.b_blocks_per_row = d->I / 64;
+    p.gu = const_cast<__nv_bfloat16*>(gu);
+    p.out_bf16 = dgu;
+    p.ld_out = 2 * d->I;
+    E4B_CUDA_TRY(launch_grouped_gemm(EPI_DGRAD_DOWN, d->codebook, a_perm, P, w->down, p.b_rows_total, d->I / 2, p,
+                                     max_m_tiles(P, d->E), st));
+
+    GemmParams q = base_params(d, ws, L, topk_w, P);   // grad_x += [dG, dU] W_gate_up
+    q.K = 2 * d->I;
+    q.N = d->H;
+    q.n_tiles = (d->H + 255) / 256;
+    q.absmax = w->gate_up_absmax;
+    q.b_rows_per_expert = 2 * d->I;
+    q.b_rows_total = (int64_t)d->E * 2 * d->I;
+    q.b_blocks_per_row = d->H / 64;
+    q.out_f32 = acc;
+    q.ld_out = d->H;
+    E4B_CUDA_TRY(launch_grouped_gemm(EPI_DGRAD_GATEUP, d->codebook, dgu, P, w->gate_up, q.b_rows_total, d->H / 2, q,
+                                     max_m_tiles(P, d->E), st));
+    E4B_CUDA_TRY(launch_f32_to_bf16(acc, T * d->H, static_cast<__nv_bfloat16*>(grad_x), st));
+    return E4B_OK;
+}
+
+}  // extern "C"

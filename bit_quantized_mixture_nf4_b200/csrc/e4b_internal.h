@@ -1,0 +1,77 @@
+// Internal host/device interfaces shared by the e4b translation units.
+#pragma once
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+#include <stdint.h>
+
+#include <algorithm>
+
+#include "e4b_device.cuh"
+
+namespace e4b {
+
+enum Epi { EPI_GATEUP = 0, EPI_DOWN = 1, EPI_DGRAD_DOWN = 2, EPI_DGRAD_GATEUP = 3 };
+
+struct GemmParams {
+    int E, K, N, n_tiles, k_top;
+    const int* offsets;       // [E+1] first grouped row of each expert
+    const int* tile_prefix;   // [E+1] prefix of ceil(M_e / 128); [E] = total m-tiles
+    const int* perm;          // [P] pair id of each grouped row
+    const float* topk_w;      // [P] routing weight by pair id
+    const float* absmax;      // absmax of the weight stack
+    int64_t b_rows_total;     // rows of the stored [rows, cols] weight matrix, all experts
+    int b_rows_per_expert;
+    int b_blocks_per_row;     // stored cols / 64
+    int up_offset;            // I (EPI_GATEUP: first up row; also the feature count)
+    __nv_bfloat16* out_bf16;  // h [P, I] or dGU [P, 2I]
+    __nv_bfloat16* gu;        // saved gate/up [P, 2I] (written by EPI_GATEUP, read by EPI_DGRAD_DOWN)
+    float* out_f32;           // [T, H] fp32 accumulation target
+    int ld_out;
+    uint32_t* status;         // device status word
+};
+
+// launch bookkeeping
+void count_launch();
+// Optional per-kernel-kind event timing (off by default): brackets one launch
+// with CUDA events on its stream.
+enum KernelKind { KK_QUANT = 0, KK_DEQUANT, KK_ROUTE, KK_GROUP, KK_GATHER, KK_CONVERT, KK_GEMM_GATEUP, KK_GEMM_DOWN,
+                  KK_GEMM_DGRAD_DOWN, KK_GEMM_DGRAD_GATEUP, KK_DECODE_GATEUP, KK_DECODE_DOWN, KK_COUNT };
+void timing_begin(int kind, cudaStream_t st);
+void timing_end(int kind, cudaStream_t st);
+int num_sms();
+uint32_t* device_status_ptr();
+
+// quant.cu
+cudaError_t launch_quantize(const float* w, int64_t nblocks, int codebook, uint8_t* packed, float* absmax,
+                            cudaStream_t st);
+cudaError_t launch_dequantize(const uint8_t* packed, const float* absmax, int64_t n, int codebook, int out_bf16,
+                              void* out, cudaStream_t st);
+
+// route.cu
+constexpr int kChunkPairs = 2048;
+cudaError_t launch_route(const float* logits, int64_t T, int E, int k, int renorm, int32_t* idx, float* w,
+                         cudaStream_t st);
+// counts/offsets/tile_prefix/perm from topk_idx; chunk scratch: [nchunks * E] ints x2
+cudaError_t launch_group(const int32_t* idx, int64_t P, int E, int tile_rows, int32_t* chunk_counts,
+                         int32_t* chunk_base, int32_t* counts, int32_t* offsets, int32_t* tile_prefix,
+                         int32_t* perm, cudaStream_t st);
+// nrows: device pointer to the number of grouped rows (offsets[E])
+cudaError_t launch_gather_rows(const __nv_bfloat16* src, const int32_t* perm, const int32_t* nrows, int k,
+                               int64_t P, int H, __nv_bfloat16* dst, cudaStream_t st);
+cudaError_t launch_f32_to_bf16(const float* src, int64_t n, __nv_bfloat16* dst, cudaStream_t st);
+
+// grouped_gemm.cu
+int gemm_tile_rows();
+cudaError_t launch_grouped_gemm(int epi, int codebook, const void* a, int64_t a_rows, const uint8_t* packed,
+                                int64_t packed_rows_total, int packed_row_bytes, GemmParams p, int max_m_tiles,
+                                cudaStream_t st);
+
+// decode.cu (T <= 8)
+cudaError_t launch_decode_forward(int codebook, int E, int H, int I, int k, int64_t T, const __nv_bfloat16* x,
+                                  const int32_t* idx, const float* w, const uint8_t* gu_packed,
+                                  const float* gu_absmax, const uint8_t* d_packed, const float* d_absmax,
+                                  float* h_scratch, __nv_bfloat16* y, cudaStream_t st);
+
+}  // namespace e4b

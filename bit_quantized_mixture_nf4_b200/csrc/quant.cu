@@ -1,0 +1,159 @@
+// Blockwise 4-bit quantize and dequantize kernels (HBM-bound).
+//
+// Quantize follows "experts4bit-qlora 0.1.0" experts.py, Experts4bit.from_float /
+// _quantize_stack: per 64 contiguous in-features of each row, absmax = max|w|,
+// every element divided by absmax and mapped to the nearest codebook value (an
+// exact tie goes to the smaller value), two codes per byte with the first
+// element in the high nibble.  Dequantize follows _dequantize_expert: code value
+// times absmax in fp32, optionally rounded to bf16 (nearest-even).
+#include "e4b_internal.h"
+
+namespace e4b {
+
+// Codes in ascending order of their value (NF4: identity; FP4: -1 .. -1/12,
+// +0, 1/12 .. 1; the -0 code is never produced).
+__device__ __forceinline__ int sorted_code(int cb, int r) {
+    if (cb == 0) return r;
+    return r < 7 ? 15 - r : r - 7;
+}
+
+// 4 threads per 64-element block; thread q of a quad holds elements
+// 16*i + 4*q + {0..3}, i = 0..3, so each quad reads 64 contiguous bytes per load.
+template <int CB>
+__global__ void __launch_bounds__(256) quantize_kernel(const float* __restrict__ w, int64_t nblocks,
+                                                       uint8_t* __restrict__ packed, float* __restrict__ absmax) {
+    __shared__ float s_mid[15];
+    __shared__ uint8_t s_code[16];
+    constexpr int NV = (CB == 0) ? 16 : 15;   // distinct codebook values
+    if (threadIdx.x < 16) {
+        const int r = threadIdx.x;
+        if (r < NV) s_code[r] = (uint8_t)sorted_code(CB, r);
+        if (r < 15) {
+            if (r < NV - 1) {
+                const float lo = c_code[CB][sorted_code(CB, r)], hi = c_code[CB][sorted_code(CB, r + 1)];
+                s_mid[r] = __fmul_rn(__fadd_rn(lo, hi), 0.5f);
+            } else {
+                s_mid[r] = __int_as_float(0x7f800000);   // +inf: never below a finite value
+            }
+        }
+    }
+    __syncthreads();
+    const int q = threadIdx.x & 3;
+    const int zero_code = (CB == 0) ? 7 : 0;
+    const int64_t stride = (int64_t)gridDim.x * blockDim.x / 4;
+    for (int64_t b = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) / 4; b < nblocks; b += stride) {
+        const float4* src = reinterpret_cast<const float4*>(w + b * 64);
+        float v[16];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const float4 f = __ldcs(src + i * 4 + q);
+            v[4 * i] = f.x; v[4 * i + 1] = f.y; v[4 * i + 2] = f.z; v[4 * i + 3] = f.w;
+        }
+        float a = 0.0f;
+#pragma unroll
+        for (int i = 0; i < 16; ++i) a = fmaxf(a, fabsf(v[i]));
+        a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, 1));
+        a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, 2));
+        if (q == 0) absmax[b] = a;
+        uint32_t code[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+            if (a == 0.0f) {
+                code[i] = zero_code;
+            } else {
+                const float n = __fdiv_rn(v[i], a);
+                int r = 0;   // number of midpoints strictly below n
+                if (s_mid[r + 7] < n) r += 8;
+                if (s_mid[r + 3] < n) r += 4;
+                if (s_mid[r + 1] < n) r += 2;
+                if (s_mid[r] < n) r += 1;
+                code[i] = s_code[r];
+            }
+        }
+        uint16_t* dst = reinterpret_cast<uint16_t*>(packed + b * 32);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const uint32_t b0 = (code[4 * i] << 4) | code[4 * i + 1];
+            const uint32_t b1 = (code[4 * i + 2] << 4) | code[4 * i + 3];
+            dst[(i * 8 + q * 2) / 2] = (uint16_t)(b0 | (b1 << 8));
+        }
+    }
+}
+
+// One thread per 16 packed bytes (32 elements, half a block).
+template <int CB, bool BF16>
+__global__ void __launch_bounds__(256) dequantize_kernel(const uint8_t* __restrict__ packed,
+                                                         const float* __restrict__ absmax, int64_t nchunks,
+                                                         void* __restrict__ out) {
+    __shared__ float s_val[16];
+    if (threadIdx.x < 16) s_val[threadIdx.x] = c_code[CB][threadIdx.x];
+    __syncthreads();
+    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+    for (int64_t c = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; c < nchunks; c += stride) {
+        const uint4 pk = __ldcs(reinterpret_cast<const uint4*>(packed) + c);
+        const float a = __ldg(absmax + (c >> 1));
+        const uint32_t words[4] = {pk.x, pk.y, pk.z, pk.w};
+        if (BF16) {
+            const BlockTable tb = make_table<CB>(a);
+            uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(out) + c * 32);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                uint32_t o[4];
+                decode_word(tb, words[i], o);
+                __stcs(dst + i, make_uint4(o[0], o[1], o[2], o[3]));
+            }
+        } else {
+            float4* dst = reinterpret_cast<float4*>(static_cast<float*>(out) + c * 32);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const uint32_t x = words[i];
+                float f[8];
+#pragma unroll
+                for (int bb = 0; bb < 4; ++bb) {
+                    const uint32_t byte = (x >> (8 * bb)) & 0xFFu;
+                    f[2 * bb] = __fmul_rn(s_val[byte >> 4], a);
+                    f[2 * bb + 1] = __fmul_rn(s_val[byte & 15u], a);
+                }
+                __stcs(dst + 2 * i, make_float4(f[0], f[1], f[2], f[3]));
+                __stcs(dst + 2 * i + 1, make_float4(f[4], f[5], f[6], f[7]));
+            }
+        }
+    }
+}
+
+static int grid_for(int64_t work_items, int threads) {
+    const int64_t blocks = (work_items + threads - 1) / threads;
+    return (int)std::max<int64_t>(1, std::min<int64_t>(blocks, (int64_t)num_sms() * 8));
+}
+
+cudaError_t launch_quantize(const float* w, int64_t nblocks, int codebook, uint8_t* packed, float* absmax,
+                            cudaStream_t st) {
+    if (nblocks == 0) return cudaSuccess;
+    const int grid = grid_for(nblocks * 4, 256);
+    timing_begin(KK_QUANT, st);
+    if (codebook == 0) quantize_kernel<0><<<grid, 256, 0, st>>>(w, nblocks, packed, absmax);
+    else quantize_kernel<1><<<grid, 256, 0, st>>>(w, nblocks, packed, absmax);
+    timing_end(KK_QUANT, st);
+    count_launch();
+    return cudaGetLastError();
+}
+
+cudaError_t launch_dequantize(const uint8_t* packed, const float* absmax, int64_t n, int codebook, int out_bf16,
+                              void* out, cudaStream_t st) {
+    const int64_t nchunks = n / 32;
+    if (nchunks == 0) return cudaSuccess;
+    const int grid = grid_for(nchunks, 256);
+    timing_begin(KK_DEQUANT, st);
+    if (codebook == 0) {
+        if (out_bf16) dequantize_kernel<0, true><<<grid, 256, 0, st>>>(packed, absmax, nchunks, out);
+        else dequantize_kernel<0, false><<<grid, 256, 0, st>>>(packed, absmax, nchunks, out);
+    } else {
+        if (out_bf16) dequantize_kernel<1, true><<<grid, 256, 0, st>>>(packed, absmax, nchunks, out);
+        else dequantize_kernel<1, false><<<grid, 256, 0, st>>>(packed, absmax, nchunks, out);
+    }
+    timing_end(KK_DEQUANT, st);
+    count_launch();
+    return cudaGetLastError();
+}
+
+}  // namespace e4b

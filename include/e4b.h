@@ -1,0 +1,176 @@
+/*
+ * e4b.h -- C ABI of the e4b library: the NF4 (and FP4) quantized Mixture-of-
+ * Experts expert path on NVIDIA B200 (sm_100a).
+ *
+ * The operations follow the expert-layer pages:
+ *   [P4] "experts4bit-qlora 0.1.0" source diff, file _vendor/experts.py, class
+ *        Experts4bit: __init__ (storage layout and validation), from_float and
+ *        _quantize_stack (quantize), _dequantize_expert (dequantize), forward.
+ *   [P5] bitsandbytes pull request #1965 "Add Experts4bit for 4-bit quantization
+ *        of fused MoE experts", section "What this adds" (recompute-in-backward
+ *        input gradient, frozen base).
+ *
+ * Conventions for every entry point:
+ *   - Tensor pointers are DEVICE pointers owned by the caller, contiguous,
+ *     row-major, 16-byte aligned.  The library allocates nothing.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default stream).
+ *     Calls are stream-ordered and asynchronous.
+ *   - Argument errors are detected on the host before any launch and return a
+ *     status without touching memory.  Launch failures return E4B_ERR_CUDA.
+ *   - Device-side waits in the grouped GEMM carry a time limit; if one expires
+ *     the kernel records it in a device status word and exits without trapping;
+ *     e4b_device_status() reports it as E4B_ERR_TIMEOUT.
+ *   - There is no CPU fallback: without a usable sm_100a device every compute
+ *     call returns E4B_ERR_CUDA.
+ *
+ * Storage of one weight stack [E, out, in] (gate_up: out = 2I, in = H, gate
+ * rows first; down: out = H, in = I):
+ *   packed  uint8 [E, out*in/2]   element 2b of an expert's row-major [out, in]
+ *                                 matrix in the HIGH nibble of byte b, element
+ *                                 2b+1 in the low nibble;
+ *   absmax  fp32  [E, out*in/64]  block j of row o at o*in/64 + j.
+ * Codes index the 16-value codebook (NF4: ascending NormalFloat values, code 7
+ * = 0; FP4: sign in bit 3, e2m1 magnitude / 6 in bits 2..0).
+ */
+#ifndef E4B_H_
+#define E4B_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define E4B_API __attribute__((visibility("default")))
+#else
+#define E4B_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    E4B_OK = 0,
+    E4B_ERR_INVALID_ARG = 1,   /* null pointer, negative or unsupported size, k > E ... */
+    E4B_ERR_BLOCKSIZE = 2,     /* in_features % blocksize != 0, or blocksize != 64      */
+    E4B_ERR_UNSUPPORTED = 3,   /* valid request outside what the kernels implement       */
+    E4B_ERR_WORKSPACE = 4,     /* workspace NULL or smaller than e4b_moe_workspace_size  */
+    E4B_ERR_CUDA = 5,          /* a CUDA runtime call or launch failed                    */
+    E4B_ERR_TIMEOUT = 6        /* a device-side wait hit its time limit                   */
+} e4b_status;
+
+typedef enum { E4B_CODEBOOK_NF4 = 0, E4B_CODEBOOK_FP4 = 1 } e4b_codebook;
+typedef enum { E4B_F32 = 0, E4B_BF16 = 1 } e4b_dtype;
+typedef enum { E4B_PATH_AUTO = 0, E4B_PATH_GROUPED = 1, E4B_PATH_DECODE = 2 } e4b_path;
+
+/* Layer description.  H and I must be multiples of 64 (blocks never straddle a
+ * row, [P4] __init__); 1 <= top_k <= min(E, 8); E <= 256; blocksize == 64.
+ * path: AUTO takes the weight-streaming decode kernels for T <= 8 and the
+ * grouped tensor-core kernels otherwise; the other values force one path. */
+typedef struct {
+    int E, H, I, top_k;
+    int renormalize;           /* divide the selected softmax weights by their sum  */
+    e4b_codebook codebook;
+    int blocksize;             /* must be 64 */
+    e4b_path path;
+} e4b_moe_desc;
+
+/* Device pointers to the two quantized stacks (see storage above). */
+typedef struct {
+    const uint8_t *gate_up;        /* [E, 2I*H/2] */
+    const uint8_t *down;           /* [E, H*I/2]  */
+    const float *gate_up_absmax;   /* [E, 2I*H/64] */
+    const float *down_absmax;      /* [E, H*I/64]  */
+} e4b_experts;
+
+/* Blockwise 4-bit quantization ([P4] from_float / _quantize_stack).
+ * w: fp32 [E, out, in].  For every 64-element block of each row: absmax =
+ * max|w| (stored as is, fp32); each element is divided by absmax (IEEE fp32
+ * division) and takes the code of the nearest codebook value, an exact tie
+ * going to the smaller value; an all-zero block stores absmax 0 and the zero
+ * code.  Writes packed [E, out*in/2] and absmax [E, out*in/64].
+ * Errors: E4B_ERR_BLOCKSIZE if blocksize != 64 or in % 64 != 0;
+ * E4B_ERR_INVALID_ARG for null pointers, negative sizes or an unknown codebook.
+ * Non-finite inputs are outside the contract. */
+E4B_API e4b_status e4b_quantize_nf4(const float *w, int64_t E, int64_t out, int64_t in, int blocksize,
+                            e4b_codebook codebook, uint8_t *packed, float *absmax, void *stream);
+
+/* Dequantization ([P4] _dequantize_expert): value = code_value * absmax with
+ * one fp32 multiply, then (out_dtype == E4B_BF16) rounded to bf16 nearest-even.
+ * w_out: [E, out, in] of out_dtype.  Same errors as quantize. */
+E4B_API e4b_status e4b_dequantize_nf4(const uint8_t *packed, const float *absmax, int64_t E, int64_t out,
+                              int64_t in, int blocksize, e4b_codebook codebook, e4b_dtype out_dtype,
+                              void *w_out, void *stream);
+
+/* Bytes of device workspace e4b_moe_forward and e4b_moe_backward_dgrad need
+ * for T tokens (the larger of the two).  Returns 0 for an invalid desc. */
+E4B_API size_t e4b_moe_workspace_size(const e4b_moe_desc *d, int64_t T);
+
+/* Forward of the expert layer ([P4] Experts4bit.forward):
+ *   y_t = sum_j w_{t,j} * (silu(x_t W_gate,e^T) * (x_t W_up,e^T)) W_down,e^T,
+ * e = topk_idx[t,j], W_gate/W_up = rows [0,I)/[I,2I) of gate_up, the weights
+ * dequantized to bf16, products accumulated in fp32, the weighted sum over the
+ * k slots in fp32, y rounded to bf16.
+ *   x            bf16 [T, H]
+ *   router_logits fp32 [T, E] or NULL.  If given, the layer routes: top-k by
+ *                logit (ties to the lower expert index), weights = softmax over
+ *                all E at the chosen experts, divided by their sum when
+ *                d->renormalize; topk_idx / topk_w are WRITTEN.  If NULL they
+ *                are read as inputs, as in [P4] forward(hidden_states,
+ *                top_k_index, top_k_weights).
+ *   topk_idx     int32 [T, k];  topk_w fp32 [T, k]
+ *   y            bf16 [T, H]
+ *   saved_gu     bf16 [T*k, 2I] or NULL: the gate/up pre-activations in grouped
+ *                row order (row r holds pair perm[r]; columns [0,I) gate,
+ *                [I,2I) up), for e4b_moe_backward_dgrad.
+ *   offsets_out  int32 [E+1] or NULL: first grouped row of each expert.
+ *   perm_out     int32 [T*k] or NULL: pair id t*k+j of each grouped row;
+ *                experts ascending, tokens ascending inside an expert.
+ *   workspace    device scratch of at least e4b_moe_workspace_size(d, T) bytes.
+ * T == 0 is a no-op.  topk_idx entries outside [0, E) are outside the contract. */
+E4B_API e4b_status e4b_moe_forward(const e4b_moe_desc *d, const e4b_experts *w, const void *x, int64_t T,
+                           const float *router_logits, int32_t *topk_idx, float *topk_w, void *y,
+                           void *saved_gu, int32_t *offsets_out, int32_t *perm_out,
+                           void *workspace, size_t ws_bytes, void *stream);
+
+/* Input gradient of the forward with routing held constant ([P5] "What this
+ * adds": recompute-in-backward; the packed base is frozen, no weight gradient):
+ *   dh   = w_{t,j} * grad_out_t W_down,e                 (contract over H)
+ *   dG   = dh * u * s(g) * (1 + g (1 - s(g))),  dU = dh * silu(g)
+ *   grad_x_t = sum_j  dG W_gate,e + dU W_up,e            (contract over 2I)
+ * with the weights re-dequantized inside the kernels and never stored.
+ * g, u come from saved_gu (as written by e4b_moe_forward for the same
+ * topk_idx) or, when saved_gu is NULL, are recomputed from x.
+ *   x bf16 [T,H] (read only when saved_gu is NULL), topk_idx int32 [T,k],
+ *   topk_w fp32 [T,k], grad_out bf16 [T,H], grad_x bf16 [T,H] (written). */
+E4B_API e4b_status e4b_moe_backward_dgrad(const e4b_moe_desc *d, const e4b_experts *w, const void *x,
+                                  int64_t T, const int32_t *topk_idx, const float *topk_w,
+                                  const void *grad_out, const void *saved_gu, void *grad_x,
+                                  void *workspace, size_t ws_bytes, void *stream);
+
+/* Synchronizes `stream`, then reads and clears the library's device status
+ * word: E4B_OK, or E4B_ERR_TIMEOUT if a kernel gave up on a wait since the last
+ * call.  E4B_ERR_CUDA if the synchronization itself fails. */
+E4B_API e4b_status e4b_device_status(void *stream);
+
+/* Static description of a status code. */
+E4B_API const char *e4b_status_string(e4b_status s);
+
+/* Number of kernels the library launched since load (a host-side counter,
+ * for benchmarks that report their launch count). */
+E4B_API uint64_t e4b_launch_count(void);
+
+/* Optional per-kernel timing for benchmarks (off by default).  When enabled,
+ * every launch of the library is bracketed by two CUDA events on its stream;
+ * e4b_timing_get synchronizes on the recorded events and returns, for one
+ * kernel kind, the summed device time (ms) and the number of timed launches.
+ * Kinds: 0 quantize, 1 dequantize, 2 route, 3 group, 4 gather, 5 convert,
+ * 6 grouped gate_up GEMM, 7 grouped down GEMM, 8 dgrad down GEMM,
+ * 9 dgrad gate_up GEMM, 10 decode gate_up GEMV, 11 decode down GEMV. */
+E4B_API void e4b_timing_enable(int on);
+E4B_API void e4b_timing_reset(void);
+E4B_API e4b_status e4b_timing_get(int kind, double *total_ms, uint64_t *launches);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* E4B_H_ */

@@ -1,0 +1,83 @@
+"""CPU checks of the C-ABI library: it builds for sm_100a, loads, exports every
+symbol include/e4b.h declares, and validates arguments on the host (no GPU
+needed: every call here returns before any launch)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from bit_quantized_mixture_nf4_b200 import build as e4b_build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    e4b_build.build()
+    import bit_quantized_mixture_nf4_b200 as e4b
+    return e4b
+
+
+def declared_functions():
+    text = open(os.path.join(ROOT, "include", "e4b.h")).read()
+    return sorted(set(re.findall(r"E4B_API\s+[\w\s\*]+?\b(e4b_\w+)\s*\(", text)))
+
+
+def test_header_declares_the_four_operations():
+    names = declared_functions()
+    for n in ("e4b_quantize_nf4", "e4b_dequantize_nf4", "e4b_moe_forward", "e4b_moe_backward_dgrad"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    so = ctypes.CDLL(lib.LIB_PATH)
+    for n in declared_functions():
+        assert hasattr(so, n), n
+    assert set(declared_functions()) == set(lib.EXPORTS)
+
+
+def test_status_strings(lib):
+    for s in range(7):
+        assert lib.e4b_status_string(s)
+
+
+def test_host_side_validation(lib):
+    L = lib.lib
+    nullp = None
+    # quantize / dequantize: blocksize and in_features rules, null pointers
+    assert L.e4b_quantize_nf4(nullp, 1, 2, 64, 32, 0, nullp, nullp, nullp) == lib.E4B_ERR_BLOCKSIZE
+    assert L.e4b_quantize_nf4(nullp, 1, 2, 96, 64, 0, nullp, nullp, nullp) == lib.E4B_ERR_BLOCKSIZE
+    assert L.e4b_quantize_nf4(nullp, 1, 2, 64, 64, 0, nullp, nullp, nullp) == lib.E4B_ERR_INVALID_ARG
+    assert L.e4b_quantize_nf4(nullp, 1, 2, 64, 64, 5, nullp, nullp, nullp) == lib.E4B_ERR_INVALID_ARG
+    assert L.e4b_quantize_nf4(nullp, 0, 2, 64, 64, 0, nullp, nullp, nullp) == lib.E4B_OK   # empty
+    assert L.e4b_dequantize_nf4(nullp, nullp, 1, 2, 96, 64, 0, 1, nullp, nullp) == lib.E4B_ERR_BLOCKSIZE
+    assert L.e4b_dequantize_nf4(nullp, nullp, 1, 2, 64, 64, 0, 7, nullp, nullp) == lib.E4B_ERR_INVALID_ARG
+    # layer descriptions
+    d = lib.make_desc(8, 256, 512, 2)
+    assert lib.e4b_moe_workspace_size(d, 64) > 0
+    for bad, code in ((lib.make_desc(8, 250, 512, 2), 0), (lib.make_desc(8, 256, 512, 9), 0),
+                      (lib.make_desc(4, 256, 512, 5), 0), (lib.make_desc(300, 256, 512, 2), 0),
+                      (lib.make_desc(8, 256, 512, 2, blocksize=128), 0)):
+        assert lib.e4b_moe_workspace_size(bad, 64) == code
+    ex = lib.e4b_experts(None, None, None, None)
+    st = lambda: L.e4b_moe_forward(ctypes.byref(d), ctypes.byref(ex), None, 4, None, None, None, None, None,
+                                   None, None, None, 0, None)
+    assert st() == lib.E4B_ERR_INVALID_ARG
+    ex2 = lib.e4b_experts(16, 16, 16, 16)   # non-null dummies: never dereferenced on these paths
+    f = lambda dd, T, x, ws, n: L.e4b_moe_forward(ctypes.byref(dd), ctypes.byref(ex2), x, T, None, 16, 16, 16, None,
+                                                  None, None, ws, n, None)
+    assert f(d, 0, None, None, 0) == lib.E4B_OK                        # T == 0: no-op
+    assert f(d, 4, None, 16, 1 << 30) == lib.E4B_ERR_INVALID_ARG       # null x
+    assert f(d, 4, 16, None, 0) == lib.E4B_ERR_WORKSPACE               # no workspace
+    assert f(d, 4, 16, 16, 10) == lib.E4B_ERR_WORKSPACE                # workspace too small
+    bad_bs = lib.make_desc(8, 256, 512, 2, blocksize=32)
+    assert f(bad_bs, 4, 16, 16, 1 << 30) == lib.E4B_ERR_BLOCKSIZE
+    bad_h = lib.make_desc(8, 96, 512, 2)
+    assert f(bad_h, 4, 16, 16, 1 << 30) == lib.E4B_ERR_BLOCKSIZE
+    dec = lib.make_desc(8, 256, 512, 2, path=lib.PATH_DECODE)
+    assert f(dec, 9, 16, 16, 1 << 40) == lib.E4B_ERR_UNSUPPORTED       # decode path is for T <= 8
+    g = lambda dd, T: L.e4b_moe_backward_dgrad(ctypes.byref(dd), ctypes.byref(ex2), None, T, 16, 16, 16, None, 16,
+                                               16, 1 << 40, None)
+    assert g(d, 4) == lib.E4B_ERR_INVALID_ARG                          # needs x when saved_gu is NULL
+    assert g(d, 0) == lib.E4B_OK
