@@ -51,6 +51,24 @@ def dist_env():
     return world, rank, local
 
 
+def max_over_ranks(value: float, device=None) -> float:
+    """Max of a per-rank number over all ranks (identity when not distributed).
+    NCCL reduces on the rank's GPU, gloo on the host."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return value
+    dev = device if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([value], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(tokens_per_rank: int, world: int, ms_per_step: float) -> float:
+    """Whole-job tokens/s: every rank processes its own batch each step (weak scaling)."""
+    return world * tokens_per_rank / (ms_per_step / 1e3)
+
+
 def peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(path):
@@ -287,13 +305,9 @@ def run_e4b(args, w):
     if world > 1:
         torch.distributed.barrier()
     step_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
-    total_ms = sum(step_ms)
-    if world > 1:
-        t = torch.tensor([total_ms], device=dev, dtype=torch.float64)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        total_ms = float(t.item())
+    total_ms = max_over_ranks(sum(step_ms), dev)
     ms_per_step = total_ms / args.steps
-    value = world * T / (ms_per_step / 1e3)
+    value = job_throughput(T, world, ms_per_step)
 
     kernels = {}
     for name in ("gemm_gateup", "gemm_down", "gemm_dgrad_down", "gemm_dgrad_gateup", "route", "group", "gather",
@@ -337,14 +351,10 @@ def run_e4b(args, w):
             e2e_step()
         ee.record(stream)
         torch.cuda.synchronize()
-        e2e_ms = es.elapsed_time(ee) / args.steps
-        if world > 1:
-            t = torch.tensor([e2e_ms], device=dev, dtype=torch.float64)
-            torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-            e2e_ms = float(t.item())
+        e2e_ms = max_over_ranks(es.elapsed_time(ee) / args.steps, dev)
         h2d = x_p.numel() * 2 + l_p.numel() * 4 + g_p.numel() * 2
         d2h = y_p.numel() * 2 + gx_p.numel() * 2
-        e2e = {"value": world * T / (e2e_ms / 1e3), "unit": UNIT, "h2d_bytes_per_step": h2d,
+        e2e = {"value": job_throughput(T, world, e2e_ms), "unit": UNIT, "h2d_bytes_per_step": h2d,
                "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms}
 
     if e4b.e4b_device_status() != e4b.E4B_OK:
