@@ -21,7 +21,6 @@ import hashlib
 import json
 import os
 import statistics
-import subprocess
 import sys
 import time
 
@@ -98,55 +97,62 @@ def recorded_traffic(kernel: str, workload: str):
 
 
 class ClockSampler:
-    """nvidia-smi clocks and throttle reasons sampled while the timed region runs."""
-    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
-         "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
-         "clocks_event_reasons.sw_power_cap")
+    """SM clock, power and clock-event (throttle) reasons sampled through NVML by a
+    host thread every ~1 ms while the timed region runs (read-only queries)."""
+    # NVML clock-event reason bits
+    REASONS = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown",
+               0x80: "hw_power_brake_slowdown"}
 
-    def __init__(self, gpu_index: int):
-        self.idx = gpu_index
-        self.proc = None
+    def __init__(self, torch_device):
+        self.dev = torch_device
+        self.samples = []
+        self.smax = None
+        self._stop = None
+        self._thr = None
 
     def __enter__(self):
+        import threading
         try:
-            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.idx), f"--query-gpu={self.Q}",
-                                          "--format=csv,noheader,nounits", "-lms", "200"],
-                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            import pynvml
+            import torch
+            pynvml.nvmlInit()
+            uuid = str(torch.cuda.get_device_properties(self.dev).uuid)
+            h = pynvml.nvmlDeviceGetHandleByUUID(uuid if uuid.startswith("GPU-") else "GPU-" + uuid)
+            self.smax = pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM)
+            get_reasons = getattr(pynvml, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+                pynvml.nvmlDeviceGetCurrentClocksThrottleReasons
         except Exception:
-            self.proc = None
+            return self
+        self._stop = threading.Event()
+
+        def loop():
+            while not self._stop.is_set():
+                try:
+                    self.samples.append((pynvml.nvmlDeviceGetClockInfo(h, pynvml.NVML_CLOCK_SM),
+                                         pynvml.nvmlDeviceGetPowerUsage(h) / 1000.0, int(get_reasons(h))))
+                except Exception:
+                    pass
+                time.sleep(0.001)
+        self._thr = threading.Thread(target=loop, daemon=True)
+        self._thr.start()
         return self
 
     def __exit__(self, *a):
-        self.out = ""
-        if self.proc is not None:
-            self.proc.terminate()
-            try:
-                self.out, _ = self.proc.communicate(timeout=5)
-            except Exception:
-                self.proc.kill()
+        if self._thr is not None:
+            self._stop.set()
+            self._thr.join(timeout=5)
 
     def summary(self):
-        rows = []
-        for line in (self.out or "").splitlines():
-            f = [x.strip() for x in line.split(",")]
-            if len(f) < 9:
-                continue
-            try:
-                rows.append(dict(sm=float(f[1]), smax=float(f[2]), power=float(f[3]), hw=f[5], hwt=f[6], swt=f[7],
-                                 swp=f[8]))
-            except ValueError:
-                continue
-        if not rows:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
-        loaded = [r for r in rows if r["power"] > 200] or rows
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.smax, "reasons": ["unsampled"]}
         reasons = set()
-        for r in rows:
-            for key, name in (("hw", "hw_slowdown"), ("hwt", "hw_thermal_slowdown"), ("swt", "sw_thermal_slowdown"),
-                              ("swp", "sw_power_cap")):
-                if r[key].lower() == "active":
+        for _, _, r in self.samples:
+            for bit, name in self.REASONS.items():
+                if r & bit:
                     reasons.add(name)
-        return {"sm_mhz": statistics.median(r["sm"] for r in loaded), "sm_max_mhz": max(r["smax"] for r in rows),
-                "reasons": sorted(reasons), "samples": len(rows)}
+        return {"sm_mhz": statistics.median(s[0] for s in self.samples), "sm_max_mhz": self.smax,
+                "reasons": sorted(reasons), "samples": len(self.samples),
+                "power_w_max": max(s[1] for s in self.samples)}
 
 
 # ------------------------------------------------------------------ CPU oracle
@@ -292,7 +298,7 @@ def run_e4b(args, w):
         torch.distributed.barrier()
     torch.cuda.synchronize()
     launches0 = e4b.e4b_launch_count()
-    with ClockSampler(local) as clk:
+    with ClockSampler(dev) as clk:
         e4b.e4b_timing_enable(True)
         for i in range(args.steps):
             flush.zero_()                       # evict L2 between timed steps (not timed)

@@ -94,7 +94,7 @@ uint32_t* device_status_ptr() {
 
 // ------------------------------------------------------------ workspace layout
 struct WsLayout {
-    size_t chunk_counts, chunk_base, counts, offsets, tile_prefix, perm, a_perm, h, gu, dgu, acc32, dec_h, total;
+    size_t chunk_counts, chunk_base, counts, offsets, tile_prefix, sched, perm, a_perm, h, gu, dgu, dec_h, total;
 };
 
 static size_t align_up(size_t v) { return (v + 255) & ~size_t(255); }
@@ -110,12 +110,12 @@ static WsLayout layout_for(const e4b_moe_desc* d, int64_t T) {
     L.counts = take((size_t)d->E * 4);
     L.offsets = take((size_t)(d->E + 1) * 4);
     L.tile_prefix = take((size_t)(d->E + 1) * 4);
+    L.sched = take(((size_t)(P + gemm_tile_rows() - 1) / gemm_tile_rows() + d->E) * 16);
     L.perm = take((size_t)P * 4);
     L.a_perm = take((size_t)P * d->H * 2);
     L.h = take((size_t)P * d->I * 2);
     L.gu = take((size_t)P * 2 * d->I * 2);
     L.dgu = take((size_t)P * 2 * d->I * 2);
-    L.acc32 = take((size_t)T * d->H * 4);
     L.dec_h = take((size_t)P * d->I * 4);
     L.total = off;
     return L;
@@ -149,6 +149,7 @@ static GemmParams base_params(const e4b_moe_desc* d, uint8_t* ws, const WsLayout
     p.k_top = d->top_k;
     p.offsets = reinterpret_cast<const int*>(ws + L.offsets);
     p.tile_prefix = reinterpret_cast<const int*>(ws + L.tile_prefix);
+    p.sched = reinterpret_cast<const int4*>(ws + L.sched);
     p.perm = reinterpret_cast<const int*>(ws + L.perm);
     p.topk_w = topk_w;
     p.status = device_status_ptr();
@@ -306,12 +307,12 @@ e4b_status e4b_moe_forward(const e4b_moe_desc* d, const e4b_experts* w, const vo
     int32_t* perm = reinterpret_cast<int32_t*>(ws + L.perm);
     E4B_CUDA_TRY(launch_group(topk_idx, P, d->E, gemm_tile_rows(), reinterpret_cast<int32_t*>(ws + L.chunk_counts),
                               reinterpret_cast<int32_t*>(ws + L.chunk_base), reinterpret_cast<int32_t*>(ws + L.counts),
-                              offsets, reinterpret_cast<int32_t*>(ws + L.tile_prefix), perm, st));
+                              offsets, reinterpret_cast<int32_t*>(ws + L.tile_prefix),
+                              reinterpret_cast<int4*>(ws + L.sched), perm, st));
     E4B_CUDA_TRY(launch_gather_rows(static_cast<const __nv_bfloat16*>(x), perm, offsets + d->E, d->top_k, P, d->H,
                                     reinterpret_cast<__nv_bfloat16*>(ws + L.a_perm), st));
-    float* acc = reinterpret_cast<float*>(ws + L.acc32);
-    E4B_CUDA_TRY(cudaMemsetAsync(acc, 0, (size_t)T * d->H * 4, st));
     __nv_bfloat16* h = reinterpret_cast<__nv_bfloat16*>(ws + L.h);
+    __nv_bfloat16* slots = reinterpret_cast<__nv_bfloat16*>(ws + L.a_perm);   // X_perm is dead after gate_up
     if ((s = run_gateup(d, w, ws, L, topk_w, P, h, static_cast<__nv_bfloat16*>(saved_gu), st)) != E4B_OK) return s;
 
     GemmParams p = base_params(d, ws, L, topk_w, P);
@@ -322,11 +323,11 @@ e4b_status e4b_moe_forward(const e4b_moe_desc* d, const e4b_experts* w, const vo
     p.b_rows_per_expert = d->H;
     p.b_rows_total = (int64_t)d->E * d->H;
     p.b_blocks_per_row = d->I / 64;
-    p.out_f32 = acc;
+    p.out_bf16 = slots;
     p.ld_out = d->H;
     E4B_CUDA_TRY(launch_grouped_gemm(EPI_DOWN, d->codebook, h, P, w->down, p.b_rows_total, d->I / 2, p,
                                      max_m_tiles(P, d->E), st));
-    E4B_CUDA_TRY(launch_f32_to_bf16(acc, T * d->H, static_cast<__nv_bfloat16*>(y), st));
+    E4B_CUDA_TRY(launch_combine(slots, topk_idx, d->E, d->top_k, T, d->H, static_cast<__nv_bfloat16*>(y), st));
     if (offsets_out) E4B_CUDA_TRY(cudaMemcpyAsync(offsets_out, offsets, (d->E + 1) * 4, cudaMemcpyDeviceToDevice, st));
     if (perm_out) E4B_CUDA_TRY(cudaMemcpyAsync(perm_out, perm, P * 4, cudaMemcpyDeviceToDevice, st));
     return E4B_OK;
@@ -351,7 +352,7 @@ e4b_status e4b_moe_backward_dgrad(const e4b_moe_desc* d, const e4b_experts* w, c
     E4B_CUDA_TRY(launch_group(topk_idx, P, d->E, gemm_tile_rows(), reinterpret_cast<int32_t*>(ws + L.chunk_counts),
                               reinterpret_cast<int32_t*>(ws + L.chunk_base), reinterpret_cast<int32_t*>(ws + L.counts),
                               reinterpret_cast<int32_t*>(ws + L.offsets), reinterpret_cast<int32_t*>(ws + L.tile_prefix),
-                              perm, st));
+                              reinterpret_cast<int4*>(ws + L.sched), perm, st));
     __nv_bfloat16* a_perm = reinterpret_cast<__nv_bfloat16*>(ws + L.a_perm);
     const int32_t* nrows = reinterpret_cast<const int32_t*>(ws + L.offsets) + d->E;
     const __nv_bfloat16* gu = static_cast<const __nv_bfloat16*>(saved_gu);
@@ -363,8 +364,6 @@ e4b_status e4b_moe_backward_dgrad(const e4b_moe_desc* d, const e4b_experts* w, c
         gu = gu_ws;
     }
     E4B_CUDA_TRY(launch_gather_rows(static_cast<const __nv_bfloat16*>(grad_out), perm, nrows, d->top_k, P, d->H, a_perm, st));
-    float* acc = reinterpret_cast<float*>(ws + L.acc32);
-    E4B_CUDA_TRY(cudaMemsetAsync(acc, 0, (size_t)T * d->H * 4, st));
     __nv_bfloat16* dgu = reinterpret_cast<__nv_bfloat16*>(ws + L.dgu);
 
     GemmParams p = base_params(d, ws, L, topk_w, P);   // dh = w * grad_out W_down, then SwiGLU backward
@@ -389,11 +388,11 @@ e4b_status e4b_moe_backward_dgrad(const e4b_moe_desc* d, const e4b_experts* w, c
     q.b_rows_per_expert = 2 * d->I;
     q.b_rows_total = (int64_t)d->E * 2 * d->I;
     q.b_blocks_per_row = d->H / 64;
-    q.out_f32 = acc;
+    q.out_bf16 = a_perm;   // slot rows; the gathered grad_out is dead after the first GEMM
     q.ld_out = d->H;
     E4B_CUDA_TRY(launch_grouped_gemm(EPI_DGRAD_GATEUP, d->codebook, dgu, P, w->gate_up, q.b_rows_total, d->H / 2, q,
                                      max_m_tiles(P, d->E), st));
-    E4B_CUDA_TRY(launch_f32_to_bf16(acc, T * d->H, static_cast<__nv_bfloat16*>(grad_x), st));
+    E4B_CUDA_TRY(launch_combine(a_perm, topk_idx, d->E, d->top_k, T, d->H, static_cast<__nv_bfloat16*>(grad_x), st));
     return E4B_OK;
 }
 

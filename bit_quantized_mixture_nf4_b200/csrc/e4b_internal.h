@@ -17,7 +17,8 @@ enum Epi { EPI_GATEUP = 0, EPI_DOWN = 1, EPI_DGRAD_DOWN = 2, EPI_DGRAD_GATEUP = 
 struct GemmParams {
     int E, K, N, n_tiles, k_top;
     const int* offsets;       // [E+1] first grouped row of each expert
-    const int* tile_prefix;   // [E+1] prefix of ceil(M_e / 128); [E] = total m-tiles
+    const int* tile_prefix;   // [E+1] prefix of ceil(M_e / tile_rows); [E] = total m-tiles
+    const int4* sched;        // per m-tile: (expert, first row, rows, 0)
     const int* perm;          // [P] pair id of each grouped row
     const float* topk_w;      // [P] routing weight by pair id
     const float* absmax;      // absmax of the weight stack
@@ -25,9 +26,9 @@ struct GemmParams {
     int b_rows_per_expert;
     int b_blocks_per_row;     // stored cols / 64
     int up_offset;            // I (EPI_GATEUP: first up row; also the feature count)
-    __nv_bfloat16* out_bf16;  // h [P, I] or dGU [P, 2I]
-    __nv_bfloat16* gu;        // saved gate/up [P, 2I] (written by EPI_GATEUP, read by EPI_DGRAD_DOWN)
-    float* out_f32;           // [T, H] fp32 accumulation target
+    __nv_bfloat16* out_bf16;  // h [P, I], dGU [P, 2I], or the slot rows [P, H] (down / dgrad gate_up)
+    __nv_bfloat16* gu;        // saved SwiGLU derivatives [P, 2I]: dh/dg | dh/du (written by EPI_GATEUP,
+                              // read by EPI_DGRAD_DOWN)
     int ld_out;
     uint32_t* status;         // device status word
 };
@@ -54,13 +55,17 @@ constexpr int kChunkPairs = 2048;
 cudaError_t launch_route(const float* logits, int64_t T, int E, int k, int renorm, int32_t* idx, float* w,
                          cudaStream_t st);
 // counts/offsets/tile_prefix/perm from topk_idx; chunk scratch: [nchunks * E] ints x2
+// sched: [ceil(P/tile_rows) + E] m-tile entries (expert, first row, rows, 0)
 cudaError_t launch_group(const int32_t* idx, int64_t P, int E, int tile_rows, int32_t* chunk_counts,
                          int32_t* chunk_base, int32_t* counts, int32_t* offsets, int32_t* tile_prefix,
-                         int32_t* perm, cudaStream_t st);
+                         int4* sched, int32_t* perm, cudaStream_t st);
 // nrows: device pointer to the number of grouped rows (offsets[E])
 cudaError_t launch_gather_rows(const __nv_bfloat16* src, const int32_t* perm, const int32_t* nrows, int k,
                                int64_t P, int H, __nv_bfloat16* dst, cudaStream_t st);
 cudaError_t launch_f32_to_bf16(const float* src, int64_t n, __nv_bfloat16* dst, cudaStream_t st);
+// y[t] = sum over the k slot rows of token t (fp32 sum in slot order, bf16 result)
+cudaError_t launch_combine(const __nv_bfloat16* slots, const int32_t* idx, int E, int k, int64_t T, int H,
+                           __nv_bfloat16* y, cudaStream_t st);
 
 // grouped_gemm.cu
 int gemm_tile_rows();

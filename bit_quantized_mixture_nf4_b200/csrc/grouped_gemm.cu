@@ -7,122 +7,155 @@
 // backward input gradient).  Rows are routed (token, slot) pairs in grouped
 // order, so expert e owns the contiguous rows [offsets[e], offsets[e+1]).
 //
-//   EPI_GATEUP        D = X_e W_gu,e^T ; epilogue h = silu(g)*u (+ saves g,u)
-//   EPI_DOWN          D = h_e W_d,e^T  ; epilogue y32[token] += w * D (atomic fp32)
-//   EPI_DGRAD_DOWN    D = dY_e W_d,e   ; epilogue dh = w*D, dG/dU (SwiGLU backward)
-//   EPI_DGRAD_GATEUP  D = dGU_e W_gu,e ; epilogue gx32[token] += D (atomic fp32)
+//   EPI_GATEUP        D = X_e W_gu,e^T ; epilogue h = silu(g)*u (+ saves dh/dg, dh/du)
+//   EPI_DOWN          D = h_e W_d,e^T  ; epilogue slot[pair] = bf16(w * D)
+//   EPI_DGRAD_DOWN    D = dY_e W_d,e   ; epilogue dh = w*D, dG = dh*dh/dg, dU = dh*dh/du
+//   EPI_DGRAD_GATEUP  D = dGU_e W_gu,e ; epilogue slot[pair] = bf16(D)
+// The slot rows of a token are summed in fp32, in slot order, by combine_kernel.
 //
-// Tile: 128 rows x 256 columns x 64-deep k-stages, 4-stage smem ring.
-//   warp 4      TMA producer: A tile (bf16, 128B swizzle) + packed 4-bit weight tile
-//   warps 8-15  dequantize the packed tile into a bf16 operand tile in smem, in the
-//               tensor cores' 128B-swizzled layout: K-major for the forward (weights
-//               stored [N, K]) and MN-major for the input gradient (weights used
-//               transposed, stored [K, N]); the transposition costs nothing
-//   warp 5      one thread issues tcgen05.mma (M=128, N=256, K=16) into TMEM
-//   warps 0-3   epilogue: tcgen05.ld from TMEM (double-buffered accumulator, 2x256
-//               columns) and the fused elementwise/scatter work
-// Every wait is bounded; on expiry the kernel records a timeout and exits.
+// Tile: (128*CTAS) rows x 256 columns, 64-deep k-stages.  With CTAS = 2 a
+// cluster of two CTAs on two SMs computes one 256-row tile with
+// tcgen05.mma.cta_group::2 (M = 256): each CTA holds 128 rows of A and HALF of
+// the dequantized B tile, so each SM dequantizes only 128 x 64 weights per
+// 512-clock stage and the B operand is read from shared memory once for both.
+// Roles per CTA (512 threads):
+//   warp 4      TMA producer: A tile (bf16, 128B swizzle) and packed 4-bit B tile
+//   warps 8-15  two groups of 4 warps, alternating k-stages: each thread turns one
+//               64-element block (one absmax) of packed codes into bf16 in the
+//               tensor cores' 128B-swizzled layout -- K-major for the forward
+//               (weights stored [N, K]), MN-major for the input gradient (weights
+//               used transposed, stored [K, N]; the transposition costs nothing)
+//   warp 5      one thread of the first CTA issues the MMAs into TMEM
+//               (double-buffered accumulator, 2 x 256 columns)
+//   warps 0-3   epilogue: tcgen05.ld of this CTA's 128 accumulator rows
+// Every mbarrier wait is bounded; on expiry the kernel records a timeout and exits.
 #include "e4b_internal.h"
 
 namespace e4b {
 
-constexpr int BM = 128, BN = 256, BK = 64, STAGES = 4;
-constexpr int A_STAGE_BYTES = BM * BK * 2;       // 16 KB
-constexpr int B_STAGE_BYTES = BN * BK * 2;       // 32 KB
-constexpr int RAW_STAGE_BYTES = BN * BK / 2;     //  8 KB
+constexpr int BN = 256, BK = 64;
 constexpr int GEMM_THREADS = 512;
-constexpr int PRODUCER_WARP = 4, MMA_WARP = 5, DEQ_WARP0 = 8;
-constexpr int TMEM_COLS = 2 * BN;                // two accumulator buffers
-constexpr int SMEM_DATA = STAGES * (A_STAGE_BYTES + B_STAGE_BYTES + RAW_STAGE_BYTES);
-constexpr int GEMM_SMEM_BYTES = SMEM_DATA + 1024 /*alignment slack*/ + 256 /*barriers*/;
+constexpr int PRODUCER_WARP = 4, MMA_WARP = 5, RAW_WARP = 6, DEQ_WARP0 = 8;
+constexpr int TMEM_COLS = 2 * BN;   // two accumulator buffers
+
+template <int CTAS>
+struct Cfg {
+    static constexpr int TILE_M = 128 * CTAS;            // rows per tile (all CTAs of the cluster)
+    static constexpr int N_CTA = BN / CTAS;              // B columns dequantized by one CTA
+    static constexpr int A_BYTES = 128 * BK * 2;         // this CTA's 128 A rows
+    static constexpr int B_BYTES = N_CTA * BK * 2;
+    static constexpr int RAW_BYTES = N_CTA * BK / 2;
+    static constexpr int ASTAGES = (CTAS == 2) ? 7 : 4;    // A (activation) ring: TMA latency under load
+    static constexpr int STAGES = (CTAS == 2) ? 4 : 2;     // dequantized-B ring
+    static constexpr int RSTAGES = (CTAS == 2) ? 8 : 6;    // packed-weight ring, prefetched far ahead
+    static constexpr int AM_BYTES = N_CTA * 4;             // the stage's absmax values, one per block
+    static constexpr int RAW_STAGE = RAW_BYTES + AM_BYTES;
+    static constexpr int BLK_PER_THREAD = N_CTA / 128;   // 64-element blocks per dequant thread per stage
+    static constexpr int SMEM_BYTES = ASTAGES * A_BYTES + STAGES * B_BYTES + RSTAGES * RAW_STAGE + 1024 + 1024;
+};
 
 struct SmemCtl {
-    uint64_t full_tma[STAGES];
-    uint64_t full_b[STAGES];
-    uint64_t empty[STAGES];
+    uint64_t a_full[8];
+    uint64_t b_full[8];
+    uint64_t empty[8];        // dequantized-B stage consumed (MMA commit)
+    uint64_t a_empty[8];      // A stage consumed (MMA commit)
+    uint64_t raw_full[16];
+    uint64_t raw_empty[16];
     uint64_t acc_full[2];
     uint64_t acc_empty[2];
     uint32_t tmem_base;
     int abort_flag;
 };
-static_assert(sizeof(SmemCtl) <= 256, "control block");
+static_assert(sizeof(SmemCtl) <= 1024, "control block");
 
 struct TileInfo {
     int e, row0, rows, nt;
 };
 
+// One load: the m-tile schedule written by the grouping scan.
 __device__ __forceinline__ TileInfo decode_tile(const GemmParams& p, int tile) {
     const int mt = tile / p.n_tiles;
-    TileInfo ti;
-    ti.nt = tile - mt * p.n_tiles;
-    int lo = 0, hi = p.E;   // tile_prefix[lo] <= mt < tile_prefix[hi]
-    while (hi - lo > 1) {
-        const int mid = (lo + hi) >> 1;
-        if (__ldg(p.tile_prefix + mid) <= mt) lo = mid; else hi = mid;
-    }
-    ti.e = lo;
-    ti.row0 = __ldg(p.offsets + lo) + (mt - __ldg(p.tile_prefix + lo)) * BM;
-    ti.rows = min(BM, __ldg(p.offsets + lo + 1) - ti.row0);
-    return ti;
+    const int4 v = __ldg(p.sched + mt);
+    return TileInfo{v.x, v.y, v.z, tile - mt * p.n_tiles};
 }
 
-// Stored weight row (within one expert) that feeds operand row n (K-major mode).
+// Stored weight row (within one expert) feeding B column `n` (0..255) of tile nt (K-major mode).
 template <int EPI>
-__device__ __forceinline__ int kmajor_row(const GemmParams& p, const TileInfo& ti, int n) {
+__device__ __forceinline__ int kmajor_row(const GemmParams& p, int nt, int n) {
     if (EPI == EPI_GATEUP)   // 128 gate rows, then the matching 128 up rows
-        return (n < 128) ? ti.nt * 128 + n : p.up_offset + ti.nt * 128 + (n - 128);
-    return ti.nt * BN + n;
+        return (n < 128) ? nt * 128 + n : p.up_offset + nt * 128 + (n - 128);
+    return nt * BN + n;
 }
 
-// absmax feeding this dequant thread's 64-element block for k-stage ks.
-template <int EPI>
-__device__ __forceinline__ float load_absmax(const GemmParams& p, const TileInfo& ti, int ks, int t) {
+// Index into the absmax array of 64-element block b (0..N_CTA-1) of this CTA's B
+// half at k-stage ks, or -1 outside the stored matrix.
+//   K-major:  block b = B column (rank*N_CTA + b), k-block ks
+//   MN-major: block b = (k-row b & 63, n-block b >> 6 of this CTA's half)
+template <int EPI, int CTAS>
+__device__ __forceinline__ int64_t absmax_index(const GemmParams& p, const TileInfo& ti, int ks, int b, int rank) {
     int64_t row;
     int blk;
-    if (EPI == EPI_GATEUP || EPI == EPI_DOWN) {         // blocks run along K
-        row = (int64_t)ti.e * p.b_rows_per_expert + kmajor_row<EPI>(p, ti, t);
+    if (EPI == EPI_GATEUP || EPI == EPI_DOWN) {
+        row = (int64_t)ti.e * p.b_rows_per_expert + kmajor_row<EPI>(p, ti.nt, rank * Cfg<CTAS>::N_CTA + b);
         blk = ks;
-    } else {                                           // blocks run along N
-        row = (int64_t)ti.e * p.b_rows_per_expert + (int64_t)ks * BK + (t >> 2);
-        blk = ti.nt * (BN / 64) + (t & 3);
-        if (blk >= p.b_blocks_per_row) return 0.0f;
+    } else {
+        row = (int64_t)ti.e * p.b_rows_per_expert + (int64_t)ks * BK + (b & 63);
+        blk = (ti.nt * BN + rank * Cfg<CTAS>::N_CTA) / 64 + (b >> 6);
+        if (blk >= p.b_blocks_per_row) return -1;
     }
-    if (row >= p.b_rows_total) return 0.0f;
-    return __ldg(p.absmax + row * p.b_blocks_per_row + blk);
+    if (row >= p.b_rows_total) return -1;
+    return row * p.b_blocks_per_row + blk;
 }
 
-__device__ __forceinline__ float silu_f(float g) { return g / (1.0f + __expf(-g)); }
-
-template <int EPI, int CB>
+template <int EPI, int CB, int CTAS>
 __global__ void __launch_bounds__(GEMM_THREADS, 1)
 grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_raw,
                     const GemmParams p) {
+    using C = Cfg<CTAS>;
+    constexpr int STAGES = C::STAGES;
+    constexpr int ASTAGES = C::ASTAGES;
+    constexpr bool kMajorB = (EPI == EPI_GATEUP || EPI == EPI_DOWN);
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t* sA = smem;
-    uint8_t* sB = smem + STAGES * A_STAGE_BYTES;
-    uint8_t* sRaw = sB + STAGES * B_STAGE_BYTES;
-    SmemCtl* ctl = reinterpret_cast<SmemCtl*>(sRaw + STAGES * RAW_STAGE_BYTES);
+    uint8_t* sB = sA + ASTAGES * C::A_BYTES;
+    uint8_t* sRaw = sB + STAGES * C::B_BYTES;
+    SmemCtl* ctl = reinterpret_cast<SmemCtl*>(sRaw + C::RSTAGES * C::RAW_STAGE);
+    constexpr int RSTAGES = C::RSTAGES;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    constexpr bool kMajorB = (EPI == EPI_GATEUP || EPI == EPI_DOWN);
+    const uint32_t rank = (CTAS == 2) ? cluster_ctarank() : 0u;
+    const bool leader = rank == 0;
+    const int cluster_id = blockIdx.x / CTAS, nclusters = gridDim.x / CTAS;
 
     if (threadIdx.x == 0) {
+        for (int s = 0; s < ASTAGES; ++s) {
+            mbar_init(smem_u32(&ctl->a_full[s]), 1);               // producer of the first CTA
+            mbar_init(smem_u32(&ctl->a_empty[s]), 1);              // MMA commit
+        }
         for (int s = 0; s < STAGES; ++s) {
-            mbar_init(smem_u32(&ctl->full_tma[s]), 1);
-            mbar_init(smem_u32(&ctl->full_b[s]), 8);      // one arrival per dequant warp
-            mbar_init(smem_u32(&ctl->empty[s]), 1);       // tcgen05.commit
+            mbar_init(smem_u32(&ctl->b_full[s]), 4 * CTAS);        // one dequant group in each CTA
+            mbar_init(smem_u32(&ctl->empty[s]), 1);                // MMA commit
+        }
+        for (int s = 0; s < RSTAGES; ++s) {
+            mbar_init(smem_u32(&ctl->raw_full[s]), 1 + 32);        // TMA + the producer warp's absmax copies
+            mbar_init(smem_u32(&ctl->raw_empty[s]), 4);            // the dequant group that read it
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(smem_u32(&ctl->acc_full[b]), 1);
-            mbar_init(smem_u32(&ctl->acc_empty[b]), 4);   // one arrival per epilogue warp
+            mbar_init(smem_u32(&ctl->acc_empty[b]), 4 * CTAS);     // epilogue warps of all CTAs
         }
         ctl->abort_flag = 0;
         fence_barrier_init();
     }
     if (warp == MMA_WARP) {
-        tmem_alloc(smem_u32(&ctl->tmem_base), TMEM_COLS);
-        tmem_relinquish();
+        if (CTAS == 2) {
+            tmem_alloc_pair(smem_u32(&ctl->tmem_base), TMEM_COLS);
+            tmem_relinquish_pair();
+        } else {
+            tmem_alloc(smem_u32(&ctl->tmem_base), TMEM_COLS);
+            tmem_relinquish();
+        }
     }
     if (warp == PRODUCER_WARP && lane == 0) {
         tma_prefetch_desc(&tmap_a);
@@ -130,121 +163,252 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_con
     }
     tc_fence_before();
     __syncthreads();
+    if (CTAS == 2) cluster_sync_all();   // peer barriers initialised before any remote arrive
     tc_fence_after();
     const uint32_t tmem_base = ctl->tmem_base;
     volatile int* abort_flag = &ctl->abort_flag;
+    auto wait = [&](uint64_t* bar, uint32_t parity) -> bool {
+        return mbar_wait(smem_u32(bar), parity, abort_flag, p.status);
+    };
+    // arrive on a barrier of the cluster's first CTA
+    auto arrive_leader = [&](uint64_t* bar) {
+        if (CTAS == 2 && !leader) mbar_arrive_cluster(mapa_shared(smem_u32(bar), 0));
+        else mbar_arrive(smem_u32(bar));
+    };
 
     const int total_tiles = __ldg(p.tile_prefix + p.E) * p.n_tiles;
     const int nk = p.K / BK;
 
     if (warp == PRODUCER_WARP) {
+        // A tiles: refilled as soon as the MMA has released a stage.  Each tile is also
+        // prefetched into L2 APF stages before its load, which hides the long HBM
+        // latency of the gathered activation rows without more shared memory.
         if (lane == 0) {
+            constexpr int APF = 8;
+            const int a_off = 128 * (int)rank;
+            int pf_tile = cluster_id, pf_ks = 0;
+            TileInfo pf_ti{};
+            if (pf_tile < total_tiles) pf_ti = decode_tile(p, pf_tile);
+            auto prefetch_next = [&]() {
+                if (pf_tile >= total_tiles) return;
+                tma_prefetch_l2_2d(&tmap_a, pf_ks * BK, pf_ti.row0 + a_off);
+                if (++pf_ks == nk) {
+                    pf_ks = 0;
+                    pf_tile += nclusters;
+                    if (pf_tile < total_tiles) pf_ti = decode_tile(p, pf_tile);
+                }
+            };
+            for (int i = 0; i < APF; ++i) prefetch_next();
             uint32_t it = 0;
             bool ok = true;
-            for (int tile = blockIdx.x; tile < total_tiles && ok; tile += gridDim.x) {
+            for (int tile = cluster_id; tile < total_tiles && ok; tile += nclusters) {
                 const TileInfo ti = decode_tile(p, tile);
                 for (int ks = 0; ks < nk; ++ks, ++it) {
-                    const int s = it % STAGES;
-                    const uint32_t r = it / STAGES;
-                    if (!mbar_wait(smem_u32(&ctl->empty[s]), (r & 1) ^ 1, abort_flag, p.status)) { ok = false; break; }
-                    const uint32_t fb = smem_u32(&ctl->full_tma[s]);
-                    mbar_arrive_expect_tx(fb, A_STAGE_BYTES + RAW_STAGE_BYTES);
-                    tma_load_2d(smem_u32(sA + s * A_STAGE_BYTES), &tmap_a, fb, ks * BK, ti.row0);
-                    const uint32_t raw = smem_u32(sRaw + s * RAW_STAGE_BYTES);
-                    if (kMajorB) {
-                        const int y0 = ti.e * p.b_rows_per_expert + kmajor_row<EPI>(p, ti, 0);
-                        const int y1 = ti.e * p.b_rows_per_expert + kmajor_row<EPI>(p, ti, 128);
-                        tma_load_2d(raw, &tmap_raw, fb, ks * (BK / 2), y0);
-                        tma_load_2d(raw + RAW_STAGE_BYTES / 2, &tmap_raw, fb, ks * (BK / 2), y1);
+                    prefetch_next();
+                    const int s = it % ASTAGES;
+                    const uint32_t r = it / ASTAGES;
+                    if (!wait(&ctl->a_empty[s], (r & 1) ^ 1)) { ok = false; break; }
+                    const uint32_t a_dst = smem_u32(sA + s * C::A_BYTES);
+                    const int a_row = ti.row0 + a_off;
+                    if (CTAS == 2) {
+                        if (leader) mbar_arrive_expect_tx(smem_u32(&ctl->a_full[s]), 2 * C::A_BYTES);
+                        tma_load_2d_pair(a_dst, &tmap_a, mapa_shared(smem_u32(&ctl->a_full[s]), 0), ks * BK, a_row);
                     } else {
-                        tma_load_2d(raw, &tmap_raw, fb, ti.nt * (BN / 2), ti.e * p.b_rows_per_expert + ks * BK);
+                        mbar_arrive_expect_tx(smem_u32(&ctl->a_full[s]), C::A_BYTES);
+                        tma_load_2d(a_dst, &tmap_a, smem_u32(&ctl->a_full[s]), ks * BK, a_row);
                     }
                 }
             }
         }
+    } else if (warp == RAW_WARP) {
+        // packed 4-bit tiles and their absmax values: a deep ring released by the
+        // dequantizing threads, so the weight loads run many stages ahead of the MMAs.
+        // Lane 0 issues the TMA; every lane copies N_CTA/32 absmax values (cp.async),
+        // so the dequantizing threads never wait on global memory.
+        constexpr int PER_LANE = C::N_CTA / 32;   // absmax values this lane copies per stage
+        uint32_t it = 0;
+        for (int tile = cluster_id; tile < total_tiles; tile += nclusters) {
+            const TileInfo ti = decode_tile(p, tile);
+            const int ebase = ti.e * p.b_rows_per_expert;
+            // per-tile source of each of this lane's absmax values at k-stage 0, and the
+            // step per k-stage (K-major: next block of the row; MN-major: 64 rows down)
+            const float* src[PER_LANE];
+            bool valid[PER_LANE];
+#pragma unroll
+            for (int i = 0; i < PER_LANE; ++i) {
+                const int64_t ix = absmax_index<EPI, CTAS>(p, ti, 0, lane + 32 * i, (int)rank);
+                valid[i] = ix >= 0;
+                src[i] = p.absmax + (valid[i] ? ix : 0);
+            }
+            const int64_t step = kMajorB ? 1 : (int64_t)BK * p.b_blocks_per_row;
+            bool ok = true;
+            for (int ks = 0; ks < nk; ++ks, ++it) {
+                const int s = it % RSTAGES;
+                const uint32_t r = it / RSTAGES;
+                if (lane == 0) ok = mbar_wait(smem_u32(&ctl->raw_empty[s]), (r & 1) ^ 1, abort_flag, p.status);
+                ok = __shfl_sync(0xffffffffu, ok, 0);
+                if (!ok) break;
+                const uint32_t rb = smem_u32(&ctl->raw_full[s]);
+                uint8_t* stage = sRaw + s * C::RAW_STAGE;
+                if (lane == 0) {
+                    mbar_arrive_expect_tx(rb, C::RAW_BYTES);
+                    const uint32_t raw = smem_u32(stage);
+                    if (kMajorB) {
+#pragma unroll
+                        for (int h = 0; h < C::N_CTA / 128; ++h)
+                            tma_load_2d(raw + h * 4096, &tmap_raw, rb, ks * (BK / 2),
+                                        ebase + kmajor_row<EPI>(p, ti.nt, (int)rank * C::N_CTA + 128 * h));
+                    } else {
+                        tma_load_2d(raw, &tmap_raw, rb, (ti.nt * BN + (int)rank * C::N_CTA) / 2, ebase + ks * BK);
+                    }
+                }
+                const uint32_t am = smem_u32(stage + C::RAW_BYTES) + 4u * lane;
+#pragma unroll
+                for (int i = 0; i < PER_LANE; ++i) {
+                    cp_async_4(am + 128u * i, valid[i] ? src[i] + ks * step : p.absmax, valid[i] ? 4u : 0u);
+                }
+                cp_async_mbar_arrive_noinc(rb);
+            }
+            if (!ok) break;
+        }
     } else if (warp == MMA_WARP) {
-        if (lane == 0) {
-            constexpr uint32_t idesc = idesc_bf16(BM, BN, kMajorB ? 0 : 1);
+        if (lane == 0 && leader) {
+            constexpr uint32_t idesc = idesc_bf16(C::TILE_M, BN, kMajorB ? 0 : 1);
             uint32_t it = 0, lt = 0;
             bool ok = true;
-            for (int tile = blockIdx.x; tile < total_tiles && ok; tile += gridDim.x, ++lt) {
+            for (int tile = cluster_id; tile < total_tiles && ok; tile += nclusters, ++lt) {
                 const uint32_t ab = lt & 1, ar = lt >> 1;
-                if (!mbar_wait(smem_u32(&ctl->acc_empty[ab]), (ar & 1) ^ 1, abort_flag, p.status)) break;
+                if (!wait(&ctl->acc_empty[ab], (ar & 1) ^ 1)) break;
                 tc_fence_after();
                 const uint32_t d_tmem = tmem_base + ab * BN;
                 for (int ks = 0; ks < nk; ++ks, ++it) {
-                    const int s = it % STAGES;
-                    const uint32_t r = it / STAGES;
-                    if (!mbar_wait(smem_u32(&ctl->full_tma[s]), r & 1, abort_flag, p.status) ||
-                        !mbar_wait(smem_u32(&ctl->full_b[s]), r & 1, abort_flag, p.status)) { ok = false; break; }
+                    const int s = it % STAGES, sa = it % ASTAGES;
+                    const uint32_t r = it / STAGES, ra = it / ASTAGES;
+                    if (!wait(&ctl->a_full[sa], ra & 1) || !wait(&ctl->b_full[s], r & 1)) { ok = false; break; }
                     tc_fence_after();
-                    const uint32_t a_addr = smem_u32(sA + s * A_STAGE_BYTES);
-                    const uint32_t b_addr = smem_u32(sB + s * B_STAGE_BYTES);
+                    const uint32_t a_addr = smem_u32(sA + sa * C::A_BYTES);
+                    const uint32_t b_addr = smem_u32(sB + s * C::B_BYTES);
 #pragma unroll
                     for (int kk = 0; kk < BK / 16; ++kk) {
                         const uint64_t adesc = smem_desc_sw128(a_addr + kk * 32, 16, 1024);
                         const uint64_t bdesc = kMajorB ? smem_desc_sw128(b_addr + kk * 32, 16, 1024)
                                                        : smem_desc_sw128(b_addr + kk * 2048, 8192, 1024);
-                        mma_bf16_ss(d_tmem, adesc, bdesc, idesc, (ks | kk) != 0);
+                        if (CTAS == 2) mma_bf16_ss_pair(d_tmem, adesc, bdesc, idesc, (ks | kk) != 0);
+                        else mma_bf16_ss(d_tmem, adesc, bdesc, idesc, (ks | kk) != 0);
                     }
-                    mma_commit(smem_u32(&ctl->empty[s]));
+                    if (CTAS == 2) {
+                        mma_commit_pair(smem_u32(&ctl->empty[s]));
+                        mma_commit_pair(smem_u32(&ctl->a_empty[sa]));
+                    } else {
+                        mma_commit(smem_u32(&ctl->empty[s]));
+                        mma_commit(smem_u32(&ctl->a_empty[sa]));
+                    }
                 }
-                if (ok) mma_commit(smem_u32(&ctl->acc_full[ab]));
+                if (ok) {
+                    if (CTAS == 2) mma_commit_pair(smem_u32(&ctl->acc_full[ab]));
+                    else mma_commit(smem_u32(&ctl->acc_full[ab]));
+                }
             }
         }
     } else if (warp >= DEQ_WARP0) {
-        const int t = threadIdx.x - DEQ_WARP0 * 32;   // 0..255
-        uint32_t it = 0;
-        int tile = blockIdx.x, ks = 0;
-        TileInfo ti{};
-        float a_next = 0.0f;
-        if (tile < total_tiles) {
-            ti = decode_tile(p, tile);
-            a_next = load_absmax<EPI>(p, ti, 0, t);
-        }
+        // two groups of 4 warps take alternate k-stages; thread tg owns blocks tg + 128*i
+        const int grp = (warp - DEQ_WARP0) >> 2;
+        const int tg = (warp - DEQ_WARP0 - 4 * grp) * 32 + lane;   // 0..127
+        constexpr int NB = C::BLK_PER_THREAD;
+        uint32_t it = grp;
+        int tile = cluster_id, ks = grp;
+        auto normalize = [&]() {   // carry ks past the end of a tile into the next tile(s)
+            while (ks >= nk && tile < total_tiles) {
+                ks -= nk;
+                tile += nclusters;
+            }
+        };
+        normalize();
         while (tile < total_tiles) {
-            const float a_cur = a_next;
             const int s = it % STAGES;
             const uint32_t r = it / STAGES;
-            // prefetch the next stage's absmax before waiting on this one
-            if (++ks == nk) {
-                ks = 0;
-                tile += gridDim.x;
-                if (tile < total_tiles) ti = decode_tile(p, tile);
-            }
-            if (tile < total_tiles) a_next = load_absmax<EPI>(p, ti, ks, t);
-
-            if (!mbar_wait(smem_u32(&ctl->full_tma[s]), r & 1, abort_flag, p.status)) break;
-            const uint8_t* raw = sRaw + s * RAW_STAGE_BYTES + (kMajorB ? t * 32 : (t >> 2) * 128 + (t & 3) * 32);
-            const uint4 p0 = *reinterpret_cast<const uint4*>(raw);
-            const uint4 p1 = *reinterpret_cast<const uint4*>(raw + 16);
-            const BlockTable tb = make_table<CB>(a_cur);
-            uint8_t* dst_tile = sB + s * B_STAGE_BYTES;
-            const uint32_t words[8] = {p0.x, p0.y, p0.z, p0.w, p1.x, p1.y, p1.z, p1.w};
+            ks += 2;   // this group's next stage
+            normalize();
+            const int rs = it % RSTAGES;
+            const uint32_t rr = it / RSTAGES;
+            if (!mbar_wait(smem_u32(&ctl->raw_full[rs]), rr & 1, abort_flag, p.status)) break;
+            const uint8_t* raw_stage = sRaw + rs * C::RAW_STAGE;
+            const float* am = reinterpret_cast<const float*>(raw_stage + C::RAW_BYTES);
+            uint4 pk[NB][2];
+            float a_cur[NB];
 #pragma unroll
-            for (int c = 0; c < 8; ++c) {
-                uint32_t o[4];
-                decode_word(tb, words[c], o);
-                const uint32_t off = kMajorB ? sw128_offset(t, c) : (t & 3) * 8192 + sw128_offset(t >> 2, c);
-                *reinterpret_cast<uint4*>(dst_tile + off) = make_uint4(o[0], o[1], o[2], o[3]);
+            for (int i = 0; i < NB; ++i) {
+                const int b = tg + 128 * i;
+                a_cur[i] = am[b];
+                if (kMajorB) {   // raw [N_CTA rows][32 B]
+                    pk[i][0] = *reinterpret_cast<const uint4*>(raw_stage + b * 32);
+                    pk[i][1] = *reinterpret_cast<const uint4*>(raw_stage + b * 32 + 16);
+                } else {         // raw [64 k-rows][N_CTA/2 B], TMA-swizzled per row
+                    const int k = b & 63, j = b >> 6;
+                    constexpr int ROWB = C::N_CTA / 2;   // 128 B (128B swizzle) or 64 B (64B swizzle)
+                    const int sw = (ROWB == 128) ? (k & 7) : ((k >> 1) & 3);
+                    pk[i][0] = *reinterpret_cast<const uint4*>(raw_stage + k * ROWB + (((2 * j) ^ sw) << 4));
+                    pk[i][1] = *reinterpret_cast<const uint4*>(raw_stage + k * ROWB + (((2 * j + 1) ^ sw) << 4));
+                }
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(smem_u32(&ctl->raw_empty[rs]));
+            // the bf16 stage is free once the MMAs that read it (STAGES stages ago) are done
+            if (!wait(&ctl->empty[s], (r & 1) ^ 1)) break;
+            uint8_t* dst_tile = sB + s * C::B_BYTES;
+#pragma unroll
+            for (int i = 0; i < NB; ++i) {
+                const int b = tg + 128 * i;
+                const BlockTable tb = make_table<CB>(a_cur[i]);
+                const uint32_t words[8] = {pk[i][0].x, pk[i][0].y, pk[i][0].z, pk[i][0].w,
+                                           pk[i][1].x, pk[i][1].y, pk[i][1].z, pk[i][1].w};
+#pragma unroll
+                for (int c = 0; c < 8; ++c) {
+                    uint32_t o[4];
+                    decode_word(tb, words[c], o);
+                    const uint32_t off = kMajorB ? sw128_offset(b, c) : (b >> 6) * 8192 + sw128_offset(b & 63, c);
+                    *reinterpret_cast<uint4*>(dst_tile + off) = make_uint4(o[0], o[1], o[2], o[3]);
+                }
             }
             fence_proxy_async_smem();
             __syncwarp();
-            if (lane == 0) mbar_arrive(smem_u32(&ctl->full_b[s]));
-            ++it;
+            if (lane == 0) arrive_leader(&ctl->b_full[s]);
+            it += 2;
         }
     } else if (warp < 4) {
         // ------------------------------------------------------------ epilogue
-        const int rloc = warp * 32 + lane;   // TMEM lane == tile row
+        const int rloc = warp * 32 + lane;   // TMEM lane == row of this CTA's half
         uint32_t lt = 0;
-        for (int tile = blockIdx.x; tile < total_tiles; tile += gridDim.x, ++lt) {
+        for (int tile = cluster_id; tile < total_tiles; tile += nclusters, ++lt) {
             const TileInfo ti = decode_tile(p, tile);
             const uint32_t ab = lt & 1, ar = lt >> 1;
-            if (!mbar_wait(smem_u32(&ctl->acc_full[ab]), ar & 1, abort_flag, p.status)) break;
+            const int rtile = 128 * (int)rank + rloc;
+            const bool valid = rtile < ti.rows;
+            const int row = ti.row0 + rtile;
+            // everything that does not depend on the accumulator is fetched before waiting for it
+            int pair = 0;
+            float wgt = 1.0f;
+            if (EPI != EPI_GATEUP && valid) {
+                pair = __ldg(p.perm + row);
+                if (EPI != EPI_DGRAD_GATEUP) wgt = __ldg(p.topk_w + pair);
+            }
+            uint4 gq[4], uq[4];   // EPI_DGRAD_DOWN: saved dh/dg, dh/du of the current 32-column chunk
+            auto load_gu = [&](int q, uint4 (&g4)[4], uint4 (&u4)[4]) {
+                const int c0 = ti.nt * BN + 32 * q;
+                if (valid && c0 < p.N) {
+                    const uint4* gsrc = reinterpret_cast<const uint4*>(p.gu + (int64_t)row * 2 * p.N + c0);
+                    const uint4* usrc = reinterpret_cast<const uint4*>(p.gu + (int64_t)row * 2 * p.N + p.N + c0);
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        g4[i] = __ldg(gsrc + i);
+                        u4[i] = __ldg(usrc + i);
+                    }
+                }
+            };
+            if (EPI == EPI_DGRAD_DOWN) load_gu(0, gq, uq);
+            if (!wait(&ctl->acc_full[ab], ar & 1)) break;
             tc_fence_after();
             const uint32_t tbase = tmem_base + ((uint32_t)(warp * 32) << 16) + ab * BN;
-            const bool valid = rloc < ti.rows;
-            const int row = ti.row0 + rloc;
             if (EPI == EPI_GATEUP) {
                 const int I = p.up_offset;
 #pragma unroll 1
@@ -254,10 +418,25 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_con
                     tmem_load32(tbase + 128 + 32 * q, u);
                     const int f0 = ti.nt * 128 + 32 * q;
                     if (valid && f0 < I) {
-                        uint32_t hv[16];
+                        // h = silu(g) * u, and the two SwiGLU derivatives the input gradient
+                        // needs: dh/dg = u s (1 + g (1 - s)), dh/du = silu(g), s = sigmoid(g)
+                        uint32_t hv[16], dgv[16], duv[16];
 #pragma unroll
-                        for (int i = 0; i < 16; ++i)
-                            hv[i] = pack_bf16x2(silu_f(g[2 * i]) * u[2 * i], silu_f(g[2 * i + 1]) * u[2 * i + 1]);
+                        for (int i = 0; i < 16; ++i) {
+                            float hh[2], dg[2], du[2];
+#pragma unroll
+                            for (int h = 0; h < 2; ++h) {
+                                const float gg = g[2 * i + h], uu = u[2 * i + h];
+                                const float sg = __fdividef(1.0f, 1.0f + __expf(-gg));
+                                const float sl = gg * sg;
+                                hh[h] = sl * uu;
+                                dg[h] = uu * sg * (1.0f + gg * (1.0f - sg));
+                                du[h] = sl;
+                            }
+                            hv[i] = pack_bf16x2(hh[0], hh[1]);
+                            dgv[i] = pack_bf16x2(dg[0], dg[1]);
+                            duv[i] = pack_bf16x2(du[0], du[1]);
+                        }
                         uint4* dst = reinterpret_cast<uint4*>(p.out_bf16 + (int64_t)row * p.ld_out + f0);
 #pragma unroll
                         for (int i = 0; i < 4; ++i) dst[i] = make_uint4(hv[4 * i], hv[4 * i + 1], hv[4 * i + 2], hv[4 * i + 3]);
@@ -266,76 +445,72 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_con
                             uint4* du = reinterpret_cast<uint4*>(p.gu + (int64_t)row * 2 * I + I + f0);
 #pragma unroll
                             for (int i = 0; i < 4; ++i) {
-                                dg[i] = make_uint4(pack_bf16x2(g[8 * i], g[8 * i + 1]), pack_bf16x2(g[8 * i + 2], g[8 * i + 3]),
-                                                   pack_bf16x2(g[8 * i + 4], g[8 * i + 5]), pack_bf16x2(g[8 * i + 6], g[8 * i + 7]));
-                                du[i] = make_uint4(pack_bf16x2(u[8 * i], u[8 * i + 1]), pack_bf16x2(u[8 * i + 2], u[8 * i + 3]),
-                                                   pack_bf16x2(u[8 * i + 4], u[8 * i + 5]), pack_bf16x2(u[8 * i + 6], u[8 * i + 7]));
+                                dg[i] = make_uint4(dgv[4 * i], dgv[4 * i + 1], dgv[4 * i + 2], dgv[4 * i + 3]);
+                                du[i] = make_uint4(duv[4 * i], duv[4 * i + 1], duv[4 * i + 2], duv[4 * i + 3]);
                             }
                         }
                     }
                 }
             } else {
-                int pair = 0;
-                float wgt = 1.0f;
-                if (valid) {
-                    pair = __ldg(p.perm + row);
-                    if (EPI != EPI_DGRAD_GATEUP) wgt = __ldg(p.topk_w + pair);
-                }
-                const int tok = pair / p.k_top;
 #pragma unroll 1
                 for (int q = 0; q < BN / 32; ++q) {
                     float v[32];
                     tmem_load32(tbase + 32 * q, v);
+                    uint4 gn[4], un[4];
+                    if (EPI == EPI_DGRAD_DOWN && q + 1 < BN / 32) load_gu(q + 1, gn, un);   // next chunk in flight
                     const int c0 = ti.nt * BN + 32 * q;
                     if (!valid || c0 >= p.N) continue;
                     if (EPI == EPI_DOWN || EPI == EPI_DGRAD_GATEUP) {
-                        float4* dst = reinterpret_cast<float4*>(p.out_f32 + (int64_t)tok * p.ld_out + c0);
+                        // this pair's contribution, rounded to bf16, into its own slot row
+                        // (summed over the k slots of each token by the combine kernel)
+                        uint4* dst = reinterpret_cast<uint4*>(p.out_bf16 + (int64_t)pair * p.ld_out + c0);
 #pragma unroll
-                        for (int i = 0; i < 8; ++i)
-                            atomicAdd(dst + i, make_float4(v[4 * i] * wgt, v[4 * i + 1] * wgt, v[4 * i + 2] * wgt, v[4 * i + 3] * wgt));
-                    } else {   // EPI_DGRAD_DOWN: SwiGLU backward with the saved pre-activations
+                        for (int i = 0; i < 4; ++i)
+                            dst[i] = make_uint4(pack_bf16x2(v[8 * i] * wgt, v[8 * i + 1] * wgt),
+                                                pack_bf16x2(v[8 * i + 2] * wgt, v[8 * i + 3] * wgt),
+                                                pack_bf16x2(v[8 * i + 4] * wgt, v[8 * i + 5] * wgt),
+                                                pack_bf16x2(v[8 * i + 6] * wgt, v[8 * i + 7] * wgt));
+                    } else {   // EPI_DGRAD_DOWN: SwiGLU backward with the saved derivatives
                         const int I = p.N;
-                        const uint4* gsrc = reinterpret_cast<const uint4*>(p.gu + (int64_t)row * 2 * I + c0);
-                        const uint4* usrc = reinterpret_cast<const uint4*>(p.gu + (int64_t)row * 2 * I + I + c0);
                         uint4* dgo = reinterpret_cast<uint4*>(p.out_bf16 + (int64_t)row * 2 * I + c0);
                         uint4* duo = reinterpret_cast<uint4*>(p.out_bf16 + (int64_t)row * 2 * I + I + c0);
 #pragma unroll
                         for (int i = 0; i < 4; ++i) {
-                            const uint4 gq = __ldg(gsrc + i), uq = __ldg(usrc + i);
-                            const uint32_t gw[4] = {gq.x, gq.y, gq.z, gq.w}, uw[4] = {uq.x, uq.y, uq.z, uq.w};
+                            const uint32_t gw[4] = {gq[i].x, gq[i].y, gq[i].z, gq[i].w};
+                            const uint32_t uw[4] = {uq[i].x, uq[i].y, uq[i].z, uq[i].w};
                             uint32_t dgw[4], duw[4];
 #pragma unroll
                             for (int j = 0; j < 4; ++j) {
-                                float dG[2], dU[2];
-#pragma unroll
-                                for (int h = 0; h < 2; ++h) {
-                                    const float gg = __uint_as_float(h ? (gw[j] & 0xFFFF0000u) : (gw[j] << 16));
-                                    const float uu = __uint_as_float(h ? (uw[j] & 0xFFFF0000u) : (uw[j] << 16));
-                                    const float dh = v[8 * i + 2 * j + h] * wgt;
-                                    const float sg = 1.0f / (1.0f + __expf(-gg));
-                                    dG[h] = dh * uu * sg * (1.0f + gg * (1.0f - sg));
-                                    dU[h] = dh * gg * sg;
-                                }
-                                dgw[j] = pack_bf16x2(dG[0], dG[1]);
-                                duw[j] = pack_bf16x2(dU[0], dU[1]);
+                                const float dh0 = v[8 * i + 2 * j] * wgt, dh1 = v[8 * i + 2 * j + 1] * wgt;
+                                dgw[j] = pack_bf16x2(dh0 * __uint_as_float(gw[j] << 16), dh1 * __uint_as_float(gw[j] & 0xFFFF0000u));
+                                duw[j] = pack_bf16x2(dh0 * __uint_as_float(uw[j] << 16), dh1 * __uint_as_float(uw[j] & 0xFFFF0000u));
                             }
                             dgo[i] = make_uint4(dgw[0], dgw[1], dgw[2], dgw[3]);
                             duo[i] = make_uint4(duw[0], duw[1], duw[2], duw[3]);
+                        }
+                        if (q + 1 < BN / 32) {
+#pragma unroll
+                            for (int i = 0; i < 4; ++i) {
+                                gq[i] = gn[i];
+                                uq[i] = un[i];
+                            }
                         }
                     }
                 }
             }
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(smem_u32(&ctl->acc_empty[ab]));
+            if (lane == 0) arrive_leader(&ctl->acc_empty[ab]);
         }
     }
 
     tc_fence_before();
     __syncthreads();
+    if (CTAS == 2) cluster_sync_all();   // the peer's smem and TMEM stay alive until the pair is done
     if (warp == MMA_WARP) {
         tc_fence_after();
-        tmem_dealloc(tmem_base, TMEM_COLS);
+        if (CTAS == 2) tmem_dealloc_pair(tmem_base, TMEM_COLS);
+        else tmem_dealloc(tmem_base, TMEM_COLS);
     }
 }
 
@@ -365,39 +540,61 @@ static bool make_map_2d(CUtensorMap* m, CUtensorMapDataType dt, const void* base
               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// CTAs per tile of the grouped GEMMs (2: cta_group::2 pairs on two SMs).
+constexpr int kCtas = 2;
+int gemm_tile_rows() { return Cfg<kCtas>::TILE_M; }
+
 template <int EPI, int CB>
 static cudaError_t launch_one(const CUtensorMap& ma, const CUtensorMap& mr, const GemmParams& p, int grid,
                               cudaStream_t st) {
-    auto kern = grouped_gemm_kernel<EPI, CB>;
+    using C = Cfg<kCtas>;
+    auto kern = grouped_gemm_kernel<EPI, CB, kCtas>;
     static bool attr_set = false;   // per instantiation
     if (!attr_set) {
-        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, GEMM_SMEM_BYTES);
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
         if (e != cudaSuccess) return e;
         attr_set = true;
     }
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(GEMM_THREADS);
+    cfg.dynamicSmemBytes = C::SMEM_BYTES;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = kCtas;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
     timing_begin(KK_GEMM_GATEUP + EPI, st);
-    kern<<<grid, GEMM_THREADS, GEMM_SMEM_BYTES, st>>>(ma, mr, p);
+    cudaError_t e = cudaLaunchKernelEx(&cfg, kern, ma, mr, p);
     timing_end(KK_GEMM_GATEUP + EPI, st);
     count_launch();
+    if (e != cudaSuccess) return e;
     return cudaGetLastError();
 }
-
-int gemm_tile_rows() { return BM; }
 
 cudaError_t launch_grouped_gemm(int epi, int codebook, const void* a, int64_t a_rows, const uint8_t* packed,
                                 int64_t packed_rows_total, int packed_row_bytes, GemmParams p, int max_m_tiles,
                                 cudaStream_t st) {
+    using C = Cfg<kCtas>;
     CUtensorMap ma, mr;
     if (!make_map_2d(&ma, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a, (uint64_t)p.K, (uint64_t)a_rows, (uint64_t)p.K * 2, 64,
-                     BM, CU_TENSOR_MAP_SWIZZLE_128B))
+                     128, CU_TENSOR_MAP_SWIZZLE_128B))
         return cudaErrorInvalidValue;
     const bool kmaj = (epi == EPI_GATEUP || epi == EPI_DOWN);
+    // K-major: boxes of 128 rows x 32 bytes; MN-major: 64 k-rows x (N_CTA/2) bytes, swizzled so the
+    // dequantizing threads read it without bank conflicts.
+    const uint32_t mn_row = C::N_CTA / 2;
     if (!make_map_2d(&mr, CU_TENSOR_MAP_DATA_TYPE_UINT8, packed, (uint64_t)packed_row_bytes,
-                     (uint64_t)packed_rows_total, (uint64_t)packed_row_bytes, kmaj ? BK / 2 : BN / 2,
-                     kmaj ? 128 : BK, CU_TENSOR_MAP_SWIZZLE_NONE))
+                     (uint64_t)packed_rows_total, (uint64_t)packed_row_bytes, kmaj ? BK / 2 : mn_row,
+                     kmaj ? 128 : BK,
+                     kmaj ? CU_TENSOR_MAP_SWIZZLE_NONE
+                          : (mn_row == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B)))
         return cudaErrorInvalidValue;
     const int64_t tiles = (int64_t)max_m_tiles * p.n_tiles;
-    const int grid = (int)std::min<int64_t>(tiles, num_sms());
+    const int grid = (int)std::min<int64_t>(tiles * kCtas, (num_sms() / kCtas) * kCtas);
     if (grid <= 0) return cudaSuccess;
 #define E4B_LAUNCH(E_, C_) return launch_one<E_, C_>(ma, mr, p, grid, st)
     if (codebook == 0) {

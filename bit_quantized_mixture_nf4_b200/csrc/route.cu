@@ -95,7 +95,7 @@ __global__ void __launch_bounds__(256) hist_kernel(const int32_t* __restrict__ i
 __global__ void __launch_bounds__(256) scan_kernel(const int32_t* __restrict__ chunk_counts, int nchunks, int E,
                                                    int tile_rows, int32_t* __restrict__ chunk_base,
                                                    int32_t* __restrict__ counts, int32_t* __restrict__ offsets,
-                                                   int32_t* __restrict__ tile_prefix) {
+                                                   int32_t* __restrict__ tile_prefix, int4* __restrict__ sched) {
     __shared__ int s_tot[256], s_tiles[256];
     const int e = threadIdx.x;
     int tot = 0;
@@ -126,6 +126,10 @@ __global__ void __launch_bounds__(256) scan_kernel(const int32_t* __restrict__ c
             chunk_base[(int64_t)c * E + e] = run;
             run += chunk_counts[(int64_t)c * E + e];
         }
+        // m-tile schedule: (expert, first row, rows) of every m-tile, experts ascending
+        const int nt = (tot + tile_rows - 1) / tile_rows;
+        for (int m = 0; m < nt; ++m)
+            sched[s_tiles[e] + m] = make_int4(e, s_tot[e] + m * tile_rows, min(tile_rows, tot - m * tile_rows), 0);
     }
 }
 
@@ -190,6 +194,36 @@ __global__ void __launch_bounds__(256) gather_rows_kernel(const __nv_bfloat16* _
     }
 }
 
+// y[t] = bf16( sum_j fp32(slot[t*k + j]) ), j ascending: the weighted combine of
+// the k expert outputs of each token in fp32 (experts4bit-qlora 0.1.0 experts.py,
+// Experts4bit.forward: per-expert outputs in the compute dtype, index_add_ into an
+// fp32 buffer).  Slots of out-of-range experts are skipped.
+__global__ void __launch_bounds__(256) combine_kernel(const __nv_bfloat16* __restrict__ slots,
+                                                      const int32_t* __restrict__ idx, int E, int k, int64_t T,
+                                                      int H, __nv_bfloat16* __restrict__ y) {
+    const int h8 = H / 8;
+    const int64_t n = T * h8;
+    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += stride) {
+        const int64_t t = i / h8;
+        const int c = (int)(i - t * h8);
+        float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+        for (int j = 0; j < k; ++j) {
+            const int e = __ldg(idx + t * k + j);
+            if (e < 0 || e >= E) continue;
+            const uint4 v = __ldcs(reinterpret_cast<const uint4*>(slots + (t * k + j) * H) + c);
+            const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                acc[2 * q] += __uint_as_float(w[q] << 16);
+                acc[2 * q + 1] += __uint_as_float(w[q] & 0xFFFF0000u);
+            }
+        }
+        reinterpret_cast<uint4*>(y)[i] = make_uint4(pack_bf16x2(acc[0], acc[1]), pack_bf16x2(acc[2], acc[3]),
+                                                    pack_bf16x2(acc[4], acc[5]), pack_bf16x2(acc[6], acc[7]));
+    }
+}
+
 __global__ void __launch_bounds__(256) f32_to_bf16_kernel(const float* __restrict__ src, int64_t n8,
                                                           __nv_bfloat16* __restrict__ dst) {
     const int64_t stride = (int64_t)gridDim.x * blockDim.x;
@@ -216,11 +250,12 @@ cudaError_t launch_route(const float* logits, int64_t T, int E, int k, int renor
 
 cudaError_t launch_group(const int32_t* idx, int64_t P, int E, int tile_rows, int32_t* chunk_counts,
                          int32_t* chunk_base, int32_t* counts, int32_t* offsets, int32_t* tile_prefix,
-                         int32_t* perm, cudaStream_t st) {
+                         int4* sched, int32_t* perm, cudaStream_t st) {
     const int nchunks = (int)((P + kChunkPairs - 1) / kChunkPairs);
     if (nchunks == 0) return cudaSuccess;
     hist_kernel<<<nchunks, 256, 0, st>>>(idx, P, E, chunk_counts);
-    scan_kernel<<<1, 256, 0, st>>>(chunk_counts, nchunks, E, tile_rows, chunk_base, counts, offsets, tile_prefix);
+    scan_kernel<<<1, 256, 0, st>>>(chunk_counts, nchunks, E, tile_rows, chunk_base, counts, offsets, tile_prefix,
+                                   sched);
     scatter_kernel<<<nchunks, 256, 0, st>>>(idx, P, E, chunk_base, perm);
     count_launch();
     count_launch();
@@ -232,6 +267,17 @@ cudaError_t launch_gather_rows(const __nv_bfloat16* src, const int32_t* perm, co
                                int64_t P, int H, __nv_bfloat16* dst, cudaStream_t st) {
     if (P == 0) return cudaSuccess;
     gather_rows_kernel<<<capped_grid((P * 32 + 255) / 256), 256, 0, st>>>(src, perm, nrows, k, P, H, dst);
+    count_launch();
+    return cudaGetLastError();
+}
+
+cudaError_t launch_combine(const __nv_bfloat16* slots, const int32_t* idx, int E, int k, int64_t T, int H,
+                           __nv_bfloat16* y, cudaStream_t st) {
+    const int64_t n = T * (H / 8);
+    if (n == 0) return cudaSuccess;
+    timing_begin(KK_CONVERT, st);
+    combine_kernel<<<capped_grid((n + 255) / 256), 256, 0, st>>>(slots, idx, E, k, T, H, y);
+    timing_end(KK_CONVERT, st);
     count_launch();
     return cudaGetLastError();
 }

@@ -119,9 +119,11 @@ E4B_API size_t e4b_moe_workspace_size(const e4b_moe_desc *d, int64_t T);
  *                top_k_index, top_k_weights).
  *   topk_idx     int32 [T, k];  topk_w fp32 [T, k]
  *   y            bf16 [T, H]
- *   saved_gu     bf16 [T*k, 2I] or NULL: the gate/up pre-activations in grouped
- *                row order (row r holds pair perm[r]; columns [0,I) gate,
- *                [I,2I) up), for e4b_moe_backward_dgrad.
+ *   saved_gu     bf16 [T*k, 2I] or NULL: what the input gradient needs from the
+ *                forward, in grouped row order (row r holds pair perm[r]): the
+ *                SwiGLU derivatives dh/dg = u s(g) (1 + g (1 - s(g))) in columns
+ *                [0,I) and dh/du = silu(g) in columns [I,2I), s the logistic
+ *                function, for e4b_moe_backward_dgrad.
  *   offsets_out  int32 [E+1] or NULL: first grouped row of each expert.
  *   perm_out     int32 [T*k] or NULL: pair id t*k+j of each grouped row;
  *                experts ascending, tokens ascending inside an expert.
@@ -138,8 +140,8 @@ E4B_API e4b_status e4b_moe_forward(const e4b_moe_desc *d, const e4b_experts *w, 
  *   dG   = dh * u * s(g) * (1 + g (1 - s(g))),  dU = dh * silu(g)
  *   grad_x_t = sum_j  dG W_gate,e + dU W_up,e            (contract over 2I)
  * with the weights re-dequantized inside the kernels and never stored.
- * g, u come from saved_gu (as written by e4b_moe_forward for the same
- * topk_idx) or, when saved_gu is NULL, are recomputed from x.
+ * The SwiGLU derivatives come from saved_gu (as written by e4b_moe_forward for
+ * the same topk_idx) or, when saved_gu is NULL, are recomputed from x.
  *   x bf16 [T,H] (read only when saved_gu is NULL), topk_idx int32 [T,k],
  *   topk_w fp32 [T,k], grad_out bf16 [T,H], grad_x bf16 [T,H] (written). */
 E4B_API e4b_status e4b_moe_backward_dgrad(const e4b_moe_desc *d, const e4b_experts *w, const void *x,
