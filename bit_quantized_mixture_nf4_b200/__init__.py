@@ -25,7 +25,7 @@ PATH_AUTO, PATH_GROUPED, PATH_DECODE = 0, 1, 2
 
 EXPORTS = ("e4b_quantize_nf4", "e4b_dequantize_nf4", "e4b_moe_workspace_size", "e4b_moe_forward",
            "e4b_moe_backward_dgrad", "e4b_device_status", "e4b_status_string", "e4b_launch_count",
-           "e4b_timing_enable", "e4b_timing_reset", "e4b_timing_get")
+           "e4b_timing_enable", "e4b_timing_reset", "e4b_timing_get", "e4b_moe_forward_noalloc")
 # kernel kinds of e4b_timing_get
 KERNEL_KINDS = ("quantize", "dequantize", "route", "group", "gather", "convert", "gemm_gateup", "gemm_down",
                 "gemm_dgrad_down", "gemm_dgrad_gateup", "decode_gateup", "decode_down")
@@ -67,6 +67,8 @@ def _load():
                                     P, P, P, P, sz, P]
     lib.e4b_moe_backward_dgrad.argtypes = [ctypes.POINTER(e4b_moe_desc), ctypes.POINTER(e4b_experts), P, i64, P, P,
                                            P, P, P, P, sz, P]
+    lib.e4b_moe_forward_noalloc.argtypes = [ctypes.POINTER(e4b_moe_desc), ctypes.POINTER(e4b_experts), P, i64, P, P,
+                                            P, P, P]
     lib.e4b_device_status.argtypes = [P]
     lib.e4b_status_string.argtypes = [i32]
     lib.e4b_status_string.restype = ctypes.c_char_p
@@ -77,7 +79,7 @@ def _load():
     lib.e4b_timing_get.argtypes = [i32, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_uint64)]
     lib.e4b_timing_get.restype = ctypes.c_int
     for f in ("e4b_quantize_nf4", "e4b_dequantize_nf4", "e4b_moe_forward", "e4b_moe_backward_dgrad",
-              "e4b_device_status"):
+              "e4b_device_status", "e4b_moe_forward_noalloc"):
         getattr(lib, f).restype = ctypes.c_int
     _lib = lib
     return lib
@@ -230,3 +232,24 @@ def e4b_moe_backward_dgrad(desc: e4b_moe_desc, experts: e4b_experts, x, topk_idx
         ctypes.byref(desc), ctypes.byref(experts), _ptr(x), T, _ptr(topk_idx), _ptr(topk_w), _ptr(grad_out),
         _ptr(saved_gu), _ptr(grad_x), _ptr(ws), ws.numel(), _stream(stream)))
     return grad_x
+
+
+def e4b_moe_forward_noalloc(desc: e4b_moe_desc, experts: e4b_experts, x: torch.Tensor, router_logits=None,
+                            topk_idx=None, topk_w=None, y=None, stream=None):
+    """The forward with the library's own fixed scratch (no workspace argument).
+    Output tensors are allocated here only when not given.  Returns (y, topk_idx, topk_w)."""
+    _cuda(x, "x", torch.bfloat16)
+    T = x.shape[0]
+    dev = x.device
+    if topk_idx is None:
+        topk_idx = torch.empty(T, desc.top_k, dtype=torch.int32, device=dev)
+    if topk_w is None:
+        topk_w = torch.empty(T, desc.top_k, dtype=torch.float32, device=dev)
+    if router_logits is not None:
+        _cuda(router_logits, "router_logits", torch.float32)
+    if y is None:
+        y = torch.empty(T, desc.H, dtype=torch.bfloat16, device=dev)
+    _check("e4b_moe_forward_noalloc", _load().e4b_moe_forward_noalloc(
+        ctypes.byref(desc), ctypes.byref(experts), _ptr(x), T, _ptr(router_logits), _ptr(topk_idx), _ptr(topk_w),
+        _ptr(y), _stream(stream)))
+    return y, topk_idx, topk_w

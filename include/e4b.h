@@ -149,6 +149,32 @@ E4B_API e4b_status e4b_moe_backward_dgrad(const e4b_moe_desc *d, const e4b_exper
                                   const void *grad_out, const void *saved_gu, void *grad_x,
                                   void *workspace, size_t ws_bytes, void *stream);
 
+/* Forward without any device memory from the caller.  The source pages have no
+ * counterpart: this is an interface for callers that cannot give the library
+ * scratch -- a caller whose device memory all belongs to its own pool, reserved
+ * up front (a serving engine that claims free memory for its caches at start-up,
+ * a process held to a hard memory budget), or a latency-critical loop that cannot
+ * afford a per-call cudaMalloc / cudaFree (both can stall or synchronize the
+ * device).  The caller still owns and passes x, topk_idx, topk_w and y.
+ *
+ * Computes exactly what e4b_moe_forward computes for the same arguments (with
+ * saved_gu, offsets_out and perm_out absent), through the same kernels.  Its
+ * scratch is a file-scope device array of 32 MiB inside the library, which every
+ * GPU that loads the library holds until the process exits.  Requests whose
+ * workspace (e4b_moe_workspace_size) exceeds 32 MiB return E4B_ERR_WORKSPACE
+ * before anything is launched.  Allocates nothing: no cudaMalloc, no cudaFree,
+ * no allocating library call.
+ *
+ * The first call on a device looks up the array's device address (once per
+ * device, with that device current); make that first call before any stream
+ * capture.  All calls share the one array and nothing in it needs to start at
+ * zero (each call writes what it reads), but calls that can overlap on the GPU
+ * -- different streams, or host threads without ordering between their calls --
+ * race on it and must be serialized by the caller. */
+E4B_API e4b_status e4b_moe_forward_noalloc(const e4b_moe_desc *d, const e4b_experts *w, const void *x,
+                                           int64_t T, const float *router_logits, int32_t *topk_idx,
+                                           float *topk_w, void *y, void *stream);
+
 /* Synchronizes `stream`, then reads and clears the library's device status
  * word: E4B_OK, or E4B_ERR_TIMEOUT if a kernel gave up on a wait since the last
  * call.  E4B_ERR_CUDA if the synchronization itself fails. */
