@@ -50,7 +50,10 @@ struct Cfg {
     static constexpr int RSTAGES = (CTAS == 2) ? 8 : 6;    // packed-weight ring, prefetched far ahead
     static constexpr int AM_BYTES = N_CTA * 4;             // the stage's absmax values, one per block
     static constexpr int RAW_STAGE = RAW_BYTES + AM_BYTES;
-    static constexpr int BLK_PER_THREAD = N_CTA / 128;   // 64-element blocks per dequant thread per stage
+    // dequantizing warps: 6 warps (none on the MMA thread's scheduler), 3 groups of 2
+    // taking every third k-stage; a thread owns N_CTA / 64 blocks of 64 elements
+    static constexpr int DEQ_GROUPS = 3, DEQ_GROUP_WARPS = 2;
+    static constexpr int BLK_PER_THREAD = N_CTA / (32 * DEQ_GROUP_WARPS);
     static constexpr int SMEM_BYTES = ASTAGES * A_BYTES + STAGES * B_BYTES + RSTAGES * RAW_STAGE + 1024 + 1024;
 };
 
@@ -134,12 +137,12 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_con
             mbar_init(smem_u32(&ctl->a_empty[s]), 1);              // MMA commit
         }
         for (int s = 0; s < STAGES; ++s) {
-            mbar_init(smem_u32(&ctl->b_full[s]), 4 * CTAS);        // one dequant group in each CTA
+            mbar_init(smem_u32(&ctl->b_full[s]), C::DEQ_GROUP_WARPS * CTAS);   // one dequant group per CTA
             mbar_init(smem_u32(&ctl->empty[s]), 1);                // MMA commit
         }
         for (int s = 0; s < RSTAGES; ++s) {
             mbar_init(smem_u32(&ctl->raw_full[s]), 1 + 32);        // TMA + the producer warp's absmax copies
-            mbar_init(smem_u32(&ctl->raw_empty[s]), 4);            // the dequant group that read it
+            mbar_init(smem_u32(&ctl->raw_empty[s]), C::DEQ_GROUP_WARPS);       // the dequant group that read it
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(smem_u32(&ctl->acc_full[b]), 1);
@@ -310,11 +313,15 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_con
                 }
             }
         }
-    } else if (warp >= DEQ_WARP0) {
-        // two groups of 4 warps take alternate k-stages; thread tg owns blocks tg + 128*i
-        const int grp = (warp - DEQ_WARP0) >> 2;
-        const int tg = (warp - DEQ_WARP0 - 4 * grp) * 32 + lane;   // 0..127
+    } else if (warp >= DEQ_WARP0 && (warp & 3) != (MMA_WARP & 3)) {
+        // warps 8, 10, 11, 12, 14, 15: the MMA-issuing thread's scheduler stays free of
+        // dequantization work.  Group g takes k-stages g, g+3, ...; thread tg owns blocks
+        // tg + 64*i of this CTA's half.
+        const int dq = (warp - DEQ_WARP0) - ((warp - DEQ_WARP0) > (MMA_WARP & 3)) - ((warp - DEQ_WARP0) > 4 + (MMA_WARP & 3));
+        const int grp = dq / C::DEQ_GROUP_WARPS;
+        const int tg = (dq % C::DEQ_GROUP_WARPS) * 32 + lane;   // 0..63
         constexpr int NB = C::BLK_PER_THREAD;
+        constexpr int TPG = 32 * C::DEQ_GROUP_WARPS;             // threads per group
         uint32_t it = grp;
         int tile = cluster_id, ks = grp;
         auto normalize = [&]() {   // carry ks past the end of a tile into the next tile(s)
@@ -327,7 +334,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_con
         while (tile < total_tiles) {
             const int s = it % STAGES;
             const uint32_t r = it / STAGES;
-            ks += 2;   // this group's next stage
+            ks += C::DEQ_GROUPS;   // this group's next stage
             normalize();
             const int rs = it % RSTAGES;
             const uint32_t rr = it / RSTAGES;
@@ -338,7 +345,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_con
             float a_cur[NB];
 #pragma unroll
             for (int i = 0; i < NB; ++i) {
-                const int b = tg + 128 * i;
+                const int b = tg + TPG * i;
                 a_cur[i] = am[b];
                 if (kMajorB) {   // raw [N_CTA rows][32 B]
                     pk[i][0] = *reinterpret_cast<const uint4*>(raw_stage + b * 32);
@@ -358,7 +365,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_con
             uint8_t* dst_tile = sB + s * C::B_BYTES;
 #pragma unroll
             for (int i = 0; i < NB; ++i) {
-                const int b = tg + 128 * i;
+                const int b = tg + TPG * i;
                 const BlockTable tb = make_table<CB>(a_cur[i]);
                 const uint32_t words[8] = {pk[i][0].x, pk[i][0].y, pk[i][0].z, pk[i][0].w,
                                            pk[i][1].x, pk[i][1].y, pk[i][1].z, pk[i][1].w};
@@ -373,7 +380,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_con
             fence_proxy_async_smem();
             __syncwarp();
             if (lane == 0) arrive_leader(&ctl->b_full[s]);
-            it += 2;
+            it += C::DEQ_GROUPS;
         }
     } else if (warp < 4) {
         // ------------------------------------------------------------ epilogue
