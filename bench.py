@@ -317,7 +317,7 @@ def run_e4b(args, w):
 
     kernels = {}
     for name in ("gemm_gateup", "gemm_down", "gemm_dgrad_down", "gemm_dgrad_gateup", "route", "group", "gather",
-                 "convert"):
+                 "combine", "decode_gateup", "decode_down"):
         ms, n = e4b.e4b_timing_get(name)
         if n:
             kernels[name] = {"launches": n, "avg_ms": ms / n}

@@ -27,7 +27,7 @@ EXPORTS = ("e4b_quantize_nf4", "e4b_dequantize_nf4", "e4b_moe_workspace_size", "
            "e4b_moe_backward_dgrad", "e4b_device_status", "e4b_status_string", "e4b_launch_count",
            "e4b_timing_enable", "e4b_timing_reset", "e4b_timing_get", "e4b_moe_forward_noalloc")
 # kernel kinds of e4b_timing_get
-KERNEL_KINDS = ("quantize", "dequantize", "route", "group", "gather", "convert", "gemm_gateup", "gemm_down",
+KERNEL_KINDS = ("quantize", "dequantize", "route", "group", "gather", "combine", "gemm_gateup", "gemm_down",
                 "gemm_dgrad_down", "gemm_dgrad_gateup", "decode_gateup", "decode_down")
 
 

@@ -37,7 +37,7 @@ struct GemmParams {
 void count_launch();
 // Optional per-kernel-kind event timing (off by default): brackets one launch
 // with CUDA events on its stream.
-enum KernelKind { KK_QUANT = 0, KK_DEQUANT, KK_ROUTE, KK_GROUP, KK_GATHER, KK_CONVERT, KK_GEMM_GATEUP, KK_GEMM_DOWN,
+enum KernelKind { KK_QUANT = 0, KK_DEQUANT, KK_ROUTE, KK_GROUP, KK_GATHER, KK_COMBINE, KK_GEMM_GATEUP, KK_GEMM_DOWN,
                   KK_GEMM_DGRAD_DOWN, KK_GEMM_DGRAD_GATEUP, KK_DECODE_GATEUP, KK_DECODE_DOWN, KK_COUNT };
 void timing_begin(int kind, cudaStream_t st);
 void timing_end(int kind, cudaStream_t st);
@@ -51,7 +51,7 @@ cudaError_t launch_dequantize(const uint8_t* packed, const float* absmax, int64_
                               void* out, cudaStream_t st);
 
 // route.cu
-constexpr int kChunkPairs = 2048;
+constexpr int kChunkPairs = 256;   // pairs per grouping block (one per thread of a 256-thread block)
 cudaError_t launch_route(const float* logits, int64_t T, int E, int k, int renorm, int32_t* idx, float* w,
                          cudaStream_t st);
 // counts/offsets/tile_prefix/perm from topk_idx; chunk scratch: [nchunks * E] ints x2
@@ -62,7 +62,6 @@ cudaError_t launch_group(const int32_t* idx, int64_t P, int E, int tile_rows, in
 // nrows: device pointer to the number of grouped rows (offsets[E])
 cudaError_t launch_gather_rows(const __nv_bfloat16* src, const int32_t* perm, const int32_t* nrows, int k,
                                int64_t P, int H, __nv_bfloat16* dst, cudaStream_t st);
-cudaError_t launch_f32_to_bf16(const float* src, int64_t n, __nv_bfloat16* dst, cudaStream_t st);
 // y[t] = sum over the k slot rows of token t (fp32 sum in slot order, bf16 result)
 cudaError_t launch_combine(const __nv_bfloat16* slots, const int32_t* idx, int E, int k, int64_t T, int H,
                            __nv_bfloat16* y, cudaStream_t st);

@@ -224,17 +224,6 @@ __global__ void __launch_bounds__(256) combine_kernel(const __nv_bfloat16* __res
     }
 }
 
-__global__ void __launch_bounds__(256) f32_to_bf16_kernel(const float* __restrict__ src, int64_t n8,
-                                                          __nv_bfloat16* __restrict__ dst) {
-    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
-    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n8; i += stride) {
-        const float4 a = __ldcs(reinterpret_cast<const float4*>(src) + 2 * i);
-        const float4 b = __ldcs(reinterpret_cast<const float4*>(src) + 2 * i + 1);
-        reinterpret_cast<uint4*>(dst)[i] =
-            make_uint4(pack_bf16x2(a.x, a.y), pack_bf16x2(a.z, a.w), pack_bf16x2(b.x, b.y), pack_bf16x2(b.z, b.w));
-    }
-}
-
 static int capped_grid(int64_t blocks) {
     return (int)std::max<int64_t>(1, std::min<int64_t>(blocks, (int64_t)num_sms() * 16));
 }
@@ -243,7 +232,9 @@ cudaError_t launch_route(const float* logits, int64_t T, int E, int k, int renor
                          cudaStream_t st) {
     if (T == 0) return cudaSuccess;
     const int64_t blocks = (T * 32 + 255) / 256;
+    timing_begin(KK_ROUTE, st);
     route_kernel<<<(unsigned)blocks, 256, 0, st>>>(logits, T, E, k, renorm, idx, w);
+    timing_end(KK_ROUTE, st);
     count_launch();
     return cudaGetLastError();
 }
@@ -253,10 +244,12 @@ cudaError_t launch_group(const int32_t* idx, int64_t P, int E, int tile_rows, in
                          int4* sched, int32_t* perm, cudaStream_t st) {
     const int nchunks = (int)((P + kChunkPairs - 1) / kChunkPairs);
     if (nchunks == 0) return cudaSuccess;
+    timing_begin(KK_GROUP, st);
     hist_kernel<<<nchunks, 256, 0, st>>>(idx, P, E, chunk_counts);
     scan_kernel<<<1, 256, 0, st>>>(chunk_counts, nchunks, E, tile_rows, chunk_base, counts, offsets, tile_prefix,
                                    sched);
     scatter_kernel<<<nchunks, 256, 0, st>>>(idx, P, E, chunk_base, perm);
+    timing_end(KK_GROUP, st);
     count_launch();
     count_launch();
     count_launch();
@@ -266,7 +259,9 @@ cudaError_t launch_group(const int32_t* idx, int64_t P, int E, int tile_rows, in
 cudaError_t launch_gather_rows(const __nv_bfloat16* src, const int32_t* perm, const int32_t* nrows, int k,
                                int64_t P, int H, __nv_bfloat16* dst, cudaStream_t st) {
     if (P == 0) return cudaSuccess;
+    timing_begin(KK_GATHER, st);
     gather_rows_kernel<<<capped_grid((P * 32 + 255) / 256), 256, 0, st>>>(src, perm, nrows, k, P, H, dst);
+    timing_end(KK_GATHER, st);
     count_launch();
     return cudaGetLastError();
 }
@@ -275,17 +270,9 @@ cudaError_t launch_combine(const __nv_bfloat16* slots, const int32_t* idx, int E
                            __nv_bfloat16* y, cudaStream_t st) {
     const int64_t n = T * (H / 8);
     if (n == 0) return cudaSuccess;
-    timing_begin(KK_CONVERT, st);
+    timing_begin(KK_COMBINE, st);
     combine_kernel<<<capped_grid((n + 255) / 256), 256, 0, st>>>(slots, idx, E, k, T, H, y);
-    timing_end(KK_CONVERT, st);
-    count_launch();
-    return cudaGetLastError();
-}
-
-cudaError_t launch_f32_to_bf16(const float* src, int64_t n, __nv_bfloat16* dst, cudaStream_t st) {
-    const int64_t n8 = n / 8;
-    if (n8 == 0) return cudaSuccess;
-    f32_to_bf16_kernel<<<capped_grid((n8 + 255) / 256), 256, 0, st>>>(src, n8, dst);
+    timing_end(KK_COMBINE, st);
     count_launch();
     return cudaGetLastError();
 }

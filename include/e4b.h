@@ -191,7 +191,7 @@ E4B_API uint64_t e4b_launch_count(void);
  * every launch of the library is bracketed by two CUDA events on its stream;
  * e4b_timing_get synchronizes on the recorded events and returns, for one
  * kernel kind, the summed device time (ms) and the number of timed launches.
- * Kinds: 0 quantize, 1 dequantize, 2 route, 3 group, 4 gather, 5 convert,
+ * Kinds: 0 quantize, 1 dequantize, 2 route, 3 group, 4 gather, 5 combine,
  * 6 grouped gate_up GEMM, 7 grouped down GEMM, 8 dgrad down GEMM,
  * 9 dgrad gate_up GEMM, 10 decode gate_up GEMV, 11 decode down GEMV. */
 E4B_API void e4b_timing_enable(int on);
