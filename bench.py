@@ -40,6 +40,7 @@ def parse():
     ap.add_argument("--tokens", type=int, default=4096)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-aux", action="store_true", help="skip the decode and quantize/dequantize legs")
     return ap.parse_args()
 
 
@@ -153,6 +154,113 @@ class ClockSampler:
         return {"sm_mhz": statistics.median(s[0] for s in self.samples), "sm_max_mhz": self.smax,
                 "reasons": sorted(reasons), "samples": len(self.samples),
                 "power_w_max": max(s[1] for s in self.samples)}
+
+
+# ------------------------------------------------------------------ secondary legs
+
+def decode_leg(w, dev, reps=20):
+    """Small-batch forward (T <= 8, the weight-streaming GEMV path) on workload w.
+
+    Metric: touched weight bytes / forward time, touched = distinct experts the
+    tokens route to x 3*H*I x 0.5625 B.  The layer's packed weights are cycled over
+    enough copies (>= 8 and > 4x the L2 size) that every forward streams its
+    experts from HBM; the forwards over all copies run as one CUDA graph (route +
+    gate_up + down per forward).  Returns a dict for the bench line."""
+    import torch
+    import bit_quantized_mixture_nf4_b200 as e4b
+    from bit_quantized_mixture_nf4_b200 import workloads as wl
+    hbm = peaks()[0]
+    x = wl.activations(w).to(dev)
+    logits = wl.router_logits(w, wl.activations(w)).to(dev)
+    gu, dn = wl.weights(w, device=dev)
+    pg, ag = e4b.e4b_quantize_nf4(gu, codebook=w.codebook)
+    pd, ad = e4b.e4b_quantize_nf4(dn, codebook=w.codebook)
+    del gu, dn
+    per_layer = pg.numel() + pd.numel() + 4 * (ag.numel() + ad.numel())
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    copies = max(8, -(-4 * l2 // per_layer))
+    layers = [(pg, ag, pd, ad)] + [(pg.clone(), ag.clone(), pd.clone(), ad.clone()) for _ in range(copies - 1)]
+    experts = [e4b.make_experts(a, c, b, d) for a, b, c, d in layers]
+    desc = e4b.make_desc(w.E, w.H, w.I, w.k, w.renorm, w.codebook, 64, e4b.PATH_DECODE)
+    idx = torch.empty(w.T, w.k, dtype=torch.int32, device=dev)
+    wts = torch.empty(w.T, w.k, dtype=torch.float32, device=dev)
+    y = torch.empty(w.T, w.H, dtype=torch.bfloat16, device=dev)
+    ws = e4b.workspace(desc, w.T, dev)
+    side = torch.cuda.Stream(dev)
+    side.wait_stream(torch.cuda.current_stream(dev))
+    with torch.cuda.stream(side):
+        for ex in experts:                      # warm-up outside the capture
+            e4b.e4b_moe_forward(desc, ex, x, logits, idx, wts, y, ws=ws)
+    torch.cuda.current_stream(dev).wait_stream(side)
+    torch.cuda.synchronize(dev)
+    graph = torch.cuda.CUDAGraph()
+    n0 = e4b.e4b_launch_count()
+    with torch.cuda.graph(graph):
+        for ex in experts:
+            e4b.e4b_moe_forward(desc, ex, x, logits, idx, wts, y, ws=ws)
+    launches_per_fwd = (e4b.e4b_launch_count() - n0) / copies
+    graph.replay()
+    torch.cuda.synchronize(dev)
+    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s.record()
+    for _ in range(reps):
+        graph.replay()
+    e.record()
+    torch.cuda.synchronize(dev)
+    us = s.elapsed_time(e) * 1e3 / (reps * copies)
+    touched = int(torch.unique(idx).numel())
+    nbytes = touched * w.weight_bytes_per_expert()
+    gbs = nbytes / (us * 1e-6) / 1e9
+    del graph
+    if e4b.e4b_device_status() != e4b.E4B_OK:
+        raise RuntimeError("device status not ok after the decode leg")
+    return {"workload": f"{w.name}-shaped E={w.E} H={w.H} I={w.I} top{w.k} T={w.T} "
+                        f"{'fp4' if w.codebook else 'nf4'}", "us_per_forward": us,
+            "experts_touched": touched, "bytes_per_forward": nbytes, "weight_stream_gbs": gbs,
+            "roofline": {"bound": "hbm", "achieved": gbs, "peak": hbm, "unit": "GB/s", "frac": gbs / hbm},
+            "layer_copies": copies, "kernels_per_forward": launches_per_fwd, "timing": "CUDA graph, events"}
+
+
+def codec_leg(w, dev, reps=10):
+    """Standalone quantize (fp32 -> packed + absmax) and bf16 dequantize over the
+    whole gate_up stack of workload w; HBM-bound: quantize moves 4 + 0.5625 B and
+    dequantize 0.5625 + 2 B per weight element."""
+    import torch
+    import bit_quantized_mixture_nf4_b200 as e4b
+    from bit_quantized_mixture_nf4_b200 import workloads as wl
+    hbm = peaks()[0]
+    gu, _ = wl.weights(w, device=dev)
+    n = gu.numel()
+    packed = torch.empty(n // 2, dtype=torch.uint8, device=dev)
+    absmax = torch.empty(n // 64, dtype=torch.float32, device=dev)
+    out = torch.empty(n, dtype=torch.bfloat16, device=dev)
+    shape = tuple(gu.shape)
+
+    def q():
+        e4b.e4b_quantize_nf4(gu, codebook=w.codebook, packed=packed, absmax=absmax)
+
+    def dq():
+        e4b.e4b_dequantize_nf4(packed, absmax, shape, codebook=w.codebook, out_dtype=e4b.BF16, out=out)
+
+    res = {}
+    for name, fn, bpe in (("quantize", q, 4.5625), ("dequantize", dq, 2.5625)):
+        for _ in range(3):
+            fn()
+        torch.cuda.synchronize(dev)
+        s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s.record()
+        for _ in range(reps):
+            fn()
+        e.record()
+        torch.cuda.synchronize(dev)
+        us = s.elapsed_time(e) * 1e3 / reps
+        gbs = n * bpe / (us * 1e-6) / 1e9
+        res[name] = {"elements": n, "us": us, "achieved": gbs, "peak": hbm, "unit": "GB/s", "frac": gbs / hbm,
+                     "bytes_per_element": bpe}
+    res["workload"] = f"{w.name}-shaped gate_up stack [{w.E},{2 * w.I},{w.H}] {'fp4' if w.codebook else 'nf4'}"
+    del gu, out
+    torch.cuda.empty_cache()
+    return res
 
 
 # ------------------------------------------------------------------ CPU oracle
@@ -366,6 +474,16 @@ def run_e4b(args, w):
     if e4b.e4b_device_status() != e4b.E4B_OK:
         raise RuntimeError("device status not ok after the timed region")
 
+    # ------------------------------------------------ secondary legs (small-batch decode, codec)
+    aux = {}
+    if not args.no_aux:
+        del saved, ws
+        torch.cuda.empty_cache()
+        aux["decode"] = [decode_leg(v, dev) for v in (wl.QWEN3.with_tokens(1), wl.GPTOSS.with_tokens(1),
+                                                      wl.QWEN3.with_tokens(8))]
+        torch.cuda.empty_cache()
+        aux["codec"] = codec_leg(wl.OLMOE, dev)
+
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         rate, info = cpu_rate(w)
@@ -390,6 +508,7 @@ def run_e4b(args, w):
             "e2e": e2e,
             "cpu_baseline": cpu,
         }
+        line.update(aux)
         print(json.dumps(line), flush=True)
     if world > 1:
         torch.distributed.barrier()

@@ -94,7 +94,8 @@ uint32_t* device_status_ptr() {
 
 // ------------------------------------------------------------ workspace layout
 struct WsLayout {
-    size_t chunk_counts, chunk_base, counts, offsets, tile_prefix, sched, perm, a_perm, h, gu, dgu, dec_h, total;
+    size_t chunk_counts, chunk_base, counts, offsets, tile_prefix, sched, perm, a_perm, h, gu, dgu, dec_h, dec_plan,
+        total;
 };
 
 static size_t align_up(size_t v) { return (v + 255) & ~size_t(255); }
@@ -116,7 +117,8 @@ static WsLayout layout_for(const e4b_moe_desc* d, int64_t T) {
     L.h = take((size_t)P * d->I * 2);
     L.gu = take((size_t)P * 2 * d->I * 2);
     L.dgu = take((size_t)P * 2 * d->I * 2);
-    L.dec_h = take((size_t)P * d->I * 4);
+    L.dec_h = take((size_t)P * d->I * 2);
+    L.dec_plan = take(decode_plan_bytes());
     L.total = off;
     return L;
 }
@@ -285,23 +287,23 @@ e4b_status e4b_moe_forward(const e4b_moe_desc* d, const e4b_experts* w, const vo
     const WsLayout L = layout_for(d, T);
     if (!workspace || ws_bytes < L.total) return E4B_ERR_WORKSPACE;
     const bool want_grouped_outputs = saved_gu || offsets_out || perm_out;
-    bool decode = (d->path == E4B_PATH_DECODE) || (d->path == E4B_PATH_AUTO && T <= 8 && !want_grouped_outputs);
-    if (d->path == E4B_PATH_DECODE && (T > 8 || want_grouped_outputs)) return E4B_ERR_UNSUPPORTED;
+    const bool dec_ok = !want_grouped_outputs && decode_supported(d->H, d->I, T, d->top_k, router_logits != nullptr);
+    const bool decode = (d->path == E4B_PATH_DECODE) || (d->path == E4B_PATH_AUTO && dec_ok);
+    if (d->path == E4B_PATH_DECODE && !dec_ok) return E4B_ERR_UNSUPPORTED;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     uint8_t* ws = static_cast<uint8_t*>(workspace);
     const int64_t P = T * d->top_k;
 
-    if (router_logits)
-        E4B_CUDA_TRY(launch_route(router_logits, T, d->E, d->top_k, d->renormalize, topk_idx, topk_w, st));
-
-    if (decode) {
-        E4B_CUDA_TRY(launch_decode_forward(d->codebook, d->E, d->H, d->I, d->top_k, T,
-                                           static_cast<const __nv_bfloat16*>(x), topk_idx, topk_w, w->gate_up,
-                                           w->gate_up_absmax, w->down, w->down_absmax,
-                                           reinterpret_cast<float*>(ws + L.dec_h), static_cast<__nv_bfloat16*>(y),
-                                           st));
+    if (decode) {   // routing, gate_up and down in two kernels
+        E4B_CUDA_TRY(launch_decode_forward(d->codebook, d->E, d->H, d->I, d->top_k, d->renormalize, T,
+                                           static_cast<const __nv_bfloat16*>(x), router_logits, topk_idx, topk_w,
+                                           w->gate_up, w->gate_up_absmax, w->down, w->down_absmax,
+                                           reinterpret_cast<__nv_bfloat16*>(ws + L.dec_h), ws + L.dec_plan,
+                                           static_cast<__nv_bfloat16*>(y), st));
         return E4B_OK;
     }
+    if (router_logits)
+        E4B_CUDA_TRY(launch_route(router_logits, T, d->E, d->top_k, d->renormalize, topk_idx, topk_w, st));
 
     int32_t* offsets = reinterpret_cast<int32_t*>(ws + L.offsets);
     int32_t* perm = reinterpret_cast<int32_t*>(ws + L.perm);

@@ -59,6 +59,84 @@ __device__ __forceinline__ uint64_t globaltimer_ns() {
     return t;
 }
 
+// ------------------------------------------------------------------ routing
+// Routing weights of one token, computed by one warp once the top-k is known:
+// v = the token's logits (lane + 32*i, -inf beyond E), lane j < k holds the
+// j-th choice's logit in sel_v, top_v = the largest logit.  softmax over all E
+// at the choices (exp(l - top) / sum), optionally divided by their sum.  The
+// summation order is fixed (per-lane sums over i, then a butterfly), so every
+// kernel that routes gets bit-identical weights.
+__device__ __forceinline__ float route_weights_warp(const float (&v)[8], int E, int k, int renorm, int lane,
+                                                    float sel_v, float top_v) {
+    float z = 0.0f;
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+        if (lane + 32 * i < E) z += expf(v[i] - top_v);
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) z += __shfl_xor_sync(0xffffffffu, z, off);
+    float p = (lane < k) ? expf(sel_v - top_v) / z : 0.0f;
+    if (renorm) {
+        float s = p;
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
+        p = p / s;
+    }
+    return p;
+}
+
+// Order-preserving 32-bit key of a finite float (-0 is taken as +0): a > b as
+// floats iff key(a) > key(b).  0 is below every key of a float, -inf included.
+__device__ __forceinline__ uint32_t float_key(float f) {
+    uint32_t b = __float_as_uint(f);
+    if ((b & 0x7fffffffu) == 0u) b = 0u;
+    return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
+}
+__device__ __forceinline__ float key_float(uint32_t k) {
+    return __uint_as_float((k & 0x80000000u) ? (k & 0x7fffffffu) : ~k);
+}
+
+// Routing of one token by one warp: top-k on the fp32 logits (descending, ties
+// to the lower expert index; E <= 256), then route_weights_warp.  Each of the k
+// rounds takes the warp-wide maximum key and, among the lanes holding it, the
+// lowest expert index (two redux.sync).  Lane j < k receives the j-th choice in
+// *e_out / *w_out.
+__device__ __forceinline__ void route_token_warp(const float* __restrict__ l, int E, int k, int renorm, int lane,
+                                                 int* e_out, float* w_out) {
+    float v[8];
+    uint32_t key[8];
+    const float NEG_INF = __int_as_float(0xff800000);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        const int e = lane + 32 * i;
+        v[i] = (e < E) ? __ldcg(l + e) : NEG_INF;
+        key[i] = (e < E) ? float_key(v[i]) : 0u;
+    }
+    uint32_t taken = 0;
+    int sel_e = -1;
+    float sel_v = 0.0f, top_v = 0.0f;
+    for (int j = 0; j < k; ++j) {
+        uint32_t bk = 0u;
+        int bi = -1;
+#pragma unroll
+        for (int i = 0; i < 8; ++i)   // first (lowest index) maximum among this lane's free experts
+            if (lane + 32 * i < E && !((taken >> i) & 1u) && (bi < 0 || key[i] > bk)) {
+                bk = key[i];
+                bi = i;
+            }
+        const uint32_t mk = __reduce_max_sync(0xffffffffu, bk);
+        const uint32_t win = __reduce_min_sync(0xffffffffu, (bi >= 0 && bk == mk) ? (uint32_t)(lane + 32 * bi) : 0xffffffffu);
+        if ((int)(win & 31u) == lane) taken |= 1u << (win >> 5);
+        const float wv = key_float(mk);
+        if (j == 0) top_v = wv;
+        if (lane == j) {
+            sel_e = (int)win;
+            sel_v = wv;
+        }
+    }
+    *e_out = sel_e;
+    *w_out = route_weights_warp(v, E, k, renorm, lane, sel_v, top_v);
+}
+
 // ------------------------------------------------- exact per-block dequantize
 // A 64-element block shares one absmax a, so its 16 possible outputs are
 // bf16_rn(code[q] * a).  Build those 16 values once (16 fp32 multiplies), keep
@@ -142,6 +220,28 @@ __device__ __forceinline__ bool mbar_wait(uint32_t addr, uint32_t parity, volati
             return false;
         }
     }
+}
+
+// Bounded wait that does not give up early on the abort flag: used to let a
+// CTA's own bulk copies land before it exits.
+__device__ __forceinline__ bool mbar_wait_drain(uint32_t addr, uint32_t parity) {
+    const uint64_t t0 = globaltimer_ns();
+    while (!mbar_try_wait(addr, parity))
+        if (globaltimer_ns() - t0 > kWaitLimitNs) return false;
+    return true;
+}
+
+// Contiguous global -> shared bulk copy (no tensor map), completing on an
+// mbarrier.  dst, src and bytes must be multiples of 16.
+__device__ __forceinline__ void bulk_g2s(uint32_t dst, const void* src, uint32_t bytes, uint32_t mbar) {
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+                 "l"(src), "r"(bytes), "r"(mbar)
+                 : "memory");
+}
+
+// Barrier over the first nthreads threads of the CTA (id != 0; 0 is __syncthreads).
+__device__ __forceinline__ void named_bar_sync(uint32_t id, uint32_t nthreads) {
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
 
 // 4-byte asynchronous global->shared copy; src_bytes = 0 writes zero without reading.

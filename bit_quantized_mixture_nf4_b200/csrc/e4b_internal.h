@@ -72,10 +72,14 @@ cudaError_t launch_grouped_gemm(int epi, int codebook, const void* a, int64_t a_
                                 int64_t packed_rows_total, int packed_row_bytes, GemmParams p, int max_m_tiles,
                                 cudaStream_t st);
 
-// decode.cu (T <= 8)
-cudaError_t launch_decode_forward(int codebook, int E, int H, int I, int k, int64_t T, const __nv_bfloat16* x,
-                                  const int32_t* idx, const float* w, const uint8_t* gu_packed,
-                                  const float* gu_absmax, const uint8_t* d_packed, const float* d_absmax,
-                                  float* h_scratch, __nv_bfloat16* y, cudaStream_t st);
+// decode.cu (T <= 8); decode_supported: the stage rings of both kernels fit in shared memory
+// (routed: the routing comes from logits, so each token's experts are distinct)
+bool decode_supported(int H, int I, int64_t T, int k, bool routed);
+size_t decode_plan_bytes();
+cudaError_t launch_decode_forward(int codebook, int E, int H, int I, int k, int renorm, int64_t T,
+                                  const __nv_bfloat16* x, const float* logits, int32_t* idx, float* w,
+                                  const uint8_t* gu_packed, const float* gu_absmax, const uint8_t* d_packed,
+                                  const float* d_absmax, __nv_bfloat16* h_scratch, void* plan_scratch,
+                                  __nv_bfloat16* y, cudaStream_t st);
 
 }  // namespace e4b

@@ -10,65 +10,19 @@
 
 namespace e4b {
 
-// One warp per token.  Top-k on the fp32 logits (descending, ties to the lower
-// expert index), weights = softmax over all E at the chosen experts, optionally
-// divided by their sum.
+// One warp per token (the per-token routing is route_token_warp, shared with
+// the small-batch kernels).
 __global__ void __launch_bounds__(256) route_kernel(const float* __restrict__ logits, int64_t T, int E, int k,
                                                     int renorm, int32_t* __restrict__ idx,
                                                     float* __restrict__ wts) {
     const int lane = threadIdx.x & 31;
     const int64_t t = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
     if (t >= T) return;
-    const float* l = logits + t * E;
-    float v[8];
-    const float NEG_INF = __int_as_float(0xff800000);
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-        const int e = lane + 32 * i;
-        v[i] = (e < E) ? __ldg(l + e) : NEG_INF;
-    }
-    uint32_t taken = 0;
-    int sel_e = -1;
-    float sel_v = 0.0f, top_v = 0.0f;
-    for (int j = 0; j < k; ++j) {
-        float best = NEG_INF;
-        int bi = 0x7fffffff;
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-            const int e = lane + 32 * i;
-            if (e < E && !((taken >> i) & 1u) && (bi == 0x7fffffff || v[i] > best)) {
-                best = v[i];
-                bi = e;
-            }
-        }
-#pragma unroll
-        for (int off = 16; off > 0; off >>= 1) {
-            const float ov = __shfl_xor_sync(0xffffffffu, best, off);
-            const int oi = __shfl_xor_sync(0xffffffffu, bi, off);
-            if (oi != 0x7fffffff && (bi == 0x7fffffff || ov > best || (ov == best && oi < bi))) {
-                best = ov;
-                bi = oi;
-            }
-        }
-        if ((bi & 31) == lane) taken |= 1u << (bi >> 5);
-        if (j == 0) top_v = best;
-        if (lane == j) { sel_e = bi; sel_v = best; }
-    }
-    float z = 0.0f;
-#pragma unroll
-    for (int i = 0; i < 8; ++i)
-        if (lane + 32 * i < E) z += expf(v[i] - top_v);
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) z += __shfl_xor_sync(0xffffffffu, z, off);
-    float p = (lane < k) ? expf(sel_v - top_v) / z : 0.0f;
-    if (renorm) {
-        float s = p;
-#pragma unroll
-        for (int off = 16; off > 0; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
-        p = p / s;
-    }
+    int e;
+    float p;
+    route_token_warp(logits + t * E, E, k, renorm, lane, &e, &p);
     if (lane < k) {
-        idx[t * k + lane] = sel_e;
+        idx[t * k + lane] = e;
         wts[t * k + lane] = p;
     }
 }

@@ -64,8 +64,13 @@ typedef enum { E4B_PATH_AUTO = 0, E4B_PATH_GROUPED = 1, E4B_PATH_DECODE = 2 } e4
 
 /* Layer description.  H and I must be multiples of 64 (blocks never straddle a
  * row, [P4] __init__); 1 <= top_k <= min(E, 8); E <= 256; blocksize == 64.
- * path: AUTO takes the weight-streaming decode kernels for T <= 8 and the
- * grouped tensor-core kernels otherwise; the other values force one path. */
+ * path: AUTO takes the weight-streaming decode kernels for T <= 8 when no
+ * grouped outputs are requested and the kernels' shared-memory stages fit
+ * (8 rows of H and 16 rows of I elements plus the h rows of one expert's
+ * tokens: H up to about 16000, I up to about 2900 with caller-given routing
+ * and about 6000 at T = 1 with routing from logits), and the grouped
+ * tensor-core kernels otherwise; the other values force one path (DECODE
+ * outside that range returns E4B_ERR_UNSUPPORTED). */
 typedef struct {
     int E, H, I, top_k;
     int renormalize;           /* divide the selected softmax weights by their sum  */

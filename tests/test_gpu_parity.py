@@ -222,6 +222,46 @@ def test_decode_path(e4b, wname, T):
     pb.assert_close_rel_max(rg["y"].float().cpu().numpy(), yref, TOL, "grouped forward")
 
 
+@pytest.mark.parametrize("E,H,I,k,T,cb", [(4, 512, 256, 1, 1, wl.NF4), (4, 512, 256, 1, 3, wl.FP4),
+                                            (6, 192, 320, 2, 5, wl.NF4), (16, 4096, 128, 2, 1, wl.NF4)])
+def test_decode_small_shapes(e4b, E, H, I, k, T, cb):
+    """Decode path where fewer than 8 (slot, tile) units exist per CTA (K split over
+    warps), K not a multiple of the per-warp split, and 16 output rows per CTA."""
+    w = pb.custom("dec", E=E, H=H, I=I, k=k, T=T, seed=31 + T, codebook=cb)
+    prob = pb.build(w)
+    r = _run_forward(e4b, prob, path=e4b.PATH_DECODE, save=False)
+    oi, ow = _check_routing(prob, r)
+    yref, _ = pb.oracle_forward_dgrad(prob, oi, ow, np.arange(T), want_dgrad=False)
+    pb.assert_close_rel_max(r["y"].float().cpu().numpy(), yref, TOL, "decode forward")
+
+
+def test_decode_given_routing_repeats_and_invalid(e4b):
+    """Caller-given routing on the decode path: an expert chosen twice by one token,
+    one expert taking more than 8 pairs (two slots), and an out-of-range id (that
+    pair contributes nothing).  Same result from the grouped path."""
+    w = pb.custom("dec-given", E=8, H=256, I=128, k=2, T=8, seed=41)
+    prob = pb.build(w)
+    idx = np.zeros((8, 2), np.int32)
+    idx[3] = (-1, 5)
+    idx[5] = (7, 0)
+    rng = np.random.default_rng(5)
+    wts = rng.uniform(0.1, 1.0, size=(8, 2)).astype(np.float32)
+    ref_idx = idx.copy()
+    ref_w = wts.astype(np.float64)
+    ref_idx[3, 0] = 0          # the out-of-range pair: weight 0 on a valid expert adds nothing
+    ref_w[3, 0] = 0.0
+    yref, _ = pb.oracle_forward_dgrad(prob, ref_idx, ref_w, np.arange(8), want_dgrad=False)
+    t, experts = _upload_experts(e4b, prob)
+    x = pb.to_dev(prob.x)
+    for path in (e4b.PATH_DECODE, e4b.PATH_GROUPED):
+        d = _desc(e4b, w, path)
+        y, gi, gw = e4b.e4b_moe_forward(d, experts, x, None, pb.to_dev(idx), pb.to_dev(wts))
+        torch.cuda.synchronize()
+        _check_status(e4b)
+        assert np.array_equal(gi.cpu().numpy(), idx)   # given routing is left as it was
+        pb.assert_close_rel_max(y.float().cpu().numpy(), yref, TOL, f"forward path {path}")
+
+
 def test_given_routing_and_zero_tokens(e4b):
     w = pb.custom("given", E=8, H=256, I=128, k=2, T=200, seed=21)
     prob = pb.build(w)
