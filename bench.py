@@ -34,13 +34,16 @@ UNIT = "tokens/s"
 def parse():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--steps", type=int, default=30)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="e4b", choices=["e4b", "reference"])
     ap.add_argument("--tokens", type=int, default=4096)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-aux", action="store_true", help="skip the decode and quantize/dequantize legs")
+    ap.add_argument("--leg", default="step", choices=["step", "decode", "codec"],
+                    help="step: the benchmark line; decode / codec: only that secondary leg (for profiling), "
+                         "decode on the Qwen3-shaped layer at --tokens (default 1)")
     return ap.parse_args()
 
 
@@ -126,17 +129,26 @@ class ClockSampler:
             return self
         self._stop = threading.Event()
 
+        def sample():
+            try:
+                self.samples.append((pynvml.nvmlDeviceGetClockInfo(h, pynvml.NVML_CLOCK_SM),
+                                     pynvml.nvmlDeviceGetPowerUsage(h) / 1000.0, int(get_reasons(h))))
+            except Exception:
+                pass
+
         def loop():
             while not self._stop.is_set():
-                try:
-                    self.samples.append((pynvml.nvmlDeviceGetClockInfo(h, pynvml.NVML_CLOCK_SM),
-                                         pynvml.nvmlDeviceGetPowerUsage(h) / 1000.0, int(get_reasons(h))))
-                except Exception:
-                    pass
+                sample()
                 time.sleep(0.001)
+        self._sample = sample
         self._thr = threading.Thread(target=loop, daemon=True)
         self._thr.start()
         return self
+
+    def sample_now(self):
+        """One sample from the calling thread (call while the GPU is busy)."""
+        if self._thr is not None:
+            self._sample()
 
     def __exit__(self, *a):
         if self._thr is not None:
@@ -413,6 +425,8 @@ def run_e4b(args, w):
             starts[i].record(stream)
             step()
             ends[i].record(stream)
+            if i % 8 == 7:
+                clk.sample_now()                # the queued steps keep the GPU busy meanwhile
         torch.cuda.synchronize()
         e4b.e4b_timing_enable(False)
     launches = e4b.e4b_launch_count() - launches0
@@ -518,6 +532,15 @@ def run_e4b(args, w):
 def main():
     args = parse()
     from bit_quantized_mixture_nf4_b200 import workloads as wl
+    if args.leg != "step":
+        import torch
+        dev = torch.device("cuda", 0)
+        if args.leg == "decode":
+            tokens = args.tokens if args.tokens <= 8 else 1
+            print(json.dumps(decode_leg(wl.QWEN3.with_tokens(tokens), dev, reps=max(args.steps, 3))), flush=True)
+        else:
+            print(json.dumps(codec_leg(wl.OLMOE, dev, reps=max(args.steps, 3))), flush=True)
+        return
     w = wl.OLMOE.with_tokens(args.tokens)
     if args.impl == "reference":
         run_reference(args, w)

@@ -19,15 +19,20 @@
 // the dequantized B tile, so each SM dequantizes only 128 x 64 weights per
 // 512-clock stage and the B operand is read from shared memory once for both.
 // Roles per CTA (512 threads):
-//   warp 4      TMA producer: A tile (bf16, 128B swizzle) and packed 4-bit B tile
-//   warps 8-15  two groups of 4 warps, alternating k-stages: each thread turns one
-//               64-element block (one absmax) of packed codes into bf16 in the
-//               tensor cores' 128B-swizzled layout -- K-major for the forward
-//               (weights stored [N, K]), MN-major for the input gradient (weights
-//               used transposed, stored [K, N]; the transposition costs nothing)
+//   warp 4      TMA producer of the A tile (bf16, 128B swizzle), 7-stage ring
+//   warp 6      producer of the packed 4-bit B tile (TMA) and its absmax values
+//               (cp.async), 8-stage ring, prefetched far ahead
+//   warps 8, 10, 11, 12, 14, 15   dequantization, 3 groups of 2 warps taking every
+//               third k-stage (none of them shares a scheduler with the MMA
+//               thread): each thread turns 64-element blocks (one absmax each) of
+//               packed codes into bf16 in the tensor cores' 128B-swizzled layout --
+//               K-major for the forward (weights stored [N, K]), MN-major for the
+//               input gradient (weights used transposed, stored [K, N]; the
+//               transposition costs nothing); 4-stage ring of dequantized tiles
 //   warp 5      one thread of the first CTA issues the MMAs into TMEM
 //               (double-buffered accumulator, 2 x 256 columns)
 //   warps 0-3   epilogue: tcgen05.ld of this CTA's 128 accumulator rows
+//   warps 7, 9, 13 idle
 // Every mbarrier wait is bounded; on expiry the kernel records a timeout and exits.
 #include "e4b_internal.h"
 

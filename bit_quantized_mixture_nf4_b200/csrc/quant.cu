@@ -24,6 +24,7 @@ __global__ void __launch_bounds__(256) quantize_kernel(const float* __restrict__
                                                        uint8_t* __restrict__ packed, float* __restrict__ absmax) {
     __shared__ float s_mid[15];
     __shared__ uint8_t s_code[16];
+    __shared__ __align__(16) uint16_t s_out[8][128];   // per warp: 8 blocks x 32 packed bytes
     constexpr int NV = (CB == 0) ? 16 : 15;   // distinct codebook values
     if (threadIdx.x < 16) {
         const int r = threadIdx.x;
@@ -41,12 +42,17 @@ __global__ void __launch_bounds__(256) quantize_kernel(const float* __restrict__
     const int q = threadIdx.x & 3;
     const int zero_code = (CB == 0) ? 7 : 0;
     const int64_t stride = (int64_t)gridDim.x * blockDim.x / 4;
-    for (int64_t b = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) / 4; b < nblocks; b += stride) {
+    // the loop bound is taken per warp (8 blocks; every lane runs the same
+    // iterations, for the __syncwarp in the body); out-of-range lanes skip work
+    const int lb = (threadIdx.x & 31) >> 2;   // block within the warp
+    for (int64_t bw = ((int64_t)blockIdx.x * blockDim.x + (threadIdx.x & ~31)) / 4; bw < nblocks; bw += stride) {
+        const int64_t b = bw + lb;
+        const bool valid = b < nblocks;
         const float4* src = reinterpret_cast<const float4*>(w + b * 64);
         float v[16];
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
-            const float4 f = __ldcs(src + i * 4 + q);
+            const float4 f = valid ? __ldcs(src + i * 4 + q) : make_float4(0.0f, 0.0f, 0.0f, 0.0f);
             v[4 * i] = f.x; v[4 * i + 1] = f.y; v[4 * i + 2] = f.z; v[4 * i + 3] = f.w;
         }
         float a = 0.0f;
@@ -54,7 +60,7 @@ __global__ void __launch_bounds__(256) quantize_kernel(const float* __restrict__
         for (int i = 0; i < 16; ++i) a = fmaxf(a, fabsf(v[i]));
         a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, 1));
         a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, 2));
-        if (q == 0) absmax[b] = a;
+        if (q == 0 && valid) absmax[b] = a;
         uint32_t code[16];
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
@@ -70,13 +76,20 @@ __global__ void __launch_bounds__(256) quantize_kernel(const float* __restrict__
                 code[i] = s_code[r];
             }
         }
-        uint16_t* dst = reinterpret_cast<uint16_t*>(packed + b * 32);
+        // The warp's 8 blocks are 256 contiguous packed bytes: assemble them in
+        // shared memory, then each lane stores 8 bytes (one coalesced 256-byte store).
+        uint16_t* stage = s_out[threadIdx.x >> 5];
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
             const uint32_t b0 = (code[4 * i] << 4) | code[4 * i + 1];
             const uint32_t b1 = (code[4 * i + 2] << 4) | code[4 * i + 3];
-            dst[(i * 8 + q * 2) / 2] = (uint16_t)(b0 | (b1 << 8));
+            stage[(lb * 32 + i * 8 + q * 2) / 2] = (uint16_t)(b0 | (b1 << 8));
         }
+        __syncwarp();
+        const int lane = threadIdx.x & 31;
+        if (bw + lane / 4 < nblocks)
+            *reinterpret_cast<uint2*>(packed + bw * 32 + lane * 8) = reinterpret_cast<const uint2*>(stage)[lane];
+        __syncwarp();
     }
 }
 
@@ -86,23 +99,43 @@ __global__ void __launch_bounds__(256) dequantize_kernel(const uint8_t* __restri
                                                          const float* __restrict__ absmax, int64_t nchunks,
                                                          void* __restrict__ out) {
     __shared__ float s_val[16];
+    __shared__ uint4 s_stage[8][128];   // per warp: 32 lanes x 4 pieces of 16 bytes
     if (threadIdx.x < 16) s_val[threadIdx.x] = c_code[CB][threadIdx.x];
     __syncthreads();
     const int64_t stride = (int64_t)gridDim.x * blockDim.x;
-    for (int64_t c = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; c < nchunks; c += stride) {
-        const uint4 pk = __ldcs(reinterpret_cast<const uint4*>(packed) + c);
-        const float a = __ldg(absmax + (c >> 1));
+    // the loop bound is taken per warp (every lane of a warp runs the same
+    // iterations, for the __syncwarp in the body); out-of-range lanes only skip work
+    for (int64_t cw = (int64_t)blockIdx.x * blockDim.x + (threadIdx.x & ~31); cw < nchunks; cw += stride) {
+        const int64_t c = cw + (threadIdx.x & 31);
+        const bool valid = c < nchunks;
+        const uint4 pk = valid ? __ldcs(reinterpret_cast<const uint4*>(packed) + c) : make_uint4(0u, 0u, 0u, 0u);
+        const float a = valid ? __ldg(absmax + (c >> 1)) : 0.0f;
         const uint32_t words[4] = {pk.x, pk.y, pk.z, pk.w};
         if (BF16) {
+            // A warp's 32 chunks are 2 KB of contiguous output.  Each lane decodes
+            // its 64 bytes into shared memory (16-byte piece s of lane l at slot
+            // (s + l/2) mod 4: conflict-free), then the warp stores 512 contiguous
+            // bytes per instruction.
             const BlockTable tb = make_table<CB>(a);
-            uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(out) + c * 32);
+            const int lane = threadIdx.x & 31;
+            uint4* stage = s_stage[threadIdx.x >> 5];
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
                 uint32_t o[4];
                 decode_word(tb, words[i], o);
-                __stcs(dst + i, make_uint4(o[0], o[1], o[2], o[3]));
+                stage[lane * 4 + ((i + (lane >> 1)) & 3)] = make_uint4(o[0], o[1], o[2], o[3]);
             }
+            __syncwarp();
+            const int64_t c0 = c - lane;   // first chunk of this warp
+            uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(out) + c0 * 32);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const int p = 32 * i + lane, t = p >> 2, sub = p & 3;   // piece p of the warp's output
+                if (c0 + t < nchunks) __stcs(dst + p, stage[t * 4 + ((sub + (t >> 1)) & 3)]);
+            }
+            __syncwarp();
         } else {
+            if (!valid) continue;
             float4* dst = reinterpret_cast<float4*>(static_cast<float*>(out) + c * 32);
 #pragma unroll
             for (int i = 0; i < 4; ++i) {

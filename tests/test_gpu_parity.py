@@ -89,6 +89,31 @@ def test_quantize_edge_blocks(e4b, cb):
     assert np.array_equal(wl.bf16_bits(bf), oracle.dequantize(pk, am, w.shape, cb, "bf16_bits"))
 
 
+@pytest.mark.parametrize("shape", [(1, 1, 64), (3, 7, 128), (2, 33, 192), (5, 41, 320)])
+@pytest.mark.parametrize("cb", [wl.NF4, wl.FP4])
+def test_quantize_dequantize_ragged_counts(e4b, shape, cb):
+    """Block and 32-element chunk counts that are not multiples of a warp's share
+    (8 blocks / 32 chunks): the partial last warp stores only its own bytes."""
+    rng = np.random.default_rng(shape[1])
+    w = (rng.standard_normal(shape) * 0.02).astype(np.float32)
+    pk, am = oracle.quantize(w, cb)
+    dev = pb.to_dev(w)
+    packed = torch.full((shape[0], shape[1] * shape[2] // 2 + 64), 0xAB, dtype=torch.uint8, device="cuda")
+    absmax = torch.full((shape[0], shape[1] * shape[2] // 64), -1.0, dtype=torch.float32, device="cuda")
+    e4b.e4b_quantize_nf4(dev, codebook=cb, packed=packed, absmax=absmax)
+    got = packed.cpu().numpy().reshape(-1)
+    n = pk.size
+    assert np.array_equal(got[:n], pk.reshape(-1))
+    assert (got[n:] == 0xAB).all()          # nothing written past the end
+    assert np.array_equal(absmax.cpu().numpy().view(np.uint32), am.view(np.uint32))
+    out = torch.full((w.size + 256,), 7.0, dtype=torch.bfloat16, device="cuda")
+    e4b.e4b_dequantize_nf4(pb.to_dev(pk), pb.to_dev(am), shape, codebook=cb, out=out)
+    bits = wl.bf16_bits(out)
+    assert np.array_equal(bits[:w.size].reshape(shape), oracle.dequantize(pk, am, shape, cb, "bf16_bits"))
+    assert (bits[w.size:] == wl.bf16_bits(torch.tensor([7.0], dtype=torch.bfloat16))[0]).all()
+    _check_status(e4b)
+
+
 @pytest.mark.parametrize("wname", ["olmoe", "qwen3", "mixtral", "gptoss"])
 def test_quantize_full_size_bit_exact(e4b, wname):
     """Full-size stacks of every layer family: GPU quantize == oracle quantize on
