@@ -11,12 +11,14 @@
 //    (PDL): each builds its lookup table before it waits on its predecessor.
 //    gate_up routes the <= 8 tokens (one warp per token, in every CTA) and CTA
 //    0 publishes the routing and its grouping for the down kernel.
-//  * Work unit = one weight tile of 8 (gate_up) or 16 (down) rows over all of K,
-//    for one routed expert.  A CTA's units stream through a ring of shared-memory
-//    stages with a classic multistage cp.async pipeline: each warp copies whole
-//    rows as 16-byte chunks NS-1 units ahead, then cp.async.wait_group and one
-//    CTA barrier per unit.  There are no spin-waits, and the padded stage rows
-//    make the reads bank-conflict free.  gate_up runs two CTAs per SM.
+//  * Work item = one 8-row weight tile over all of K for one routed expert
+//    (gate_up: 4 gate and 4 up rows; down: 8 output rows).  Each warp owns
+//    whole items and streams them through its own ring of shared-memory
+//    sub-stages (8 blocks of 64 elements of the 8 rows, plus their absmax, and
+//    for down the h rows of the expert's tokens) with a multistage cp.async
+//    pipeline.  A warp accumulates the full K itself: no CTA barrier and no
+//    cross-warp reduction in the main loop, no spin-waits.  The padded sub-stage
+//    rows make the reads bank-conflict free.
 //  * Weight decode: a 256-entry table maps a packed byte (two 4-bit codes) to a
 //    bf16x2 pair of code values.  The table is replicated for each of the 32
 //    lanes, so a warp's 32 lookups hit 32 distinct banks.  The lookup address
@@ -25,8 +27,7 @@
 //    operand (8 rows); the activation rows (the tokens routed to the expert,
 //    <= 8) are the A operand.  Each MMA covers 16 elements of one 64-element
 //    block, so the block's absmax multiplies the fp32 block partial once
-//    (w = code * absmax, code in bf16, scale applied in fp32).  The warps of a
-//    CTA split K; their partials are summed in shared memory in warp order.
+//    (w = code * absmax, code in bf16, scale applied in fp32).
 #include "e4b_internal.h"
 
 namespace e4b {
@@ -35,29 +36,24 @@ constexpr int DK_THREADS = 256;
 constexpr int DK_WARPS = DK_THREADS / 32;
 constexpr int DK_MAXP = 64;                 // T * k <= 8 * 8 routed pairs
 constexpr int DK_MAXE = 256;
-constexpr int DK_NS_MAX = 16;               // ring stages
-constexpr int DK_DN_MAX_ROWS = 64;          // down: output rows per CTA
+constexpr int DK_NS_MAX = 8;                // sub-stages per warp ring
+constexpr int DK_KC = 8;                    // 64-element blocks per sub-stage
+constexpr int DK_DN_MAX_RT = 8;             // down: 8-row tiles per CTA
 constexpr uint32_t DK_LUT_BYTES = 32768;    // 256 byte values x 32 lanes x 4 B
+// sub-stage layout: 8 weight rows of DK_KC*32 bytes padded to 288 (72 words = 8 mod 32:
+// the 4 rows a half-warp reads fall in distinct banks), 8 absmax rows of DK_KC floats
+// padded to 12 words (4 mod 8), then (down) up to 8 activation rows of DK_KC*128
+// bytes padded to 1040 (an odd count of 16-byte units)
+constexpr int DK_SUB_RS = DK_KC * 32 + 32;
+constexpr int DK_SUB_ABS = 8 * DK_SUB_RS;
+constexpr int DK_SUB_ASW = DK_KC + 4;
+constexpr int DK_SUB_A = DK_SUB_ABS + 8 * DK_SUB_ASW * 4;
+constexpr int DK_SUB_AS = DK_KC * 128 + 16;
 
 // e2m1 values (sign in bit 3).  The FP4 codebook is these divided by 6; the
 // division is applied to the fp32 result, so the table is exact in bf16.
 static __constant__ float c_e2m1[16] = {0.0f,  0.5f,  1.0f,  1.5f,  2.0f,  3.0f,  4.0f,  6.0f,
                                         -0.0f, -0.5f, -1.0f, -1.5f, -2.0f, -3.0f, -4.0f, -6.0f};
-
-// Layout of one ring stage: R packed weight rows, R absmax rows, then (down
-// only) up to 8 activation rows.
-struct StageLayout {
-    int rows;        // R
-    int rowstride;   // bytes between weight rows: K/2 + pad, (rowstride/4) = 8 (mod 32)
-    int absoff;      // offset of the absmax rows
-    int absw;        // words between absmax rows: odd, 2 (mod 4) or 4 (mod 8)
-    int aoff;        // offset of the activation rows
-    int astride;     // bytes between activation rows: (astride/16) odd
-    int bytes;       // stage size (multiple of 128)
-    int ns;          // stages in the ring
-    int ring_off;    // offset of the ring in dynamic shared memory
-    int smem;        // dynamic shared memory of the kernel
-};
 
 struct DecArgs {
     const __nv_bfloat16* x;   // [T, H]
@@ -72,9 +68,10 @@ struct DecArgs {
     __nv_bfloat16* h;           // [T*k, I] scratch
     __nv_bfloat16* y;           // [T, H]
     struct DecPlan* gplan;      // routing / grouping published by gate_up CTA 0 for the down kernel
-    int dn_rows;                // down: output rows per CTA (multiple of 16, <= 64)
     int xs_off, xs_stride;      // gate_up: staged activations
-    StageLayout gl, dl;         // gate_up / down stage layouts
+    int gu_ring_off, gu_ns;     // gate_up: per-warp rings (offset, sub-stages)
+    int dn_rt;                  // down: 8-row tiles per CTA
+    int dn_yslot_off, dn_ring_off, dn_ns, dn_sub;   // down: y slots, per-warp rings, sub-stage bytes
 };
 
 // Routing and grouping of the <= 64 pairs.  A "slot" is one expert with up to
@@ -95,10 +92,7 @@ struct __align__(16) DecPlan {
 };
 
 constexpr uint32_t DK_PLAN_OFF = DK_LUT_BYTES;
-constexpr uint32_t DK_PART_OFF = DK_PLAN_OFF + ((sizeof(DecPlan) + 127) / 128) * 128;
-constexpr uint32_t DK_PART_BYTES = 2 * DK_WARPS * 32 * 8;                  // [2][WARPS][32] float2
-constexpr uint32_t DK_YSLOT_OFF = DK_PART_OFF + DK_PART_BYTES;
-constexpr uint32_t DK_YSLOT_BYTES = DK_MAXP * DK_DN_MAX_ROWS * 4;           // down: [MAXP][rows] fp32
+constexpr uint32_t DK_FIXED = DK_PLAN_OFF + ((sizeof(DecPlan) + 127) / 128) * 128;
 
 __device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 __device__ __forceinline__ void griddep_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;"); }
@@ -158,55 +152,58 @@ __device__ __forceinline__ void mma_16816(float d[4], uint32_t a0, uint32_t a2, 
 // activation rows, accumulated as acc += absmax[block] * (block dot product).
 // Lane (g = lane/4, c = lane%4) reads bytes [8c, 8c+8) of each block of weight
 // row g (elements 16c..16c+15) and elements 16c..16c+15 of each block of
-// activation row g (xrow; null: the row is zero).  MMA m of a block takes elements 16c+4m..16c+4m+3 from every lane:
+// activation row g (xrow).  Rows g past the slot's tokens may read any valid
+// row: MMA rows are independent and those results are never stored.  MMA m of a block takes elements 16c+4m..16c+4m+3 from every lane:
 // the same permutation of k on both operands, so D[g][n] is the block's dot
 // product; d[0], d[1] = activation row g against weight rows 2c and 2c+1.  The
 // MMAs are issued m-major over the blocks: consecutive MMAs are independent,
 // so their latencies overlap.
-__device__ __forceinline__ void mma_batch4(int nb, const uint8_t* wrow, const uint8_t* xrow, const float* a0,
-                                           const float* a1, uint32_t lane8, const uint8_t* lut, float& acc0,
-                                           float& acc1) {
-    uint2 w[4];
-    uint4 xa[4][2];
+template <int NB>
+__device__ __forceinline__ void mma_batch(const uint8_t* wrow, const uint8_t* xrow, const float* a0, const float* a1,
+                                          uint32_t lane8, const uint8_t* lut, float& acc0, float& acc1) {
+    uint2 w[NB];
+    uint4 xa[NB][2];
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-        w[j] = (j < nb) ? *reinterpret_cast<const uint2*>(wrow + j * 32) : make_uint2(0u, 0u);
-        if (xrow && j < nb) {
-            xa[j][0] = *reinterpret_cast<const uint4*>(xrow + j * 128);
-            xa[j][1] = *reinterpret_cast<const uint4*>(xrow + j * 128 + 16);
-        } else {
-            xa[j][0] = xa[j][1] = make_uint4(0u, 0u, 0u, 0u);
-        }
+    for (int j = 0; j < NB; ++j) {
+        w[j] = *reinterpret_cast<const uint2*>(wrow + j * 32);
+        xa[j][0] = *reinterpret_cast<const uint4*>(xrow + j * 128);
+        xa[j][1] = *reinterpret_cast<const uint4*>(xrow + j * 128 + 16);
     }
-    float d[4][4];
+    float d[NB][4];
 #pragma unroll
-    for (int j = 0; j < 4; ++j) d[j][0] = d[j][1] = d[j][2] = d[j][3] = 0.0f;
+    for (int j = 0; j < NB; ++j) d[j][0] = d[j][1] = d[j][2] = d[j][3] = 0.0f;
 #pragma unroll
     for (int m = 0; m < 4; ++m) {
         const uint32_t bi = (2 * m) & 3;
-        uint32_t b0[4], b1[4];
+        uint32_t b0[NB], b1[NB];
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
+        for (int j = 0; j < NB; ++j) {
             const uint32_t word = (m < 2) ? w[j].x : w[j].y;
             b0[j] = lut_lookup(lut, word, lane8, 0x5504u | (bi << 4));
             b1[j] = lut_lookup(lut, word, lane8, 0x5504u | ((bi + 1) << 4));
         }
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            if (j < nb) {
-                const uint32_t x0 = (m < 2) ? (m == 0 ? xa[j][0].x : xa[j][0].z) : (m == 2 ? xa[j][1].x : xa[j][1].z);
-                const uint32_t x1 = (m < 2) ? (m == 0 ? xa[j][0].y : xa[j][0].w) : (m == 2 ? xa[j][1].y : xa[j][1].w);
-                mma_16816(d[j], x0, x1, b0[j], b1[j]);
-            }
+        for (int j = 0; j < NB; ++j) {
+            const uint32_t x0 = (m < 2) ? (m == 0 ? xa[j][0].x : xa[j][0].z) : (m == 2 ? xa[j][1].x : xa[j][1].z);
+            const uint32_t x1 = (m < 2) ? (m == 0 ? xa[j][0].y : xa[j][0].w) : (m == 2 ? xa[j][1].y : xa[j][1].w);
+            mma_16816(d[j], x0, x1, b0[j], b1[j]);
         }
     }
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-        if (j < nb) {
-            acc0 = fmaf(a0[j], d[j][0], acc0);
-            acc1 = fmaf(a1[j], d[j][1], acc1);
-        }
+    for (int j = 0; j < NB; ++j) {
+        acc0 = fmaf(a0[j], d[j][0], acc0);
+        acc1 = fmaf(a1[j], d[j][1], acc1);
     }
+}
+
+// nb (<= 8) consecutive blocks: batches of 4, then the remainder one block at a time.
+__device__ __forceinline__ void mma_blocks(int nb, const uint8_t* wrow, const uint8_t* xrow, const float* a0,
+                                           const float* a1, uint32_t lane8, const uint8_t* lut, float& acc0,
+                                           float& acc1) {
+    int j = 0;
+    for (; j + 4 <= nb; j += 4)
+        mma_batch<4>(wrow + j * 32, xrow + j * 128, a0 + j, a1 + j, lane8, lut, acc0, acc1);
+    for (; j < nb; ++j) mma_batch<1>(wrow + j * 32, xrow + j * 128, a0 + j, a1 + j, lane8, lut, acc0, acc1);
 }
 
 // Routing (one warp per token, from logits; or the given routing) and the
@@ -281,42 +278,36 @@ __device__ void dec_build_plan(DecPlan& pl, const DecArgs& a, bool store) {
     __syncthreads();
 }
 
-// Copies weight rows grow(0) .. grow(R-1) (K/2 bytes each) and their absmax
-// rows (K/64 floats each) into a stage: warp w copies rows w, w+8, ... as 16-byte
-// chunks (absmax rows whose length is not a multiple of 16 bytes go as 4-byte
-// copies).
+// Copies one sub-stage: blocks [kb0, kb0 + nb) (nb <= DK_KC) of the 8 weight
+// rows grow(0..7) of K elements and their absmax.  Lane l takes row l/4 and
+// every 4th 16-byte chunk of it; absmax goes as 16-byte chunks when aligned,
+// else as 4-byte copies.
 template <typename RowFn>
-__device__ __forceinline__ void stage_rows(uint32_t st, const StageLayout& L, int K, const uint8_t* packed,
-                                           const float* absmax, RowFn grow) {
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int rc = K / 32, kb = K / 64;   // 16-byte chunks per row, absmax per row
-    for (int r = warp; r < L.rows; r += DK_WARPS) {
-        const size_t gr = grow(r);
-        const uint8_t* src = packed + gr * (size_t)(K / 2);
-        const uint32_t dst = st + r * L.rowstride;
-        for (int q = lane; q < rc; q += 32) cp_async16(dst + q * 16, src + q * 16);
-        const float* asrc = absmax + gr * (size_t)kb;
-        const uint32_t adst = st + L.absoff + r * L.absw * 4;
-        if (kb % 4 == 0) {
-            for (int q = lane; q < kb / 4; q += 32) cp_async16(adst + q * 16, asrc + q * 4);
-        } else {
-            for (int q = lane; q < kb; q += 32) cp_async_4(adst + q * 4, asrc + q, 4);
-        }
+__device__ __forceinline__ void copy_sub(uint32_t st, int K, int kb0, int nb, const uint8_t* packed,
+                                         const float* absmax, int lane, RowFn grow) {
+    const int r = lane >> 2, part = lane & 3, kbr = K / 64;
+    const size_t gr = grow(r);
+    const uint8_t* src = packed + gr * (size_t)(K / 2) + kb0 * 32;
+    for (int q = part; q < 2 * nb; q += 4) cp_async16(st + r * DK_SUB_RS + q * 16, src + q * 16);
+    const float* asrc = absmax + gr * (size_t)kbr + kb0;
+    const uint32_t adst = st + DK_SUB_ABS + r * DK_SUB_ASW * 4;
+    if ((kbr & 3) == 0 && (kb0 & 3) == 0 && (nb & 3) == 0) {
+        for (int q = part; q < nb / 4; q += 4) cp_async16(adst + q * 16, asrc + q * 4);
+    } else {
+        for (int q = part; q < nb; q += 4) cp_async_4(adst + q * 4, asrc + q, 4);
     }
 }
 
 // ------------------------------------------------------------------ gate_up
 // h[p, f] = silu(x_t . W_gate,e[f]) * (x_t . W_up,e[f]) for every routed pair
-// p = (t, j).  Unit = (slot, 4 features): its 8-row tile holds gate rows
+// p = (t, j).  Item = (slot, 4 features): its 8-row tile holds gate rows
 // f0..f0+3 at tile rows 0, 2, 4, 6 and up rows at 1, 3, 5, 7, so after the MMA
-// each lane holds G and U of one feature for one token.  Units are split evenly
-// over the CTAs (one per SM); the 8 warps split K.
+// each lane holds G and U of one feature for one token.  Items go round-robin
+// to all warps of the grid.
 template <int CB>
 __global__ void __launch_bounds__(DK_THREADS, 2) dec_gateup_kernel(DecArgs a) {
     extern __shared__ __align__(128) uint8_t dsm[];
     DecPlan& pl = *reinterpret_cast<DecPlan*>(dsm + DK_PLAN_OFF);
-    float2* part = reinterpret_cast<float2*>(dsm + DK_PART_OFF);   // [2][WARPS][32]
-    const StageLayout& L = a.gl;
     build_lut<CB>(dsm);
     griddep_wait();
     dec_build_plan(pl, a, a.logits != nullptr && blockIdx.x == 0);
@@ -325,113 +316,90 @@ __global__ void __launch_bounds__(DK_THREADS, 2) dec_gateup_kernel(DecArgs a) {
         int* dst = reinterpret_cast<int*>(a.gplan);
         for (int i = threadIdx.x; i < (int)(sizeof(DecPlan) / 4); i += DK_THREADS) dst[i] = src[i];
     }
-
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int H = a.H, I = a.I, KB = H / 64, FT = I / 4;
-    const int N = pl.n_slots * FT;
-    const int u0 = (int)((int64_t)blockIdx.x * N / gridDim.x);
-    const int n_units = (int)((int64_t)(blockIdx.x + 1) * N / gridDim.x) - u0;
-    const uint32_t ring = smem_u32(dsm + L.ring_off), xs = smem_u32(dsm + a.xs_off);
-
-    // activations of the T tokens (first copy group, with unit 0)
+    // activations of the T tokens
+    const uint32_t xs = smem_u32(dsm + a.xs_off);
     for (int i = tid; i < a.T * (H / 8); i += DK_THREADS) {
         const int t = i / (H / 8), q = i - t * (H / 8);
         cp_async16(xs + t * a.xs_stride + q * 16, a.x + (size_t)t * H + q * 8);
     }
-    griddep_launch_dependents();
-    // Unit cursors (slot, first feature, ring stage) advance by one unit at a
-    // time: no divisions in the loop.
-    struct Cur {
-        int s, f0, stg;
-    };
-    const int ns = L.ns;
-    auto advance = [&](Cur& q) {
-        q.f0 += 4;
-        if (q.f0 == I) {
-            q.f0 = 0;
-            ++q.s;
-        }
-        q.stg = (q.stg + 1 == ns) ? 0 : q.stg + 1;
-    };
-    const Cur first = {u0 / FT, (u0 % FT) * 4, 0};
-    auto issue = [&](const Cur& q) {
-        const size_t r0 = (size_t)pl.slot_e[q.s] * 2 * I + q.f0;
-        stage_rows(ring + q.stg * L.bytes, L, H, a.gu_packed, a.gu_absmax,
-                   [&](int r) { return r0 + (r & 1) * I + (r >> 1); });
-    };
-    Cur iq = first;
-    for (int j = 0; j < ns - 1; ++j) {
-        if (j < n_units) {
-            issue(iq);
-            advance(iq);
-        }
-        cp_async_commit();
-    }
-
-    const int g = lane >> 2, c = lane & 3;
-    const int kb0 = warp * KB / DK_WARPS, kb1 = (warp + 1) * KB / DK_WARPS;
-    const uint32_t lane8 = (uint32_t)lane * 8u;
-    const float mu = CB == 0 ? 1.0f : (1.0f / 6.0f);
-    // Sum of the 8 warps' partials of a unit (one warp does it), SwiGLU, store h.
-    auto reduce = [&](const Cur& q, int parity) {
-        const float2* pb = part + (size_t)parity * DK_WARPS * 32;
-        float G = 0.0f, U = 0.0f;
-#pragma unroll
-        for (int w = 0; w < DK_WARPS; ++w) {
-            const float2 v = pb[w * 32 + lane];
-            G += v.x;
-            U += v.y;
-        }
-        if (g < pl.slot_n[q.s]) {
-            G *= mu;
-            U *= mu;
-            const float hv = G / (1.0f + expf(-G)) * U;
-            a.h[(int64_t)pl.slot_pair[q.s][g] * I + q.f0 + c] = __float2bfloat16_rn(hv);
-        }
-    };
-    Cur cq = first, prev = first;
-    for (int i = 0; i < n_units; ++i) {
-        cp_async_wait_pending(ns - 2);
-        __syncthreads();   // unit i's stage complete; unit i-1's partials written, its stage free
-        if (i > 0 && warp == (i & (DK_WARPS - 1))) reduce(prev, (i - 1) & 1);
-        if (i + ns - 1 < n_units) {
-            issue(iq);
-            advance(iq);
-        }
-        cp_async_commit();
-
-        const uint8_t* xrow =   // activation row of token slot g (staged x)
-            (g < pl.slot_n[cq.s]) ? dsm + a.xs_off + pl.slot_tok[cq.s][g] * a.xs_stride + c * 32 : nullptr;
-        const uint8_t* st = dsm + L.ring_off + cq.stg * L.bytes;
-        const uint8_t* wrow = st + g * L.rowstride + c * 8;
-        const float* ag = reinterpret_cast<const float*>(st + L.absoff) + (2 * c) * L.absw;
-        const float* au = ag + L.absw;
-        float acc0 = 0.0f, acc1 = 0.0f;
-        for (int kb = kb0; kb < kb1; kb += 4)
-            mma_batch4(min(4, kb1 - kb), wrow + kb * 32, xrow ? xrow + kb * 128 : nullptr, ag + kb, au + kb, lane8,
-                       dsm, acc0, acc1);
-        part[((size_t)(i & 1) * DK_WARPS + warp) * 32 + lane] = make_float2(acc0, acc1);
-        prev = cq;
-        advance(cq);
-    }
     cp_async_wait_all();
     __syncthreads();
-    if (n_units > 0 && warp == (n_units & (DK_WARPS - 1))) reduce(prev, (n_units - 1) & 1);
+    griddep_launch_dependents();
+
+    const int N = pl.n_slots * FT, W = gridDim.x * DK_WARPS, gw = blockIdx.x * DK_WARPS + warp;
+    const int nsub = (KB + DK_KC - 1) / DK_KC;
+    const int n_items = gw < N ? (N - gw + W - 1) / W : 0;
+    const int total = n_items * nsub;   // this warp's sub-stages
+    const int ns = a.gu_ns;
+    const uint32_t ring = smem_u32(dsm + a.gu_ring_off) + warp * ns * DK_SUB_A;
+    const uint8_t* ring_p = dsm + a.gu_ring_off + warp * ns * DK_SUB_A;
+
+    // issue cursor: item m, sub-stage sb
+    int im = 0, isb = 0;
+    auto issue = [&]() {
+        const int it = gw + im * W, s = it / FT, f0 = (it - s * FT) * 4;
+        const size_t r0 = (size_t)pl.slot_e[s] * 2 * I + f0;
+        const int kb0 = isb * DK_KC;
+        copy_sub(ring + ((im * nsub + isb) % ns) * DK_SUB_A, H, kb0, min(DK_KC, KB - kb0), a.gu_packed, a.gu_absmax,
+                 lane, [&](int r) { return r0 + (r & 1) * I + (r >> 1); });
+        if (++isb == nsub) {
+            isb = 0;
+            ++im;
+        }
+    };
+    for (int j = 0; j < ns - 1; ++j) {
+        if (j < total) issue();
+        cp_async_commit();
+    }
+    const int g = lane >> 2, c = lane & 3;
+    const uint32_t lane8 = (uint32_t)lane * 8u;
+    const float mu = CB == 0 ? 1.0f : (1.0f / 6.0f);
+    float acc0 = 0.0f, acc1 = 0.0f;
+    int s = 0, f0 = 0, sb = 0, m = 0;
+    const uint8_t* xrow = dsm;
+    for (int i = 0; i < total; ++i) {
+        if (sb == 0) {   // new item
+            const int it = gw + m * W;
+            s = it / FT;
+            f0 = (it - s * FT) * 4;
+            xrow = dsm + a.xs_off + pl.slot_tok[s][g < pl.slot_n[s] ? g : 0] * a.xs_stride + c * 32;
+        }
+        cp_async_wait_pending(ns - 2);
+        __syncwarp();   // this warp's copies of sub-stage i landed; sub-stage i-1 consumed by every lane
+        if (i + ns - 1 < total) issue();
+        cp_async_commit();
+        const uint8_t* st = ring_p + (i % ns) * DK_SUB_A;
+        const int kb0 = sb * DK_KC, nb = min(DK_KC, KB - kb0);
+        const uint8_t* wrow = st + g * DK_SUB_RS + c * 8;
+        const float* ag = reinterpret_cast<const float*>(st + DK_SUB_ABS) + (2 * c) * DK_SUB_ASW;
+        const float* au = ag + DK_SUB_ASW;
+        mma_blocks(nb, wrow, xrow + kb0 * 128, ag, au, lane8, dsm, acc0, acc1);
+        if (++sb == nsub) {   // item done: SwiGLU, store h
+            if (g < pl.slot_n[s]) {
+                const float G = acc0 * mu, U = acc1 * mu;
+                const float hv = G / (1.0f + expf(-G)) * U;
+                a.h[(int64_t)pl.slot_pair[s][g] * I + f0 + c] = __float2bfloat16_rn(hv);
+            }
+            acc0 = acc1 = 0.0f;
+            sb = 0;
+            ++m;
+        }
+    }
+    cp_async_wait_all();
 }
 
 // --------------------------------------------------------------------- down
 // y[t, r] = sum_j w[t,j] * (W_down,e_j[r] . h[t*k+j]), summed over j in slot order.
-// A CTA owns dn_rows output rows for all routed experts.  Unit = (slot, 16
-// rows): warps 0-3 take rows 0-7 and warps 4-7 rows 8-15, each a quarter of K.
-// The unit's stage also holds the h rows of the slot's pairs.  Weighted
-// per-pair rows go to shared memory and are summed per token in j order.
+// A CTA owns dn_rt 8-row tiles of the output for all routed experts.  Item =
+// (slot, tile); items go round-robin to the CTA's warps, and an item's
+// sub-stages also carry the h rows of the slot's pairs.  Weighted per-pair rows
+// go to shared memory and are summed per token in j order.
 template <int CB>
-__global__ void __launch_bounds__(DK_THREADS, 2) dec_down_kernel(DecArgs a) {
+__global__ void __launch_bounds__(DK_THREADS, 1) dec_down_kernel(DecArgs a) {
     extern __shared__ __align__(128) uint8_t dsm[];
     DecPlan& pl = *reinterpret_cast<DecPlan*>(dsm + DK_PLAN_OFF);
-    float2* part = reinterpret_cast<float2*>(dsm + DK_PART_OFF);   // [2][WARPS][32]
-    float* yslot = reinterpret_cast<float*>(dsm + DK_YSLOT_OFF);    // [MAXP][dn_rows]
-    const StageLayout& L = a.dl;
     build_lut<CB>(dsm);
     griddep_launch_dependents();   // the next layer's gate_up may build its table meanwhile
     griddep_wait();                // routing plan and h come from gate_up
@@ -443,101 +411,85 @@ __global__ void __launch_bounds__(DK_THREADS, 2) dec_down_kernel(DecArgs a) {
     __syncthreads();
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int H = a.H, I = a.I, KB = I / 64, RW = a.dn_rows;
+    const int H = a.H, I = a.I, KB = I / 64, RW = a.dn_rt * 8;
     const int r0 = blockIdx.x * RW;
-    const int ng = min(RW, H - r0) / 16;   // 16-row groups in this CTA
-    const int n_units = pl.n_slots * ng;
-    const uint32_t ring = smem_u32(dsm + L.ring_off);
-    struct Cur {
-        int s, tg, stg;
-    };
-    const int ns = L.ns;
-    auto advance = [&](Cur& q) {
-        if (++q.tg == ng) {
-            q.tg = 0;
-            ++q.s;
+    const int nt = min(RW, H - r0) / 8;   // 8-row tiles in this CTA
+    float* yslot = reinterpret_cast<float*>(dsm + a.dn_yslot_off);   // [P][RW]
+    const int N = pl.n_slots * nt;
+    const int nsub = (KB + DK_KC - 1) / DK_KC;
+    const int n_items = warp < N ? (N - warp + DK_WARPS - 1) / DK_WARPS : 0;
+    const int total = n_items * nsub;
+    const int ns = a.dn_ns, sub = a.dn_sub;
+    const uint32_t ring = smem_u32(dsm + a.dn_ring_off) + warp * ns * sub;
+    const uint8_t* ring_p = dsm + a.dn_ring_off + warp * ns * sub;
+
+    int im = 0, isb = 0;
+    auto issue = [&]() {
+        const int it = warp + im * DK_WARPS, s = it / nt, t = it - s * nt;
+        const size_t rb = (size_t)pl.slot_e[s] * H + r0 + t * 8;
+        const int kb0 = isb * DK_KC, nb = min(DK_KC, KB - kb0);
+        const uint32_t st = ring + ((im * nsub + isb) % ns) * sub;
+        copy_sub(st, I, kb0, nb, a.d_packed, a.d_absmax, lane, [&](int r) { return rb + r; });
+        const int n = pl.slot_n[s];
+        for (int gg = 0; gg < n; ++gg) {   // h rows of the slot's pairs, these blocks
+            const __nv_bfloat16* hsrc = a.h + (size_t)pl.slot_pair[s][gg] * I + kb0 * 64;
+            for (int q = lane; q < nb * 8; q += 32) cp_async16(st + DK_SUB_A + gg * DK_SUB_AS + q * 16, hsrc + q * 8);
         }
-        q.stg = (q.stg + 1 == ns) ? 0 : q.stg + 1;
-    };
-    auto issue = [&](const Cur& q) {   // weight rows and the h rows of the unit's pairs
-        const size_t rb = (size_t)pl.slot_e[q.s] * H + r0 + q.tg * 16;
-        const uint32_t st = ring + q.stg * L.bytes;
-        stage_rows(st, L, I, a.d_packed, a.d_absmax, [&](int r) { return rb + r; });
-        const int n = pl.slot_n[q.s], rc = I / 8;
-        for (int gg = warp; gg < n; gg += DK_WARPS) {
-            const __nv_bfloat16* src = a.h + (size_t)pl.slot_pair[q.s][gg] * I;
-            for (int qq = lane; qq < rc; qq += 32) cp_async16(st + L.aoff + gg * L.astride + qq * 16, src + qq * 8);
+        if (++isb == nsub) {
+            isb = 0;
+            ++im;
         }
     };
-    Cur iq = {0, 0, 0};
     for (int j = 0; j < ns - 1; ++j) {
-        if (j < n_units) {
-            issue(iq);
-            advance(iq);
-        }
+        if (j < total) issue();
         cp_async_commit();
     }
-
-    const int g = lane >> 2, c = lane & 3, t8 = warp >> 2, kp = warp & 3;
-    const int kb0 = kp * KB / 4, kb1 = (kp + 1) * KB / 4;
+    const int g = lane >> 2, c = lane & 3;
     const uint32_t lane8 = (uint32_t)lane * 8u;
     const float mu = CB == 0 ? 1.0f : (1.0f / 6.0f);
-    // Sum of the 4 K-part partials of each of a unit's two 8-row tiles (two warps), weight, stash.
-    auto reduce = [&](const Cur& q, int parity) {
-        const int t = (warp & 1);
-        const float2* pb = part + (size_t)parity * DK_WARPS * 32;
-        float v0 = 0.0f, v1 = 0.0f;
-#pragma unroll
-        for (int qq = 0; qq < 4; ++qq) {
-            const float2 v = pb[(t * 4 + qq) * 32 + lane];
-            v0 += v.x;
-            v1 += v.y;
+    float acc0 = 0.0f, acc1 = 0.0f;
+    int s = 0, t = 0, sb = 0, m = 0, n = 0;
+    for (int i = 0; i < total; ++i) {
+        if (sb == 0) {
+            const int it = warp + m * DK_WARPS;
+            s = it / nt;
+            t = it - s * nt;
+            n = pl.slot_n[s];
         }
-        if (g < pl.slot_n[q.s]) {
-            const int p = pl.slot_pair[q.s][g];
-            yslot[p * RW + q.tg * 16 + t * 8 + 2 * c] = pl.pw[p] * (v0 * mu);
-            yslot[p * RW + q.tg * 16 + t * 8 + 2 * c + 1] = pl.pw[p] * (v1 * mu);
-        }
-    };
-    Cur cq = {0, 0, 0}, prev = cq;
-    for (int i = 0; i < n_units; ++i) {
         cp_async_wait_pending(ns - 2);
-        __syncthreads();
-        if (i > 0 && (warp >> 1) == (i & 3)) reduce(prev, (i - 1) & 1);
-        if (i + ns - 1 < n_units) {
-            issue(iq);
-            advance(iq);
-        }
+        __syncwarp();
+        if (i + ns - 1 < total) issue();
         cp_async_commit();
-
-        const int n = pl.slot_n[cq.s];
-        const uint8_t* st = dsm + L.ring_off + cq.stg * L.bytes;
-        const uint8_t* wrow = st + (t8 * 8 + g) * L.rowstride + c * 8;
-        const float* a0p = reinterpret_cast<const float*>(st + L.absoff) + (t8 * 8 + 2 * c) * L.absw;
-        const float* a1p = a0p + L.absw;
-        const uint8_t* hrow = (g < n) ? st + L.aoff + g * L.astride + c * 32 : nullptr;
-        float acc0 = 0.0f, acc1 = 0.0f;
-        for (int kb = kb0; kb < kb1; kb += 4)
-            mma_batch4(min(4, kb1 - kb), wrow + kb * 32, hrow ? hrow + kb * 128 : nullptr, a0p + kb, a1p + kb, lane8,
-                       dsm, acc0, acc1);
-        part[((size_t)(i & 1) * DK_WARPS + warp) * 32 + lane] = make_float2(acc0, acc1);
-        prev = cq;
-        advance(cq);
+        const uint8_t* st = ring_p + (i % ns) * sub;
+        const int kb0 = sb * DK_KC, nb = min(DK_KC, KB - kb0);
+        const uint8_t* wrow = st + g * DK_SUB_RS + c * 8;
+        const float* a0p = reinterpret_cast<const float*>(st + DK_SUB_ABS) + (2 * c) * DK_SUB_ASW;
+        const float* a1p = a0p + DK_SUB_ASW;
+        const uint8_t* hrow = st + DK_SUB_A + (g < n ? g : 0) * DK_SUB_AS + c * 32;
+        mma_blocks(nb, wrow, hrow, a0p, a1p, lane8, dsm, acc0, acc1);
+        if (++sb == nsub) {   // item done: weight by the routing weight, stash per pair
+            if (g < n) {
+                const int p = pl.slot_pair[s][g];
+                yslot[p * RW + t * 8 + 2 * c] = pl.pw[p] * (acc0 * mu);
+                yslot[p * RW + t * 8 + 2 * c + 1] = pl.pw[p] * (acc1 * mu);
+            }
+            acc0 = acc1 = 0.0f;
+            sb = 0;
+            ++m;
+        }
     }
     cp_async_wait_all();
     __syncthreads();
-    if (n_units > 0 && (warp >> 1) == (n_units & 3)) reduce(prev, (n_units - 1) & 1);
-    __syncthreads();
-    const int rows = ng * 16;
+    const int rows = nt * 8;
     for (int i = tid; i < a.T * rows; i += DK_THREADS) {
-        const int t = i / rows, rl = i - t * rows;
+        const int tt = i / rows, rl = i - tt * rows;
         float v = 0.0f;
         for (int j = 0; j < a.k; ++j) {
-            const int p = t * a.k + j;
+            const int p = tt * a.k + j;
             const int e = pl.pe[p];
             if (e >= 0 && e < a.E) v += yslot[p * RW + rl];
         }
-        a.y[(int64_t)t * H + r0 + rl] = __float2bfloat16_rn(v);
+        a.y[(int64_t)tt * H + r0 + rl] = __float2bfloat16_rn(v);
     }
 }
 
@@ -555,39 +507,58 @@ static int sm_count() {
     return cache[dev];
 }
 
-// Stage layout for R weight rows of K elements (+ a_rows activation rows).
-// Weight rows are padded so that (row stride / 4) = 8 (mod 32): the lanes of
-// 4 consecutive rows then read distinct banks.  Absmax rows use a word stride
-// that is odd, 2 (mod 4) or 4 (mod 8) (the last keeps rows 16-byte aligned for
-// 16-byte copies): the lanes reading rows 2c (or 2c+1), c = 0..3, hit distinct
-// banks.  Activation rows use a 16-byte stride count that is odd.
-static StageLayout stage_layout(int K, int R, int a_rows, int ring_off, int ring_budget) {
-    StageLayout L{};
-    const int rowb = K / 2, kb = K / 64;
-    L.rows = R;
-    L.rowstride = rowb + 4 * (((8 - rowb / 4) % 32 + 32) % 32);
-    L.absoff = R * L.rowstride;
-    L.absw = (kb % 4 != 0) ? kb : (kb % 8 == 0 ? kb + 4 : kb);   // odd, 2 or 4 (mod 8): distinct banks
-    L.aoff = (L.absoff + R * L.absw * 4 + 15) / 16 * 16;
-    L.astride = (K * 2 / 16) % 2 ? K * 2 : K * 2 + 16;
-    L.bytes = (L.aoff + a_rows * L.astride + 127) / 128 * 128;
-    L.ns = std::max(2, std::min(DK_NS_MAX, ring_budget / L.bytes));
-    L.ring_off = ring_off;
-    L.smem = ring_off + L.ns * L.bytes;
-    return L;
-}
-
 static int xs_stride(int H) { return (H * 2 / 16) % 2 ? H * 2 : H * 2 + 16; }
-
-// h rows per down stage: a slot holds at most T pairs when the routing comes from
-// logits (distinct experts per token), at most 8 with caller-given routing.
+static int align128(int v) { return (v + 127) / 128 * 128; }
+// h rows per down sub-stage: a slot holds at most T pairs when the routing comes
+// from logits (distinct experts per token), at most 8 with caller-given routing.
 static int down_arows(int64_t T, int k, bool routed) { return routed ? (int)T : (int)std::min<int64_t>(8, T * k); }
 
-bool decode_supported(int H, int I, int64_t T, int k, bool routed) {
+struct DecLaunch {
+    int gu_grid, gu_smem, dn_grid, dn_smem;
+};
+
+// Shared-memory plan of both kernels: gate_up two CTAs per SM (up to 112 KB
+// each) while a 3-deep per-warp ring fits, else one; down one CTA per SM.
+static bool decode_plan_launch(int H, int I, int64_t T, int k, bool routed, DecArgs* a, DecLaunch* l) {
     if (T < 1 || T > 8 || T * k > DK_MAXP) return false;
-    const int gu = (int)DK_PART_OFF + (int)DK_PART_BYTES + (int)T * xs_stride(H) + 128;
-    return stage_layout(H, 8, 0, gu, 0).smem <= 200 * 1024 &&
-           stage_layout(I, 16, down_arows(T, k, routed), (int)(DK_YSLOT_OFF + DK_YSLOT_BYTES), 0).smem <= 200 * 1024;
+    const int nsm = sm_count();
+    const int sub_g = DK_SUB_A;   // already a multiple of 128
+    const int xs_off = (int)DK_FIXED, xst = xs_stride(H);
+    const int gu_ring = align128(xs_off + (int)T * xst);
+    int gu_ns = std::min(DK_NS_MAX, (112 * 1024 - gu_ring) / (DK_WARPS * sub_g));
+    int gu_grid = 2 * nsm;
+    if (gu_ns < 3) {
+        gu_ns = std::min(DK_NS_MAX, (220 * 1024 - gu_ring) / (DK_WARPS * sub_g));
+        gu_grid = nsm;
+    }
+    const int rt = std::max(1, std::min(DK_DN_MAX_RT, (H / 8 + nsm - 1) / nsm));
+    const int yslot_off = (int)DK_FIXED;
+    const int dn_ring = align128(yslot_off + (int)(T * k) * rt * 8 * 4);
+    const int sub_d = align128(DK_SUB_A + down_arows(T, k, routed) * DK_SUB_AS);
+    const int dn_ns = std::min(DK_NS_MAX, (220 * 1024 - dn_ring) / (DK_WARPS * sub_d));
+    if (gu_ns < 2 || dn_ns < 2) return false;
+    if (a) {
+        a->xs_off = xs_off;
+        a->xs_stride = xst;
+        a->gu_ring_off = gu_ring;
+        a->gu_ns = gu_ns;
+        a->dn_rt = rt;
+        a->dn_yslot_off = yslot_off;
+        a->dn_ring_off = dn_ring;
+        a->dn_ns = dn_ns;
+        a->dn_sub = sub_d;
+    }
+    if (l) {
+        l->gu_grid = gu_grid;
+        l->gu_smem = gu_ring + DK_WARPS * gu_ns * sub_g;
+        l->dn_grid = (H / 8 + rt - 1) / rt;
+        l->dn_smem = dn_ring + DK_WARPS * dn_ns * sub_d;
+    }
+    return true;
+}
+
+bool decode_supported(int H, int I, int64_t T, int k, bool routed) {
+    return decode_plan_launch(H, I, T, k, routed, nullptr, nullptr);
 }
 
 template <typename K>
@@ -606,12 +577,12 @@ static cudaError_t launch_pdl(K kernel, int grid, int smem, cudaStream_t st, con
 }
 
 template <int CB>
-static cudaError_t decode_impl(const DecArgs& a, cudaStream_t st) {
-    cudaError_t err = cudaFuncSetAttribute(dec_gateup_kernel<CB>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                           a.gl.smem);
+static cudaError_t decode_impl(const DecArgs& a, const DecLaunch& l, cudaStream_t st) {
+    cudaError_t err =
+        cudaFuncSetAttribute(dec_gateup_kernel<CB>, cudaFuncAttributeMaxDynamicSharedMemorySize, l.gu_smem);
     if (err == cudaSuccess)
-        err = cudaFuncSetAttribute(dec_down_kernel<CB>, cudaFuncAttributeMaxDynamicSharedMemorySize, a.dl.smem);
-    // the whole unified L1 / shared array as shared memory, so two CTAs fit per SM
+        err = cudaFuncSetAttribute(dec_down_kernel<CB>, cudaFuncAttributeMaxDynamicSharedMemorySize, l.dn_smem);
+    // the whole unified L1 / shared array as shared memory, so two gate_up CTAs fit per SM
     if (err == cudaSuccess)
         err = cudaFuncSetAttribute(dec_gateup_kernel<CB>, cudaFuncAttributePreferredSharedMemoryCarveout,
                                    (int)cudaSharedmemCarveoutMaxShared);
@@ -620,12 +591,12 @@ static cudaError_t decode_impl(const DecArgs& a, cudaStream_t st) {
                                    (int)cudaSharedmemCarveoutMaxShared);
     if (err != cudaSuccess) return err;
     timing_begin(KK_DECODE_GATEUP, st);
-    err = launch_pdl(dec_gateup_kernel<CB>, 2 * sm_count(), a.gl.smem, st, a);
+    err = launch_pdl(dec_gateup_kernel<CB>, l.gu_grid, l.gu_smem, st, a);
     timing_end(KK_DECODE_GATEUP, st);
     count_launch();
     if (err != cudaSuccess) return err;
     timing_begin(KK_DECODE_DOWN, st);
-    err = launch_pdl(dec_down_kernel<CB>, (a.H + a.dn_rows - 1) / a.dn_rows, a.dl.smem, st, a);
+    err = launch_pdl(dec_down_kernel<CB>, l.dn_grid, l.dn_smem, st, a);
     timing_end(KK_DECODE_DOWN, st);
     count_launch();
     return err;
@@ -639,8 +610,9 @@ cudaError_t launch_decode_forward(int codebook, int E, int H, int I, int k, int 
                                   const float* d_absmax, __nv_bfloat16* h_scratch, void* plan_scratch,
                                   __nv_bfloat16* y, cudaStream_t st) {
     if (T == 0) return cudaSuccess;
-    if (E > DK_MAXE || !decode_supported(H, I, T, k, logits != nullptr)) return cudaErrorInvalidValue;
     DecArgs a;
+    DecLaunch l;
+    if (E > DK_MAXE || !decode_plan_launch(H, I, T, k, logits != nullptr, &a, &l)) return cudaErrorInvalidValue;
     a.x = x;
     a.logits = logits;
     a.idx = idx;
@@ -658,19 +630,7 @@ cudaError_t launch_decode_forward(int codebook, int E, int H, int I, int k, int 
     a.h = h_scratch;
     a.gplan = static_cast<DecPlan*>(plan_scratch);
     a.y = y;
-    const int nsm = sm_count();
-    // down: 16-row groups spread over about one CTA per SM (H is a multiple of 64)
-    const int groups = H / 16;
-    a.dn_rows = 16 * std::min(DK_DN_MAX_ROWS / 16, (groups + nsm - 1) / nsm);
-    a.xs_off = (int)(DK_PART_OFF + DK_PART_BYTES);
-    a.xs_stride = xs_stride(H);
-    const int gu_ring = (a.xs_off + (int)T * a.xs_stride + 127) / 128 * 128;
-    // gate_up: two CTAs per SM, each up to 112 KB (an SM has 228 KB, 1 KB per CTA
-    // reserved); down: one CTA per SM with up to about 150 KB.
-    a.gl = stage_layout(H, 8, 0, gu_ring, 112 * 1024 - gu_ring);
-    const int dn_fixed = (int)(DK_YSLOT_OFF + DK_YSLOT_BYTES);
-    a.dl = stage_layout(I, 16, down_arows(T, k, logits != nullptr), dn_fixed, 150 * 1024 - dn_fixed);
-    return codebook == 0 ? decode_impl<0>(a, st) : decode_impl<1>(a, st);
+    return codebook == 0 ? decode_impl<0>(a, l, st) : decode_impl<1>(a, l, st);
 }
 
 }  // namespace e4b
