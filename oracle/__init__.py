@@ -62,11 +62,12 @@ def _L():
             lib.e4bo_permute.argtypes = [P, i64, i32, i32, P, P, P]
             lib.e4bo_forward.argtypes = [P, i64, i32, i32, i32, i32, P, P, P, P, P, i64, P]
             lib.e4bo_dgrad.argtypes = [P, P, i64, i32, i32, i32, i32, P, P, P, P, P, i64, P]
+            lib.e4bo_router_grad.argtypes = [P, P, P, i64, i32, i32, i32, i32, i32, P, P, P, P, i64, P, P]
             lib.e4bo_codebook.argtypes = [i32, P]
             lib.e4bo_f32_to_bf16.argtypes = [ctypes.c_float]
             lib.e4bo_f32_to_bf16.restype = ctypes.c_uint16
             for f in ("e4bo_quantize", "e4bo_dequantize_f32", "e4bo_dequantize_bf16",
-                      "e4bo_route", "e4bo_permute", "e4bo_forward", "e4bo_dgrad"):
+                      "e4bo_route", "e4bo_permute", "e4bo_forward", "e4bo_dgrad", "e4bo_router_grad"):
                 getattr(lib, f).restype = ctypes.c_int
             lib.e4bo_num_threads.restype = ctypes.c_int
             _lib = lib
@@ -199,3 +200,28 @@ def dgrad(x: np.ndarray, grad_out: np.ndarray, idx: np.ndarray, w: np.ndarray, w
     _check("e4bo_dgrad", _L().e4bo_dgrad(_p(x), _p(g), T, E, H, I2 // 2, k, _p(idx), _p(w), _p(wgu), _p(wd),
                                          None if tok is None else _p(tok), nt, _p(gx)))
     return gx
+
+
+def router_grad(x: np.ndarray, grad_out: np.ndarray, logits, idx: np.ndarray, renorm: bool, wgu: np.ndarray,
+                wd: np.ndarray, tokens=None):
+    """fp64 gradient of L = <grad_out, y> with respect to the routing weights
+    (dw [nt, k]) and, when logits are given, to the router logits (dlogits
+    [nt, E]; else None), with the routing indices held."""
+    x = np.ascontiguousarray(x, np.float64)
+    g = np.ascontiguousarray(grad_out, np.float64)
+    idx = np.ascontiguousarray(idx, np.int32)
+    wgu = np.ascontiguousarray(wgu, np.float32)
+    wd = np.ascontiguousarray(wd, np.float32)
+    T, H = x.shape
+    E, I2, _ = wgu.shape
+    k = idx.shape[1]
+    lg = None if logits is None else np.ascontiguousarray(logits, np.float32)
+    El = E if lg is None else lg.shape[1]
+    tok = None if tokens is None else np.ascontiguousarray(tokens, np.int64)
+    nt = T if tok is None else tok.shape[0]
+    dw = np.zeros((nt, k), np.float64)
+    dl = None if lg is None else np.zeros((nt, El), np.float64)
+    _check("e4bo_router_grad", _L().e4bo_router_grad(
+        _p(x), _p(g), None if lg is None else _p(lg), T, El, H, I2 // 2, k, int(bool(renorm)), _p(idx), _p(wgu),
+        _p(wd), None if tok is None else _p(tok), nt, _p(dw), None if dl is None else _p(dl)))
+    return dw, dl

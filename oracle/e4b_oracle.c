@@ -347,6 +347,91 @@ int e4bo_dgrad(const double *x, const double *gout, int64_t T, int E, int H, int
     return ORC_OK;
 }
 
+/* ---- routing gradient (the other half of the layer backward) ------------- */
+
+/* With the routing indices held, the layer output is y_t = sum_j w_{t,j} Y_{t,j},
+ * Y_{t,j} = h_{t,j} W_down,e^T the expert output before its routing weight
+ * ([P4] forward: the routing weight multiplies the expert output).  So
+ *   dL/dw_{t,j} = <grad_out_t, Y_{t,j}>.
+ * The weights come from the logits (e4bo_route):
+ *   no renormalisation: w_j = p_{e_j}, p = softmax(l) over all E, and
+ *     dL/dl_i = p_i * (sum_{j: e_j = i} dw_j - sum_j dw_j p_{e_j});
+ *   renormalisation: w_j = exp(l_{e_j}) / sum_j' exp(l_{e_j'}) (the full softmax
+ *     denominator cancels), and
+ *     dL/dl_i = sum_{j: e_j = i} w_j * (dw_j - sum_j' w_j' dw_j').
+ * dw: [nt, k]; dlogits (may be NULL): [nt, E]; row i belongs to tokens[i]. */
+int e4bo_router_grad(const double *x, const double *gout, const float *logits, int64_t T, int E, int H, int I,
+                     int k, int renorm, const int32_t *idx, const float *wgu, const float *wd,
+                     const int64_t *tokens, int64_t nt, double *dw, double *dlogits) {
+    if (!x || !gout || !idx || !wgu || !wd || !dw || T < 0 || E <= 0 || k <= 0) return ORC_ERR_ARG;
+    if (dlogits && !logits) return ORC_ERR_ARG;
+    if (!tokens) nt = T;
+    for (int64_t p = 0; p < T * k; ++p)
+        if (idx[p] < 0 || idx[p] >= E) return ORC_ERR_ARG;
+#pragma omp parallel
+    {
+        double *h = (double *)malloc(sizeof(double) * (size_t)I);
+        double *pr = (double *)malloc(sizeof(double) * (size_t)E);
+#pragma omp for schedule(dynamic, 1)
+        for (int64_t i = 0; i < nt; ++i) {
+            int64_t t = tokens ? tokens[i] : i;
+            const double *xt = x + t * H;
+            const double *go = gout + t * H;
+            for (int j = 0; j < k; ++j) {
+                int e = idx[t * k + j];
+                const float *Wg = wgu + (int64_t)e * 2 * I * H;
+                const float *Wu = Wg + (int64_t)I * H;
+                const float *Wd = wd + (int64_t)e * H * I;
+                for (int r = 0; r < I; ++r) {
+                    double g = 0.0, u = 0.0;
+                    for (int c = 0; c < H; ++c) {
+                        g += xt[c] * (double)Wg[(int64_t)r * H + c];
+                        u += xt[c] * (double)Wu[(int64_t)r * H + c];
+                    }
+                    h[r] = silu(g) * u;
+                }
+                double d = 0.0;
+                for (int c = 0; c < H; ++c) {
+                    double yc = 0.0;
+                    for (int r = 0; r < I; ++r) yc += h[r] * (double)Wd[(int64_t)c * I + r];
+                    d += go[c] * yc;
+                }
+                dw[i * k + j] = d;
+            }
+            if (!dlogits) continue;
+            const float *l = logits + t * E;
+            const int32_t *o = idx + t * k;
+            double *dl = dlogits + i * E;
+            for (int e = 0; e < E; ++e) dl[e] = 0.0;
+            if (renorm) {
+                double mx = (double)l[o[0]];
+                for (int j = 1; j < k; ++j) mx = fmax(mx, (double)l[o[j]]);
+                double z = 0.0;
+                for (int j = 0; j < k; ++j) z += exp((double)l[o[j]] - mx);
+                double a = 0.0;
+                for (int j = 0; j < k; ++j) a += exp((double)l[o[j]] - mx) / z * dw[i * k + j];
+                for (int j = 0; j < k; ++j) {
+                    double wj = exp((double)l[o[j]] - mx) / z;
+                    dl[o[j]] += wj * (dw[i * k + j] - a);
+                }
+            } else {
+                double mx = (double)l[0];
+                for (int e = 1; e < E; ++e) mx = fmax(mx, (double)l[e]);
+                double z = 0.0;
+                for (int e = 0; e < E; ++e) z += exp((double)l[e] - mx);
+                for (int e = 0; e < E; ++e) pr[e] = exp((double)l[e] - mx) / z;
+                double a = 0.0;
+                for (int j = 0; j < k; ++j) a += dw[i * k + j] * pr[o[j]];
+                for (int e = 0; e < E; ++e) dl[e] = -pr[e] * a;
+                for (int j = 0; j < k; ++j) dl[o[j]] += pr[o[j]] * dw[i * k + j];
+            }
+        }
+        free(h);
+        free(pr);
+    }
+    return ORC_OK;
+}
+
 int e4bo_num_threads(void) {
 #ifdef _OPENMP
     return omp_get_max_threads();

@@ -339,6 +339,80 @@ def test_dgrad_adjoint_identity():
     assert abs(lhs - rhs) <= 1e-7 * abs(rhs) + 1e-9
 
 
+# -------------------------------------------------------------- routing gradient
+
+def _weights_from_logits(l, idx, renorm):
+    """fp64 routing weights at fixed indices: softmax over all E at idx, or over the selected."""
+    l = np.asarray(l, np.float64)
+    if renorm:
+        sel = np.take_along_axis(l, idx, 1)
+        ex = np.exp(sel - sel.max(1, keepdims=True))
+        return ex / ex.sum(1, keepdims=True)
+    ex = np.exp(l - l.max(1, keepdims=True))
+    return np.take_along_axis(ex / ex.sum(1, keepdims=True), idx, 1)
+
+
+@pytest.mark.parametrize("renorm", [True, False])
+def test_router_grad_dw_matches_central_finite_differences(renorm):
+    """dL/dw by differencing L(w) = <grad_out, y(w)> (y is linear in w)."""
+    x, idx, w, wgu, wd, *_ = _tiny_problem(E=5, H=64, I=64, T=6, k=2, seed=21, renorm=renorm)
+    go = np.random.default_rng(22).standard_normal(x.shape)
+    dw, _ = oracle.router_grad(x, go, None, idx, renorm, wgu, wd)
+    eps = 1e-3
+    num = np.zeros_like(dw)
+    for t in range(x.shape[0]):
+        for j in range(idx.shape[1]):
+            wp, wm = w.copy(), w.copy()
+            wp[t, j] += eps
+            wm[t, j] -= eps
+            num[t, j] = ((oracle.forward(x, idx, wp, wgu, wd) - oracle.forward(x, idx, wm, wgu, wd)) * go).sum() / (2 * eps)
+    np.testing.assert_allclose(dw, num, rtol=1e-8, atol=1e-10 * np.abs(num).max())
+
+
+@pytest.mark.parametrize("renorm", [True, False])
+def test_router_grad_logits_match_central_finite_differences(renorm):
+    """dL/dlogits by differencing L(l) = <grad_out, y(w(l))> with the indices held."""
+    rng = np.random.default_rng(31)
+    E, H, I, T, k = 6, 64, 64, 5, 3
+    x, _, _, wgu, wd, *_ = _tiny_problem(E=E, H=H, I=I, T=T, k=k, seed=32)
+    l = rng.standard_normal((T, E)).astype(np.float32)
+    idx, w = oracle.route(l, k, renorm)
+    np.testing.assert_allclose(_weights_from_logits(l, idx, renorm), w, rtol=1e-12)
+    go = rng.standard_normal(x.shape)
+    _, dl = oracle.router_grad(x, go, l, idx, renorm, wgu, wd)
+    eps = 1e-4
+    num = np.zeros((T, E))
+    l64 = l.astype(np.float64)
+    for t in range(T):
+        for e in range(E):
+            lp, lm = l64.copy(), l64.copy()
+            lp[t, e] += eps
+            lm[t, e] -= eps
+            fp = (oracle.forward(x, idx, _weights_from_logits(lp, idx, renorm), wgu, wd) * go).sum()
+            fm = (oracle.forward(x, idx, _weights_from_logits(lm, idx, renorm), wgu, wd) * go).sum()
+            num[t, e] = (fp - fm) / (2 * eps)
+    np.testing.assert_allclose(dl, num, rtol=1e-6, atol=1e-7 * np.abs(num).max())
+    if renorm:   # logits outside the top-k do not move renormalised weights
+        for t in range(T):
+            assert np.all(np.delete(dl[t], idx[t]) == 0.0)
+
+
+@pytest.mark.parametrize("renorm", [True, False])
+def test_router_grad_logits_sum_to_zero_and_k1_renorm_is_zero(renorm):
+    """Softmax gradients sum to zero over the logits; with k = 1 and renormalisation the
+    weight is the constant 1, so the logit gradient vanishes."""
+    rng = np.random.default_rng(41)
+    x, _, _, wgu, wd, *_ = _tiny_problem(E=7, H=64, I=64, T=9, k=2, seed=42)
+    l = rng.standard_normal((9, 7)).astype(np.float32)
+    go = rng.standard_normal(x.shape)
+    idx, _ = oracle.route(l, 2, renorm)
+    _, dl = oracle.router_grad(x, go, l, idx, renorm, wgu, wd)
+    assert np.abs(dl.sum(1)).max() <= 1e-12 * np.abs(dl).max()
+    idx1, _ = oracle.route(l, 1, True)
+    _, dl1 = oracle.router_grad(x, go, l, idx1, True, wgu, wd)
+    assert np.all(dl1 == 0.0)
+
+
 # ------------------------------------------------------ seeded workloads
 
 def test_zipf_router_hot_set():
