@@ -488,8 +488,38 @@ def run_e4b(args, w):
     if e4b.e4b_device_status() != e4b.E4B_OK:
         raise RuntimeError("device status not ok after the timed region")
 
-    # ------------------------------------------------ secondary legs (small-batch decode, codec)
+    # ------------------------------------------------ routing gradient (the other half of the backward)
     aux = {}
+    if not args.no_aux:
+        dwt = torch.empty(T, w.k, dtype=torch.float32, device=dev)
+        dlg = torch.empty(T, w.E, dtype=torch.float32, device=dev)
+
+        def rstep():
+            e4b.e4b_moe_backward_router(desc, experts, x, idx, wts, go, router_logits=logits, grad_topk_w=dwt,
+                                        grad_logits=dlg, ws=ws, stream=stream)
+
+        for _ in range(3):
+            rstep()
+        torch.cuda.synchronize()
+        rs = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+        re_ = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+        for i in range(args.steps):
+            flush.zero_()
+            rs[i].record(stream)
+            rstep()
+            re_[i].record(stream)
+        torch.cuda.synchronize()
+        r_ms = sum(a.elapsed_time(b) for a, b in zip(rs, re_)) / args.steps
+        r_flops = 6 * w.H * w.I * P
+        aux["router_backward"] = {
+            "workload": f"same layer and batch as the step (T={T})", "us": r_ms * 1e3,
+            "roofline": {"bound": "tensor", "achieved": r_flops / (r_ms / 1e3) / 1e12, "peak": bf16_burst,
+                         "unit": "TFLOP/s", "frac": r_flops / (r_ms / 1e3) / 1e12 / bf16_burst},
+            "work": "h and the unweighted expert outputs recomputed by the grouped GEMMs (6*H*I FLOP per pair), "
+                    "then one fp32 dot product per pair and the softmax backward per token"}
+        del dwt, dlg
+
+    # ------------------------------------------------ secondary legs (small-batch decode, codec)
     if not args.no_aux:
         del saved, ws
         torch.cuda.empty_cache()

@@ -24,8 +24,8 @@ F32, BF16 = 0, 1
 PATH_AUTO, PATH_GROUPED, PATH_DECODE = 0, 1, 2
 
 EXPORTS = ("e4b_quantize_nf4", "e4b_dequantize_nf4", "e4b_moe_workspace_size", "e4b_moe_forward",
-           "e4b_moe_backward_dgrad", "e4b_device_status", "e4b_status_string", "e4b_launch_count",
-           "e4b_timing_enable", "e4b_timing_reset", "e4b_timing_get", "e4b_moe_forward_noalloc")
+           "e4b_moe_backward_dgrad", "e4b_moe_backward_router", "e4b_device_status", "e4b_status_string",
+           "e4b_launch_count", "e4b_timing_enable", "e4b_timing_reset", "e4b_timing_get", "e4b_moe_forward_noalloc")
 # kernel kinds of e4b_timing_get
 KERNEL_KINDS = ("quantize", "dequantize", "route", "group", "gather", "combine", "gemm_gateup", "gemm_down",
                 "gemm_dgrad_down", "gemm_dgrad_gateup", "decode_gateup", "decode_down")
@@ -69,6 +69,8 @@ def _load():
                                            P, P, P, P, sz, P]
     lib.e4b_moe_forward_noalloc.argtypes = [ctypes.POINTER(e4b_moe_desc), ctypes.POINTER(e4b_experts), P, i64, P, P,
                                             P, P, P]
+    lib.e4b_moe_backward_router.argtypes = [ctypes.POINTER(e4b_moe_desc), ctypes.POINTER(e4b_experts), P, i64, P, P,
+                                            P, P, P, P, P, sz, P]
     lib.e4b_device_status.argtypes = [P]
     lib.e4b_status_string.argtypes = [i32]
     lib.e4b_status_string.restype = ctypes.c_char_p
@@ -79,7 +81,7 @@ def _load():
     lib.e4b_timing_get.argtypes = [i32, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_uint64)]
     lib.e4b_timing_get.restype = ctypes.c_int
     for f in ("e4b_quantize_nf4", "e4b_dequantize_nf4", "e4b_moe_forward", "e4b_moe_backward_dgrad",
-              "e4b_device_status", "e4b_moe_forward_noalloc"):
+              "e4b_device_status", "e4b_moe_forward_noalloc", "e4b_moe_backward_router"):
         getattr(lib, f).restype = ctypes.c_int
     _lib = lib
     return lib
@@ -253,3 +255,26 @@ def e4b_moe_forward_noalloc(desc: e4b_moe_desc, experts: e4b_experts, x: torch.T
         ctypes.byref(desc), ctypes.byref(experts), _ptr(x), T, _ptr(router_logits), _ptr(topk_idx), _ptr(topk_w),
         _ptr(y), _stream(stream)))
     return y, topk_idx, topk_w
+
+
+def e4b_moe_backward_router(desc: e4b_moe_desc, experts: e4b_experts, x, topk_idx, topk_w, grad_out,
+                            router_logits=None, grad_topk_w=None, grad_logits=None, want_logits=True, ws=None,
+                            stream=None):
+    """Routing gradient with the indices held: (grad_topk_w fp32 [T, k],
+    grad_logits fp32 [T, E] or None).  grad_logits needs router_logits."""
+    _cuda(x, "x", torch.bfloat16)
+    _cuda(grad_out, "grad_out", torch.bfloat16)
+    T = x.shape[0]
+    dev = x.device
+    if grad_topk_w is None:
+        grad_topk_w = torch.empty(T, desc.top_k, dtype=torch.float32, device=dev)
+    if router_logits is not None:
+        _cuda(router_logits, "router_logits", torch.float32)
+        if grad_logits is None and want_logits:
+            grad_logits = torch.empty(T, desc.E, dtype=torch.float32, device=dev)
+    if ws is None:
+        ws = workspace(desc, T, dev)
+    _check("e4b_moe_backward_router", _load().e4b_moe_backward_router(
+        ctypes.byref(desc), ctypes.byref(experts), _ptr(x), T, _ptr(router_logits), _ptr(topk_idx), _ptr(topk_w),
+        _ptr(grad_out), _ptr(grad_topk_w), _ptr(grad_logits), _ptr(ws), ws.numel(), _stream(stream)))
+    return grad_topk_w, grad_logits

@@ -8,6 +8,7 @@
 
 #include "../../include/e4b.h"
 #include "e4b_internal.h"
+#include "router_backward.h"
 
 namespace e4b {
 
@@ -95,7 +96,7 @@ uint32_t* device_status_ptr() {
 // ------------------------------------------------------------ workspace layout
 struct WsLayout {
     size_t chunk_counts, chunk_base, counts, offsets, tile_prefix, sched, perm, a_perm, h, gu, dgu, dec_h, dec_plan,
-        total;
+        ones, total;
 };
 
 static size_t align_up(size_t v) { return (v + 255) & ~size_t(255); }
@@ -119,6 +120,7 @@ static WsLayout layout_for(const e4b_moe_desc* d, int64_t T) {
     L.dgu = take((size_t)P * 2 * d->I * 2);
     L.dec_h = take((size_t)P * d->I * 2);
     L.dec_plan = take(decode_plan_bytes());
+    L.ones = take((size_t)P * 4);
     L.total = off;
     return L;
 }
@@ -395,6 +397,54 @@ e4b_status e4b_moe_backward_dgrad(const e4b_moe_desc* d, const e4b_experts* w, c
     E4B_CUDA_TRY(launch_grouped_gemm(EPI_DGRAD_GATEUP, d->codebook, dgu, P, w->gate_up, q.b_rows_total, d->H / 2, q,
                                      max_m_tiles(P, d->E), st));
     E4B_CUDA_TRY(launch_combine(a_perm, topk_idx, d->E, d->top_k, T, d->H, static_cast<__nv_bfloat16*>(grad_x), st));
+    return E4B_OK;
+}
+
+e4b_status e4b_moe_backward_router(const e4b_moe_desc* d, const e4b_experts* w, const void* x, int64_t T,
+                                   const float* router_logits, const int32_t* topk_idx, const float* topk_w,
+                                   const void* grad_out, float* grad_topk_w, float* grad_logits, void* workspace,
+                                   size_t ws_bytes, void* stream) {
+    e4b_status s = check_desc(d);
+    if (s != E4B_OK) return s;
+    if ((s = check_experts(w)) != E4B_OK) return s;
+    if (T < 0 || T * d->top_k > (int64_t)INT32_MAX) return E4B_ERR_INVALID_ARG;
+    if (T == 0) return E4B_OK;
+    if (!x || !topk_idx || !topk_w || !grad_out || !grad_topk_w || (grad_logits && !router_logits))
+        return E4B_ERR_INVALID_ARG;
+    const WsLayout L = layout_for(d, T);
+    if (!workspace || ws_bytes < L.total) return E4B_ERR_WORKSPACE;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
+    const int64_t P = T * d->top_k;
+    // h recomputed through the grouped gate_up GEMM, then the unweighted expert
+    // outputs Y (the down GEMM with unit weights) into the slot rows
+    int32_t* perm = reinterpret_cast<int32_t*>(ws + L.perm);
+    E4B_CUDA_TRY(launch_group(topk_idx, P, d->E, gemm_tile_rows(), reinterpret_cast<int32_t*>(ws + L.chunk_counts),
+                              reinterpret_cast<int32_t*>(ws + L.chunk_base), reinterpret_cast<int32_t*>(ws + L.counts),
+                              reinterpret_cast<int32_t*>(ws + L.offsets), reinterpret_cast<int32_t*>(ws + L.tile_prefix),
+                              reinterpret_cast<int4*>(ws + L.sched), perm, st));
+    const int32_t* nrows = reinterpret_cast<const int32_t*>(ws + L.offsets) + d->E;
+    __nv_bfloat16* a_perm = reinterpret_cast<__nv_bfloat16*>(ws + L.a_perm);
+    E4B_CUDA_TRY(launch_gather_rows(static_cast<const __nv_bfloat16*>(x), perm, nrows, d->top_k, P, d->H, a_perm, st));
+    __nv_bfloat16* h = reinterpret_cast<__nv_bfloat16*>(ws + L.h);
+    if ((s = run_gateup(d, w, ws, L, topk_w, P, h, nullptr, st)) != E4B_OK) return s;
+    float* ones = reinterpret_cast<float*>(ws + L.ones);
+    E4B_CUDA_TRY(launch_fill_f32(ones, P, 1.0f, st));
+    GemmParams p = base_params(d, ws, L, ones, P);
+    p.K = d->I;
+    p.N = d->H;
+    p.n_tiles = (d->H + 255) / 256;
+    p.absmax = w->down_absmax;
+    p.b_rows_per_expert = d->H;
+    p.b_rows_total = (int64_t)d->E * d->H;
+    p.b_blocks_per_row = d->I / 64;
+    p.out_bf16 = a_perm;   // Y, one row per pair
+    p.ld_out = d->H;
+    E4B_CUDA_TRY(launch_grouped_gemm(EPI_DOWN, d->codebook, h, P, w->down, p.b_rows_total, d->I / 2, p,
+                                     max_m_tiles(P, d->E), st));
+    E4B_CUDA_TRY(launch_router_grad(static_cast<const __nv_bfloat16*>(grad_out), a_perm, topk_idx, topk_w,
+                                    router_logits, T, d->E, d->top_k, d->H, d->renormalize, grad_topk_w, grad_logits,
+                                    st));
     return E4B_OK;
 }
 

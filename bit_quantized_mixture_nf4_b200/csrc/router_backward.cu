@@ -1,0 +1,131 @@
+// Routing-weight and router-logit gradient of the expert layer (routing indices
+// held).  The layer output is y_t = sum_j w_{t,j} Y_{t,j}, with Y_{t,j} the
+// expert output before its routing weight ("experts4bit-qlora 0.1.0"
+// experts.py, Experts4bit.forward: the routing weight multiplies the expert
+// output).  Hence dL/dw_{t,j} = <grad_out_t, Y_{t,j}>, and the logit gradient
+// follows through the softmax that produced the weights:
+//   no renormalisation: dL/dl_i = p_i (sum_{j: e_j = i} dw_j - sum_j dw_j p_{e_j}),
+//     p = softmax over all E experts;
+//   renormalisation: dL/dl_i = sum_{j: e_j = i} w_j (dw_j - sum_j' w_j' dw_j').
+// The unweighted Y comes from the grouped down GEMM run with unit weights.
+#include "router_backward.h"
+
+namespace e4b {
+
+__global__ void __launch_bounds__(256) fill_f32_kernel(float* __restrict__ p, int64_t n, float v) {
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x)
+        p[i] = v;
+}
+
+// One warp per token: the k dot products <grad_out_t, Y_{t,j}> over H (fp32, a
+// fixed order: per-lane sums over 16-byte chunks, then a butterfly), then the
+// logit gradient of the token.
+__global__ void __launch_bounds__(256) router_grad_kernel(const __nv_bfloat16* __restrict__ grad_out,
+                                                          const __nv_bfloat16* __restrict__ Y,
+                                                          const int32_t* __restrict__ idx,
+                                                          const float* __restrict__ wts,
+                                                          const float* __restrict__ logits, int64_t T, int E,
+                                                          int k, int H, int renorm, float* __restrict__ dw_out,
+                                                          float* __restrict__ dl_out) {
+    const int lane = threadIdx.x & 31;
+    const int64_t t = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    if (t >= T) return;
+    float dw[8];
+    int ej[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+        dw[j] = 0.0f;
+        ej[j] = -1;
+        if (j >= k) continue;
+        const int64_t p = t * k + j;
+        const int e = __ldg(idx + p);
+        const bool valid = e >= 0 && e < E;
+        float acc = 0.0f;
+        if (valid) {
+            const uint4* g4 = reinterpret_cast<const uint4*>(grad_out + t * H);
+            const uint4* y4 = reinterpret_cast<const uint4*>(Y + p * H);
+            for (int c = lane; c < H / 8; c += 32) {
+                const uint4 gv = __ldg(g4 + c), yv = __ldcs(y4 + c);
+                const uint32_t gw[4] = {gv.x, gv.y, gv.z, gv.w}, yw[4] = {yv.x, yv.y, yv.z, yv.w};
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    acc = fmaf(__uint_as_float(gw[q] << 16), __uint_as_float(yw[q] << 16), acc);
+                    acc = fmaf(__uint_as_float(gw[q] & 0xFFFF0000u), __uint_as_float(yw[q] & 0xFFFF0000u), acc);
+                }
+            }
+        }
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+        dw[j] = acc;
+        ej[j] = valid ? e : -1;
+        if (lane == 0) dw_out[p] = acc;
+    }
+    if (!dl_out) return;
+    const float* l = logits + t * E;
+    float v[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) v[i] = (lane + 32 * i < E) ? __ldg(l + lane + 32 * i) : __int_as_float(0xff800000);
+    float dl[8];
+    if (renorm) {
+        float a = 0.0f;
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+            if (j < k && ej[j] >= 0) a = fmaf(__ldg(wts + t * k + j), dw[j], a);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            dl[i] = 0.0f;
+#pragma unroll
+            for (int j = 0; j < 8; ++j)
+                if (j < k && ej[j] == lane + 32 * i) dl[i] = fmaf(__ldg(wts + t * k + j), dw[j] - a, dl[i]);
+        }
+    } else {
+        float top = v[0];
+#pragma unroll
+        for (int i = 1; i < 8; ++i) top = fmaxf(top, v[i]);
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) top = fmaxf(top, __shfl_xor_sync(0xffffffffu, top, off));
+        float z = 0.0f;
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+            if (lane + 32 * i < E) z += expf(v[i] - top);
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) z += __shfl_xor_sync(0xffffffffu, z, off);
+        float a = 0.0f;
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+            if (j < k && ej[j] >= 0) a = fmaf(dw[j], expf(__ldg(l + ej[j]) - top) / z, a);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const float pi = (lane + 32 * i < E) ? expf(v[i] - top) / z : 0.0f;
+            float sel = 0.0f;
+#pragma unroll
+            for (int j = 0; j < 8; ++j)
+                if (j < k && ej[j] == lane + 32 * i) sel += dw[j];
+            dl[i] = pi * (sel - a);
+        }
+    }
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+        if (lane + 32 * i < E) dl_out[t * E + lane + 32 * i] = dl[i];
+}
+
+cudaError_t launch_fill_f32(float* p, int64_t n, float v, cudaStream_t st) {
+    if (n == 0) return cudaSuccess;
+    const int grid = (int)std::min<int64_t>((n + 255) / 256, 1184);
+    fill_f32_kernel<<<grid, 256, 0, st>>>(p, n, v);
+    count_launch();
+    return cudaGetLastError();
+}
+
+cudaError_t launch_router_grad(const __nv_bfloat16* grad_out, const __nv_bfloat16* Y, const int32_t* idx,
+                               const float* wts, const float* logits, int64_t T, int E, int k, int H, int renorm,
+                               float* dw, float* dlogits, cudaStream_t st) {
+    if (T == 0) return cudaSuccess;
+    const int64_t grid = (T * 32 + 255) / 256;
+    router_grad_kernel<<<(unsigned)grid, 256, 0, st>>>(grad_out, Y, idx, wts, logits, T, E, k, H, renorm, dw,
+                                                       dlogits);
+    count_launch();
+    return cudaGetLastError();
+}
+
+}  // namespace e4b

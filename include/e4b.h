@@ -106,8 +106,9 @@ E4B_API e4b_status e4b_dequantize_nf4(const uint8_t *packed, const float *absmax
                               int64_t in, int blocksize, e4b_codebook codebook, e4b_dtype out_dtype,
                               void *w_out, void *stream);
 
-/* Bytes of device workspace e4b_moe_forward and e4b_moe_backward_dgrad need
- * for T tokens (the larger of the two).  Returns 0 for an invalid desc. */
+/* Bytes of device workspace e4b_moe_forward, e4b_moe_backward_dgrad and
+ * e4b_moe_backward_router need for T tokens (the largest of them).  Returns 0
+ * for an invalid desc. */
 E4B_API size_t e4b_moe_workspace_size(const e4b_moe_desc *d, int64_t T);
 
 /* Forward of the expert layer ([P4] Experts4bit.forward):
@@ -153,6 +154,30 @@ E4B_API e4b_status e4b_moe_backward_dgrad(const e4b_moe_desc *d, const e4b_exper
                                   int64_t T, const int32_t *topk_idx, const float *topk_w,
                                   const void *grad_out, const void *saved_gu, void *grad_x,
                                   void *workspace, size_t ws_bytes, void *stream);
+
+/* Gradient of the layer output with respect to the routing, indices held
+ * constant: the other half of the layer backward next to e4b_moe_backward_dgrad.
+ * The forward gives y_t = sum_j w_{t,j} Y_{t,j}, with Y_{t,j} the expert output
+ * before its routing weight ([P4] Experts4bit.forward), so
+ *   grad_topk_w[t,j] = <grad_out_t, Y_{t,j}>                       (fp32 [T,k])
+ * and, through the softmax that made the weights from router_logits,
+ *   no renormalisation: grad_logits[t,i] = p_i (sum_{j: e_j = i} dw_j - sum_j dw_j p_{e_j}),
+ *                       p = softmax of the token's logits over all E;
+ *   renormalisation:    grad_logits[t,i] = sum_{j: e_j = i} w_j (dw_j - sum_j' w_j' dw_j'),
+ *                       w = topk_w (logits outside the top-k get 0).
+ * Y is recomputed from x through the grouped GEMMs (gate_up, then down with unit
+ * weights), rounded to bf16 like every slot row; the dot products and the
+ * softmax backward run in fp32.
+ *   x bf16 [T,H], router_logits fp32 [T,E] (needed only for grad_logits),
+ *   topk_idx int32 [T,k], topk_w fp32 [T,k] (the forward's), grad_out bf16 [T,H],
+ *   grad_topk_w fp32 [T,k] (written; 0 for an out-of-range expert),
+ *   grad_logits fp32 [T,E] (written) or NULL,
+ *   workspace as for e4b_moe_forward (e4b_moe_workspace_size bytes).
+ * Returns E4B_ERR_INVALID_ARG when grad_logits is given without router_logits. */
+E4B_API e4b_status e4b_moe_backward_router(const e4b_moe_desc *d, const e4b_experts *w, const void *x,
+                                   int64_t T, const float *router_logits, const int32_t *topk_idx,
+                                   const float *topk_w, const void *grad_out, float *grad_topk_w,
+                                   float *grad_logits, void *workspace, size_t ws_bytes, void *stream);
 
 /* Forward without any device memory from the caller.  The source pages have no
  * counterpart: this is an interface for callers that cannot give the library
