@@ -25,7 +25,8 @@ PATH_AUTO, PATH_GROUPED, PATH_DECODE = 0, 1, 2
 
 EXPORTS = ("e4b_quantize_nf4", "e4b_dequantize_nf4", "e4b_moe_workspace_size", "e4b_moe_forward",
            "e4b_moe_backward_dgrad", "e4b_moe_backward_router", "e4b_device_status", "e4b_status_string",
-           "e4b_launch_count", "e4b_timing_enable", "e4b_timing_reset", "e4b_timing_get", "e4b_moe_forward_noalloc")
+           "e4b_launch_count", "e4b_timing_enable", "e4b_timing_reset", "e4b_timing_get", "e4b_moe_forward_noalloc",
+           "e4b_watchdog_selftest")
 # kernel kinds of e4b_timing_get
 KERNEL_KINDS = ("quantize", "dequantize", "route", "group", "gather", "combine", "gemm_gateup", "gemm_down",
                 "gemm_dgrad_down", "gemm_dgrad_gateup", "decode_gateup", "decode_down")
@@ -72,6 +73,7 @@ def _load():
     lib.e4b_moe_backward_router.argtypes = [ctypes.POINTER(e4b_moe_desc), ctypes.POINTER(e4b_experts), P, i64, P, P,
                                             P, P, P, P, P, sz, P]
     lib.e4b_device_status.argtypes = [P]
+    lib.e4b_watchdog_selftest.argtypes = [P]
     lib.e4b_status_string.argtypes = [i32]
     lib.e4b_status_string.restype = ctypes.c_char_p
     lib.e4b_launch_count.restype = ctypes.c_uint64
@@ -81,7 +83,7 @@ def _load():
     lib.e4b_timing_get.argtypes = [i32, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_uint64)]
     lib.e4b_timing_get.restype = ctypes.c_int
     for f in ("e4b_quantize_nf4", "e4b_dequantize_nf4", "e4b_moe_forward", "e4b_moe_backward_dgrad",
-              "e4b_device_status", "e4b_moe_forward_noalloc", "e4b_moe_backward_router"):
+              "e4b_device_status", "e4b_moe_forward_noalloc", "e4b_moe_backward_router", "e4b_watchdog_selftest"):
         getattr(lib, f).restype = ctypes.c_int
     _lib = lib
     return lib
@@ -278,3 +280,8 @@ def e4b_moe_backward_router(desc: e4b_moe_desc, experts: e4b_experts, x, topk_id
         ctypes.byref(desc), ctypes.byref(experts), _ptr(x), T, _ptr(router_logits), _ptr(topk_idx), _ptr(topk_w),
         _ptr(grad_out), _ptr(grad_topk_w), _ptr(grad_logits), _ptr(ws), ws.numel(), _stream(stream)))
     return grad_topk_w, grad_logits
+
+
+def e4b_watchdog_selftest(stream=None):
+    """Launch the watchdog self-test kernel (a bounded wait that must time out)."""
+    _check("e4b_watchdog_selftest", _load().e4b_watchdog_selftest(_stream(stream)))

@@ -210,6 +210,14 @@ E4B_API e4b_status e4b_moe_forward_noalloc(const e4b_moe_desc *d, const e4b_expe
  * call.  E4B_ERR_CUDA if the synchronization itself fails. */
 E4B_API e4b_status e4b_device_status(void *stream);
 
+/* Diagnostic: launches one kernel whose single thread waits, through the same
+ * bounded mbarrier wait every pipelined kernel uses, on a barrier nothing
+ * arrives at.  After the wait's 2 s limit the kernel records the timeout in the
+ * device status word and returns (nothing faults, traps or hangs), so the next
+ * e4b_device_status() returns E4B_ERR_TIMEOUT and clears it; the context stays
+ * usable.  Returns E4B_OK once the kernel is launched. */
+E4B_API e4b_status e4b_watchdog_selftest(void *stream);
+
 /* Static description of a status code. */
 E4B_API const char *e4b_status_string(e4b_status s);
 
