@@ -25,8 +25,9 @@ PATH_AUTO, PATH_GROUPED, PATH_DECODE = 0, 1, 2
 
 EXPORTS = ("e4b_quantize_nf4", "e4b_dequantize_nf4", "e4b_moe_workspace_size", "e4b_moe_forward",
            "e4b_moe_backward_dgrad", "e4b_moe_backward_router", "e4b_device_status", "e4b_status_string",
-           "e4b_launch_count", "e4b_timing_enable", "e4b_timing_reset", "e4b_timing_get", "e4b_moe_forward_noalloc",
-           "e4b_watchdog_selftest")
+           "e4b_launch_count", "e4b_timing_enable", "e4b_timing_enable_kinds", "e4b_timing_reset", "e4b_timing_get",
+           "e4b_moe_forward_noalloc", "e4b_watchdog_selftest", "e4b_pipe_arena_size", "e4b_pipe_create",
+           "e4b_pipe_submit", "e4b_pipe_join", "e4b_pipe_sync", "e4b_pipe_destroy")
 # kernel kinds of e4b_timing_get
 KERNEL_KINDS = ("quantize", "dequantize", "route", "group", "gather", "combine", "gemm_gateup", "gemm_down",
                 "gemm_dgrad_down", "gemm_dgrad_gateup", "decode_gateup", "decode_down")
@@ -79,6 +80,17 @@ def _load():
     lib.e4b_launch_count.restype = ctypes.c_uint64
     lib.e4b_timing_enable.argtypes = [i32]
     lib.e4b_timing_enable.restype = None
+    lib.e4b_timing_enable_kinds.argtypes = [ctypes.c_uint32]
+    lib.e4b_pipe_arena_size.argtypes = [ctypes.POINTER(e4b_moe_desc), i64]
+    lib.e4b_pipe_arena_size.restype = sz
+    lib.e4b_pipe_create.argtypes = [ctypes.POINTER(e4b_moe_desc), ctypes.POINTER(e4b_experts), i64, P, sz, P,
+                                    ctypes.POINTER(ctypes.c_void_p)]
+    lib.e4b_pipe_submit.argtypes = [P, i64, P, P, P, P, P]
+    lib.e4b_pipe_join.argtypes = [P]
+    lib.e4b_pipe_sync.argtypes = [P]
+    lib.e4b_pipe_destroy.argtypes = [P]
+    lib.e4b_pipe_destroy.restype = None
+    lib.e4b_timing_enable_kinds.restype = None
     lib.e4b_timing_reset.restype = None
     lib.e4b_timing_get.argtypes = [i32, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_uint64)]
     lib.e4b_timing_get.restype = ctypes.c_int
@@ -130,6 +142,14 @@ def e4b_launch_count() -> int:
 
 def e4b_timing_enable(on: bool = True):
     _load().e4b_timing_enable(int(bool(on)))
+
+
+def e4b_timing_enable_kinds(kinds):
+    """Time only the given kernel kinds (indices or names in KERNEL_KINDS); empty turns timing off."""
+    mask = 0
+    for k in kinds:
+        mask |= 1 << (KERNEL_KINDS.index(k) if isinstance(k, str) else int(k))
+    _load().e4b_timing_enable_kinds(mask)
 
 
 def e4b_timing_reset():
@@ -285,3 +305,62 @@ def e4b_moe_backward_router(desc: e4b_moe_desc, experts: e4b_experts, x, topk_id
 def e4b_watchdog_selftest(stream=None):
     """Launch the watchdog self-test kernel (a bounded wait that must time out)."""
     _check("e4b_watchdog_selftest", _load().e4b_watchdog_selftest(_stream(stream)))
+
+
+# ------------------------------------------------------------- pipelined host-buffer steps
+
+def _host(t: torch.Tensor, name: str, dtype, shape):
+    if t.is_cuda or not t.is_pinned():
+        raise ValueError(f"{name} must be a page-locked host tensor (pin_memory())")
+    if t.dtype != dtype or tuple(t.shape) != tuple(shape) or not t.is_contiguous():
+        raise ValueError(f"{name} must be a contiguous {dtype} tensor of shape {tuple(shape)}")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def e4b_pipe_arena_size(desc: e4b_moe_desc, T_max: int) -> int:
+    return int(_load().e4b_pipe_arena_size(ctypes.byref(desc), T_max))
+
+
+class e4b_pipe:
+    """Handle of a pipelined host-buffer step runner (e4b_pipe_create): owns the
+    device arena tensor and keeps the descriptor and expert tensors alive."""
+
+    def __init__(self, handle, arena, desc, experts, T_max):
+        self.handle, self.arena, self.desc, self.experts, self.T_max = handle, arena, desc, experts, T_max
+
+
+def e4b_pipe_create(desc: e4b_moe_desc, experts: e4b_experts, T_max: int, device="cuda", stream=None) -> e4b_pipe:
+    size = e4b_pipe_arena_size(desc, T_max)
+    if size == 0:
+        raise ValueError("invalid descriptor or T_max")
+    arena = torch.empty(size, dtype=torch.uint8, device=device)
+    h = ctypes.c_void_p()
+    _check("e4b_pipe_create", _load().e4b_pipe_create(ctypes.byref(desc), ctypes.byref(experts), T_max,
+                                                      _ptr(arena), size, _stream(stream), ctypes.byref(h)))
+    return e4b_pipe(h, arena, desc, experts, T_max)
+
+
+def e4b_pipe_submit(pipe: e4b_pipe, x, router_logits, grad_out, y, grad_x):
+    """Enqueue one batch: pinned host x [T,H] bf16, router_logits [T,E] fp32,
+    grad_out [T,H] bf16 in; pinned host y and grad_x [T,H] bf16 out (valid after
+    a later e4b_pipe_join/e4b_pipe_sync)."""
+    d = pipe.desc
+    T = x.shape[0]
+    args = (_host(x, "x", torch.bfloat16, (T, d.H)), _host(router_logits, "router_logits", torch.float32, (T, d.E)),
+            _host(grad_out, "grad_out", torch.bfloat16, (T, d.H)), _host(y, "y", torch.bfloat16, (T, d.H)),
+            _host(grad_x, "grad_x", torch.bfloat16, (T, d.H)))
+    _check("e4b_pipe_submit", _load().e4b_pipe_submit(pipe.handle, T, *args))
+
+
+def e4b_pipe_join(pipe: e4b_pipe):
+    _check("e4b_pipe_join", _load().e4b_pipe_join(pipe.handle))
+
+
+def e4b_pipe_sync(pipe: e4b_pipe):
+    _check("e4b_pipe_sync", _load().e4b_pipe_sync(pipe.handle))
+
+
+def e4b_pipe_destroy(pipe: e4b_pipe):
+    if pipe.handle:
+        _load().e4b_pipe_destroy(pipe.handle)
+        pipe.handle = None

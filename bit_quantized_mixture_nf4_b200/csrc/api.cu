@@ -19,6 +19,7 @@ void count_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
 struct TimingState {
     std::mutex mu;
     bool on = false;
+    uint32_t mask = 0;   // bit k set: launches of kind k are timed
     std::vector<std::pair<cudaEvent_t, cudaEvent_t>> pending[KK_COUNT];
     cudaEvent_t open[KK_COUNT] = {};
     double total_ms[KK_COUNT] = {};
@@ -34,7 +35,7 @@ static cudaEvent_t new_event() {
 
 void timing_begin(int kind, cudaStream_t st) {
     std::lock_guard<std::mutex> lock(g_timing.mu);
-    if (!g_timing.on) return;
+    if (!g_timing.on || !((g_timing.mask >> kind) & 1u)) return;
     g_timing.open[kind] = new_event();
     cudaEventRecord(g_timing.open[kind], st);
 }
@@ -205,10 +206,19 @@ const char* e4b_status_string(e4b_status s) {
 
 uint64_t e4b_launch_count(void) { return g_launches.load(); }
 
-void e4b_timing_enable(int on) {
+void e4b_timing_enable(int on) { e4b_timing_enable_kinds(on ? 0xFFFFFFFFu : 0u); }
+
+void e4b_timing_enable_kinds(uint32_t mask) {
     std::lock_guard<std::mutex> lock(g_timing.mu);
     timing_collect();
-    g_timing.on = on != 0;
+    for (int k = 0; k < KK_COUNT; ++k) {   // a kind switched off mid-launch drops its open event
+        if (g_timing.open[k] && !((mask >> k) & 1u)) {
+            cudaEventDestroy(g_timing.open[k]);
+            g_timing.open[k] = nullptr;
+        }
+    }
+    g_timing.mask = mask;
+    g_timing.on = mask != 0;
 }
 
 void e4b_timing_reset(void) {

@@ -10,6 +10,19 @@
 
 namespace e4b {
 
+// Programmatic dependent launch: the grouping chain (route, histogram, scan,
+// scatter, gather) is launched with programmatic stream serialization, so a
+// kernel's blocks are resident while its predecessor drains.  Every kernel of
+// the chain waits for its predecessor's completion (and memory) before it reads
+// anything the predecessor wrote; since each one waits before it can finish,
+// completion is ordered along the whole chain.  A chained kernel's lifetime
+// overlaps its predecessors', so what they write is not read-only for it: the
+// chain reads through L2 (ld.global.cg), never through the non-coherent path.
+__device__ __forceinline__ void chain_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void chain_release() { asm volatile("griddepcontrol.launch_dependents;"); }
+
+constexpr int kMaxTopK = 8;   // the entry points reject top_k > 8
+
 // One warp per token (the per-token routing is route_token_warp, shared with
 // the small-batch kernels).
 __global__ void __launch_bounds__(256) route_kernel(const float* __restrict__ logits, int64_t T, int E, int k,
@@ -17,6 +30,8 @@ __global__ void __launch_bounds__(256) route_kernel(const float* __restrict__ lo
                                                     float* __restrict__ wts) {
     const int lane = threadIdx.x & 31;
     const int64_t t = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    chain_release();
+    chain_wait();
     if (t >= T) return;
     int e;
     float p;
@@ -28,62 +43,96 @@ __global__ void __launch_bounds__(256) route_kernel(const float* __restrict__ lo
 }
 
 // Per-chunk expert histogram (order-independent, so atomics keep it exact).
+// chunk_counts is expert-major: [E][nchunks].
 __global__ void __launch_bounds__(256) hist_kernel(const int32_t* __restrict__ idx, int64_t P, int E,
                                                    int32_t* __restrict__ chunk_counts) {
     __shared__ int cnt[256];
     for (int e = threadIdx.x; e < E; e += blockDim.x) cnt[e] = 0;
+    chain_release();
+    chain_wait();
     __syncthreads();
     const int64_t p0 = (int64_t)blockIdx.x * kChunkPairs;
     for (int i = threadIdx.x; i < kChunkPairs; i += blockDim.x) {
         const int64_t pp = p0 + i;
         if (pp < P) {
-            const int e = __ldg(idx + pp);
+            const int e = __ldcg(idx + pp);
             if (e >= 0 && e < E) atomicAdd(&cnt[e], 1);   // out-of-range experts are dropped
         }
     }
     __syncthreads();
-    for (int e = threadIdx.x; e < E; e += blockDim.x) chunk_counts[(int64_t)blockIdx.x * E + e] = cnt[e];
+    for (int e = threadIdx.x; e < E; e += blockDim.x) chunk_counts[(int64_t)e * gridDim.x + blockIdx.x] = cnt[e];
 }
 
-// Single block: totals, exclusive scan over experts, per-chunk bases, m-tile prefix.
-__global__ void __launch_bounds__(256) scan_kernel(const int32_t* __restrict__ chunk_counts, int nchunks, int E,
-                                                   int tile_rows, int32_t* __restrict__ chunk_base,
-                                                   int32_t* __restrict__ counts, int32_t* __restrict__ offsets,
-                                                   int32_t* __restrict__ tile_prefix, int4* __restrict__ sched) {
-    __shared__ int s_tot[256], s_tiles[256];
-    const int e = threadIdx.x;
-    int tot = 0;
-    if (e < E)
-        for (int c = 0; c < nchunks; ++c) tot += chunk_counts[(int64_t)c * E + e];
-    s_tot[e] = (e < E) ? tot : 0;
-    s_tiles[e] = (e < E) ? (tot + tile_rows - 1) / tile_rows : 0;
-    __syncthreads();
-    if (e == 0) {   // E <= 256: a serial scan is short and exact
-        int run = 0, trun = 0;
-        for (int i = 0; i < E; ++i) {
-            const int a = s_tot[i], b = s_tiles[i];
-            s_tot[i] = run;
-            s_tiles[i] = trun;
-            run += a;
-            trun += b;
-        }
-        offsets[E] = run;
-        tile_prefix[E] = trun;
+__device__ __forceinline__ int warp_inclusive_scan(int v, int lane) {
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int u = __shfl_up_sync(0xffffffffu, v, o);
+        if (lane >= o) v += u;
+    }
+    return v;
+}
+
+// Single block of 1024 threads: expert totals, exclusive scans over experts (rows
+// and m-tiles), per-chunk bases and the m-tile schedule.  A warp owns experts
+// warp, warp+32, ...; it walks an expert's chunk counts (contiguous, expert-major)
+// 32 at a time with a running carry.
+__global__ void __launch_bounds__(1024) scan_kernel(const int32_t* __restrict__ chunk_counts, int nchunks, int E,
+                                                    int tile_rows, int32_t* __restrict__ chunk_base,
+                                                    int32_t* __restrict__ counts, int32_t* __restrict__ offsets,
+                                                    int32_t* __restrict__ tile_prefix, int4* __restrict__ sched) {
+    __shared__ int s_tot[256], s_off[256], s_toff[256];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
+    chain_release();
+    chain_wait();
+    for (int e = warp; e < E; e += nw) {
+        const int32_t* c = chunk_counts + (int64_t)e * nchunks;
+        int sum = 0;
+        for (int i = lane; i < nchunks; i += 32) sum += __ldcg(c + i);
+        sum = __reduce_add_sync(0xffffffffu, sum);
+        if (lane == 0) s_tot[e] = sum;
     }
     __syncthreads();
-    if (e < E) {
-        counts[e] = tot;
-        offsets[e] = s_tot[e];
-        tile_prefix[e] = s_tiles[e];
-        int run = s_tot[e];
-        for (int c = 0; c < nchunks; ++c) {
-            chunk_base[(int64_t)c * E + e] = run;
-            run += chunk_counts[(int64_t)c * E + e];
+    if (warp == 0) {   // exclusive scans of the row counts and m-tile counts over experts
+        int run = 0, trun = 0;
+        for (int e0 = 0; e0 < E; e0 += 32) {
+            const int e = e0 + lane;
+            const int v = e < E ? s_tot[e] : 0;
+            const int tv = (v + tile_rows - 1) / tile_rows;
+            const int x = warp_inclusive_scan(v, lane), tx = warp_inclusive_scan(tv, lane);
+            if (e < E) {
+                s_off[e] = run + x - v;
+                s_toff[e] = trun + tx - tv;
+            }
+            run += __shfl_sync(0xffffffffu, x, 31);
+            trun += __shfl_sync(0xffffffffu, tx, 31);
+        }
+        if (lane == 0) {
+            offsets[E] = run;
+            tile_prefix[E] = trun;
+        }
+    }
+    __syncthreads();
+    for (int e = warp; e < E; e += nw) {
+        const int32_t* c = chunk_counts + (int64_t)e * nchunks;
+        int32_t* b = chunk_base + (int64_t)e * nchunks;
+        const int tot = s_tot[e], off = s_off[e], toff = s_toff[e];
+        int run = off;
+        for (int i0 = 0; i0 < nchunks; i0 += 32) {
+            const int i = i0 + lane;
+            const int v = i < nchunks ? __ldcg(c + i) : 0;
+            const int x = warp_inclusive_scan(v, lane);
+            if (i < nchunks) b[i] = run + x - v;
+            run += __shfl_sync(0xffffffffu, x, 31);
+        }
+        if (lane == 0) {
+            counts[e] = tot;
+            offsets[e] = off;
+            tile_prefix[e] = toff;
         }
         // m-tile schedule: (expert, first row, rows) of every m-tile, experts ascending
         const int nt = (tot + tile_rows - 1) / tile_rows;
-        for (int m = 0; m < nt; ++m)
-            sched[s_tiles[e] + m] = make_int4(e, s_tot[e] + m * tile_rows, min(tile_rows, tot - m * tile_rows), 0);
+        for (int m = lane; m < nt; m += 32)
+            sched[toff + m] = make_int4(e, off + m * tile_rows, min(tile_rows, tot - m * tile_rows), 0);
     }
 }
 
@@ -95,18 +144,20 @@ __global__ void __launch_bounds__(256) scatter_kernel(const int32_t* __restrict_
     __shared__ int wbase[WARPS][256];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     for (int i = threadIdx.x; i < WARPS * 256; i += blockDim.x) (&wbase[0][0])[i] = 0;
+    chain_release();
+    chain_wait();
     __syncthreads();
     const int64_t p0 = (int64_t)blockIdx.x * kChunkPairs + warp * PER_WARP;
     for (int it = 0; it < PER_WARP; it += 32) {
         const int64_t pp = p0 + it + lane;
         if (pp < P) {
-            const int e = __ldg(idx + pp);
+            const int e = __ldcg(idx + pp);
             if (e >= 0 && e < E) atomicAdd(&wbase[warp][e], 1);
         }
     }
     __syncthreads();
     for (int e = threadIdx.x; e < E; e += blockDim.x) {
-        int run = chunk_base[(int64_t)blockIdx.x * E + e];
+        int run = __ldcg(chunk_base + (int64_t)e * gridDim.x + blockIdx.x);
         for (int w = 0; w < WARPS; ++w) {
             const int c = wbase[w][e];
             wbase[w][e] = run;
@@ -117,7 +168,7 @@ __global__ void __launch_bounds__(256) scatter_kernel(const int32_t* __restrict_
     const uint32_t lt_mask = (1u << lane) - 1u;
     for (int it = 0; it < PER_WARP; it += 32) {
         const int64_t pp = p0 + it + lane;
-        int e = (pp < P) ? __ldg(idx + pp) : -1;
+        int e = (pp < P) ? __ldcg(idx + pp) : -1;
         if (e >= E) e = -1;
         const uint32_t peers = __match_any_sync(0xffffffffu, e);
         const int rank = __popc(peers & lt_mask);
@@ -131,20 +182,32 @@ __global__ void __launch_bounds__(256) scatter_kernel(const int32_t* __restrict_
     }
 }
 
-// dst[r] = src[perm[r] / k]: one warp per row, 16-byte vectors.
+// dst[r] = src[perm[r] / k]: one warp per row, 16-byte vectors, four loads in
+// flight per lane before the stores.
 __global__ void __launch_bounds__(256) gather_rows_kernel(const __nv_bfloat16* __restrict__ src,
                                                           const int32_t* __restrict__ perm,
                                                           const int32_t* __restrict__ nrows, int k, int64_t P,
                                                           int H, __nv_bfloat16* __restrict__ dst) {
     const int lane = threadIdx.x & 31;
-    P = min(P, (int64_t)__ldg(nrows));   // rows that belong to a valid expert
+    chain_release();
+    chain_wait();
+    P = min(P, (int64_t)__ldcg(nrows));   // rows that belong to a valid expert
     const int64_t wstride = (int64_t)gridDim.x * blockDim.x / 32;
     const int vec = H / 8;
     for (int64_t r = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) / 32; r < P; r += wstride) {
-        const int64_t t = __ldg(perm + r) / k;
+        const int64_t t = __ldcg(perm + r) / k;
         const uint4* s = reinterpret_cast<const uint4*>(src + t * H);
         uint4* d = reinterpret_cast<uint4*>(dst + r * H);
-        for (int i = lane; i < vec; i += 32) d[i] = __ldg(s + i);
+#pragma unroll 1
+        for (int i0 = lane; i0 < vec; i0 += 128) {
+            uint4 v[4];
+#pragma unroll
+            for (int q = 0; q < 4; ++q)
+                if (i0 + 32 * q < vec) v[q] = __ldcg(s + i0 + 32 * q);
+#pragma unroll
+            for (int q = 0; q < 4; ++q)
+                if (i0 + 32 * q < vec) d[i0 + 32 * q] = v[q];
+        }
     }
 }
 
@@ -162,11 +225,19 @@ __global__ void __launch_bounds__(256) combine_kernel(const __nv_bfloat16* __res
         const int64_t t = i / h8;
         const int c = (int)(i - t * h8);
         float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-        for (int j = 0; j < k; ++j) {
-            const int e = __ldg(idx + t * k + j);
-            if (e < 0 || e >= E) continue;
-            const uint4 v = __ldcs(reinterpret_cast<const uint4*>(slots + (t * k + j) * H) + c);
-            const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+        uint4 v[kMaxTopK];
+#pragma unroll
+        for (int j = 0; j < kMaxTopK; ++j) {   // every slot's vector in flight before the sums
+            v[j] = make_uint4(0u, 0u, 0u, 0u);
+            if (j < k) {
+                const int e = __ldg(idx + t * k + j);
+                if (e >= 0 && e < E) v[j] = __ldcs(reinterpret_cast<const uint4*>(slots + (t * k + j) * H) + c);
+            }
+        }
+#pragma unroll
+        for (int j = 0; j < kMaxTopK; ++j) {
+            if (j >= k) break;
+            const uint32_t w[4] = {v[j].x, v[j].y, v[j].z, v[j].w};
 #pragma unroll
             for (int q = 0; q < 4; ++q) {
                 acc[2 * q] += __uint_as_float(w[q] << 16);
@@ -182,15 +253,33 @@ static int capped_grid(int64_t blocks) {
     return (int)std::max<int64_t>(1, std::min<int64_t>(blocks, (int64_t)num_sms() * 16));
 }
 
+// Launch with programmatic stream serialization (the kernel calls chain_wait
+// before it reads its predecessors' output).
+template <typename... KArgs, typename... Args>
+static cudaError_t launch_chained(void (*kernel)(KArgs...), unsigned grid, unsigned block, cudaStream_t st,
+                                  Args... args) {
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(block);
+    cfg.dynamicSmemBytes = 0;
+    cfg.stream = st;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
+}
+
 cudaError_t launch_route(const float* logits, int64_t T, int E, int k, int renorm, int32_t* idx, float* w,
                          cudaStream_t st) {
     if (T == 0) return cudaSuccess;
     const int64_t blocks = (T * 32 + 255) / 256;
     timing_begin(KK_ROUTE, st);
-    route_kernel<<<(unsigned)blocks, 256, 0, st>>>(logits, T, E, k, renorm, idx, w);
+    const cudaError_t err = launch_chained(route_kernel, (unsigned)blocks, 256, st, logits, T, E, k, renorm, idx, w);
     timing_end(KK_ROUTE, st);
     count_launch();
-    return cudaGetLastError();
+    return err;
 }
 
 cudaError_t launch_group(const int32_t* idx, int64_t P, int E, int tile_rows, int32_t* chunk_counts,
@@ -199,25 +288,27 @@ cudaError_t launch_group(const int32_t* idx, int64_t P, int E, int tile_rows, in
     const int nchunks = (int)((P + kChunkPairs - 1) / kChunkPairs);
     if (nchunks == 0) return cudaSuccess;
     timing_begin(KK_GROUP, st);
-    hist_kernel<<<nchunks, 256, 0, st>>>(idx, P, E, chunk_counts);
-    scan_kernel<<<1, 256, 0, st>>>(chunk_counts, nchunks, E, tile_rows, chunk_base, counts, offsets, tile_prefix,
-                                   sched);
-    scatter_kernel<<<nchunks, 256, 0, st>>>(idx, P, E, chunk_base, perm);
+    cudaError_t err = launch_chained(hist_kernel, nchunks, 256, st, idx, P, E, chunk_counts);
+    if (err == cudaSuccess)
+        err = launch_chained(scan_kernel, 1, 1024, st, chunk_counts, nchunks, E, tile_rows, chunk_base, counts, offsets,
+                             tile_prefix, sched);
+    if (err == cudaSuccess) err = launch_chained(scatter_kernel, nchunks, 256, st, idx, P, E, chunk_base, perm);
     timing_end(KK_GROUP, st);
     count_launch();
     count_launch();
     count_launch();
-    return cudaGetLastError();
+    return err;
 }
 
 cudaError_t launch_gather_rows(const __nv_bfloat16* src, const int32_t* perm, const int32_t* nrows, int k,
                                int64_t P, int H, __nv_bfloat16* dst, cudaStream_t st) {
     if (P == 0) return cudaSuccess;
     timing_begin(KK_GATHER, st);
-    gather_rows_kernel<<<capped_grid((P * 32 + 255) / 256), 256, 0, st>>>(src, perm, nrows, k, P, H, dst);
+    const cudaError_t err =
+        launch_chained(gather_rows_kernel, capped_grid((P * 32 + 255) / 256), 256, st, src, perm, nrows, k, P, H, dst);
     timing_end(KK_GATHER, st);
     count_launch();
-    return cudaGetLastError();
+    return err;
 }
 
 cudaError_t launch_combine(const __nv_bfloat16* slots, const int32_t* idx, int E, int k, int64_t T, int H,

@@ -205,6 +205,47 @@ E4B_API e4b_status e4b_moe_forward_noalloc(const e4b_moe_desc *d, const e4b_expe
                                            int64_t T, const float *router_logits, int32_t *topk_idx,
                                            float *topk_w, void *y, void *stream);
 
+/* Pipelined steps through PINNED host buffers: the expert layer's forward
+ * (routed from router logits) and its input gradient for a stream of batches
+ * that live in host memory.  Each e4b_pipe_submit
+ *   - copies the batch's x [T,H] bf16, router logits [T,E] fp32 and grad_out
+ *     [T,H] bf16 to the device on the pipe's copy-in stream,
+ *   - runs e4b_moe_forward (g/u saved) and e4b_moe_backward_dgrad on the
+ *     compute stream given at creation,
+ *   - copies y [T,H] and grad_x [T,H] (bf16) back on the pipe's copy-out
+ *     stream, y as soon as the forward is done.
+ * Two device buffer sets alternate between consecutive submits, so batch n+1's
+ * input copies and batch n-1's output copies run under batch n's kernels; the
+ * saved g/u and the workspace are shared (the compute stream orders them).
+ * Results are exactly those of the two calls on device copies of the inputs.
+ *
+ * arena: caller-owned device memory of e4b_pipe_arena_size(d, T_max) bytes,
+ * 256-byte aligned, alive until e4b_pipe_destroy.  Host pointers passed to
+ * submit must be page-locked (cudaHostAlloc / cudaHostRegister); the inputs
+ * must stay unchanged and the outputs unread until a later e4b_pipe_join or
+ * e4b_pipe_sync covers the submit.  `w` is copied at creation (the weight
+ * memory it points to must stay alive).  A pipe is used from one host thread
+ * at a time.  Creation makes two non-blocking CUDA streams and a few events
+ * (host-side driver objects; no device memory is allocated). */
+typedef struct e4b_pipe e4b_pipe;
+E4B_API size_t e4b_pipe_arena_size(const e4b_moe_desc *d, int64_t T_max);
+E4B_API e4b_status e4b_pipe_create(const e4b_moe_desc *d, const e4b_experts *w, int64_t T_max, void *arena,
+                                   size_t arena_bytes, void *stream, e4b_pipe **out);
+/* Enqueues one batch (0 <= T <= T_max; T = 0 is a no-op) and returns without
+ * waiting for it.  Shape and pointer errors return before anything is enqueued. */
+E4B_API e4b_status e4b_pipe_submit(e4b_pipe *p, int64_t T, const void *x_host, const float *logits_host,
+                                   const void *grad_out_host, void *y_host, void *grad_x_host);
+/* Fork/join point, without waiting on the host: work enqueued on the compute
+ * stream after the call runs after every batch submitted so far (copies
+ * included), and the pipe's copies of later submits run after the work already
+ * enqueued on the compute stream. */
+E4B_API e4b_status e4b_pipe_join(e4b_pipe *p);
+/* e4b_pipe_join, then waits on the host for the compute stream and returns
+ * e4b_device_status of it. */
+E4B_API e4b_status e4b_pipe_sync(e4b_pipe *p);
+/* Waits for the pipe's streams, then releases its streams and events.  NULL is a no-op. */
+E4B_API void e4b_pipe_destroy(e4b_pipe *p);
+
 /* Synchronizes `stream`, then reads and clears the library's device status
  * word: E4B_OK, or E4B_ERR_TIMEOUT if a kernel gave up on a wait since the last
  * call.  E4B_ERR_CUDA if the synchronization itself fails. */
@@ -233,6 +274,10 @@ E4B_API uint64_t e4b_launch_count(void);
  * 6 grouped gate_up GEMM, 7 grouped down GEMM, 8 dgrad down GEMM,
  * 9 dgrad gate_up GEMM, 10 decode gate_up GEMV, 11 decode down GEMV. */
 E4B_API void e4b_timing_enable(int on);
+/* Times only the kinds whose bit is set in mask (bit k = kind k above); 0 turns
+ * timing off.  e4b_timing_enable(1) equals a mask with every bit set.  A kind
+ * left untimed records no events, so its launches run back to back. */
+E4B_API void e4b_timing_enable_kinds(uint32_t mask);
 E4B_API void e4b_timing_reset(void);
 E4B_API e4b_status e4b_timing_get(int kind, double *total_ms, uint64_t *launches);
 

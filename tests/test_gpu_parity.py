@@ -311,3 +311,28 @@ def test_single_expert_dense_mlp(e4b):
     oi, ow = _check_routing(prob, r)
     yref, gref = pb.oracle_forward_dgrad(prob, oi, ow, np.arange(w.T))
     pb.assert_close_rel_max(r["y"].float().cpu().numpy(), yref, TOL, "dense forward")
+
+
+def test_consecutive_shapes_share_workspace(e4b):
+    """Back-to-back grouped forwards of different layers through one workspace:
+    the second call's routing, grouping and output must not see anything the
+    first call left in the workspace (or in any cache in front of it)."""
+    ws_shapes = [pb.custom("seqA", E=16, H=256, I=192, k=4, T=700, seed=41),
+                 pb.custom("seqB", E=6, H=320, I=128, k=2, renorm=False, T=450, seed=42),
+                 pb.custom("seqC", E=16, H=256, I=192, k=3, T=523, seed=43)]
+    probs = [pb.build(w) for w in ws_shapes]
+    size = max(e4b.e4b_moe_workspace_size(_desc(e4b, w, e4b.PATH_GROUPED), w.T) for w in ws_shapes)
+    ws = torch.empty(size, dtype=torch.uint8, device="cuda")
+    for rnd in range(2):
+        for w, prob in zip(ws_shapes, probs):
+            _, experts = _upload_experts(e4b, prob)
+            d = _desc(e4b, w, e4b.PATH_GROUPED)
+            x, logits = pb.to_dev(prob.x), pb.to_dev(prob.logits)
+            offs = torch.empty(w.E + 1, dtype=torch.int32, device="cuda")
+            perm = torch.empty(w.T * w.k, dtype=torch.int32, device="cuda")
+            y, idx, wts = e4b.e4b_moe_forward(d, experts, x, logits, offsets_out=offs, perm_out=perm, ws=ws)
+            torch.cuda.synchronize()
+            _check_status(e4b)
+            oi, ow = _check_routing(prob, dict(idx=idx, wts=wts, offs=offs, perm=perm))
+            yref, _ = pb.oracle_forward_dgrad(prob, oi, ow, np.arange(w.T), want_dgrad=False)
+            pb.assert_close_rel_max(y.float().cpu().numpy(), yref, TOL, f"forward {w.name} (pass {rnd})")
