@@ -96,7 +96,7 @@ uint32_t* device_status_ptr() {
 
 // ------------------------------------------------------------ workspace layout
 struct WsLayout {
-    size_t chunk_counts, chunk_base, counts, offsets, tile_prefix, sched, perm, a_perm, h, gu, dgu, dec_h, dec_plan,
+    size_t chunk_counts, chunk_base, counts, offsets, tile_prefix, sched, perm, inv_perm, a_perm, h, gu, dgu, dec_h, dec_plan,
         ones, total;
 };
 
@@ -115,6 +115,7 @@ static WsLayout layout_for(const e4b_moe_desc* d, int64_t T) {
     L.tile_prefix = take((size_t)(d->E + 1) * 4);
     L.sched = take(((size_t)(P + gemm_tile_rows() - 1) / gemm_tile_rows() + d->E) * 16);
     L.perm = take((size_t)P * 4);
+    L.inv_perm = take((size_t)P * 4);
     L.a_perm = take((size_t)P * d->H * 2);
     L.h = take((size_t)P * d->I * 2);
     L.gu = take((size_t)P * 2 * d->I * 2);
@@ -322,7 +323,8 @@ e4b_status e4b_moe_forward(const e4b_moe_desc* d, const e4b_experts* w, const vo
     E4B_CUDA_TRY(launch_group(topk_idx, P, d->E, gemm_tile_rows(), reinterpret_cast<int32_t*>(ws + L.chunk_counts),
                               reinterpret_cast<int32_t*>(ws + L.chunk_base), reinterpret_cast<int32_t*>(ws + L.counts),
                               offsets, reinterpret_cast<int32_t*>(ws + L.tile_prefix),
-                              reinterpret_cast<int4*>(ws + L.sched), perm, st));
+                              reinterpret_cast<int4*>(ws + L.sched), perm, reinterpret_cast<int32_t*>(ws + L.inv_perm),
+                              st));
     E4B_CUDA_TRY(launch_gather_rows(static_cast<const __nv_bfloat16*>(x), perm, offsets + d->E, d->top_k, P, d->H,
                                     reinterpret_cast<__nv_bfloat16*>(ws + L.a_perm), st));
     __nv_bfloat16* h = reinterpret_cast<__nv_bfloat16*>(ws + L.h);
@@ -341,7 +343,8 @@ e4b_status e4b_moe_forward(const e4b_moe_desc* d, const e4b_experts* w, const vo
     p.ld_out = d->H;
     E4B_CUDA_TRY(launch_grouped_gemm(EPI_DOWN, d->codebook, h, P, w->down, p.b_rows_total, d->I / 2, p,
                                      max_m_tiles(P, d->E), st));
-    E4B_CUDA_TRY(launch_combine(slots, topk_idx, d->E, d->top_k, T, d->H, static_cast<__nv_bfloat16*>(y), st));
+    E4B_CUDA_TRY(launch_combine(slots, reinterpret_cast<const int32_t*>(ws + L.inv_perm), d->top_k, T, d->H,
+                                static_cast<__nv_bfloat16*>(y), st));
     if (offsets_out) E4B_CUDA_TRY(cudaMemcpyAsync(offsets_out, offsets, (d->E + 1) * 4, cudaMemcpyDeviceToDevice, st));
     if (perm_out) E4B_CUDA_TRY(cudaMemcpyAsync(perm_out, perm, P * 4, cudaMemcpyDeviceToDevice, st));
     return E4B_OK;
@@ -366,7 +369,8 @@ e4b_status e4b_moe_backward_dgrad(const e4b_moe_desc* d, const e4b_experts* w, c
     E4B_CUDA_TRY(launch_group(topk_idx, P, d->E, gemm_tile_rows(), reinterpret_cast<int32_t*>(ws + L.chunk_counts),
                               reinterpret_cast<int32_t*>(ws + L.chunk_base), reinterpret_cast<int32_t*>(ws + L.counts),
                               reinterpret_cast<int32_t*>(ws + L.offsets), reinterpret_cast<int32_t*>(ws + L.tile_prefix),
-                              reinterpret_cast<int4*>(ws + L.sched), perm, st));
+                              reinterpret_cast<int4*>(ws + L.sched), perm, reinterpret_cast<int32_t*>(ws + L.inv_perm),
+                              st));
     __nv_bfloat16* a_perm = reinterpret_cast<__nv_bfloat16*>(ws + L.a_perm);
     const int32_t* nrows = reinterpret_cast<const int32_t*>(ws + L.offsets) + d->E;
     const __nv_bfloat16* gu = static_cast<const __nv_bfloat16*>(saved_gu);
@@ -402,11 +406,12 @@ e4b_status e4b_moe_backward_dgrad(const e4b_moe_desc* d, const e4b_experts* w, c
     q.b_rows_per_expert = 2 * d->I;
     q.b_rows_total = (int64_t)d->E * 2 * d->I;
     q.b_blocks_per_row = d->H / 64;
-    q.out_bf16 = a_perm;   // slot rows; the gathered grad_out is dead after the first GEMM
+    q.out_bf16 = a_perm;   // per-pair rows in grouped order; the gathered grad_out is dead by now
     q.ld_out = d->H;
     E4B_CUDA_TRY(launch_grouped_gemm(EPI_DGRAD_GATEUP, d->codebook, dgu, P, w->gate_up, q.b_rows_total, d->H / 2, q,
                                      max_m_tiles(P, d->E), st));
-    E4B_CUDA_TRY(launch_combine(a_perm, topk_idx, d->E, d->top_k, T, d->H, static_cast<__nv_bfloat16*>(grad_x), st));
+    E4B_CUDA_TRY(launch_combine(a_perm, reinterpret_cast<const int32_t*>(ws + L.inv_perm), d->top_k, T, d->H,
+                                static_cast<__nv_bfloat16*>(grad_x), st));
     return E4B_OK;
 }
 
@@ -427,12 +432,13 @@ e4b_status e4b_moe_backward_router(const e4b_moe_desc* d, const e4b_experts* w, 
     uint8_t* ws = static_cast<uint8_t*>(workspace);
     const int64_t P = T * d->top_k;
     // h recomputed through the grouped gate_up GEMM, then the unweighted expert
-    // outputs Y (the down GEMM with unit weights) into the slot rows
+    // outputs Y (the down GEMM with unit weights), one grouped row per pair
     int32_t* perm = reinterpret_cast<int32_t*>(ws + L.perm);
     E4B_CUDA_TRY(launch_group(topk_idx, P, d->E, gemm_tile_rows(), reinterpret_cast<int32_t*>(ws + L.chunk_counts),
                               reinterpret_cast<int32_t*>(ws + L.chunk_base), reinterpret_cast<int32_t*>(ws + L.counts),
                               reinterpret_cast<int32_t*>(ws + L.offsets), reinterpret_cast<int32_t*>(ws + L.tile_prefix),
-                              reinterpret_cast<int4*>(ws + L.sched), perm, st));
+                              reinterpret_cast<int4*>(ws + L.sched), perm, reinterpret_cast<int32_t*>(ws + L.inv_perm),
+                              st));
     const int32_t* nrows = reinterpret_cast<const int32_t*>(ws + L.offsets) + d->E;
     __nv_bfloat16* a_perm = reinterpret_cast<__nv_bfloat16*>(ws + L.a_perm);
     E4B_CUDA_TRY(launch_gather_rows(static_cast<const __nv_bfloat16*>(x), perm, nrows, d->top_k, P, d->H, a_perm, st));
@@ -448,11 +454,12 @@ e4b_status e4b_moe_backward_router(const e4b_moe_desc* d, const e4b_experts* w, 
     p.b_rows_per_expert = d->H;
     p.b_rows_total = (int64_t)d->E * d->H;
     p.b_blocks_per_row = d->I / 64;
-    p.out_bf16 = a_perm;   // Y, one row per pair
+    p.out_bf16 = a_perm;   // Y, one grouped row per pair
     p.ld_out = d->H;
     E4B_CUDA_TRY(launch_grouped_gemm(EPI_DOWN, d->codebook, h, P, w->down, p.b_rows_total, d->I / 2, p,
                                      max_m_tiles(P, d->E), st));
-    E4B_CUDA_TRY(launch_router_grad(static_cast<const __nv_bfloat16*>(grad_out), a_perm, topk_idx, topk_w,
+    E4B_CUDA_TRY(launch_router_grad(static_cast<const __nv_bfloat16*>(grad_out), a_perm,
+                                    reinterpret_cast<const int32_t*>(ws + L.inv_perm), topk_idx, topk_w,
                                     router_logits, T, d->E, d->top_k, d->H, d->renormalize, grad_topk_w, grad_logits,
                                     st));
     return E4B_OK;

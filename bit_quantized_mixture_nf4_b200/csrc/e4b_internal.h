@@ -56,14 +56,16 @@ cudaError_t launch_route(const float* logits, int64_t T, int E, int k, int renor
                          cudaStream_t st);
 // counts/offsets/tile_prefix/perm from topk_idx; chunk scratch: [nchunks * E] ints x2
 // sched: [ceil(P/tile_rows) + E] m-tile entries (expert, first row, rows, 0)
+// inv_perm[pair] = grouped row of the pair, -1 for a pair of an out-of-range expert
 cudaError_t launch_group(const int32_t* idx, int64_t P, int E, int tile_rows, int32_t* chunk_counts,
                          int32_t* chunk_base, int32_t* counts, int32_t* offsets, int32_t* tile_prefix,
-                         int4* sched, int32_t* perm, cudaStream_t st);
+                         int4* sched, int32_t* perm, int32_t* inv_perm, cudaStream_t st);
 // nrows: device pointer to the number of grouped rows (offsets[E])
 cudaError_t launch_gather_rows(const __nv_bfloat16* src, const int32_t* perm, const int32_t* nrows, int k,
                                int64_t P, int H, __nv_bfloat16* dst, cudaStream_t st);
-// y[t] = sum over the k slot rows of token t (fp32 sum in slot order, bf16 result)
-cudaError_t launch_combine(const __nv_bfloat16* slots, const int32_t* idx, int E, int k, int64_t T, int H,
+// y[t] = sum over the grouped rows inv_perm[t*k + j] of token t (fp32 sum in slot
+// order j, bf16 result; rows of out-of-range experts skipped)
+cudaError_t launch_combine(const __nv_bfloat16* rows, const int32_t* inv_perm, int k, int64_t T, int H,
                            __nv_bfloat16* y, cudaStream_t st);
 
 // grouped_gemm.cu

@@ -8,10 +8,12 @@
 // order, so expert e owns the contiguous rows [offsets[e], offsets[e+1]).
 //
 //   EPI_GATEUP        D = X_e W_gu,e^T ; epilogue h = silu(g)*u (+ saves dh/dg, dh/du)
-//   EPI_DOWN          D = h_e W_d,e^T  ; epilogue slot[pair] = bf16(w * D)
+//   EPI_DOWN          D = h_e W_d,e^T  ; epilogue out[row] = bf16(w * D)
 //   EPI_DGRAD_DOWN    D = dY_e W_d,e   ; epilogue dh = w*D, dG = dh*dh/dg, dU = dh*dh/du
-//   EPI_DGRAD_GATEUP  D = dGU_e W_gu,e ; epilogue slot[pair] = bf16(D)
-// The slot rows of a token are summed in fp32, in slot order, by combine_kernel.
+//   EPI_DGRAD_GATEUP  D = dGU_e W_gu,e ; epilogue out[row] = bf16(D)
+// Every output row is the grouped row itself (a contiguous slab per tile); the
+// k rows of a token are found through the inverse permutation and summed in
+// fp32, in slot order, by combine_kernel.
 //
 // Tile: (128*CTAS) rows x 256 columns, 64-deep k-stages.  With CTAS = 2 a
 // cluster of two CTAs on two SMs computes one 256-row tile with
@@ -19,7 +21,7 @@
 // the dequantized B tile, so each SM dequantizes only 128 x 64 weights per
 // 512-clock stage and the B operand is read from shared memory once for both.
 // Roles per CTA (512 threads):
-//   warp 4      TMA producer of the A tile (bf16, 128B swizzle), 7-stage ring
+//   warp 4      TMA producer of the A tile (bf16, 128B swizzle), 6-stage ring
 //   warp 6      producer of the packed 4-bit B tile (TMA) and its absmax values
 //               (cp.async), 8-stage ring, prefetched far ahead
 //   warps 8, 10, 11, 12, 14, 15   dequantization, 3 groups of 2 warps taking every
@@ -31,7 +33,11 @@
 //               transposition costs nothing); 4-stage ring of dequantized tiles
 //   warp 5      one thread of the first CTA issues the MMAs into TMEM
 //               (double-buffered accumulator, 2 x 256 columns)
-//   warps 0-3   epilogue: tcgen05.ld of this CTA's 128 accumulator rows
+//   warps 0-3   epilogue: tcgen05.ld of this CTA's 128 accumulator rows; a warp's
+//               32 x 32 output chunks go through shared memory (64B-swizzled)
+//               and leave with TMA tensor stores, so the epilogue issues no
+//               per-thread global stores that would compete with the
+//               dequantizing warps for the load/store pipeline
 //   warps 7, 9, 13 idle
 // Every mbarrier wait is bounded; on expiry the kernel records a timeout and exits.
 #include "e4b_internal.h"
@@ -50,7 +56,7 @@ struct Cfg {
     static constexpr int A_BYTES = 128 * BK * 2;         // this CTA's 128 A rows
     static constexpr int B_BYTES = N_CTA * BK * 2;
     static constexpr int RAW_BYTES = N_CTA * BK / 2;
-    static constexpr int ASTAGES = (CTAS == 2) ? 7 : 4;    // A (activation) ring: TMA latency under load
+    static constexpr int ASTAGES = (CTAS == 2) ? 6 : 4;    // A (activation) ring: TMA latency under load
     static constexpr int STAGES = (CTAS == 2) ? 4 : 2;     // dequantized-B ring
     static constexpr int RSTAGES = (CTAS == 2) ? 8 : 6;    // packed-weight ring, prefetched far ahead
     static constexpr int AM_BYTES = N_CTA * 4;             // the stage's absmax values, one per block
@@ -59,8 +65,27 @@ struct Cfg {
     // taking every third k-stage; a thread owns N_CTA / 64 blocks of 64 elements
     static constexpr int DEQ_GROUPS = 3, DEQ_GROUP_WARPS = 2;
     static constexpr int BLK_PER_THREAD = N_CTA / (32 * DEQ_GROUP_WARPS);
-    static constexpr int SMEM_BYTES = ASTAGES * A_BYTES + STAGES * B_BYTES + RSTAGES * RAW_STAGE + 1024 + 1024;
+    // epilogue staging: per epilogue warp three 32 x 32 bf16 buffers (2 KB each)
+    static constexpr int STAGE_BUF = 2048, STAGE_BUFS = 3, STAGE_WARP = STAGE_BUF * STAGE_BUFS;
+    static constexpr int RINGS_BYTES = ASTAGES * A_BYTES + STAGES * B_BYTES + RSTAGES * RAW_STAGE;
+    static constexpr int SMEM_BYTES = RINGS_BYTES + 1024 + 4 * STAGE_WARP + 1024;
 };
+static_assert(Cfg<2>::RINGS_BYTES % 1024 == 0, "staging buffers stay 1024-byte aligned");
+static_assert(Cfg<2>::SMEM_BYTES <= 232448, "shared memory per block");
+
+// TMA tensor store of a 32 x 32 bf16 box from shared memory, and its bulk-group
+// bookkeeping (issued and awaited by one thread).
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap* m, uint32_t src, int x, int y) {
+    asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];"
+                 ::"l"(reinterpret_cast<uint64_t>(m)), "r"(src), "r"(x), "r"(y)
+                 : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void bulk_wait_read() {
+    asm volatile("cp.async.bulk.wait_group.read %0;" ::"n"(N) : "memory");
+}
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 
 struct SmemCtl {
     uint64_t a_full[8];
@@ -118,6 +143,7 @@ __device__ __forceinline__ int64_t absmax_index(const GemmParams& p, const TileI
 template <int EPI, int CB, int CTAS>
 __global__ void __launch_bounds__(GEMM_THREADS, 1)
 grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_raw,
+                    const __grid_constant__ CUtensorMap tmap_out, const __grid_constant__ CUtensorMap tmap_gu,
                     const GemmParams p) {
     using C = Cfg<CTAS>;
     constexpr int STAGES = C::STAGES;
@@ -129,6 +155,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_con
     uint8_t* sB = sA + ASTAGES * C::A_BYTES;
     uint8_t* sRaw = sB + STAGES * C::B_BYTES;
     SmemCtl* ctl = reinterpret_cast<SmemCtl*>(sRaw + C::RSTAGES * C::RAW_STAGE);
+    uint8_t* sStage = reinterpret_cast<uint8_t*>(ctl) + 1024;
     constexpr int RSTAGES = C::RSTAGES;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -389,21 +416,48 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_con
         }
     } else if (warp < 4) {
         // ------------------------------------------------------------ epilogue
+        // Lane l holds accumulator row (32*warp + l) of this CTA's half.  A warp whose 32
+        // rows all lie inside the tile writes each 32 x 32 output chunk into one of its
+        // three staging buffers (row l at 64*l, 16-byte chunks 64B-swizzled: chunk c at
+        // c ^ ((l >> 1) & 3), which is also conflict-free for the 16-byte stores) and
+        // lane 0 sends it out with a TMA tensor store; the tail warp of a partial tile
+        // stores its valid rows directly.
         const int rloc = warp * 32 + lane;   // TMEM lane == row of this CTA's half
+        uint8_t* stg = sStage + warp * C::STAGE_WARP;
+        uint32_t nbuf = 0;                   // staging buffers used so far (rotating)
+        auto stage_store = [&](const uint32_t (&v)[16], const CUtensorMap* m, int x, int y) {
+            uint8_t* buf = stg + (nbuf % C::STAGE_BUFS) * C::STAGE_BUF;
+            if (nbuf >= (uint32_t)C::STAGE_BUFS) {   // the store that last read this buffer is done reading
+                if (lane == 0) bulk_wait_read<C::STAGE_BUFS - 1>();
+                __syncwarp();
+            }
+            const int sw = (lane >> 1) & 3;
+#pragma unroll
+            for (int c = 0; c < 4; ++c)
+                *reinterpret_cast<uint4*>(buf + lane * 64 + ((c ^ sw) << 4)) =
+                    make_uint4(v[4 * c], v[4 * c + 1], v[4 * c + 2], v[4 * c + 3]);
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+                tma_store_2d(m, smem_u32(buf), x, y);
+                bulk_commit();
+            }
+            ++nbuf;
+        };
         uint32_t lt = 0;
         for (int tile = cluster_id; tile < total_tiles; tile += nclusters, ++lt) {
             const TileInfo ti = decode_tile(p, tile);
             const uint32_t ab = lt & 1, ar = lt >> 1;
             const int rtile = 128 * (int)rank + rloc;
+            const int wrow0 = 128 * (int)rank + 32 * warp;   // this warp's first row in the tile
+            const bool bulk = ti.rows - wrow0 >= 32;          // all 32 rows inside the tile
+            const bool any = ti.rows > wrow0;
             const bool valid = rtile < ti.rows;
             const int row = ti.row0 + rtile;
+            const int srow = ti.row0 + wrow0;                 // first row of the warp's TMA boxes
             // everything that does not depend on the accumulator is fetched before waiting for it
-            int pair = 0;
             float wgt = 1.0f;
-            if (EPI != EPI_GATEUP && valid) {
-                pair = __ldg(p.perm + row);
-                if (EPI != EPI_DGRAD_GATEUP) wgt = __ldg(p.topk_w + pair);
-            }
+            if ((EPI == EPI_DOWN || EPI == EPI_DGRAD_DOWN) && valid) wgt = __ldg(p.topk_w + __ldg(p.perm + row));
             uint4 gq[4], uq[4];   // EPI_DGRAD_DOWN: saved dh/dg, dh/du of the current 32-column chunk
             auto load_gu = [&](int q, uint4 (&g4)[4], uint4 (&u4)[4]) {
                 const int c0 = ti.nt * BN + 32 * q;
@@ -429,36 +483,56 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_con
                     tmem_load32(tbase + 32 * q, g);
                     tmem_load32(tbase + 128 + 32 * q, u);
                     const int f0 = ti.nt * 128 + 32 * q;
-                    if (valid && f0 < I) {
+                    if (any && f0 < I) {
                         // h = silu(g) * u, and the two SwiGLU derivatives the input gradient
                         // needs: dh/dg = u s (1 + g (1 - s)), dh/du = silu(g), s = sigmoid(g)
-                        uint32_t hv[16], dgv[16], duv[16];
+                        // in place: u <- dh/dg, g <- dh/du, so few registers stay live
+                        uint32_t hv[16];
 #pragma unroll
                         for (int i = 0; i < 16; ++i) {
-                            float hh[2], dg[2], du[2];
+                            float hh[2];
 #pragma unroll
                             for (int h = 0; h < 2; ++h) {
-                                const float gg = g[2 * i + h], uu = u[2 * i + h];
+                                const int j = 2 * i + h;
+                                const float gg = g[j], uu = u[j];
                                 const float sg = __fdividef(1.0f, 1.0f + __expf(-gg));
                                 const float sl = gg * sg;
                                 hh[h] = sl * uu;
-                                dg[h] = uu * sg * (1.0f + gg * (1.0f - sg));
-                                du[h] = sl;
+                                u[j] = uu * sg * (1.0f + gg * (1.0f - sg));
+                                g[j] = sl;
                             }
                             hv[i] = pack_bf16x2(hh[0], hh[1]);
-                            dgv[i] = pack_bf16x2(dg[0], dg[1]);
-                            duv[i] = pack_bf16x2(du[0], du[1]);
                         }
-                        uint4* dst = reinterpret_cast<uint4*>(p.out_bf16 + (int64_t)row * p.ld_out + f0);
+                        auto pack32 = [&](const float (&f)[32], uint32_t (&o)[16]) {
 #pragma unroll
-                        for (int i = 0; i < 4; ++i) dst[i] = make_uint4(hv[4 * i], hv[4 * i + 1], hv[4 * i + 2], hv[4 * i + 3]);
-                        if (p.gu) {
-                            uint4* dg = reinterpret_cast<uint4*>(p.gu + (int64_t)row * 2 * I + f0);
-                            uint4* du = reinterpret_cast<uint4*>(p.gu + (int64_t)row * 2 * I + I + f0);
+                            for (int i = 0; i < 16; ++i) o[i] = pack_bf16x2(f[2 * i], f[2 * i + 1]);
+                        };
+                        if (bulk) {
+                            stage_store(hv, &tmap_out, f0, srow);
+                            if (p.gu) {
+                                uint32_t pk[16];
+                                pack32(u, pk);
+                                stage_store(pk, &tmap_gu, f0, srow);
+                                pack32(g, pk);
+                                stage_store(pk, &tmap_gu, I + f0, srow);
+                            }
+                        } else if (valid) {
+                            uint4* dst = reinterpret_cast<uint4*>(p.out_bf16 + (int64_t)row * p.ld_out + f0);
 #pragma unroll
-                            for (int i = 0; i < 4; ++i) {
-                                dg[i] = make_uint4(dgv[4 * i], dgv[4 * i + 1], dgv[4 * i + 2], dgv[4 * i + 3]);
-                                du[i] = make_uint4(duv[4 * i], duv[4 * i + 1], duv[4 * i + 2], duv[4 * i + 3]);
+                            for (int i = 0; i < 4; ++i)
+                                dst[i] = make_uint4(hv[4 * i], hv[4 * i + 1], hv[4 * i + 2], hv[4 * i + 3]);
+                            if (p.gu) {
+                                uint32_t pk[16];
+                                pack32(u, pk);
+                                uint4* dg = reinterpret_cast<uint4*>(p.gu + (int64_t)row * 2 * I + f0);
+#pragma unroll
+                                for (int i = 0; i < 4; ++i)
+                                    dg[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
+                                pack32(g, pk);
+                                uint4* du = reinterpret_cast<uint4*>(p.gu + (int64_t)row * 2 * I + I + f0);
+#pragma unroll
+                                for (int i = 0; i < 4; ++i)
+                                    du[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
                             }
                         }
                     }
@@ -471,41 +545,56 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_con
                     uint4 gn[4], un[4];
                     if (EPI == EPI_DGRAD_DOWN && q + 1 < BN / 32) load_gu(q + 1, gn, un);   // next chunk in flight
                     const int c0 = ti.nt * BN + 32 * q;
-                    if (!valid || c0 >= p.N) continue;
-                    if (EPI == EPI_DOWN || EPI == EPI_DGRAD_GATEUP) {
-                        // this pair's contribution, rounded to bf16, into its own slot row
-                        // (summed over the k slots of each token by the combine kernel)
-                        uint4* dst = reinterpret_cast<uint4*>(p.out_bf16 + (int64_t)pair * p.ld_out + c0);
+                    if (any && c0 < p.N) {
+                        if (EPI == EPI_DOWN || EPI == EPI_DGRAD_GATEUP) {
+                            // this pair's contribution, rounded to bf16, into its grouped row
+                            // (summed over the k rows of each token by the combine kernel)
+                            uint32_t ov[16];
 #pragma unroll
-                        for (int i = 0; i < 4; ++i)
-                            dst[i] = make_uint4(pack_bf16x2(v[8 * i] * wgt, v[8 * i + 1] * wgt),
-                                                pack_bf16x2(v[8 * i + 2] * wgt, v[8 * i + 3] * wgt),
-                                                pack_bf16x2(v[8 * i + 4] * wgt, v[8 * i + 5] * wgt),
-                                                pack_bf16x2(v[8 * i + 6] * wgt, v[8 * i + 7] * wgt));
-                    } else {   // EPI_DGRAD_DOWN: SwiGLU backward with the saved derivatives
-                        const int I = p.N;
-                        uint4* dgo = reinterpret_cast<uint4*>(p.out_bf16 + (int64_t)row * 2 * I + c0);
-                        uint4* duo = reinterpret_cast<uint4*>(p.out_bf16 + (int64_t)row * 2 * I + I + c0);
+                            for (int i = 0; i < 16; ++i) ov[i] = pack_bf16x2(v[2 * i] * wgt, v[2 * i + 1] * wgt);
+                            if (bulk) {
+                                stage_store(ov, &tmap_out, c0, srow);
+                            } else if (valid) {
+                                uint4* dst = reinterpret_cast<uint4*>(p.out_bf16 + (int64_t)row * p.ld_out + c0);
 #pragma unroll
-                        for (int i = 0; i < 4; ++i) {
-                            const uint32_t gw[4] = {gq[i].x, gq[i].y, gq[i].z, gq[i].w};
-                            const uint32_t uw[4] = {uq[i].x, uq[i].y, uq[i].z, uq[i].w};
-                            uint32_t dgw[4], duw[4];
-#pragma unroll
-                            for (int j = 0; j < 4; ++j) {
-                                const float dh0 = v[8 * i + 2 * j] * wgt, dh1 = v[8 * i + 2 * j + 1] * wgt;
-                                dgw[j] = pack_bf16x2(dh0 * __uint_as_float(gw[j] << 16), dh1 * __uint_as_float(gw[j] & 0xFFFF0000u));
-                                duw[j] = pack_bf16x2(dh0 * __uint_as_float(uw[j] << 16), dh1 * __uint_as_float(uw[j] & 0xFFFF0000u));
+                                for (int i = 0; i < 4; ++i)
+                                    dst[i] = make_uint4(ov[4 * i], ov[4 * i + 1], ov[4 * i + 2], ov[4 * i + 3]);
                             }
-                            dgo[i] = make_uint4(dgw[0], dgw[1], dgw[2], dgw[3]);
-                            duo[i] = make_uint4(duw[0], duw[1], duw[2], duw[3]);
-                        }
-                        if (q + 1 < BN / 32) {
+                        } else {   // EPI_DGRAD_DOWN: SwiGLU backward with the saved derivatives
+                            const int I = p.N;
+                            uint32_t dgw[16], duw[16];
 #pragma unroll
                             for (int i = 0; i < 4; ++i) {
-                                gq[i] = gn[i];
-                                uq[i] = un[i];
+                                const uint32_t gw[4] = {gq[i].x, gq[i].y, gq[i].z, gq[i].w};
+                                const uint32_t uw[4] = {uq[i].x, uq[i].y, uq[i].z, uq[i].w};
+#pragma unroll
+                                for (int j = 0; j < 4; ++j) {
+                                    const float dh0 = v[8 * i + 2 * j] * wgt, dh1 = v[8 * i + 2 * j + 1] * wgt;
+                                    dgw[4 * i + j] = pack_bf16x2(dh0 * __uint_as_float(gw[j] << 16),
+                                                                 dh1 * __uint_as_float(gw[j] & 0xFFFF0000u));
+                                    duw[4 * i + j] = pack_bf16x2(dh0 * __uint_as_float(uw[j] << 16),
+                                                                 dh1 * __uint_as_float(uw[j] & 0xFFFF0000u));
+                                }
                             }
+                            if (bulk) {
+                                stage_store(dgw, &tmap_out, c0, srow);
+                                stage_store(duw, &tmap_out, I + c0, srow);
+                            } else if (valid) {
+                                uint4* dgo = reinterpret_cast<uint4*>(p.out_bf16 + (int64_t)row * 2 * I + c0);
+                                uint4* duo = reinterpret_cast<uint4*>(p.out_bf16 + (int64_t)row * 2 * I + I + c0);
+#pragma unroll
+                                for (int i = 0; i < 4; ++i) {
+                                    dgo[i] = make_uint4(dgw[4 * i], dgw[4 * i + 1], dgw[4 * i + 2], dgw[4 * i + 3]);
+                                    duo[i] = make_uint4(duw[4 * i], duw[4 * i + 1], duw[4 * i + 2], duw[4 * i + 3]);
+                                }
+                            }
+                        }
+                    }
+                    if (EPI == EPI_DGRAD_DOWN && q + 1 < BN / 32) {
+#pragma unroll
+                        for (int i = 0; i < 4; ++i) {
+                            gq[i] = gn[i];
+                            uq[i] = un[i];
                         }
                     }
                 }
@@ -514,6 +603,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_con
             __syncwarp();
             if (lane == 0) arrive_leader(&ctl->acc_empty[ab]);
         }
+        if (lane == 0) bulk_wait_all();   // this warp's tensor stores have left shared memory
     }
 
     tc_fence_before();
@@ -557,8 +647,8 @@ constexpr int kCtas = 2;
 int gemm_tile_rows() { return Cfg<kCtas>::TILE_M; }
 
 template <int EPI, int CB>
-static cudaError_t launch_one(const CUtensorMap& ma, const CUtensorMap& mr, const GemmParams& p, int grid,
-                              cudaStream_t st) {
+static cudaError_t launch_one(const CUtensorMap& ma, const CUtensorMap& mr, const CUtensorMap& mo,
+                              const CUtensorMap& mg, const GemmParams& p, int grid, cudaStream_t st) {
     using C = Cfg<kCtas>;
     auto kern = grouped_gemm_kernel<EPI, CB, kCtas>;
     static bool attr_set = false;   // per instantiation
@@ -580,7 +670,7 @@ static cudaError_t launch_one(const CUtensorMap& ma, const CUtensorMap& mr, cons
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     timing_begin(KK_GEMM_GATEUP + EPI, st);
-    cudaError_t e = cudaLaunchKernelEx(&cfg, kern, ma, mr, p);
+    cudaError_t e = cudaLaunchKernelEx(&cfg, kern, ma, mr, mo, mg, p);
     timing_end(KK_GEMM_GATEUP + EPI, st);
     count_launch();
     if (e != cudaSuccess) return e;
@@ -605,10 +695,21 @@ cudaError_t launch_grouped_gemm(int epi, int codebook, const void* a, int64_t a_
                      kmaj ? CU_TENSOR_MAP_SWIZZLE_NONE
                           : (mn_row == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B)))
         return cudaErrorInvalidValue;
+    // epilogue outputs: 32 x 32 boxes, 64B-swizzled, of the [rows, ld_out] output (h, the
+    // input-gradient halves or the per-pair rows) and of the saved derivatives [rows, 2I]
+    CUtensorMap mo, mg;
+    if (!make_map_2d(&mo, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, p.out_bf16, (uint64_t)p.ld_out, (uint64_t)a_rows,
+                     (uint64_t)p.ld_out * 2, 32, 32, CU_TENSOR_MAP_SWIZZLE_64B))
+        return cudaErrorInvalidValue;
+    mg = mo;
+    if (epi == EPI_GATEUP && p.gu &&
+        !make_map_2d(&mg, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, p.gu, (uint64_t)p.up_offset * 2, (uint64_t)a_rows,
+                     (uint64_t)p.up_offset * 4, 32, 32, CU_TENSOR_MAP_SWIZZLE_64B))
+        return cudaErrorInvalidValue;
     const int64_t tiles = (int64_t)max_m_tiles * p.n_tiles;
     const int grid = (int)std::min<int64_t>(tiles * kCtas, (num_sms() / kCtas) * kCtas);
     if (grid <= 0) return cudaSuccess;
-#define E4B_LAUNCH(E_, C_) return launch_one<E_, C_>(ma, mr, p, grid, st)
+#define E4B_LAUNCH(E_, C_) return launch_one<E_, C_>(ma, mr, mo, mg, p, grid, st)
     if (codebook == 0) {
         switch (epi) {
             case EPI_GATEUP: E4B_LAUNCH(EPI_GATEUP, 0);

@@ -136,10 +136,11 @@ __global__ void __launch_bounds__(1024) scan_kernel(const int32_t* __restrict__ 
     }
 }
 
-// Stable scatter: pairs of a chunk keep their order inside each expert.
+// Stable scatter: pairs of a chunk keep their order inside each expert.  Also the
+// inverse map pair -> grouped row (-1 for pairs of out-of-range experts).
 __global__ void __launch_bounds__(256) scatter_kernel(const int32_t* __restrict__ idx, int64_t P, int E,
                                                       const int32_t* __restrict__ chunk_base,
-                                                      int32_t* __restrict__ perm) {
+                                                      int32_t* __restrict__ perm, int32_t* __restrict__ inv_perm) {
     constexpr int WARPS = 8, PER_WARP = kChunkPairs / WARPS;
     __shared__ int wbase[WARPS][256];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -176,7 +177,10 @@ __global__ void __launch_bounds__(256) scatter_kernel(const int32_t* __restrict_
         __syncwarp();
         if (e >= 0) {
             perm[base + rank] = (int32_t)pp;
+            inv_perm[pp] = base + rank;
             if (rank == 0) wbase[warp][e] = base + __popc(peers);
+        } else if (pp < P) {
+            inv_perm[pp] = -1;
         }
         __syncwarp();
     }
@@ -211,12 +215,13 @@ __global__ void __launch_bounds__(256) gather_rows_kernel(const __nv_bfloat16* _
     }
 }
 
-// y[t] = bf16( sum_j fp32(slot[t*k + j]) ), j ascending: the weighted combine of
-// the k expert outputs of each token in fp32 (experts4bit-qlora 0.1.0 experts.py,
-// Experts4bit.forward: per-expert outputs in the compute dtype, index_add_ into an
-// fp32 buffer).  Slots of out-of-range experts are skipped.
-__global__ void __launch_bounds__(256) combine_kernel(const __nv_bfloat16* __restrict__ slots,
-                                                      const int32_t* __restrict__ idx, int E, int k, int64_t T,
+// y[t] = bf16( sum_j fp32(rows[inv_perm[t*k + j]]) ), j ascending: the weighted
+// combine of the k expert outputs of each token in fp32 (experts4bit-qlora 0.1.0
+// experts.py, Experts4bit.forward: per-expert outputs in the compute dtype,
+// index_add_ into an fp32 buffer).  Pairs of out-of-range experts (inv_perm -1)
+// are skipped.
+__global__ void __launch_bounds__(256) combine_kernel(const __nv_bfloat16* __restrict__ rows,
+                                                      const int32_t* __restrict__ inv_perm, int k, int64_t T,
                                                       int H, __nv_bfloat16* __restrict__ y) {
     const int h8 = H / 8;
     const int64_t n = T * h8;
@@ -230,8 +235,8 @@ __global__ void __launch_bounds__(256) combine_kernel(const __nv_bfloat16* __res
         for (int j = 0; j < kMaxTopK; ++j) {   // every slot's vector in flight before the sums
             v[j] = make_uint4(0u, 0u, 0u, 0u);
             if (j < k) {
-                const int e = __ldg(idx + t * k + j);
-                if (e >= 0 && e < E) v[j] = __ldcs(reinterpret_cast<const uint4*>(slots + (t * k + j) * H) + c);
+                const int r = __ldg(inv_perm + t * k + j);
+                if (r >= 0) v[j] = __ldcs(reinterpret_cast<const uint4*>(rows + (int64_t)r * H) + c);
             }
         }
 #pragma unroll
@@ -284,7 +289,7 @@ cudaError_t launch_route(const float* logits, int64_t T, int E, int k, int renor
 
 cudaError_t launch_group(const int32_t* idx, int64_t P, int E, int tile_rows, int32_t* chunk_counts,
                          int32_t* chunk_base, int32_t* counts, int32_t* offsets, int32_t* tile_prefix,
-                         int4* sched, int32_t* perm, cudaStream_t st) {
+                         int4* sched, int32_t* perm, int32_t* inv_perm, cudaStream_t st) {
     const int nchunks = (int)((P + kChunkPairs - 1) / kChunkPairs);
     if (nchunks == 0) return cudaSuccess;
     timing_begin(KK_GROUP, st);
@@ -292,7 +297,8 @@ cudaError_t launch_group(const int32_t* idx, int64_t P, int E, int tile_rows, in
     if (err == cudaSuccess)
         err = launch_chained(scan_kernel, 1, 1024, st, chunk_counts, nchunks, E, tile_rows, chunk_base, counts, offsets,
                              tile_prefix, sched);
-    if (err == cudaSuccess) err = launch_chained(scatter_kernel, nchunks, 256, st, idx, P, E, chunk_base, perm);
+    if (err == cudaSuccess)
+        err = launch_chained(scatter_kernel, nchunks, 256, st, idx, P, E, chunk_base, perm, inv_perm);
     timing_end(KK_GROUP, st);
     count_launch();
     count_launch();
@@ -311,12 +317,12 @@ cudaError_t launch_gather_rows(const __nv_bfloat16* src, const int32_t* perm, co
     return err;
 }
 
-cudaError_t launch_combine(const __nv_bfloat16* slots, const int32_t* idx, int E, int k, int64_t T, int H,
+cudaError_t launch_combine(const __nv_bfloat16* rows, const int32_t* inv_perm, int k, int64_t T, int H,
                            __nv_bfloat16* y, cudaStream_t st) {
     const int64_t n = T * (H / 8);
     if (n == 0) return cudaSuccess;
     timing_begin(KK_COMBINE, st);
-    combine_kernel<<<capped_grid((n + 255) / 256), 256, 0, st>>>(slots, idx, E, k, T, H, y);
+    combine_kernel<<<capped_grid((n + 255) / 256), 256, 0, st>>>(rows, inv_perm, k, T, H, y);
     timing_end(KK_COMBINE, st);
     count_launch();
     return cudaGetLastError();

@@ -22,6 +22,7 @@ __global__ void __launch_bounds__(256) fill_f32_kernel(float* __restrict__ p, in
 // logit gradient of the token.
 __global__ void __launch_bounds__(256) router_grad_kernel(const __nv_bfloat16* __restrict__ grad_out,
                                                           const __nv_bfloat16* __restrict__ Y,
+                                                          const int32_t* __restrict__ inv_perm,
                                                           const int32_t* __restrict__ idx,
                                                           const float* __restrict__ wts,
                                                           const float* __restrict__ logits, int64_t T, int E,
@@ -43,7 +44,7 @@ __global__ void __launch_bounds__(256) router_grad_kernel(const __nv_bfloat16* _
         float acc = 0.0f;
         if (valid) {
             const uint4* g4 = reinterpret_cast<const uint4*>(grad_out + t * H);
-            const uint4* y4 = reinterpret_cast<const uint4*>(Y + p * H);
+            const uint4* y4 = reinterpret_cast<const uint4*>(Y + (int64_t)__ldg(inv_perm + p) * H);
             for (int c = lane; c < H / 8; c += 32) {
                 const uint4 gv = __ldg(g4 + c), yv = __ldcs(y4 + c);
                 const uint32_t gw[4] = {gv.x, gv.y, gv.z, gv.w}, yw[4] = {yv.x, yv.y, yv.z, yv.w};
@@ -117,13 +118,13 @@ cudaError_t launch_fill_f32(float* p, int64_t n, float v, cudaStream_t st) {
     return cudaGetLastError();
 }
 
-cudaError_t launch_router_grad(const __nv_bfloat16* grad_out, const __nv_bfloat16* Y, const int32_t* idx,
-                               const float* wts, const float* logits, int64_t T, int E, int k, int H, int renorm,
-                               float* dw, float* dlogits, cudaStream_t st) {
+cudaError_t launch_router_grad(const __nv_bfloat16* grad_out, const __nv_bfloat16* Y, const int32_t* inv_perm,
+                               const int32_t* idx, const float* wts, const float* logits, int64_t T, int E, int k,
+                               int H, int renorm, float* dw, float* dlogits, cudaStream_t st) {
     if (T == 0) return cudaSuccess;
     const int64_t grid = (T * 32 + 255) / 256;
-    router_grad_kernel<<<(unsigned)grid, 256, 0, st>>>(grad_out, Y, idx, wts, logits, T, E, k, H, renorm, dw,
-                                                       dlogits);
+    router_grad_kernel<<<(unsigned)grid, 256, 0, st>>>(grad_out, Y, inv_perm, idx, wts, logits, T, E, k, H, renorm,
+                                                       dw, dlogits);
     count_launch();
     return cudaGetLastError();
 }

@@ -5,10 +5,11 @@
 namespace e4b {
 
 cudaError_t launch_fill_f32(float* p, int64_t n, float v, cudaStream_t st);
-// dw [T*k] = <grad_out_t, Y_p> for every pair p = t*k + j (0 for an out-of-range
-// expert); dlogits [T, E] (skipped when null) through the routing softmax.
-cudaError_t launch_router_grad(const __nv_bfloat16* grad_out, const __nv_bfloat16* Y, const int32_t* idx,
-                               const float* wts, const float* logits, int64_t T, int E, int k, int H, int renorm,
-                               float* dw, float* dlogits, cudaStream_t st);
+// dw [T*k] = <grad_out_t, Y[inv_perm[p]]> for every pair p = t*k + j (Y in grouped
+// row order; 0 for an out-of-range expert); dlogits [T, E] (skipped when null)
+// through the routing softmax.
+cudaError_t launch_router_grad(const __nv_bfloat16* grad_out, const __nv_bfloat16* Y, const int32_t* inv_perm,
+                               const int32_t* idx, const float* wts, const float* logits, int64_t T, int E, int k,
+                               int H, int renorm, float* dw, float* dlogits, cudaStream_t st);
 
 }  // namespace e4b
