@@ -191,6 +191,7 @@ MEDIUM = [
     pb.custom("ragged", E=4, H=320, I=192, k=2, T=500, seed=11),                    # M, N and K tails
     pb.custom("skew", E=16, H=256, I=256, k=4, T=777, seed=12, router="zipf"),      # empty experts, skew
     pb.custom("fp4med", E=6, H=192, I=320, k=3, T=333, seed=13, codebook=wl.FP4),
+    pb.custom("even6", E=8, H=384, I=128, k=2, T=300, seed=14),                     # 6 / 2 blocks per row
     wl.TINY,
 ]
 
