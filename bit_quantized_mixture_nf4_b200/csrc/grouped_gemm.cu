@@ -49,7 +49,7 @@ constexpr int GEMM_THREADS = 512;
 constexpr int PRODUCER_WARP = 4, MMA_WARP = 5, RAW_WARP = 6, DEQ_WARP0 = 8;
 constexpr int TMEM_COLS = 2 * BN;   // two accumulator buffers
 
-template <int CTAS>
+template <int CTAS, int EPI = 0>
 struct Cfg {
     static constexpr int TILE_M = 128 * CTAS;            // rows per tile (all CTAs of the cluster)
     static constexpr int N_CTA = BN / CTAS;              // B columns dequantized by one CTA
@@ -58,20 +58,26 @@ struct Cfg {
     static constexpr int RAW_BYTES = N_CTA * BK / 2;
     static constexpr int ASTAGES = (CTAS == 2) ? 6 : 4;    // A (activation) ring: TMA latency under load
     static constexpr int STAGES = (CTAS == 2) ? 4 : 2;     // dequantized-B ring
-    static constexpr int RSTAGES = (CTAS == 2) ? 8 : 6;    // packed-weight ring, prefetched far ahead
+    // packed-weight ring, prefetched far ahead (the input gradient's down^T GEMM gives two
+    // stages to the epilogue buffers that bring in the saved SwiGLU derivatives)
+    static constexpr int RSTAGES = (CTAS == 2) ? (EPI == EPI_DGRAD_DOWN ? 6 : 8) : 6;
     static constexpr int AM_BYTES = N_CTA * 4;             // the stage's absmax values, one per block
     static constexpr int RAW_STAGE = RAW_BYTES + AM_BYTES;
     // dequantizing warps: 6 warps (none on the MMA thread's scheduler), 3 groups of 2
     // taking every third k-stage; a thread owns N_CTA / 64 blocks of 64 elements
     static constexpr int DEQ_GROUPS = 3, DEQ_GROUP_WARPS = 2;
     static constexpr int BLK_PER_THREAD = N_CTA / (32 * DEQ_GROUP_WARPS);
-    // epilogue staging: per epilogue warp three 32 x 32 bf16 buffers (2 KB each)
-    static constexpr int STAGE_BUF = 2048, STAGE_BUFS = 3, STAGE_WARP = STAGE_BUF * STAGE_BUFS;
+    // epilogue staging: per epilogue warp three 32 x 32 bf16 buffers (2 KB each); four (two
+    // pairs of saved-derivative chunks, loaded and stored in place) for the down^T GEMM
+    static constexpr int STAGE_BUF = 2048, STAGE_BUFS = (EPI == EPI_DGRAD_DOWN) ? 4 : 3;
+    static constexpr int STAGE_WARP = STAGE_BUF * STAGE_BUFS;
     static constexpr int RINGS_BYTES = ASTAGES * A_BYTES + STAGES * B_BYTES + RSTAGES * RAW_STAGE;
     static constexpr int SMEM_BYTES = RINGS_BYTES + 1024 + 4 * STAGE_WARP + 1024;
 };
-static_assert(Cfg<2>::RINGS_BYTES % 1024 == 0, "staging buffers stay 1024-byte aligned");
-static_assert(Cfg<2>::SMEM_BYTES <= 232448, "shared memory per block");
+static_assert(Cfg<2, EPI_GATEUP>::RINGS_BYTES % 1024 == 0 && Cfg<2, EPI_DGRAD_DOWN>::RINGS_BYTES % 1024 == 0,
+              "staging buffers stay 1024-byte aligned");
+static_assert(Cfg<2, EPI_GATEUP>::SMEM_BYTES <= 232448 && Cfg<2, EPI_DGRAD_DOWN>::SMEM_BYTES <= 232448,
+              "shared memory per block");
 
 // TMA tensor store of a 32 x 32 bf16 box from shared memory, and its bulk-group
 // bookkeeping (issued and awaited by one thread).
@@ -96,6 +102,7 @@ struct SmemCtl {
     uint64_t raw_empty[16];
     uint64_t acc_full[2];
     uint64_t acc_empty[2];
+    uint64_t ld_full[4][2];   // EPI_DGRAD_DOWN: saved-derivative chunk pair landed (per epilogue warp)
     uint32_t tmem_base;
     int abort_flag;
 };
@@ -145,7 +152,7 @@ __global__ void __launch_bounds__(GEMM_THREADS, 1)
 grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_raw,
                     const __grid_constant__ CUtensorMap tmap_out, const __grid_constant__ CUtensorMap tmap_gu,
                     const GemmParams p) {
-    using C = Cfg<CTAS>;
+    using C = Cfg<CTAS, EPI>;
     constexpr int STAGES = C::STAGES;
     constexpr int ASTAGES = C::ASTAGES;
     constexpr bool kMajorB = (EPI == EPI_GATEUP || EPI == EPI_DOWN);
@@ -179,6 +186,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_con
         for (int b = 0; b < 2; ++b) {
             mbar_init(smem_u32(&ctl->acc_full[b]), 1);
             mbar_init(smem_u32(&ctl->acc_empty[b]), 4 * CTAS);     // epilogue warps of all CTAs
+            for (int w = 0; w < 4; ++w) mbar_init(smem_u32(&ctl->ld_full[w][b]), 1);
         }
         ctl->abort_flag = 0;
         fence_barrier_init();
@@ -425,6 +433,23 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_con
         const int rloc = warp * 32 + lane;   // TMEM lane == row of this CTA's half
         uint8_t* stg = sStage + warp * C::STAGE_WARP;
         uint32_t nbuf = 0;                   // staging buffers used so far (rotating)
+        // EPI_DGRAD_DOWN, whole-slab warps: the saved dh/dg and dh/du chunks of a 32 x 32
+        // output chunk come in by TMA (pair n & 1 of the warp's four buffers, barrier
+        // ld_full[warp][n & 1]), are turned into dG, dU in place and leave by TMA
+        uint32_t nld = 0, ncons = 0;         // chunk pairs requested / consumed
+        auto issue_pair = [&](int c0, int srow) {
+            uint8_t* gb = stg + (nld & 1) * 2 * C::STAGE_BUF;
+            if (lane == 0) {
+                bulk_wait_read<0>();          // the stores that last read this pair are done with it
+                const uint32_t bar = smem_u32(&ctl->ld_full[warp][nld & 1]);
+                mbar_arrive_expect_tx(bar, 2 * C::STAGE_BUF);
+                tma_load_2d(smem_u32(gb), &tmap_gu, bar, c0, srow);
+                tma_load_2d(smem_u32(gb + C::STAGE_BUF), &tmap_gu, bar, p.N + c0, srow);
+            }
+            __syncwarp();
+            ++nld;
+        };
+        bool aborted = false;
         auto stage_store = [&](const uint32_t (&v)[16], const CUtensorMap* m, int x, int y) {
             uint8_t* buf = stg + (nbuf % C::STAGE_BUFS) * C::STAGE_BUF;
             if (nbuf >= (uint32_t)C::STAGE_BUFS) {   // the store that last read this buffer is done reading
@@ -471,7 +496,13 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_con
                     }
                 }
             };
-            if (EPI == EPI_DGRAD_DOWN) load_gu(0, gq, uq);
+            if (EPI == EPI_DGRAD_DOWN) {
+                if (bulk) {
+                    if (ti.nt * BN < p.N) issue_pair(ti.nt * BN, srow);
+                } else {
+                    load_gu(0, gq, uq);
+                }
+            }
             if (!wait(&ctl->acc_full[ab], ar & 1)) break;
             tc_fence_after();
             const uint32_t tbase = tmem_base + ((uint32_t)(warp * 32) << 16) + ab * BN;
@@ -537,6 +568,51 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_con
                         }
                     }
                 }
+            } else if (EPI == EPI_DGRAD_DOWN && bulk) {
+                const int I = p.N;
+#pragma unroll 1
+                for (int q = 0; q < BN / 32; ++q) {
+                    const int c0 = ti.nt * BN + 32 * q;
+                    if (c0 >= I) break;
+                    float v[32];
+                    tmem_load32(tbase + 32 * q, v);
+                    if (q + 1 < BN / 32 && c0 + 32 < I) issue_pair(c0 + 32, srow);   // next pair in flight
+                    const uint32_t n = ncons++;
+                    if (!wait(&ctl->ld_full[warp][n & 1], (n >> 1) & 1)) {
+                        aborted = true;
+                        break;
+                    }
+                    uint8_t* gb = stg + (n & 1) * 2 * C::STAGE_BUF;
+                    uint8_t* ub = gb + C::STAGE_BUF;
+                    const int sw = (lane >> 1) & 3;
+#pragma unroll
+                    for (int c = 0; c < 4; ++c) {   // row `lane`, 16-byte chunk c (64B swizzle)
+                        uint4* gp = reinterpret_cast<uint4*>(gb + lane * 64 + ((c ^ sw) << 4));
+                        uint4* up = reinterpret_cast<uint4*>(ub + lane * 64 + ((c ^ sw) << 4));
+                        const uint4 g4 = *gp, u4 = *up;
+                        const uint32_t gw[4] = {g4.x, g4.y, g4.z, g4.w};
+                        const uint32_t uw[4] = {u4.x, u4.y, u4.z, u4.w};
+                        uint32_t dgw[4], duw[4];
+#pragma unroll
+                        for (int j = 0; j < 4; ++j) {
+                            const float dh0 = v[8 * c + 2 * j] * wgt, dh1 = v[8 * c + 2 * j + 1] * wgt;
+                            dgw[j] = pack_bf16x2(dh0 * __uint_as_float(gw[j] << 16),
+                                                 dh1 * __uint_as_float(gw[j] & 0xFFFF0000u));
+                            duw[j] = pack_bf16x2(dh0 * __uint_as_float(uw[j] << 16),
+                                                 dh1 * __uint_as_float(uw[j] & 0xFFFF0000u));
+                        }
+                        *gp = make_uint4(dgw[0], dgw[1], dgw[2], dgw[3]);
+                        *up = make_uint4(duw[0], duw[1], duw[2], duw[3]);
+                    }
+                    fence_proxy_async_smem();
+                    __syncwarp();
+                    if (lane == 0) {
+                        tma_store_2d(&tmap_out, smem_u32(gb), c0, srow);
+                        tma_store_2d(&tmap_out, smem_u32(ub), I + c0, srow);
+                        bulk_commit();
+                    }
+                }
+                if (aborted) break;
             } else {
 #pragma unroll 1
                 for (int q = 0; q < BN / 32; ++q) {
@@ -603,7 +679,11 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_con
             __syncwarp();
             if (lane == 0) arrive_leader(&ctl->acc_empty[ab]);
         }
-        if (lane == 0) bulk_wait_all();   // this warp's tensor stores have left shared memory
+        if (lane == 0) {
+            bulk_wait_all();   // this warp's tensor stores have left shared memory
+            for (; ncons < nld; ++ncons)   // and its derivative loads have landed (bounded)
+                mbar_wait_drain(smem_u32(&ctl->ld_full[warp][ncons & 1]), (ncons >> 1) & 1);
+        }
     }
 
     tc_fence_before();
@@ -649,7 +729,7 @@ int gemm_tile_rows() { return Cfg<kCtas>::TILE_M; }
 template <int EPI, int CB>
 static cudaError_t launch_one(const CUtensorMap& ma, const CUtensorMap& mr, const CUtensorMap& mo,
                               const CUtensorMap& mg, const GemmParams& p, int grid, cudaStream_t st) {
-    using C = Cfg<kCtas>;
+    using C = Cfg<kCtas, EPI>;
     auto kern = grouped_gemm_kernel<EPI, CB, kCtas>;
     static bool attr_set = false;   // per instantiation
     if (!attr_set) {
@@ -702,9 +782,11 @@ cudaError_t launch_grouped_gemm(int epi, int codebook, const void* a, int64_t a_
                      (uint64_t)p.ld_out * 2, 32, 32, CU_TENSOR_MAP_SWIZZLE_64B))
         return cudaErrorInvalidValue;
     mg = mo;
-    if (epi == EPI_GATEUP && p.gu &&
-        !make_map_2d(&mg, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, p.gu, (uint64_t)p.up_offset * 2, (uint64_t)a_rows,
-                     (uint64_t)p.up_offset * 4, 32, 32, CU_TENSOR_MAP_SWIZZLE_64B))
+    // saved derivatives [rows, 2I]: written by the gate_up epilogue, read by the down^T epilogue
+    const int64_t n_feat = (epi == EPI_GATEUP) ? p.up_offset : p.N;
+    if ((epi == EPI_GATEUP || epi == EPI_DGRAD_DOWN) && p.gu &&
+        !make_map_2d(&mg, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, p.gu, (uint64_t)n_feat * 2, (uint64_t)a_rows,
+                     (uint64_t)n_feat * 4, 32, 32, CU_TENSOR_MAP_SWIZZLE_64B))
         return cudaErrorInvalidValue;
     const int64_t tiles = (int64_t)max_m_tiles * p.n_tiles;
     const int grid = (int)std::min<int64_t>(tiles * kCtas, (num_sms() / kCtas) * kCtas);
