@@ -166,7 +166,7 @@ E4B_API e4b_status e4b_moe_backward_dgrad(const e4b_moe_desc *d, const e4b_exper
  *   renormalisation:    grad_logits[t,i] = sum_{j: e_j = i} w_j (dw_j - sum_j' w_j' dw_j'),
  *                       w = topk_w (logits outside the top-k get 0).
  * Y is recomputed from x through the grouped GEMMs (gate_up, then down with unit
- * weights), rounded to bf16 like every slot row; the dot products and the
+ * weights), rounded to bf16 like every per-pair row; the dot products and the
  * softmax backward run in fp32.
  *   x bf16 [T,H], router_logits fp32 [T,E] (needed only for grad_logits),
  *   topk_idx int32 [T,k], topk_w fp32 [T,k] (the forward's), grad_out bf16 [T,H],
