@@ -22,23 +22,20 @@ __device__ __forceinline__ int sorted_code(int cb, int r) {
 template <int CB>
 __global__ void __launch_bounds__(256) quantize_kernel(const float* __restrict__ w, int64_t nblocks,
                                                        uint8_t* __restrict__ packed, float* __restrict__ absmax) {
-    __shared__ float s_mid[15];
-    __shared__ uint8_t s_code[16];
     __shared__ __align__(16) uint16_t s_out[8][128];   // per warp: 8 blocks x 32 packed bytes
     constexpr int NV = (CB == 0) ? 16 : 15;   // distinct codebook values
-    if (threadIdx.x < 16) {
-        const int r = threadIdx.x;
-        if (r < NV) s_code[r] = (uint8_t)sorted_code(CB, r);
-        if (r < 15) {
-            if (r < NV - 1) {
-                const float lo = c_code[CB][sorted_code(CB, r)], hi = c_code[CB][sorted_code(CB, r + 1)];
-                s_mid[r] = __fmul_rn(__fadd_rn(lo, hi), 0.5f);
-            } else {
-                s_mid[r] = __int_as_float(0x7f800000);   // +inf: never below a finite value
-            }
+    // the 15 midpoints between consecutive sorted codebook values, in registers (+inf past
+    // the last one); the nearest-value search below selects among them without memory loads
+    float m[15];
+#pragma unroll
+    for (int r = 0; r < 15; ++r) {
+        if (r < NV - 1) {
+            const float lo = c_code[CB][sorted_code(CB, r)], hi = c_code[CB][sorted_code(CB, r + 1)];
+            m[r] = __fmul_rn(__fadd_rn(lo, hi), 0.5f);
+        } else {
+            m[r] = __int_as_float(0x7f800000);   // +inf: never below a finite value
         }
     }
-    __syncthreads();
     const int q = threadIdx.x & 3;
     const int zero_code = (CB == 0) ? 7 : 0;
     const int64_t stride = (int64_t)gridDim.x * blockDim.x / 4;
@@ -68,12 +65,16 @@ __global__ void __launch_bounds__(256) quantize_kernel(const float* __restrict__
                 code[i] = zero_code;
             } else {
                 const float n = __fdiv_rn(v[i], a);
-                int r = 0;   // number of midpoints strictly below n
-                if (s_mid[r + 7] < n) r += 8;
-                if (s_mid[r + 3] < n) r += 4;
-                if (s_mid[r + 1] < n) r += 2;
-                if (s_mid[r] < n) r += 1;
-                code[i] = s_code[r];
+                // r = number of midpoints strictly below n: a 4-level binary search whose
+                // pivots m[7], m[r+3], m[r+1], m[r] are picked by selects on r's bits
+                const bool b3 = m[7] < n;
+                const bool b2 = (b3 ? m[11] : m[3]) < n;
+                const float p1 = b3 ? (b2 ? m[13] : m[9]) : (b2 ? m[5] : m[1]);
+                const bool b1 = p1 < n;
+                const float p0 = b3 ? (b2 ? (b1 ? m[14] : m[12]) : (b1 ? m[10] : m[8]))
+                                    : (b2 ? (b1 ? m[6] : m[4]) : (b1 ? m[2] : m[0]));
+                const int r = (b3 ? 8 : 0) + (b2 ? 4 : 0) + (b1 ? 2 : 0) + ((p0 < n) ? 1 : 0);
+                code[i] = (uint32_t)sorted_code(CB, r);
             }
         }
         // The warp's 8 blocks are 256 contiguous packed bytes: assemble them in
