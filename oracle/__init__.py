@@ -60,9 +60,11 @@ def _L():
             lib.e4bo_dequantize_bf16.argtypes = [P, P, i64, i32, i32, P]
             lib.e4bo_route.argtypes = [P, i64, i32, i32, i32, P, P]
             lib.e4bo_permute.argtypes = [P, i64, i32, i32, P, P, P]
-            lib.e4bo_forward.argtypes = [P, i64, i32, i32, i32, i32, P, P, P, P, P, i64, P]
-            lib.e4bo_dgrad.argtypes = [P, P, i64, i32, i32, i32, i32, P, P, P, P, P, i64, P]
-            lib.e4bo_router_grad.argtypes = [P, P, P, i64, i32, i32, i32, i32, i32, P, P, P, P, i64, P, P]
+            dbl = ctypes.c_double
+            lib.e4bo_forward.argtypes = [P, i64, i32, i32, i32, i32, P, P, P, P, P, i64, i32, dbl, dbl, P, P, P]
+            lib.e4bo_dgrad.argtypes = [P, P, i64, i32, i32, i32, i32, P, P, P, P, P, i64, i32, dbl, dbl, P, P]
+            lib.e4bo_router_grad.argtypes = [P, P, P, i64, i32, i32, i32, i32, i32, P, P, P, P, i64, i32, dbl, dbl,
+                                             P, P, P, P]
             lib.e4bo_codebook.argtypes = [i32, P]
             lib.e4bo_f32_to_bf16.argtypes = [ctypes.c_float]
             lib.e4bo_f32_to_bf16.restype = ctypes.c_uint16
@@ -161,11 +163,19 @@ def permute(idx: np.ndarray, E: int):
     return counts, offsets, perm
 
 
+ACT_SWIGLU, ACT_CLAMPED_GLU = 0, 1
+
+
+def _bias(b, shape):
+    return None if b is None else np.ascontiguousarray(np.broadcast_to(b, shape), np.float32)
+
+
 def forward(x: np.ndarray, idx: np.ndarray, w: np.ndarray, wgu: np.ndarray, wd: np.ndarray,
-            tokens=None) -> np.ndarray:
+            tokens=None, act=ACT_SWIGLU, alpha=1.702, limit=7.0, bgu=None, bd=None) -> np.ndarray:
     """fp64 forward.  x [T,H] (any float dtype, widened to fp64), idx [T,k], w [T,k],
-    wgu [E,2I,H] / wd [E,H,I] dequantized weights.  Returns y [nt, H] fp64 for
-    ``tokens`` (all tokens when None)."""
+    wgu [E,2I,H] / wd [E,H,I] dequantized weights; act SwiGLU or the clamped GLU
+    (alpha, limit); optional biases bgu [E,2I] (gate then up) and bd [E,H].  Returns
+    y [nt, H] fp64 for ``tokens`` (all tokens when None)."""
     x = np.ascontiguousarray(x, np.float64)
     idx = np.ascontiguousarray(idx, np.int32)
     w = np.ascontiguousarray(w, np.float64)
@@ -177,14 +187,18 @@ def forward(x: np.ndarray, idx: np.ndarray, w: np.ndarray, wgu: np.ndarray, wd: 
     tok = None if tokens is None else np.ascontiguousarray(tokens, np.int64)
     nt = T if tok is None else tok.shape[0]
     y = np.zeros((nt, H), np.float64)
+    bgu, bd = _bias(bgu, (E, I2)), _bias(bd, (E, H))
     _check("e4bo_forward", _L().e4bo_forward(_p(x), T, E, H, I2 // 2, k, _p(idx), _p(w), _p(wgu), _p(wd),
-                                             None if tok is None else _p(tok), nt, _p(y)))
+                                             None if tok is None else _p(tok), nt, int(act), float(alpha),
+                                             float(limit), None if bgu is None else _p(bgu),
+                                             None if bd is None else _p(bd), _p(y)))
     return y
 
 
 def dgrad(x: np.ndarray, grad_out: np.ndarray, idx: np.ndarray, w: np.ndarray, wgu: np.ndarray,
-          wd: np.ndarray, tokens=None) -> np.ndarray:
-    """fp64 input gradient of the forward above with routing held constant."""
+          wd: np.ndarray, tokens=None, act=ACT_SWIGLU, alpha=1.702, limit=7.0, bgu=None) -> np.ndarray:
+    """fp64 input gradient of the forward above with routing held constant (the
+    down bias does not enter it)."""
     x = np.ascontiguousarray(x, np.float64)
     g = np.ascontiguousarray(grad_out, np.float64)
     idx = np.ascontiguousarray(idx, np.int32)
@@ -197,13 +211,15 @@ def dgrad(x: np.ndarray, grad_out: np.ndarray, idx: np.ndarray, w: np.ndarray, w
     tok = None if tokens is None else np.ascontiguousarray(tokens, np.int64)
     nt = T if tok is None else tok.shape[0]
     gx = np.zeros((nt, H), np.float64)
+    bgu = _bias(bgu, (E, I2))
     _check("e4bo_dgrad", _L().e4bo_dgrad(_p(x), _p(g), T, E, H, I2 // 2, k, _p(idx), _p(w), _p(wgu), _p(wd),
-                                         None if tok is None else _p(tok), nt, _p(gx)))
+                                         None if tok is None else _p(tok), nt, int(act), float(alpha), float(limit),
+                                         None if bgu is None else _p(bgu), _p(gx)))
     return gx
 
 
 def router_grad(x: np.ndarray, grad_out: np.ndarray, logits, idx: np.ndarray, renorm: bool, wgu: np.ndarray,
-                wd: np.ndarray, tokens=None):
+                wd: np.ndarray, tokens=None, act=ACT_SWIGLU, alpha=1.702, limit=7.0, bgu=None, bd=None):
     """fp64 gradient of L = <grad_out, y> with respect to the routing weights
     (dw [nt, k]) and, when logits are given, to the router logits (dlogits
     [nt, E]; else None), with the routing indices held."""
@@ -221,7 +237,9 @@ def router_grad(x: np.ndarray, grad_out: np.ndarray, logits, idx: np.ndarray, re
     nt = T if tok is None else tok.shape[0]
     dw = np.zeros((nt, k), np.float64)
     dl = None if lg is None else np.zeros((nt, El), np.float64)
+    bgu, bd = _bias(bgu, (E, I2)), _bias(bd, (E, H))
     _check("e4bo_router_grad", _L().e4bo_router_grad(
         _p(x), _p(g), None if lg is None else _p(lg), T, El, H, I2 // 2, k, int(bool(renorm)), _p(idx), _p(wgu),
-        _p(wd), None if tok is None else _p(tok), nt, _p(dw), None if dl is None else _p(dl)))
+        _p(wd), None if tok is None else _p(tok), nt, int(act), float(alpha), float(limit),
+        None if bgu is None else _p(bgu), None if bd is None else _p(bd), _p(dw), None if dl is None else _p(dl)))
     return dw, dl

@@ -16,6 +16,14 @@
  *         modes: the support matrix".
  *   [QLoRA] Dettmers et al. 2023, "QLoRA", appendix on the NormalFloat data
  *         type (the 16 NF4 values; the pages only call get_4bit_type("nf4")).
+ *   [P2]  "experts4bit-qlora 0.31.1" PyPI project page, section "Scope": the
+ *         gpt-oss experts carry per-expert biases and a clamped GLU.  The pages
+ *         give no formula; the reading taken is the published gpt-oss expert
+ *         (gpt-oss model card, OpenAI 2025): g' = min(g, limit), u' = clamp(u,
+ *         -limit, limit), h = (u' + 1) g' sigmoid(alpha g'), with alpha and limit
+ *         parameters (1.702 and 7 in gpt-oss), biases added to g, u and to the
+ *         down projection's output, and the clamp passing the gradient where its
+ *         input lies inside the closed interval.
  *
  * Precision.  Quantize takes its decisions in fp32 (the pages quantize fp32
  * weights with fp32 absmax); dequantize multiplies in fp32 and rounds once to
@@ -241,20 +249,40 @@ int e4bo_permute(const int32_t *idx, int64_t T, int k, int E, int32_t *counts,
 
 /* ---- forward ([P4] Experts4bit.forward) ---------------------------------- */
 
-static double silu(double g) { return g / (1.0 + exp(-g)); }
+/* The expert's gated activation of the pre-activations g, u and its two partial
+ * derivatives.  act 0 (SwiGLU, [P4] forward): h = silu(g) u.  act 1 (the clamped
+ * GLU of [P2], reading above): h = (u' + 1) g' sigmoid(alpha g').  dhdg / dhdu may
+ * be NULL. */
+static double expert_act(int act, double alpha, double limit, double g, double u, double *dhdg, double *dhdu) {
+    if (act == 0) {
+        double s = 1.0 / (1.0 + exp(-g));
+        if (dhdg) *dhdg = u * s * (1.0 + g * (1.0 - s));
+        if (dhdu) *dhdu = g * s;
+        return g * s * u;
+    }
+    double gc = g <= limit ? g : limit;                 /* min(g, limit) */
+    double uc = u < -limit ? -limit : (u > limit ? limit : u);
+    double s = 1.0 / (1.0 + exp(-alpha * gc));
+    if (dhdg) *dhdg = (g <= limit) ? (uc + 1.0) * s * (1.0 + alpha * gc * (1.0 - s)) : 0.0;
+    if (dhdu) *dhdu = (u >= -limit && u <= limit) ? gc * s : 0.0;
+    return (uc + 1.0) * gc * s;
+}
 
 /* For each token t in tokens[0..nt) (all tokens when tokens == NULL) and each
  * slot j with expert e = idx[t,j]:
- *   g = x_t W_gate,e^T,  u = x_t W_up,e^T   (W_gate = rows [0,I), W_up = rows
- *   [I,2I) of gate_up, i.e. proj.chunk(2) with gate first),
- *   h = silu(g) * u,
- *   y_t += w_{t,j} * h W_down,e^T,  summed over j in slot order.
+ *   g = x_t W_gate,e^T + bg_e,  u = x_t W_up,e^T + bu_e   (W_gate = rows [0,I),
+ *   W_up = rows [I,2I) of gate_up, i.e. proj.chunk(2) with gate first; the
+ *   biases bgu [E,2I] in the same order, zero when bgu == NULL),
+ *   h = expert_act(g, u)   (silu(g) * u for act 0),
+ *   y_t += w_{t,j} * (h W_down,e^T + bd_e),  summed over j in slot order
+ *   (bd [E,H], zero when NULL).
  * x: [T,H] fp64, wgu: [E,2I,H] fp32 (dequantized), wd: [E,H,I] fp32,
  * y: [nt,H] fp64 (row i belongs to tokens[i]). */
 int e4bo_forward(const double *x, int64_t T, int E, int H, int I, int k,
                  const int32_t *idx, const double *wts, const float *wgu,
-                 const float *wd, const int64_t *tokens, int64_t nt, double *y) {
-    if (!x || !idx || !wts || !wgu || !wd || !y || T < 0 || E <= 0 || k <= 0) return ORC_ERR_ARG;
+                 const float *wd, const int64_t *tokens, int64_t nt, int act, double alpha, double limit,
+                 const float *bgu, const float *bd, double *y) {
+    if (!x || !idx || !wts || !wgu || !wd || !y || T < 0 || E <= 0 || k <= 0 || act < 0 || act > 1) return ORC_ERR_ARG;
     if (!tokens) nt = T;
 #pragma omp parallel
     {
@@ -271,16 +299,17 @@ int e4bo_forward(const double *x, int64_t T, int E, int H, int I, int k,
                 const float *Wu = Wg + (int64_t)I * H;
                 const float *Wd = wd + (int64_t)e * H * I;
                 for (int r = 0; r < I; ++r) {
-                    double g = 0.0, u = 0.0;
+                    double g = bgu ? (double)bgu[(int64_t)e * 2 * I + r] : 0.0;
+                    double u = bgu ? (double)bgu[(int64_t)e * 2 * I + I + r] : 0.0;
                     for (int c = 0; c < H; ++c) {
                         g += xt[c] * (double)Wg[(int64_t)r * H + c];
                         u += xt[c] * (double)Wu[(int64_t)r * H + c];
                     }
-                    h[r] = silu(g) * u;
+                    h[r] = expert_act(act, alpha, limit, g, u, NULL, NULL);
                 }
                 double w = wts[t * k + j];
                 for (int c = 0; c < H; ++c) {
-                    double acc = 0.0;
+                    double acc = bd ? (double)bd[(int64_t)e * H + c] : 0.0;
                     for (int r = 0; r < I; ++r) acc += h[r] * (double)Wd[(int64_t)c * I + r];
                     yt[c] += w * acc;
                 }
@@ -295,15 +324,17 @@ int e4bo_forward(const double *x, int64_t T, int E, int H, int I, int k,
 
 /* grad_x_t = sum_j dx_{t,j}, routing held constant:
  *   dY   = w_{t,j} * grad_out_t
- *   dh   = dY W_down,e                    (contract over H)
- *   dG   = dh * u * s(g) * (1 + g (1 - s(g)))   with s the logistic function
- *   dU   = dh * silu(g)
+ *   dh   = dY W_down,e                    (contract over H; the down bias drops out)
+ *   dG   = dh * dh/dg,  dU = dh * dh/du   (expert_act's partials; for SwiGLU
+ *          dh/dg = u s(g) (1 + g (1 - s(g))), dh/du = silu(g), s the logistic function)
  *   dx   = dG W_gate,e + dU W_up,e        (contract over 2I)
- * with g, u recomputed from x and the dequantized weights (never saved). */
+ * with g, u (biases included) recomputed from x and the dequantized weights. */
 int e4bo_dgrad(const double *x, const double *gout, int64_t T, int E, int H, int I, int k,
                const int32_t *idx, const double *wts, const float *wgu, const float *wd,
-               const int64_t *tokens, int64_t nt, double *gx) {
-    if (!x || !gout || !idx || !wts || !wgu || !wd || !gx || T < 0 || E <= 0 || k <= 0) return ORC_ERR_ARG;
+               const int64_t *tokens, int64_t nt, int act, double alpha, double limit, const float *bgu,
+               double *gx) {
+    if (!x || !gout || !idx || !wts || !wgu || !wd || !gx || T < 0 || E <= 0 || k <= 0 || act < 0 || act > 1)
+        return ORC_ERR_ARG;
     if (!tokens) nt = T;
 #pragma omp parallel
     {
@@ -323,15 +354,18 @@ int e4bo_dgrad(const double *x, const double *gout, int64_t T, int E, int H, int
                 const float *Wd = wd + (int64_t)e * H * I;
                 double w = wts[t * k + j];
                 for (int r = 0; r < I; ++r) {
-                    double g = 0.0, u = 0.0, dh = 0.0;
+                    double g = bgu ? (double)bgu[(int64_t)e * 2 * I + r] : 0.0;
+                    double u = bgu ? (double)bgu[(int64_t)e * 2 * I + I + r] : 0.0;
+                    double dh = 0.0;
                     for (int c = 0; c < H; ++c) {
                         g += xt[c] * (double)Wg[(int64_t)r * H + c];
                         u += xt[c] * (double)Wu[(int64_t)r * H + c];
                         dh += w * go[c] * (double)Wd[(int64_t)c * I + r];
                     }
-                    double s = 1.0 / (1.0 + exp(-g));
-                    dG[r] = dh * u * s * (1.0 + g * (1.0 - s));
-                    dU[r] = dh * g * s;
+                    double dhdg, dhdu;
+                    expert_act(act, alpha, limit, g, u, &dhdg, &dhdu);
+                    dG[r] = dh * dhdg;
+                    dU[r] = dh * dhdu;
                 }
                 for (int c = 0; c < H; ++c) {
                     double acc = 0.0;
@@ -362,8 +396,10 @@ int e4bo_dgrad(const double *x, const double *gout, int64_t T, int E, int H, int
  * dw: [nt, k]; dlogits (may be NULL): [nt, E]; row i belongs to tokens[i]. */
 int e4bo_router_grad(const double *x, const double *gout, const float *logits, int64_t T, int E, int H, int I,
                      int k, int renorm, const int32_t *idx, const float *wgu, const float *wd,
-                     const int64_t *tokens, int64_t nt, double *dw, double *dlogits) {
-    if (!x || !gout || !idx || !wgu || !wd || !dw || T < 0 || E <= 0 || k <= 0) return ORC_ERR_ARG;
+                     const int64_t *tokens, int64_t nt, int act, double alpha, double limit, const float *bgu,
+                     const float *bd, double *dw, double *dlogits) {
+    if (!x || !gout || !idx || !wgu || !wd || !dw || T < 0 || E <= 0 || k <= 0 || act < 0 || act > 1)
+        return ORC_ERR_ARG;
     if (dlogits && !logits) return ORC_ERR_ARG;
     if (!tokens) nt = T;
     for (int64_t p = 0; p < T * k; ++p)
@@ -383,16 +419,17 @@ int e4bo_router_grad(const double *x, const double *gout, const float *logits, i
                 const float *Wu = Wg + (int64_t)I * H;
                 const float *Wd = wd + (int64_t)e * H * I;
                 for (int r = 0; r < I; ++r) {
-                    double g = 0.0, u = 0.0;
+                    double g = bgu ? (double)bgu[(int64_t)e * 2 * I + r] : 0.0;
+                    double u = bgu ? (double)bgu[(int64_t)e * 2 * I + I + r] : 0.0;
                     for (int c = 0; c < H; ++c) {
                         g += xt[c] * (double)Wg[(int64_t)r * H + c];
                         u += xt[c] * (double)Wu[(int64_t)r * H + c];
                     }
-                    h[r] = silu(g) * u;
+                    h[r] = expert_act(act, alpha, limit, g, u, NULL, NULL);
                 }
                 double d = 0.0;
                 for (int c = 0; c < H; ++c) {
-                    double yc = 0.0;
+                    double yc = bd ? (double)bd[(int64_t)e * H + c] : 0.0;
                     for (int r = 0; r < I; ++r) yc += h[r] * (double)Wd[(int64_t)c * I + r];
                     d += go[c] * yc;
                 }

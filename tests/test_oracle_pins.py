@@ -424,3 +424,119 @@ def test_zipf_router_hot_set():
     c = np.sort(np.bincount(idx.ravel(), minlength=w.E))[::-1]
     share = c[:8].sum() / c.sum()
     assert 0.35 < share < 0.65
+
+
+# -------------------------------------------------------------- gpt-oss expert variant
+# Clamped GLU h = (u' + 1) g' sigmoid(alpha g'), g' = min(g, L), u' = clamp(u, -L, L),
+# with per-expert biases on g, u (bgu [E, 2I], gate half first) and on the down output.
+
+GLU = oracle.ACT_CLAMPED_GLU
+
+
+def _biases(E, H, I, seed, scale=0.5):
+    rng = np.random.default_rng(seed)
+    return (rng.standard_normal((E, 2 * I)) * scale).astype(np.float32), \
+        (rng.standard_normal((E, H)) * scale).astype(np.float32)
+
+
+def test_clamped_glu_alpha1_unclamped_is_swiglu_with_unit_up_bias():
+    """alpha = 1, L = inf: (u + 1) silu(g) is SwiGLU with the up pre-activation
+    shifted by one, i.e. SwiGLU with up bias 1 (gate bias 0)."""
+    x, idx, w, wgu, wd, *_ = _tiny_problem(E=5, H=64, I=64, T=12, k=2, seed=31)
+    E, I2, H = wgu.shape
+    bgu1 = np.concatenate([np.zeros((E, I2 // 2)), np.ones((E, I2 // 2))], 1).astype(np.float32)
+    y_glu = oracle.forward(x, idx, w, wgu, wd, act=GLU, alpha=1.0, limit=np.inf)
+    y_sw = oracle.forward(x, idx, w, wgu, wd, bgu=bgu1)
+    np.testing.assert_allclose(y_glu, y_sw, rtol=1e-12, atol=1e-14 * np.abs(y_sw).max())
+
+
+def test_clamped_glu_large_alpha_is_relu_gated():
+    """alpha -> inf turns sigmoid(alpha g) into the unit step: h -> (u' + 1) relu(g')."""
+    x, idx, w, wgu, wd, *_ = _tiny_problem(E=4, H=64, I=64, T=10, k=2, seed=32)
+    E, I2, H = wgu.shape
+    I = I2 // 2
+    y = oracle.forward(x, idx, w, wgu, wd, act=GLU, alpha=1e9, limit=0.3)
+    xd = x.astype(np.float64)
+    ref = np.zeros_like(y)
+    for t in range(x.shape[0]):
+        for j in range(idx.shape[1]):
+            e = idx[t, j]
+            g = wgu[e, :I].astype(np.float64) @ xd[t]
+            u = wgu[e, I:].astype(np.float64) @ xd[t]
+            h = (np.clip(u, -0.3, 0.3) + 1.0) * np.maximum(np.minimum(g, 0.3), 0.0)
+            ref[t] += w[t, j] * (wd[e].astype(np.float64) @ h)
+    np.testing.assert_allclose(y, ref, rtol=1e-9, atol=1e-12 * np.abs(ref).max())
+
+
+def test_clamped_glu_clamp_invariances():
+    """Outside the clamp the up pre-activation does not matter; inside it the limit does not."""
+    x, idx, w, wgu, wd, *_ = _tiny_problem(E=4, H=64, I=64, T=9, k=2, seed=33)
+    E, I2, H = wgu.shape
+    I = I2 // 2
+    # every |g|, |u| below 10: a limit of 10 equals no limit
+    np.testing.assert_allclose(oracle.forward(x, idx, w, wgu, wd, act=GLU, limit=10.0),
+                               oracle.forward(x, idx, w, wgu, wd, act=GLU, limit=np.inf), rtol=0, atol=0)
+    # up bias 5 pushes every u above L = 1: scaling the up weights changes nothing
+    b = np.concatenate([np.zeros((E, I)), np.full((E, I), 5.0)], 1).astype(np.float32)
+    w2 = wgu.copy()
+    w2[:, I:] *= 0.5
+    y1 = oracle.forward(x, idx, w, wgu, wd, act=GLU, limit=1.0, bgu=b)
+    y2 = oracle.forward(x, idx, w, w2, wd, act=GLU, limit=1.0, bgu=b)
+    np.testing.assert_array_equal(y1, y2)
+
+
+def test_down_bias_adds_routing_weighted_bias():
+    """y(bd) - y(0) = sum_j w_{t,j} bd[e_{t,j}] for every token."""
+    x, idx, w, wgu, wd, *_ = _tiny_problem(E=6, H=64, I=64, T=11, k=3, seed=34)
+    E, I2, H = wgu.shape
+    bgu, bd = _biases(E, H, I2 // 2, 35)
+    d = oracle.forward(x, idx, w, wgu, wd, act=GLU, bgu=bgu, bd=bd) - oracle.forward(x, idx, w, wgu, wd, act=GLU,
+                                                                                      bgu=bgu)
+    ref = np.einsum("tj,tjh->th", w, bd[idx].astype(np.float64))
+    np.testing.assert_allclose(d, ref, rtol=1e-10, atol=1e-12)
+
+
+def test_clamped_glu_dgrad_matches_central_finite_differences():
+    """Biases and a limit that clamps part of g and u (no pre-activation within eps of a kink)."""
+    x, idx, w, wgu, wd, *_ = _tiny_problem(E=4, H=64, I=64, T=6, k=2, seed=36)
+    E, I2, H = wgu.shape
+    bgu, bd = _biases(E, H, I2 // 2, 37)
+    kw = dict(act=GLU, alpha=1.702, limit=0.8, bgu=bgu)
+    go = np.random.default_rng(38).standard_normal(x.shape)
+    gx = oracle.dgrad(x, go, idx, w, wgu, wd, **kw)
+    eps = 1e-6
+    num = np.zeros_like(gx)
+    for t in range(x.shape[0]):
+        for c in range(x.shape[1]):
+            xp = x.astype(np.float64).copy()
+            xm = xp.copy()
+            xp[t, c] += eps
+            xm[t, c] -= eps
+            fp = (oracle.forward(xp, idx, w, wgu, wd, tokens=[t], bd=bd, **kw) * go[t]).sum()
+            fm = (oracle.forward(xm, idx, w, wgu, wd, tokens=[t], bd=bd, **kw) * go[t]).sum()
+            num[t, c] = (fp - fm) / (2 * eps)
+    np.testing.assert_allclose(gx, num, rtol=1e-6, atol=1e-6 * np.abs(num).max())
+    # the clamp is active somewhere, so the test exercises the zero-gradient branch
+    xd = x.astype(np.float64)
+    g = np.einsum("th,eih->eti", xd, wgu[:, :I2 // 2]) + bgu[:, None, :I2 // 2]
+    u = np.einsum("th,eih->eti", xd, wgu[:, I2 // 2:]) + bgu[:, None, I2 // 2:]
+    assert (g > 0.8).any() and (np.abs(u) > 0.8).any()
+
+
+def test_clamped_glu_router_grad_dw_matches_central_finite_differences():
+    x, idx, w, wgu, wd, *_ = _tiny_problem(E=5, H=64, I=64, T=6, k=2, seed=39)
+    E, I2, H = wgu.shape
+    bgu, bd = _biases(E, H, I2 // 2, 40)
+    kw = dict(act=GLU, alpha=1.702, limit=0.8, bgu=bgu, bd=bd)
+    go = np.random.default_rng(41).standard_normal(x.shape)
+    dw, _ = oracle.router_grad(x, go, None, idx, True, wgu, wd, **kw)
+    eps = 1e-3
+    num = np.zeros_like(dw)
+    for t in range(x.shape[0]):
+        for j in range(idx.shape[1]):
+            wp, wm = w.copy(), w.copy()
+            wp[t, j] += eps
+            wm[t, j] -= eps
+            num[t, j] = ((oracle.forward(x, idx, wp, wgu, wd, **kw) - oracle.forward(x, idx, wm, wgu, wd, **kw))
+                         * go).sum() / (2 * eps)
+    np.testing.assert_allclose(dw, num, rtol=1e-8, atol=1e-10 * np.abs(num).max())
