@@ -41,8 +41,8 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-aux", action="store_true", help="skip the decode and quantize/dequantize legs")
-    ap.add_argument("--leg", default="step", choices=["step", "decode", "codec"],
-                    help="step: the benchmark line; decode / codec: only that secondary leg (for profiling), "
+    ap.add_argument("--leg", default="step", choices=["step", "decode", "codec", "variant"],
+                    help="step: the benchmark line; decode / codec / variant: only that secondary leg (for profiling), "
                          "decode on the Qwen3-shaped layer at --tokens (default 1)")
     return ap.parse_args()
 
@@ -231,6 +231,64 @@ def decode_leg(w, dev, reps=20):
             "experts_touched": touched, "bytes_per_forward": nbytes, "weight_stream_gbs": gbs,
             "roofline": {"bound": "hbm", "achieved": gbs, "peak": hbm, "unit": "GB/s", "frac": gbs / hbm},
             "layer_copies": copies, "kernels_per_forward": launches_per_fwd, "timing": "CUDA graph, events"}
+
+
+def variant_leg(w, dev, reps=10):
+    """The gpt-oss expert variant (per-expert biases, clamped GLU alpha 1.702 and
+    limit 7) on workload w: forward (routed from logits, derivatives saved) plus
+    input gradient, L2 flushed between steps; tokens/s and the whole step against
+    the dense-bf16 peak (12*H*I FLOP per pair)."""
+    import torch
+    import bit_quantized_mixture_nf4_b200 as e4b
+    from bit_quantized_mixture_nf4_b200 import workloads as wl
+    bf16 = peaks()[1]
+    x = wl.activations(w).to(dev)
+    logits = wl.router_logits(w, wl.activations(w)).to(dev)
+    go = wl.grad_output(w).to(dev)
+    gu, dn = wl.weights(w, device=dev)
+    pg, ag = e4b.e4b_quantize_nf4(gu, codebook=w.codebook)
+    pd, ad = e4b.e4b_quantize_nf4(dn, codebook=w.codebook)
+    del gu, dn
+    g = torch.Generator(device=dev)
+    g.manual_seed(w.seed + 7)
+    bgu = torch.randn(w.E, 2 * w.I, device=dev, generator=g) * 0.3
+    bd = torch.randn(w.E, w.H, device=dev, generator=g) * 0.3
+    experts = e4b.make_experts(pg, pd, ag, ad, bgu, bd)
+    desc = e4b.make_desc(w.E, w.H, w.I, w.k, w.renorm, w.codebook, 64, e4b.PATH_GROUPED, e4b.ACT_CLAMPED_GLU,
+                         1.702, 7.0)
+    P = w.T * w.k
+    idx = torch.empty(w.T, w.k, dtype=torch.int32, device=dev)
+    wts = torch.empty(w.T, w.k, dtype=torch.float32, device=dev)
+    y = torch.empty(w.T, w.H, dtype=torch.bfloat16, device=dev)
+    gx = torch.empty(w.T, w.H, dtype=torch.bfloat16, device=dev)
+    saved = torch.empty(P, 2 * w.I, dtype=torch.bfloat16, device=dev)
+    ws = e4b.workspace(desc, w.T, dev)
+    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
+
+    def step():
+        e4b.e4b_moe_forward(desc, experts, x, logits, idx, wts, y, saved_gu=saved, ws=ws)
+        e4b.e4b_moe_backward_dgrad(desc, experts, x, idx, wts, go, saved_gu=saved, grad_x=gx, ws=ws)
+
+    for _ in range(3):
+        step()
+    torch.cuda.synchronize(dev)
+    ss = [torch.cuda.Event(enable_timing=True) for _ in range(reps)]
+    ee = [torch.cuda.Event(enable_timing=True) for _ in range(reps)]
+    for i in range(reps):
+        flush.zero_()
+        ss[i].record()
+        step()
+        ee[i].record()
+    torch.cuda.synchronize(dev)
+    ms = sum(a.elapsed_time(b) for a, b in zip(ss, ee)) / reps
+    if e4b.e4b_device_status() != e4b.E4B_OK:
+        raise RuntimeError("device status not ok after the variant leg")
+    tf = 12 * w.H * w.I * P / (ms / 1e3) / 1e12
+    return {"workload": f"{w.name}-shaped E={w.E} H={w.H} I={w.I} top{w.k} T={w.T} "
+                        f"{'fp4' if w.codebook else 'nf4'}, clamped GLU + per-expert biases, fwd + dgrad",
+            "ms_per_step": ms, "tokens_per_s": w.T / (ms / 1e3),
+            "roofline": {"bound": "tensor", "achieved": tf, "peak": bf16, "unit": "TFLOP/s", "frac": tf / bf16},
+            "l2": "flushed between steps"}
 
 
 def codec_leg(w, dev, reps=10):
@@ -547,6 +605,8 @@ def run_e4b(args, w):
                                                       wl.QWEN3.with_tokens(8))]
         torch.cuda.empty_cache()
         aux["codec"] = codec_leg(wl.OLMOE, dev)
+        torch.cuda.empty_cache()
+        aux["gptoss_variant"] = variant_leg(wl.GPTOSS.with_tokens(2048), dev)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -589,6 +649,8 @@ def main():
         if args.leg == "decode":
             tokens = args.tokens if args.tokens <= 8 else 1
             print(json.dumps(decode_leg(wl.QWEN3.with_tokens(tokens), dev, reps=max(args.steps, 3))), flush=True)
+        elif args.leg == "variant":
+            print(json.dumps(variant_leg(wl.GPTOSS.with_tokens(2048), dev, reps=max(args.steps, 3))), flush=True)
         else:
             print(json.dumps(codec_leg(wl.OLMOE, dev, reps=max(args.steps, 3))), flush=True)
         return

@@ -22,6 +22,7 @@ E4B_OK, E4B_ERR_INVALID_ARG, E4B_ERR_BLOCKSIZE, E4B_ERR_UNSUPPORTED, E4B_ERR_WOR
 NF4, FP4 = 0, 1
 F32, BF16 = 0, 1
 PATH_AUTO, PATH_GROUPED, PATH_DECODE = 0, 1, 2
+ACT_SWIGLU, ACT_CLAMPED_GLU = 0, 1
 
 EXPORTS = ("e4b_quantize_nf4", "e4b_dequantize_nf4", "e4b_moe_workspace_size", "e4b_moe_forward",
            "e4b_moe_backward_dgrad", "e4b_moe_backward_router", "e4b_device_status", "e4b_status_string",
@@ -36,12 +37,13 @@ KERNEL_KINDS = ("quantize", "dequantize", "route", "group", "gather", "combine",
 class e4b_moe_desc(ctypes.Structure):
     _fields_ = [("E", ctypes.c_int), ("H", ctypes.c_int), ("I", ctypes.c_int), ("top_k", ctypes.c_int),
                 ("renormalize", ctypes.c_int), ("codebook", ctypes.c_int), ("blocksize", ctypes.c_int),
-                ("path", ctypes.c_int)]
+                ("path", ctypes.c_int), ("activation", ctypes.c_int), ("glu_alpha", ctypes.c_float),
+                ("glu_limit", ctypes.c_float)]
 
 
 class e4b_experts(ctypes.Structure):
     _fields_ = [("gate_up", ctypes.c_void_p), ("down", ctypes.c_void_p), ("gate_up_absmax", ctypes.c_void_p),
-                ("down_absmax", ctypes.c_void_p)]
+                ("down_absmax", ctypes.c_void_p), ("gate_up_bias", ctypes.c_void_p), ("down_bias", ctypes.c_void_p)]
 
 
 class E4BError(RuntimeError):
@@ -198,16 +200,26 @@ def e4b_dequantize_nf4(packed: torch.Tensor, absmax: torch.Tensor, shape, blocks
     return out
 
 
-def make_desc(E, H, I, top_k, renormalize=True, codebook=NF4, blocksize=64, path=PATH_AUTO) -> e4b_moe_desc:
-    return e4b_moe_desc(E, H, I, top_k, int(bool(renormalize)), codebook, blocksize, path)
+def make_desc(E, H, I, top_k, renormalize=True, codebook=NF4, blocksize=64, path=PATH_AUTO, activation=ACT_SWIGLU,
+              glu_alpha=1.702, glu_limit=7.0) -> e4b_moe_desc:
+    return e4b_moe_desc(E, H, I, top_k, int(bool(renormalize)), codebook, blocksize, path, activation, glu_alpha,
+                        glu_limit)
 
 
-def make_experts(gate_up, down, gate_up_absmax, down_absmax) -> e4b_experts:
+def make_experts(gate_up, down, gate_up_absmax, down_absmax, gate_up_bias=None, down_bias=None) -> e4b_experts:
+    """The two packed stacks and their absmax (device tensors), plus optional fp32
+    per-expert biases gate_up_bias [E, 2I] and down_bias [E, H].  The tensors must
+    outlive every call that uses the returned struct."""
     for n, t in (("gate_up", gate_up), ("down", down)):
         _cuda(t, n, torch.uint8)
     for n, t in (("gate_up_absmax", gate_up_absmax), ("down_absmax", down_absmax)):
         _cuda(t, n, torch.float32)
-    return e4b_experts(gate_up.data_ptr(), down.data_ptr(), gate_up_absmax.data_ptr(), down_absmax.data_ptr())
+    for n, t in (("gate_up_bias", gate_up_bias), ("down_bias", down_bias)):
+        if t is not None:
+            _cuda(t, n, torch.float32)
+    return e4b_experts(gate_up.data_ptr(), down.data_ptr(), gate_up_absmax.data_ptr(), down_absmax.data_ptr(),
+                       None if gate_up_bias is None else gate_up_bias.data_ptr(),
+                       None if down_bias is None else down_bias.data_ptr())
 
 
 def e4b_moe_workspace_size(desc: e4b_moe_desc, T: int) -> int:

@@ -1,6 +1,7 @@
 // C ABI of the e4b library (declared in include/e4b.h): argument validation,
 // workspace layout and the launch sequence of each entry point.
 #include <atomic>
+#include <cmath>
 #include <cstring>
 #include <mutex>
 #include <utility>
@@ -135,6 +136,9 @@ static e4b_status check_desc(const e4b_moe_desc* d) {
     if (d->top_k < 1 || d->top_k > 8 || d->top_k > d->E) return E4B_ERR_INVALID_ARG;
     if (d->codebook != E4B_CODEBOOK_NF4 && d->codebook != E4B_CODEBOOK_FP4) return E4B_ERR_INVALID_ARG;
     if (d->path < E4B_PATH_AUTO || d->path > E4B_PATH_DECODE) return E4B_ERR_INVALID_ARG;
+    if (d->activation != E4B_ACT_SWIGLU && d->activation != E4B_ACT_CLAMPED_GLU) return E4B_ERR_INVALID_ARG;
+    if (d->activation == E4B_ACT_CLAMPED_GLU && (!std::isfinite(d->glu_alpha) || !(d->glu_limit > 0.0f)))
+        return E4B_ERR_INVALID_ARG;
     return E4B_OK;
 }
 
@@ -152,8 +156,6 @@ static GemmParams base_params(const e4b_moe_desc* d, uint8_t* ws, const WsLayout
                               int64_t P) {
     GemmParams p{};
     p.E = d->E;
-    p.k_top = d->top_k;
-    p.offsets = reinterpret_cast<const int*>(ws + L.offsets);
     p.tile_prefix = reinterpret_cast<const int*>(ws + L.tile_prefix);
     p.sched = reinterpret_cast<const int4*>(ws + L.sched);
     p.perm = reinterpret_cast<const int*>(ws + L.perm);
@@ -181,6 +183,10 @@ static e4b_status run_gateup(const e4b_moe_desc* d, const e4b_experts* w, uint8_
     p.out_bf16 = h_out;
     p.gu = gu_out;
     p.ld_out = d->I;
+    p.act = (int)d->activation;
+    p.alpha = d->glu_alpha;
+    p.limit = d->glu_limit;
+    p.bias = w->gate_up_bias;
     E4B_CUDA_TRY(launch_grouped_gemm(EPI_GATEUP, d->codebook, ws + L.a_perm, P, w->gate_up, p.b_rows_total, d->H / 2,
                                      p, max_m_tiles(P, d->E), st));
     return E4B_OK;
@@ -300,7 +306,10 @@ e4b_status e4b_moe_forward(const e4b_moe_desc* d, const e4b_experts* w, const vo
     const WsLayout L = layout_for(d, T);
     if (!workspace || ws_bytes < L.total) return E4B_ERR_WORKSPACE;
     const bool want_grouped_outputs = saved_gu || offsets_out || perm_out;
-    const bool dec_ok = !want_grouped_outputs && decode_supported(d->H, d->I, T, d->top_k, router_logits != nullptr);
+    // the decode kernels implement SwiGLU without biases
+    const bool plain_experts = d->activation == E4B_ACT_SWIGLU && !w->gate_up_bias && !w->down_bias;
+    const bool dec_ok = !want_grouped_outputs && plain_experts &&
+                        decode_supported(d->H, d->I, T, d->top_k, router_logits != nullptr);
     const bool decode = (d->path == E4B_PATH_DECODE) || (d->path == E4B_PATH_AUTO && dec_ok);
     if (d->path == E4B_PATH_DECODE && !dec_ok) return E4B_ERR_UNSUPPORTED;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
@@ -340,6 +349,7 @@ e4b_status e4b_moe_forward(const e4b_moe_desc* d, const e4b_experts* w, const vo
     p.b_rows_total = (int64_t)d->E * d->H;
     p.b_blocks_per_row = d->I / 64;
     p.out_bf16 = slots;
+    p.bias = w->down_bias;
     p.ld_out = d->H;
     E4B_CUDA_TRY(launch_grouped_gemm(EPI_DOWN, d->codebook, h, P, w->down, p.b_rows_total, d->I / 2, p,
                                      max_m_tiles(P, d->E), st));
@@ -455,6 +465,7 @@ e4b_status e4b_moe_backward_router(const e4b_moe_desc* d, const e4b_experts* w, 
     p.b_rows_total = (int64_t)d->E * d->H;
     p.b_blocks_per_row = d->I / 64;
     p.out_bf16 = a_perm;   // Y, one grouped row per pair
+    p.bias = w->down_bias;
     p.ld_out = d->H;
     E4B_CUDA_TRY(launch_grouped_gemm(EPI_DOWN, d->codebook, h, P, w->down, p.b_rows_total, d->I / 2, p,
                                      max_m_tiles(P, d->E), st));

@@ -15,8 +15,7 @@ namespace e4b {
 enum Epi { EPI_GATEUP = 0, EPI_DOWN = 1, EPI_DGRAD_DOWN = 2, EPI_DGRAD_GATEUP = 3 };
 
 struct GemmParams {
-    int E, K, N, n_tiles, k_top;
-    const int* offsets;       // [E+1] first grouped row of each expert
+    int E, K, N, n_tiles;
     const int* tile_prefix;   // [E+1] prefix of ceil(M_e / tile_rows); [E] = total m-tiles
     const int4* sched;        // per m-tile: (expert, first row, rows, 0)
     const int* perm;          // [P] pair id of each grouped row
@@ -26,10 +25,13 @@ struct GemmParams {
     int b_rows_per_expert;
     int b_blocks_per_row;     // stored cols / 64
     int up_offset;            // I (EPI_GATEUP: first up row; also the feature count)
-    __nv_bfloat16* out_bf16;  // h [P, I], dGU [P, 2I], or the slot rows [P, H] (down / dgrad gate_up)
-    __nv_bfloat16* gu;        // saved SwiGLU derivatives [P, 2I]: dh/dg | dh/du (written by EPI_GATEUP,
-                              // read by EPI_DGRAD_DOWN)
+    int act;                  // EPI_GATEUP: 0 SwiGLU, 1 clamped GLU (alpha, limit below)
+    __nv_bfloat16* out_bf16;  // h [P, I], dGU [P, 2I], or the per-pair rows [P, H] (down / dgrad gate_up)
+    __nv_bfloat16* gu;        // saved activation derivatives [P, 2I]: dh/dg | dh/du (written by
+                              // EPI_GATEUP, read by EPI_DGRAD_DOWN)
+    const float* bias;        // optional per-expert bias: [E, 2I] (EPI_GATEUP) or [E, H] (EPI_DOWN)
     int ld_out;
+    float alpha, limit;
     uint32_t* status;         // device status word
 };
 

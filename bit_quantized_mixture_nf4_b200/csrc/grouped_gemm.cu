@@ -147,7 +147,9 @@ __device__ __forceinline__ int64_t absmax_index(const GemmParams& p, const TileI
     return row * p.b_blocks_per_row + blk;
 }
 
-template <int EPI, int CB, int CTAS>
+// XACT (EPI_GATEUP only): the epilogue handles per-expert biases and the clamped GLU
+// (p.bias, p.act); the plain SwiGLU instance carries none of that code.
+template <int EPI, int CB, int CTAS, bool XACT = false>
 __global__ void __launch_bounds__(GEMM_THREADS, 1)
 grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_raw,
                     const __grid_constant__ CUtensorMap tmap_out, const __grid_constant__ CUtensorMap tmap_gu,
@@ -515,24 +517,57 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_con
                     tmem_load32(tbase + 128 + 32 * q, u);
                     const int f0 = ti.nt * 128 + 32 * q;
                     if (any && f0 < I) {
-                        // h = silu(g) * u, and the two SwiGLU derivatives the input gradient
-                        // needs: dh/dg = u s (1 + g (1 - s)), dh/du = silu(g), s = sigmoid(g)
-                        // in place: u <- dh/dg, g <- dh/du, so few registers stay live
-                        uint32_t hv[16];
+                        if (XACT && p.bias) {   // per-expert bias: lane l loads column f0 + l, shuffles share it
+                            const float bgl = __ldg(p.bias + (int64_t)ti.e * 2 * I + f0 + lane);
+                            const float bul = __ldg(p.bias + (int64_t)ti.e * 2 * I + I + f0 + lane);
 #pragma unroll
-                        for (int i = 0; i < 16; ++i) {
-                            float hh[2];
-#pragma unroll
-                            for (int h = 0; h < 2; ++h) {
-                                const int j = 2 * i + h;
-                                const float gg = g[j], uu = u[j];
-                                const float sg = __fdividef(1.0f, 1.0f + __expf(-gg));
-                                const float sl = gg * sg;
-                                hh[h] = sl * uu;
-                                u[j] = uu * sg * (1.0f + gg * (1.0f - sg));
-                                g[j] = sl;
+                            for (int j = 0; j < 32; ++j) {
+                                g[j] += __shfl_sync(0xffffffffu, bgl, j);
+                                u[j] += __shfl_sync(0xffffffffu, bul, j);
                             }
-                            hv[i] = pack_bf16x2(hh[0], hh[1]);
+                        }
+                        // h = act(g, u) and the two derivatives the input gradient needs, in
+                        // place: u <- dh/dg, g <- dh/du, so few registers stay live.
+                        //   SwiGLU: h = silu(g) u, dh/dg = u s (1 + g (1 - s)), dh/du = silu(g),
+                        //           s = sigmoid(g)
+                        //   clamped GLU: g' = min(g, L), u' = clamp(u, -L, L), s = sigmoid(a g'),
+                        //           h = (u' + 1) g' s, dh/dg = [g <= L] (u' + 1) s (1 + a g' (1 - s)),
+                        //           dh/du = [-L <= u <= L] g' s
+                        uint32_t hv[16];
+                        if (!XACT || p.act == 0) {
+#pragma unroll
+                            for (int i = 0; i < 16; ++i) {
+                                float hh[2];
+#pragma unroll
+                                for (int h = 0; h < 2; ++h) {
+                                    const int j = 2 * i + h;
+                                    const float gg = g[j], uu = u[j];
+                                    const float sg = __fdividef(1.0f, 1.0f + __expf(-gg));
+                                    const float sl = gg * sg;
+                                    hh[h] = sl * uu;
+                                    u[j] = uu * sg * (1.0f + gg * (1.0f - sg));
+                                    g[j] = sl;
+                                }
+                                hv[i] = pack_bf16x2(hh[0], hh[1]);
+                            }
+                        } else {
+                            const float al = p.alpha, L = p.limit;
+#pragma unroll
+                            for (int i = 0; i < 16; ++i) {
+                                float hh[2];
+#pragma unroll
+                                for (int h = 0; h < 2; ++h) {
+                                    const int j = 2 * i + h;
+                                    const float gg = g[j], uu = u[j];
+                                    const float gc = fminf(gg, L), uc = fminf(fmaxf(uu, -L), L);
+                                    const float sg = __fdividef(1.0f, 1.0f + __expf(-al * gc));
+                                    const float gs = gc * sg;
+                                    hh[h] = (uc + 1.0f) * gs;
+                                    u[j] = (gg <= L) ? (uc + 1.0f) * sg * (1.0f + al * gc * (1.0f - sg)) : 0.0f;
+                                    g[j] = (uu >= -L && uu <= L) ? gs : 0.0f;
+                                }
+                                hv[i] = pack_bf16x2(hh[0], hh[1]);
+                            }
                         }
                         auto pack32 = [&](const float (&f)[32], uint32_t (&o)[16]) {
 #pragma unroll
@@ -624,7 +659,16 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_con
                     if (any && c0 < p.N) {
                         if (EPI == EPI_DOWN || EPI == EPI_DGRAD_GATEUP) {
                             // this pair's contribution, rounded to bf16, into its grouped row
-                            // (summed over the k rows of each token by the combine kernel)
+                            // (summed over the k rows of each token by the combine kernel);
+                            // the down projection's per-expert bias joins before the weight
+                            if (EPI == EPI_DOWN && p.bias) {
+                                const float4* bd = reinterpret_cast<const float4*>(p.bias + (int64_t)ti.e * p.N + c0);
+#pragma unroll
+                                for (int i = 0; i < 8; ++i) {
+                                    const float4 b = __ldg(bd + i);
+                                    v[4 * i] += b.x; v[4 * i + 1] += b.y; v[4 * i + 2] += b.z; v[4 * i + 3] += b.w;
+                                }
+                            }
                             uint32_t ov[16];
 #pragma unroll
                             for (int i = 0; i < 16; ++i) ov[i] = pack_bf16x2(v[2 * i] * wgt, v[2 * i + 1] * wgt);
@@ -726,11 +770,11 @@ static bool make_map_2d(CUtensorMap* m, CUtensorMapDataType dt, const void* base
 constexpr int kCtas = 2;
 int gemm_tile_rows() { return Cfg<kCtas>::TILE_M; }
 
-template <int EPI, int CB>
+template <int EPI, int CB, bool XACT = false>
 static cudaError_t launch_one(const CUtensorMap& ma, const CUtensorMap& mr, const CUtensorMap& mo,
                               const CUtensorMap& mg, const GemmParams& p, int grid, cudaStream_t st) {
     using C = Cfg<kCtas, EPI>;
-    auto kern = grouped_gemm_kernel<EPI, CB, kCtas>;
+    auto kern = grouped_gemm_kernel<EPI, CB, kCtas, XACT>;
     static bool attr_set = false;   // per instantiation
     if (!attr_set) {
         cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
@@ -792,6 +836,11 @@ cudaError_t launch_grouped_gemm(int epi, int codebook, const void* a, int64_t a_
     const int grid = (int)std::min<int64_t>(tiles * kCtas, (num_sms() / kCtas) * kCtas);
     if (grid <= 0) return cudaSuccess;
 #define E4B_LAUNCH(E_, C_) return launch_one<E_, C_>(ma, mr, mo, mg, p, grid, st)
+    const bool xact = epi == EPI_GATEUP && (p.act != 0 || p.bias != nullptr);
+    if (xact) {
+        if (codebook == 0) return launch_one<EPI_GATEUP, 0, true>(ma, mr, mo, mg, p, grid, st);
+        return launch_one<EPI_GATEUP, 1, true>(ma, mr, mo, mg, p, grid, st);
+    }
     if (codebook == 0) {
         switch (epi) {
             case EPI_GATEUP: E4B_LAUNCH(EPI_GATEUP, 0);

@@ -9,6 +9,8 @@
  *   [P5] bitsandbytes pull request #1965 "Add Experts4bit for 4-bit quantization
  *        of fused MoE experts", section "What this adds" (recompute-in-backward
  *        input gradient, frozen base).
+ *   [P2] "experts4bit-qlora 0.31.1" PyPI project page, section "Scope": the
+ *        gpt-oss experts (per-expert biases and a clamped GLU).
  *
  * Conventions for every entry point:
  *   - Tensor pointers are DEVICE pointers owned by the caller, contiguous,
@@ -61,6 +63,14 @@ typedef enum {
 typedef enum { E4B_CODEBOOK_NF4 = 0, E4B_CODEBOOK_FP4 = 1 } e4b_codebook;
 typedef enum { E4B_F32 = 0, E4B_BF16 = 1 } e4b_dtype;
 typedef enum { E4B_PATH_AUTO = 0, E4B_PATH_GROUPED = 1, E4B_PATH_DECODE = 2 } e4b_path;
+/* The experts' gated activation of the pre-activations g (gate rows) and u (up rows):
+ *   SWIGLU       h = silu(g) u                                   ([P4] forward)
+ *   CLAMPED_GLU  h = (u' + 1) g' sigmoid(alpha g'),  g' = min(g, limit),
+ *                u' = clamp(u, -limit, limit)                    ([P2] gpt-oss experts;
+ *                the pages give no formula: this is the published gpt-oss expert,
+ *                alpha = 1.702 and limit = 7 there).  The clamp passes the gradient
+ *                where its input lies inside the closed interval. */
+typedef enum { E4B_ACT_SWIGLU = 0, E4B_ACT_CLAMPED_GLU = 1 } e4b_activation;
 
 /* Layer description.  H and I must be multiples of 64 (blocks never straddle a
  * row, [P4] __init__); 1 <= top_k <= min(E, 8); E <= 256; blocksize == 64.
@@ -70,21 +80,33 @@ typedef enum { E4B_PATH_AUTO = 0, E4B_PATH_GROUPED = 1, E4B_PATH_DECODE = 2 } e4
  * tokens: H up to about 16000, I up to about 2900 with caller-given routing
  * and about 6000 at T = 1 with routing from logits), and the grouped
  * tensor-core kernels otherwise; the other values force one path (DECODE
- * outside that range returns E4B_ERR_UNSUPPORTED). */
+ * outside that range returns E4B_ERR_UNSUPPORTED).  The decode kernels implement
+ * SwiGLU without biases only: AUTO takes the grouped kernels for the clamped GLU
+ * or biased experts at every T, and DECODE returns E4B_ERR_UNSUPPORTED for them.
+ * activation: E4B_ACT_SWIGLU (zero-initialised descriptors) or
+ * E4B_ACT_CLAMPED_GLU with glu_alpha finite and glu_limit > 0 (+inf allowed). */
 typedef struct {
     int E, H, I, top_k;
     int renormalize;           /* divide the selected softmax weights by their sum  */
     e4b_codebook codebook;
     int blocksize;             /* must be 64 */
     e4b_path path;
+    e4b_activation activation;
+    float glu_alpha, glu_limit;   /* E4B_ACT_CLAMPED_GLU only */
 } e4b_moe_desc;
 
-/* Device pointers to the two quantized stacks (see storage above). */
+/* Device pointers to the two quantized stacks (see storage above) and the
+ * optional per-expert biases ([P2] gpt-oss experts; NULL = none): gate_up_bias
+ * is added to the gate_up pre-activations (gate half first, like the rows),
+ * down_bias to each expert's output before its routing weight multiplies it.
+ * Bias pointers are 16-byte aligned. */
 typedef struct {
     const uint8_t *gate_up;        /* [E, 2I*H/2] */
     const uint8_t *down;           /* [E, H*I/2]  */
     const float *gate_up_absmax;   /* [E, 2I*H/64] */
     const float *down_absmax;      /* [E, H*I/64]  */
+    const float *gate_up_bias;     /* fp32 [E, 2I] or NULL */
+    const float *down_bias;        /* fp32 [E, H] or NULL  */
 } e4b_experts;
 
 /* Blockwise 4-bit quantization ([P4] from_float / _quantize_stack).
@@ -112,10 +134,11 @@ E4B_API e4b_status e4b_dequantize_nf4(const uint8_t *packed, const float *absmax
 E4B_API size_t e4b_moe_workspace_size(const e4b_moe_desc *d, int64_t T);
 
 /* Forward of the expert layer ([P4] Experts4bit.forward):
- *   y_t = sum_j w_{t,j} * (silu(x_t W_gate,e^T) * (x_t W_up,e^T)) W_down,e^T,
- * e = topk_idx[t,j], W_gate/W_up = rows [0,I)/[I,2I) of gate_up, the weights
- * dequantized to bf16, products accumulated in fp32, the weighted sum over the
- * k slots in fp32, y rounded to bf16.
+ *   y_t = sum_j w_{t,j} * (act(x_t W_gate,e^T + bg_e, x_t W_up,e^T + bu_e) W_down,e^T + bd_e),
+ * e = topk_idx[t,j], W_gate/W_up = rows [0,I)/[I,2I) of gate_up, act the
+ * descriptor's activation (silu(g) * u by default), the biases zero unless
+ * given, the weights dequantized to bf16, products accumulated in fp32, the
+ * weighted sum over the k slots in fp32, y rounded to bf16.
  *   x            bf16 [T, H]
  *   router_logits fp32 [T, E] or NULL.  If given, the layer routes: top-k by
  *                logit (ties to the lower expert index), weights = softmax over
@@ -127,9 +150,9 @@ E4B_API size_t e4b_moe_workspace_size(const e4b_moe_desc *d, int64_t T);
  *   y            bf16 [T, H]
  *   saved_gu     bf16 [T*k, 2I] or NULL: what the input gradient needs from the
  *                forward, in grouped row order (row r holds pair perm[r]): the
- *                SwiGLU derivatives dh/dg = u s(g) (1 + g (1 - s(g))) in columns
- *                [0,I) and dh/du = silu(g) in columns [I,2I), s the logistic
- *                function, for e4b_moe_backward_dgrad.
+ *                activation's derivatives dh/dg in columns [0,I) and dh/du in
+ *                columns [I,2I) (SwiGLU: u s(g) (1 + g (1 - s(g))) and silu(g), s
+ *                the logistic function), for e4b_moe_backward_dgrad.
  *   offsets_out  int32 [E+1] or NULL: first grouped row of each expert.
  *   perm_out     int32 [T*k] or NULL: pair id t*k+j of each grouped row;
  *                experts ascending, tokens ascending inside an expert.
@@ -143,7 +166,8 @@ E4B_API e4b_status e4b_moe_forward(const e4b_moe_desc *d, const e4b_experts *w, 
 /* Input gradient of the forward with routing held constant ([P5] "What this
  * adds": recompute-in-backward; the packed base is frozen, no weight gradient):
  *   dh   = w_{t,j} * grad_out_t W_down,e                 (contract over H)
- *   dG   = dh * u * s(g) * (1 + g (1 - s(g))),  dU = dh * silu(g)
+ *   dG   = dh * dh/dg,  dU = dh * dh/du   (the activation's derivatives; SwiGLU:
+ *          u * s(g) * (1 + g (1 - s(g))) and silu(g))
  *   grad_x_t = sum_j  dG W_gate,e + dU W_up,e            (contract over 2I)
  * with the weights re-dequantized inside the kernels and never stored.
  * The SwiGLU derivatives come from saved_gu (as written by e4b_moe_forward for

@@ -65,8 +65,11 @@ def oracle_weights(prob: Problem, experts=None):
     return wgu, wd
 
 
-def oracle_forward_dgrad(prob: Problem, idx: np.ndarray, wts: np.ndarray, tokens, want_dgrad=True):
-    """Oracle y (and grad_x) for the given tokens, using only the experts they touch."""
+def oracle_forward_dgrad(prob: Problem, idx: np.ndarray, wts: np.ndarray, tokens, want_dgrad=True, act=0,
+                         alpha=1.702, limit=7.0, bgu=None, bd=None):
+    """Oracle y (and grad_x) for the given tokens, using only the experts they touch;
+    act / alpha / limit and the per-expert biases bgu [E, 2I], bd [E, H] as in the
+    oracle's forward."""
     tokens = np.asarray(tokens, np.int64)
     used = np.unique(idx[tokens])
     remap = np.full(prob.w.E, -1, np.int32)
@@ -75,11 +78,12 @@ def oracle_forward_dgrad(prob: Problem, idx: np.ndarray, wts: np.ndarray, tokens
     sub_idx = remap[idx[tokens]]
     sub_w = wts[tokens]
     xs = prob.x.float().numpy()[tokens]
-    y = oracle.forward(xs, sub_idx, sub_w, wgu, wd)
+    kw = dict(act=act, alpha=alpha, limit=limit, bgu=None if bgu is None else np.asarray(bgu)[used])
+    y = oracle.forward(xs, sub_idx, sub_w, wgu, wd, bd=None if bd is None else np.asarray(bd)[used], **kw)
     gx = None
     if want_dgrad:
         gos = prob.grad_out.float().numpy()[tokens]
-        gx = oracle.dgrad(xs, gos, sub_idx, sub_w, wgu, wd)
+        gx = oracle.dgrad(xs, gos, sub_idx, sub_w, wgu, wd, **kw)
     return y, gx
 
 

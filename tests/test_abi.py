@@ -77,6 +77,21 @@ def test_host_side_validation(lib):
     assert f(bad_h, 4, 16, 16, 1 << 30) == lib.E4B_ERR_BLOCKSIZE
     dec = lib.make_desc(8, 256, 512, 2, path=lib.PATH_DECODE)
     assert f(dec, 9, 16, 16, 1 << 40) == lib.E4B_ERR_UNSUPPORTED       # decode path is for T <= 8
+    # activation: known kind, finite alpha, positive (possibly infinite) limit
+    for bad in (lib.make_desc(8, 256, 512, 2, activation=2), lib.make_desc(8, 256, 512, 2, activation=-1),
+                lib.make_desc(8, 256, 512, 2, activation=lib.ACT_CLAMPED_GLU, glu_limit=0.0),
+                lib.make_desc(8, 256, 512, 2, activation=lib.ACT_CLAMPED_GLU, glu_limit=float("nan")),
+                lib.make_desc(8, 256, 512, 2, activation=lib.ACT_CLAMPED_GLU, glu_alpha=float("inf"))):
+        assert lib.e4b_moe_workspace_size(bad, 64) == 0
+        assert f(bad, 4, 16, 16, 1 << 40) == lib.E4B_ERR_INVALID_ARG
+    glu = lib.make_desc(8, 256, 512, 2, activation=lib.ACT_CLAMPED_GLU, glu_limit=float("inf"))
+    assert lib.e4b_moe_workspace_size(glu, 64) == lib.e4b_moe_workspace_size(d, 64)
+    # the decode kernels implement SwiGLU without biases: forcing them is refused before any launch
+    glu_dec = lib.make_desc(8, 256, 512, 2, path=lib.PATH_DECODE, activation=lib.ACT_CLAMPED_GLU)
+    assert f(glu_dec, 2, 16, 16, 1 << 40) == lib.E4B_ERR_UNSUPPORTED
+    exb = lib.e4b_experts(16, 16, 16, 16, 16, None)
+    assert L.e4b_moe_forward(ctypes.byref(dec), ctypes.byref(exb), 16, 2, None, 16, 16, 16, None, None, None, 16,
+                             1 << 40, None) == lib.E4B_ERR_UNSUPPORTED
     g = lambda dd, T: L.e4b_moe_backward_dgrad(ctypes.byref(dd), ctypes.byref(ex2), None, T, 16, 16, 16, None, 16,
                                                16, 1 << 40, None)
     assert g(d, 4) == lib.E4B_ERR_INVALID_ARG                          # needs x when saved_gu is NULL
