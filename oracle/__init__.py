@@ -65,6 +65,10 @@ def _L():
             lib.e4bo_dgrad.argtypes = [P, P, i64, i32, i32, i32, i32, P, P, P, P, P, i64, i32, dbl, dbl, P, P]
             lib.e4bo_router_grad.argtypes = [P, P, P, i64, i32, i32, i32, i32, i32, P, P, P, P, i64, i32, dbl, dbl,
                                              P, P, P, P]
+            lib.e4bo_lora_forward.argtypes = [P, i64, i32, i32, i32, i32, P, P, P, P, P, P, P, P, i32, dbl, i32, dbl,
+                                              dbl, P, P, P]
+            lib.e4bo_lora_backward.argtypes = [P, P, i64, i32, i32, i32, i32, P, P, P, P, P, P, P, P, i32, dbl, i32,
+                                               dbl, dbl, P, P, P, P, P, P]
             lib.e4bo_codebook.argtypes = [i32, P]
             lib.e4bo_f32_to_bf16.argtypes = [ctypes.c_float]
             lib.e4bo_f32_to_bf16.restype = ctypes.c_uint16
@@ -243,3 +247,54 @@ def router_grad(x: np.ndarray, grad_out: np.ndarray, logits, idx: np.ndarray, re
         _p(wd), None if tok is None else _p(tok), nt, int(act), float(alpha), float(limit),
         None if bgu is None else _p(bgu), None if bd is None else _p(bd), _p(dw), None if dl is None else _p(dl)))
     return dw, dl
+
+
+def _lora(agu, bgu_l, ad, bd_l):
+    agu, bgu_l, ad, bd_l = (np.ascontiguousarray(a, np.float32) for a in (agu, bgu_l, ad, bd_l))
+    return agu, bgu_l, ad, bd_l, agu.shape[1]
+
+
+def lora_forward(x, idx, w, wgu, wd, agu, bgu_l, ad, bd_l, scale, act=ACT_SWIGLU, alpha=1.702, limit=7.0, bgu=None,
+                 bd=None) -> np.ndarray:
+    """fp64 forward with per-expert LoRA adapters on both stacks: A_gu [E,r,H],
+    B_gu [E,2I,r], A_d [E,r,I], B_d [E,H,r], update scale (alpha / r)."""
+    x = np.ascontiguousarray(x, np.float64)
+    idx = np.ascontiguousarray(idx, np.int32)
+    w = np.ascontiguousarray(w, np.float64)
+    wgu = np.ascontiguousarray(wgu, np.float32)
+    wd = np.ascontiguousarray(wd, np.float32)
+    agu, bgu_l, ad, bd_l, r = _lora(agu, bgu_l, ad, bd_l)
+    T, H = x.shape
+    E, I2, _ = wgu.shape
+    k = idx.shape[1]
+    y = np.zeros((T, H), np.float64)
+    bgu, bd = _bias(bgu, (E, I2)), _bias(bd, (E, H))
+    _check("e4bo_lora_forward", _L().e4bo_lora_forward(
+        _p(x), T, E, H, I2 // 2, k, _p(idx), _p(w), _p(wgu), _p(wd), _p(agu), _p(bgu_l), _p(ad), _p(bd_l), r,
+        float(scale), int(act), float(alpha), float(limit), None if bgu is None else _p(bgu),
+        None if bd is None else _p(bd), _p(y)))
+    return y
+
+
+def lora_backward(x, grad_out, idx, w, wgu, wd, agu, bgu_l, ad, bd_l, scale, act=ACT_SWIGLU, alpha=1.702, limit=7.0,
+                  bgu=None):
+    """fp64 gradients of <grad_out, y> of lora_forward with the routing held and the
+    base frozen: (grad_x [T,H], dA_gu, dB_gu, dA_d, dB_d) shaped like the adapters."""
+    x = np.ascontiguousarray(x, np.float64)
+    g = np.ascontiguousarray(grad_out, np.float64)
+    idx = np.ascontiguousarray(idx, np.int32)
+    w = np.ascontiguousarray(w, np.float64)
+    wgu = np.ascontiguousarray(wgu, np.float32)
+    wd = np.ascontiguousarray(wd, np.float32)
+    agu, bgu_l, ad, bd_l, r = _lora(agu, bgu_l, ad, bd_l)
+    T, H = x.shape
+    E, I2, _ = wgu.shape
+    k = idx.shape[1]
+    gx = np.zeros((T, H), np.float64)
+    out = [np.zeros(a.shape, np.float64) for a in (agu, bgu_l, ad, bd_l)]
+    bgu = _bias(bgu, (E, I2))
+    _check("e4bo_lora_backward", _L().e4bo_lora_backward(
+        _p(x), _p(g), T, E, H, I2 // 2, k, _p(idx), _p(w), _p(wgu), _p(wd), _p(agu), _p(bgu_l), _p(ad), _p(bd_l), r,
+        float(scale), int(act), float(alpha), float(limit), None if bgu is None else _p(bgu), _p(gx),
+        *[_p(o) for o in out]))
+    return (gx, *out)

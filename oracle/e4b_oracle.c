@@ -469,6 +469,173 @@ int e4bo_router_grad(const double *x, const double *gout, const float *logits, i
     return ORC_OK;
 }
 
+/* ---- per-expert LoRA over the frozen base ([P1] "ExpertsLoRA(base, r, alpha)",
+ * "only the LoRA adapters train"; [P2] section "Prior art": stacked per-expert
+ * adapters [num_experts, r, in] / [num_experts, out, r]).  Reading: both stacks
+ * carry an adapter, the update is the standard LoRA one, scale = alpha / r, no
+ * dropout:
+ *   gu   = x W_gu,e^T + s (x A_gu,e^T) B_gu,e^T          A_gu [E,r,H], B_gu [E,2I,r]
+ *   h    = expert_act(g, u)        (g = gu[0,I), u = gu[I,2I), biases as above)
+ *   Y    = h W_d,e^T + s (h A_d,e^T) B_d,e^T + bd_e       A_d [E,r,I],  B_d [E,H,r]
+ *   y_t  = sum_j w_{t,j} Y_{t,j}
+ * Backward, routing held, base frozen (gradients summed over the pairs of each expert):
+ *   dY = w grad_out_t
+ *   dB_d += s dY (h A_d^T)^T   [H,r];   dA_d += s (dY B_d)^T h   [r,I]
+ *   dh  = dY W_d + s (dY B_d) A_d
+ *   dG, dU = dh * dh/dg, dh * dh/du;  dGU = [dG | dU]
+ *   dB_gu += s dGU (x A_gu^T)^T [2I,r]; dA_gu += s (dGU B_gu)^T x [r,H]
+ *   dx  = dGU W_gu + s (dGU B_gu) A_gu
+ * All in fp64 over the fp32 inputs. */
+static void lora_pair(const double *xt, int H, int I, int r, double s, const float *Wg, const float *Wd,
+                      const float *Ag, const float *Bg, const float *Ad, const float *Bd, int act, double alpha,
+                      double limit, const float *bg, const float *bd, double *za, double *gu, double *h,
+                      double *zd, double *Y) {
+    /* za = x A_gu^T [r]; gu = x W^T + s za B^T (+ bias) [2I] */
+    for (int q = 0; q < r; ++q) {
+        double a = 0.0;
+        for (int c = 0; c < H; ++c) a += xt[c] * (double)Ag[(int64_t)q * H + c];
+        za[q] = a;
+    }
+    for (int o = 0; o < 2 * I; ++o) {
+        double a = bg ? (double)bg[o] : 0.0;
+        for (int c = 0; c < H; ++c) a += xt[c] * (double)Wg[(int64_t)o * H + c];
+        double l = 0.0;
+        for (int q = 0; q < r; ++q) l += za[q] * (double)Bg[(int64_t)o * r + q];
+        gu[o] = a + s * l;
+    }
+    for (int i = 0; i < I; ++i) h[i] = expert_act(act, alpha, limit, gu[i], gu[I + i], NULL, NULL);
+    for (int q = 0; q < r; ++q) {
+        double a = 0.0;
+        for (int i = 0; i < I; ++i) a += h[i] * (double)Ad[(int64_t)q * I + i];
+        zd[q] = a;
+    }
+    if (!Y) return;
+    for (int c = 0; c < H; ++c) {
+        double a = bd ? (double)bd[c] : 0.0;
+        for (int i = 0; i < I; ++i) a += h[i] * (double)Wd[(int64_t)c * I + i];
+        double l = 0.0;
+        for (int q = 0; q < r; ++q) l += zd[q] * (double)Bd[(int64_t)c * r + q];
+        Y[c] = a + s * l;
+    }
+}
+
+int e4bo_lora_forward(const double *x, int64_t T, int E, int H, int I, int k, const int32_t *idx,
+                      const double *wts, const float *wgu, const float *wd, const float *agu, const float *bgu_l,
+                      const float *ad, const float *bd_l, int r, double scale, int act, double alpha,
+                      double limit, const float *bgu, const float *bd, double *y) {
+    if (!x || !idx || !wts || !wgu || !wd || !agu || !bgu_l || !ad || !bd_l || !y || T < 0 || E <= 0 || k <= 0 ||
+        r <= 0 || act < 0 || act > 1)
+        return ORC_ERR_ARG;
+#pragma omp parallel
+    {
+        double *za = (double *)malloc(sizeof(double) * (size_t)r);
+        double *zd = (double *)malloc(sizeof(double) * (size_t)r);
+        double *gu = (double *)malloc(sizeof(double) * (size_t)(2 * I));
+        double *h = (double *)malloc(sizeof(double) * (size_t)I);
+        double *Y = (double *)malloc(sizeof(double) * (size_t)H);
+#pragma omp for schedule(dynamic, 1)
+        for (int64_t t = 0; t < T; ++t) {
+            double *yt = y + t * H;
+            for (int c = 0; c < H; ++c) yt[c] = 0.0;
+            for (int j = 0; j < k; ++j) {
+                int e = idx[t * k + j];
+                lora_pair(x + t * H, H, I, r, scale, wgu + (int64_t)e * 2 * I * H, wd + (int64_t)e * H * I,
+                          agu + (int64_t)e * r * H, bgu_l + (int64_t)e * 2 * I * r, ad + (int64_t)e * r * I,
+                          bd_l + (int64_t)e * H * r, act, alpha, limit, bgu ? bgu + (int64_t)e * 2 * I : NULL,
+                          bd ? bd + (int64_t)e * H : NULL, za, gu, h, zd, Y);
+                for (int c = 0; c < H; ++c) yt[c] += wts[t * k + j] * Y[c];
+            }
+        }
+        free(za); free(zd); free(gu); free(h); free(Y);
+    }
+    return ORC_OK;
+}
+
+/* Gradients of L = <grad_out, y>: gx [T,H], and the adapter gradients dagu [E,r,H],
+ * dbgu [E,2I,r], dad [E,r,I], dbd [E,H,r] (zeroed here, summed over pairs in token
+ * order, so the result does not depend on the thread count). */
+int e4bo_lora_backward(const double *x, const double *gout, int64_t T, int E, int H, int I, int k,
+                       const int32_t *idx, const double *wts, const float *wgu, const float *wd, const float *agu,
+                       const float *bgu_l, const float *ad, const float *bd_l, int r, double scale, int act,
+                       double alpha, double limit, const float *bgu, double *gx, double *dagu, double *dbgu,
+                       double *dad, double *dbd) {
+    if (!x || !gout || !idx || !wts || !wgu || !wd || !agu || !bgu_l || !ad || !bd_l || !gx || !dagu || !dbgu ||
+        !dad || !dbd || T < 0 || E <= 0 || k <= 0 || r <= 0 || act < 0 || act > 1)
+        return ORC_ERR_ARG;
+    memset(dagu, 0, sizeof(double) * (size_t)E * r * H);
+    memset(dbgu, 0, sizeof(double) * (size_t)E * 2 * I * r);
+    memset(dad, 0, sizeof(double) * (size_t)E * r * I);
+    memset(dbd, 0, sizeof(double) * (size_t)E * H * r);
+    double *za = (double *)malloc(sizeof(double) * (size_t)r);
+    double *zd = (double *)malloc(sizeof(double) * (size_t)r);
+    double *gu = (double *)malloc(sizeof(double) * (size_t)(2 * I));
+    double *h = (double *)malloc(sizeof(double) * (size_t)I);
+    double *dY = (double *)malloc(sizeof(double) * (size_t)H);
+    double *vb = (double *)malloc(sizeof(double) * (size_t)r);   /* dY B_d, then dGU B_gu */
+    double *dh = (double *)malloc(sizeof(double) * (size_t)I);
+    double *dgu = (double *)malloc(sizeof(double) * (size_t)(2 * I));
+    for (int64_t t = 0; t < T; ++t) {
+        const double *xt = x + t * H;
+        double *gt = gx + t * H;
+        for (int c = 0; c < H; ++c) gt[c] = 0.0;
+        for (int j = 0; j < k; ++j) {
+            int e = idx[t * k + j];
+            const float *Wg = wgu + (int64_t)e * 2 * I * H, *Wd = wd + (int64_t)e * H * I;
+            const float *Ag = agu + (int64_t)e * r * H, *Bg = bgu_l + (int64_t)e * 2 * I * r;
+            const float *Ad = ad + (int64_t)e * r * I, *Bd = bd_l + (int64_t)e * H * r;
+            double *dAg = dagu + (int64_t)e * r * H, *dBg = dbgu + (int64_t)e * 2 * I * r;
+            double *dAd = dad + (int64_t)e * r * I, *dBd = dbd + (int64_t)e * H * r;
+            lora_pair(xt, H, I, r, scale, Wg, Wd, Ag, Bg, Ad, Bd, act, alpha, limit,
+                      bgu ? bgu + (int64_t)e * 2 * I : NULL, NULL, za, gu, h, zd, NULL);
+            double w = wts[t * k + j];
+            for (int c = 0; c < H; ++c) dY[c] = w * gout[t * H + c];
+            /* down adapter */
+            for (int q = 0; q < r; ++q) {
+                double a = 0.0;
+                for (int c = 0; c < H; ++c) a += dY[c] * (double)Bd[(int64_t)c * r + q];
+                vb[q] = a;
+            }
+            for (int c = 0; c < H; ++c)
+                for (int q = 0; q < r; ++q) dBd[(int64_t)c * r + q] += scale * dY[c] * zd[q];
+            for (int q = 0; q < r; ++q)
+                for (int i = 0; i < I; ++i) dAd[(int64_t)q * I + i] += scale * vb[q] * h[i];
+            for (int i = 0; i < I; ++i) {
+                double a = 0.0;
+                for (int c = 0; c < H; ++c) a += dY[c] * (double)Wd[(int64_t)c * I + i];
+                double l = 0.0;
+                for (int q = 0; q < r; ++q) l += vb[q] * (double)Ad[(int64_t)q * I + i];
+                dh[i] = a + scale * l;
+            }
+            /* activation */
+            for (int i = 0; i < I; ++i) {
+                double dg, du;
+                expert_act(act, alpha, limit, gu[i], gu[I + i], &dg, &du);
+                dgu[i] = dh[i] * dg;
+                dgu[I + i] = dh[i] * du;
+            }
+            /* gate_up adapter and the input gradient */
+            for (int q = 0; q < r; ++q) {
+                double a = 0.0;
+                for (int o = 0; o < 2 * I; ++o) a += dgu[o] * (double)Bg[(int64_t)o * r + q];
+                vb[q] = a;
+            }
+            for (int o = 0; o < 2 * I; ++o)
+                for (int q = 0; q < r; ++q) dBg[(int64_t)o * r + q] += scale * dgu[o] * za[q];
+            for (int q = 0; q < r; ++q)
+                for (int c = 0; c < H; ++c) dAg[(int64_t)q * H + c] += scale * vb[q] * xt[c];
+            for (int c = 0; c < H; ++c) {
+                double a = 0.0;
+                for (int o = 0; o < 2 * I; ++o) a += dgu[o] * (double)Wg[(int64_t)o * H + c];
+                double l = 0.0;
+                for (int q = 0; q < r; ++q) l += vb[q] * (double)Ag[(int64_t)q * H + c];
+                gt[c] += a + scale * l;
+            }
+        }
+    }
+    free(za); free(zd); free(gu); free(h); free(dY); free(vb); free(dh); free(dgu);
+    return ORC_OK;
+}
+
 int e4bo_num_threads(void) {
 #ifdef _OPENMP
     return omp_get_max_threads();

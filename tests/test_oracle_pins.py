@@ -540,3 +540,105 @@ def test_clamped_glu_router_grad_dw_matches_central_finite_differences():
             num[t, j] = ((oracle.forward(x, idx, wp, wgu, wd, **kw) - oracle.forward(x, idx, wm, wgu, wd, **kw))
                          * go).sum() / (2 * eps)
     np.testing.assert_allclose(dw, num, rtol=1e-8, atol=1e-10 * np.abs(num).max())
+
+
+# -------------------------------------------------------------- per-expert LoRA (next row)
+# Adapters A_gu [E,r,H], B_gu [E,2I,r], A_d [E,r,I], B_d [E,H,r]; update scale s = alpha / r.
+
+def _adapters(E, H, I, r, seed, zero_b=False):
+    rng = np.random.default_rng(seed)
+    agu = (rng.standard_normal((E, r, H)) * 0.1).astype(np.float32)
+    bgu_l = np.zeros((E, 2 * I, r), np.float32) if zero_b else (rng.standard_normal((E, 2 * I, r)) * 0.1).astype(np.float32)
+    ad = (rng.standard_normal((E, r, I)) * 0.1).astype(np.float32)
+    bd_l = np.zeros((E, H, r), np.float32) if zero_b else (rng.standard_normal((E, H, r)) * 0.1).astype(np.float32)
+    return agu, bgu_l, ad, bd_l
+
+
+@pytest.mark.parametrize("act", [oracle.ACT_SWIGLU, GLU])
+def test_lora_zero_b_is_the_base_layer(act):
+    """LoRA's B starts at zero: the adapted layer is then exactly the base layer."""
+    x, idx, w, wgu, wd, *_ = _tiny_problem(E=5, H=64, I=64, T=10, k=2, seed=81)
+    ad_ = _adapters(5, 64, 64, 8, 82, zero_b=True)
+    bgu, bd = _biases(5, 64, 64, 83)
+    np.testing.assert_array_equal(oracle.lora_forward(x, idx, w, wgu, wd, *ad_, 2.0, act=act, bgu=bgu, bd=bd),
+                                  oracle.forward(x, idx, w, wgu, wd, act=act, bgu=bgu, bd=bd))
+
+
+def test_lora_equals_base_with_merged_weights():
+    """x W^T + s (x A^T) B^T = x (W + s B A)^T: the adapted layer equals the base layer
+    evaluated with the merged dense weights."""
+    x, idx, w, wgu, wd, *_ = _tiny_problem(E=4, H=64, I=64, T=12, k=2, seed=84)
+    agu, bgu_l, ad, bd_l = _adapters(4, 64, 64, 4, 85)
+    s = 16.0 / 4
+    mg = (wgu.astype(np.float64) + s * np.einsum("eor,erh->eoh", bgu_l, agu)).astype(np.float32)
+    md = (wd.astype(np.float64) + s * np.einsum("ehr,eri->ehi", bd_l, ad)).astype(np.float32)
+    y = oracle.lora_forward(x, idx, w, wgu, wd, agu, bgu_l, ad, bd_l, s)
+    ref = oracle.forward(x, idx, w, mg, md)
+    np.testing.assert_allclose(y, ref, rtol=2e-5, atol=2e-6 * np.abs(ref).max())
+
+
+@pytest.mark.parametrize("act", [oracle.ACT_SWIGLU, GLU])
+def test_lora_single_expert_matches_torch_autograd(act):
+    """E = 1, k = 1, w = 1: a dense MLP with LoRA on both projections; forward and every
+    gradient against torch autograd in fp64."""
+    E, H, I, r, T = 1, 64, 64, 4, 7
+    x, _, _, wgu, wd, *_ = _tiny_problem(E=E, H=H, I=I, T=T, k=1, seed=86)
+    idx = np.zeros((T, 1), np.int32)
+    w = np.ones((T, 1))
+    agu, bgu_l, ad, bd_l = _adapters(E, H, I, r, 87)
+    bgu, bd = _biases(E, H, I, 88)
+    s, al, L = 2.5, 1.702, 0.9
+    go = np.random.default_rng(89).standard_normal((T, H))
+    y = oracle.lora_forward(x, idx, w, wgu, wd, agu, bgu_l, ad, bd_l, s, act=act, alpha=al, limit=L, bgu=bgu, bd=bd)
+    gx, dag, dbg, dad, dbd = oracle.lora_backward(x, go, idx, w, wgu, wd, agu, bgu_l, ad, bd_l, s, act=act, alpha=al,
+                                                  limit=L, bgu=bgu)
+    tt = lambda a, grad=False: torch.tensor(np.asarray(a, np.float64), requires_grad=grad)
+    X, Ag, Bg, Ad, Bd = tt(x, True), tt(agu[0], True), tt(bgu_l[0], True), tt(ad[0], True), tt(bd_l[0], True)
+    gu = X @ tt(wgu[0]).T + s * (X @ Ag.T) @ Bg.T + tt(bgu[0])
+    g, u = gu[:, :I], gu[:, I:]
+    if act == oracle.ACT_SWIGLU:
+        h = torch.nn.functional.silu(g) * u
+    else:
+        gc, uc = torch.clamp(g, max=L), torch.clamp(u, -L, L)
+        h = (uc + 1) * gc * torch.sigmoid(al * gc)
+    Y = h @ tt(wd[0]).T + s * (h @ Ad.T) @ Bd.T + tt(bd[0])
+    (Y * tt(go)).sum().backward()
+    np.testing.assert_allclose(y, Y.detach().numpy(), rtol=1e-11, atol=1e-13)
+    for mine, ref in ((gx, X.grad), (dag[0], Ag.grad), (dbg[0], Bg.grad), (dad[0], Ad.grad), (dbd[0], Bd.grad)):
+        np.testing.assert_allclose(mine, ref.numpy(), rtol=1e-10, atol=1e-12 * np.abs(ref.numpy()).max())
+
+
+def test_lora_routed_gradients_match_central_finite_differences():
+    """Several experts, k = 2, routing weights: the adapter gradients sum over each
+    expert's pairs (sampled entries) and grad_x (all entries) by central differences."""
+    E, H, I, r = 4, 64, 64, 4
+    x, idx, w, wgu, wd, *_ = _tiny_problem(E=E, H=H, I=I, T=6, k=2, seed=90)
+    ad_ = list(_adapters(E, H, I, r, 91))
+    s = 4.0
+    go = np.random.default_rng(92).standard_normal(x.shape)
+    grads = oracle.lora_backward(x, go, idx, w, wgu, wd, *ad_, s)
+    L = lambda xx, aa: (oracle.lora_forward(xx, idx, w, wgu, wd, *aa, s) * go).sum()
+    eps = 1e-6
+    xd = x.astype(np.float64)
+    num = np.zeros_like(xd)
+    for t in range(x.shape[0]):
+        for c in range(0, H, 5):
+            xp, xm = xd.copy(), xd.copy()
+            xp[t, c] += eps
+            xm[t, c] -= eps
+            num[t, c] = (L(xp, ad_) - L(xm, ad_)) / (2 * eps)
+    sel = np.zeros_like(xd, bool)
+    sel[:, 0:H:5] = True
+    np.testing.assert_allclose(grads[0][sel], num[sel], rtol=1e-6, atol=1e-6 * np.abs(num).max())
+    rng = np.random.default_rng(93)
+    for which in range(4):
+        g_an = grads[1 + which]
+        for _ in range(12):
+            pos = tuple(int(rng.integers(0, n)) for n in ad_[which].shape)
+            eps_w = 1e-3   # the adapters are fp32 inputs: perturb by a representable step
+            ap, am = [a.copy() for a in ad_], [a.copy() for a in ad_]
+            ap[which][pos] += eps_w
+            am[which][pos] -= eps_w
+            d = (ap[which][pos] - am[which][pos])   # the exact fp32 step taken
+            num_w = (L(xd, ap) - L(xd, am)) / d
+            assert abs(num_w - g_an[pos]) <= 1e-5 * max(1.0, abs(g_an[pos])), (which, pos, num_w, g_an[pos])
