@@ -96,3 +96,26 @@ def test_host_side_validation(lib):
                                                16, 1 << 40, None)
     assert g(d, 4) == lib.E4B_ERR_INVALID_ARG                          # needs x when saved_gu is NULL
     assert g(d, 0) == lib.E4B_OK
+
+
+def test_pipe_host_side_validation(lib):
+    """The pipelined runner rejects bad arguments before touching the device."""
+    L = lib.lib
+    d = lib.make_desc(8, 256, 512, 2)
+    ex = lib.e4b_experts(16, 16, 16, 16)
+    n = lib.e4b_pipe_arena_size(d, 64)
+    assert n > lib.e4b_moe_workspace_size(d, 64)   # two input/output sets, saved g/u and the workspace
+    assert lib.e4b_pipe_arena_size(lib.make_desc(8, 250, 512, 2), 64) == 0          # invalid desc
+    out = ctypes.c_void_p()
+    create = lambda dd, e, T, arena, nbytes: L.e4b_pipe_create(ctypes.byref(dd), ctypes.byref(e), T, arena, nbytes,
+                                                               None, ctypes.byref(out))
+    assert create(d, ex, 64, None, n) == lib.E4B_ERR_INVALID_ARG                    # no arena
+    assert create(d, ex, 64, 256 + 16, n) == lib.E4B_ERR_INVALID_ARG                # arena not 256-byte aligned
+    assert create(d, ex, -1, 256, n) == lib.E4B_ERR_INVALID_ARG                     # negative T_max
+    assert create(d, ex, 64, 256, n - 1) == lib.E4B_ERR_WORKSPACE                   # arena too small
+    assert create(d, lib.e4b_experts(None, 16, 16, 16), 64, 256, n) == lib.E4B_ERR_INVALID_ARG
+    assert out.value is None
+    assert L.e4b_pipe_submit(None, 4, 16, 16, 16, 16, 16) == lib.E4B_ERR_INVALID_ARG
+    assert L.e4b_pipe_join(None) == lib.E4B_ERR_INVALID_ARG
+    assert L.e4b_pipe_sync(None) == lib.E4B_ERR_INVALID_ARG
+    L.e4b_pipe_destroy(None)   # a no-op
