@@ -1,12 +1,20 @@
 #!/usr/bin/env python
-"""Benchmark of the NF4 Mixture-of-Experts expert layer: forward + input
-gradient (recompute-in-backward) on the OLMoE-1B-7B-shaped layer (E=64, H=2048,
-I=1024, top-8 without renormalisation, T=4096 tokens per GPU), NF4 weights with
-blocksize-64 fp32 absmax, synthetic seeded inputs.
+"""Benchmark of the NF4 Mixture-of-Experts expert layer.
 
-One step = route (softmax/top-k from fp32 logits) + group + grouped gate_up GEMM
-with SwiGLU + grouped down GEMM with the weighted combine + dgrad (two grouped
-GEMMs with the weights re-dequantized in-kernel), all through the C ABI.
+Headline: one training step (forward routed from fp32 logits + the input
+gradient with the weights re-dequantized in-kernel) of the Mixtral-8x7B-shaped
+layer (E=8, H=4096, I=14336, top-2 renormalised, T=16384 tokens per GPU), NF4
+weights with blocksize-64 fp32 absmax, synthetic seeded inputs, through the C
+ABI.  Metric: routed tokens/s of forward + input gradient; the dominant kernel
+and the whole step are reported against the dense-bf16 tensor peak
+(12*H*I FLOP per routed pair for a step).
+
+Secondary legs on the same line: the other large layers (OLMoE T=4096, Qwen3
+prefill T=8192 with Zipf-skewed routing, gpt-oss FP4 T=2048), the small-batch
+decode path (Qwen3 T=1,2,4,8 and gpt-oss T=1: touched weight bytes / time
+against HBM peak), the routing gradient, the gpt-oss expert variant, the
+standalone codec kernels and the NF4-vs-FP4 reconstruction error of the
+gpt-oss-shaped stacks.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl e4b|reference]
 
@@ -29,6 +37,7 @@ sys.path.insert(0, ROOT)
 
 METRIC = "routed tokens/s, NF4 MoE layer fwd+dgrad"
 UNIT = "tokens/s"
+GEMM_FLOPS = {"gemm_gateup": 4, "gemm_down": 2, "gemm_dgrad_down": 2, "gemm_dgrad_gateup": 4}   # x H*I per pair
 
 
 def parse():
@@ -37,14 +46,35 @@ def parse():
     ap.add_argument("--steps", type=int, default=30)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="e4b", choices=["e4b", "reference"])
-    ap.add_argument("--tokens", type=int, default=4096)
+    ap.add_argument("--workload", default="mixtral", choices=["mixtral", "olmoe", "qwen3", "gptoss"],
+                    help="layer of the headline step (default: the Mixtral-shaped layer, the largest config)")
+    ap.add_argument("--tokens", type=int, default=0, help="tokens per GPU (0: the workload's own T)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
-    ap.add_argument("--no-aux", action="store_true", help="skip the decode and quantize/dequantize legs")
+    ap.add_argument("--no-aux", action="store_true", help="skip the secondary legs")
     ap.add_argument("--leg", default="step", choices=["step", "decode", "codec", "variant"],
-                    help="step: the benchmark line; decode / codec / variant: only that secondary leg (for profiling), "
-                         "decode on the Qwen3-shaped layer at --tokens (default 1)")
+                    help="step: the benchmark line; decode / codec / variant: only that secondary leg (for "
+                         "profiling); decode runs the Qwen3-shaped layer at --tokens (default 1)")
     return ap.parse_args()
+
+
+def headline_workload(args):
+    from bit_quantized_mixture_nf4_b200 import workloads as wl
+    w = wl.ALL[args.workload]
+    return w.with_tokens(args.tokens) if args.tokens > 0 else w
+
+
+def workload_desc(w) -> str:
+    rt = "zipf-skewed routing, " if w.router == "zipf" else ""
+    return (f"{w.name}-shaped E={w.E} H={w.H} I={w.I} top{w.k} {'renorm' if w.renorm else 'no-renorm'} T={w.T}/GPU, "
+            f"{'fp4' if w.codebook else 'nf4'} blocksize 64, {rt}fwd (routed from logits, g/u saved) + dgrad")
+
+
+def bench_config(w, world):
+    """The config dict both arms print for the headline workload."""
+    return {"workload": workload_desc(w), "global_batch": w.T * world, "routed_pairs_per_gpu": w.P,
+            "parallelism": f"dp{world} (independent batches)",
+            "l2": "flushed between timed steps (256 MB write)"}
 
 
 def dist_env():
@@ -70,6 +100,22 @@ def max_over_ranks(value: float, device=None) -> float:
 def job_throughput(tokens_per_rank: int, world: int, ms_per_step: float) -> float:
     """Whole-job tokens/s: every rank processes its own batch each step (weak scaling)."""
     return world * tokens_per_rank / (ms_per_step / 1e3)
+
+
+def pct(values, q):
+    """q-th percentile (0..100) by linear interpolation."""
+    v = sorted(values)
+    if not v:
+        return None
+    pos = (len(v) - 1) * q / 100.0
+    lo = int(pos)
+    hi = min(lo + 1, len(v) - 1)
+    return v[lo] + (v[hi] - v[lo]) * (pos - lo)
+
+
+def step_stats(ms):
+    return {"median": statistics.median(ms), "p10": pct(ms, 10), "p90": pct(ms, 90), "mean": sum(ms) / len(ms),
+            "n": len(ms)}
 
 
 def peaks():
@@ -168,16 +214,131 @@ class ClockSampler:
                 "power_w_max": max(s[1] for s in self.samples)}
 
 
+# ------------------------------------------------------------------ GPU layer set-up
+
+class Layer:
+    """One quantized layer on the device with its seeded inputs (drawn on the host,
+    so the CPU oracle can be fed the same values) and output buffers."""
+
+    def __init__(self, w, dev, path=0, act=0, biases=False):
+        import torch
+        import bit_quantized_mixture_nf4_b200 as e4b
+        from bit_quantized_mixture_nf4_b200 import workloads as wl
+        self.w, self.dev = w, dev
+        self.x_h = wl.activations(w)
+        self.logits_h = wl.router_logits(w, self.x_h)
+        self.go_h = wl.grad_output(w)
+        gu, dn = wl.weights(w, device=dev)
+        self.pg, self.ag = e4b.e4b_quantize_nf4(gu, codebook=w.codebook)
+        self.pd, self.ad = e4b.e4b_quantize_nf4(dn, codebook=w.codebook)
+        del gu, dn
+        self.bgu = self.bd = None
+        if biases:
+            g = torch.Generator(device=dev)
+            g.manual_seed(w.seed + 7)
+            self.bgu = torch.randn(w.E, 2 * w.I, device=dev, generator=g) * 0.3
+            self.bd = torch.randn(w.E, w.H, device=dev, generator=g) * 0.3
+        self.experts = e4b.make_experts(self.pg, self.pd, self.ag, self.ad, self.bgu, self.bd)
+        self.desc = e4b.make_desc(w.E, w.H, w.I, w.k, w.renorm, w.codebook, 64, path, act, 1.702, 7.0)
+        T, P = w.T, w.P
+        self.x = self.x_h.to(dev)
+        self.logits = self.logits_h.to(dev)
+        self.go = self.go_h.to(dev)
+        self.idx = torch.empty(T, w.k, dtype=torch.int32, device=dev)
+        self.wts = torch.empty(T, w.k, dtype=torch.float32, device=dev)
+        self.y = torch.empty(T, w.H, dtype=torch.bfloat16, device=dev)
+        self.gx = torch.empty(T, w.H, dtype=torch.bfloat16, device=dev)
+        self.saved = torch.empty(P, 2 * w.I, dtype=torch.bfloat16, device=dev)
+        self.ws = e4b.workspace(self.desc, T, dev)
+        torch.cuda.empty_cache()
+
+    def step(self, stream=None):
+        import bit_quantized_mixture_nf4_b200 as e4b
+        e4b.e4b_moe_forward(self.desc, self.experts, self.x, self.logits, self.idx, self.wts, self.y,
+                            saved_gu=self.saved, ws=self.ws, stream=stream)
+        e4b.e4b_moe_backward_dgrad(self.desc, self.experts, self.x, self.idx, self.wts, self.go,
+                                   saved_gu=self.saved, grad_x=self.gx, ws=self.ws, stream=stream)
+
+
+def timed_steps(layer, steps, warmup, flush, stream, clk=None, kinds=tuple(GEMM_FLOPS)):
+    """Per-step device times (ms) of `steps` fwd+dgrad steps after `warmup` untimed
+    ones, L2 flushed between steps; the grouped GEMMs carry per-launch events."""
+    import torch
+    import bit_quantized_mixture_nf4_b200 as e4b
+    for _ in range(max(warmup, 3)):
+        layer.step(stream)
+    torch.cuda.synchronize()
+    if e4b.e4b_device_status() != e4b.E4B_OK:
+        raise RuntimeError("device status not ok after warm-up")
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    e4b.e4b_timing_reset()
+    torch.cuda.synchronize()
+    n0 = e4b.e4b_launch_count()
+    e4b.e4b_timing_enable_kinds(kinds)
+    for i in range(steps):
+        flush.zero_()                       # evict L2 between timed steps (not timed)
+        starts[i].record(stream)
+        layer.step(stream)
+        ends[i].record(stream)
+        if clk is not None and i % 4 == 3:
+            clk.sample_now()                # the queued steps keep the GPU busy meanwhile
+    torch.cuda.synchronize()
+    e4b.e4b_timing_enable(False)
+    launches = e4b.e4b_launch_count() - n0
+    ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
+    kernels = {}
+    for name in kinds:
+        t, n = e4b.e4b_timing_get(name)
+        if n:
+            kernels[name] = {"launches": n, "avg_ms": t / n}
+    if e4b.e4b_device_status() != e4b.E4B_OK:
+        raise RuntimeError("device status not ok after the timed steps")
+    return ms, kernels, launches
+
+
+def gemm_roofline(w, kernels, bf16, peak_kind):
+    """The dominant grouped GEMM (largest total time) against the dense-bf16 peak."""
+    dom = max((k for k in GEMM_FLOPS if k in kernels), key=lambda k: kernels[k]["avg_ms"] * kernels[k]["launches"])
+    flops = GEMM_FLOPS[dom] * w.H * w.I * w.P
+    achieved = flops / (kernels[dom]["avg_ms"] / 1e3) / 1e12
+    per_kernel = {k: {"avg_ms": v["avg_ms"], "tflops": GEMM_FLOPS[k] * w.H * w.I * w.P / (v["avg_ms"] / 1e3) / 1e12,
+                      "frac": GEMM_FLOPS[k] * w.H * w.I * w.P / (v["avg_ms"] / 1e3) / 1e12 / bf16}
+                  for k, v in kernels.items() if k in GEMM_FLOPS}
+    return {"kernel": dom, "bound": "tensor", "achieved": achieved, "peak": bf16, "unit": "TFLOP/s",
+            "frac": achieved / bf16, "peak_kind": peak_kind, "flops_per_launch": flops,
+            "avg_launch_ms": kernels[dom]["avg_ms"]}, per_kernel
+
+
 # ------------------------------------------------------------------ secondary legs
 
+def step_leg(w, dev, flush, steps=10):
+    """fwd+dgrad of another large layer: tokens/s, whole step and dominant GEMM vs dense bf16."""
+    import torch
+    _, bf16, _, src = peaks()
+    layer = Layer(w, dev)
+    stream = torch.cuda.current_stream()
+    ms, kernels, _ = timed_steps(layer, steps, 3, flush, stream)
+    st = step_stats(ms)
+    roof, per_kernel = gemm_roofline(w, kernels, bf16, f"{src} bf16 dense (burst)")
+    step_tf = 12 * w.H * w.I * w.P / (st["median"] / 1e3) / 1e12
+    del layer
+    torch.cuda.empty_cache()
+    return {"workload": workload_desc(w), "tokens_per_s": w.T / (st["median"] / 1e3), "step_ms": st,
+            "step_roofline": {"bound": "tensor", "achieved": step_tf, "peak": bf16, "unit": "TFLOP/s",
+                              "frac": step_tf / bf16, "flops_per_step": 12 * w.H * w.I * w.P},
+            "roofline": roof, "kernels": per_kernel}
+
+
 def decode_leg(w, dev, reps=20):
-    """Small-batch forward (T <= 8, the weight-streaming GEMV path) on workload w.
+    """Small-batch forward (T <= 8, the weight-streaming decode kernels) on workload w.
 
     Metric: touched weight bytes / forward time, touched = distinct experts the
-    tokens route to x 3*H*I x 0.5625 B.  The layer's packed weights are cycled over
-    enough copies (>= 8 and > 4x the L2 size) that every forward streams its
-    experts from HBM; the forwards over all copies run as one CUDA graph (route +
-    gate_up + down per forward).  Returns a dict for the bench line."""
+    tokens route to x 3*H*I x 0.5625 B.  The layer's packed weights are cycled
+    over enough copies that the TOUCHED bytes of all copies exceed 4x the L2 (and
+    at least 8 copies), so every forward streams its experts from HBM; the
+    forwards over all copies run as one CUDA graph (routing + gate_up + down per
+    forward)."""
     import torch
     import bit_quantized_mixture_nf4_b200 as e4b
     from bit_quantized_mixture_nf4_b200 import workloads as wl
@@ -188,16 +349,19 @@ def decode_leg(w, dev, reps=20):
     pg, ag = e4b.e4b_quantize_nf4(gu, codebook=w.codebook)
     pd, ad = e4b.e4b_quantize_nf4(dn, codebook=w.codebook)
     del gu, dn
-    per_layer = pg.numel() + pd.numel() + 4 * (ag.numel() + ad.numel())
-    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
-    copies = max(8, -(-4 * l2 // per_layer))
-    layers = [(pg, ag, pd, ad)] + [(pg.clone(), ag.clone(), pd.clone(), ad.clone()) for _ in range(copies - 1)]
-    experts = [e4b.make_experts(a, c, b, d) for a, b, c, d in layers]
     desc = e4b.make_desc(w.E, w.H, w.I, w.k, w.renorm, w.codebook, 64, e4b.PATH_DECODE)
     idx = torch.empty(w.T, w.k, dtype=torch.int32, device=dev)
     wts = torch.empty(w.T, w.k, dtype=torch.float32, device=dev)
     y = torch.empty(w.T, w.H, dtype=torch.bfloat16, device=dev)
     ws = e4b.workspace(desc, w.T, dev)
+    e4b.e4b_moe_forward(desc, e4b.make_experts(pg, pd, ag, ad), x, logits, idx, wts, y, ws=ws)
+    torch.cuda.synchronize()
+    touched = int(torch.unique(idx).numel())
+    nbytes = touched * w.weight_bytes_per_expert()
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    copies = max(8, -(-4 * l2 // int(nbytes)))
+    layers = [(pg, ag, pd, ad)] + [(pg.clone(), ag.clone(), pd.clone(), ad.clone()) for _ in range(copies - 1)]
+    experts = [e4b.make_experts(a, c, b, d) for a, b, c, d in layers]
     side = torch.cuda.Stream(dev)
     side.wait_stream(torch.cuda.current_stream(dev))
     with torch.cuda.stream(side):
@@ -213,82 +377,81 @@ def decode_leg(w, dev, reps=20):
     launches_per_fwd = (e4b.e4b_launch_count() - n0) / copies
     graph.replay()
     torch.cuda.synchronize(dev)
-    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    s.record()
+    us = []
     for _ in range(reps):
+        s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s.record()
         graph.replay()
-    e.record()
-    torch.cuda.synchronize(dev)
-    us = s.elapsed_time(e) * 1e3 / (reps * copies)
-    touched = int(torch.unique(idx).numel())
-    nbytes = touched * w.weight_bytes_per_expert()
-    gbs = nbytes / (us * 1e-6) / 1e9
+        e.record()
+        torch.cuda.synchronize(dev)
+        us.append(s.elapsed_time(e) * 1e3 / copies)
+    st = step_stats(us)
+    gbs = nbytes / (st["median"] * 1e-6) / 1e9
     del graph
     if e4b.e4b_device_status() != e4b.E4B_OK:
         raise RuntimeError("device status not ok after the decode leg")
     return {"workload": f"{w.name}-shaped E={w.E} H={w.H} I={w.I} top{w.k} T={w.T} "
-                        f"{'fp4' if w.codebook else 'nf4'}", "us_per_forward": us,
+                        f"{'fp4' if w.codebook else 'nf4'}", "us_per_forward": st,
             "experts_touched": touched, "bytes_per_forward": nbytes, "weight_stream_gbs": gbs,
             "roofline": {"bound": "hbm", "achieved": gbs, "peak": hbm, "unit": "GB/s", "frac": gbs / hbm},
-            "layer_copies": copies, "kernels_per_forward": launches_per_fwd, "timing": "CUDA graph, events"}
+            "layer_copies": copies, "touched_bytes_all_copies": nbytes * copies,
+            "kernels_per_forward": launches_per_fwd, "timing": "CUDA graph over all copies, events, median of reps"}
 
 
-def variant_leg(w, dev, reps=10):
+def variant_leg(w, dev, flush, steps=10):
     """The gpt-oss expert variant (per-expert biases, clamped GLU alpha 1.702 and
-    limit 7) on workload w: forward (routed from logits, derivatives saved) plus
-    input gradient, L2 flushed between steps; tokens/s and the whole step against
-    the dense-bf16 peak (12*H*I FLOP per pair)."""
+    limit 7) on workload w: forward + input gradient, L2 flushed between steps."""
     import torch
     import bit_quantized_mixture_nf4_b200 as e4b
-    from bit_quantized_mixture_nf4_b200 import workloads as wl
-    bf16 = peaks()[1]
-    x = wl.activations(w).to(dev)
-    logits = wl.router_logits(w, wl.activations(w)).to(dev)
-    go = wl.grad_output(w).to(dev)
-    gu, dn = wl.weights(w, device=dev)
-    pg, ag = e4b.e4b_quantize_nf4(gu, codebook=w.codebook)
-    pd, ad = e4b.e4b_quantize_nf4(dn, codebook=w.codebook)
-    del gu, dn
-    g = torch.Generator(device=dev)
-    g.manual_seed(w.seed + 7)
-    bgu = torch.randn(w.E, 2 * w.I, device=dev, generator=g) * 0.3
-    bd = torch.randn(w.E, w.H, device=dev, generator=g) * 0.3
-    experts = e4b.make_experts(pg, pd, ag, ad, bgu, bd)
-    desc = e4b.make_desc(w.E, w.H, w.I, w.k, w.renorm, w.codebook, 64, e4b.PATH_GROUPED, e4b.ACT_CLAMPED_GLU,
-                         1.702, 7.0)
-    P = w.T * w.k
-    idx = torch.empty(w.T, w.k, dtype=torch.int32, device=dev)
-    wts = torch.empty(w.T, w.k, dtype=torch.float32, device=dev)
-    y = torch.empty(w.T, w.H, dtype=torch.bfloat16, device=dev)
-    gx = torch.empty(w.T, w.H, dtype=torch.bfloat16, device=dev)
-    saved = torch.empty(P, 2 * w.I, dtype=torch.bfloat16, device=dev)
-    ws = e4b.workspace(desc, w.T, dev)
-    flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
+    _, bf16, _, src = peaks()
+    layer = Layer(w, dev, path=e4b.PATH_GROUPED, act=e4b.ACT_CLAMPED_GLU, biases=True)
+    ms, kernels, _ = timed_steps(layer, steps, 3, flush, torch.cuda.current_stream())
+    st = step_stats(ms)
+    tf = 12 * w.H * w.I * w.P / (st["median"] / 1e3) / 1e12
+    del layer
+    torch.cuda.empty_cache()
+    return {"workload": workload_desc(w).replace("fwd (", "clamped GLU + per-expert biases, fwd ("),
+            "step_ms": st, "tokens_per_s": w.T / (st["median"] / 1e3),
+            "roofline": {"bound": "tensor", "achieved": tf, "peak": bf16, "unit": "TFLOP/s", "frac": tf / bf16,
+                         "peak_kind": f"{src} bf16 dense (burst)"}}
 
-    def step():
-        e4b.e4b_moe_forward(desc, experts, x, logits, idx, wts, y, saved_gu=saved, ws=ws)
-        e4b.e4b_moe_backward_dgrad(desc, experts, x, idx, wts, go, saved_gu=saved, grad_x=gx, ws=ws)
+
+def router_leg(layer, flush, steps=10):
+    """Routing gradient (weights and logits) on the headline layer and batch."""
+    import torch
+    import bit_quantized_mixture_nf4_b200 as e4b
+    _, bf16, _, src = peaks()
+    w = layer.w
+    dev = layer.dev
+    dwt = torch.empty(w.T, w.k, dtype=torch.float32, device=dev)
+    dlg = torch.empty(w.T, w.E, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def rstep():
+        e4b.e4b_moe_backward_router(layer.desc, layer.experts, layer.x, layer.idx, layer.wts, layer.go,
+                                    router_logits=layer.logits, grad_topk_w=dwt, grad_logits=dlg, ws=layer.ws,
+                                    stream=stream)
 
     for _ in range(3):
-        step()
-    torch.cuda.synchronize(dev)
-    ss = [torch.cuda.Event(enable_timing=True) for _ in range(reps)]
-    ee = [torch.cuda.Event(enable_timing=True) for _ in range(reps)]
-    for i in range(reps):
+        rstep()
+    torch.cuda.synchronize()
+    ms = []
+    for _ in range(steps):
         flush.zero_()
-        ss[i].record()
-        step()
-        ee[i].record()
-    torch.cuda.synchronize(dev)
-    ms = sum(a.elapsed_time(b) for a, b in zip(ss, ee)) / reps
-    if e4b.e4b_device_status() != e4b.E4B_OK:
-        raise RuntimeError("device status not ok after the variant leg")
-    tf = 12 * w.H * w.I * P / (ms / 1e3) / 1e12
-    return {"workload": f"{w.name}-shaped E={w.E} H={w.H} I={w.I} top{w.k} T={w.T} "
-                        f"{'fp4' if w.codebook else 'nf4'}, clamped GLU + per-expert biases, fwd + dgrad",
-            "ms_per_step": ms, "tokens_per_s": w.T / (ms / 1e3),
-            "roofline": {"bound": "tensor", "achieved": tf, "peak": bf16, "unit": "TFLOP/s", "frac": tf / bf16},
-            "l2": "flushed between steps"}
+        s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s.record(stream)
+        rstep()
+        e.record(stream)
+        torch.cuda.synchronize()
+        ms.append(s.elapsed_time(e))
+    st = step_stats(ms)
+    r_flops = 6 * w.H * w.I * w.P
+    tf = r_flops / (st["median"] / 1e3) / 1e12
+    return {"workload": f"same layer and batch as the headline step (T={w.T})", "ms": st,
+            "roofline": {"bound": "tensor", "achieved": tf, "peak": bf16, "unit": "TFLOP/s", "frac": tf / bf16,
+                         "peak_kind": f"{src} bf16 dense (burst)"},
+            "work": "h and the unweighted expert outputs recomputed by the grouped GEMMs (6*H*I FLOP per pair), "
+                    "then one fp32 dot product per pair and the softmax backward per token"}
 
 
 def codec_leg(w, dev, reps=10):
@@ -333,91 +496,193 @@ def codec_leg(w, dev, reps=10):
     return res
 
 
+def reconstruction_leg(w, dev):
+    """NF4 vs FP4 reconstruction error of the same seeded N(0, 0.02) stacks (the
+    gpt-oss-shaped layer): relative RMSE ||w - deq(q(w))|| / ||w|| of the bf16
+    dequantized weights, quantized and dequantized by the library."""
+    import torch
+    import bit_quantized_mixture_nf4_b200 as e4b
+    from bit_quantized_mixture_nf4_b200 import workloads as wl
+    gu, dn = wl.weights(w, device=dev)
+    res = {"workload": f"{w.name}-shaped stacks gate_up [{w.E},{2 * w.I},{w.H}] + down [{w.E},{w.H},{w.I}], "
+                       f"N(0, 0.02)"}
+    for name, cb in (("nf4", e4b.NF4), ("fp4", e4b.FP4)):
+        num = den = 0.0
+        for stack in (gu, dn):
+            p, a = e4b.e4b_quantize_nf4(stack, codebook=cb)
+            d = e4b.e4b_dequantize_nf4(p, a, tuple(stack.shape), codebook=cb, out_dtype=e4b.BF16)
+            num += float((stack - d.float()).double().pow(2).sum())
+            den += float(stack.double().pow(2).sum())
+            del p, a, d
+        res[f"{name}_rel_rmse"] = (num / den) ** 0.5
+    del gu, dn
+    torch.cuda.empty_cache()
+    return res
+
+
 # ------------------------------------------------------------------ CPU oracle
 
-def oracle_step(w, x, logits, go, packed, sample_tokens, dequant_cache):
-    """One oracle pass: route + group all tokens, dequantize the experts (from the
-    packed bytes), forward + input gradient of the sampled tokens.  Returns
-    (seconds for the whole-batch fixed part, seconds for the sampled tokens)."""
-    import numpy as np
-    import oracle
-    t0 = time.perf_counter()
-    idx, wts = oracle.route(logits, w.k, w.renorm)
-    oracle.permute(idx, w.E)
-    pg, ag, pd, ad = packed
-    wgu = oracle.dequantize(pg, ag, (w.E, 2 * w.I, w.H), w.codebook)
-    wd = oracle.dequantize(pd, ad, (w.E, w.H, w.I), w.codebook)
-    t1 = time.perf_counter()
-    toks = np.asarray(sample_tokens, np.int64)
-    oracle.forward(x, idx, wts, wgu, wd, tokens=toks)
-    oracle.dgrad(x, go, idx, wts, wgu, wd, tokens=toks)
-    t2 = time.perf_counter()
-    return t1 - t0, t2 - t1
+class OracleSample:
+    """The CPU oracle on a bounded sample of a workload.
+
+    One step of the oracle = routing and grouping of all T tokens, dequantization
+    of both weight stacks, forward + input gradient of all T tokens.  Routing and
+    grouping run in full; dequantization is timed on a fixed sample of blocks and
+    scaled to the whole stacks; forward + input gradient are timed on S sampled
+    tokens (chosen among the tokens whose experts lie in a subset X whose
+    dequantized weights fit a bounded host budget) and scaled linearly to T."""
+
+    MAX_X_ELEMENTS = 400_000_000
+    DEQ_SAMPLE = 1 << 24
+
+    def __init__(self, w, seed=0):
+        import numpy as np
+        import oracle
+        from bit_quantized_mixture_nf4_b200 import workloads as wl
+        self.w = w
+        self.cores = oracle.num_threads()
+        x = wl.activations(w)
+        self.x = x.float().numpy()
+        self.logits = wl.router_logits(w, x).numpy()
+        self.go = wl.grad_output(w).float().numpy()
+        gu, dn = wl.weights(w)
+        self.pg, self.ag = oracle.quantize(gu.numpy(), w.codebook)
+        self.pd, self.ad = oracle.quantize(dn.numpy(), w.codebook)
+        del gu, dn
+        self.idx, self.wts = oracle.route(self.logits, w.k, w.renorm)
+        per_expert = 3 * w.H * w.I
+        rng = np.random.default_rng(seed)
+        X, toks = set(), []
+        for t in rng.permutation(w.T):
+            ex = set(int(e) for e in self.idx[t])
+            if (len(X | ex)) * per_expert <= max(self.MAX_X_ELEMENTS, w.k * per_expert):
+                X |= ex
+                toks.append(int(t))
+        self.X = np.array(sorted(X), np.int64)
+        self.pool = np.array(toks, np.int64)
+        remap = np.full(w.E, -1, np.int32)
+        remap[self.X] = np.arange(len(self.X), dtype=np.int32)
+        self.sub_idx = remap[self.idx]
+        xs = self.X
+        self.wgu = oracle.dequantize(self.pg[xs], self.ag[xs], (len(xs), 2 * w.I, w.H), w.codebook)
+        self.wd = oracle.dequantize(self.pd[xs], self.ad[xs], (len(xs), w.H, w.I), w.codebook)
+
+    def step(self, S):
+        """Seconds of one extrapolated oracle step; S = sampled tokens."""
+        import numpy as np
+        import oracle
+        w = self.w
+        t0 = time.perf_counter()
+        idx, _ = oracle.route(self.logits, w.k, w.renorm)
+        oracle.permute(idx, w.E)
+        t1 = time.perf_counter()
+        rows = self.deq_rows()
+        oracle.dequantize(self.pg[0][: rows * w.H // 2], self.ag[0][: rows * w.H // 64], (1, rows, w.H), w.codebook)
+        t2 = time.perf_counter()
+        total = w.E * 3 * w.H * w.I
+        toks = self.pool[:min(S, len(self.pool))]
+        oracle.forward(self.x[toks], self.sub_idx[toks], self.wts[toks], self.wgu, self.wd)
+        oracle.dgrad(self.x[toks], self.go[toks], self.sub_idx[toks], self.wts[toks], self.wgu, self.wd)
+        t3 = time.perf_counter()
+        parts = {"route_s": t1 - t0, "deq_s": (t2 - t1) * total / (rows * w.H), "tok_s": t3 - t2,
+                 "sampled_s": t3 - t0}
+        return parts["route_s"] + parts["deq_s"] + parts["tok_s"] * w.T / len(toks), len(toks), parts
+
+    def deq_rows(self):
+        """Rows of expert 0's gate_up stack in the dequantization sample."""
+        return min(self.DEQ_SAMPLE, self.pg.shape[1] * 2) // self.w.H
+
+    def sample_text(self, S):
+        w = self.w
+        return (f"routing + grouping of all {w.T} tokens; dequantization timed on {self.deq_rows() * w.H} elements and "
+                f"scaled to both stacks ({w.E * 3 * w.H * w.I} elements); fwd+dgrad timed on {S} of {w.T} tokens "
+                f"(tokens routed within {len(self.X)} of {w.E} experts) and scaled linearly in tokens")
 
 
-def oracle_inputs(w):
-    import oracle
-    from bit_quantized_mixture_nf4_b200 import workloads as wl
-    x = wl.activations(w)
-    gu, dn = wl.weights(w)
-    logits = wl.router_logits(w, x).numpy()
-    go = wl.grad_output(w).float().numpy()
-    packed = oracle.quantize(gu.numpy(), w.codebook) + oracle.quantize(dn.numpy(), w.codebook)
-    return x.float().numpy(), logits, go, packed
-
-
-def cpu_rate(w, target_s=12.0, inputs=None):
-    """Oracle throughput in routed tokens/s on a bounded sample, scaled to a full batch."""
-    import numpy as np
-    import oracle
-    x, logits, go, packed = inputs if inputs is not None else oracle_inputs(w)
-    nth = oracle.num_threads()
-    rng = np.random.default_rng(0)
-    cal = rng.choice(w.T, size=min(w.T, nth), replace=False)
-    fixed, tcal = oracle_step(w, x, logits, go, packed, cal, None)
-    per_tok = tcal / len(cal)
-    S = int(max(len(cal), min(w.T, (target_s - fixed) / max(per_tok, 1e-9))))
-    S = max(nth, (S // nth) * nth)
-    toks = rng.choice(w.T, size=min(S, w.T), replace=False)
-    fixed, ttok = oracle_step(w, x, logits, go, packed, toks, None)
-    step = fixed + ttok * w.T / len(toks)
-    return w.T / step, dict(cores=nth, sample=f"{len(toks)} of {w.T} tokens (fwd+dgrad), whole-batch routing, "
-                                               f"grouping and dequantization; step time extrapolated linearly in "
-                                               f"tokens", fixed_s=fixed, sample_s=ttok)
+def cpu_rate(w, target_s=15.0):
+    """Oracle throughput in routed tokens/s on a bounded sample (one extrapolated step)."""
+    o = OracleSample(w)
+    _, used, parts = o.step(o.cores)                   # calibration: per-token cost
+    per_tok = parts["tok_s"] / used
+    S = int((target_s - parts["route_s"] - parts["sampled_s"] + parts["tok_s"]) / max(per_tok, 1e-9))
+    S = max(o.cores, min(len(o.pool), (S // o.cores) * o.cores))
+    step, used, _ = o.step(S)
+    return w.T / step, dict(cores=o.cores, sample=o.sample_text(used))
 
 
 def run_reference(args, w):
+    """The reference arm: the CPU oracle as it stands, on the host cores.  Each
+    step runs the bounded sample of OracleSample (8 sampled tokens per core);
+    value = T / the extrapolated full step, ms_per_step = the sampled step's own
+    wall time."""
     world, rank, _ = dist_env()
     if rank != 0:
         return
-    inputs = oracle_inputs(w)
-    import numpy as np
-    import oracle
-    nth = oracle.num_threads()
-    rng = np.random.default_rng(1)
-    S = max(nth, 2 * nth)
-    toks = rng.choice(w.T, size=min(S, w.T), replace=False)
+    o = OracleSample(w, seed=1)
+    S = 8 * o.cores
+    used = S
     for _ in range(args.warmup):
-        oracle_step(w, *inputs, toks, None)
-    steps = []
+        _, used, _ = o.step(S)
+    full, wall = [], []
     for _ in range(args.steps):
-        fixed, ttok = oracle_step(w, *inputs, toks, None)
-        steps.append(fixed + ttok * w.T / len(toks))
-    step = statistics.median(steps)
+        s, used, parts = o.step(S)
+        full.append(s)
+        wall.append(parts["sampled_s"])
+    step = statistics.median(full)
     value = w.T / step
-    sample = (f"{len(toks)} of {w.T} tokens per step (fwd+dgrad), whole-batch routing, grouping and "
-              f"dequantization; step time extrapolated linearly in tokens")
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
-            "steps": args.steps, "warmup": args.warmup, "ms_per_step": step * 1e3, "higher_is_better": True,
-            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": f"olmoe-shaped E={w.E} H={w.H} I={w.I} top{w.k} T={w.T} nf4 fwd+dgrad",
-                       "global_batch": w.T * world, "l2": "n/a (CPU)"},
-            "cpu_baseline": {"value": value, "unit": UNIT, "cores": nth, "kind": "oracle", "sample": sample},
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": statistics.median(wall) * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": bench_config(w, world),
+            "extrapolated_full_step_ms": step_stats([s * 1e3 for s in full]),
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": o.cores, "kind": "oracle",
+                             "sample": o.sample_text(used)},
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
 
 
 # ------------------------------------------------------------------ GPU arm
+
+def e2e_leg(layer, steps, world, stream):
+    """The same step end to end through the C-ABI's pipelined host-buffer runner:
+    every step copies its inputs in from pinned host memory and its y and grad_x
+    out, on copy streams that overlap one batch's copies with the neighbouring
+    batches' kernels.  The L2 is not flushed: the copies stream ~0.5 GB per step."""
+    import torch
+    import bit_quantized_mixture_nf4_b200 as e4b
+    w = layer.w
+    T = w.T
+    x_p = layer.x_h.pin_memory()
+    l_p = layer.logits_h.pin_memory()
+    g_p = layer.go_h.pin_memory()
+    y_p = torch.empty(T, w.H, dtype=torch.bfloat16).pin_memory()
+    gx_p = torch.empty(T, w.H, dtype=torch.bfloat16).pin_memory()
+    pipe = e4b.e4b_pipe_create(layer.desc, layer.experts, T, layer.dev, stream)
+    try:
+        for _ in range(3):
+            e4b.e4b_pipe_submit(pipe, x_p, l_p, g_p, y_p, gx_p)
+        e4b.e4b_pipe_sync(pipe)
+        if world > 1:
+            torch.distributed.barrier()
+        es, ee = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        es.record(stream)
+        e4b.e4b_pipe_join(pipe)          # the pipe's copies start after es
+        for _ in range(steps):
+            e4b.e4b_pipe_submit(pipe, x_p, l_p, g_p, y_p, gx_p)
+        e4b.e4b_pipe_join(pipe)          # ee after the last copy out
+        ee.record(stream)
+        e4b.e4b_pipe_sync(pipe)
+        torch.cuda.synchronize()
+    finally:
+        e4b.e4b_pipe_destroy(pipe)
+    e2e_ms = max_over_ranks(es.elapsed_time(ee) / steps, layer.dev)
+    h2d = x_p.numel() * 2 + l_p.numel() * 4 + g_p.numel() * 2
+    d2h = y_p.numel() * 2 + gx_p.numel() * 2
+    return {"value": job_throughput(T, world, e2e_ms), "unit": UNIT, "h2d_bytes_per_step": h2d,
+            "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms,
+            "api": "e4b_pipe_submit (pinned host buffers; copies of one batch overlap the kernels of the "
+                   "neighbouring batches)"}
+
 
 def run_e4b(args, w):
     import torch
@@ -433,180 +698,61 @@ def run_e4b(args, w):
                                 device_id=torch.device("cuda", local))
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
-
-    # inputs: activations / logits / grad_out drawn on the host (seeded), weights on the device
-    x_h = wl.activations(w)
-    logits_h = wl.router_logits(w, x_h)
-    go_h = wl.grad_output(w)
-    gu, dn = wl.weights(w, device=dev)
-    pg, ag = e4b.e4b_quantize_nf4(gu, codebook=w.codebook)
-    pd, ad = e4b.e4b_quantize_nf4(dn, codebook=w.codebook)
-    del gu, dn
-    torch.cuda.empty_cache()
-    experts = e4b.make_experts(pg, pd, ag, ad)
-    desc = e4b.make_desc(w.E, w.H, w.I, w.k, w.renorm, w.codebook, 64, e4b.PATH_AUTO)
-    T, P = w.T, w.P
-    x = x_h.to(dev)
-    logits = logits_h.to(dev)
-    go = go_h.to(dev)
-    idx = torch.empty(T, w.k, dtype=torch.int32, device=dev)
-    wts = torch.empty(T, w.k, dtype=torch.float32, device=dev)
-    y = torch.empty(T, w.H, dtype=torch.bfloat16, device=dev)
-    gx = torch.empty(T, w.H, dtype=torch.bfloat16, device=dev)
-    saved = torch.empty(P, 2 * w.I, dtype=torch.bfloat16, device=dev)
-    ws = e4b.workspace(desc, T, dev)
+    hbm, bf16_burst, bf16_sus, peak_src = peaks()
     flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)   # > 126 MB L2
     stream = torch.cuda.current_stream()
-
-    def step():
-        e4b.e4b_moe_forward(desc, experts, x, logits, idx, wts, y, saved_gu=saved, ws=ws, stream=stream)
-        e4b.e4b_moe_backward_dgrad(desc, experts, x, idx, wts, go, saved_gu=saved, grad_x=gx, ws=ws, stream=stream)
-
-    for _ in range(max(args.warmup, 3)):
-        step()
-    torch.cuda.synchronize()
-    if e4b.e4b_device_status() != e4b.E4B_OK:
-        raise RuntimeError("device status not ok after warm-up")
+    layer = Layer(w, dev)
 
     # ------------------------------------------------ device-timed region
-    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
-    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
-    e4b.e4b_timing_reset()
     if world > 1:
         torch.distributed.barrier()
     torch.cuda.synchronize()
-    launches0 = e4b.e4b_launch_count()
-    gemm_kinds = ("gemm_gateup", "gemm_down", "gemm_dgrad_down", "gemm_dgrad_gateup")
     with ClockSampler(dev) as clk:
-        # only the grouped GEMMs carry events inside the timed region; the small
-        # kernels between them run back to back (their breakdown is taken below)
-        e4b.e4b_timing_enable_kinds(gemm_kinds)
-        for i in range(args.steps):
-            flush.zero_()                       # evict L2 between timed steps (not timed)
-            starts[i].record(stream)
-            step()
-            ends[i].record(stream)
-            if i % 8 == 7:
-                clk.sample_now()                # the queued steps keep the GPU busy meanwhile
-        torch.cuda.synchronize()
-        e4b.e4b_timing_enable(False)
-    launches = e4b.e4b_launch_count() - launches0
+        step_ms, kernels, launches = timed_steps(layer, args.steps, args.warmup, flush, stream, clk)
     if world > 1:
         torch.distributed.barrier()
-    step_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
     total_ms = max_over_ranks(sum(step_ms), dev)
     ms_per_step = total_ms / args.steps
-    value = job_throughput(T, world, ms_per_step)
-
-    kernels = {}
-    for name in gemm_kinds:
-        ms, n = e4b.e4b_timing_get(name)
-        if n:
-            kernels[name] = {"launches": n, "avg_ms": ms / n}
+    value = job_throughput(w.T, world, ms_per_step)
+    roof, per_kernel = gemm_roofline(w, kernels, bf16_burst, f"{peak_src} bf16 dense (burst)")
+    roof["traffic"] = recorded_traffic(roof["kernel"], f"{w.name}_T{w.T}")
+    step_tf = 12 * w.H * w.I * w.P / (ms_per_step / 1e3) / 1e12
 
     # per-kernel breakdown of the rest of the step: a short separate pass with every
     # kind bracketed by events (which serialises the chained small kernels)
     e4b.e4b_timing_reset()
     e4b.e4b_timing_enable(True)
-    for _ in range(5):
+    for _ in range(3):
         flush.zero_()
-        step()
+        layer.step(stream)
     torch.cuda.synchronize()
     e4b.e4b_timing_enable(False)
     small_kernels = {}
     for name in ("route", "group", "gather", "combine"):
-        ms, n = e4b.e4b_timing_get(name)
+        t, n = e4b.e4b_timing_get(name)
         if n:
-            small_kernels[name] = {"launches": n, "avg_ms": ms / n}
-    flops = {"gemm_gateup": 4, "gemm_down": 2, "gemm_dgrad_down": 2, "gemm_dgrad_gateup": 4}
-    dom = max((k for k in flops if k in kernels), key=lambda k: kernels[k]["avg_ms"] * kernels[k]["launches"])
-    hbm, bf16_burst, bf16_sus, peak_src = peaks()
-    dom_flops = flops[dom] * w.H * w.I * P
-    achieved = dom_flops / (kernels[dom]["avg_ms"] / 1e3) / 1e12
-    wl_name = f"olmoe_T{T}"
-    traffic = recorded_traffic(dom, wl_name)
+            small_kernels[name] = {"launches": n, "avg_ms": t / n}
 
-    # ------------------------------------------------ end-to-end through host buffers
-    # The C-ABI's pipelined host-buffer runner: every step copies its inputs in
-    # from pinned host memory and its y and grad_x out, on copy streams that
-    # overlap one batch's copies with the neighbouring batches' kernels.
-    e2e = None
-    if not args.no_e2e:
-        x_p = x_h.pin_memory()
-        l_p = logits_h.pin_memory()
-        g_p = go_h.pin_memory()
-        y_p = torch.empty(T, w.H, dtype=torch.bfloat16).pin_memory()
-        gx_p = torch.empty(T, w.H, dtype=torch.bfloat16).pin_memory()
-        pipe = e4b.e4b_pipe_create(desc, experts, T, dev, stream)
-        try:
-            for _ in range(3):
-                e4b.e4b_pipe_submit(pipe, x_p, l_p, g_p, y_p, gx_p)
-            e4b.e4b_pipe_sync(pipe)
-            if world > 1:
-                torch.distributed.barrier()
-            es, ee = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            es.record(stream)
-            e4b.e4b_pipe_join(pipe)          # the pipe's copies start after es
-            for _ in range(args.steps):
-                e4b.e4b_pipe_submit(pipe, x_p, l_p, g_p, y_p, gx_p)
-            e4b.e4b_pipe_join(pipe)          # ee after the last copy out
-            ee.record(stream)
-            e4b.e4b_pipe_sync(pipe)
-            torch.cuda.synchronize()
-        finally:
-            e4b.e4b_pipe_destroy(pipe)
-        e2e_ms = max_over_ranks(es.elapsed_time(ee) / args.steps, dev)
-        h2d = x_p.numel() * 2 + l_p.numel() * 4 + g_p.numel() * 2
-        d2h = y_p.numel() * 2 + gx_p.numel() * 2
-        e2e = {"value": job_throughput(T, world, e2e_ms), "unit": UNIT, "h2d_bytes_per_step": h2d,
-               "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms,
-               "api": "e4b_pipe_submit (pinned host buffers; copies of one batch overlap the kernels of the "
-                      "neighbouring batches)"}
+    e2e = None if args.no_e2e else e2e_leg(layer, args.steps, world, stream)
 
-    if e4b.e4b_device_status() != e4b.E4B_OK:
-        raise RuntimeError("device status not ok after the timed region")
-
-    # ------------------------------------------------ routing gradient (the other half of the backward)
     aux = {}
     if not args.no_aux:
-        dwt = torch.empty(T, w.k, dtype=torch.float32, device=dev)
-        dlg = torch.empty(T, w.E, dtype=torch.float32, device=dev)
-
-        def rstep():
-            e4b.e4b_moe_backward_router(desc, experts, x, idx, wts, go, router_logits=logits, grad_topk_w=dwt,
-                                        grad_logits=dlg, ws=ws, stream=stream)
-
-        for _ in range(3):
-            rstep()
-        torch.cuda.synchronize()
-        rs = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
-        re_ = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
-        for i in range(args.steps):
-            flush.zero_()
-            rs[i].record(stream)
-            rstep()
-            re_[i].record(stream)
-        torch.cuda.synchronize()
-        r_ms = sum(a.elapsed_time(b) for a, b in zip(rs, re_)) / args.steps
-        r_flops = 6 * w.H * w.I * P
-        aux["router_backward"] = {
-            "workload": f"same layer and batch as the step (T={T})", "us": r_ms * 1e3,
-            "roofline": {"bound": "tensor", "achieved": r_flops / (r_ms / 1e3) / 1e12, "peak": bf16_burst,
-                         "unit": "TFLOP/s", "frac": r_flops / (r_ms / 1e3) / 1e12 / bf16_burst},
-            "work": "h and the unweighted expert outputs recomputed by the grouped GEMMs (6*H*I FLOP per pair), "
-                    "then one fp32 dot product per pair and the softmax backward per token"}
-        del dwt, dlg
-
-    # ------------------------------------------------ secondary legs (small-batch decode, codec)
+        aux["router_backward"] = router_leg(layer, flush)
+    del layer
+    torch.cuda.empty_cache()
     if not args.no_aux:
-        del saved, ws
-        torch.cuda.empty_cache()
-        aux["decode"] = [decode_leg(v, dev) for v in (wl.QWEN3.with_tokens(1), wl.GPTOSS.with_tokens(1),
-                                                      wl.QWEN3.with_tokens(8))]
+        legs = {}
+        for v in (wl.OLMOE, wl.QWEN3, wl.GPTOSS, wl.MIXTRAL):
+            if v.name != w.name:
+                legs[f"{v.name}_T{v.T}"] = step_leg(v, dev, flush)
+        aux["large_layers"] = legs
+        aux["decode"] = [decode_leg(v, dev) for v in (wl.QWEN3.with_tokens(1), wl.QWEN3.with_tokens(2),
+                                                      wl.QWEN3.with_tokens(4), wl.QWEN3.with_tokens(8),
+                                                      wl.GPTOSS.with_tokens(1))]
         torch.cuda.empty_cache()
         aux["codec"] = codec_leg(wl.OLMOE, dev)
-        torch.cuda.empty_cache()
-        aux["gptoss_variant"] = variant_leg(wl.GPTOSS.with_tokens(2048), dev)
+        aux["reconstruction_nf4_vs_fp4"] = reconstruction_leg(wl.GPTOSS, dev)
+        aux["gptoss_variant"] = variant_leg(wl.GPTOSS.with_tokens(2048), dev, flush)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -618,16 +764,15 @@ def run_e4b(args, w):
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": max(args.warmup, 3), "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-            "config": {"workload": f"olmoe-shaped E={w.E} H={w.H} I={w.I} top{w.k} no-renorm T={T}/GPU, nf4 "
-                                   f"blocksize 64, fwd (routed from logits, g/u saved) + dgrad",
-                       "global_batch": T * world, "parallelism": f"dp{world} (independent batches)",
-                       "l2": "flushed between timed steps (256 MB write)", "routed_pairs_per_gpu": P},
-            "roofline": {"kernel": dom, "bound": "tensor", "achieved": achieved, "peak": bf16_burst,
-                         "unit": "TFLOP/s", "frac": achieved / bf16_burst, "traffic": traffic,
-                         "peak_kind": f"{peak_src} bf16 dense (burst)",
-                         "flops_per_launch": dom_flops, "avg_launch_ms": kernels[dom]["avg_ms"]},
-            "kernels": kernels,
-            "small_kernels": {"timed": "separate 5-step pass, every launch bracketed by events", **small_kernels},
+            "config": bench_config(w, world),
+            "step_ms": step_stats(step_ms),
+            "roofline": roof,
+            "step_roofline": {"bound": "tensor", "achieved": step_tf, "peak": bf16_burst, "unit": "TFLOP/s",
+                              "frac": step_tf / bf16_burst, "flops_per_step": 12 * w.H * w.I * w.P,
+                              "peak_kind": f"{peak_src} bf16 dense (burst)",
+                              "vs_sustained_peak": step_tf / bf16_sus if bf16_sus else None},
+            "kernels": per_kernel,
+            "small_kernels": {"timed": "separate 3-step pass, every launch bracketed by events", **small_kernels},
             "clocks": clk.summary(),
             "gpu_launches": launches,
             "e2e": e2e,
@@ -646,15 +791,17 @@ def main():
     if args.leg != "step":
         import torch
         dev = torch.device("cuda", 0)
+        flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
         if args.leg == "decode":
-            tokens = args.tokens if args.tokens <= 8 else 1
+            tokens = args.tokens if 0 < args.tokens <= 8 else 1
             print(json.dumps(decode_leg(wl.QWEN3.with_tokens(tokens), dev, reps=max(args.steps, 3))), flush=True)
         elif args.leg == "variant":
-            print(json.dumps(variant_leg(wl.GPTOSS.with_tokens(2048), dev, reps=max(args.steps, 3))), flush=True)
+            print(json.dumps(variant_leg(wl.GPTOSS.with_tokens(2048), dev, flush, steps=max(args.steps, 3))),
+                  flush=True)
         else:
             print(json.dumps(codec_leg(wl.OLMOE, dev, reps=max(args.steps, 3))), flush=True)
         return
-    w = wl.OLMOE.with_tokens(args.tokens)
+    w = headline_workload(args)
     if args.impl == "reference":
         run_reference(args, w)
     else:

@@ -95,13 +95,19 @@ __device__ __forceinline__ float key_float(uint32_t k) {
     return __uint_as_float((k & 0x80000000u) ? (k & 0x7fffffffu) : ~k);
 }
 
+struct NoPickHook {
+    __device__ __forceinline__ void operator()(int, int) const {}
+};
+
 // Routing of one token by one warp: top-k on the fp32 logits (descending, ties
 // to the lower expert index; E <= 256), then route_weights_warp.  Each of the k
 // rounds takes the warp-wide maximum key and, among the lanes holding it, the
 // lowest expert index (two redux.sync).  Lane j < k receives the j-th choice in
-// *e_out / *w_out.
+// *e_out / *w_out.  on_pick(expert, j) runs on every lane as soon as round j has
+// picked its expert (the decode kernels start that expert's weight stream there).
+template <typename PickHook = NoPickHook>
 __device__ __forceinline__ void route_token_warp(const float* __restrict__ l, int E, int k, int renorm, int lane,
-                                                 int* e_out, float* w_out) {
+                                                 int* e_out, float* w_out, const PickHook& on_pick = PickHook()) {
     float v[8];
     uint32_t key[8];
     const float NEG_INF = __int_as_float(0xff800000);
@@ -126,6 +132,7 @@ __device__ __forceinline__ void route_token_warp(const float* __restrict__ l, in
         const uint32_t mk = __reduce_max_sync(0xffffffffu, bk);
         const uint32_t win = __reduce_min_sync(0xffffffffu, (bi >= 0 && bk == mk) ? (uint32_t)(lane + 32 * bi) : 0xffffffffu);
         if ((int)(win & 31u) == lane) taken |= 1u << (win >> 5);
+        on_pick((int)win, j);
         const float wv = key_float(mk);
         if (j == 0) top_v = wv;
         if (lane == j) {

@@ -40,6 +40,8 @@
 //               dequantizing warps for the load/store pipeline
 //   warps 7, 9, 13 idle
 // Every mbarrier wait is bounded; on expiry the kernel records a timeout and exits.
+#include <mutex>
+
 #include "e4b_internal.h"
 
 namespace e4b {
@@ -754,6 +756,22 @@ static PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
     return fn;
 }
 
+bool make_tensor_map(CUtensorMap* m, CUtensorMapDataType dt, int rank, const void* base, const uint64_t* dims,
+                     const uint64_t* strides_bytes, const uint32_t* box, CUtensorMapSwizzle sw) {
+    auto fn = encode_fn();
+    if (!fn || rank < 1 || rank > 5) return false;
+    cuuint64_t d[5], s[4];
+    cuuint32_t b[5], e[5];
+    for (int i = 0; i < rank; ++i) {
+        d[i] = dims[i];
+        b[i] = box[i];
+        e[i] = 1;
+        if (i + 1 < rank) s[i] = strides_bytes[i];
+    }
+    return fn(m, dt, rank, const_cast<void*>(base), d, s, b, e, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
+              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 static bool make_map_2d(CUtensorMap* m, CUtensorMapDataType dt, const void* base, uint64_t inner, uint64_t outer,
                         uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer, CUtensorMapSwizzle sw) {
     auto fn = encode_fn();
@@ -775,11 +793,21 @@ static cudaError_t launch_one(const CUtensorMap& ma, const CUtensorMap& mr, cons
                               const CUtensorMap& mg, const GemmParams& p, int grid, cudaStream_t st) {
     using C = Cfg<kCtas, EPI>;
     auto kern = grouped_gemm_kernel<EPI, CB, kCtas, XACT>;
-    static bool attr_set = false;   // per instantiation
-    if (!attr_set) {
-        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
+    // The shared-memory limit is a per-device function attribute: set it once per
+    // device and instantiation, under a lock.
+    {
+        static std::mutex mu;
+        static bool attr_set[64] = {false};
+        int dev = 0;
+        cudaError_t e = cudaGetDevice(&dev);
         if (e != cudaSuccess) return e;
-        attr_set = true;
+        if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+        std::lock_guard<std::mutex> lock(mu);
+        if (!attr_set[dev]) {
+            e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
+            if (e != cudaSuccess) return e;
+            attr_set[dev] = true;
+        }
     }
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(grid);

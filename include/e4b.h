@@ -221,7 +221,12 @@ E4B_API e4b_status e4b_moe_backward_router(const e4b_moe_desc *d, const e4b_expe
  *
  * The first call on a device looks up the array's device address (once per
  * device, with that device current); make that first call before any stream
- * capture.  All calls share the one array and nothing in it needs to start at
+ * capture.  CUDA loads a library's device code lazily, at its first use on a
+ * device, and the 32 MiB array is claimed then, not when the library is loaded:
+ * a caller that reserves the device's free memory for its own pool must make one
+ * call on each device BEFORE reserving it (a call with T = 0 does only this set-up
+ * and launches nothing), or that first call can fail with E4B_ERR_CUDA.
+ * All calls share the one array and nothing in it needs to start at
  * zero (each call writes what it reads), but calls that can overlap on the GPU
  * -- different streams, or host threads without ordering between their calls --
  * race on it and must be serialized by the caller. */
