@@ -794,7 +794,8 @@ def main():
         flush = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev)
         if args.leg == "decode":
             tokens = args.tokens if 0 < args.tokens <= 8 else 1
-            print(json.dumps(decode_leg(wl.QWEN3.with_tokens(tokens), dev, reps=max(args.steps, 3))), flush=True)
+            base = wl.QWEN3 if args.workload == "mixtral" else wl.ALL[args.workload]   # decode: Qwen3 by default
+            print(json.dumps(decode_leg(base.with_tokens(tokens), dev, reps=max(args.steps, 3))), flush=True)
         elif args.leg == "variant":
             print(json.dumps(variant_leg(wl.GPTOSS.with_tokens(2048), dev, flush, steps=max(args.steps, 3))),
                   flush=True)

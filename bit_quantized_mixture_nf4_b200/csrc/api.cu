@@ -97,8 +97,8 @@ uint32_t* device_status_ptr() {
 
 // ------------------------------------------------------------ workspace layout
 struct WsLayout {
-    size_t chunk_counts, chunk_base, counts, offsets, tile_prefix, sched, perm, inv_perm, a_perm, h, gu, dgu, dec_h, dec_plan,
-        ones, total;
+    size_t chunk_counts, chunk_base, counts, offsets, tile_prefix, sched, perm, inv_perm, a_perm, h, gu, dgu, dec, ones,
+        total;
 };
 
 static size_t align_up(size_t v) { return (v + 255) & ~size_t(255); }
@@ -121,8 +121,7 @@ static WsLayout layout_for(const e4b_moe_desc* d, int64_t T) {
     L.h = take((size_t)P * d->I * 2);
     L.gu = take((size_t)P * 2 * d->I * 2);
     L.dgu = take((size_t)P * 2 * d->I * 2);
-    L.dec_h = take((size_t)P * d->I * 2);
-    L.dec_plan = take(decode_plan_bytes());
+    L.dec = take(decode_scratch_bytes(d->E, d->H, d->I, T, d->top_k));
     L.ones = take((size_t)P * 4);
     L.total = off;
     return L;
@@ -308,8 +307,7 @@ e4b_status e4b_moe_forward(const e4b_moe_desc* d, const e4b_experts* w, const vo
     const bool want_grouped_outputs = saved_gu || offsets_out || perm_out;
     // the decode kernels implement SwiGLU without biases
     const bool plain_experts = d->activation == E4B_ACT_SWIGLU && !w->gate_up_bias && !w->down_bias;
-    const bool dec_ok = !want_grouped_outputs && plain_experts &&
-                        decode_supported(d->H, d->I, T, d->top_k, router_logits != nullptr);
+    const bool dec_ok = !want_grouped_outputs && plain_experts && decode_supported(d->E, d->H, d->I, T, d->top_k);
     const bool decode = (d->path == E4B_PATH_DECODE) || (d->path == E4B_PATH_AUTO && dec_ok);
     if (d->path == E4B_PATH_DECODE && !dec_ok) return E4B_ERR_UNSUPPORTED;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
@@ -319,8 +317,7 @@ e4b_status e4b_moe_forward(const e4b_moe_desc* d, const e4b_experts* w, const vo
     if (decode) {   // routing, gate_up and down in two kernels
         E4B_CUDA_TRY(launch_decode_forward(d->codebook, d->E, d->H, d->I, d->top_k, d->renormalize, T,
                                            static_cast<const __nv_bfloat16*>(x), router_logits, topk_idx, topk_w,
-                                           w->gate_up, w->gate_up_absmax, w->down, w->down_absmax,
-                                           reinterpret_cast<__nv_bfloat16*>(ws + L.dec_h), ws + L.dec_plan,
+                                           w->gate_up, w->gate_up_absmax, w->down, w->down_absmax, ws + L.dec,
                                            static_cast<__nv_bfloat16*>(y), st));
         return E4B_OK;
     }

@@ -1,61 +1,55 @@
-// Small-batch (T <= 8) forward.  At a handful of tokens the layer is a
-// weight-streaming GEMV: every touched expert's packed weights are read once,
-// so HBM bandwidth bounds it and tensor-core throughput does not matter.
+// Small-batch (T <= 8) forward.  At a handful of tokens the expert layer is a
+// weight-streaming GEMV: each touched expert's packed weights are read once, so
+// HBM bandwidth bounds it, and at ~20 MB per layer the fixed latencies (routing,
+// the first bytes, the gate_up -> down dependency) weigh as much as the stream.
 //
 // This is the decode fast path of the expert-layer pages ("experts4bit-qlora"
 // 0.4.0 description, section "Inference": single-token forward over the token's
-// top-k experts with no host synchronisation, 4-bit GEMV reading packed NF4
-// directly), designed for B200:
+// top-k experts, a 4-bit GEMV that reads the packed codes directly), designed for
+// B200:
 //
-//  * Two kernels, gate_up and down, chained with programmatic dependent launch
-//    (PDL): each builds its lookup table before it waits on its predecessor.
-//    gate_up routes the <= 8 tokens (one warp per token, in every CTA) and CTA
-//    0 publishes the routing and its grouping for the down kernel.
-//  * Work item = one 8-row weight tile over all of K for one routed expert
-//    (gate_up: 4 gate and 4 up rows; down: 8 output rows).  Each warp owns
-//    whole items and streams them through its own ring of shared-memory
-//    sub-stages (8 blocks of 64 elements of the 8 rows, plus their absmax, and
-//    for down the h rows of the expert's tokens) with a multistage cp.async
-//    pipeline.  A warp accumulates the full K itself: no CTA barrier and no
-//    cross-warp reduction in the main loop, no spin-waits.  The padded sub-stage
-//    rows make the reads bank-conflict free.
-//  * Weight decode: a 256-entry table maps a packed byte (two 4-bit codes) to a
-//    bf16x2 pair of code values.  The table is replicated for each of the 32
-//    lanes, so a warp's 32 lookups hit 32 distinct banks.  The lookup address
-//    takes one byte permute and one shift.
-//  * Math: mma.sync m16n8k16 (bf16 in, fp32 out).  The weight tile is the B
-//    operand (8 rows); the activation rows (the tokens routed to the expert,
-//    <= 8) are the A operand.  Each MMA covers 16 elements of one 64-element
-//    block, so the block's absmax multiplies the fp32 block partial once
-//    (w = code * absmax, code in bf16, scale applied in fp32).
+//  * Two kernels, gate_up then down (a programmatic dependent), one CTA per SM.
+//  * Both kernels route the tokens themselves (one warp per token, from fp32
+//    logits, the routing of the grouped path) and build the same "slots": the
+//    distinct routed experts, ascending.  Every slot is computed for all T tokens
+//    (the MMA's 8 columns); a token's weight for a slot is 0 when it does not
+//    route there, and only routed tokens' h rows are stored and read.
+//  * gate_up: unit = (slot, 8 features) = 8 gate + 8 up rows over all of K = H;
+//    the units are split evenly over the CTAs and round-robin over the 8 warps.
+//    While it streams its own weights it asks L2 for the down weights of the
+//    down CTA with the same index.
+//  * down: CTA c owns whole output tiles (16 rows of H); unit = (tile, slot),
+//    tile-major.  It starts streaming its weights before it waits for gate_up
+//    (only the h rows wait); each warp keeps its own sums per output tile and
+//    the warps' sums are added in warp order, so the result is deterministic and
+//    no CTA waits for another.
+//  * Each warp computes whole units: it streams a unit's 16 rows (codes and
+//    absmax; for down also the h rows) in chunks of KC 64-element blocks from
+//    global memory with 16-byte cp.async into its own ring of shared-memory
+//    stages, lanes running along a row so every copy instruction reads whole
+//    128-byte lines, and computes on the stage copied D-1 chunks earlier.
+//  * Math: mma.sync m16n8k16 (bf16 in, fp32 out) with the WEIGHTS as the A
+//    operand (16 rows) and the <= 8 tokens' activations as B (8 columns): one MMA
+//    covers 256 weights.  K is permuted identically on both operands so a lane
+//    reads 8 contiguous bytes of a row per 64-element block.  Codes become bf16
+//    code values through a 256-entry byte -> bf16x2 table replicated per lane
+//    (conflict-free).  Every MMA starts from zero (no accumulation chain between
+//    MMAs); a block's partial sums are added and scaled by its absmax in fp32.
+#include <mutex>
+
 #include "e4b_internal.h"
 
 namespace e4b {
 
-constexpr int DK_THREADS = 256;
-constexpr int DK_WARPS = DK_THREADS / 32;
-constexpr int DK_MAXP = 64;                 // T * k <= 8 * 8 routed pairs
-constexpr int DK_MAXE = 256;
-constexpr int DK_NS_MAX = 8;                // sub-stages per warp ring
-constexpr int DK_KC = 8;                    // 64-element blocks per sub-stage
-constexpr int DK_DN_MAX_RT = 8;             // down: 8-row tiles per CTA
-constexpr uint32_t DK_LUT_BYTES = 32768;    // 256 byte values x 32 lanes x 4 B
-// sub-stage layout: 8 weight rows of DK_KC*32 bytes padded to 288 (72 words = 8 mod 32:
-// the 4 rows a half-warp reads fall in distinct banks), 8 absmax rows of DK_KC floats
-// padded to 12 words (4 mod 8), then (down) up to 8 activation rows of DK_KC*128
-// bytes padded to 1040 (an odd count of 16-byte units)
-constexpr int DK_SUB_RS = DK_KC * 32 + 32;
-constexpr int DK_SUB_ABS = 8 * DK_SUB_RS;
-constexpr int DK_SUB_ASW = DK_KC + 4;
-constexpr int DK_SUB_A = DK_SUB_ABS + 8 * DK_SUB_ASW * 4;
-constexpr int DK_SUB_AS = DK_KC * 128 + 16;
+constexpr int DV_WARPS = 8;
+constexpr int DV_THREADS = 32 * DV_WARPS;
+constexpr int DV_MAXT = 8, DV_MAXP = 64, DV_MAXS = 64, DV_MAXE = 256;
+constexpr int DV_MAXTL = 8;        // output tiles per down CTA
+constexpr int DV_MAXD = 8;         // ring stages per warp
+constexpr int DV_LUT_WORDS = 256 * 32;   // byte value x lane
+static_assert(DV_MAXE <= DV_THREADS, "one thread per expert in the slot builder");
 
-// e2m1 values (sign in bit 3).  The FP4 codebook is these divided by 6; the
-// division is applied to the fp32 result, so the table is exact in bf16.
-static __constant__ float c_e2m1[16] = {0.0f,  0.5f,  1.0f,  1.5f,  2.0f,  3.0f,  4.0f,  6.0f,
-                                        -0.0f, -0.5f, -1.0f, -1.5f, -2.0f, -3.0f, -4.0f, -6.0f};
-
-struct DecArgs {
+struct DvArgs {
     const __nv_bfloat16* x;   // [T, H]
     const float* logits;      // [T, E] or null (routing given in idx / wts)
     int32_t* idx;             // [T, k]
@@ -65,507 +59,635 @@ struct DecArgs {
     const float* gu_absmax;     // [E, 2I, H/64]
     const uint8_t* d_packed;    // [E, H, I/2]
     const float* d_absmax;      // [E, H, I/64]
-    __nv_bfloat16* h;           // [T*k, I] scratch
-    __nv_bfloat16* y;           // [T, H]
-    struct DecPlan* gplan;      // routing / grouping published by gate_up CTA 0 for the down kernel
-    int xs_off, xs_stride;      // gate_up: staged activations
-    int gu_ring_off, gu_ns;     // gate_up: per-warp rings (offset, sub-stages)
-    int dn_rt;                  // down: 8-row tiles per CTA
-    int dn_yslot_off, dn_ring_off, dn_ns, dn_sub;   // down: y slots, per-warp rings, sub-stage bytes
+    __nv_bfloat16* h;         // [n_slots, T, I] (scratch)
+    __nv_bfloat16* y;         // [T, H]
+    int kc;                   // 64-element blocks per streamed chunk of a unit
+    int depth;                // ring stages per warp
+    int stage_bytes;          // one stage: codes [16][rs] + absmax [16][ss] (+ h [T][hrs])
+    int rs, ss, hrs;          // row strides of a stage (bytes, floats, bytes)
+    int ring_off;             // shared-memory offset of the rings
 };
 
-// Routing and grouping of the <= 64 pairs.  A "slot" is one expert with up to
-// 8 of its pairs (tokens ascending); an expert with more pairs (only possible
-// with caller-given routing that repeats an expert within a token) takes
-// several slots.
-struct __align__(16) DecPlan {
+// The slots: distinct routed experts, ascending, with each token's summed
+// routing weight (0 where the token does not route there).
+struct __align__(16) DvSlots {
     int n_slots;
-    int warp_reps[2];
-    int pe[DK_MAXP];
-    float pw[DK_MAXP];
-    int tslot[DK_MAXP];
-    int rep_rank[DK_MAXP];
-    int slot_e[DK_MAXP];
-    int slot_n[DK_MAXP];
-    int slot_pair[DK_MAXP][8];
-    int slot_tok[DK_MAXP][8];   // token of slot_pair
+    int pad[3];
+    int slot_e[DV_MAXS];
+    unsigned slot_tmask[DV_MAXS];
+    float slot_w[DV_MAXS][DV_MAXT];
 };
 
-constexpr uint32_t DK_PLAN_OFF = DK_LUT_BYTES;
-constexpr uint32_t DK_FIXED = DK_PLAN_OFF + ((sizeof(DecPlan) + 127) / 128) * 128;
+// Dynamic shared memory of both kernels: the slots, the routing pairs and
+// bookkeeping; then
+// (gate_up) the activations or (down) the warps' tile sums; then the warps'
+// rings.
+constexpr int DV_SLOTS_OFF = 0, DV_PAIRS_OFF = 3072, DV_MISC_OFF = 3584;
+constexpr int DV_HDR = 4096;
+static_assert(sizeof(DvSlots) <= DV_PAIRS_OFF, "slots");
+static_assert(DV_PAIRS_OFF + 2 * DV_MAXP * 4 <= DV_MISC_OFF, "pairs");
+struct DvMisc {
+    int warp_cnt[DV_WARPS];   // slot builder: routed experts per warp
+};
+static_assert(sizeof(DvMisc) <= DV_HDR - DV_MISC_OFF, "misc");
 
 __device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 __device__ __forceinline__ void griddep_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;"); }
 
-__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
+__device__ __forceinline__ uint32_t bfe15(uint32_t v) {   // (v >> 1) & 0x7fff
+    uint32_t d;
+    asm("bfe.u32 %0, %1, 1, 15;" : "=r"(d) : "r"(v));
+    return d;
+}
+
+__device__ __forceinline__ void dv_cp16(uint32_t dst, const void* src) {
     asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
 }
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
-// cp.async.wait_group takes an immediate: at most n of this thread's groups pending.
-__device__ __forceinline__ void cp_async_wait_pending(int n) {
-#define DK_WAIT_CASE(N) \
-    case N: asm volatile("cp.async.wait_group " #N ";" ::: "memory"); break;
+__device__ __forceinline__ void dv_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void dv_wait_groups() {
+    asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+// At most n (0 <= n < DV_MAXD) of this thread's copy groups still pending.
+__device__ __forceinline__ void dv_wait_pending(int n) {
     switch (n) {
-        DK_WAIT_CASE(0) DK_WAIT_CASE(1) DK_WAIT_CASE(2) DK_WAIT_CASE(3) DK_WAIT_CASE(4) DK_WAIT_CASE(5)
-        DK_WAIT_CASE(6) DK_WAIT_CASE(7) DK_WAIT_CASE(8) DK_WAIT_CASE(9) DK_WAIT_CASE(10) DK_WAIT_CASE(11)
-        DK_WAIT_CASE(12) DK_WAIT_CASE(13)
-        default: asm volatile("cp.async.wait_group 14;" ::: "memory"); break;
-    }
-#undef DK_WAIT_CASE
-}
-
-template <int CB>
-__device__ __forceinline__ float dec_table(int q) {
-    return CB == 0 ? c_code[0][q] : c_e2m1[q];
-}
-
-// Entry for byte v: bf16x2 {value(high nibble), value(low nibble)} (low half =
-// the element that comes first), stored at v*128 + lane*4 for every lane.
-template <int CB>
-__device__ __forceinline__ void build_lut(uint8_t* lut) {
-    const float cv = dec_table<CB>(threadIdx.x & 15);   // lane q (and q+16) holds code value q
-#pragma unroll
-    for (int k = 0; k < 256 * 8 / DK_THREADS; ++k) {
-        const int i = threadIdx.x + k * DK_THREADS, v = i >> 3, q = i & 7;
-        const float hi = __shfl_sync(0xffffffffu, cv, v >> 4), lo = __shfl_sync(0xffffffffu, cv, v & 15);
-        const uint32_t val = pack_bf16x2(hi, lo);
-        *reinterpret_cast<uint4*>(lut + v * 128 + q * 16) = make_uint4(val, val, val, val);
+        case 0: dv_wait_groups<0>(); break;
+        case 1: dv_wait_groups<1>(); break;
+        case 2: dv_wait_groups<2>(); break;
+        case 3: dv_wait_groups<3>(); break;
+        case 4: dv_wait_groups<4>(); break;
+        case 5: dv_wait_groups<5>(); break;
+        case 6: dv_wait_groups<6>(); break;
+        default: dv_wait_groups<7>(); break;
     }
 }
-
-// One permute builds (byte << 8) | lane*8 (byte 0 <- lane8.byte0, byte 1 <-
-// word.byte[i], bytes 2, 3 <- 0); halved, it is byte*128 + lane*4.
-__device__ __forceinline__ uint32_t lut_lookup(const uint8_t* lut, uint32_t word, uint32_t lane8, uint32_t sel) {
-    return *reinterpret_cast<const uint32_t*>(lut + (prmt(word, lane8, sel) >> 1));
+// Request the 128-byte line at p into L2 (no data returned to the thread).
+__device__ __forceinline__ void dv_prefetch_l2(const void* p) {
+    asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
 }
 
-__device__ __forceinline__ void mma_16816(float d[4], uint32_t a0, uint32_t a2, uint32_t b0, uint32_t b1) {
+// D = A * B with zero accumulator input (every MMA independent of the others).
+__device__ __forceinline__ void mma_16816_z(float d[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                            uint32_t b0, uint32_t b1) {
     asm(
         "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
-        "{%0,%1,%2,%3};"
-        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
-        : "r"(a0), "r"(0u), "r"(a2), "r"(0u), "r"(b0), "r"(b1));
+        "{%10,%10,%10,%10};"
+        : "=f"(d[0]), "=f"(d[1]), "=f"(d[2]), "=f"(d[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1), "f"(0.0f));
 }
 
-// Up to 4 consecutive 64-element blocks of an 8-row weight tile against up to 8
-// activation rows, accumulated as acc += absmax[block] * (block dot product).
-// Lane (g = lane/4, c = lane%4) reads bytes [8c, 8c+8) of each block of weight
-// row g (elements 16c..16c+15) and elements 16c..16c+15 of each block of
-// activation row g (xrow).  Rows g past the slot's tokens may read any valid
-// row: MMA rows are independent and those results are never stored.  MMA m of a block takes elements 16c+4m..16c+4m+3 from every lane:
-// the same permutation of k on both operands, so D[g][n] is the block's dot
-// product; d[0], d[1] = activation row g against weight rows 2c and 2c+1.  The
-// MMAs are issued m-major over the blocks: consecutive MMAs are independent,
-// so their latencies overlap.
-template <int NB>
-__device__ __forceinline__ void mma_batch(const uint8_t* wrow, const uint8_t* xrow, const float* a0, const float* a1,
-                                          uint32_t lane8, const uint8_t* lut, float& acc0, float& acc1) {
-    uint2 w[NB];
-    uint4 xa[NB][2];
-#pragma unroll
-    for (int j = 0; j < NB; ++j) {
-        w[j] = *reinterpret_cast<const uint2*>(wrow + j * 32);
-        xa[j][0] = *reinterpret_cast<const uint4*>(xrow + j * 128);
-        xa[j][1] = *reinterpret_cast<const uint4*>(xrow + j * 128 + 16);
+// Code value q of the codebook (NF4: the NormalFloat values; FP4: the e2m1
+// values, divided by 6 in fp32 after the dot product so they stay exact in bf16).
+template <int CB>
+__device__ __forceinline__ float dv_code(int q) {
+    if (CB == 1) {
+        const float m = (q & 7) < 4 ? 0.5f * (q & 7) : ((q & 7) == 4 ? 2.0f : ((q & 7) == 5 ? 3.0f : ((q & 7) == 6 ? 4.0f : 6.0f)));
+        return (q & 8) ? -m : m;
     }
-    float d[NB][4];
+    float v;
+    switch (q & 15) {
+        case 0: v = -1.0f; break;
+        case 1: v = -0.6961928009986877f; break;
+        case 2: v = -0.5250730514526367f; break;
+        case 3: v = -0.39491748809814453f; break;
+        case 4: v = -0.28444138169288635f; break;
+        case 5: v = -0.18477343022823334f; break;
+        case 6: v = -0.09105003625154495f; break;
+        case 7: v = 0.0f; break;
+        case 8: v = 0.07958029955625534f; break;
+        case 9: v = 0.16093020141124725f; break;
+        case 10: v = 0.24611230194568634f; break;
+        case 11: v = 0.33791524171829224f; break;
+        case 12: v = 0.44070982933044434f; break;
+        case 13: v = 0.5626170039176941f; break;
+        case 14: v = 0.7229568362236023f; break;
+        default: v = 1.0f; break;
+    }
+    return v;
+}
+
+// Table entry of byte v for lane l at word v*32 + l: bf16x2 {value(high nibble),
+// value(low nibble)} (low half = the element that comes first).  The 16 code
+// values go through the small table cv first.  Ends with a block barrier.
+template <int CB>
+__device__ __forceinline__ void dv_build_lut(uint32_t* lut, float* cv) {
+    if (threadIdx.x < 16) cv[threadIdx.x] = dv_code<CB>((int)threadIdx.x);
+    __syncthreads();
+    for (int i = threadIdx.x; i < 256 * 8; i += DV_THREADS) {
+        const int v = i >> 3;
+        const uint32_t val = pack_bf16x2(cv[v >> 4], cv[v & 15]);
+        reinterpret_cast<uint4*>(lut)[i] = make_uint4(val, val, val, val);
+    }
+    __syncthreads();
+}
+
+// Four table lookups for the bytes of w: byte b's entry for this lane sits at
+// byte offset b*128 + lane*4.  One byte permute builds two offsets at once
+// ([lane8, b_i, lane8, b_j], lane8 = lane*8).
+__device__ __forceinline__ void dv_lut4(const uint32_t* lut, uint32_t w, uint32_t lane8, uint32_t& v0, uint32_t& v1,
+                                        uint32_t& v2, uint32_t& v3) {
+    const uint8_t* base = reinterpret_cast<const uint8_t*>(lut);
+    const uint32_t d01 = prmt(w, lane8, 0x1404u);
+    const uint32_t d23 = prmt(w, lane8, 0x3424u);
+    v0 = *reinterpret_cast<const uint32_t*>(base + bfe15(d01));
+    v1 = *reinterpret_cast<const uint32_t*>(base + (d01 >> 17));
+    v2 = *reinterpret_cast<const uint32_t*>(base + bfe15(d23));
+    v3 = *reinterpret_cast<const uint32_t*>(base + (d23 >> 17));
+}
+
+// One 64-element block (column bl of the slot) of the 16 slot rows against the
+// activation fragments of its two halves; h0 / h1: the half is in range.
+// acc += absmax * (block dot products).
+__device__ __forceinline__ void dv_block(const uint8_t* slot, const float* sabs, int rs, int nbs, int bl, bool h0,
+                                         bool h1, uint4 x0, uint4 x1, const uint32_t* lut, uint32_t lane8, int g, int c,
+                                         float acc[4]) {
+    const uint2 wlo = *reinterpret_cast<const uint2*>(slot + g * rs + bl * 32 + c * 8);
+    const uint2 whi = *reinterpret_cast<const uint2*>(slot + (g + 8) * rs + bl * 32 + c * 8);
+    const float alo = sabs[g * nbs + bl], ahi = sabs[(g + 8) * nbs + bl];
+    float s[4] = {0.f, 0.f, 0.f, 0.f};
+    if (h0) {
+        uint32_t l0, l1, l2, l3, m0, m1, m2, m3;
+        dv_lut4(lut, wlo.x, lane8, l0, l1, l2, l3);
+        dv_lut4(lut, whi.x, lane8, m0, m1, m2, m3);
+        float d0[4], d1[4];
+        mma_16816_z(d0, l0, m0, l1, m1, x0.x, x0.y);
+        mma_16816_z(d1, l2, m2, l3, m3, x0.z, x0.w);
 #pragma unroll
-    for (int j = 0; j < NB; ++j) d[j][0] = d[j][1] = d[j][2] = d[j][3] = 0.0f;
+        for (int j = 0; j < 4; ++j) s[j] += d0[j] + d1[j];
+    }
+    if (h1) {
+        uint32_t l0, l1, l2, l3, m0, m1, m2, m3;
+        dv_lut4(lut, wlo.y, lane8, l0, l1, l2, l3);
+        dv_lut4(lut, whi.y, lane8, m0, m1, m2, m3);
+        float d0[4], d1[4];
+        mma_16816_z(d0, l0, m0, l1, m1, x1.x, x1.y);
+        mma_16816_z(d1, l2, m2, l3, m3, x1.z, x1.w);
 #pragma unroll
-    for (int m = 0; m < 4; ++m) {
-        const uint32_t bi = (2 * m) & 3;
-        uint32_t b0[NB], b1[NB];
-#pragma unroll
-        for (int j = 0; j < NB; ++j) {
-            const uint32_t word = (m < 2) ? w[j].x : w[j].y;
-            b0[j] = lut_lookup(lut, word, lane8, 0x5504u | (bi << 4));
-            b1[j] = lut_lookup(lut, word, lane8, 0x5504u | ((bi + 1) << 4));
+        for (int j = 0; j < 4; ++j) s[j] += d0[j] + d1[j];
+    }
+    acc[0] = fmaf(alo, s[0], acc[0]);
+    acc[1] = fmaf(alo, s[1], acc[1]);
+    acc[2] = fmaf(ahi, s[2], acc[2]);
+    acc[3] = fmaf(ahi, s[3], acc[3]);
+}
+
+// First unit of CTA c when U units are split evenly over G CTAs (c * U < 2^31).
+__device__ __forceinline__ int dv_lo(int c, int U, int G) { return c * U / G; }
+
+// Stored row (within the stack) of row r of a unit.  gate_up unit u = (slot,
+// 8 features): rows 0..7 the gate rows, 8..15 the up rows.  down unit u =
+// (tile of 16 output rows, slot), tile-major over S slots.
+__device__ __forceinline__ int64_t dv_gu_row(const DvSlots& sl, int I, int u, int r) {
+    const int FT = I / 8, s = u / FT, f0 = (u - s * FT) * 8;
+    return (int64_t)sl.slot_e[s] * 2 * I + (r < 8 ? f0 + r : I + f0 + r - 8);
+}
+__device__ __forceinline__ int64_t dv_dn_row(const DvSlots& sl, int H, int S, int u, int r) {
+    const int tile = u / S, s = u - tile * S;
+    return (int64_t)sl.slot_e[s] * H + tile * 16 + r;
+}
+
+
+// i / d for 0 <= i < 1024 and 1 <= d <= 64, with inv = ceil(65536 / d).
+__device__ __forceinline__ int dv_div(int i, uint32_t inv) { return (int)(((uint32_t)i * inv) >> 16); }
+__device__ __forceinline__ uint32_t dv_inv(int d) { return (65536u + (uint32_t)d - 1u) / (uint32_t)d; }
+
+// One warp: cp.async copies of blocks [b0, b0 + nb) of a unit's 16 rows into the
+// stage at shared address st: codes (row r at codes + row_of(r) * rb) into
+// [16][rs] and absmax (absmax + row_of(r) * kb) into [16][ss].  Lanes run along
+// a row, so each copy instruction reads whole 128-byte lines.
+template <typename RowFn>
+__device__ __forceinline__ void dv_copy_chunk(uint32_t st, int lane, int b0, int nb, const uint8_t* codes, int rb,
+                                              const float* absmax, int kb, int rs, int ss, RowFn row_of) {
+    const int cpr = 2 * nb;   // 16-byte units per row
+    const uint32_t inv = dv_inv(cpr);
+    for (int i = lane; i < 16 * cpr; i += 32) {
+        const int r = dv_div(i, inv), j = i - r * cpr;
+        dv_cp16(st + r * rs + j * 16, codes + row_of(r) * rb + b0 * 32 + j * 16);
+    }
+    const uint32_t sab = st + 16 * rs;
+    if (((kb | b0 | nb) & 3) == 0) {   // 16-byte aligned absmax runs
+        const int cpa = nb >> 2;
+        const uint32_t inva = dv_inv(cpa);
+        for (int i = lane; i < 16 * cpa; i += 32) {
+            const int r = dv_div(i, inva), j = i - r * cpa;
+            dv_cp16(sab + r * ss * 4 + j * 16, absmax + row_of(r) * kb + b0 + j * 4);
         }
-#pragma unroll
-        for (int j = 0; j < NB; ++j) {
-            const uint32_t x0 = (m < 2) ? (m == 0 ? xa[j][0].x : xa[j][0].z) : (m == 2 ? xa[j][1].x : xa[j][1].z);
-            const uint32_t x1 = (m < 2) ? (m == 0 ? xa[j][0].y : xa[j][0].w) : (m == 2 ? xa[j][1].y : xa[j][1].w);
-            mma_16816(d[j], x0, x1, b0[j], b1[j]);
+    } else {
+        const uint32_t inva = dv_inv(nb);
+        for (int i = lane; i < 16 * nb; i += 32) {
+            const int r = dv_div(i, inva), j = i - r * nb;
+            cp_async_4(sab + (r * ss + j) * 4, absmax + row_of(r) * kb + b0 + j, 4);
         }
     }
-#pragma unroll
-    for (int j = 0; j < NB; ++j) {
-        acc0 = fmaf(a0[j], d[j][0], acc0);
-        acc1 = fmaf(a1[j], d[j][1], acc1);
-    }
 }
 
-// nb (<= 8) consecutive blocks: batches of 4, then the remainder one block at a time.
-__device__ __forceinline__ void mma_blocks(int nb, const uint8_t* wrow, const uint8_t* xrow, const float* a0,
-                                           const float* a1, uint32_t lane8, const uint8_t* lut, float& acc0,
-                                           float& acc1) {
-    int j = 0;
-    for (; j + 4 <= nb; j += 4)
-        mma_batch<4>(wrow + j * 32, xrow + j * 128, a0 + j, a1 + j, lane8, lut, acc0, acc1);
-    for (; j < nb; ++j) mma_batch<1>(wrow + j * 32, xrow + j * 128, a0 + j, a1 + j, lane8, lut, acc0, acc1);
-}
+// Chunk geometry of a kernel: kc blocks of 64 K per chunk (nc chunks per unit),
+// ring of `depth` stages of stage_bytes per warp.
+__device__ __forceinline__ int dv_chunk_blocks(int c, int kc, int kb) { return min(kc, kb - c * kc); }
 
-// Routing (one warp per token, from logits; or the given routing) and the
-// slots.  Inputs are read through L2 (ld.global.cg): the down kernel runs this
-// before its dependency wait.  store: write topk_idx / topk_w.
-__device__ void dec_build_plan(DecPlan& pl, const DecArgs& a, bool store) {
+// -------------------------------------------------------------------- routing
+// The routing and the slots of the T tokens, computed identically by every CTA
+// of both kernels (shared memory only; ends with a block barrier).  From
+// logits: one warp per token (route_token_warp, the routing of the grouped
+// path).  Given routing: the pairs are read from idx / wts.  Slots: the
+// distinct routed experts in ascending order; a token's weight for a slot is
+// the sum of its pairs' weights there, in pair order.
+__device__ __forceinline__ void dv_plan(const DvArgs& a, uint8_t* dsm, bool write_out) {
+    DvSlots& sl = *reinterpret_cast<DvSlots*>(dsm + DV_SLOTS_OFF);
+    int* pe = reinterpret_cast<int*>(dsm + DV_PAIRS_OFF);
+    float* pw = reinterpret_cast<float*>(dsm + DV_PAIRS_OFF + DV_MAXP * 4);
+    DvMisc& misc = *reinterpret_cast<DvMisc*>(dsm + DV_MISC_OFF);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int k = a.k, E = a.E, T = a.T, P = T * k;
+    const int T = a.T, E = a.E, k = a.k, P = T * k;
     if (a.logits) {
         if (warp < T) {
-            const int t = warp;
             int e;
             float p;
-            route_token_warp(a.logits + (int64_t)t * E, E, k, a.renorm, lane, &e, &p);
+            route_token_warp(a.logits + (int64_t)warp * E, E, k, a.renorm, lane, &e, &p);
             if (lane < k) {
-                pl.pe[t * k + lane] = e;
-                pl.pw[t * k + lane] = p;
-                if (store) {
-                    a.idx[t * k + lane] = e;
-                    a.wts[t * k + lane] = p;
+                pe[warp * k + lane] = e;
+                pw[warp * k + lane] = p;
+                if (write_out) {
+                    a.idx[warp * k + lane] = e;
+                    a.wts[warp * k + lane] = p;
                 }
             }
         }
-    } else {
-        for (int p = tid; p < P; p += blockDim.x) {
-            pl.pe[p] = __ldcg(a.idx + p);
-            pl.pw[p] = __ldcg(a.wts + p);
-        }
+    } else if (tid < P) {
+        pe[tid] = __ldcg(a.idx + tid);
+        pw[tid] = __ldcg(a.wts + tid);
     }
     __syncthreads();
-    int e = -1, ts = 0, cnt = 0;
-    bool rep = false;
-    if (tid < P) {
-        e = pl.pe[tid];
-        if (e >= 0 && e < E) {
-            for (int q = 0; q < P; ++q)
-                if (pl.pe[q] == e) {
-                    ts += (q < tid);
-                    ++cnt;
-                }
-            rep = (ts & 7) == 0;
-        } else {
-            e = -1;
-        }
-    }
-    const unsigned bal = __ballot_sync(0xffffffffu, rep);
-    if (lane == 0 && warp < 2) pl.warp_reps[warp] = __popc(bal);
-    int r = __popc(bal & ((1u << lane) - 1u));
-    __syncthreads();
-    if (warp == 1) r += pl.warp_reps[0];
-    if (tid < P) {
-        pl.rep_rank[tid] = rep ? r : -1;
-        pl.tslot[tid] = ts;
-    }
-    if (tid == 0) pl.n_slots = pl.warp_reps[0] + pl.warp_reps[1];
-    __syncthreads();
-    if (tid < P && e >= 0) {
-        int rq = tid;
-        for (int q = 0; q <= tid; ++q)
-            if (pl.pe[q] == e && pl.tslot[q] == (ts & ~7)) {
-                rq = q;
-                break;
+    // thread e marks the tokens routed to expert e
+    const int e = tid;
+    unsigned tm = 0u;
+    if (e < E) {
+        int t = 0, j = 0;
+        for (int p = 0; p < P; ++p) {
+            if (pe[p] == e) tm |= 1u << t;
+            if (++j == k) {
+                j = 0;
+                ++t;
             }
-        const int s = pl.rep_rank[rq];
-        pl.slot_pair[s][ts & 7] = tid;
-        pl.slot_tok[s][ts & 7] = tid / k;
-        if (rep) {
-            pl.slot_e[s] = e;
-            pl.slot_n[s] = min(8, cnt - ts);
         }
+    }
+    const unsigned bal = __ballot_sync(0xffffffffu, tm != 0u);
+    if (lane == 0) misc.warp_cnt[warp] = __popc(bal);
+    __syncthreads();
+    int base = 0;
+    for (int w = 0; w < warp; ++w) base += misc.warp_cnt[w];
+    if (tm) {
+        const int s = base + __popc(bal & ((1u << lane) - 1u));
+        sl.slot_e[s] = e;
+        sl.slot_tmask[s] = tm;
+        for (int t = 0; t < T; ++t) {
+            float wsum = 0.0f;
+            for (int j = 0; j < k; ++j)
+                if (pe[t * k + j] == e) wsum += pw[t * k + j];
+            sl.slot_w[s][t] = wsum;
+        }
+    }
+    if (tid == DV_THREADS - 1) {
+        int n = 0;
+        for (int w = 0; w < DV_WARPS; ++w) n += misc.warp_cnt[w];
+        sl.n_slots = n;
     }
     __syncthreads();
 }
 
-// Copies one sub-stage: blocks [kb0, kb0 + nb) (nb <= DK_KC) of the 8 weight
-// rows grow(0..7) of K elements and their absmax.  Lane l takes row l/4 and
-// every 4th 16-byte chunk of it; absmax goes as 16-byte chunks when aligned,
-// else as 4-byte copies.
-template <typename RowFn>
-__device__ __forceinline__ void copy_sub(uint32_t st, int K, int kb0, int nb, const uint8_t* packed,
-                                         const float* absmax, int lane, RowFn grow) {
-    const int r = lane >> 2, part = lane & 3, kbr = K / 64;
-    const size_t gr = grow(r);
-    const uint8_t* src = packed + gr * (size_t)(K / 2) + kb0 * 32;
-    for (int q = part; q < 2 * nb; q += 4) cp_async16(st + r * DK_SUB_RS + q * 16, src + q * 16);
-    const float* asrc = absmax + gr * (size_t)kbr + kb0;
-    const uint32_t adst = st + DK_SUB_ABS + r * DK_SUB_ASW * 4;
-    if ((kbr & 3) == 0 && (kb0 & 3) == 0 && (nb & 3) == 0) {
-        for (int q = part; q < nb / 4; q += 4) cp_async16(adst + q * 16, asrc + q * 4);
-    } else {
-        for (int q = part; q < nb; q += 4) cp_async_4(adst + q * 4, asrc + q, 4);
+// The compute of one streamed chunk of KC blocks (all of them in range): the
+// unit's 16 rows in the stage against the activation rows at act (row stride
+// ars bytes, token g of the lane).
+template <int KC>
+__device__ __forceinline__ void dv_chunk(const uint8_t* st, const float* sabs, int rs, int ss, const uint8_t* act,
+                                         bool gvalid, const uint32_t* lut, uint32_t lane8, int g, int q4,
+                                         float acc[4]) {
+#pragma unroll
+    for (int bl = 0; bl < KC; ++bl) {
+        const uint4 zero = make_uint4(0u, 0u, 0u, 0u);
+        const uint4 x0 = gvalid ? *reinterpret_cast<const uint4*>(act + bl * 128) : zero;
+        const uint4 x1 = gvalid ? *reinterpret_cast<const uint4*>(act + bl * 128 + 16) : zero;
+        dv_block(st, sabs, rs, ss, bl, true, true, x0, x1, lut, lane8, g, q4, acc);
     }
+}
+// A chunk of nb < KC blocks (the last of a unit whose K is not a multiple of KC).
+__device__ __forceinline__ void dv_chunk_tail(int nb, const uint8_t* st, const float* sabs, int rs, int ss,
+                                              const uint8_t* act, bool gvalid, const uint32_t* lut, uint32_t lane8,
+                                              int g, int q4, float acc[4]) {
+#pragma unroll 1
+    for (int bl = 0; bl < nb; ++bl) {
+        const uint4 zero = make_uint4(0u, 0u, 0u, 0u);
+        const uint4 x0 = gvalid ? *reinterpret_cast<const uint4*>(act + bl * 128) : zero;
+        const uint4 x1 = gvalid ? *reinterpret_cast<const uint4*>(act + bl * 128 + 16) : zero;
+        dv_block(st, sabs, rs, ss, bl, true, true, x0, x1, lut, lane8, g, q4, acc);
+    }
+}
+
+// Code table and zeroed slot records (both kernels, before the wait on the
+// preceding grid: shared memory only).
+template <int CB>
+__device__ __forceinline__ void dv_prologue(uint32_t* lut, float* cv, uint8_t* dsm) {
+    DvSlots& sl = *reinterpret_cast<DvSlots*>(dsm + DV_SLOTS_OFF);
+    const int tid = threadIdx.x;
+    if (tid < DV_MAXS) sl.slot_tmask[tid] = 0u;
+    dv_build_lut<CB>(lut, cv);   // ends with a barrier
 }
 
 // ------------------------------------------------------------------ gate_up
-// h[p, f] = silu(x_t . W_gate,e[f]) * (x_t . W_up,e[f]) for every routed pair
-// p = (t, j).  Item = (slot, 4 features): its 8-row tile holds gate rows
-// f0..f0+3 at tile rows 0, 2, 4, 6 and up rows at 1, 3, 5, 7, so after the MMA
-// each lane holds G and U of one feature for one token.  Items go round-robin
-// to all warps of the grid.
-template <int CB>
-__global__ void __launch_bounds__(DK_THREADS, 2) dec_gateup_kernel(DecArgs a) {
+// h[s, t, f] = silu(x_t . W_gate,e[f]) * (x_t . W_up,e[f]) for every slot s
+// (expert e) and every token t.  Unit = (slot, 8 features): a warp computes a
+// whole unit (all of K = H), streaming it in chunks of KC blocks through its
+// ring.
+template <int CB, int KC>
+__global__ void __launch_bounds__(DV_THREADS, 1) dv_gateup_kernel(DvArgs a) {
+    __shared__ __align__(16) uint32_t lut[DV_LUT_WORDS];
+    __shared__ float cv[16];
     extern __shared__ __align__(128) uint8_t dsm[];
-    DecPlan& pl = *reinterpret_cast<DecPlan*>(dsm + DK_PLAN_OFF);
-    build_lut<CB>(dsm);
-    griddep_wait();
-    dec_build_plan(pl, a, a.logits != nullptr && blockIdx.x == 0);
-    if (blockIdx.x == 0) {   // publish the plan for the down kernel
-        const int* src = reinterpret_cast<const int*>(&pl);
-        int* dst = reinterpret_cast<int*>(a.gplan);
-        for (int i = threadIdx.x; i < (int)(sizeof(DecPlan) / 4); i += DK_THREADS) dst[i] = src[i];
-    }
+    DvSlots& sl = *reinterpret_cast<DvSlots*>(dsm + DV_SLOTS_OFF);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int H = a.H, I = a.I, KB = H / 64, FT = I / 4;
-    // activations of the T tokens
-    const uint32_t xs = smem_u32(dsm + a.xs_off);
-    for (int i = tid; i < a.T * (H / 8); i += DK_THREADS) {
-        const int t = i / (H / 8), q = i - t * (H / 8);
-        cp_async16(xs + t * a.xs_stride + q * 16, a.x + (size_t)t * H + q * 8);
-    }
-    cp_async_wait_all();
-    __syncthreads();
-    griddep_launch_dependents();
+    const int I = a.I, H = a.H, T = a.T, G = gridDim.x;
 
-    const int N = pl.n_slots * FT, W = gridDim.x * DK_WARPS, gw = blockIdx.x * DK_WARPS + warp;
-    const int nsub = (KB + DK_KC - 1) / DK_KC;
-    const int n_items = gw < N ? (N - gw + W - 1) / W : 0;
-    const int total = n_items * nsub;   // this warp's sub-stages
-    const int ns = a.gu_ns;
-    const uint32_t ring = smem_u32(dsm + a.gu_ring_off) + warp * ns * DK_SUB_A;
-    const uint8_t* ring_p = dsm + a.gu_ring_off + warp * ns * DK_SUB_A;
+    dv_prologue<CB>(lut, cv, dsm);
+    griddep_wait();               // everything before this kernel (inputs included) is complete
+    griddep_launch_dependents();  // the down kernel may take the SMs this grid leaves
 
-    // issue cursor: item m, sub-stage sb
-    int im = 0, isb = 0;
-    auto issue = [&]() {
-        const int it = gw + im * W, s = it / FT, f0 = (it - s * FT) * 4;
-        const size_t r0 = (size_t)pl.slot_e[s] * 2 * I + f0;
-        const int kb0 = isb * DK_KC;
-        copy_sub(ring + ((im * nsub + isb) % ns) * DK_SUB_A, H, kb0, min(DK_KC, KB - kb0), a.gu_packed, a.gu_absmax,
-                 lane, [&](int r) { return r0 + (r & 1) * I + (r >> 1); });
-        if (++isb == nsub) {
-            isb = 0;
-            ++im;
+    // activations x [T][H] into shared memory (rows of H*2 + 16 bytes), one copy group
+    uint8_t* xs = dsm + DV_HDR;
+    const int xrs = H * 2 + 16;
+    {
+        const int cpr = H / 8;
+        for (int i = tid; i < T * cpr; i += DV_THREADS) {
+            const int t = i / cpr, j = i - t * cpr;
+            dv_cp16(smem_u32(xs) + t * xrs + j * 16, a.x + (int64_t)t * H + j * 8);
         }
-    };
-    for (int j = 0; j < ns - 1; ++j) {
-        if (j < total) issue();
-        cp_async_commit();
+        dv_commit();
     }
-    const int g = lane >> 2, c = lane & 3;
+    dv_plan(a, dsm, blockIdx.x == 0);
+
+    const int FT = I / 8, KB = H / 64, RB = H / 2, S = sl.n_slots, NC = (KB + KC - 1) / KC;
+    const int U = S * FT;
+    const int u0 = dv_lo(blockIdx.x, U, G), u1 = dv_lo(blockIdx.x + 1, U, G);
+    const int nu = u1 - u0 > warp ? (u1 - u0 - warp + DV_WARPS - 1) / DV_WARPS : 0;   // this warp's units
+    const int L = nu * NC;                                                           // its chunk stream
+    const int D = a.depth;
+    const uint32_t ring = smem_u32(dsm + a.ring_off) + warp * D * a.stage_bytes;
+    int ij = 0, ic = 0;   // issue cursor: unit index j of this warp, chunk c
+    auto issue = [&]() {
+        if (ij < nu) {
+            const int u = u0 + warp + ij * DV_WARPS, s = u / FT, f0 = (u - s * FT) * 8;
+            const int64_t gb = (int64_t)sl.slot_e[s] * 2 * I + f0, ub = gb + I;
+            const int i = ij * NC + ic;
+            dv_copy_chunk(ring + (i % D) * a.stage_bytes, lane, ic * KC, dv_chunk_blocks(ic, KC, KB), a.gu_packed, RB,
+                          a.gu_absmax, KB, a.rs, a.ss, [&](int r) { return r < 8 ? gb + r : ub + r - 8; });
+            if (++ic == NC) {
+                ic = 0;
+                ++ij;
+            }
+        }
+        dv_commit();
+    };
+    for (int i = 0; i < D - 1; ++i) issue();
+    // The weights of the down CTA of this index, requested into L2 while this
+    // grid streams its own: output tiles [t0, t1) of every slot.
+    if (S > 0) {
+        const int NT = H / 16, t0 = dv_lo(blockIdx.x, NT, G), t1 = dv_lo(blockIdx.x + 1, NT, G);
+        const int lcode = 16 * (I / 2) / 128, labs = (16 * (I / 64) * 4 + 127) / 128, lpu = lcode + labs;
+        const int n = (t1 - t0) * S * lpu;
+        for (int i = tid; i < n; i += DV_THREADS) {
+            const int uu = i / lpu, l = i - uu * lpu, tile = t0 + uu / S, s = uu - (uu / S) * S;
+            const int64_t row0 = (int64_t)sl.slot_e[s] * H + tile * 16;
+            if (l < lcode) dv_prefetch_l2(a.d_packed + row0 * (I / 2) + l * 128);
+            else dv_prefetch_l2(reinterpret_cast<const uint8_t*>(a.d_absmax + row0 * (I / 64)) + (l - lcode) * 128);
+        }
+    }
+    dv_wait_pending(D - 1);   // this thread's part of the activations has landed ...
+    __syncthreads();          // ... and everyone's
+
+    const int g = lane >> 2, q4 = lane & 3;
+    const bool gvalid = g < T;
     const uint32_t lane8 = (uint32_t)lane * 8u;
     const float mu = CB == 0 ? 1.0f : (1.0f / 6.0f);
-    float acc0 = 0.0f, acc1 = 0.0f;
-    int s = 0, f0 = 0, sb = 0, m = 0;
-    const uint8_t* xrow = dsm;
-    for (int i = 0; i < total; ++i) {
-        if (sb == 0) {   // new item
-            const int it = gw + m * W;
-            s = it / FT;
-            f0 = (it - s * FT) * 4;
-            xrow = dsm + a.xs_off + pl.slot_tok[s][g < pl.slot_n[s] ? g : 0] * a.xs_stride + c * 32;
-        }
-        cp_async_wait_pending(ns - 2);
-        __syncwarp();   // this warp's copies of sub-stage i landed; sub-stage i-1 consumed by every lane
-        if (i + ns - 1 < total) issue();
-        cp_async_commit();
-        const uint8_t* st = ring_p + (i % ns) * DK_SUB_A;
-        const int kb0 = sb * DK_KC, nb = min(DK_KC, KB - kb0);
-        const uint8_t* wrow = st + g * DK_SUB_RS + c * 8;
-        const float* ag = reinterpret_cast<const float*>(st + DK_SUB_ABS) + (2 * c) * DK_SUB_ASW;
-        const float* au = ag + DK_SUB_ASW;
-        mma_blocks(nb, wrow, xrow + kb0 * 128, ag, au, lane8, dsm, acc0, acc1);
-        if (++sb == nsub) {   // item done: SwiGLU, store h
-            if (g < pl.slot_n[s]) {
-                const float G = acc0 * mu, U = acc1 * mu;
-                const float hv = G / (1.0f + expf(-G)) * U;
-                a.h[(int64_t)pl.slot_pair[s][g] * I + f0 + c] = __float2bfloat16_rn(hv);
+    const uint8_t* xrow = xs + g * xrs + 32 * q4;
+    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+    int cj = 0, cc = 0;   // compute cursor
+    for (int i = 0; i < L; ++i) {
+        __syncwarp();               // every lane is done with the stage chunk i-1 used
+        issue();
+        dv_wait_pending(D - 1);     // this lane's copies of chunk i landed
+        __syncwarp();               // ... and every lane's
+        const uint8_t* st = dsm + a.ring_off + (warp * D + (i % D)) * a.stage_bytes;
+        const float* sabs = reinterpret_cast<const float*>(st + 16 * a.rs);
+        const int nb = dv_chunk_blocks(cc, KC, KB);
+        if (nb == KC) dv_chunk<KC>(st, sabs, a.rs, a.ss, xrow + cc * KC * 128, gvalid, lut, lane8, g, q4, acc);
+        else dv_chunk_tail(nb, st, sabs, a.rs, a.ss, xrow + cc * KC * 128, gvalid, lut, lane8, g, q4, acc);
+        if (++cc == NC) {   // unit done: SwiGLU, store h
+            const int u = u0 + warp + cj * DV_WARPS, s = u / FT, f = (u - s * FT) * 8 + g;
+#pragma unroll
+            for (int jj = 0; jj < 2; ++jj) {
+                const int t = 2 * q4 + jj;
+                if (t < T && ((sl.slot_tmask[s] >> t) & 1u)) {   // h of the tokens routed here
+                    const float gv = acc[jj] * mu, uv = acc[2 + jj] * mu;
+                    const float hv = gv / (1.0f + expf(-gv)) * uv;
+                    a.h[((int64_t)s * T + t) * I + f] = __float2bfloat16_rn(hv);
+                }
             }
-            acc0 = acc1 = 0.0f;
-            sb = 0;
-            ++m;
+            acc[0] = acc[1] = acc[2] = acc[3] = 0.f;
+            cc = 0;
+            ++cj;
         }
     }
-    cp_async_wait_all();
+    dv_wait_groups<0>();
 }
 
 // --------------------------------------------------------------------- down
-// y[t, r] = sum_j w[t,j] * (W_down,e_j[r] . h[t*k+j]), summed over j in slot order.
-// A CTA owns dn_rt 8-row tiles of the output for all routed experts.  Item =
-// (slot, tile); items go round-robin to the CTA's warps, and an item's
-// sub-stages also carry the h rows of the slot's pairs.  Weighted per-pair rows
-// go to shared memory and are summed per token in j order.
-template <int CB>
-__global__ void __launch_bounds__(DK_THREADS, 1) dec_down_kernel(DecArgs a) {
+// y[t, r] = sum over slots s of w[s, t] * (W_down,e_s[r] . h[s, t]).  CTA c owns
+// whole output tiles of 16 rows, [c NT / G, (c+1) NT / G) of NT = H / 16; a unit
+// is (tile, slot), tile-major, and a warp computes whole units (all of K = I).
+// The kernel repeats the routing itself and starts its weight stream before it
+// waits for gate_up; only the h rows wait.
+template <int CB, int KC>
+__global__ void __launch_bounds__(DV_THREADS, 1) dv_down_kernel(DvArgs a) {
+    __shared__ __align__(16) uint32_t lut[DV_LUT_WORDS];
+    __shared__ float cv[16];
     extern __shared__ __align__(128) uint8_t dsm[];
-    DecPlan& pl = *reinterpret_cast<DecPlan*>(dsm + DK_PLAN_OFF);
-    build_lut<CB>(dsm);
-    griddep_launch_dependents();   // the next layer's gate_up may build its table meanwhile
-    griddep_wait();                // routing plan and h come from gate_up
-    {
-        const int* src = reinterpret_cast<const int*>(a.gplan);
-        int* dst = reinterpret_cast<int*>(&pl);
-        for (int i = threadIdx.x; i < (int)(sizeof(DecPlan) / 4); i += DK_THREADS) dst[i] = __ldcg(src + i);
-    }
-    __syncthreads();
-
+    DvSlots& sl = *reinterpret_cast<DvSlots*>(dsm + DV_SLOTS_OFF);
+    float* yw = reinterpret_cast<float*>(dsm + DV_HDR);   // [warp][ntl][16][8] per-warp tile sums
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int H = a.H, I = a.I, KB = I / 64, RW = a.dn_rt * 8;
-    const int r0 = blockIdx.x * RW;
-    const int nt = min(RW, H - r0) / 8;   // 8-row tiles in this CTA
-    float* yslot = reinterpret_cast<float*>(dsm + a.dn_yslot_off);   // [P][RW]
-    const int N = pl.n_slots * nt;
-    const int nsub = (KB + DK_KC - 1) / DK_KC;
-    const int n_items = warp < N ? (N - warp + DK_WARPS - 1) / DK_WARPS : 0;
-    const int total = n_items * nsub;
-    const int ns = a.dn_ns, sub = a.dn_sub;
-    const uint32_t ring = smem_u32(dsm + a.dn_ring_off) + warp * ns * sub;
-    const uint8_t* ring_p = dsm + a.dn_ring_off + warp * ns * sub;
+    const int I = a.I, H = a.H, T = a.T, KBI = I / 64, RB = I / 2, G = gridDim.x;
+    const int NT = H / 16, t0 = dv_lo(blockIdx.x, NT, G), t1 = dv_lo(blockIdx.x + 1, NT, G);
+    const int ntl = (NT + G - 1) / G;   // output tiles per CTA at most
 
-    int im = 0, isb = 0;
-    auto issue = [&]() {
-        const int it = warp + im * DK_WARPS, s = it / nt, t = it - s * nt;
-        const size_t rb = (size_t)pl.slot_e[s] * H + r0 + t * 8;
-        const int kb0 = isb * DK_KC, nb = min(DK_KC, KB - kb0);
-        const uint32_t st = ring + ((im * nsub + isb) % ns) * sub;
-        copy_sub(st, I, kb0, nb, a.d_packed, a.d_absmax, lane, [&](int r) { return rb + r; });
-        const int n = pl.slot_n[s];
-        for (int gg = 0; gg < n; ++gg) {   // h rows of the slot's pairs, these blocks
-            const __nv_bfloat16* hsrc = a.h + (size_t)pl.slot_pair[s][gg] * I + kb0 * 64;
-            for (int q = lane; q < nb * 8; q += 32) cp_async16(st + DK_SUB_A + gg * DK_SUB_AS + q * 16, hsrc + q * 8);
+    for (int i = tid; i < DV_WARPS * ntl * 128; i += DV_THREADS) yw[i] = 0.0f;
+    dv_prologue<CB>(lut, cv, dsm);
+    // This grid starts once every gate_up CTA has passed its own wait, so the
+    // inputs of the layer are complete here; the routing is recomputed.
+    dv_plan(a, dsm, false);
+    const int S = sl.n_slots;
+    const int n = (t1 - t0) * S, u0 = t0 * S;   // this CTA's units [u0, u0 + n)
+    const int NC = (KBI + KC - 1) / KC;
+    const int nu = n > warp ? (n - warp + DV_WARPS - 1) / DV_WARPS : 0;
+    const int L = nu * NC;
+    const int D = a.depth;
+    const uint32_t ring = smem_u32(dsm + a.ring_off) + warp * D * a.stage_bytes;
+    const int h_off = 16 * a.rs + 16 * a.ss * 4;
+    // chunk i of this warp's stream: weights (part & 1) and h rows (part & 2)
+    auto copy = [&](int i, int part) {
+        const int ij = i / NC, ic = i - ij * NC;
+        const int u = u0 + warp + ij * DV_WARPS, s = u % S;
+        const int b0 = ic * KC, nb = dv_chunk_blocks(ic, KC, KBI);
+        const uint32_t st = ring + (i % D) * a.stage_bytes;
+        if (part & 1) {
+            const int64_t rb0 = dv_dn_row(sl, H, S, u, 0);
+            dv_copy_chunk(st, lane, b0, nb, a.d_packed, RB, a.d_absmax, KBI, a.rs, a.ss,
+                          [&](int r) { return rb0 + r; });
         }
-        if (++isb == nsub) {
-            isb = 0;
-            ++im;
+        if (part & 2) {   // the h rows of the tokens routed to this slot (the others stay unread)
+            const int cpr = nb * 8;   // 16-byte units of a token's h row in this chunk
+            const uint32_t inv = dv_inv(cpr);
+            const unsigned tms = sl.slot_tmask[s];
+            const __nv_bfloat16* src = a.h + (int64_t)s * T * I + b0 * 64;
+            for (int q = lane; q < T * cpr; q += 32) {
+                const int t = dv_div(q, inv), j = q - t * cpr;
+                if ((tms >> t) & 1u) dv_cp16(st + h_off + t * a.hrs + j * 16, src + (int64_t)t * I + j * 8);
+            }
         }
     };
-    for (int j = 0; j < ns - 1; ++j) {
-        if (j < total) issue();
-        cp_async_commit();
+    const int npre = min(D - 1, L);
+    for (int i = 0; i < D - 1; ++i) {   // weights of the first chunks: inputs, ready now
+        if (i < npre) copy(i, 1);
+        dv_commit();
     }
-    const int g = lane >> 2, c = lane & 3;
+    griddep_wait();   // gate_up is complete: h is visible
+    griddep_launch_dependents();
+    for (int i = 0; i < D - 1; ++i) {
+        if (i < npre) copy(i, 2);
+        dv_commit();
+    }
+
+    if (S == 0) {   // no valid expert anywhere: y = 0 on this CTA's tiles
+        for (int i = tid; i < (t1 - t0) * 16 * T; i += DV_THREADS) {
+            const int t = i / ((t1 - t0) * 16), r = i - t * (t1 - t0) * 16;
+            a.y[(int64_t)t * H + t0 * 16 + r] = __float2bfloat16_rn(0.0f);
+        }
+        dv_wait_groups<0>();
+        return;
+    }
+    const int g = lane >> 2, q4 = lane & 3;
+    const bool gvalid = g < T;
     const uint32_t lane8 = (uint32_t)lane * 8u;
     const float mu = CB == 0 ? 1.0f : (1.0f / 6.0f);
-    float acc0 = 0.0f, acc1 = 0.0f;
-    int s = 0, t = 0, sb = 0, m = 0, n = 0;
-    for (int i = 0; i < total; ++i) {
-        if (sb == 0) {
-            const int it = warp + m * DK_WARPS;
-            s = it / nt;
-            t = it - s * nt;
-            n = pl.slot_n[s];
-        }
-        cp_async_wait_pending(ns - 2);
+    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+    int cj = 0, cc = 0;
+    for (int i = 0; i < L; ++i) {
         __syncwarp();
-        if (i + ns - 1 < total) issue();
-        cp_async_commit();
-        const uint8_t* st = ring_p + (i % ns) * sub;
-        const int kb0 = sb * DK_KC, nb = min(DK_KC, KB - kb0);
-        const uint8_t* wrow = st + g * DK_SUB_RS + c * 8;
-        const float* a0p = reinterpret_cast<const float*>(st + DK_SUB_ABS) + (2 * c) * DK_SUB_ASW;
-        const float* a1p = a0p + DK_SUB_ASW;
-        const uint8_t* hrow = st + DK_SUB_A + (g < n ? g : 0) * DK_SUB_AS + c * 32;
-        mma_blocks(nb, wrow, hrow, a0p, a1p, lane8, dsm, acc0, acc1);
-        if (++sb == nsub) {   // item done: weight by the routing weight, stash per pair
-            if (g < n) {
-                const int p = pl.slot_pair[s][g];
-                yslot[p * RW + t * 8 + 2 * c] = pl.pw[p] * (acc0 * mu);
-                yslot[p * RW + t * 8 + 2 * c + 1] = pl.pw[p] * (acc1 * mu);
+        if (i + D - 1 < L) copy(i + D - 1, 3);
+        dv_commit();
+        dv_wait_pending(D - 1);
+        __syncwarp();
+        const uint8_t* st = dsm + a.ring_off + (warp * D + (i % D)) * a.stage_bytes;
+        const float* sabs = reinterpret_cast<const float*>(st + 16 * a.rs);
+        const uint8_t* hrow = st + h_off + g * a.hrs + 32 * q4;
+        const int nb = dv_chunk_blocks(cc, KC, KBI);
+        const int su = (u0 + warp + cj * DV_WARPS) % S;
+        const bool hv = gvalid && ((sl.slot_tmask[su] >> g) & 1u);   // token g routed to this slot
+        if (nb == KC) dv_chunk<KC>(st, sabs, a.rs, a.ss, hrow, hv, lut, lane8, g, q4, acc);
+        else dv_chunk_tail(nb, st, sabs, a.rs, a.ss, hrow, hv, lut, lane8, g, q4, acc);
+        if (++cc == NC) {   // unit done: weight by the routing and add into this warp's tile sums
+            const int u = u0 + warp + cj * DV_WARPS, tile = u / S, s = u - tile * S, tl = tile - t0;
+            const unsigned tms = sl.slot_tmask[s];
+            float* yb = yw + (warp * ntl + tl) * 128;
+#pragma unroll
+            for (int jj = 0; jj < 2; ++jj) {
+                const int t = 2 * q4 + jj;
+                if (t < T && ((tms >> t) & 1u)) {
+                    const float wgt = sl.slot_w[s][t] * mu;
+                    yb[g * 8 + t] += wgt * acc[jj];
+                    yb[(g + 8) * 8 + t] += wgt * acc[2 + jj];
+                }
             }
-            acc0 = acc1 = 0.0f;
-            sb = 0;
-            ++m;
+            acc[0] = acc[1] = acc[2] = acc[3] = 0.f;
+            cc = 0;
+            ++cj;
         }
     }
-    cp_async_wait_all();
+    dv_wait_groups<0>();
     __syncthreads();
-    const int rows = nt * 8;
-    for (int i = tid; i < a.T * rows; i += DK_THREADS) {
-        const int tt = i / rows, rl = i - tt * rows;
+    // this CTA's tiles: the warps' sums added in warp order
+    for (int i = tid; i < (t1 - t0) * 16 * T; i += DV_THREADS) {
+        const int tl = i / (16 * T), rem = i - tl * 16 * T, t = rem >> 4, r = rem & 15;
         float v = 0.0f;
-        for (int j = 0; j < a.k; ++j) {
-            const int p = tt * a.k + j;
-            const int e = pl.pe[p];
-            if (e >= 0 && e < a.E) v += yslot[p * RW + rl];
-        }
-        a.y[(int64_t)tt * H + r0 + rl] = __float2bfloat16_rn(v);
+        for (int w = 0; w < DV_WARPS; ++w) v += yw[(w * ntl + tl) * 128 + r * 8 + t];
+        a.y[(int64_t)t * H + (t0 + tl) * 16 + r] = __float2bfloat16_rn(v);
     }
 }
 
 // ------------------------------------------------------------------- host side
 
-static int sm_count() {
-    static int cache[64] = {0};
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
-    if (!cache[dev]) {
-        int n = 0;
-        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
-        cache[dev] = n;
-    }
-    return cache[dev];
-}
-
-static int xs_stride(int H) { return (H * 2 / 16) % 2 ? H * 2 : H * 2 + 16; }
-static int align128(int v) { return (v + 127) / 128 * 128; }
-// h rows per down sub-stage: a slot holds at most T pairs when the routing comes
-// from logits (distinct experts per token), at most 8 with caller-given routing.
-static int down_arows(int64_t T, int k, bool routed) { return routed ? (int)T : (int)std::min<int64_t>(8, T * k); }
-
-struct DecLaunch {
-    int gu_grid, gu_smem, dn_grid, dn_smem;
+struct DvGeom {
+    int kc, depth, stage_bytes, rs, ss, hrs, ring_off, smem;
+};
+struct DvCfg {
+    int G;
+    DvGeom a, b;
 };
 
-// Shared-memory plan of both kernels: gate_up two CTAs per SM (up to 112 KB
-// each) while a 3-deep per-warp ring fits, else one; down one CTA per SM.
-static bool decode_plan_launch(int H, int I, int64_t T, int k, bool routed, DecArgs* a, DecLaunch* l) {
-    if (T < 1 || T > 8 || T * k > DK_MAXP) return false;
-    const int nsm = sm_count();
-    const int sub_g = DK_SUB_A;   // already a multiple of 128
-    const int xs_off = (int)DK_FIXED, xst = xs_stride(H);
-    const int gu_ring = align128(xs_off + (int)T * xst);
-    int gu_ns = std::min(DK_NS_MAX, (112 * 1024 - gu_ring) / (DK_WARPS * sub_g));
-    int gu_grid = 2 * nsm;
-    if (gu_ns < 3) {
-        gu_ns = std::min(DK_NS_MAX, (220 * 1024 - gu_ring) / (DK_WARPS * sub_g));
-        gu_grid = nsm;
+constexpr int DV_SMEM_MAX = 227 * 1024 - DV_LUT_WORDS * 4;   // dynamic shared memory per CTA
+
+// Stage geometry for chunks of kc blocks: code rows of an odd number of 32-byte
+// units keep the warp's 8-byte row reads at two wavefronts; an absmax stride of
+// 4 mod 8 floats and h rows of an odd number of 16-byte units keep those reads
+// conflict-free.  fixed: shared bytes before the rings.
+static bool dv_geom(int K, int hrows, int fixed, DvGeom* g) {
+    const int kb = K / 64;
+    for (int kc = std::min(kb, 8); kc >= 1; kc = kc > 2 ? kc / 2 : kc - 1) {
+        DvGeom t{};
+        t.kc = kc;
+        t.rs = kc * 32 + ((kc & 1) ? 0 : 32);
+        t.ss = 4;
+        while (t.ss < kc || t.ss % 8 != 4) t.ss += 4;
+        t.hrs = kc * 128 + 16;
+        t.stage_bytes = (16 * t.rs + 16 * t.ss * 4 + hrows * t.hrs + 127) / 128 * 128;
+        t.ring_off = (fixed + 127) / 128 * 128;
+        t.depth = std::min(DV_MAXD, (DV_SMEM_MAX - t.ring_off) / (DV_WARPS * t.stage_bytes));
+        if (t.depth >= 3 || (t.depth >= 2 && kc == 1)) {
+            t.smem = t.ring_off + t.depth * DV_WARPS * t.stage_bytes;
+            *g = t;
+            return true;
+        }
     }
-    const int rt = std::max(1, std::min(DK_DN_MAX_RT, (H / 8 + nsm - 1) / nsm));
-    const int yslot_off = (int)DK_FIXED;
-    const int dn_ring = align128(yslot_off + (int)(T * k) * rt * 8 * 4);
-    const int sub_d = align128(DK_SUB_A + down_arows(T, k, routed) * DK_SUB_AS);
-    const int dn_ns = std::min(DK_NS_MAX, (220 * 1024 - dn_ring) / (DK_WARPS * sub_d));
-    if (gu_ns < 2 || dn_ns < 2) return false;
-    if (a) {
-        a->xs_off = xs_off;
-        a->xs_stride = xst;
-        a->gu_ring_off = gu_ring;
-        a->gu_ns = gu_ns;
-        a->dn_rt = rt;
-        a->dn_yslot_off = yslot_off;
-        a->dn_ring_off = dn_ring;
-        a->dn_ns = dn_ns;
-        a->dn_sub = sub_d;
-    }
-    if (l) {
-        l->gu_grid = gu_grid;
-        l->gu_smem = gu_ring + DK_WARPS * gu_ns * sub_g;
-        l->dn_grid = (H / 8 + rt - 1) / rt;
-        l->dn_smem = dn_ring + DK_WARPS * dn_ns * sub_d;
-    }
+    return false;
+}
+
+static bool dv_config(int E, int H, int I, int64_t T, int k, DvCfg* c) {
+    if (T < 1 || T > DV_MAXT || T * k > DV_MAXP || E > DV_MAXE) return false;
+    if (H % 64 || I % 64 || H > 8192) return false;
+    DvCfg d{};
+    d.G = num_sms();
+    if ((H / 16 + d.G - 1) / d.G > DV_MAXTL) return false;   // output tiles per down CTA
+    // gate_up: the activations [T][H*2 + 16] after the header; down: the warps' tile sums
+    if (!dv_geom(H, 0, DV_HDR + (int)T * (H * 2 + 16), &d.a)) return false;
+    const int ntl = (H / 16 + d.G - 1) / d.G;
+    if (!dv_geom(I, (int)T, DV_HDR + DV_WARPS * ntl * 128 * 4, &d.b)) return false;
+    if (c) *c = d;
     return true;
 }
 
-bool decode_supported(int H, int I, int64_t T, int k, bool routed) {
-    return decode_plan_launch(H, I, T, k, routed, nullptr, nullptr);
+bool decode_supported(int E, int H, int I, int64_t T, int k) { return dv_config(E, H, I, T, k, nullptr); }
+
+static size_t al256(size_t v) { return (v + 255) & ~size_t(255); }
+
+// h per (slot, token).
+size_t decode_scratch_bytes(int E, int H, int I, int64_t T, int k) {
+    if (!decode_supported(E, H, I, T, k)) return 0;
+    const int64_t slots = std::min<int64_t>(E, T * k);
+    return al256((size_t)slots * T * I * 2);
 }
 
 template <typename K>
-static cudaError_t launch_pdl(K kernel, int grid, int smem, cudaStream_t st, const DecArgs& a) {
+static cudaError_t dv_launch(K kernel, int grid, int smem, cudaStream_t st, const DvArgs& a) {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(grid);
-    cfg.blockDim = dim3(DK_THREADS);
+    cfg.blockDim = dim3(DV_THREADS);
     cfg.dynamicSmemBytes = (size_t)smem;
     cfg.stream = st;
     cudaLaunchAttribute at[1];
@@ -576,43 +698,89 @@ static cudaError_t launch_pdl(K kernel, int grid, int smem, cudaStream_t st, con
     return cudaLaunchKernelEx(&cfg, kernel, a);
 }
 
-template <int CB>
-static cudaError_t decode_impl(const DecArgs& a, const DecLaunch& l, cudaStream_t st) {
-    cudaError_t err =
-        cudaFuncSetAttribute(dec_gateup_kernel<CB>, cudaFuncAttributeMaxDynamicSharedMemorySize, l.gu_smem);
-    if (err == cudaSuccess)
-        err = cudaFuncSetAttribute(dec_down_kernel<CB>, cudaFuncAttributeMaxDynamicSharedMemorySize, l.dn_smem);
-    // the whole unified L1 / shared array as shared memory, so two gate_up CTAs fit per SM
-    if (err == cudaSuccess)
-        err = cudaFuncSetAttribute(dec_gateup_kernel<CB>, cudaFuncAttributePreferredSharedMemoryCarveout,
-                                   (int)cudaSharedmemCarveoutMaxShared);
-    if (err == cudaSuccess)
-        err = cudaFuncSetAttribute(dec_down_kernel<CB>, cudaFuncAttributePreferredSharedMemoryCarveout,
-                                   (int)cudaSharedmemCarveoutMaxShared);
+// Per-device function attributes: the largest dynamic shared memory any call
+// asked for so far, and the whole unified L1 / shared array as shared memory.
+// kind: one slot per kernel instance.
+constexpr int DV_KINDS = 16;
+template <typename K>
+static cudaError_t dv_attr(K kernel, int smem, int kind) {
+    static std::mutex mu;
+    static int set_bytes[64][DV_KINDS] = {};
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+    std::lock_guard<std::mutex> lock(mu);
+    if (set_bytes[dev][kind] >= smem) return cudaSuccess;
+    e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                 (int)cudaSharedmemCarveoutMaxShared);
+    if (e == cudaSuccess) set_bytes[dev][kind] = smem;
+    return e;
+}
+
+static void dv_apply(DvArgs& a, const DvGeom& g) {
+    a.kc = g.kc;
+    a.depth = g.depth;
+    a.stage_bytes = g.stage_bytes;
+    a.rs = g.rs;
+    a.ss = g.ss;
+    a.hrs = g.hrs;
+    a.ring_off = g.ring_off;
+}
+
+// Kernel instances by chunk size (kc in {1, 2, 4, 8}).
+template <int CB, int KC>
+static cudaError_t dv_launch_gateup(const DvCfg& c, const DvArgs& a, cudaStream_t st) {
+    cudaError_t err = dv_attr(dv_gateup_kernel<CB, KC>, c.a.smem, CB * 8 + (KC == 8 ? 3 : KC == 4 ? 2 : KC - 1));
     if (err != cudaSuccess) return err;
+    return dv_launch(dv_gateup_kernel<CB, KC>, c.G, c.a.smem, st, a);
+}
+template <int CB, int KC>
+static cudaError_t dv_launch_down(const DvCfg& c, const DvArgs& a, cudaStream_t st) {
+    cudaError_t err = dv_attr(dv_down_kernel<CB, KC>, c.b.smem, CB * 8 + 4 + (KC == 8 ? 3 : KC == 4 ? 2 : KC - 1));
+    if (err != cudaSuccess) return err;
+    return dv_launch(dv_down_kernel<CB, KC>, c.G, c.b.smem, st, a);
+}
+
+template <int CB>
+static cudaError_t dv_impl(const DvCfg& c, const DvArgs& a, cudaStream_t st) {
+    DvArgs aa = a;
+    dv_apply(aa, c.a);
     timing_begin(KK_DECODE_GATEUP, st);
-    err = launch_pdl(dec_gateup_kernel<CB>, l.gu_grid, l.gu_smem, st, a);
+    cudaError_t err;
+    switch (c.a.kc) {
+        case 8: err = dv_launch_gateup<CB, 8>(c, aa, st); break;
+        case 4: err = dv_launch_gateup<CB, 4>(c, aa, st); break;
+        case 2: err = dv_launch_gateup<CB, 2>(c, aa, st); break;
+        default: err = dv_launch_gateup<CB, 1>(c, aa, st); break;
+    }
     timing_end(KK_DECODE_GATEUP, st);
     count_launch();
     if (err != cudaSuccess) return err;
+    DvArgs ab = a;
+    dv_apply(ab, c.b);
     timing_begin(KK_DECODE_DOWN, st);
-    err = launch_pdl(dec_down_kernel<CB>, l.dn_grid, l.dn_smem, st, a);
+    switch (c.b.kc) {
+        case 8: err = dv_launch_down<CB, 8>(c, ab, st); break;
+        case 4: err = dv_launch_down<CB, 4>(c, ab, st); break;
+        case 2: err = dv_launch_down<CB, 2>(c, ab, st); break;
+        default: err = dv_launch_down<CB, 1>(c, ab, st); break;
+    }
     timing_end(KK_DECODE_DOWN, st);
     count_launch();
     return err;
 }
 
-size_t decode_plan_bytes() { return sizeof(DecPlan); }
-
 cudaError_t launch_decode_forward(int codebook, int E, int H, int I, int k, int renorm, int64_t T,
                                   const __nv_bfloat16* x, const float* logits, int32_t* idx, float* w,
                                   const uint8_t* gu_packed, const float* gu_absmax, const uint8_t* d_packed,
-                                  const float* d_absmax, __nv_bfloat16* h_scratch, void* plan_scratch,
-                                  __nv_bfloat16* y, cudaStream_t st) {
+                                  const float* d_absmax, void* scratch, __nv_bfloat16* y, cudaStream_t st) {
     if (T == 0) return cudaSuccess;
-    DecArgs a;
-    DecLaunch l;
-    if (E > DK_MAXE || !decode_plan_launch(H, I, T, k, logits != nullptr, &a, &l)) return cudaErrorInvalidValue;
+    DvCfg c;
+    if (!dv_config(E, H, I, T, k, &c)) return cudaErrorInvalidValue;
+    DvArgs a{};
     a.x = x;
     a.logits = logits;
     a.idx = idx;
@@ -627,10 +795,9 @@ cudaError_t launch_decode_forward(int codebook, int E, int H, int I, int k, int 
     a.gu_absmax = gu_absmax;
     a.d_packed = d_packed;
     a.d_absmax = d_absmax;
-    a.h = h_scratch;
-    a.gplan = static_cast<DecPlan*>(plan_scratch);
+    a.h = static_cast<__nv_bfloat16*>(scratch);
     a.y = y;
-    return codebook == 0 ? decode_impl<0>(a, l, st) : decode_impl<1>(a, l, st);
+    return codebook == 0 ? dv_impl<0>(c, a, st) : dv_impl<1>(c, a, st);
 }
 
 }  // namespace e4b

@@ -76,14 +76,19 @@ cudaError_t launch_grouped_gemm(int epi, int codebook, const void* a, int64_t a_
                                 int64_t packed_rows_total, int packed_row_bytes, GemmParams p, int max_m_tiles,
                                 cudaStream_t st);
 
-// decode.cu (T <= 8); decode_supported: the stage rings of both kernels fit in shared memory
-// (routed: the routing comes from logits, so each token's experts are distinct)
-bool decode_supported(int H, int I, int64_t T, int k, bool routed);
-size_t decode_plan_bytes();
+// Tiled TMA descriptor of a rank-`rank` tensor (dims innermost first, strides in bytes of
+// dims 1..rank-1); grouped_gemm.cu.
+bool make_tensor_map(CUtensorMap* m, CUtensorMapDataType dt, int rank, const void* base, const uint64_t* dims,
+                     const uint64_t* strides_bytes, const uint32_t* box, CUtensorMapSwizzle sw);
+
+// decode.cu (T <= 8): the weight-streaming forward.  decode_supported: the shapes the
+// kernels take (H, I multiples of 64, H <= 8192, the stage rings fit in shared memory).
+bool decode_supported(int E, int H, int I, int64_t T, int k);
+// Scratch bytes of the decode path: h per (slot, token) [min(E, T*k), T, I] bf16.
+size_t decode_scratch_bytes(int E, int H, int I, int64_t T, int k);
 cudaError_t launch_decode_forward(int codebook, int E, int H, int I, int k, int renorm, int64_t T,
                                   const __nv_bfloat16* x, const float* logits, int32_t* idx, float* w,
                                   const uint8_t* gu_packed, const float* gu_absmax, const uint8_t* d_packed,
-                                  const float* d_absmax, __nv_bfloat16* h_scratch, void* plan_scratch,
-                                  __nv_bfloat16* y, cudaStream_t st);
+                                  const float* d_absmax, void* scratch, __nv_bfloat16* y, cudaStream_t st);
 
 }  // namespace e4b
