@@ -52,9 +52,10 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-aux", action="store_true", help="skip the secondary legs")
-    ap.add_argument("--leg", default="step", choices=["step", "decode", "codec", "variant"],
-                    help="step: the benchmark line; decode / codec / variant: only that secondary leg (for "
-                         "profiling); decode runs the Qwen3-shaped layer at --tokens (default 1)")
+    ap.add_argument("--leg", default="step", choices=["step", "decode", "codec", "variant", "router"],
+                    help="step: the benchmark line; decode / codec / variant / router: only that secondary leg "
+                         "(for profiling); decode runs the Qwen3-shaped layer (or --workload) at --tokens "
+                         "(default 1); router runs the routing-gradient legs on --workload")
     return ap.parse_args()
 
 
@@ -250,14 +251,31 @@ class Layer:
         self.gx = torch.empty(T, w.H, dtype=torch.bfloat16, device=dev)
         self.saved = torch.empty(P, 2 * w.I, dtype=torch.bfloat16, device=dev)
         self.ws = e4b.workspace(self.desc, T, dev)
+        self.routing = False   # True: the step also takes the routing gradient (fused backward)
+        self.saved_h = self.dwt = self.dlg = None
         torch.cuda.empty_cache()
+
+    def with_routing_gradient(self):
+        """Switch the step to forward (saving h) + the one-pass layer backward with
+        grad_x, grad_topk_w and grad_logits."""
+        import torch
+        w, dev = self.w, self.dev
+        self.saved_h = torch.empty(w.P, w.I, dtype=torch.bfloat16, device=dev)
+        self.dwt = torch.empty(w.T, w.k, dtype=torch.float32, device=dev)
+        self.dlg = torch.empty(w.T, w.E, dtype=torch.float32, device=dev)
+        self.routing = True
 
     def step(self, stream=None):
         import bit_quantized_mixture_nf4_b200 as e4b
         e4b.e4b_moe_forward(self.desc, self.experts, self.x, self.logits, self.idx, self.wts, self.y,
-                            saved_gu=self.saved, ws=self.ws, stream=stream)
-        e4b.e4b_moe_backward_dgrad(self.desc, self.experts, self.x, self.idx, self.wts, self.go,
-                                   saved_gu=self.saved, grad_x=self.gx, ws=self.ws, stream=stream)
+                            saved_gu=self.saved, ws=self.ws, stream=stream, saved_h=self.saved_h)
+        if self.routing:
+            e4b.e4b_moe_backward(self.desc, self.experts, self.x, self.idx, self.wts, self.go, saved_gu=self.saved,
+                                 saved_h=self.saved_h, router_logits=self.logits, grad_x=self.gx,
+                                 grad_topk_w=self.dwt, grad_logits=self.dlg, ws=self.ws, stream=stream)
+        else:
+            e4b.e4b_moe_backward_dgrad(self.desc, self.experts, self.x, self.idx, self.wts, self.go,
+                                       saved_gu=self.saved, grad_x=self.gx, ws=self.ws, stream=stream)
 
 
 def timed_steps(layer, steps, warmup, flush, stream, clk=None, kinds=tuple(GEMM_FLOPS)):
@@ -452,6 +470,38 @@ def router_leg(layer, flush, steps=10):
                          "peak_kind": f"{src} bf16 dense (burst)"},
             "work": "h and the unweighted expert outputs recomputed by the grouped GEMMs (6*H*I FLOP per pair), "
                     "then one fp32 dot product per pair and the softmax backward per token"}
+
+
+def router_fused_leg(layer, flush, steps=10):
+    """The training step with the routing gradient (grad_topk_w and grad_logits)
+    fused into the input gradient, against the same step without it.  The extra
+    work is one dot product per pair over I, fed from the down^T GEMM's
+    accumulator and the saved h, plus the per-token softmax backward; its
+    algorithmic bytes: h read (2I B per pair), the per-tile partials written and
+    read (8 B per pair and 256-column tile), the routing gradient written (4 B per
+    pair), the logits read and their gradient written (8E B per token)."""
+    import torch
+    hbm = peaks()[0]
+    w = layer.w
+    stream = torch.cuda.current_stream()
+    ms0, _, _ = timed_steps(layer, steps, 3, flush, stream, kinds=())
+    layer.with_routing_gradient()
+    ms1, _, _ = timed_steps(layer, steps, 3, flush, stream, kinds=())
+    layer.routing = False
+    s0, s1 = step_stats(ms0), step_stats(ms1)
+    nt = -(-w.I // 256)
+    extra_bytes = w.P * (2 * w.I + 8 * nt + 4) + w.T * 8 * w.E
+    added_ms = s1["median"] - s0["median"]
+    roof = None
+    if added_ms > 0:
+        gbs = extra_bytes / (added_ms / 1e3) / 1e9
+        roof = {"bound": "hbm", "achieved": gbs, "peak": hbm, "unit": "GB/s", "frac": gbs / hbm,
+                "basis": "extra algorithmic bytes / added step time"}
+    return {"workload": f"same layer and batch as the headline step (T={w.T})",
+            "step_ms_without": s0, "step_ms_with": s1, "added_frac": added_ms / s0["median"],
+            "extra_bytes_per_step": extra_bytes, "roofline": roof,
+            "work": "forward saves h; e4b_moe_backward: the down^T GEMM epilogue leaves <grad_out W_d, h> per "
+                    "row and 256-column tile, a per-token kernel sums them and runs the softmax backward"}
 
 
 def codec_leg(w, dev, reps=10):
@@ -738,6 +788,7 @@ def run_e4b(args, w):
     aux = {}
     if not args.no_aux:
         aux["router_backward"] = router_leg(layer, flush)
+        aux["router_fused"] = router_fused_leg(layer, flush)
     del layer
     torch.cuda.empty_cache()
     if not args.no_aux:
@@ -796,6 +847,11 @@ def main():
             tokens = args.tokens if 0 < args.tokens <= 8 else 1
             base = wl.QWEN3 if args.workload == "mixtral" else wl.ALL[args.workload]   # decode: Qwen3 by default
             print(json.dumps(decode_leg(base.with_tokens(tokens), dev, reps=max(args.steps, 3))), flush=True)
+        elif args.leg == "router":
+            w = headline_workload(args)
+            layer = Layer(w, dev)
+            print(json.dumps({"router_fused": router_fused_leg(layer, flush, steps=max(args.steps, 3)),
+                              "router_backward": router_leg(layer, flush, steps=max(args.steps, 3))}), flush=True)
         elif args.leg == "variant":
             print(json.dumps(variant_leg(wl.GPTOSS.with_tokens(2048), dev, flush, steps=max(args.steps, 3))),
                   flush=True)

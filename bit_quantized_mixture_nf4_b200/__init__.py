@@ -25,7 +25,7 @@ PATH_AUTO, PATH_GROUPED, PATH_DECODE = 0, 1, 2
 ACT_SWIGLU, ACT_CLAMPED_GLU = 0, 1
 
 EXPORTS = ("e4b_quantize_nf4", "e4b_dequantize_nf4", "e4b_moe_workspace_size", "e4b_moe_forward",
-           "e4b_moe_backward_dgrad", "e4b_moe_backward_router", "e4b_device_status", "e4b_status_string",
+           "e4b_moe_backward", "e4b_moe_backward_dgrad", "e4b_moe_backward_router", "e4b_device_status", "e4b_status_string",
            "e4b_launch_count", "e4b_timing_enable", "e4b_timing_enable_kinds", "e4b_timing_reset", "e4b_timing_get",
            "e4b_moe_forward_noalloc", "e4b_watchdog_selftest", "e4b_pipe_arena_size", "e4b_pipe_create",
            "e4b_pipe_submit", "e4b_pipe_join", "e4b_pipe_sync", "e4b_pipe_destroy")
@@ -68,7 +68,9 @@ def _load():
     lib.e4b_moe_workspace_size.argtypes = [ctypes.POINTER(e4b_moe_desc), i64]
     lib.e4b_moe_workspace_size.restype = sz
     lib.e4b_moe_forward.argtypes = [ctypes.POINTER(e4b_moe_desc), ctypes.POINTER(e4b_experts), P, i64, P, P, P, P,
-                                    P, P, P, P, sz, P]
+                                    P, P, P, P, P, sz, P]
+    lib.e4b_moe_backward.argtypes = [ctypes.POINTER(e4b_moe_desc), ctypes.POINTER(e4b_experts), P, i64, P, P, P, P,
+                                     P, P, P, P, P, P, sz, P]
     lib.e4b_moe_backward_dgrad.argtypes = [ctypes.POINTER(e4b_moe_desc), ctypes.POINTER(e4b_experts), P, i64, P, P,
                                            P, P, P, P, sz, P]
     lib.e4b_moe_forward_noalloc.argtypes = [ctypes.POINTER(e4b_moe_desc), ctypes.POINTER(e4b_experts), P, i64, P, P,
@@ -96,7 +98,7 @@ def _load():
     lib.e4b_timing_reset.restype = None
     lib.e4b_timing_get.argtypes = [i32, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_uint64)]
     lib.e4b_timing_get.restype = ctypes.c_int
-    for f in ("e4b_quantize_nf4", "e4b_dequantize_nf4", "e4b_moe_forward", "e4b_moe_backward_dgrad",
+    for f in ("e4b_quantize_nf4", "e4b_dequantize_nf4", "e4b_moe_forward", "e4b_moe_backward", "e4b_moe_backward_dgrad",
               "e4b_device_status", "e4b_moe_forward_noalloc", "e4b_moe_backward_router", "e4b_watchdog_selftest"):
         getattr(lib, f).restype = ctypes.c_int
     _lib = lib
@@ -231,7 +233,8 @@ def workspace(desc: e4b_moe_desc, T: int, device="cuda") -> torch.Tensor:
 
 
 def e4b_moe_forward(desc: e4b_moe_desc, experts: e4b_experts, x: torch.Tensor, router_logits=None, topk_idx=None,
-                    topk_w=None, y=None, saved_gu=None, offsets_out=None, perm_out=None, ws=None, stream=None):
+                    topk_w=None, y=None, saved_gu=None, offsets_out=None, perm_out=None, ws=None, stream=None,
+                    saved_h=None):
     """Expert-layer forward.  With router_logits the layer routes and fills
     topk_idx / topk_w (allocated here when not given); without, they are inputs.
     Returns (y, topk_idx, topk_w)."""
@@ -250,8 +253,36 @@ def e4b_moe_forward(desc: e4b_moe_desc, experts: e4b_experts, x: torch.Tensor, r
         ws = workspace(desc, T, dev)
     _check("e4b_moe_forward", _load().e4b_moe_forward(
         ctypes.byref(desc), ctypes.byref(experts), _ptr(x), T, _ptr(router_logits), _ptr(topk_idx), _ptr(topk_w),
-        _ptr(y), _ptr(saved_gu), _ptr(offsets_out), _ptr(perm_out), _ptr(ws), ws.numel(), _stream(stream)))
+        _ptr(y), _ptr(saved_gu), _ptr(saved_h), _ptr(offsets_out), _ptr(perm_out), _ptr(ws), ws.numel(),
+        _stream(stream)))
     return y, topk_idx, topk_w
+
+
+def e4b_moe_backward(desc: e4b_moe_desc, experts: e4b_experts, x, topk_idx, topk_w, grad_out, saved_gu=None,
+                     saved_h=None, router_logits=None, grad_x=None, grad_topk_w=None, grad_logits=None,
+                     want_grad_x=True, want_routing=True, ws=None, stream=None):
+    """The layer backward in one pass: (grad_x bf16 [T, H] or None, grad_topk_w fp32
+    [T, k] or None, grad_logits fp32 [T, E] or None).  The routing-weight gradient
+    is fused into the input gradient's down^T GEMM; with saved_gu it needs
+    saved_h (both from e4b_moe_forward), without them x is used to recompute."""
+    _cuda(grad_out, "grad_out", torch.bfloat16)
+    T = grad_out.shape[0]
+    dev = grad_out.device
+    if grad_x is None and want_grad_x:
+        grad_x = torch.empty(T, desc.H, dtype=torch.bfloat16, device=dev)
+    if grad_topk_w is None and want_routing:
+        grad_topk_w = torch.empty(T, desc.top_k, dtype=torch.float32, device=dev)
+    if router_logits is not None:
+        _cuda(router_logits, "router_logits", torch.float32)
+        if grad_logits is None and want_routing:
+            grad_logits = torch.empty(T, desc.E, dtype=torch.float32, device=dev)
+    if ws is None:
+        ws = workspace(desc, T, dev)
+    _check("e4b_moe_backward", _load().e4b_moe_backward(
+        ctypes.byref(desc), ctypes.byref(experts), _ptr(x), T, _ptr(router_logits), _ptr(topk_idx), _ptr(topk_w),
+        _ptr(grad_out), _ptr(saved_gu), _ptr(saved_h), _ptr(grad_x), _ptr(grad_topk_w), _ptr(grad_logits), _ptr(ws),
+        ws.numel(), _stream(stream)))
+    return grad_x, grad_topk_w, grad_logits
 
 
 def e4b_moe_backward_dgrad(desc: e4b_moe_desc, experts: e4b_experts, x, topk_idx, topk_w, grad_out, saved_gu=None,

@@ -98,10 +98,14 @@ uint32_t* device_status_ptr() {
 // ------------------------------------------------------------ workspace layout
 struct WsLayout {
     size_t chunk_counts, chunk_base, counts, offsets, tile_prefix, sched, perm, inv_perm, a_perm, h, gu, dgu, dec, ones,
-        total;
+        dw_part, total;
 };
 
 static size_t align_up(size_t v) { return (v + 255) & ~size_t(255); }
+
+// n-tiles of the input-gradient down^T GEMM (N = I): the per-row dot products of
+// the fused routing-weight gradient come one per n-tile.
+static int dw_tiles(const e4b_moe_desc* d) { return (d->I + 255) / 256; }
 
 static WsLayout layout_for(const e4b_moe_desc* d, int64_t T) {
     WsLayout L{};
@@ -123,6 +127,7 @@ static WsLayout layout_for(const e4b_moe_desc* d, int64_t T) {
     L.dgu = take((size_t)P * 2 * d->I * 2);
     L.dec = take(decode_scratch_bytes(d->E, d->H, d->I, T, d->top_k));
     L.ones = take((size_t)P * 4);
+    L.dw_part = take((size_t)P * dw_tiles(d) * 4);
     L.total = off;
     return L;
 }
@@ -294,7 +299,7 @@ size_t e4b_moe_workspace_size(const e4b_moe_desc* d, int64_t T) {
 
 e4b_status e4b_moe_forward(const e4b_moe_desc* d, const e4b_experts* w, const void* x, int64_t T,
                            const float* router_logits, int32_t* topk_idx, float* topk_w, void* y, void* saved_gu,
-                           int32_t* offsets_out, int32_t* perm_out, void* workspace, size_t ws_bytes,
+                           void* saved_h, int32_t* offsets_out, int32_t* perm_out, void* workspace, size_t ws_bytes,
                            void* stream) {
     e4b_status s = check_desc(d);
     if (s != E4B_OK) return s;
@@ -304,7 +309,7 @@ e4b_status e4b_moe_forward(const e4b_moe_desc* d, const e4b_experts* w, const vo
     if (!x || !topk_idx || !topk_w || !y) return E4B_ERR_INVALID_ARG;
     const WsLayout L = layout_for(d, T);
     if (!workspace || ws_bytes < L.total) return E4B_ERR_WORKSPACE;
-    const bool want_grouped_outputs = saved_gu || offsets_out || perm_out;
+    const bool want_grouped_outputs = saved_gu || saved_h || offsets_out || perm_out;
     // the decode kernels implement SwiGLU without biases
     const bool plain_experts = d->activation == E4B_ACT_SWIGLU && !w->gate_up_bias && !w->down_bias;
     const bool dec_ok = !want_grouped_outputs && plain_experts && decode_supported(d->E, d->H, d->I, T, d->top_k);
@@ -333,7 +338,8 @@ e4b_status e4b_moe_forward(const e4b_moe_desc* d, const e4b_experts* w, const vo
                               st));
     E4B_CUDA_TRY(launch_gather_rows(static_cast<const __nv_bfloat16*>(x), perm, offsets + d->E, d->top_k, P, d->H,
                                     reinterpret_cast<__nv_bfloat16*>(ws + L.a_perm), st));
-    __nv_bfloat16* h = reinterpret_cast<__nv_bfloat16*>(ws + L.h);
+    // h goes straight to the caller's saved_h when asked for (the down GEMM reads it there)
+    __nv_bfloat16* h = saved_h ? static_cast<__nv_bfloat16*>(saved_h) : reinterpret_cast<__nv_bfloat16*>(ws + L.h);
     __nv_bfloat16* slots = reinterpret_cast<__nv_bfloat16*>(ws + L.a_perm);   // X_perm is dead after gate_up
     if ((s = run_gateup(d, w, ws, L, topk_w, P, h, static_cast<__nv_bfloat16*>(saved_gu), st)) != E4B_OK) return s;
 
@@ -357,22 +363,26 @@ e4b_status e4b_moe_forward(const e4b_moe_desc* d, const e4b_experts* w, const vo
     return E4B_OK;
 }
 
-e4b_status e4b_moe_backward_dgrad(const e4b_moe_desc* d, const e4b_experts* w, const void* x, int64_t T,
-                                  const int32_t* topk_idx, const float* topk_w, const void* grad_out,
-                                  const void* saved_gu, void* grad_x, void* workspace, size_t ws_bytes,
-                                  void* stream) {
+e4b_status e4b_moe_backward(const e4b_moe_desc* d, const e4b_experts* w, const void* x, int64_t T,
+                            const float* router_logits, const int32_t* topk_idx, const float* topk_w,
+                            const void* grad_out, const void* saved_gu, const void* saved_h, void* grad_x,
+                            float* grad_topk_w, float* grad_logits, void* workspace, size_t ws_bytes, void* stream) {
     e4b_status s = check_desc(d);
     if (s != E4B_OK) return s;
     if ((s = check_experts(w)) != E4B_OK) return s;
     if (T < 0 || T * d->top_k > (int64_t)INT32_MAX) return E4B_ERR_INVALID_ARG;
     if (T == 0) return E4B_OK;
-    if (!topk_idx || !topk_w || !grad_out || !grad_x || (!saved_gu && !x)) return E4B_ERR_INVALID_ARG;
+    if (!topk_idx || !topk_w || !grad_out || (!grad_x && !grad_topk_w)) return E4B_ERR_INVALID_ARG;
+    if (!saved_gu && !x) return E4B_ERR_INVALID_ARG;                 // nothing to recompute from
+    if (grad_topk_w && saved_gu && !saved_h) return E4B_ERR_INVALID_ARG;   // h saved with the derivatives
+    if (grad_logits && (!router_logits || !grad_topk_w)) return E4B_ERR_INVALID_ARG;
     const WsLayout L = layout_for(d, T);
     if (!workspace || ws_bytes < L.total) return E4B_ERR_WORKSPACE;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     uint8_t* ws = static_cast<uint8_t*>(workspace);
     const int64_t P = T * d->top_k;
     int32_t* perm = reinterpret_cast<int32_t*>(ws + L.perm);
+    const int32_t* inv_perm = reinterpret_cast<const int32_t*>(ws + L.inv_perm);
     E4B_CUDA_TRY(launch_group(topk_idx, P, d->E, gemm_tile_rows(), reinterpret_cast<int32_t*>(ws + L.chunk_counts),
                               reinterpret_cast<int32_t*>(ws + L.chunk_base), reinterpret_cast<int32_t*>(ws + L.counts),
                               reinterpret_cast<int32_t*>(ws + L.offsets), reinterpret_cast<int32_t*>(ws + L.tile_prefix),
@@ -381,20 +391,24 @@ e4b_status e4b_moe_backward_dgrad(const e4b_moe_desc* d, const e4b_experts* w, c
     __nv_bfloat16* a_perm = reinterpret_cast<__nv_bfloat16*>(ws + L.a_perm);
     const int32_t* nrows = reinterpret_cast<const int32_t*>(ws + L.offsets) + d->E;
     const __nv_bfloat16* gu = static_cast<const __nv_bfloat16*>(saved_gu);
-    if (!gu) {   // recompute the gate/up pre-activations from x
+    const __nv_bfloat16* h = static_cast<const __nv_bfloat16*>(saved_h);
+    if (!gu) {   // recompute the gate/up pre-activations (and h) from x
         E4B_CUDA_TRY(launch_gather_rows(static_cast<const __nv_bfloat16*>(x), perm, nrows, d->top_k, P, d->H, a_perm, st));
         __nv_bfloat16* gu_ws = reinterpret_cast<__nv_bfloat16*>(ws + L.gu);
-        if ((s = run_gateup(d, w, ws, L, topk_w, P, reinterpret_cast<__nv_bfloat16*>(ws + L.h), gu_ws, st)) != E4B_OK)
-            return s;
+        __nv_bfloat16* h_ws = reinterpret_cast<__nv_bfloat16*>(ws + L.h);
+        if ((s = run_gateup(d, w, ws, L, topk_w, P, h_ws, gu_ws, st)) != E4B_OK) return s;
         gu = gu_ws;
+        h = h_ws;
     }
     E4B_CUDA_TRY(launch_gather_rows(static_cast<const __nv_bfloat16*>(grad_out), perm, nrows, d->top_k, P, d->H, a_perm, st));
     __nv_bfloat16* dgu = reinterpret_cast<__nv_bfloat16*>(ws + L.dgu);
 
-    GemmParams p = base_params(d, ws, L, topk_w, P);   // dh = w * grad_out W_down, then SwiGLU backward
+    // dh = w * grad_out W_down, then the activation backward; with grad_topk_w the
+    // epilogue also leaves <grad_out W_down, h> per row and n-tile
+    GemmParams p = base_params(d, ws, L, topk_w, P);
     p.K = d->H;
     p.N = d->I;
-    p.n_tiles = (d->I + 255) / 256;
+    p.n_tiles = dw_tiles(d);
     p.absmax = w->down_absmax;
     p.b_rows_per_expert = d->H;
     p.b_rows_total = (int64_t)d->E * d->H;
@@ -402,8 +416,18 @@ e4b_status e4b_moe_backward_dgrad(const e4b_moe_desc* d, const e4b_experts* w, c
     p.gu = const_cast<__nv_bfloat16*>(gu);
     p.out_bf16 = dgu;
     p.ld_out = 2 * d->I;
+    float* dw_part = reinterpret_cast<float*>(ws + L.dw_part);
+    if (grad_topk_w) {
+        p.h_in = h;
+        p.dw_part = dw_part;
+    }
     E4B_CUDA_TRY(launch_grouped_gemm(EPI_DGRAD_DOWN, d->codebook, a_perm, P, w->down, p.b_rows_total, d->I / 2, p,
                                      max_m_tiles(P, d->E), st));
+    if (grad_topk_w)   // reads the gathered grad_out rows' source, grad_out itself, before a_perm is reused
+        E4B_CUDA_TRY(launch_router_grad_parts(static_cast<const __nv_bfloat16*>(grad_out), dw_part, dw_tiles(d),
+                                              w->down_bias, inv_perm, topk_idx, topk_w, router_logits, T, d->E,
+                                              d->top_k, d->H, d->renormalize, grad_topk_w, grad_logits, st));
+    if (!grad_x) return E4B_OK;
 
     GemmParams q = base_params(d, ws, L, topk_w, P);   // grad_x += [dG, dU] W_gate_up
     q.K = 2 * d->I;
@@ -417,9 +441,17 @@ e4b_status e4b_moe_backward_dgrad(const e4b_moe_desc* d, const e4b_experts* w, c
     q.ld_out = d->H;
     E4B_CUDA_TRY(launch_grouped_gemm(EPI_DGRAD_GATEUP, d->codebook, dgu, P, w->gate_up, q.b_rows_total, d->H / 2, q,
                                      max_m_tiles(P, d->E), st));
-    E4B_CUDA_TRY(launch_combine(a_perm, reinterpret_cast<const int32_t*>(ws + L.inv_perm), d->top_k, T, d->H,
-                                static_cast<__nv_bfloat16*>(grad_x), st));
+    E4B_CUDA_TRY(launch_combine(a_perm, inv_perm, d->top_k, T, d->H, static_cast<__nv_bfloat16*>(grad_x), st));
     return E4B_OK;
+}
+
+e4b_status e4b_moe_backward_dgrad(const e4b_moe_desc* d, const e4b_experts* w, const void* x, int64_t T,
+                                  const int32_t* topk_idx, const float* topk_w, const void* grad_out,
+                                  const void* saved_gu, void* grad_x, void* workspace, size_t ws_bytes,
+                                  void* stream) {
+    if (T > 0 && !grad_x) return E4B_ERR_INVALID_ARG;
+    return e4b_moe_backward(d, w, x, T, nullptr, topk_idx, topk_w, grad_out, saved_gu, nullptr, grad_x, nullptr,
+                            nullptr, workspace, ws_bytes, stream);
 }
 
 e4b_status e4b_moe_backward_router(const e4b_moe_desc* d, const e4b_experts* w, const void* x, int64_t T,

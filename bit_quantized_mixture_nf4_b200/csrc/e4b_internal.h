@@ -33,6 +33,9 @@ struct GemmParams {
     int ld_out;
     float alpha, limit;
     uint32_t* status;         // device status word
+    const __nv_bfloat16* h_in;   // EPI_DGRAD_DOWN, optional: the forward's h [P, I] in grouped order
+    float* dw_part;           // with h_in: [P, n_tiles] fp32, row r / n-tile nt: sum over the tile's
+                              // columns c of (grad_out_r W_d,e)[c] * h[r, c] (before the routing weight)
 };
 
 // launch bookkeeping

@@ -9,7 +9,9 @@
 //
 //   EPI_GATEUP        D = X_e W_gu,e^T ; epilogue h = silu(g)*u (+ saves dh/dg, dh/du)
 //   EPI_DOWN          D = h_e W_d,e^T  ; epilogue out[row] = bf16(w * D)
-//   EPI_DGRAD_DOWN    D = dY_e W_d,e   ; epilogue dh = w*D, dG = dh*dh/dg, dU = dh*dh/du
+//   EPI_DGRAD_DOWN    D = dY_e W_d,e   ; epilogue dh = w*D, dG = dh*dh/dg, dU = dh*dh/du, and
+//                                        optionally the per-tile dot products <D, h> of the
+//                                        routing-weight gradient
 //   EPI_DGRAD_GATEUP  D = dGU_e W_gu,e ; epilogue out[row] = bf16(D)
 // Every output row is the grouped row itself (a contiguous slab per tile); the
 // k rows of a token are found through the inverse permutation and summed in
@@ -149,8 +151,27 @@ __device__ __forceinline__ int64_t absmax_index(const GemmParams& p, const TileI
     return row * p.b_blocks_per_row + blk;
 }
 
-// XACT (EPI_GATEUP only): the epilogue handles per-expert biases and the clamped GLU
-// (p.bias, p.act); the plain SwiGLU instance carries none of that code.
+// This row's part of the routing-weight gradient over one 32-column chunk:
+// acc += sum_j v[j] * h[row, c0 + j] (fp32, columns in order).
+__device__ __forceinline__ void dw_dot_chunk(const GemmParams& p, int64_t row, int c0, const float (&v)[32],
+                                             float& acc) {
+    const uint4* hs = reinterpret_cast<const uint4*>(p.h_in + row * p.N + c0);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const uint4 hv = __ldg(hs + i);
+        const uint32_t hw[4] = {hv.x, hv.y, hv.z, hv.w};
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            acc = fmaf(v[8 * i + 2 * j], __uint_as_float(hw[j] << 16), acc);
+            acc = fmaf(v[8 * i + 2 * j + 1], __uint_as_float(hw[j] & 0xFFFF0000u), acc);
+        }
+    }
+}
+
+// XACT, the extended epilogue: EPI_GATEUP handles per-expert biases and the clamped
+// GLU (p.bias, p.act); EPI_DGRAD_DOWN also takes the dot products of the
+// routing-weight gradient (p.h_in, p.dw_part).  The plain instances carry none of
+// that code.
 template <int EPI, int CB, int CTAS, bool XACT = false>
 __global__ void __launch_bounds__(GEMM_THREADS, 1)
 grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_raw,
@@ -487,6 +508,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_con
             // everything that does not depend on the accumulator is fetched before waiting for it
             float wgt = 1.0f;
             if ((EPI == EPI_DOWN || EPI == EPI_DGRAD_DOWN) && valid) wgt = __ldg(p.topk_w + __ldg(p.perm + row));
+            float dwdot = 0.0f;   // EPI_DGRAD_DOWN, XACT: <grad_out W_d, h> over the tile's columns
             uint4 gq[4], uq[4];   // EPI_DGRAD_DOWN: saved dh/dg, dh/du of the current 32-column chunk
             auto load_gu = [&](int q, uint4 (&g4)[4], uint4 (&u4)[4]) {
                 const int c0 = ti.nt * BN + 32 * q;
@@ -614,6 +636,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_con
                     float v[32];
                     tmem_load32(tbase + 32 * q, v);
                     if (q + 1 < BN / 32 && c0 + 32 < I) issue_pair(c0 + 32, srow);   // next pair in flight
+                    if (XACT) dw_dot_chunk(p, row, c0, v, dwdot);
                     const uint32_t n = ncons++;
                     if (!wait(&ctl->ld_full[warp][n & 1], (n >> 1) & 1)) {
                         aborted = true;
@@ -650,6 +673,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_con
                     }
                 }
                 if (aborted) break;
+                if (XACT) p.dw_part[(int64_t)row * p.n_tiles + ti.nt] = dwdot;
             } else {
 #pragma unroll 1
                 for (int q = 0; q < BN / 32; ++q) {
@@ -684,6 +708,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_con
                             }
                         } else {   // EPI_DGRAD_DOWN: SwiGLU backward with the saved derivatives
                             const int I = p.N;
+                            if (XACT && valid) dw_dot_chunk(p, row, c0, v, dwdot);
                             uint32_t dgw[16], duw[16];
 #pragma unroll
                             for (int i = 0; i < 4; ++i) {
@@ -720,6 +745,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_con
                         }
                     }
                 }
+                if (EPI == EPI_DGRAD_DOWN && XACT && valid) p.dw_part[(int64_t)row * p.n_tiles + ti.nt] = dwdot;
             }
             tc_fence_before();
             __syncwarp();
@@ -864,10 +890,14 @@ cudaError_t launch_grouped_gemm(int epi, int codebook, const void* a, int64_t a_
     const int grid = (int)std::min<int64_t>(tiles * kCtas, (num_sms() / kCtas) * kCtas);
     if (grid <= 0) return cudaSuccess;
 #define E4B_LAUNCH(E_, C_) return launch_one<E_, C_>(ma, mr, mo, mg, p, grid, st)
-    const bool xact = epi == EPI_GATEUP && (p.act != 0 || p.bias != nullptr);
-    if (xact) {
+    if (epi == EPI_GATEUP && (p.act != 0 || p.bias != nullptr)) {
         if (codebook == 0) return launch_one<EPI_GATEUP, 0, true>(ma, mr, mo, mg, p, grid, st);
         return launch_one<EPI_GATEUP, 1, true>(ma, mr, mo, mg, p, grid, st);
+    }
+    if (epi == EPI_DGRAD_DOWN && p.dw_part) {
+        if (!p.h_in) return cudaErrorInvalidValue;
+        if (codebook == 0) return launch_one<EPI_DGRAD_DOWN, 0, true>(ma, mr, mo, mg, p, grid, st);
+        return launch_one<EPI_DGRAD_DOWN, 1, true>(ma, mr, mo, mg, p, grid, st);
     }
     if (codebook == 0) {
         switch (epi) {

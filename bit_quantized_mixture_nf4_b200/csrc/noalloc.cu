@@ -63,6 +63,6 @@ extern "C" e4b_status e4b_moe_forward_noalloc(const e4b_moe_desc* d, const e4b_e
     if (!scratch) return st;
     // Every byte of the scratch the forward reads is written earlier in the same
     // call, so nothing has to be cleared between calls.
-    return e4b_moe_forward(d, w, x, T, router_logits, topk_idx, topk_w, y, nullptr, nullptr, nullptr, scratch,
+    return e4b_moe_forward(d, w, x, T, router_logits, topk_idx, topk_w, y, nullptr, nullptr, nullptr, nullptr, scratch,
                            kNoAllocScratchBytes, stream);
 }

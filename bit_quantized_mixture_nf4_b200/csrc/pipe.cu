@@ -154,7 +154,7 @@ e4b_status e4b_pipe_submit(e4b_pipe* p, int64_t T, const void* x_host, const flo
     PIPE_TRY(cudaStreamWaitEvent(p->compute, p->in_ready[b], 0));
     if (p->used[b]) PIPE_TRY(cudaStreamWaitEvent(p->compute, p->out_done[b], 0));
     e4b_status s = e4b_moe_forward(&p->d, &p->w, p->x[b], T, p->logits[b], p->idx[b], p->wts[b], p->y[b], p->saved,
-                                   nullptr, nullptr, p->ws, p->ws_bytes, p->compute);
+                                   nullptr, nullptr, nullptr, p->ws, p->ws_bytes, p->compute);
     if (s != E4B_OK) return s;
     PIPE_TRY(cudaEventRecord(p->y_ready[b], p->compute));
     s = e4b_moe_backward_dgrad(&p->d, &p->w, p->x[b], T, p->idx[b], p->wts[b], p->go[b], p->saved, p->gx[b], p->ws,

@@ -7,7 +7,9 @@
 //   no renormalisation: dL/dl_i = p_i (sum_{j: e_j = i} dw_j - sum_j dw_j p_{e_j}),
 //     p = softmax over all E experts;
 //   renormalisation: dL/dl_i = sum_{j: e_j = i} w_j (dw_j - sum_j' w_j' dw_j').
-// The unweighted Y comes from the grouped down GEMM run with unit weights.
+// The unweighted Y comes from the grouped down GEMM run with unit weights, or,
+// fused into the input gradient, dL/dw = <grad_out_t W_d, h_{t,j}> (+ <grad_out_t,
+// b_e> with a down bias) from the dot products the down^T GEMM leaves per tile.
 #include "router_backward.h"
 
 namespace e4b {
@@ -17,11 +19,17 @@ __global__ void __launch_bounds__(256) fill_f32_kernel(float* __restrict__ p, in
         p[i] = v;
 }
 
-// One warp per token: the k dot products <grad_out_t, Y_{t,j}> over H (fp32, a
-// fixed order: per-lane sums over 16-byte chunks, then a butterfly), then the
-// logit gradient of the token.
+// One warp per token: the k routing-weight gradients of the token, then its
+// logit gradient.  FROM_PARTS = false: dw_j = <grad_out_t, Y_{t,j}> over H
+// (fp32, a fixed order: per-lane sums over 16-byte chunks, then a butterfly).
+// FROM_PARTS = true: dw_j = the sum of the pair's per-tile dot products
+// <grad_out_t W_d, h> (written by the input-gradient down^T GEMM; lane-strided
+// over the tiles, then a butterfly) plus, with a down bias, <grad_out_t, b_e>.
+template <bool FROM_PARTS>
 __global__ void __launch_bounds__(256) router_grad_kernel(const __nv_bfloat16* __restrict__ grad_out,
                                                           const __nv_bfloat16* __restrict__ Y,
+                                                          const float* __restrict__ parts, int n_parts,
+                                                          const float* __restrict__ down_bias,
                                                           const int32_t* __restrict__ inv_perm,
                                                           const int32_t* __restrict__ idx,
                                                           const float* __restrict__ wts,
@@ -43,15 +51,36 @@ __global__ void __launch_bounds__(256) router_grad_kernel(const __nv_bfloat16* _
         const bool valid = e >= 0 && e < E;
         float acc = 0.0f;
         if (valid) {
+            const int64_t r = __ldg(inv_perm + p);
             const uint4* g4 = reinterpret_cast<const uint4*>(grad_out + t * H);
-            const uint4* y4 = reinterpret_cast<const uint4*>(Y + (int64_t)__ldg(inv_perm + p) * H);
-            for (int c = lane; c < H / 8; c += 32) {
-                const uint4 gv = __ldg(g4 + c), yv = __ldcs(y4 + c);
-                const uint32_t gw[4] = {gv.x, gv.y, gv.z, gv.w}, yw[4] = {yv.x, yv.y, yv.z, yv.w};
+            if (FROM_PARTS) {
+                for (int c = lane; c < n_parts; c += 32) acc += __ldcs(parts + r * n_parts + c);
+                if (down_bias) {
+                    float b = 0.0f;
+                    const float4* b4 = reinterpret_cast<const float4*>(down_bias + (int64_t)e * H);
+                    for (int c = lane; c < H / 8; c += 32) {
+                        const uint4 gv = __ldg(g4 + c);
+                        const float4 bl = __ldg(b4 + 2 * c), bh = __ldg(b4 + 2 * c + 1);
+                        const float bv[8] = {bl.x, bl.y, bl.z, bl.w, bh.x, bh.y, bh.z, bh.w};
+                        const uint32_t gw[4] = {gv.x, gv.y, gv.z, gv.w};
 #pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    acc = fmaf(__uint_as_float(gw[q] << 16), __uint_as_float(yw[q] << 16), acc);
-                    acc = fmaf(__uint_as_float(gw[q] & 0xFFFF0000u), __uint_as_float(yw[q] & 0xFFFF0000u), acc);
+                        for (int q = 0; q < 4; ++q) {
+                            b = fmaf(__uint_as_float(gw[q] << 16), bv[2 * q], b);
+                            b = fmaf(__uint_as_float(gw[q] & 0xFFFF0000u), bv[2 * q + 1], b);
+                        }
+                    }
+                    acc += b;
+                }
+            } else {
+                const uint4* y4 = reinterpret_cast<const uint4*>(Y + r * H);
+                for (int c = lane; c < H / 8; c += 32) {
+                    const uint4 gv = __ldg(g4 + c), yv = __ldcs(y4 + c);
+                    const uint32_t gw[4] = {gv.x, gv.y, gv.z, gv.w}, yw[4] = {yv.x, yv.y, yv.z, yv.w};
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        acc = fmaf(__uint_as_float(gw[q] << 16), __uint_as_float(yw[q] << 16), acc);
+                        acc = fmaf(__uint_as_float(gw[q] & 0xFFFF0000u), __uint_as_float(yw[q] & 0xFFFF0000u), acc);
+                    }
                 }
             }
         }
@@ -123,8 +152,20 @@ cudaError_t launch_router_grad(const __nv_bfloat16* grad_out, const __nv_bfloat1
                                int H, int renorm, float* dw, float* dlogits, cudaStream_t st) {
     if (T == 0) return cudaSuccess;
     const int64_t grid = (T * 32 + 255) / 256;
-    router_grad_kernel<<<(unsigned)grid, 256, 0, st>>>(grad_out, Y, inv_perm, idx, wts, logits, T, E, k, H, renorm,
-                                                       dw, dlogits);
+    router_grad_kernel<false><<<(unsigned)grid, 256, 0, st>>>(grad_out, Y, nullptr, 0, nullptr, inv_perm, idx, wts,
+                                                              logits, T, E, k, H, renorm, dw, dlogits);
+    count_launch();
+    return cudaGetLastError();
+}
+
+cudaError_t launch_router_grad_parts(const __nv_bfloat16* grad_out, const float* parts, int n_parts,
+                                     const float* down_bias, const int32_t* inv_perm, const int32_t* idx,
+                                     const float* wts, const float* logits, int64_t T, int E, int k, int H,
+                                     int renorm, float* dw, float* dlogits, cudaStream_t st) {
+    if (T == 0) return cudaSuccess;
+    const int64_t grid = (T * 32 + 255) / 256;
+    router_grad_kernel<true><<<(unsigned)grid, 256, 0, st>>>(grad_out, nullptr, parts, n_parts, down_bias, inv_perm,
+                                                             idx, wts, logits, T, E, k, H, renorm, dw, dlogits);
     count_launch();
     return cudaGetLastError();
 }

@@ -12,4 +12,12 @@ cudaError_t launch_router_grad(const __nv_bfloat16* grad_out, const __nv_bfloat1
                                const int32_t* idx, const float* wts, const float* logits, int64_t T, int E, int k,
                                int H, int renorm, float* dw, float* dlogits, cudaStream_t st);
 
+// The same from the per-tile dot products parts [P, n_parts] (grouped row order)
+// that the input-gradient down^T GEMM writes: dw = sum of the row's parts, plus
+// <grad_out_t, b_e> when down_bias is given.
+cudaError_t launch_router_grad_parts(const __nv_bfloat16* grad_out, const float* parts, int n_parts,
+                                     const float* down_bias, const int32_t* inv_perm, const int32_t* idx,
+                                     const float* wts, const float* logits, int64_t T, int E, int k, int H,
+                                     int renorm, float* dw, float* dlogits, cudaStream_t st);
+
 }  // namespace e4b

@@ -153,6 +153,9 @@ E4B_API size_t e4b_moe_workspace_size(const e4b_moe_desc *d, int64_t T);
  *                activation's derivatives dh/dg in columns [0,I) and dh/du in
  *                columns [I,2I) (SwiGLU: u s(g) (1 + g (1 - s(g))) and silu(g), s
  *                the logistic function), for e4b_moe_backward_dgrad.
+ *   saved_h      bf16 [T*k, I] or NULL: the activation output h of every pair in
+ *                grouped row order, for the routing-weight gradient of
+ *                e4b_moe_backward.  The forward's down GEMM reads h from here.
  *   offsets_out  int32 [E+1] or NULL: first grouped row of each expert.
  *   perm_out     int32 [T*k] or NULL: pair id t*k+j of each grouped row;
  *                experts ascending, tokens ascending inside an expert.
@@ -160,8 +163,35 @@ E4B_API size_t e4b_moe_workspace_size(const e4b_moe_desc *d, int64_t T);
  * T == 0 is a no-op.  topk_idx entries outside [0, E) are outside the contract. */
 E4B_API e4b_status e4b_moe_forward(const e4b_moe_desc *d, const e4b_experts *w, const void *x, int64_t T,
                            const float *router_logits, int32_t *topk_idx, float *topk_w, void *y,
-                           void *saved_gu, int32_t *offsets_out, int32_t *perm_out,
+                           void *saved_gu, void *saved_h, int32_t *offsets_out, int32_t *perm_out,
                            void *workspace, size_t ws_bytes, void *stream);
+
+/* The layer backward: the input gradient and the routing gradient in one pass.
+ *   grad_x       as in e4b_moe_backward_dgrad (written), or NULL;
+ *   grad_topk_w  fp32 [T,k] = <grad_out_t, Y_{t,j}> as in e4b_moe_backward_router
+ *                (written; 0 for an out-of-range expert), or NULL;
+ *   grad_logits  fp32 [T,E] through the routing softmax as in
+ *                e4b_moe_backward_router (written), or NULL.
+ * The routing-weight gradient is fused into the input gradient's down^T GEMM:
+ * its accumulator is grad_out_t W_down,e before the routing weight, so
+ *   <grad_out_t, Y_{t,j}> = <grad_out_t W_down,e, h_{t,j}> (+ <grad_out_t, b_e>
+ *                                                           with a down bias)
+ * and the epilogue leaves one fp32 partial dot product per row and 256-column
+ * tile; a per-token kernel adds them in tile order and runs the softmax
+ * backward.  No GEMM is repeated for it.  h comes from saved_h (as written by
+ * e4b_moe_forward for the same topk_idx, with saved_gu) or, when saved_gu is
+ * NULL, is recomputed from x together with the derivatives.
+ *   x bf16 [T,H] (read only when saved_gu is NULL); router_logits fp32 [T,E]
+ *   (needed only for grad_logits); topk_idx, topk_w, grad_out as for
+ *   e4b_moe_backward_dgrad; workspace: e4b_moe_workspace_size(d, T) bytes.
+ * Returns E4B_ERR_INVALID_ARG when no output is asked for, when grad_topk_w is
+ * asked for with saved_gu but without saved_h, or when grad_logits is asked for
+ * without router_logits or grad_topk_w. */
+E4B_API e4b_status e4b_moe_backward(const e4b_moe_desc *d, const e4b_experts *w, const void *x, int64_t T,
+                            const float *router_logits, const int32_t *topk_idx, const float *topk_w,
+                            const void *grad_out, const void *saved_gu, const void *saved_h,
+                            void *grad_x, float *grad_topk_w, float *grad_logits,
+                            void *workspace, size_t ws_bytes, void *stream);
 
 /* Input gradient of the forward with routing held constant ([P5] "What this
  * adds": recompute-in-backward; the packed base is frozen, no weight gradient):

@@ -62,11 +62,11 @@ def test_host_side_validation(lib):
         assert lib.e4b_moe_workspace_size(bad, 64) == code
     ex = lib.e4b_experts(None, None, None, None)
     st = lambda: L.e4b_moe_forward(ctypes.byref(d), ctypes.byref(ex), None, 4, None, None, None, None, None,
-                                   None, None, None, 0, None)
+                                   None, None, None, None, 0, None)
     assert st() == lib.E4B_ERR_INVALID_ARG
     ex2 = lib.e4b_experts(16, 16, 16, 16)   # non-null dummies: never dereferenced on these paths
     f = lambda dd, T, x, ws, n: L.e4b_moe_forward(ctypes.byref(dd), ctypes.byref(ex2), x, T, None, 16, 16, 16, None,
-                                                  None, None, ws, n, None)
+                                                  None, None, None, ws, n, None)
     assert f(d, 0, None, None, 0) == lib.E4B_OK                        # T == 0: no-op
     assert f(d, 4, None, 16, 1 << 30) == lib.E4B_ERR_INVALID_ARG       # null x
     assert f(d, 4, 16, None, 0) == lib.E4B_ERR_WORKSPACE               # no workspace
@@ -90,12 +90,26 @@ def test_host_side_validation(lib):
     glu_dec = lib.make_desc(8, 256, 512, 2, path=lib.PATH_DECODE, activation=lib.ACT_CLAMPED_GLU)
     assert f(glu_dec, 2, 16, 16, 1 << 40) == lib.E4B_ERR_UNSUPPORTED
     exb = lib.e4b_experts(16, 16, 16, 16, 16, None)
-    assert L.e4b_moe_forward(ctypes.byref(dec), ctypes.byref(exb), 16, 2, None, 16, 16, 16, None, None, None, 16,
-                             1 << 40, None) == lib.E4B_ERR_UNSUPPORTED
+    assert L.e4b_moe_forward(ctypes.byref(dec), ctypes.byref(exb), 16, 2, None, 16, 16, 16, None, None, None, None,
+                             16, 1 << 40, None) == lib.E4B_ERR_UNSUPPORTED
+    # saved_h asks for the grouped path's intermediates: the decode path is refused
+    assert L.e4b_moe_forward(ctypes.byref(dec), ctypes.byref(ex2), 16, 2, None, 16, 16, 16, None, 16, None, None,
+                             16, 1 << 40, None) == lib.E4B_ERR_UNSUPPORTED
     g = lambda dd, T: L.e4b_moe_backward_dgrad(ctypes.byref(dd), ctypes.byref(ex2), None, T, 16, 16, 16, None, 16,
                                                16, 1 << 40, None)
     assert g(d, 4) == lib.E4B_ERR_INVALID_ARG                          # needs x when saved_gu is NULL
     assert g(d, 0) == lib.E4B_OK
+    # the fused layer backward: argument rules, checked before any launch
+    def b(T, x=16, logits=None, saved_gu=16, saved_h=16, gx=16, gw=16, gl=None):
+        return L.e4b_moe_backward(ctypes.byref(d), ctypes.byref(ex2), x, T, logits, 16, 16, 16, saved_gu, saved_h,
+                                  gx, gw, gl, None, 0, None)
+    assert b(0) == lib.E4B_OK                                           # T == 0: no-op
+    assert b(4, gx=None, gw=None) == lib.E4B_ERR_INVALID_ARG           # no output asked for
+    assert b(4, x=None, saved_gu=None) == lib.E4B_ERR_INVALID_ARG      # nothing to recompute from
+    assert b(4, saved_h=None) == lib.E4B_ERR_INVALID_ARG               # routing gradient needs the saved h
+    assert b(4, gl=16) == lib.E4B_ERR_INVALID_ARG                      # grad_logits needs router_logits
+    assert b(4, logits=16, gw=None, gl=16) == lib.E4B_ERR_INVALID_ARG  # ... and grad_topk_w
+    assert b(4) == lib.E4B_ERR_WORKSPACE                               # valid request, no workspace
 
 
 def test_pipe_host_side_validation(lib):
