@@ -38,12 +38,19 @@ class e4b_moe_desc(ctypes.Structure):
     _fields_ = [("E", ctypes.c_int), ("H", ctypes.c_int), ("I", ctypes.c_int), ("top_k", ctypes.c_int),
                 ("renormalize", ctypes.c_int), ("codebook", ctypes.c_int), ("blocksize", ctypes.c_int),
                 ("path", ctypes.c_int), ("activation", ctypes.c_int), ("glu_alpha", ctypes.c_float),
-                ("glu_limit", ctypes.c_float)]
+                ("glu_limit", ctypes.c_float), ("lora_rank", ctypes.c_int), ("lora_scale", ctypes.c_float)]
 
 
 class e4b_experts(ctypes.Structure):
     _fields_ = [("gate_up", ctypes.c_void_p), ("down", ctypes.c_void_p), ("gate_up_absmax", ctypes.c_void_p),
-                ("down_absmax", ctypes.c_void_p), ("gate_up_bias", ctypes.c_void_p), ("down_bias", ctypes.c_void_p)]
+                ("down_absmax", ctypes.c_void_p), ("gate_up_bias", ctypes.c_void_p), ("down_bias", ctypes.c_void_p),
+                ("lora_A_gu", ctypes.c_void_p), ("lora_B_gu", ctypes.c_void_p), ("lora_A_d", ctypes.c_void_p),
+                ("lora_B_d", ctypes.c_void_p)]
+
+
+class e4b_lora_grads(ctypes.Structure):
+    _fields_ = [("dA_gu", ctypes.c_void_p), ("dB_gu", ctypes.c_void_p), ("dA_d", ctypes.c_void_p),
+                ("dB_d", ctypes.c_void_p)]
 
 
 class E4BError(RuntimeError):
@@ -70,7 +77,7 @@ def _load():
     lib.e4b_moe_forward.argtypes = [ctypes.POINTER(e4b_moe_desc), ctypes.POINTER(e4b_experts), P, i64, P, P, P, P,
                                     P, P, P, P, P, sz, P]
     lib.e4b_moe_backward.argtypes = [ctypes.POINTER(e4b_moe_desc), ctypes.POINTER(e4b_experts), P, i64, P, P, P, P,
-                                     P, P, P, P, P, P, sz, P]
+                                     P, P, P, P, P, P, P, sz, P]
     lib.e4b_moe_backward_dgrad.argtypes = [ctypes.POINTER(e4b_moe_desc), ctypes.POINTER(e4b_experts), P, i64, P, P,
                                            P, P, P, P, sz, P]
     lib.e4b_moe_forward_noalloc.argtypes = [ctypes.POINTER(e4b_moe_desc), ctypes.POINTER(e4b_experts), P, i64, P, P,
@@ -203,15 +210,18 @@ def e4b_dequantize_nf4(packed: torch.Tensor, absmax: torch.Tensor, shape, blocks
 
 
 def make_desc(E, H, I, top_k, renormalize=True, codebook=NF4, blocksize=64, path=PATH_AUTO, activation=ACT_SWIGLU,
-              glu_alpha=1.702, glu_limit=7.0) -> e4b_moe_desc:
+              glu_alpha=1.702, glu_limit=7.0, lora_rank=0, lora_scale=1.0) -> e4b_moe_desc:
     return e4b_moe_desc(E, H, I, top_k, int(bool(renormalize)), codebook, blocksize, path, activation, glu_alpha,
-                        glu_limit)
+                        glu_limit, lora_rank, lora_scale)
 
 
-def make_experts(gate_up, down, gate_up_absmax, down_absmax, gate_up_bias=None, down_bias=None) -> e4b_experts:
+def make_experts(gate_up, down, gate_up_absmax, down_absmax, gate_up_bias=None, down_bias=None,
+                 lora=None) -> e4b_experts:
     """The two packed stacks and their absmax (device tensors), plus optional fp32
-    per-expert biases gate_up_bias [E, 2I] and down_bias [E, H].  The tensors must
-    outlive every call that uses the returned struct."""
+    per-expert biases gate_up_bias [E, 2I] and down_bias [E, H], and optional bf16
+    LoRA adapters lora = (A_gu [E, r, H], B_gu [E, 2I, r], A_d [E, r, I], B_d [E, H, r])
+    (the descriptor's lora_rank must be r).  The tensors must outlive every call
+    that uses the returned struct."""
     for n, t in (("gate_up", gate_up), ("down", down)):
         _cuda(t, n, torch.uint8)
     for n, t in (("gate_up_absmax", gate_up_absmax), ("down_absmax", down_absmax)):
@@ -219,9 +229,16 @@ def make_experts(gate_up, down, gate_up_absmax, down_absmax, gate_up_bias=None, 
     for n, t in (("gate_up_bias", gate_up_bias), ("down_bias", down_bias)):
         if t is not None:
             _cuda(t, n, torch.float32)
+    ad = [None] * 4
+    if lora is not None:
+        for i, (n, t) in enumerate(zip(("A_gu", "B_gu", "A_d", "B_d"), lora)):
+            _cuda(t, n, torch.bfloat16)
+            if not t.is_contiguous():
+                raise ValueError(f"{n} must be contiguous")
+            ad[i] = t.data_ptr()
     return e4b_experts(gate_up.data_ptr(), down.data_ptr(), gate_up_absmax.data_ptr(), down_absmax.data_ptr(),
                        None if gate_up_bias is None else gate_up_bias.data_ptr(),
-                       None if down_bias is None else down_bias.data_ptr())
+                       None if down_bias is None else down_bias.data_ptr(), *ad)
 
 
 def e4b_moe_workspace_size(desc: e4b_moe_desc, T: int) -> int:
@@ -260,11 +277,13 @@ def e4b_moe_forward(desc: e4b_moe_desc, experts: e4b_experts, x: torch.Tensor, r
 
 def e4b_moe_backward(desc: e4b_moe_desc, experts: e4b_experts, x, topk_idx, topk_w, grad_out, saved_gu=None,
                      saved_h=None, router_logits=None, grad_x=None, grad_topk_w=None, grad_logits=None,
-                     want_grad_x=True, want_routing=True, ws=None, stream=None):
+                     want_grad_x=True, want_routing=True, lora_grads=None, ws=None, stream=None):
     """The layer backward in one pass: (grad_x bf16 [T, H] or None, grad_topk_w fp32
     [T, k] or None, grad_logits fp32 [T, E] or None).  The routing-weight gradient
     is fused into the input gradient's down^T GEMM; with saved_gu it needs
-    saved_h (both from e4b_moe_forward), without them x is used to recompute."""
+    saved_h (both from e4b_moe_forward), without them x is used to recompute.
+    lora_grads: fp32 tensors (dA_gu, dB_gu, dA_d, dB_d) shaped like the adapters,
+    written with the adapter gradients (needs x)."""
     _cuda(grad_out, "grad_out", torch.bfloat16)
     T = grad_out.shape[0]
     dev = grad_out.device
@@ -278,10 +297,15 @@ def e4b_moe_backward(desc: e4b_moe_desc, experts: e4b_experts, x, topk_idx, topk
             grad_logits = torch.empty(T, desc.E, dtype=torch.float32, device=dev)
     if ws is None:
         ws = workspace(desc, T, dev)
+    lg = None
+    if lora_grads is not None:
+        for n, t in zip(("dA_gu", "dB_gu", "dA_d", "dB_d"), lora_grads):
+            _cuda(t, n, torch.float32)
+        lg = e4b_lora_grads(*[t.data_ptr() for t in lora_grads])
     _check("e4b_moe_backward", _load().e4b_moe_backward(
         ctypes.byref(desc), ctypes.byref(experts), _ptr(x), T, _ptr(router_logits), _ptr(topk_idx), _ptr(topk_w),
-        _ptr(grad_out), _ptr(saved_gu), _ptr(saved_h), _ptr(grad_x), _ptr(grad_topk_w), _ptr(grad_logits), _ptr(ws),
-        ws.numel(), _stream(stream)))
+        _ptr(grad_out), _ptr(saved_gu), _ptr(saved_h), _ptr(grad_x), _ptr(grad_topk_w), _ptr(grad_logits),
+        None if lg is None else ctypes.byref(lg), _ptr(ws), ws.numel(), _stream(stream)))
     return grad_x, grad_topk_w, grad_logits
 
 

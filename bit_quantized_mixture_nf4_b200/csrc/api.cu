@@ -9,6 +9,7 @@
 
 #include "../../include/e4b.h"
 #include "e4b_internal.h"
+#include "lora.h"
 #include "router_backward.h"
 
 namespace e4b {
@@ -98,7 +99,7 @@ uint32_t* device_status_ptr() {
 // ------------------------------------------------------------ workspace layout
 struct WsLayout {
     size_t chunk_counts, chunk_base, counts, offsets, tile_prefix, sched, perm, inv_perm, a_perm, h, gu, dgu, dec, ones,
-        dw_part, total;
+        dw_part, lz_gu, lz_d, lv_d, lv_gu, x_perm, total;
 };
 
 static size_t align_up(size_t v) { return (v + 255) & ~size_t(255); }
@@ -128,6 +129,13 @@ static WsLayout layout_for(const e4b_moe_desc* d, int64_t T) {
     L.dec = take(decode_scratch_bytes(d->E, d->H, d->I, T, d->top_k));
     L.ones = take((size_t)P * 4);
     L.dw_part = take((size_t)P * dw_tiles(d) * 4);
+    if (d->lora_rank > 0) {   // the thin LoRA operands [P, 64] bf16 and the kept gathered x
+        L.lz_gu = take((size_t)P * 64 * 2);
+        L.lz_d = take((size_t)P * 64 * 2);
+        L.lv_d = take((size_t)P * 64 * 2);
+        L.lv_gu = take((size_t)P * 64 * 2);
+        L.x_perm = take((size_t)P * d->H * 2);
+    }
     L.total = off;
     return L;
 }
@@ -143,11 +151,15 @@ static e4b_status check_desc(const e4b_moe_desc* d) {
     if (d->activation != E4B_ACT_SWIGLU && d->activation != E4B_ACT_CLAMPED_GLU) return E4B_ERR_INVALID_ARG;
     if (d->activation == E4B_ACT_CLAMPED_GLU && (!std::isfinite(d->glu_alpha) || !(d->glu_limit > 0.0f)))
         return E4B_ERR_INVALID_ARG;
+    if (d->lora_rank < 0 || d->lora_rank > 64 || d->lora_rank % 8) return E4B_ERR_INVALID_ARG;
+    if (d->lora_rank > 0 && !std::isfinite(d->lora_scale)) return E4B_ERR_INVALID_ARG;
     return E4B_OK;
 }
 
-static e4b_status check_experts(const e4b_experts* w) {
+static e4b_status check_experts(const e4b_moe_desc* d, const e4b_experts* w) {
     if (!w || !w->gate_up || !w->down || !w->gate_up_absmax || !w->down_absmax) return E4B_ERR_INVALID_ARG;
+    if (d->lora_rank > 0 && (!w->lora_A_gu || !w->lora_B_gu || !w->lora_A_d || !w->lora_B_d))
+        return E4B_ERR_INVALID_ARG;
     return E4B_OK;
 }
 
@@ -171,10 +183,28 @@ static GemmParams base_params(const e4b_moe_desc* d, uint8_t* ws, const WsLayout
 
 static int max_m_tiles(int64_t P, int E) { return (int)((P + gemm_tile_rows() - 1) / gemm_tile_rows()) + E; }
 
-// gate_up GEMM + SwiGLU over the grouped rows in ws.a_perm.
+static const __nv_bfloat16* bf(const void* p) { return static_cast<const __nv_bfloat16*>(p); }
+
+// The thin LoRA operand out [P, 64] = s * in [P, K] M_e^T (M an A adapter [E, r, K]
+// when q_major, else a B adapter [E, K, r]).
+static e4b_status lora_thin(const e4b_moe_desc* d, uint8_t* ws, const WsLayout& L, int64_t P, const void* in, int K,
+                            const void* m, bool q_major, size_t out_off, cudaStream_t st) {
+    E4B_CUDA_TRY(launch_lora_thin(bf(in), K, bf(m), q_major, d->lora_rank, d->lora_scale,
+                                  reinterpret_cast<const int4*>(ws + L.sched),
+                                  reinterpret_cast<const int*>(ws + L.tile_prefix), d->E, max_m_tiles(P, d->E),
+                                  reinterpret_cast<__nv_bfloat16*>(ws + out_off), st));
+    return E4B_OK;
+}
+
+// gate_up GEMM + activation over the grouped rows a (ws.a_perm unless given); with
+// adapters, the LoRA stage takes ws.lz_gu (made here from a) against B_gu.
 static e4b_status run_gateup(const e4b_moe_desc* d, const e4b_experts* w, uint8_t* ws, const WsLayout& L,
                              const float* topk_w, int64_t P, __nv_bfloat16* h_out, __nv_bfloat16* gu_out,
-                             cudaStream_t st) {
+                             cudaStream_t st, const void* a = nullptr) {
+    if (!a) a = ws + L.a_perm;
+    e4b_status s;
+    if (d->lora_rank > 0 && (s = lora_thin(d, ws, L, P, a, d->H, w->lora_A_gu, true, L.lz_gu, st)) != E4B_OK)
+        return s;
     GemmParams p = base_params(d, ws, L, topk_w, P);
     p.K = d->H;
     p.N = d->I;
@@ -191,8 +221,36 @@ static e4b_status run_gateup(const e4b_moe_desc* d, const e4b_experts* w, uint8_
     p.alpha = d->glu_alpha;
     p.limit = d->glu_limit;
     p.bias = w->gate_up_bias;
-    E4B_CUDA_TRY(launch_grouped_gemm(EPI_GATEUP, d->codebook, ws + L.a_perm, P, w->gate_up, p.b_rows_total, d->H / 2,
-                                     p, max_m_tiles(P, d->E), st));
+    p.lora_r = d->lora_rank;
+    p.lora_b = bf(w->lora_B_gu);
+    E4B_CUDA_TRY(launch_grouped_gemm(EPI_GATEUP, d->codebook, a, P, w->gate_up, p.b_rows_total, d->H / 2, p,
+                                     max_m_tiles(P, d->E), st, d->lora_rank > 0 ? ws + L.lz_gu : nullptr));
+    return E4B_OK;
+}
+
+// down GEMM over h [P, I] into the per-pair rows out (weights w applied); with
+// adapters, the LoRA stage takes ws.lz_d = s h A_d^T (made here) against B_d.
+static e4b_status run_down(const e4b_moe_desc* d, const e4b_experts* w, uint8_t* ws, const WsLayout& L,
+                           const float* wts, int64_t P, const __nv_bfloat16* h, __nv_bfloat16* out,
+                           cudaStream_t st) {
+    e4b_status s;
+    if (d->lora_rank > 0 && (s = lora_thin(d, ws, L, P, h, d->I, w->lora_A_d, true, L.lz_d, st)) != E4B_OK)
+        return s;
+    GemmParams p = base_params(d, ws, L, wts, P);
+    p.K = d->I;
+    p.N = d->H;
+    p.n_tiles = (d->H + 255) / 256;
+    p.absmax = w->down_absmax;
+    p.b_rows_per_expert = d->H;
+    p.b_rows_total = (int64_t)d->E * d->H;
+    p.b_blocks_per_row = d->I / 64;
+    p.out_bf16 = out;
+    p.bias = w->down_bias;
+    p.ld_out = d->H;
+    p.lora_r = d->lora_rank;
+    p.lora_b = bf(w->lora_B_d);
+    E4B_CUDA_TRY(launch_grouped_gemm(EPI_DOWN, d->codebook, h, P, w->down, p.b_rows_total, d->I / 2, p,
+                                     max_m_tiles(P, d->E), st, d->lora_rank > 0 ? ws + L.lz_d : nullptr));
     return E4B_OK;
 }
 
@@ -303,7 +361,7 @@ e4b_status e4b_moe_forward(const e4b_moe_desc* d, const e4b_experts* w, const vo
                            void* stream) {
     e4b_status s = check_desc(d);
     if (s != E4B_OK) return s;
-    if ((s = check_experts(w)) != E4B_OK) return s;
+    if ((s = check_experts(d, w)) != E4B_OK) return s;
     if (T < 0 || T * d->top_k > (int64_t)INT32_MAX) return E4B_ERR_INVALID_ARG;
     if (T == 0) return E4B_OK;
     if (!x || !topk_idx || !topk_w || !y) return E4B_ERR_INVALID_ARG;
@@ -311,7 +369,8 @@ e4b_status e4b_moe_forward(const e4b_moe_desc* d, const e4b_experts* w, const vo
     if (!workspace || ws_bytes < L.total) return E4B_ERR_WORKSPACE;
     const bool want_grouped_outputs = saved_gu || saved_h || offsets_out || perm_out;
     // the decode kernels implement SwiGLU without biases
-    const bool plain_experts = d->activation == E4B_ACT_SWIGLU && !w->gate_up_bias && !w->down_bias;
+    const bool plain_experts =
+        d->activation == E4B_ACT_SWIGLU && !w->gate_up_bias && !w->down_bias && d->lora_rank == 0;
     const bool dec_ok = !want_grouped_outputs && plain_experts && decode_supported(d->E, d->H, d->I, T, d->top_k);
     const bool decode = (d->path == E4B_PATH_DECODE) || (d->path == E4B_PATH_AUTO && dec_ok);
     if (d->path == E4B_PATH_DECODE && !dec_ok) return E4B_ERR_UNSUPPORTED;
@@ -343,19 +402,7 @@ e4b_status e4b_moe_forward(const e4b_moe_desc* d, const e4b_experts* w, const vo
     __nv_bfloat16* slots = reinterpret_cast<__nv_bfloat16*>(ws + L.a_perm);   // X_perm is dead after gate_up
     if ((s = run_gateup(d, w, ws, L, topk_w, P, h, static_cast<__nv_bfloat16*>(saved_gu), st)) != E4B_OK) return s;
 
-    GemmParams p = base_params(d, ws, L, topk_w, P);
-    p.K = d->I;
-    p.N = d->H;
-    p.n_tiles = (d->H + 255) / 256;
-    p.absmax = w->down_absmax;
-    p.b_rows_per_expert = d->H;
-    p.b_rows_total = (int64_t)d->E * d->H;
-    p.b_blocks_per_row = d->I / 64;
-    p.out_bf16 = slots;
-    p.bias = w->down_bias;
-    p.ld_out = d->H;
-    E4B_CUDA_TRY(launch_grouped_gemm(EPI_DOWN, d->codebook, h, P, w->down, p.b_rows_total, d->I / 2, p,
-                                     max_m_tiles(P, d->E), st));
+    if ((s = run_down(d, w, ws, L, topk_w, P, h, slots, st)) != E4B_OK) return s;
     E4B_CUDA_TRY(launch_combine(slots, reinterpret_cast<const int32_t*>(ws + L.inv_perm), d->top_k, T, d->H,
                                 static_cast<__nv_bfloat16*>(y), st));
     if (offsets_out) E4B_CUDA_TRY(cudaMemcpyAsync(offsets_out, offsets, (d->E + 1) * 4, cudaMemcpyDeviceToDevice, st));
@@ -366,45 +413,61 @@ e4b_status e4b_moe_forward(const e4b_moe_desc* d, const e4b_experts* w, const vo
 e4b_status e4b_moe_backward(const e4b_moe_desc* d, const e4b_experts* w, const void* x, int64_t T,
                             const float* router_logits, const int32_t* topk_idx, const float* topk_w,
                             const void* grad_out, const void* saved_gu, const void* saved_h, void* grad_x,
-                            float* grad_topk_w, float* grad_logits, void* workspace, size_t ws_bytes, void* stream) {
+                            float* grad_topk_w, float* grad_logits, const e4b_lora_grads* lora_grads,
+                            void* workspace, size_t ws_bytes, void* stream) {
     e4b_status s = check_desc(d);
     if (s != E4B_OK) return s;
-    if ((s = check_experts(w)) != E4B_OK) return s;
+    if ((s = check_experts(d, w)) != E4B_OK) return s;
     if (T < 0 || T * d->top_k > (int64_t)INT32_MAX) return E4B_ERR_INVALID_ARG;
     if (T == 0) return E4B_OK;
-    if (!topk_idx || !topk_w || !grad_out || (!grad_x && !grad_topk_w)) return E4B_ERR_INVALID_ARG;
-    if (!saved_gu && !x) return E4B_ERR_INVALID_ARG;                 // nothing to recompute from
-    if (grad_topk_w && saved_gu && !saved_h) return E4B_ERR_INVALID_ARG;   // h saved with the derivatives
+    const bool lg = d->lora_rank > 0 && lora_grads;   // adapter gradients asked for
+    if (lg && (!lora_grads->dA_gu || !lora_grads->dB_gu || !lora_grads->dA_d || !lora_grads->dB_d))
+        return E4B_ERR_INVALID_ARG;
+    if (!topk_idx || !topk_w || !grad_out || (!grad_x && !grad_topk_w && !lg)) return E4B_ERR_INVALID_ARG;
+    if (!saved_gu && !x) return E4B_ERR_INVALID_ARG;                            // nothing to recompute from
+    if ((grad_topk_w || lg) && saved_gu && !saved_h) return E4B_ERR_INVALID_ARG;   // h saved with the derivatives
+    if (lg && !x) return E4B_ERR_INVALID_ARG;                                   // dA_gu contracts with x
     if (grad_logits && (!router_logits || !grad_topk_w)) return E4B_ERR_INVALID_ARG;
     const WsLayout L = layout_for(d, T);
     if (!workspace || ws_bytes < L.total) return E4B_ERR_WORKSPACE;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     uint8_t* ws = static_cast<uint8_t*>(workspace);
     const int64_t P = T * d->top_k;
+    const bool lora = d->lora_rank > 0;
     int32_t* perm = reinterpret_cast<int32_t*>(ws + L.perm);
     const int32_t* inv_perm = reinterpret_cast<const int32_t*>(ws + L.inv_perm);
+    const int32_t* offsets = reinterpret_cast<const int32_t*>(ws + L.offsets);
     E4B_CUDA_TRY(launch_group(topk_idx, P, d->E, gemm_tile_rows(), reinterpret_cast<int32_t*>(ws + L.chunk_counts),
                               reinterpret_cast<int32_t*>(ws + L.chunk_base), reinterpret_cast<int32_t*>(ws + L.counts),
                               reinterpret_cast<int32_t*>(ws + L.offsets), reinterpret_cast<int32_t*>(ws + L.tile_prefix),
                               reinterpret_cast<int4*>(ws + L.sched), perm, reinterpret_cast<int32_t*>(ws + L.inv_perm),
                               st));
     __nv_bfloat16* a_perm = reinterpret_cast<__nv_bfloat16*>(ws + L.a_perm);
-    const int32_t* nrows = reinterpret_cast<const int32_t*>(ws + L.offsets) + d->E;
+    const int32_t* nrows = offsets + d->E;
     const __nv_bfloat16* gu = static_cast<const __nv_bfloat16*>(saved_gu);
     const __nv_bfloat16* h = static_cast<const __nv_bfloat16*>(saved_h);
+    // the gathered x: kept in its own buffer when the adapters need it to the end
+    __nv_bfloat16* xg = lora ? reinterpret_cast<__nv_bfloat16*>(ws + L.x_perm) : a_perm;
+    if (!gu || lg) {
+        E4B_CUDA_TRY(launch_gather_rows(bf(x), perm, nrows, d->top_k, P, d->H, xg, st));
+        // s x A_gu^T for dB_gu (recompute mode makes it inside run_gateup)
+        if (gu && (s = lora_thin(d, ws, L, P, xg, d->H, w->lora_A_gu, true, L.lz_gu, st)) != E4B_OK) return s;
+    }
     if (!gu) {   // recompute the gate/up pre-activations (and h) from x
-        E4B_CUDA_TRY(launch_gather_rows(static_cast<const __nv_bfloat16*>(x), perm, nrows, d->top_k, P, d->H, a_perm, st));
         __nv_bfloat16* gu_ws = reinterpret_cast<__nv_bfloat16*>(ws + L.gu);
         __nv_bfloat16* h_ws = reinterpret_cast<__nv_bfloat16*>(ws + L.h);
-        if ((s = run_gateup(d, w, ws, L, topk_w, P, h_ws, gu_ws, st)) != E4B_OK) return s;
+        if ((s = run_gateup(d, w, ws, L, topk_w, P, h_ws, gu_ws, st, xg)) != E4B_OK) return s;
         gu = gu_ws;
         h = h_ws;
     }
-    E4B_CUDA_TRY(launch_gather_rows(static_cast<const __nv_bfloat16*>(grad_out), perm, nrows, d->top_k, P, d->H, a_perm, st));
+    if (lg && (s = lora_thin(d, ws, L, P, h, d->I, w->lora_A_d, true, L.lz_d, st)) != E4B_OK) return s;
+    E4B_CUDA_TRY(launch_gather_rows(bf(grad_out), perm, nrows, d->top_k, P, d->H, a_perm, st));
+    // LoRA: the down^T GEMM's extra stage is s (grad_out B_d) against A_d
+    if (lora && (s = lora_thin(d, ws, L, P, a_perm, d->H, w->lora_B_d, false, L.lv_d, st)) != E4B_OK) return s;
     __nv_bfloat16* dgu = reinterpret_cast<__nv_bfloat16*>(ws + L.dgu);
 
-    // dh = w * grad_out W_down, then the activation backward; with grad_topk_w the
-    // epilogue also leaves <grad_out W_down, h> per row and n-tile
+    // dh = w * grad_out W_down (+ the adapter term), then the activation backward; with
+    // grad_topk_w the epilogue also leaves <grad_out W_down, h> per row and n-tile
     GemmParams p = base_params(d, ws, L, topk_w, P);
     p.K = d->H;
     p.N = d->I;
@@ -416,20 +479,42 @@ e4b_status e4b_moe_backward(const e4b_moe_desc* d, const e4b_experts* w, const v
     p.gu = const_cast<__nv_bfloat16*>(gu);
     p.out_bf16 = dgu;
     p.ld_out = 2 * d->I;
+    p.lora_r = d->lora_rank;
+    p.lora_b = bf(w->lora_A_d);
     float* dw_part = reinterpret_cast<float*>(ws + L.dw_part);
     if (grad_topk_w) {
         p.h_in = h;
         p.dw_part = dw_part;
     }
     E4B_CUDA_TRY(launch_grouped_gemm(EPI_DGRAD_DOWN, d->codebook, a_perm, P, w->down, p.b_rows_total, d->I / 2, p,
-                                     max_m_tiles(P, d->E), st));
-    if (grad_topk_w)   // reads the gathered grad_out rows' source, grad_out itself, before a_perm is reused
-        E4B_CUDA_TRY(launch_router_grad_parts(static_cast<const __nv_bfloat16*>(grad_out), dw_part, dw_tiles(d),
-                                              w->down_bias, inv_perm, topk_idx, topk_w, router_logits, T, d->E,
-                                              d->top_k, d->H, d->renormalize, grad_topk_w, grad_logits, st));
+                                     max_m_tiles(P, d->E), st, lora ? ws + L.lv_d : nullptr));
+    if (grad_topk_w)
+        E4B_CUDA_TRY(launch_router_grad_parts(bf(grad_out), dw_part, dw_tiles(d), w->down_bias, inv_perm, topk_idx,
+                                              topk_w, router_logits, T, d->E, d->top_k, d->H, d->renormalize,
+                                              grad_topk_w, grad_logits, st));
+    if (lg) {   // down adapter: dB_d = sum w g (x) s z_d,  dA_d = sum w s (g B_d) (x) h
+        const __nv_bfloat16* lzd = reinterpret_cast<const __nv_bfloat16*>(ws + L.lz_d);
+        const __nv_bfloat16* lvd = reinterpret_cast<const __nv_bfloat16*>(ws + L.lv_d);
+        E4B_CUDA_TRY(launch_lora_grad(a_perm, d->H, lzd, d->lora_rank, offsets, d->E, topk_w, perm, true, false,
+                                      lora_grads->dB_d, st));
+        E4B_CUDA_TRY(launch_lora_grad(h, d->I, lvd, d->lora_rank, offsets, d->E, topk_w, perm, true, true,
+                                      lora_grads->dA_d, st));
+    }
+    // LoRA: the gate_up^T GEMM's extra stage is s (dGU B_gu) against A_gu
+    if (lora && (grad_x || lg) &&
+        (s = lora_thin(d, ws, L, P, dgu, 2 * d->I, w->lora_B_gu, false, L.lv_gu, st)) != E4B_OK)
+        return s;
+    if (lg) {   // gate_up adapter: dB_gu = sum dGU (x) s z_gu,  dA_gu = sum s (dGU B_gu) (x) x
+        const __nv_bfloat16* lzg = reinterpret_cast<const __nv_bfloat16*>(ws + L.lz_gu);
+        const __nv_bfloat16* lvg = reinterpret_cast<const __nv_bfloat16*>(ws + L.lv_gu);
+        E4B_CUDA_TRY(launch_lora_grad(dgu, 2 * d->I, lzg, d->lora_rank, offsets, d->E, topk_w, perm, false, false,
+                                      lora_grads->dB_gu, st));
+        E4B_CUDA_TRY(launch_lora_grad(xg, d->H, lvg, d->lora_rank, offsets, d->E, topk_w, perm, false, true,
+                                      lora_grads->dA_gu, st));
+    }
     if (!grad_x) return E4B_OK;
 
-    GemmParams q = base_params(d, ws, L, topk_w, P);   // grad_x += [dG, dU] W_gate_up
+    GemmParams q = base_params(d, ws, L, topk_w, P);   // grad_x += [dG, dU] W_gate_up (+ the adapter term)
     q.K = 2 * d->I;
     q.N = d->H;
     q.n_tiles = (d->H + 255) / 256;
@@ -439,8 +524,10 @@ e4b_status e4b_moe_backward(const e4b_moe_desc* d, const e4b_experts* w, const v
     q.b_blocks_per_row = d->H / 64;
     q.out_bf16 = a_perm;   // per-pair rows in grouped order; the gathered grad_out is dead by now
     q.ld_out = d->H;
+    q.lora_r = d->lora_rank;
+    q.lora_b = bf(w->lora_A_gu);
     E4B_CUDA_TRY(launch_grouped_gemm(EPI_DGRAD_GATEUP, d->codebook, dgu, P, w->gate_up, q.b_rows_total, d->H / 2, q,
-                                     max_m_tiles(P, d->E), st));
+                                     max_m_tiles(P, d->E), st, lora ? ws + L.lv_gu : nullptr));
     E4B_CUDA_TRY(launch_combine(a_perm, inv_perm, d->top_k, T, d->H, static_cast<__nv_bfloat16*>(grad_x), st));
     return E4B_OK;
 }
@@ -451,7 +538,7 @@ e4b_status e4b_moe_backward_dgrad(const e4b_moe_desc* d, const e4b_experts* w, c
                                   void* stream) {
     if (T > 0 && !grad_x) return E4B_ERR_INVALID_ARG;
     return e4b_moe_backward(d, w, x, T, nullptr, topk_idx, topk_w, grad_out, saved_gu, nullptr, grad_x, nullptr,
-                            nullptr, workspace, ws_bytes, stream);
+                            nullptr, nullptr, workspace, ws_bytes, stream);
 }
 
 e4b_status e4b_moe_backward_router(const e4b_moe_desc* d, const e4b_experts* w, const void* x, int64_t T,
@@ -460,7 +547,7 @@ e4b_status e4b_moe_backward_router(const e4b_moe_desc* d, const e4b_experts* w, 
                                    size_t ws_bytes, void* stream) {
     e4b_status s = check_desc(d);
     if (s != E4B_OK) return s;
-    if ((s = check_experts(w)) != E4B_OK) return s;
+    if ((s = check_experts(d, w)) != E4B_OK) return s;
     if (T < 0 || T * d->top_k > (int64_t)INT32_MAX) return E4B_ERR_INVALID_ARG;
     if (T == 0) return E4B_OK;
     if (!x || !topk_idx || !topk_w || !grad_out || !grad_topk_w || (grad_logits && !router_logits))
@@ -485,19 +572,7 @@ e4b_status e4b_moe_backward_router(const e4b_moe_desc* d, const e4b_experts* w, 
     if ((s = run_gateup(d, w, ws, L, topk_w, P, h, nullptr, st)) != E4B_OK) return s;
     float* ones = reinterpret_cast<float*>(ws + L.ones);
     E4B_CUDA_TRY(launch_fill_f32(ones, P, 1.0f, st));
-    GemmParams p = base_params(d, ws, L, ones, P);
-    p.K = d->I;
-    p.N = d->H;
-    p.n_tiles = (d->H + 255) / 256;
-    p.absmax = w->down_absmax;
-    p.b_rows_per_expert = d->H;
-    p.b_rows_total = (int64_t)d->E * d->H;
-    p.b_blocks_per_row = d->I / 64;
-    p.out_bf16 = a_perm;   // Y, one grouped row per pair
-    p.bias = w->down_bias;
-    p.ld_out = d->H;
-    E4B_CUDA_TRY(launch_grouped_gemm(EPI_DOWN, d->codebook, h, P, w->down, p.b_rows_total, d->I / 2, p,
-                                     max_m_tiles(P, d->E), st));
+    if ((s = run_down(d, w, ws, L, ones, P, h, a_perm, st)) != E4B_OK) return s;   // Y, one grouped row per pair
     E4B_CUDA_TRY(launch_router_grad(static_cast<const __nv_bfloat16*>(grad_out), a_perm,
                                     reinterpret_cast<const int32_t*>(ws + L.inv_perm), topk_idx, topk_w,
                                     router_logits, T, d->E, d->top_k, d->H, d->renormalize, grad_topk_w, grad_logits,

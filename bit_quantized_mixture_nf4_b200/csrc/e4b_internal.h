@@ -36,6 +36,13 @@ struct GemmParams {
     const __nv_bfloat16* h_in;   // EPI_DGRAD_DOWN, optional: the forward's h [P, I] in grouped order
     float* dw_part;           // with h_in: [P, n_tiles] fp32, row r / n-tile nt: sum over the tile's
                               // columns c of (grad_out_r W_d,e)[c] * h[r, c] (before the routing weight)
+    // Per-expert LoRA as one more 64-deep k-stage: A gets the thin operand [rows, 64] bf16
+    // (the lora_a argument of launch_grouped_gemm), B the adapter: K-major B (gate_up, down)
+    // reads lora_b as [E, b_rows_per_expert, lora_r] (the B_gu / B_d adapter rows), MN-major
+    // B (the two input-gradient GEMMs) as [E, lora_r, N] (A_d / A_gu).  Ranks above lora_r
+    // and rows or columns outside the expert read as 0.  lora_r = 0: no extra stage.
+    const __nv_bfloat16* lora_b;
+    int lora_r;               // 0 or a multiple of 8 up to 64
 };
 
 // launch bookkeeping
@@ -75,9 +82,11 @@ cudaError_t launch_combine(const __nv_bfloat16* rows, const int32_t* inv_perm, i
 
 // grouped_gemm.cu
 int gemm_tile_rows();
+// lora_a: the thin A operand of the LoRA k-stage, [a_rows, 64] bf16 (rank padded with
+// zeros), when p.lora_r > 0; otherwise null.
 cudaError_t launch_grouped_gemm(int epi, int codebook, const void* a, int64_t a_rows, const uint8_t* packed,
                                 int64_t packed_rows_total, int packed_row_bytes, GemmParams p, int max_m_tiles,
-                                cudaStream_t st);
+                                cudaStream_t st, const void* lora_a = nullptr);
 
 // Tiled TMA descriptor of a rank-`rank` tensor (dims innermost first, strides in bytes of
 // dims 1..rank-1); grouped_gemm.cu.

@@ -176,7 +176,7 @@ template <int EPI, int CB, int CTAS, bool XACT = false>
 __global__ void __launch_bounds__(GEMM_THREADS, 1)
 grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_raw,
                     const __grid_constant__ CUtensorMap tmap_out, const __grid_constant__ CUtensorMap tmap_gu,
-                    const GemmParams p) {
+                    const __grid_constant__ CUtensorMap tmap_lora, const GemmParams p) {
     using C = Cfg<CTAS, EPI>;
     constexpr int STAGES = C::STAGES;
     constexpr int ASTAGES = C::ASTAGES;
@@ -245,7 +245,8 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_con
     };
 
     const int total_tiles = __ldg(p.tile_prefix + p.E) * p.n_tiles;
-    const int nk = p.K / BK;
+    const int nk = p.K / BK;              // k-stages of the quantized weights
+    const int nkt = nk + (p.lora_r > 0);  // plus the LoRA stage (the last one of a tile)
 
     if (warp == PRODUCER_WARP) {
         // A tiles: refilled as soon as the MMA has released a stage.  Each tile is also
@@ -259,8 +260,8 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_con
             if (pf_tile < total_tiles) pf_ti = decode_tile(p, pf_tile);
             auto prefetch_next = [&]() {
                 if (pf_tile >= total_tiles) return;
-                tma_prefetch_l2_2d(&tmap_a, pf_ks * BK, pf_ti.row0 + a_off);
-                if (++pf_ks == nk) {
+                if (pf_ks < nk) tma_prefetch_l2_2d(&tmap_a, pf_ks * BK, pf_ti.row0 + a_off);
+                if (++pf_ks == nkt) {
                     pf_ks = 0;
                     pf_tile += nclusters;
                     if (pf_tile < total_tiles) pf_ti = decode_tile(p, pf_tile);
@@ -271,19 +272,22 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_con
             bool ok = true;
             for (int tile = cluster_id; tile < total_tiles && ok; tile += nclusters) {
                 const TileInfo ti = decode_tile(p, tile);
-                for (int ks = 0; ks < nk; ++ks, ++it) {
+                for (int ks = 0; ks < nkt; ++ks, ++it) {
                     prefetch_next();
                     const int s = it % ASTAGES;
                     const uint32_t r = it / ASTAGES;
                     if (!wait(&ctl->a_empty[s], (r & 1) ^ 1)) { ok = false; break; }
                     const uint32_t a_dst = smem_u32(sA + s * C::A_BYTES);
                     const int a_row = ti.row0 + a_off;
+                    // the LoRA stage reads the thin operand [rows, 64] instead of A
+                    const CUtensorMap* am = ks < nk ? &tmap_a : &tmap_lora;
+                    const int ax = ks < nk ? ks * BK : 0;
                     if (CTAS == 2) {
                         if (leader) mbar_arrive_expect_tx(smem_u32(&ctl->a_full[s]), 2 * C::A_BYTES);
-                        tma_load_2d_pair(a_dst, &tmap_a, mapa_shared(smem_u32(&ctl->a_full[s]), 0), ks * BK, a_row);
+                        tma_load_2d_pair(a_dst, am, mapa_shared(smem_u32(&ctl->a_full[s]), 0), ax, a_row);
                     } else {
                         mbar_arrive_expect_tx(smem_u32(&ctl->a_full[s]), C::A_BYTES);
-                        tma_load_2d(a_dst, &tmap_a, smem_u32(&ctl->a_full[s]), ks * BK, a_row);
+                        tma_load_2d(a_dst, am, smem_u32(&ctl->a_full[s]), ax, a_row);
                     }
                 }
             }
@@ -310,13 +314,18 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_con
             }
             const int64_t step = kMajorB ? 1 : (int64_t)BK * p.b_blocks_per_row;
             bool ok = true;
-            for (int ks = 0; ks < nk; ++ks, ++it) {
+            for (int ks = 0; ks < nkt; ++ks, ++it) {
                 const int s = it % RSTAGES;
                 const uint32_t r = it / RSTAGES;
                 if (lane == 0) ok = mbar_wait(smem_u32(&ctl->raw_empty[s]), (r & 1) ^ 1, abort_flag, p.status);
                 ok = __shfl_sync(0xffffffffu, ok, 0);
                 if (!ok) break;
                 const uint32_t rb = smem_u32(&ctl->raw_full[s]);
+                if (ks == nk) {   // the LoRA stage brings no packed weights: the same 1 + 32 arrivals
+                    if (lane == 0) mbar_arrive(rb);
+                    mbar_arrive(rb);
+                    continue;
+                }
                 uint8_t* stage = sRaw + s * C::RAW_STAGE;
                 if (lane == 0) {
                     mbar_arrive_expect_tx(rb, C::RAW_BYTES);
@@ -349,7 +358,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_con
                 if (!wait(&ctl->acc_empty[ab], (ar & 1) ^ 1)) break;
                 tc_fence_after();
                 const uint32_t d_tmem = tmem_base + ab * BN;
-                for (int ks = 0; ks < nk; ++ks, ++it) {
+                for (int ks = 0; ks < nkt; ++ks, ++it) {
                     const int s = it % STAGES, sa = it % ASTAGES;
                     const uint32_t r = it / STAGES, ra = it / ASTAGES;
                     if (!wait(&ctl->a_full[sa], ra & 1) || !wait(&ctl->b_full[s], r & 1)) { ok = false; break; }
@@ -390,8 +399,8 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_con
         uint32_t it = grp;
         int tile = cluster_id, ks = grp;
         auto normalize = [&]() {   // carry ks past the end of a tile into the next tile(s)
-            while (ks >= nk && tile < total_tiles) {
-                ks -= nk;
+            while (ks >= nkt && tile < total_tiles) {
+                ks -= nkt;
                 tile += nclusters;
             }
         };
@@ -399,11 +408,55 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_con
         while (tile < total_tiles) {
             const int s = it % STAGES;
             const uint32_t r = it / STAGES;
+            const int cur_tile = tile, cur_ks = ks;
             ks += C::DEQ_GROUPS;   // this group's next stage
             normalize();
             const int rs = it % RSTAGES;
             const uint32_t rr = it / RSTAGES;
             if (!mbar_wait(smem_u32(&ctl->raw_full[rs]), rr & 1, abort_flag, p.status)) break;
+            if (cur_ks == nk) {
+                // LoRA stage: the adapter tile in bf16 straight from global memory, in the
+                // same shared-memory layout as a dequantized tile
+                __syncwarp();
+                if (lane == 0) mbar_arrive(smem_u32(&ctl->raw_empty[rs]));
+                if (!wait(&ctl->empty[s], (r & 1) ^ 1)) break;
+                const TileInfo ti = decode_tile(p, cur_tile);
+                uint8_t* dst_tile = sB + s * C::B_BYTES;
+#pragma unroll
+                for (int i = 0; i < NB; ++i) {
+                    const int b = tg + TPG * i;
+                    const __nv_bfloat16* src = nullptr;   // 64 consecutive bf16 of the tile row b, or null
+                    int nvalid = 0;                        // of which the first nvalid are in range
+                    if (kMajorB) {   // row b of this CTA's half; the adapter's r values, zeros after
+                        const int n = (int)rank * C::N_CTA + b;
+                        const int row = kmajor_row<EPI>(p, ti.nt, n);
+                        const bool in = (EPI == EPI_GATEUP) ? (ti.nt * 128 + (n & 127) < p.up_offset)
+                                                            : (row < p.b_rows_per_expert);
+                        if (in) {
+                            src = p.lora_b + ((int64_t)ti.e * p.b_rows_per_expert + row) * p.lora_r;
+                            nvalid = p.lora_r;
+                        }
+                    } else {         // k-row q = b & 63 (the rank index), columns of block b >> 6
+                        const int q = b & 63, col = ti.nt * BN + (int)rank * C::N_CTA + (b >> 6) * 64;
+                        if (q < p.lora_r && col < p.N) {
+                            src = p.lora_b + ((int64_t)ti.e * p.lora_r + q) * p.N + col;
+                            nvalid = min(64, p.N - col);
+                        }
+                    }
+#pragma unroll
+                    for (int c = 0; c < 8; ++c) {
+                        uint4 v = make_uint4(0u, 0u, 0u, 0u);
+                        if (src && 8 * c < nvalid) v = __ldg(reinterpret_cast<const uint4*>(src) + c);
+                        const uint32_t off = kMajorB ? sw128_offset(b, c) : (b >> 6) * 8192 + sw128_offset(b & 63, c);
+                        *reinterpret_cast<uint4*>(dst_tile + off) = v;
+                    }
+                }
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) arrive_leader(&ctl->b_full[s]);
+                it += C::DEQ_GROUPS;
+                continue;
+            }
             const uint8_t* raw_stage = sRaw + rs * C::RAW_STAGE;
             const float* am = reinterpret_cast<const float*>(raw_stage + C::RAW_BYTES);
             uint4 pk[NB][2];
@@ -816,7 +869,8 @@ int gemm_tile_rows() { return Cfg<kCtas>::TILE_M; }
 
 template <int EPI, int CB, bool XACT = false>
 static cudaError_t launch_one(const CUtensorMap& ma, const CUtensorMap& mr, const CUtensorMap& mo,
-                              const CUtensorMap& mg, const GemmParams& p, int grid, cudaStream_t st) {
+                              const CUtensorMap& mg, const CUtensorMap& ml, const GemmParams& p, int grid,
+                              cudaStream_t st) {
     using C = Cfg<kCtas, EPI>;
     auto kern = grouped_gemm_kernel<EPI, CB, kCtas, XACT>;
     // The shared-memory limit is a per-device function attribute: set it once per
@@ -848,7 +902,7 @@ static cudaError_t launch_one(const CUtensorMap& ma, const CUtensorMap& mr, cons
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     timing_begin(KK_GEMM_GATEUP + EPI, st);
-    cudaError_t e = cudaLaunchKernelEx(&cfg, kern, ma, mr, mo, mg, p);
+    cudaError_t e = cudaLaunchKernelEx(&cfg, kern, ma, mr, mo, mg, ml, p);
     timing_end(KK_GEMM_GATEUP + EPI, st);
     count_launch();
     if (e != cudaSuccess) return e;
@@ -857,7 +911,7 @@ static cudaError_t launch_one(const CUtensorMap& ma, const CUtensorMap& mr, cons
 
 cudaError_t launch_grouped_gemm(int epi, int codebook, const void* a, int64_t a_rows, const uint8_t* packed,
                                 int64_t packed_rows_total, int packed_row_bytes, GemmParams p, int max_m_tiles,
-                                cudaStream_t st) {
+                                cudaStream_t st, const void* lora_a) {
     using C = Cfg<kCtas>;
     CUtensorMap ma, mr;
     if (!make_map_2d(&ma, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a, (uint64_t)p.K, (uint64_t)a_rows, (uint64_t)p.K * 2, 64,
@@ -886,18 +940,26 @@ cudaError_t launch_grouped_gemm(int epi, int codebook, const void* a, int64_t a_
         !make_map_2d(&mg, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, p.gu, (uint64_t)n_feat * 2, (uint64_t)a_rows,
                      (uint64_t)n_feat * 4, 32, 32, CU_TENSOR_MAP_SWIZZLE_64B))
         return cudaErrorInvalidValue;
+    // the LoRA stage's thin A operand [rows, 64] bf16: one 64-deep box per tile row block
+    CUtensorMap ml = ma;
+    if (p.lora_r > 0) {
+        if (!lora_a || !p.lora_b || p.lora_r % 8 || p.lora_r > 64 ||
+            !make_map_2d(&ml, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, lora_a, 64, (uint64_t)a_rows, 128, 64, 128,
+                         CU_TENSOR_MAP_SWIZZLE_128B))
+            return cudaErrorInvalidValue;
+    }
     const int64_t tiles = (int64_t)max_m_tiles * p.n_tiles;
     const int grid = (int)std::min<int64_t>(tiles * kCtas, (num_sms() / kCtas) * kCtas);
     if (grid <= 0) return cudaSuccess;
-#define E4B_LAUNCH(E_, C_) return launch_one<E_, C_>(ma, mr, mo, mg, p, grid, st)
+#define E4B_LAUNCH(E_, C_) return launch_one<E_, C_>(ma, mr, mo, mg, ml, p, grid, st)
     if (epi == EPI_GATEUP && (p.act != 0 || p.bias != nullptr)) {
-        if (codebook == 0) return launch_one<EPI_GATEUP, 0, true>(ma, mr, mo, mg, p, grid, st);
-        return launch_one<EPI_GATEUP, 1, true>(ma, mr, mo, mg, p, grid, st);
+        if (codebook == 0) return launch_one<EPI_GATEUP, 0, true>(ma, mr, mo, mg, ml, p, grid, st);
+        return launch_one<EPI_GATEUP, 1, true>(ma, mr, mo, mg, ml, p, grid, st);
     }
     if (epi == EPI_DGRAD_DOWN && p.dw_part) {
         if (!p.h_in) return cudaErrorInvalidValue;
-        if (codebook == 0) return launch_one<EPI_DGRAD_DOWN, 0, true>(ma, mr, mo, mg, p, grid, st);
-        return launch_one<EPI_DGRAD_DOWN, 1, true>(ma, mr, mo, mg, p, grid, st);
+        if (codebook == 0) return launch_one<EPI_DGRAD_DOWN, 0, true>(ma, mr, mo, mg, ml, p, grid, st);
+        return launch_one<EPI_DGRAD_DOWN, 1, true>(ma, mr, mo, mg, ml, p, grid, st);
     }
     if (codebook == 0) {
         switch (epi) {

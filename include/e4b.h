@@ -75,16 +75,20 @@ typedef enum { E4B_ACT_SWIGLU = 0, E4B_ACT_CLAMPED_GLU = 1 } e4b_activation;
 /* Layer description.  H and I must be multiples of 64 (blocks never straddle a
  * row, [P4] __init__); 1 <= top_k <= min(E, 8); E <= 256; blocksize == 64.
  * path: AUTO takes the weight-streaming decode kernels for T <= 8 when no
- * grouped outputs are requested and the kernels' shared-memory stages fit
- * (8 rows of H and 16 rows of I elements plus the h rows of one expert's
- * tokens: H up to about 16000, I up to about 2900 with caller-given routing
- * and about 6000 at T = 1 with routing from logits), and the grouped
- * tensor-core kernels otherwise; the other values force one path (DECODE
- * outside that range returns E4B_ERR_UNSUPPORTED).  The decode kernels implement
- * SwiGLU without biases only: AUTO takes the grouped kernels for the clamped GLU
- * or biased experts at every T, and DECODE returns E4B_ERR_UNSUPPORTED for them.
+ * grouped outputs are requested and the shapes fit them (H <= 8192, and the
+ * per-warp stage rings of 16 rows plus the tokens' activation rows fit in
+ * shared memory), and the grouped tensor-core kernels otherwise; the other
+ * values force one path (DECODE outside that range returns
+ * E4B_ERR_UNSUPPORTED).  The decode kernels implement SwiGLU without biases or
+ * adapters only: AUTO takes the grouped kernels for the clamped GLU, biased
+ * experts or LoRA at every T, and DECODE returns E4B_ERR_UNSUPPORTED for them.
  * activation: E4B_ACT_SWIGLU (zero-initialised descriptors) or
- * E4B_ACT_CLAMPED_GLU with glu_alpha finite and glu_limit > 0 (+inf allowed). */
+ * E4B_ACT_CLAMPED_GLU with glu_alpha finite and glu_limit > 0 (+inf allowed).
+ * lora_rank: 0 (no adapters; zero-initialised descriptors) or the rank r of the
+ * per-expert LoRA adapters in e4b_experts, a multiple of 8 up to 64 ([P1]
+ * "ExpertsLoRA(base, r, alpha)": the base stays frozen, only the adapters
+ * train); lora_scale = alpha / r multiplies each adapter update:
+ *   gate_up pre-activations += s (x A_gu^T) B_gu^T,  expert output += s (h A_d^T) B_d^T. */
 typedef struct {
     int E, H, I, top_k;
     int renormalize;           /* divide the selected softmax weights by their sum  */
@@ -93,13 +97,17 @@ typedef struct {
     e4b_path path;
     e4b_activation activation;
     float glu_alpha, glu_limit;   /* E4B_ACT_CLAMPED_GLU only */
+    int lora_rank;                /* 0, or 8, 16, ..., 64 */
+    float lora_scale;             /* alpha / r, finite */
 } e4b_moe_desc;
 
-/* Device pointers to the two quantized stacks (see storage above) and the
+/* Device pointers to the two quantized stacks (see storage above), the
  * optional per-expert biases ([P2] gpt-oss experts; NULL = none): gate_up_bias
  * is added to the gate_up pre-activations (gate half first, like the rows),
- * down_bias to each expert's output before its routing weight multiplies it.
- * Bias pointers are 16-byte aligned. */
+ * down_bias to each expert's output before its routing weight multiplies it;
+ * and, when the descriptor's lora_rank r > 0, the four bf16 LoRA adapters of
+ * every expert (stacked [E, r, in] / [E, out, r] as in [P2] "Prior art"; all
+ * four required then, ignored otherwise).  Pointers are 16-byte aligned. */
 typedef struct {
     const uint8_t *gate_up;        /* [E, 2I*H/2] */
     const uint8_t *down;           /* [E, H*I/2]  */
@@ -107,7 +115,17 @@ typedef struct {
     const float *down_absmax;      /* [E, H*I/64]  */
     const float *gate_up_bias;     /* fp32 [E, 2I] or NULL */
     const float *down_bias;        /* fp32 [E, H] or NULL  */
+    const void *lora_A_gu;         /* bf16 [E, r, H]  */
+    const void *lora_B_gu;         /* bf16 [E, 2I, r] (gate rows first, like the stack) */
+    const void *lora_A_d;          /* bf16 [E, r, I]  */
+    const void *lora_B_d;          /* bf16 [E, H, r]  */
 } e4b_experts;
+
+/* Gradients of the four adapters (fp32, shaped like them; each fully written),
+ * summed over every routed pair of the expert. */
+typedef struct {
+    float *dA_gu, *dB_gu, *dA_d, *dB_d;
+} e4b_lora_grads;
 
 /* Blockwise 4-bit quantization ([P4] from_float / _quantize_stack).
  * w: fp32 [E, out, in].  For every 64-element block of each row: absmax =
@@ -184,13 +202,21 @@ E4B_API e4b_status e4b_moe_forward(const e4b_moe_desc *d, const e4b_experts *w, 
  *   x bf16 [T,H] (read only when saved_gu is NULL); router_logits fp32 [T,E]
  *   (needed only for grad_logits); topk_idx, topk_w, grad_out as for
  *   e4b_moe_backward_dgrad; workspace: e4b_moe_workspace_size(d, T) bytes.
- * Returns E4B_ERR_INVALID_ARG when no output is asked for, when grad_topk_w is
- * asked for with saved_gu but without saved_h, or when grad_logits is asked for
- * without router_logits or grad_topk_w. */
+ * With adapters (d->lora_rank > 0), every gradient includes their updates, and
+ * lora_grads (or NULL) receives the adapter gradients, with s = lora_scale, dY =
+ * w grad_out_t, z_gu = x A_gu^T, z_d = h A_d^T:
+ *   dB_d += s dY (x) z_d,   dA_d += s (dY B_d) (x) h,
+ *   dB_gu += s dGU (x) z_gu,  dA_gu += s (dGU B_gu) (x) x      (dGU = [dG | dU]).
+ * lora_grads needs x (and h: saved_h, or recompute mode).
+ * Returns E4B_ERR_INVALID_ARG when no output is asked for, when grad_topk_w or
+ * lora_grads is asked for with saved_gu but without saved_h, when lora_grads is
+ * asked for without x, or when grad_logits is asked for without router_logits or
+ * grad_topk_w. */
 E4B_API e4b_status e4b_moe_backward(const e4b_moe_desc *d, const e4b_experts *w, const void *x, int64_t T,
                             const float *router_logits, const int32_t *topk_idx, const float *topk_w,
                             const void *grad_out, const void *saved_gu, const void *saved_h,
                             void *grad_x, float *grad_topk_w, float *grad_logits,
+                            const e4b_lora_grads *lora_grads,
                             void *workspace, size_t ws_bytes, void *stream);
 
 /* Input gradient of the forward with routing held constant ([P5] "What this

@@ -102,7 +102,7 @@ def test_host_side_validation(lib):
     # the fused layer backward: argument rules, checked before any launch
     def b(T, x=16, logits=None, saved_gu=16, saved_h=16, gx=16, gw=16, gl=None):
         return L.e4b_moe_backward(ctypes.byref(d), ctypes.byref(ex2), x, T, logits, 16, 16, 16, saved_gu, saved_h,
-                                  gx, gw, gl, None, 0, None)
+                                  gx, gw, gl, None, None, 0, None)
     assert b(0) == lib.E4B_OK                                           # T == 0: no-op
     assert b(4, gx=None, gw=None) == lib.E4B_ERR_INVALID_ARG           # no output asked for
     assert b(4, x=None, saved_gu=None) == lib.E4B_ERR_INVALID_ARG      # nothing to recompute from
@@ -110,6 +110,21 @@ def test_host_side_validation(lib):
     assert b(4, gl=16) == lib.E4B_ERR_INVALID_ARG                      # grad_logits needs router_logits
     assert b(4, logits=16, gw=None, gl=16) == lib.E4B_ERR_INVALID_ARG  # ... and grad_topk_w
     assert b(4) == lib.E4B_ERR_WORKSPACE                               # valid request, no workspace
+    # LoRA: rank a multiple of 8 up to 64, finite scale, all four adapters present
+    for bad in (lib.make_desc(8, 256, 512, 2, lora_rank=12), lib.make_desc(8, 256, 512, 2, lora_rank=72),
+                lib.make_desc(8, 256, 512, 2, lora_rank=-8),
+                lib.make_desc(8, 256, 512, 2, lora_rank=16, lora_scale=float("nan"))):
+        assert lib.e4b_moe_workspace_size(bad, 64) == 0
+    ld = lib.make_desc(8, 256, 512, 2, lora_rank=16, lora_scale=2.0)
+    assert lib.e4b_moe_workspace_size(ld, 64) > lib.e4b_moe_workspace_size(d, 64)   # the thin operands
+    assert f(ld, 4, 16, 16, 1 << 40) == lib.E4B_ERR_INVALID_ARG       # adapters missing
+    exl = lib.e4b_experts(16, 16, 16, 16, None, None, 16, 16, 16, 16)
+    ldec = lib.make_desc(8, 256, 512, 2, path=lib.PATH_DECODE, lora_rank=16, lora_scale=2.0)
+    assert L.e4b_moe_forward(ctypes.byref(ldec), ctypes.byref(exl), 16, 2, None, 16, 16, 16, None, None, None, None,
+                             16, 1 << 40, None) == lib.E4B_ERR_UNSUPPORTED   # decode kernels take no adapters
+    gl = lib.e4b_lora_grads(16, 16, 16, 16)
+    assert L.e4b_moe_backward(ctypes.byref(ld), ctypes.byref(exl), None, 4, None, 16, 16, 16, 16, 16, 16, None, None,
+                              ctypes.byref(gl), None, 0, None) == lib.E4B_ERR_INVALID_ARG   # adapter grads need x
 
 
 def test_pipe_host_side_validation(lib):
