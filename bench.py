@@ -52,7 +52,7 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-aux", action="store_true", help="skip the secondary legs")
-    ap.add_argument("--leg", default="step", choices=["step", "decode", "codec", "variant", "router"],
+    ap.add_argument("--leg", default="step", choices=["step", "decode", "codec", "variant", "router", "lora"],
                     help="step: the benchmark line; decode / codec / variant / router: only that secondary leg "
                          "(for profiling); decode runs the Qwen3-shaped layer (or --workload) at --tokens "
                          "(default 1); router runs the routing-gradient legs on --workload")
@@ -221,7 +221,7 @@ class Layer:
     """One quantized layer on the device with its seeded inputs (drawn on the host,
     so the CPU oracle can be fed the same values) and output buffers."""
 
-    def __init__(self, w, dev, path=0, act=0, biases=False):
+    def __init__(self, w, dev, path=0, act=0, biases=False, lora_rank=0):
         import torch
         import bit_quantized_mixture_nf4_b200 as e4b
         from bit_quantized_mixture_nf4_b200 import workloads as wl
@@ -239,8 +239,19 @@ class Layer:
             g.manual_seed(w.seed + 7)
             self.bgu = torch.randn(w.E, 2 * w.I, device=dev, generator=g) * 0.3
             self.bd = torch.randn(w.E, w.H, device=dev, generator=g) * 0.3
-        self.experts = e4b.make_experts(self.pg, self.pd, self.ag, self.ad, self.bgu, self.bd)
-        self.desc = e4b.make_desc(w.E, w.H, w.I, w.k, w.renorm, w.codebook, 64, path, act, 1.702, 7.0)
+        self.lora = self.lora_grads = None
+        if lora_rank:   # per-expert adapters (A ~ N(0, 1/in), B ~ N(0, 0.01/r)), bf16
+            g = torch.Generator(device=dev)
+            g.manual_seed(w.seed + 11)
+            r = lora_rank
+            shapes = ((w.E, r, w.H, 1 / w.H), (w.E, 2 * w.I, r, 0.01 / r), (w.E, r, w.I, 1 / w.I),
+                      (w.E, w.H, r, 0.01 / r))
+            self.lora = tuple((torch.randn(a, b, c, device=dev, generator=g) * v ** 0.5).to(torch.bfloat16)
+                              for a, b, c, v in shapes)
+            self.lora_grads = tuple(torch.empty(t.shape, dtype=torch.float32, device=dev) for t in self.lora)
+        self.experts = e4b.make_experts(self.pg, self.pd, self.ag, self.ad, self.bgu, self.bd, lora=self.lora)
+        self.desc = e4b.make_desc(w.E, w.H, w.I, w.k, w.renorm, w.codebook, 64, path, act, 1.702, 7.0,
+                                  lora_rank=lora_rank, lora_scale=2.0)
         T, P = w.T, w.P
         self.x = self.x_h.to(dev)
         self.logits = self.logits_h.to(dev)
@@ -269,10 +280,11 @@ class Layer:
         import bit_quantized_mixture_nf4_b200 as e4b
         e4b.e4b_moe_forward(self.desc, self.experts, self.x, self.logits, self.idx, self.wts, self.y,
                             saved_gu=self.saved, ws=self.ws, stream=stream, saved_h=self.saved_h)
-        if self.routing:
+        if self.routing or self.lora is not None:
             e4b.e4b_moe_backward(self.desc, self.experts, self.x, self.idx, self.wts, self.go, saved_gu=self.saved,
-                                 saved_h=self.saved_h, router_logits=self.logits, grad_x=self.gx,
-                                 grad_topk_w=self.dwt, grad_logits=self.dlg, ws=self.ws, stream=stream)
+                                 saved_h=self.saved_h, router_logits=self.logits if self.routing else None,
+                                 grad_x=self.gx, grad_topk_w=self.dwt, grad_logits=self.dlg,
+                                 want_routing=self.routing, lora_grads=self.lora_grads, ws=self.ws, stream=stream)
         else:
             e4b.e4b_moe_backward_dgrad(self.desc, self.experts, self.x, self.idx, self.wts, self.go,
                                        saved_gu=self.saved, grad_x=self.gx, ws=self.ws, stream=stream)
@@ -502,6 +514,38 @@ def router_fused_leg(layer, flush, steps=10):
             "extra_bytes_per_step": extra_bytes, "roofline": roof,
             "work": "forward saves h; e4b_moe_backward: the down^T GEMM epilogue leaves <grad_out W_d, h> per "
                     "row and 256-column tile, a per-token kernel sums them and runs the softmax backward"}
+
+
+def lora_leg(w, dev, flush, rank=16, steps=10):
+    """The training step with per-expert LoRA adapters of rank r on both stacks:
+    forward (saving g/u and h) + the one-pass backward with the input gradient and
+    the four adapter gradients, against the same step of the base layer alone."""
+    import torch
+    _, bf16, _, src = peaks()
+    stream = torch.cuda.current_stream()
+    base = Layer(w, dev)
+    ms0, _, _ = timed_steps(base, steps, 3, flush, stream, kinds=())
+    del base
+    torch.cuda.empty_cache()
+    layer = Layer(w, dev, lora_rank=rank)
+    layer.saved_h = torch.empty(w.P, w.I, dtype=torch.bfloat16, device=dev)
+    ms1, _, _ = timed_steps(layer, steps, 3, flush, stream, kinds=())
+    del layer
+    torch.cuda.empty_cache()
+    s0, s1 = step_stats(ms0), step_stats(ms1)
+    base_flops = 12 * w.H * w.I * w.P
+    # adapter work: the extra 64-deep k-stage in the four GEMMs (rank padded to 64), the
+    # four thin projections and the four adapter gradients (2 FLOP per multiply-add)
+    k64 = 2 * w.P * 64 * (2 * w.I + w.H + w.I + w.H)
+    thin = 2 * w.P * rank * (w.H + w.I + w.H + 2 * w.I)
+    grads = 2 * w.P * rank * (w.H + w.I + 2 * w.I + w.H)
+    tf = base_flops / (s1["median"] / 1e3) / 1e12
+    return {"workload": workload_desc(w).replace("+ dgrad", f"+ dgrad, LoRA r={rank} on both stacks"),
+            "step_ms_base": s0, "step_ms_lora": s1, "added_frac": s1["median"] / s0["median"] - 1.0,
+            "tokens_per_s": w.T / (s1["median"] / 1e3), "adapter_flops_per_step": k64 + thin + grads,
+            "roofline": {"bound": "tensor", "achieved": tf, "peak": bf16, "unit": "TFLOP/s", "frac": tf / bf16,
+                         "basis": "base-layer FLOP (12 H I per pair) / LoRA step time",
+                         "peak_kind": f"{src} bf16 dense (burst)"}}
 
 
 def codec_leg(w, dev, reps=10):
@@ -797,6 +841,7 @@ def run_e4b(args, w):
             if v.name != w.name:
                 legs[f"{v.name}_T{v.T}"] = step_leg(v, dev, flush)
         aux["large_layers"] = legs
+        aux["lora"] = lora_leg(wl.OLMOE, dev, flush)
         aux["decode"] = [decode_leg(v, dev) for v in (wl.QWEN3.with_tokens(1), wl.QWEN3.with_tokens(2),
                                                       wl.QWEN3.with_tokens(4), wl.QWEN3.with_tokens(8),
                                                       wl.GPTOSS.with_tokens(1))]
@@ -847,6 +892,9 @@ def main():
             tokens = args.tokens if 0 < args.tokens <= 8 else 1
             base = wl.QWEN3 if args.workload == "mixtral" else wl.ALL[args.workload]   # decode: Qwen3 by default
             print(json.dumps(decode_leg(base.with_tokens(tokens), dev, reps=max(args.steps, 3))), flush=True)
+        elif args.leg == "lora":
+            w = headline_workload(args)
+            print(json.dumps(lora_leg(w, dev, flush, steps=max(args.steps, 3))), flush=True)
         elif args.leg == "router":
             w = headline_workload(args)
             layer = Layer(w, dev)

@@ -99,7 +99,7 @@ uint32_t* device_status_ptr() {
 // ------------------------------------------------------------ workspace layout
 struct WsLayout {
     size_t chunk_counts, chunk_base, counts, offsets, tile_prefix, sched, perm, inv_perm, a_perm, h, gu, dgu, dec, ones,
-        dw_part, lz_gu, lz_d, lv_d, lv_gu, x_perm, total;
+        dw_part, lz_gu, lz_d, lv_d, lv_gu, x_perm, lbt_gu, lbt_d, total;
 };
 
 static size_t align_up(size_t v) { return (v + 255) & ~size_t(255); }
@@ -135,6 +135,8 @@ static WsLayout layout_for(const e4b_moe_desc* d, int64_t T) {
         L.lv_d = take((size_t)P * 64 * 2);
         L.lv_gu = take((size_t)P * 64 * 2);
         L.x_perm = take((size_t)P * d->H * 2);
+        L.lbt_gu = take((size_t)d->E * d->lora_rank * 2 * d->I * 2);   // B_gu as [E, r, 2I]
+        L.lbt_d = take((size_t)d->E * d->lora_rank * d->H * 2);        // B_d as [E, r, H]
     }
     L.total = off;
     return L;
@@ -462,8 +464,12 @@ e4b_status e4b_moe_backward(const e4b_moe_desc* d, const e4b_experts* w, const v
     }
     if (lg && (s = lora_thin(d, ws, L, P, h, d->I, w->lora_A_d, true, L.lz_d, st)) != E4B_OK) return s;
     E4B_CUDA_TRY(launch_gather_rows(bf(grad_out), perm, nrows, d->top_k, P, d->H, a_perm, st));
-    // LoRA: the down^T GEMM's extra stage is s (grad_out B_d) against A_d
-    if (lora && (s = lora_thin(d, ws, L, P, a_perm, d->H, w->lora_B_d, false, L.lv_d, st)) != E4B_OK) return s;
+    // LoRA: the down^T GEMM's extra stage is s (grad_out B_d) against A_d (B_d transposed first)
+    if (lora) {
+        E4B_CUDA_TRY(launch_lora_transpose(bf(w->lora_B_d), d->E, d->H, d->lora_rank,
+                                           reinterpret_cast<__nv_bfloat16*>(ws + L.lbt_d), st));
+        if ((s = lora_thin(d, ws, L, P, a_perm, d->H, ws + L.lbt_d, true, L.lv_d, st)) != E4B_OK) return s;
+    }
     __nv_bfloat16* dgu = reinterpret_cast<__nv_bfloat16*>(ws + L.dgu);
 
     // dh = w * grad_out W_down (+ the adapter term), then the activation backward; with
@@ -501,9 +507,11 @@ e4b_status e4b_moe_backward(const e4b_moe_desc* d, const e4b_experts* w, const v
                                       lora_grads->dA_d, st));
     }
     // LoRA: the gate_up^T GEMM's extra stage is s (dGU B_gu) against A_gu
-    if (lora && (grad_x || lg) &&
-        (s = lora_thin(d, ws, L, P, dgu, 2 * d->I, w->lora_B_gu, false, L.lv_gu, st)) != E4B_OK)
-        return s;
+    if (lora && (grad_x || lg)) {
+        E4B_CUDA_TRY(launch_lora_transpose(bf(w->lora_B_gu), d->E, 2 * d->I, d->lora_rank,
+                                           reinterpret_cast<__nv_bfloat16*>(ws + L.lbt_gu), st));
+        if ((s = lora_thin(d, ws, L, P, dgu, 2 * d->I, ws + L.lbt_gu, true, L.lv_gu, st)) != E4B_OK) return s;
+    }
     if (lg) {   // gate_up adapter: dB_gu = sum dGU (x) s z_gu,  dA_gu = sum s (dGU B_gu) (x) x
         const __nv_bfloat16* lzg = reinterpret_cast<const __nv_bfloat16*>(ws + L.lz_gu);
         const __nv_bfloat16* lvg = reinterpret_cast<const __nv_bfloat16*>(ws + L.lv_gu);

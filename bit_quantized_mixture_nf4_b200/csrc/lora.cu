@@ -7,76 +7,153 @@
 // padded to 64 with zeros, bf16) against the adapter B.  The two input
 // gradients take s (dy B) against A the same way.  The kernels here make those
 // thin operands and the four adapter gradients, which are sums over each
-// expert's rows in grouped order (a fixed order: deterministic).
+// expert's rows in grouped order (a fixed order: deterministic).  Both are
+// small-N contractions (N = r <= 64): mma.sync m16n8k16 tiles fed from
+// cp.async-staged shared memory, fp32 accumulation.
+#include <mutex>
+
 #include "lora.h"
 
 namespace e4b {
 
-// out[row, q] = s * sum_c in[row, c] * M_e(q, c) for the rows of one m-tile (one
-// expert), q < r; columns r..63 of out are zero.  M_e(q, c) = m[e][q][c]
-// (Q_MAJOR, an A adapter [E, r, K]) or m[e][c][q] (a B adapter [E, K, r]).
-// One thread per row; the adapter goes through shared memory in chunks of 64
-// columns of K as fp32 [64][r].
+namespace {
+
+__device__ __forceinline__ void mma16816(float d[4], const uint32_t a[4], uint32_t b0, uint32_t b1) {
+    asm("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+        "{%0,%1,%2,%3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+__device__ __forceinline__ void ldsm_x4(uint32_t r[4], uint32_t addr) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]) : "r"(addr));
+}
+__device__ __forceinline__ void ldsm_x4_t(uint32_t r[4], uint32_t addr) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]) : "r"(addr));
+}
+__device__ __forceinline__ void ldsm_x2(uint32_t& r0, uint32_t& r1, uint32_t addr) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x2.shared.b16 {%0,%1}, [%2];" : "=r"(r0), "=r"(r1) : "r"(addr));
+}
+__device__ __forceinline__ void ldsm_x2_t(uint32_t& r0, uint32_t& r1, uint32_t addr) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x2.trans.shared.b16 {%0,%1}, [%2];" : "=r"(r0), "=r"(r1) : "r"(addr));
+}
+// 16-byte copy global -> shared; src_bytes = 0 fills zeros
+__device__ __forceinline__ void cp16z(uint32_t dst, const void* src, uint32_t src_bytes) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_bytes) : "memory");
+}
+__device__ __forceinline__ void cp_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void cp_wait1() { asm volatile("cp.async.wait_group 1;" ::: "memory"); }
+
+constexpr int THIN_ROWS = 256, THIN_SA = 72;   // rows per CTA (8 warps x 32); smem row stride (bf16)
+constexpr int THIN_SMEM = 2 * (THIN_ROWS + 64) * THIN_SA * 2;
+constexpr int GR_P = 32, GR_A = 128, GR_SU = GR_A + 8, GR_SV = 72;   // rows per chunk, columns per CTA
+
+}  // namespace
+
+// out[row, q] = s * sum_k in[row, k] * M_e(q, k) for the rows of one m-tile (one
+// expert, up to 256 rows), q < r; columns r..63 of out are zero.  M_e(q, k) =
+// m[e][q][k] (Q_MAJOR, an A adapter [E, r, K]) or m[e][k][q] (a B adapter
+// [E, K, r]).  K in chunks of 64, double-buffered: the rows' chunk and M_e's
+// chunk as [q][k] in shared memory; warp w owns rows 32w..32w+31 (two m16 tiles).
 template <bool Q_MAJOR>
 __global__ void __launch_bounds__(256) lora_thin_kernel(const __nv_bfloat16* __restrict__ in, int K,
                                                         const __nv_bfloat16* __restrict__ m, int r, float s,
                                                         const int4* __restrict__ sched,
                                                         const int* __restrict__ tile_prefix, int E,
                                                         __nv_bfloat16* __restrict__ out) {
-    __shared__ __align__(16) float ms[64 * 64];
+    extern __shared__ __align__(16) uint8_t sm[];
     const int mt = blockIdx.x;
     if (mt >= __ldg(tile_prefix + E)) return;
     const int4 tl = __ldg(sched + mt);   // (expert, first row, rows, 0)
-    const int e = tl.x, row = tl.y + (int)threadIdx.x;
-    const bool valid = (int)threadIdx.x < tl.z;
-    float acc[64];
-#pragma unroll
-    for (int q = 0; q < 64; ++q) acc[q] = 0.0f;
+    const int e = tl.x, row0 = tl.y, rows = tl.z;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    __nv_bfloat16* sA = reinterpret_cast<__nv_bfloat16*>(sm);                 // [2][256][72]
+    __nv_bfloat16* sM = sA + 2 * THIN_ROWS * THIN_SA;                         // [2][64][72]
     const __nv_bfloat16* me = m + (int64_t)e * r * K;
-    const uint4* xin = reinterpret_cast<const uint4*>(in + (int64_t)row * K);
-    for (int c0 = 0; c0 < K; c0 += 64) {
+    const int nch = K / 64;
+    auto stage = [&](int c, int b) {
+        __nv_bfloat16* a = sA + b * THIN_ROWS * THIN_SA;
+        for (int i = tid; i < THIN_ROWS * 8; i += 256) {
+            const int rr = i >> 3, sg = i & 7;
+            const bool ok = rr < rows;
+            cp16z(smem_u32(a + rr * THIN_SA + sg * 8), in + (int64_t)(row0 + (ok ? rr : 0)) * K + c * 64 + sg * 8,
+                  ok ? 16u : 0u);
+        }
+        __nv_bfloat16* mm = sM + b * 64 * THIN_SA;
+        if (Q_MAJOR) {
+            for (int i = tid; i < 64 * 8; i += 256) {
+                const int q = i >> 3, sg = i & 7;
+                const bool ok = q < r;
+                cp16z(smem_u32(mm + q * THIN_SA + sg * 8), me + (int64_t)(ok ? q : 0) * K + c * 64 + sg * 8,
+                      ok ? 16u : 0u);
+            }
+        } else {   // m[e][k][q]: transposed through registers, zeros past r
+            for (int i = tid; i < 64 * 8; i += 256) {
+                const int k = i >> 3, q0 = (i & 7) * 8;
+                uint4 v = make_uint4(0u, 0u, 0u, 0u);
+                if (q0 < r) v = __ldg(reinterpret_cast<const uint4*>(me + (int64_t)(c * 64 + k) * r + q0));
+                const __nv_bfloat16* hv = reinterpret_cast<const __nv_bfloat16*>(&v);
+#pragma unroll
+                for (int j = 0; j < 8; ++j) mm[(q0 + j) * THIN_SA + k] = hv[j];
+            }
+        }
+        cp_commit();
+    };
+    float acc[2][8][4];
+#pragma unroll
+    for (int i = 0; i < 2; ++i)
+#pragma unroll
+        for (int j = 0; j < 8; ++j) acc[i][j][0] = acc[i][j][1] = acc[i][j][2] = acc[i][j][3] = 0.0f;
+    const int nt_n = r / 8;
+    stage(0, 0);
+    for (int c = 0; c < nch; ++c) {
+        if (c + 1 < nch) stage(c + 1, (c + 1) & 1);
+        else cp_commit();
+        cp_wait1();
         __syncthreads();
-        for (int i = threadIdx.x; i < 64 * r; i += blockDim.x) {   // ms[c][q] = M_e(q, c0 + c)
-            const int c = i / r, q = i - c * r;
-            const float v = Q_MAJOR ? __bfloat162float(me[(int64_t)q * K + c0 + c])
-                                    : __bfloat162float(me[(int64_t)(c0 + c) * r + q]);
-            ms[c * r + q] = v;
+        const __nv_bfloat16* a = sA + (c & 1) * THIN_ROWS * THIN_SA;
+        const __nv_bfloat16* mm = sM + (c & 1) * 64 * THIN_SA;
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) {
+            uint32_t af[2][4];
+#pragma unroll
+            for (int t = 0; t < 2; ++t)
+                ldsm_x4(af[t], smem_u32(a + (32 * warp + 16 * t + (lane & 15)) * THIN_SA + kk * 16 + (lane >> 4) * 8));
+#pragma unroll
+            for (int nt = 0; nt < 8; ++nt) {
+                if (nt >= nt_n) break;
+                uint32_t b0, b1;
+                ldsm_x2(b0, b1, smem_u32(mm + (8 * nt + (lane & 7)) * THIN_SA + kk * 16 + ((lane >> 3) & 1) * 8));
+                mma16816(acc[0][nt], af[0], b0, b1);
+                mma16816(acc[1][nt], af[1], b0, b1);
+            }
         }
         __syncthreads();
-        if (!valid) continue;
-#pragma unroll 1
-        for (int c8 = 0; c8 < 64; c8 += 8) {
-            const uint4 xv = __ldg(xin + (c0 + c8) / 8);
-            const uint32_t xw[4] = {xv.x, xv.y, xv.z, xv.w};
+    }
+    const int g = lane >> 2, c2 = (lane & 3) * 2;
 #pragma unroll
-            for (int j = 0; j < 8; ++j) {
-                const float x = __uint_as_float(j & 1 ? (xw[j >> 1] & 0xFFFF0000u) : (xw[j >> 1] << 16));
-                const float* mr = ms + (c8 + j) * r;
+    for (int t = 0; t < 2; ++t) {
 #pragma unroll
-                for (int q = 0; q < 64; ++q)
-                    if (q < r) acc[q] = fmaf(x, mr[q], acc[q]);
+        for (int h = 0; h < 2; ++h) {
+            const int rr = 32 * warp + 16 * t + g + 8 * h;
+            if (rr >= rows) continue;
+            uint32_t* o = reinterpret_cast<uint32_t*>(out + (int64_t)(row0 + rr) * 64);
+#pragma unroll
+            for (int nt = 0; nt < 8; ++nt) {
+                const float v0 = nt < nt_n ? s * acc[t][nt][2 * h] : 0.0f;
+                const float v1 = nt < nt_n ? s * acc[t][nt][2 * h + 1] : 0.0f;
+                o[(8 * nt + c2) >> 1] = pack_bf16x2(v0, v1);
             }
         }
     }
-    if (!valid) return;
-    uint4* o = reinterpret_cast<uint4*>(out + (int64_t)row * 64);
-#pragma unroll
-    for (int q8 = 0; q8 < 8; ++q8) {
-        uint32_t w[4];
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            const int q = 8 * q8 + 2 * j;
-            w[j] = pack_bf16x2(q < r ? s * acc[q] : 0.0f, q + 1 < r ? s * acc[q + 1] : 0.0f);
-        }
-        o[q8] = make_uint4(w[0], w[1], w[2], w[3]);
-    }
 }
 
-// out for expert e = sum over its grouped rows p (ascending) of coef_p * U[p, a] *
-// V[p, q], a < N (the big dimension), q < r; coef_p = topk_w[perm[p]] when
-// coef_w, else 1.  Written as out[e][a][q] (B adapters) or, with Q_MAJOR_OUT,
-// out[e][q][a] (A adapters), fp32.  Block (e, 256 columns): one thread per
-// column a, V rows staged through shared memory 32 at a time.
+// out for expert e = sum over its grouped rows p (offsets[e] .. offsets[e+1], in
+// chunks of 32, ascending) of coef_p U[p, a] V[p, q], a < N, q < r: out[e][a][q],
+// or out[e][q][a] with Q_MAJOR_OUT; fp32.  coef_p = topk_w[perm[p]] when coef_w,
+// else 1 (applied to V's rows while they are staged).  Block: 128 columns a of
+// one expert; warp w owns a = 16w..16w+15 as an m16 tile of U^T.
 template <bool Q_MAJOR_OUT>
 __global__ void __launch_bounds__(256) lora_grad_kernel(const __nv_bfloat16* __restrict__ U, int N,
                                                         const __nv_bfloat16* __restrict__ V, int r,
@@ -84,48 +161,135 @@ __global__ void __launch_bounds__(256) lora_grad_kernel(const __nv_bfloat16* __r
                                                         const float* __restrict__ topk_w,
                                                         const int* __restrict__ perm, int coef_w,
                                                         float* __restrict__ out) {
-    __shared__ float vs[32][65];
-    __shared__ float cs[32];
-    const int e = blockIdx.y, a = blockIdx.x * 256 + (int)threadIdx.x;
+    __shared__ __align__(16) __nv_bfloat16 sU[2][GR_P][GR_SU];
+    __shared__ __align__(16) __nv_bfloat16 sV[2][GR_P][GR_SV];
+    const int e = blockIdx.y, a0 = blockIdx.x * GR_A;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int p0 = __ldg(offsets + e), p1 = __ldg(offsets + e + 1);
-    float acc[64];
-#pragma unroll
-    for (int q = 0; q < 64; ++q) acc[q] = 0.0f;
-    for (int pb = p0; pb < p1; pb += 32) {
-        const int np = min(32, p1 - pb);
-        __syncthreads();
-        for (int i = threadIdx.x; i < np * 64; i += blockDim.x) {
-            const int pp = i >> 6, q = i & 63;
-            vs[pp][q] = __bfloat162float(V[(int64_t)(pb + pp) * 64 + q]);
+    const int nchunks = (p1 - p0 + GR_P - 1) / GR_P;
+    auto stage = [&](int c, int b) {
+        const int pb = p0 + c * GR_P;
+        for (int i = tid; i < GR_P * (GR_A / 8); i += 256) {   // U rows: 32 x 128 columns
+            const int pp = i / (GR_A / 8), sg = i % (GR_A / 8);
+            const int a = a0 + sg * 8;
+            const bool ok = pb + pp < p1 && a < N;
+            cp16z(smem_u32(&sU[b][pp][sg * 8]), U + (int64_t)(ok ? pb + pp : p0) * N + (ok ? a : 0), ok ? 16u : 0u);
         }
-        if ((int)threadIdx.x < np)
-            cs[threadIdx.x] = coef_w ? __ldg(topk_w + __ldg(perm + pb + threadIdx.x)) : 1.0f;
+        cp_commit();
+        {   // V rows scaled by coef_p: 32 x 64 (ranks past r are zero in V already)
+            const int pp = tid >> 3, q0 = (tid & 7) * 8;
+            uint4 v = make_uint4(0u, 0u, 0u, 0u);
+            if (pb + pp < p1) {
+                v = __ldg(reinterpret_cast<const uint4*>(V + (int64_t)(pb + pp) * 64 + q0));
+                if (coef_w) {
+                    const float cf = __ldg(topk_w + __ldg(perm + pb + pp));
+                    uint32_t* w = reinterpret_cast<uint32_t*>(&v);
+#pragma unroll
+                    for (int j = 0; j < 4; ++j)
+                        w[j] = pack_bf16x2(cf * __uint_as_float(w[j] << 16), cf * __uint_as_float(w[j] & 0xFFFF0000u));
+                }
+            }
+            *reinterpret_cast<uint4*>(&sV[b][pp][q0]) = v;
+        }
+    };
+    float acc[8][4];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) acc[j][0] = acc[j][1] = acc[j][2] = acc[j][3] = 0.0f;
+    const int nt_n = r / 8;
+    if (nchunks > 0) stage(0, 0);
+    for (int c = 0; c < nchunks; ++c) {
+        if (c + 1 < nchunks) stage(c + 1, (c + 1) & 1);
+        else cp_commit();
+        cp_wait1();
         __syncthreads();
+        const int b = c & 1;
+#pragma unroll
+        for (int kk = 0; kk < GR_P / 16; ++kk) {
+            uint32_t af[4];   // A = U^T: 16 columns a x 16 rows p
+            const int mtx = lane >> 3;
+            ldsm_x4_t(af, smem_u32(&sU[b][kk * 16 + (mtx >> 1) * 8 + (lane & 7)][16 * warp + (mtx & 1) * 8]));
+#pragma unroll
+            for (int nt = 0; nt < 8; ++nt) {
+                if (nt >= nt_n) break;
+                uint32_t b0, b1;   // B = V: 16 rows p x 8 ranks q
+                ldsm_x2_t(b0, b1, smem_u32(&sV[b][kk * 16 + ((lane >> 3) & 1) * 8 + (lane & 7)][8 * nt]));
+                mma16816(acc[nt], af, b0, b1);
+            }
+        }
+        __syncthreads();
+    }
+    const int g = lane >> 2, c2 = (lane & 3) * 2;
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+        const int a = a0 + 16 * warp + g + 8 * h;
         if (a >= N) continue;
-#pragma unroll 1
-        for (int pp = 0; pp < np; ++pp) {
-            const float u = cs[pp] * __bfloat162float(U[(int64_t)(pb + pp) * N + a]);
 #pragma unroll
-            for (int q = 0; q < 64; ++q)
-                if (q < r) acc[q] = fmaf(u, vs[pp][q], acc[q]);
+        for (int nt = 0; nt < 8; ++nt) {
+            if (nt >= nt_n) break;
+            const int q = 8 * nt + c2;
+            if (Q_MAJOR_OUT) {
+                out[((int64_t)e * r + q) * N + a] = acc[nt][2 * h];
+                out[((int64_t)e * r + q + 1) * N + a] = acc[nt][2 * h + 1];
+            } else {
+                *reinterpret_cast<float2*>(out + ((int64_t)e * N + a) * r + q) =
+                    make_float2(acc[nt][2 * h], acc[nt][2 * h + 1]);
+            }
         }
     }
-    if (a >= N) return;
-#pragma unroll
-    for (int q = 0; q < 64; ++q) {
-        if (q >= r) break;
-        if (Q_MAJOR_OUT) out[((int64_t)e * r + q) * N + a] = acc[q];
-        else out[((int64_t)e * N + a) * r + q] = acc[q];
+}
+
+// t[e][q][k] = m[e][k][q]: a B adapter [E, K, r] in the [E, r, K] layout of the thin
+// kernel (tiled through shared memory; K a multiple of 64).
+__global__ void __launch_bounds__(256) lora_transpose_kernel(const __nv_bfloat16* __restrict__ m, int K, int r,
+                                                             __nv_bfloat16* __restrict__ t) {
+    __shared__ __nv_bfloat16 tile[64][65];
+    const int e = blockIdx.y, k0 = blockIdx.x * 64;
+    const __nv_bfloat16* me = m + (int64_t)e * K * r;
+    for (int i = threadIdx.x; i < 64 * r; i += blockDim.x) {   // rows k0..k0+63, r contiguous each
+        const int k = i / r, q = i - k * r;
+        tile[q][k] = me[(int64_t)(k0 + k) * r + q];
     }
+    __syncthreads();
+    __nv_bfloat16* te = t + (int64_t)e * r * K;
+    for (int i = threadIdx.x; i < 64 * r; i += blockDim.x) {   // rows q, 64 contiguous k each
+        const int q = i >> 6, k = i & 63;
+        te[(int64_t)q * K + k0 + k] = tile[q][k];
+    }
+}
+
+cudaError_t launch_lora_transpose(const __nv_bfloat16* m, int E, int K, int r, __nv_bfloat16* t, cudaStream_t st) {
+    if (K % 64 || r < 8 || r > 64) return cudaErrorInvalidValue;
+    lora_transpose_kernel<<<dim3(K / 64, E), 256, 0, st>>>(m, K, r, t);
+    count_launch();
+    return cudaGetLastError();
 }
 
 cudaError_t launch_lora_thin(const __nv_bfloat16* in, int K, const __nv_bfloat16* m, bool m_q_major, int r, float s,
                              const int4* sched, const int* tile_prefix, int E, int max_m_tiles, __nv_bfloat16* out,
                              cudaStream_t st) {
     if (max_m_tiles <= 0) return cudaSuccess;
-    if (K % 64 || r < 1 || r > 64) return cudaErrorInvalidValue;
-    if (m_q_major) lora_thin_kernel<true><<<max_m_tiles, 256, 0, st>>>(in, K, m, r, s, sched, tile_prefix, E, out);
-    else lora_thin_kernel<false><<<max_m_tiles, 256, 0, st>>>(in, K, m, r, s, sched, tile_prefix, E, out);
+    if (K % 64 || r < 8 || r > 64 || r % 8) return cudaErrorInvalidValue;
+    static std::mutex mu;
+    static bool set[64][2] = {};
+    int dev = 0;
+    cudaError_t err = cudaGetDevice(&dev);
+    if (err != cudaSuccess) return err;
+    if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+    {
+        std::lock_guard<std::mutex> lock(mu);
+        if (!set[dev][m_q_major]) {
+            err = m_q_major ? cudaFuncSetAttribute(lora_thin_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                   THIN_SMEM)
+                            : cudaFuncSetAttribute(lora_thin_kernel<false>,
+                                                   cudaFuncAttributeMaxDynamicSharedMemorySize, THIN_SMEM);
+            if (err != cudaSuccess) return err;
+            set[dev][m_q_major] = true;
+        }
+    }
+    if (m_q_major)
+        lora_thin_kernel<true><<<max_m_tiles, 256, THIN_SMEM, st>>>(in, K, m, r, s, sched, tile_prefix, E, out);
+    else
+        lora_thin_kernel<false><<<max_m_tiles, 256, THIN_SMEM, st>>>(in, K, m, r, s, sched, tile_prefix, E, out);
     count_launch();
     return cudaGetLastError();
 }
@@ -133,8 +297,8 @@ cudaError_t launch_lora_thin(const __nv_bfloat16* in, int K, const __nv_bfloat16
 cudaError_t launch_lora_grad(const __nv_bfloat16* U, int N, const __nv_bfloat16* V, int r, const int* offsets,
                              int E, const float* topk_w, const int* perm, bool coef_w, bool q_major_out, float* out,
                              cudaStream_t st) {
-    if (r < 1 || r > 64) return cudaErrorInvalidValue;
-    const dim3 grid((N + 255) / 256, E);
+    if (r < 8 || r > 64 || r % 8 || N % 64) return cudaErrorInvalidValue;
+    const dim3 grid((N + GR_A - 1) / GR_A, E);
     if (q_major_out)
         lora_grad_kernel<true><<<grid, 256, 0, st>>>(U, N, V, r, offsets, topk_w, perm, coef_w ? 1 : 0, out);
     else

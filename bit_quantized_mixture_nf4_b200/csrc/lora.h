@@ -10,6 +10,8 @@ namespace e4b {
 cudaError_t launch_lora_thin(const __nv_bfloat16* in, int K, const __nv_bfloat16* m, bool m_q_major, int r, float s,
                              const int4* sched, const int* tile_prefix, int E, int max_m_tiles, __nv_bfloat16* out,
                              cudaStream_t st);
+// t [E, r, K] = the B adapter m [E, K, r] transposed (K a multiple of 64).
+cudaError_t launch_lora_transpose(const __nv_bfloat16* m, int E, int K, int r, __nv_bfloat16* t, cudaStream_t st);
 // out (fp32) for each expert e = sum over its grouped rows p (offsets[e] .. offsets[e+1])
 // of coef_p U[p, :] (x) V[p, :r], U [rows, N] bf16, V [rows, 64] bf16; coef_p =
 // topk_w[perm[p]] when coef_w, else 1; out [E, N, r], or [E, r, N] when q_major_out.
