@@ -16,6 +16,10 @@ Parity status of each function (what pins it is in ``tests/test_oracle_pins.py``
   route / permute        pinned (brute-force sort, softmax ratio closed form, bijection)
   forward                pinned (fp64 dense all-experts reference; E=1 dense SwiGLU MLP)
   dgrad                  pinned (central finite differences; adjoint identity)
+  MXFP4 quantize / dequantize
+                         pinned (exact reproduction of scaled E2M1 values, the scale
+                         exponent on hand-picked maxima and its clamp, ties to even,
+                         saturation, round-trip bound, idempotence, padding)
   FP4 codebook vs bitsandbytes' own fp4 table: parity unpinned (not on the pages).
 """
 from __future__ import annotations
@@ -58,6 +62,10 @@ def _L():
             lib.e4bo_quantize.argtypes = [P, i64, i64, i64, i32, i32, P, P]
             lib.e4bo_dequantize_f32.argtypes = [P, P, i64, i32, i32, P]
             lib.e4bo_dequantize_bf16.argtypes = [P, P, i64, i32, i32, P]
+            lib.e4bo_quantize_mxfp4.argtypes = [P, i64, i64, i64, P, P]
+            lib.e4bo_dequantize_mxfp4.argtypes = [P, P, i64, i64, i64, i32, P]
+            lib.e4bo_mxfp4_scale_stride.argtypes = [i64]
+            lib.e4bo_mxfp4_scale_stride.restype = i64
             lib.e4bo_route.argtypes = [P, i64, i32, i32, i32, P, P]
             lib.e4bo_permute.argtypes = [P, i64, i32, i32, P, P, P]
             dbl = ctypes.c_double
@@ -142,6 +150,40 @@ def dequantize(packed: np.ndarray, absmax: np.ndarray, shape, cb: int = NF4,
         return out.reshape(shape)
     bits = np.zeros(n, np.uint16)
     _check("e4bo_dequantize_bf16", _L().e4bo_dequantize_bf16(_p(packed), _p(absmax), n, blocksize, cb, _p(bits)))
+    bits = bits.reshape(shape)
+    return bits if out_dtype == "bf16_bits" else bf16_bits_to_f32(bits)
+
+
+def mxfp4_scale_stride(cols: int) -> int:
+    """Bytes per row of an MXFP4 scale array: cols/32 rounded up to a multiple of 16."""
+    return int(_L().e4bo_mxfp4_scale_stride(cols))
+
+
+def quantize_mxfp4(w: np.ndarray):
+    """w: fp32 [E, out, in] -> (packed uint8 [E, out*in/2], scales uint8 [E, out, S]),
+    OCP MX v1.0 MXFP4: 32-element blocks, E8M0 scales (byte X + 127), E2M1 codes."""
+    w = np.ascontiguousarray(w, np.float32)
+    if w.ndim != 3:
+        raise ValueError("quantize_mxfp4 expects a 3-D [E, out, in] stack")
+    E, o, i = w.shape
+    packed = np.zeros((E, o * i // 2), np.uint8)
+    scales = np.zeros((E, o, mxfp4_scale_stride(i)), np.uint8)
+    _check("e4bo_quantize_mxfp4", _L().e4bo_quantize_mxfp4(_p(w), E, o, i, _p(packed), _p(scales)))
+    return packed, scales
+
+
+def dequantize_mxfp4(packed: np.ndarray, scales: np.ndarray, shape, out_dtype: str = "bf16") -> np.ndarray:
+    """MXFP4 packed codes + E8M0 scales -> [E, out, in]: e2m1(q) * 2^(s - 127) in fp32
+    (exact), then bf16 (nearest-even; exact for these values) unless out_dtype 'f32'."""
+    packed = np.ascontiguousarray(packed, np.uint8)
+    scales = np.ascontiguousarray(scales, np.uint8)
+    E, o, i = shape
+    if out_dtype == "f32":
+        out = np.zeros(E * o * i, np.float32)
+        _check("e4bo_dequantize_mxfp4", _L().e4bo_dequantize_mxfp4(_p(packed), _p(scales), E, o, i, 0, _p(out)))
+        return out.reshape(shape)
+    bits = np.zeros(E * o * i, np.uint16)
+    _check("e4bo_dequantize_mxfp4", _L().e4bo_dequantize_mxfp4(_p(packed), _p(scales), E, o, i, 1, _p(bits)))
     bits = bits.reshape(shape)
     return bits if out_dtype == "bf16_bits" else bf16_bits_to_f32(bits)
 

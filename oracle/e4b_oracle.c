@@ -188,6 +188,90 @@ int e4bo_dequantize_bf16(const uint8_t *packed, const float *absmax, int64_t n,
     return ORC_OK;
 }
 
+/* ---- MXFP4 ([P2] "Scope": the gpt-oss experts ship MXFP4 weights) --------
+ * The pages name the format only; the reading taken is the OCP Microscaling
+ * Formats (MX) v1.0 specification: blocks of 32 consecutive elements of a row
+ * share one E8M0 scale 2^X (stored as the byte X + 127), and each element is an
+ * FP4 E2M1 value (sign in bit 3, magnitudes {0, .5, 1, 1.5, 2, 3, 4, 6} in bits
+ * 2..0).  Quantization (the spec's conversion): X = floor(log2(amax)) - 2 (2 is
+ * the largest E2M1 exponent), clamped to [-127, 127]; each element is v / 2^X
+ * rounded to the nearest E2M1 value, ties to the even code, saturating at 6.
+ * Readings where the spec leaves room: an all-zero block stores X = -127 and zero
+ * codes; a value that rounds to zero is stored as +0.  Storage: codes packed like
+ * the 4-bit stacks (element 2b in the high nibble of byte b); scales uint8
+ * [E, out, S] with S = in/32 rounded up to a multiple of 16 (padding bytes 0). */
+
+static const float kE2M1[8] = {0.0f, 0.5f, 1.0f, 1.5f, 2.0f, 3.0f, 4.0f, 6.0f};
+
+int64_t e4bo_mxfp4_scale_stride(int64_t in) { return ((in / 32) + 15) / 16 * 16; }
+
+/* nearest E2M1 magnitude code of |p| (p finite), ties to the even code, saturating */
+static int e2m1_code(float a) {
+    if (a >= 6.0f) return 7;
+    int best = 0;
+    for (int c = 1; c < 8; ++c) {
+        float dc = fabsf(a - kE2M1[c]), db = fabsf(a - kE2M1[best]);
+        if (dc < db || (dc == db && (c & 1) == 0)) best = c;
+    }
+    return best;
+}
+
+int e4bo_quantize_mxfp4(const float *w, int64_t E, int64_t out, int64_t in, uint8_t *packed, uint8_t *scales) {
+    if (!w || !packed || !scales || E < 0 || out < 0 || in < 0) return ORC_ERR_ARG;
+    if (in % 32 != 0) return ORC_ERR_BLOCKSIZE;
+    const int64_t S = e4bo_mxfp4_scale_stride(in), rows = E * out;
+    memset(scales, 0, (size_t)(rows * S));
+#pragma omp parallel for schedule(static)
+    for (int64_t r = 0; r < rows; ++r) {
+        for (int64_t j = 0; j < in / 32; ++j) {
+            const float *src = w + r * in + j * 32;
+            float amax = 0.0f;
+            for (int i = 0; i < 32; ++i) amax = fmaxf(amax, fabsf(src[i]));
+            int X = -127;
+            if (amax > 0.0f) {
+                int e;
+                frexpf(amax, &e);          /* amax = m 2^e, m in [0.5, 1): floor(log2 amax) = e - 1 */
+                X = (e - 1) - 2;
+                if (X < -127) X = -127;
+                if (X > 127) X = 127;
+            }
+            scales[r * S + j] = (uint8_t)(X + 127);
+            uint8_t *dst = packed + (r * in + j * 32) / 2;
+            for (int i = 0; i < 32; i += 2) {
+                int q[2];
+                for (int t = 0; t < 2; ++t) {
+                    float p = ldexpf(src[i + t], -X);   /* exact scaling by a power of two */
+                    int c = amax > 0.0f ? e2m1_code(fabsf(p)) : 0;
+                    q[t] = (c != 0 && p < 0.0f) ? (8 | c) : c;
+                }
+                dst[i / 2] = (uint8_t)((q[0] << 4) | q[1]);
+            }
+        }
+    }
+    return ORC_OK;
+}
+
+static inline float mx_one(const uint8_t *packed, const uint8_t *scales, int64_t in, int64_t S, int64_t i) {
+    const int64_t r = i / in, c = i % in;
+    const uint8_t byte = packed[i >> 1];
+    const int q = (i & 1) ? (byte & 15) : (byte >> 4);
+    const float m = kE2M1[q & 7];
+    return ldexpf((q & 8) ? -m : m, (int)scales[r * S + c / 32] - 127);
+}
+
+int e4bo_dequantize_mxfp4(const uint8_t *packed, const uint8_t *scales, int64_t E, int64_t out, int64_t in,
+                          int bf16, void *dst) {
+    if (!packed || !scales || !dst || E < 0 || out < 0 || in < 0 || in % 32) return ORC_ERR_ARG;
+    const int64_t S = e4bo_mxfp4_scale_stride(in), n = E * out * in;
+#pragma omp parallel for schedule(static)
+    for (int64_t i = 0; i < n; ++i) {
+        const float v = mx_one(packed, scales, in, S, i);
+        if (bf16) ((uint16_t *)dst)[i] = e4bo_f32_to_bf16(v);
+        else ((float *)dst)[i] = v;
+    }
+    return ORC_OK;
+}
+
 /* ---- routing ------------------------------------------------------------- */
 
 /* logits fp32 [T, E] -> idx [T, k] (descending logit, ties to lower index) and
