@@ -19,12 +19,13 @@ LIB_PATH = os.path.join(_HERE, "libe4b.so")
 
 E4B_OK, E4B_ERR_INVALID_ARG, E4B_ERR_BLOCKSIZE, E4B_ERR_UNSUPPORTED, E4B_ERR_WORKSPACE, E4B_ERR_CUDA, \
     E4B_ERR_TIMEOUT = range(7)
-NF4, FP4 = 0, 1
+NF4, FP4, MXFP4 = 0, 1, 2
 F32, BF16 = 0, 1
 PATH_AUTO, PATH_GROUPED, PATH_DECODE = 0, 1, 2
 ACT_SWIGLU, ACT_CLAMPED_GLU = 0, 1
 
-EXPORTS = ("e4b_quantize_nf4", "e4b_dequantize_nf4", "e4b_moe_workspace_size", "e4b_moe_forward",
+EXPORTS = ("e4b_quantize_nf4", "e4b_dequantize_nf4", "e4b_quantize_mxfp4", "e4b_dequantize_mxfp4",
+           "e4b_mxfp4_scale_stride", "e4b_moe_workspace_size", "e4b_moe_forward",
            "e4b_moe_backward", "e4b_moe_backward_dgrad", "e4b_moe_backward_router", "e4b_device_status", "e4b_status_string",
            "e4b_launch_count", "e4b_timing_enable", "e4b_timing_enable_kinds", "e4b_timing_reset", "e4b_timing_get",
            "e4b_moe_forward_noalloc", "e4b_watchdog_selftest", "e4b_pipe_arena_size", "e4b_pipe_create",
@@ -45,7 +46,7 @@ class e4b_experts(ctypes.Structure):
     _fields_ = [("gate_up", ctypes.c_void_p), ("down", ctypes.c_void_p), ("gate_up_absmax", ctypes.c_void_p),
                 ("down_absmax", ctypes.c_void_p), ("gate_up_bias", ctypes.c_void_p), ("down_bias", ctypes.c_void_p),
                 ("lora_A_gu", ctypes.c_void_p), ("lora_B_gu", ctypes.c_void_p), ("lora_A_d", ctypes.c_void_p),
-                ("lora_B_d", ctypes.c_void_p)]
+                ("lora_B_d", ctypes.c_void_p), ("gate_up_scales", ctypes.c_void_p), ("down_scales", ctypes.c_void_p)]
 
 
 class e4b_lora_grads(ctypes.Structure):
@@ -72,6 +73,10 @@ def _load():
     P, i64, i32, sz = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_size_t
     lib.e4b_quantize_nf4.argtypes = [P, i64, i64, i64, i32, i32, P, P, P]
     lib.e4b_dequantize_nf4.argtypes = [P, P, i64, i64, i64, i32, i32, i32, P, P]
+    lib.e4b_quantize_mxfp4.argtypes = [P, i64, i64, i64, P, P, P]
+    lib.e4b_dequantize_mxfp4.argtypes = [P, P, i64, i64, i64, i32, P, P]
+    lib.e4b_mxfp4_scale_stride.argtypes = [i64]
+    lib.e4b_mxfp4_scale_stride.restype = i64
     lib.e4b_moe_workspace_size.argtypes = [ctypes.POINTER(e4b_moe_desc), i64]
     lib.e4b_moe_workspace_size.restype = sz
     lib.e4b_moe_forward.argtypes = [ctypes.POINTER(e4b_moe_desc), ctypes.POINTER(e4b_experts), P, i64, P, P, P, P,
@@ -105,7 +110,8 @@ def _load():
     lib.e4b_timing_reset.restype = None
     lib.e4b_timing_get.argtypes = [i32, ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_uint64)]
     lib.e4b_timing_get.restype = ctypes.c_int
-    for f in ("e4b_quantize_nf4", "e4b_dequantize_nf4", "e4b_moe_forward", "e4b_moe_backward", "e4b_moe_backward_dgrad",
+    for f in ("e4b_quantize_nf4", "e4b_dequantize_nf4", "e4b_quantize_mxfp4", "e4b_dequantize_mxfp4",
+              "e4b_moe_forward", "e4b_moe_backward", "e4b_moe_backward_dgrad",
               "e4b_device_status", "e4b_moe_forward_noalloc", "e4b_moe_backward_router", "e4b_watchdog_selftest"):
         getattr(lib, f).restype = ctypes.c_int
     _lib = lib
@@ -215,8 +221,37 @@ def make_desc(E, H, I, top_k, renormalize=True, codebook=NF4, blocksize=64, path
                         glu_limit, lora_rank, lora_scale)
 
 
+def e4b_mxfp4_scale_stride(cols: int) -> int:
+    return int(_load().e4b_mxfp4_scale_stride(cols))
+
+
+def e4b_quantize_mxfp4(w: torch.Tensor, stream=None):
+    """fp32 [E, out, in] (CUDA) -> (packed uint8 [E, out*in/2], scales uint8 [E, out, S]):
+    OCP MX v1.0 MXFP4 (32-element blocks, E8M0 scales, E2M1 codes)."""
+    _cuda(w, "w", torch.float32)
+    if w.dim() != 3 or not w.is_contiguous():
+        raise ValueError("w must be a contiguous [E, out, in] tensor")
+    E, o, i = w.shape
+    packed = torch.empty(E, o * i // 2, dtype=torch.uint8, device=w.device)
+    scales = torch.empty(E, o, e4b_mxfp4_scale_stride(i), dtype=torch.uint8, device=w.device)
+    _check("e4b_quantize_mxfp4", _load().e4b_quantize_mxfp4(_ptr(w), E, o, i, _ptr(packed), _ptr(scales),
+                                                          _stream(stream)))
+    return packed, scales
+
+
+def e4b_dequantize_mxfp4(packed: torch.Tensor, scales: torch.Tensor, shape, out_dtype=torch.bfloat16, stream=None):
+    _cuda(packed, "packed", torch.uint8)
+    _cuda(scales, "scales", torch.uint8)
+    E, o, i = shape
+    out = torch.empty(E, o, i, dtype=out_dtype, device=packed.device)
+    _check("e4b_dequantize_mxfp4", _load().e4b_dequantize_mxfp4(
+        _ptr(packed), _ptr(scales), E, o, i, BF16 if out_dtype == torch.bfloat16 else F32, _ptr(out),
+        _stream(stream)))
+    return out
+
+
 def make_experts(gate_up, down, gate_up_absmax, down_absmax, gate_up_bias=None, down_bias=None,
-                 lora=None) -> e4b_experts:
+                 lora=None, gate_up_scales=None, down_scales=None) -> e4b_experts:
     """The two packed stacks and their absmax (device tensors), plus optional fp32
     per-expert biases gate_up_bias [E, 2I] and down_bias [E, H], and optional bf16
     LoRA adapters lora = (A_gu [E, r, H], B_gu [E, 2I, r], A_d [E, r, I], B_d [E, H, r])
@@ -225,7 +260,11 @@ def make_experts(gate_up, down, gate_up_absmax, down_absmax, gate_up_bias=None, 
     for n, t in (("gate_up", gate_up), ("down", down)):
         _cuda(t, n, torch.uint8)
     for n, t in (("gate_up_absmax", gate_up_absmax), ("down_absmax", down_absmax)):
-        _cuda(t, n, torch.float32)
+        if t is not None:
+            _cuda(t, n, torch.float32)
+    for n, t in (("gate_up_scales", gate_up_scales), ("down_scales", down_scales)):
+        if t is not None:
+            _cuda(t, n, torch.uint8)
     for n, t in (("gate_up_bias", gate_up_bias), ("down_bias", down_bias)):
         if t is not None:
             _cuda(t, n, torch.float32)
@@ -236,9 +275,9 @@ def make_experts(gate_up, down, gate_up_absmax, down_absmax, gate_up_bias=None, 
             if not t.is_contiguous():
                 raise ValueError(f"{n} must be contiguous")
             ad[i] = t.data_ptr()
-    return e4b_experts(gate_up.data_ptr(), down.data_ptr(), gate_up_absmax.data_ptr(), down_absmax.data_ptr(),
-                       None if gate_up_bias is None else gate_up_bias.data_ptr(),
-                       None if down_bias is None else down_bias.data_ptr(), *ad)
+    ptr = lambda t: None if t is None else t.data_ptr()
+    return e4b_experts(gate_up.data_ptr(), down.data_ptr(), ptr(gate_up_absmax), ptr(down_absmax),
+                       ptr(gate_up_bias), ptr(down_bias), *ad, ptr(gate_up_scales), ptr(down_scales))
 
 
 def e4b_moe_workspace_size(desc: e4b_moe_desc, T: int) -> int:

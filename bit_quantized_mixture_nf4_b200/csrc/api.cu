@@ -144,11 +144,12 @@ static WsLayout layout_for(const e4b_moe_desc* d, int64_t T) {
 
 static e4b_status check_desc(const e4b_moe_desc* d) {
     if (!d) return E4B_ERR_INVALID_ARG;
-    if (d->blocksize != 64) return E4B_ERR_BLOCKSIZE;
+    if (d->blocksize != (d->codebook == E4B_CODEBOOK_MXFP4 ? 32 : 64)) return E4B_ERR_BLOCKSIZE;
     if (d->E < 1 || d->E > 256 || d->H <= 0 || d->I <= 0) return E4B_ERR_INVALID_ARG;
     if (d->H % 64 || d->I % 64) return E4B_ERR_BLOCKSIZE;
     if (d->top_k < 1 || d->top_k > 8 || d->top_k > d->E) return E4B_ERR_INVALID_ARG;
-    if (d->codebook != E4B_CODEBOOK_NF4 && d->codebook != E4B_CODEBOOK_FP4) return E4B_ERR_INVALID_ARG;
+    if (d->codebook != E4B_CODEBOOK_NF4 && d->codebook != E4B_CODEBOOK_FP4 && d->codebook != E4B_CODEBOOK_MXFP4)
+        return E4B_ERR_INVALID_ARG;
     if (d->path < E4B_PATH_AUTO || d->path > E4B_PATH_DECODE) return E4B_ERR_INVALID_ARG;
     if (d->activation != E4B_ACT_SWIGLU && d->activation != E4B_ACT_CLAMPED_GLU) return E4B_ERR_INVALID_ARG;
     if (d->activation == E4B_ACT_CLAMPED_GLU && (!std::isfinite(d->glu_alpha) || !(d->glu_limit > 0.0f)))
@@ -159,7 +160,10 @@ static e4b_status check_desc(const e4b_moe_desc* d) {
 }
 
 static e4b_status check_experts(const e4b_moe_desc* d, const e4b_experts* w) {
-    if (!w || !w->gate_up || !w->down || !w->gate_up_absmax || !w->down_absmax) return E4B_ERR_INVALID_ARG;
+    if (!w || !w->gate_up || !w->down) return E4B_ERR_INVALID_ARG;
+    if (d->codebook == E4B_CODEBOOK_MXFP4 ? (!w->gate_up_scales || !w->down_scales)
+                                          : (!w->gate_up_absmax || !w->down_absmax))
+        return E4B_ERR_INVALID_ARG;
     if (d->lora_rank > 0 && (!w->lora_A_gu || !w->lora_B_gu || !w->lora_A_d || !w->lora_B_d))
         return E4B_ERR_INVALID_ARG;
     return E4B_OK;
@@ -181,6 +185,13 @@ static GemmParams base_params(const e4b_moe_desc* d, uint8_t* ws, const WsLayout
     p.status = device_status_ptr();
     (void)P;
     return p;
+}
+
+// MXFP4 stacks: the scale bytes of the stored matrix (cols = its row length).
+static void set_mx(const e4b_moe_desc* d, const uint8_t* scales, int64_t cols, GemmParams* p) {
+    if (d->codebook != E4B_CODEBOOK_MXFP4) return;
+    p->mx_scales = scales;
+    p->mx_stride = mxfp4_scale_stride(cols);
 }
 
 static int max_m_tiles(int64_t P, int E) { return (int)((P + gemm_tile_rows() - 1) / gemm_tile_rows()) + E; }
@@ -215,6 +226,7 @@ static e4b_status run_gateup(const e4b_moe_desc* d, const e4b_experts* w, uint8_
     p.b_rows_per_expert = 2 * d->I;
     p.b_rows_total = (int64_t)d->E * 2 * d->I;
     p.b_blocks_per_row = d->H / 64;
+    set_mx(d, w->gate_up_scales, d->H, &p);
     p.up_offset = d->I;
     p.out_bf16 = h_out;
     p.gu = gu_out;
@@ -246,6 +258,7 @@ static e4b_status run_down(const e4b_moe_desc* d, const e4b_experts* w, uint8_t*
     p.b_rows_per_expert = d->H;
     p.b_rows_total = (int64_t)d->E * d->H;
     p.b_blocks_per_row = d->I / 64;
+    set_mx(d, w->down_scales, d->I, &p);
     p.out_bf16 = out;
     p.bias = w->down_bias;
     p.ld_out = d->H;
@@ -337,6 +350,30 @@ e4b_status e4b_quantize_nf4(const float* w, int64_t E, int64_t out, int64_t in, 
     return E4B_OK;
 }
 
+int64_t e4b_mxfp4_scale_stride(int64_t in) { return in < 0 ? 0 : mxfp4_scale_stride(in); }
+
+e4b_status e4b_quantize_mxfp4(const float* w, int64_t E, int64_t out, int64_t in, uint8_t* packed, uint8_t* scales,
+                              void* stream) {
+    if (E < 0 || out < 0 || in < 0) return E4B_ERR_INVALID_ARG;
+    if (in % 32) return E4B_ERR_BLOCKSIZE;
+    if (E * out * in == 0) return E4B_OK;
+    if (!w || !packed || !scales) return E4B_ERR_INVALID_ARG;
+    E4B_CUDA_TRY(launch_quantize_mxfp4(w, E * out, in, packed, scales, static_cast<cudaStream_t>(stream)));
+    return E4B_OK;
+}
+
+e4b_status e4b_dequantize_mxfp4(const uint8_t* packed, const uint8_t* scales, int64_t E, int64_t out, int64_t in,
+                                e4b_dtype out_dtype, void* w_out, void* stream) {
+    if (E < 0 || out < 0 || in < 0) return E4B_ERR_INVALID_ARG;
+    if (in % 32) return E4B_ERR_BLOCKSIZE;
+    if (out_dtype != E4B_F32 && out_dtype != E4B_BF16) return E4B_ERR_INVALID_ARG;
+    if (E * out * in == 0) return E4B_OK;
+    if (!packed || !scales || !w_out) return E4B_ERR_INVALID_ARG;
+    E4B_CUDA_TRY(launch_dequantize_mxfp4(packed, scales, E * out, in, out_dtype == E4B_BF16, w_out,
+                                         static_cast<cudaStream_t>(stream)));
+    return E4B_OK;
+}
+
 e4b_status e4b_dequantize_nf4(const uint8_t* packed, const float* absmax, int64_t E, int64_t out, int64_t in,
                               int blocksize, e4b_codebook cb, e4b_dtype out_dtype, void* w_out, void* stream) {
     if (blocksize != 64) return E4B_ERR_BLOCKSIZE;
@@ -371,8 +408,8 @@ e4b_status e4b_moe_forward(const e4b_moe_desc* d, const e4b_experts* w, const vo
     if (!workspace || ws_bytes < L.total) return E4B_ERR_WORKSPACE;
     const bool want_grouped_outputs = saved_gu || saved_h || offsets_out || perm_out;
     // the decode kernels implement SwiGLU without biases
-    const bool plain_experts =
-        d->activation == E4B_ACT_SWIGLU && !w->gate_up_bias && !w->down_bias && d->lora_rank == 0;
+    const bool plain_experts = d->activation == E4B_ACT_SWIGLU && !w->gate_up_bias && !w->down_bias &&
+                               d->lora_rank == 0 && d->codebook != E4B_CODEBOOK_MXFP4;
     const bool dec_ok = !want_grouped_outputs && plain_experts && decode_supported(d->E, d->H, d->I, T, d->top_k);
     const bool decode = (d->path == E4B_PATH_DECODE) || (d->path == E4B_PATH_AUTO && dec_ok);
     if (d->path == E4B_PATH_DECODE && !dec_ok) return E4B_ERR_UNSUPPORTED;
@@ -482,6 +519,7 @@ e4b_status e4b_moe_backward(const e4b_moe_desc* d, const e4b_experts* w, const v
     p.b_rows_per_expert = d->H;
     p.b_rows_total = (int64_t)d->E * d->H;
     p.b_blocks_per_row = d->I / 64;
+    set_mx(d, w->down_scales, d->I, &p);
     p.gu = const_cast<__nv_bfloat16*>(gu);
     p.out_bf16 = dgu;
     p.ld_out = 2 * d->I;
@@ -530,6 +568,7 @@ e4b_status e4b_moe_backward(const e4b_moe_desc* d, const e4b_experts* w, const v
     q.b_rows_per_expert = 2 * d->I;
     q.b_rows_total = (int64_t)d->E * 2 * d->I;
     q.b_blocks_per_row = d->H / 64;
+    set_mx(d, w->gate_up_scales, d->H, &q);
     q.out_bf16 = a_perm;   // per-pair rows in grouped order; the gathered grad_out is dead by now
     q.ld_out = d->H;
     q.lora_r = d->lora_rank;

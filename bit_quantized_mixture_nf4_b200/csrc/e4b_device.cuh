@@ -20,13 +20,22 @@ enum : uint32_t { kStatusTimeout = 1u };
 // NF4: the 16 NormalFloat values (QLoRA appendix, the "standard" table the
 // expert-layer pages refer to via get_4bit_type("nf4")), ascending, code 7 = 0.
 // FP4: e2m1 magnitudes {0, .5, 1, 1.5, 2, 3, 4, 6} / 6 with the sign in bit 3.
-static __constant__ float c_code[2][16] = {
+// MXFP4 (index 2): the same codes unscaled, {0, .5, ..., 6}; a 32-element block's
+// E8M0 scale 2^(s - 127) multiplies them (OCP Microscaling Formats v1.0).
+static __constant__ float c_code[3][16] = {
     {-1.0f, -0.6961928009986877f, -0.5250730514526367f, -0.39491748809814453f,
      -0.28444138169288635f, -0.18477343022823334f, -0.09105003625154495f, 0.0f,
      0.07958029955625534f, 0.16093020141124725f, 0.24611230194568634f, 0.33791524171829224f,
      0.44070982933044434f, 0.5626170039176941f, 0.7229568362236023f, 1.0f},
     {0.0f, 0.5f / 6.0f, 1.0f / 6.0f, 1.5f / 6.0f, 2.0f / 6.0f, 3.0f / 6.0f, 4.0f / 6.0f, 1.0f,
-     -0.0f, -0.5f / 6.0f, -1.0f / 6.0f, -1.5f / 6.0f, -2.0f / 6.0f, -3.0f / 6.0f, -4.0f / 6.0f, -1.0f}};
+     -0.0f, -0.5f / 6.0f, -1.0f / 6.0f, -1.5f / 6.0f, -2.0f / 6.0f, -3.0f / 6.0f, -4.0f / 6.0f, -1.0f},
+    {0.0f, 0.5f, 1.0f, 1.5f, 2.0f, 3.0f, 4.0f, 6.0f, -0.0f, -0.5f, -1.0f, -1.5f, -2.0f, -3.0f, -4.0f, -6.0f}};
+
+// The E8M0 scale byte s as the fp32 value 2^(s - 127) (s = 0: the subnormal 2^-127;
+// s = 255, the format's NaN, is never produced by the quantizer).
+__device__ __forceinline__ float mx_scale(uint32_t s) {
+    return s == 0u ? __int_as_float(0x00400000) : __int_as_float((int)(s << 23));
+}
 
 // --------------------------------------------------------------- small utils
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {

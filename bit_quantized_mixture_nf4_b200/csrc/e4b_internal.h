@@ -43,6 +43,9 @@ struct GemmParams {
     // and rows or columns outside the expert read as 0.  lora_r = 0: no extra stage.
     const __nv_bfloat16* lora_b;
     int lora_r;               // 0 or a multiple of 8 up to 64
+    // MXFP4 weights (codebook 2): the E8M0 scale bytes [rows, mx_stride] replace absmax
+    const uint8_t* mx_scales;
+    int64_t mx_stride;
 };
 
 // launch bookkeeping
@@ -61,6 +64,12 @@ cudaError_t launch_quantize(const float* w, int64_t nblocks, int codebook, uint8
                             cudaStream_t st);
 cudaError_t launch_dequantize(const uint8_t* packed, const float* absmax, int64_t n, int codebook, int out_bf16,
                               void* out, cudaStream_t st);
+// MXFP4 (32-element blocks, E8M0 scales [rows, S], S = mxfp4_scale_stride(in) bytes per row)
+int64_t mxfp4_scale_stride(int64_t in);
+cudaError_t launch_quantize_mxfp4(const float* w, int64_t rows, int64_t in, uint8_t* packed, uint8_t* scales,
+                                  cudaStream_t st);
+cudaError_t launch_dequantize_mxfp4(const uint8_t* packed, const uint8_t* scales, int64_t rows, int64_t in,
+                                    int out_bf16, void* out, cudaStream_t st);
 
 // route.cu
 constexpr int kChunkPairs = 256;   // pairs per grouping block (one per thread of a 256-thread block)

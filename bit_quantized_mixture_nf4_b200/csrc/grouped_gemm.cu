@@ -151,6 +151,22 @@ __device__ __forceinline__ int64_t absmax_index(const GemmParams& p, const TileI
     return row * p.b_blocks_per_row + blk;
 }
 
+// MXFP4: byte offset, in p.mx_scales, of the 4 scale bytes the raw warp copies for
+// block b at k-stage 0 (-1 outside the stack).  K-major: row b's bytes for 32-blocks
+// 0..3 (k-stage ks reads bytes 2ks, 2ks+1 of the group starting at 4 (ks / 2));
+// MN-major: k-row (b & 63)'s bytes for the 4 32-column groups of this CTA's 128
+// columns (n-block b >> 6 takes bytes 2 (b >> 6), +1).
+template <int EPI, int CTAS>
+__device__ __forceinline__ int64_t mx_offset(const GemmParams& p, const TileInfo& ti, int b, int rank) {
+    if (absmax_index<EPI, CTAS>(p, ti, 0, b, rank) < 0) return -1;
+    if (EPI == EPI_GATEUP || EPI == EPI_DOWN) {
+        const int64_t row = (int64_t)ti.e * p.b_rows_per_expert + kmajor_row<EPI>(p, ti.nt, rank * Cfg<CTAS>::N_CTA + b);
+        return row * p.mx_stride;
+    }
+    const int64_t row = (int64_t)ti.e * p.b_rows_per_expert + (b & 63);
+    return row * p.mx_stride + (ti.nt * BN + rank * Cfg<CTAS>::N_CTA) / 32;
+}
+
 // This row's part of the routing-weight gradient over one 32-column chunk:
 // acc += sum_j v[j] * h[row, c0 + j] (fp32, columns in order).
 __device__ __forceinline__ void dw_dot_chunk(const GemmParams& p, int64_t row, int c0, const float (&v)[32],
@@ -304,15 +320,23 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_con
             const int ebase = ti.e * p.b_rows_per_expert;
             // per-tile source of each of this lane's absmax values at k-stage 0, and the
             // step per k-stage (K-major: next block of the row; MN-major: 64 rows down)
-            const float* src[PER_LANE];
+            // (MXFP4: the 4 E8M0 scale bytes that hold this block's two 32-block scales)
+            const uint8_t* src[PER_LANE];
             bool valid[PER_LANE];
 #pragma unroll
             for (int i = 0; i < PER_LANE; ++i) {
-                const int64_t ix = absmax_index<EPI, CTAS>(p, ti, 0, lane + 32 * i, (int)rank);
-                valid[i] = ix >= 0;
-                src[i] = p.absmax + (valid[i] ? ix : 0);
+                if (CB == 2) {
+                    const int64_t off = mx_offset<EPI, CTAS>(p, ti, lane + 32 * i, (int)rank);
+                    valid[i] = off >= 0;
+                    src[i] = p.mx_scales + (valid[i] ? off : 0);
+                } else {
+                    const int64_t ix = absmax_index<EPI, CTAS>(p, ti, 0, lane + 32 * i, (int)rank);
+                    valid[i] = ix >= 0;
+                    src[i] = reinterpret_cast<const uint8_t*>(p.absmax + (valid[i] ? ix : 0));
+                }
             }
-            const int64_t step = kMajorB ? 1 : (int64_t)BK * p.b_blocks_per_row;
+            const int64_t step = CB == 2 ? (kMajorB ? 0 : (int64_t)BK * p.mx_stride)
+                                         : 4 * (kMajorB ? 1 : (int64_t)BK * p.b_blocks_per_row);
             bool ok = true;
             for (int ks = 0; ks < nkt; ++ks, ++it) {
                 const int s = it % RSTAGES;
@@ -342,7 +366,8 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_con
                 const uint32_t am = smem_u32(stage + C::RAW_BYTES) + 4u * lane;
 #pragma unroll
                 for (int i = 0; i < PER_LANE; ++i) {
-                    cp_async_4(am + 128u * i, valid[i] ? src[i] + ks * step : p.absmax, valid[i] ? 4u : 0u);
+                    const uint8_t* a = src[i] + ks * step + ((CB == 2 && kMajorB) ? 4 * (ks >> 1) : 0);
+                    cp_async_4(am + 128u * i, valid[i] ? a : src[i], valid[i] ? 4u : 0u);
                 }
                 cp_async_mbar_arrive_noinc(rb);
             }
@@ -484,13 +509,23 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_con
 #pragma unroll
             for (int i = 0; i < NB; ++i) {
                 const int b = tg + TPG * i;
-                const BlockTable tb = make_table<CB>(a_cur[i]);
+                // MXFP4: the block's two 32-element halves have their own scales, bytes
+                // sel and sel+1 of the 4 copied (K-major: by k-stage; MN-major: by n-block)
+                BlockTable tb, tb1;
+                if (CB == 2) {
+                    const uint32_t sc = __float_as_uint(a_cur[i]);
+                    const int sel = kMajorB ? 2 * (cur_ks & 1) : 2 * (b >> 6);
+                    tb = make_table<CB>(mx_scale((sc >> (8 * sel)) & 0xFFu));
+                    tb1 = make_table<CB>(mx_scale((sc >> (8 * sel + 8)) & 0xFFu));
+                } else {
+                    tb = make_table<CB>(a_cur[i]);
+                }
                 const uint32_t words[8] = {pk[i][0].x, pk[i][0].y, pk[i][0].z, pk[i][0].w,
                                            pk[i][1].x, pk[i][1].y, pk[i][1].z, pk[i][1].w};
 #pragma unroll
                 for (int c = 0; c < 8; ++c) {
                     uint32_t o[4];
-                    decode_word(tb, words[c], o);
+                    decode_word((CB == 2 && c >= 4) ? tb1 : tb, words[c], o);
                     const uint32_t off = kMajorB ? sw128_offset(b, c) : (b >> 6) * 8192 + sw128_offset(b & 63, c);
                     *reinterpret_cast<uint4*>(dst_tile + off) = make_uint4(o[0], o[1], o[2], o[3]);
                 }
@@ -909,6 +944,23 @@ static cudaError_t launch_one(const CUtensorMap& ma, const CUtensorMap& mr, cons
     return cudaGetLastError();
 }
 
+// The instance for the epilogue kind and codebook: the extended epilogue (XACT) for the
+// gate_up variant (clamped GLU or biases) and for the routing-gradient dot products.
+template <int CB>
+static cudaError_t launch_cb(int epi, const CUtensorMap& ma, const CUtensorMap& mr, const CUtensorMap& mo,
+                             const CUtensorMap& mg, const CUtensorMap& ml, const GemmParams& p, int grid,
+                             cudaStream_t st) {
+    if (epi == EPI_GATEUP && (p.act != 0 || p.bias != nullptr))
+        return launch_one<EPI_GATEUP, CB, true>(ma, mr, mo, mg, ml, p, grid, st);
+    if (epi == EPI_DGRAD_DOWN && p.dw_part) return launch_one<EPI_DGRAD_DOWN, CB, true>(ma, mr, mo, mg, ml, p, grid, st);
+    switch (epi) {
+        case EPI_GATEUP: return launch_one<EPI_GATEUP, CB>(ma, mr, mo, mg, ml, p, grid, st);
+        case EPI_DOWN: return launch_one<EPI_DOWN, CB>(ma, mr, mo, mg, ml, p, grid, st);
+        case EPI_DGRAD_DOWN: return launch_one<EPI_DGRAD_DOWN, CB>(ma, mr, mo, mg, ml, p, grid, st);
+        default: return launch_one<EPI_DGRAD_GATEUP, CB>(ma, mr, mo, mg, ml, p, grid, st);
+    }
+}
+
 cudaError_t launch_grouped_gemm(int epi, int codebook, const void* a, int64_t a_rows, const uint8_t* packed,
                                 int64_t packed_rows_total, int packed_row_bytes, GemmParams p, int max_m_tiles,
                                 cudaStream_t st, const void* lora_a) {
@@ -951,32 +1003,14 @@ cudaError_t launch_grouped_gemm(int epi, int codebook, const void* a, int64_t a_
     const int64_t tiles = (int64_t)max_m_tiles * p.n_tiles;
     const int grid = (int)std::min<int64_t>(tiles * kCtas, (num_sms() / kCtas) * kCtas);
     if (grid <= 0) return cudaSuccess;
-#define E4B_LAUNCH(E_, C_) return launch_one<E_, C_>(ma, mr, mo, mg, ml, p, grid, st)
-    if (epi == EPI_GATEUP && (p.act != 0 || p.bias != nullptr)) {
-        if (codebook == 0) return launch_one<EPI_GATEUP, 0, true>(ma, mr, mo, mg, ml, p, grid, st);
-        return launch_one<EPI_GATEUP, 1, true>(ma, mr, mo, mg, ml, p, grid, st);
+if (epi == EPI_DGRAD_DOWN && p.dw_part && !p.h_in) return cudaErrorInvalidValue;
+    if (codebook == 2 && (!p.mx_scales || p.mx_stride < (p.b_blocks_per_row * 2 + 15) / 16 * 16))
+        return cudaErrorInvalidValue;
+    switch (codebook) {
+        case 0: return launch_cb<0>(epi, ma, mr, mo, mg, ml, p, grid, st);
+        case 1: return launch_cb<1>(epi, ma, mr, mo, mg, ml, p, grid, st);
+        default: return launch_cb<2>(epi, ma, mr, mo, mg, ml, p, grid, st);
     }
-    if (epi == EPI_DGRAD_DOWN && p.dw_part) {
-        if (!p.h_in) return cudaErrorInvalidValue;
-        if (codebook == 0) return launch_one<EPI_DGRAD_DOWN, 0, true>(ma, mr, mo, mg, ml, p, grid, st);
-        return launch_one<EPI_DGRAD_DOWN, 1, true>(ma, mr, mo, mg, ml, p, grid, st);
-    }
-    if (codebook == 0) {
-        switch (epi) {
-            case EPI_GATEUP: E4B_LAUNCH(EPI_GATEUP, 0);
-            case EPI_DOWN: E4B_LAUNCH(EPI_DOWN, 0);
-            case EPI_DGRAD_DOWN: E4B_LAUNCH(EPI_DGRAD_DOWN, 0);
-            default: E4B_LAUNCH(EPI_DGRAD_GATEUP, 0);
-        }
-    } else {
-        switch (epi) {
-            case EPI_GATEUP: E4B_LAUNCH(EPI_GATEUP, 1);
-            case EPI_DOWN: E4B_LAUNCH(EPI_DOWN, 1);
-            case EPI_DGRAD_DOWN: E4B_LAUNCH(EPI_DGRAD_DOWN, 1);
-            default: E4B_LAUNCH(EPI_DGRAD_GATEUP, 1);
-        }
-    }
-#undef E4B_LAUNCH
 }
 
 }  // namespace e4b

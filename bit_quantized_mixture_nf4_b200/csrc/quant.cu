@@ -95,10 +95,13 @@ __global__ void __launch_bounds__(256) quantize_kernel(const float* __restrict__
 }
 
 // One thread per 16 packed bytes (32 elements, half a block).
+// CB 2 (MXFP4): chunk c is one 32-element block; its scale byte is mx[row * S + j]
+// with row = c / nb, j = c % nb (nb = in / 32 blocks per row).
 template <int CB, bool BF16>
 __global__ void __launch_bounds__(256) dequantize_kernel(const uint8_t* __restrict__ packed,
                                                          const float* __restrict__ absmax, int64_t nchunks,
-                                                         void* __restrict__ out) {
+                                                         void* __restrict__ out, const uint8_t* __restrict__ mx,
+                                                         int64_t nb, int64_t S) {
     __shared__ float s_val[16];
     __shared__ uint4 s_stage[8][128];   // per warp: 32 lanes x 4 pieces of 16 bytes
     if (threadIdx.x < 16) s_val[threadIdx.x] = c_code[CB][threadIdx.x];
@@ -110,7 +113,8 @@ __global__ void __launch_bounds__(256) dequantize_kernel(const uint8_t* __restri
         const int64_t c = cw + (threadIdx.x & 31);
         const bool valid = c < nchunks;
         const uint4 pk = valid ? __ldcs(reinterpret_cast<const uint4*>(packed) + c) : make_uint4(0u, 0u, 0u, 0u);
-        const float a = valid ? __ldg(absmax + (c >> 1)) : 0.0f;
+        float a = 0.0f;
+        if (valid) a = (CB == 2) ? mx_scale(__ldg(mx + (c / nb) * S + c % nb)) : __ldg(absmax + (c >> 1));
         const uint32_t words[4] = {pk.x, pk.y, pk.z, pk.w};
         if (BF16) {
             // A warp's 32 chunks are 2 KB of contiguous output.  Each lane decodes
@@ -179,12 +183,95 @@ cudaError_t launch_dequantize(const uint8_t* packed, const float* absmax, int64_
     const int grid = grid_for(nchunks, 256);
     timing_begin(KK_DEQUANT, st);
     if (codebook == 0) {
-        if (out_bf16) dequantize_kernel<0, true><<<grid, 256, 0, st>>>(packed, absmax, nchunks, out);
-        else dequantize_kernel<0, false><<<grid, 256, 0, st>>>(packed, absmax, nchunks, out);
+        if (out_bf16) dequantize_kernel<0, true><<<grid, 256, 0, st>>>(packed, absmax, nchunks, out, nullptr, 1, 1);
+        else dequantize_kernel<0, false><<<grid, 256, 0, st>>>(packed, absmax, nchunks, out, nullptr, 1, 1);
     } else {
-        if (out_bf16) dequantize_kernel<1, true><<<grid, 256, 0, st>>>(packed, absmax, nchunks, out);
-        else dequantize_kernel<1, false><<<grid, 256, 0, st>>>(packed, absmax, nchunks, out);
+        if (out_bf16) dequantize_kernel<1, true><<<grid, 256, 0, st>>>(packed, absmax, nchunks, out, nullptr, 1, 1);
+        else dequantize_kernel<1, false><<<grid, 256, 0, st>>>(packed, absmax, nchunks, out, nullptr, 1, 1);
     }
+    timing_end(KK_DEQUANT, st);
+    count_launch();
+    return cudaGetLastError();
+}
+
+int64_t mxfp4_scale_stride(int64_t in) { return ((in / 32) + 15) / 16 * 16; }
+
+// MXFP4 quantize (OCP Microscaling Formats v1.0, the gpt-oss expert storage):
+// one thread per (row, scale byte j); j < in/32 quantizes the 32-element block j:
+// X = floor(log2 amax) - 2 = (biased exponent of amax) - 129, at least -127 (an
+// all-zero block: -127); each element v * 2^-X (exact) goes to the nearest E2M1
+// value, ties to the even code, saturating at 6; a zero result is +0.  Bytes
+// j >= in/32 are the row's zero padding.
+__global__ void __launch_bounds__(256) quantize_mxfp4_kernel(const float* __restrict__ w, int64_t rows, int64_t in,
+                                                             int64_t S, uint8_t* __restrict__ packed,
+                                                             uint8_t* __restrict__ scales) {
+    const int64_t nb = in / 32, total = rows * S;
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < total; i += (int64_t)gridDim.x * blockDim.x) {
+        const int64_t r = i / S, j = i - r * S;
+        if (j >= nb) {
+            scales[i] = 0;
+            continue;
+        }
+        const float4* src = reinterpret_cast<const float4*>(w + r * in + j * 32);
+        float v[32];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+            const float4 f = __ldcs(src + k);
+            v[4 * k] = f.x; v[4 * k + 1] = f.y; v[4 * k + 2] = f.z; v[4 * k + 3] = f.w;
+        }
+        float amax = 0.0f;
+#pragma unroll
+        for (int k = 0; k < 32; ++k) amax = fmaxf(amax, fabsf(v[k]));
+        const int eb = (int)((__float_as_uint(amax) >> 23) & 0xFFu);   // biased exponent (0: zero / subnormal)
+        const int X = max(eb - 129, -127);
+        scales[i] = (uint8_t)(X + 127);
+        const float inv = __int_as_float((127 - X) << 23);   // 2^-X, a normal float for X in [-127, 125]
+        uint32_t words[4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            uint32_t wv = 0;
+#pragma unroll
+            for (int t = 0; t < 8; ++t) {
+                const float p = __fmul_rn(v[8 * k + t], inv);
+                const float a = fabsf(p);
+                // nearest E2M1 magnitude: ties at 0.25, 1.25, 2.5, 5 go down (even code below),
+                // at 0.75, 1.75, 3.5 up (even code above); 6 and beyond saturate to code 7
+                uint32_t c = (a > 0.25f) + (a >= 0.75f) + (a > 1.25f) + (a >= 1.75f) + (a > 2.5f) + (a >= 3.5f) +
+                             (a > 5.0f);
+                if (amax == 0.0f) c = 0;
+                if (c != 0 && p < 0.0f) c |= 8u;
+                // element 2b in the high nibble of byte b: byte t/2 of the word, high nibble for even t
+                wv |= c << (8 * (t >> 1) + ((t & 1) ? 0 : 4));
+            }
+            words[k] = wv;
+        }
+        *reinterpret_cast<uint4*>(packed + (r * in + j * 32) / 2) = make_uint4(words[0], words[1], words[2], words[3]);
+    }
+}
+
+cudaError_t launch_quantize_mxfp4(const float* w, int64_t rows, int64_t in, uint8_t* packed, uint8_t* scales,
+                                  cudaStream_t st) {
+    if (rows == 0 || in == 0) return cudaSuccess;
+    if (in % 32) return cudaErrorInvalidValue;
+    const int64_t S = mxfp4_scale_stride(in);
+    const int grid = grid_for(rows * S, 256);
+    timing_begin(KK_QUANT, st);
+    quantize_mxfp4_kernel<<<grid, 256, 0, st>>>(w, rows, in, S, packed, scales);
+    timing_end(KK_QUANT, st);
+    count_launch();
+    return cudaGetLastError();
+}
+
+cudaError_t launch_dequantize_mxfp4(const uint8_t* packed, const uint8_t* scales, int64_t rows, int64_t in,
+                                    int out_bf16, void* out, cudaStream_t st) {
+    if (in % 32) return cudaErrorInvalidValue;
+    const int64_t nchunks = rows * (in / 32);
+    if (nchunks == 0) return cudaSuccess;
+    const int grid = grid_for(nchunks, 256);
+    const int64_t nb = in / 32, S = mxfp4_scale_stride(in);
+    timing_begin(KK_DEQUANT, st);
+    if (out_bf16) dequantize_kernel<2, true><<<grid, 256, 0, st>>>(packed, nullptr, nchunks, out, scales, nb, S);
+    else dequantize_kernel<2, false><<<grid, 256, 0, st>>>(packed, nullptr, nchunks, out, scales, nb, S);
     timing_end(KK_DEQUANT, st);
     count_launch();
     return cudaGetLastError();

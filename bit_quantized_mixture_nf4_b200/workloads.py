@@ -18,7 +18,7 @@ import math
 
 import torch
 
-NF4, FP4 = 0, 1
+NF4, FP4, MXFP4 = 0, 1, 2   # MXFP4: the gpt-oss experts' native storage (32-element E8M0 blocks)
 
 
 @dataclasses.dataclass(frozen=True)

@@ -60,7 +60,14 @@ typedef enum {
     E4B_ERR_TIMEOUT = 6        /* a device-side wait hit its time limit                   */
 } e4b_status;
 
-typedef enum { E4B_CODEBOOK_NF4 = 0, E4B_CODEBOOK_FP4 = 1 } e4b_codebook;
+/* NF4 / FP4: 64-element blocks with an fp32 absmax (the 4-bit stacks above).
+ * MXFP4: the gpt-oss experts' native storage ([P2] "Scope"), read as the OCP
+ * Microscaling Formats v1.0 MXFP4: 32-element blocks sharing an E8M0 scale
+ * 2^(s - 127) (one byte s), FP4 E2M1 elements (sign in bit 3, magnitudes
+ * {0, .5, 1, 1.5, 2, 3, 4, 6}), packed like the 4-bit stacks; scales uint8
+ * [E, out, S] with S = e4b_mxfp4_scale_stride(in) (in/32 rounded up to a multiple
+ * of 16, padding bytes 0).  The descriptor's blocksize is 32 for MXFP4. */
+typedef enum { E4B_CODEBOOK_NF4 = 0, E4B_CODEBOOK_FP4 = 1, E4B_CODEBOOK_MXFP4 = 2 } e4b_codebook;
 typedef enum { E4B_F32 = 0, E4B_BF16 = 1 } e4b_dtype;
 typedef enum { E4B_PATH_AUTO = 0, E4B_PATH_GROUPED = 1, E4B_PATH_DECODE = 2 } e4b_path;
 /* The experts' gated activation of the pre-activations g (gate rows) and u (up rows):
@@ -73,7 +80,8 @@ typedef enum { E4B_PATH_AUTO = 0, E4B_PATH_GROUPED = 1, E4B_PATH_DECODE = 2 } e4
 typedef enum { E4B_ACT_SWIGLU = 0, E4B_ACT_CLAMPED_GLU = 1 } e4b_activation;
 
 /* Layer description.  H and I must be multiples of 64 (blocks never straddle a
- * row, [P4] __init__); 1 <= top_k <= min(E, 8); E <= 256; blocksize == 64.
+ * row, [P4] __init__); 1 <= top_k <= min(E, 8); E <= 256; blocksize == 64
+ * (32 for E4B_CODEBOOK_MXFP4).
  * path: AUTO takes the weight-streaming decode kernels for T <= 8 when no
  * grouped outputs are requested and the shapes fit them (H <= 8192, and the
  * per-warp stage rings of 16 rows plus the tokens' activation rows fit in
@@ -119,6 +127,8 @@ typedef struct {
     const void *lora_B_gu;         /* bf16 [E, 2I, r] (gate rows first, like the stack) */
     const void *lora_A_d;          /* bf16 [E, r, I]  */
     const void *lora_B_d;          /* bf16 [E, H, r]  */
+    const uint8_t *gate_up_scales; /* MXFP4 only (then the absmax pointers are unused): [E, 2I, S(H)] */
+    const uint8_t *down_scales;    /*                                                    [E, H, S(I)]  */
 } e4b_experts;
 
 /* Gradients of the four adapters (fp32, shaped like them; each fully written),
@@ -138,6 +148,21 @@ typedef struct {
  * Non-finite inputs are outside the contract. */
 E4B_API e4b_status e4b_quantize_nf4(const float *w, int64_t E, int64_t out, int64_t in, int blocksize,
                             e4b_codebook codebook, uint8_t *packed, float *absmax, void *stream);
+
+/* MXFP4 quantization (OCP MX v1.0 conversion): for every 32-element block of
+ * each row, X = floor(log2(max|w|)) - 2 clamped to [-127, 127] (an all-zero block:
+ * -127), scale byte X + 127; each element w / 2^X rounded to the nearest E2M1
+ * value, ties to the even code, saturating at 6, a zero result stored as +0.
+ * Writes packed [E, out*in/2] and scales [E, out, e4b_mxfp4_scale_stride(in)].
+ * Errors: E4B_ERR_BLOCKSIZE if in % 32 != 0; E4B_ERR_INVALID_ARG for null
+ * pointers or negative sizes. */
+E4B_API int64_t e4b_mxfp4_scale_stride(int64_t in);
+E4B_API e4b_status e4b_quantize_mxfp4(const float *w, int64_t E, int64_t out, int64_t in, uint8_t *packed,
+                              uint8_t *scales, void *stream);
+/* MXFP4 dequantization: e2m1(code) * 2^(s - 127) in fp32 (exact), then bf16
+ * nearest-even (exact for these values) when out_dtype == E4B_BF16. */
+E4B_API e4b_status e4b_dequantize_mxfp4(const uint8_t *packed, const uint8_t *scales, int64_t E, int64_t out,
+                                int64_t in, e4b_dtype out_dtype, void *w_out, void *stream);
 
 /* Dequantization ([P4] _dequantize_expert): value = code_value * absmax with
  * one fp32 multiply, then (out_dtype == E4B_BF16) rounded to bf16 nearest-even.

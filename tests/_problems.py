@@ -45,8 +45,12 @@ def build(w: wl.Workload) -> Problem:
     go = wl.grad_output(w)
     gu = gu.numpy()
     dn = dn.numpy()
-    pg, ag = oracle.quantize(gu, w.codebook)
-    pd, ad = oracle.quantize(dn, w.codebook)
+    if w.codebook == wl.MXFP4:   # packed codes + E8M0 scale bytes (in ag / ad)
+        pg, ag = oracle.quantize_mxfp4(gu)
+        pd, ad = oracle.quantize_mxfp4(dn)
+    else:
+        pg, ag = oracle.quantize(gu, w.codebook)
+        pd, ad = oracle.quantize(dn, w.codebook)
     prob = Problem(w, x, logits, go, gu, dn, pg, ag, pd, ad)
     if len(_cache) > 2:
         _cache.clear()
@@ -60,6 +64,10 @@ def oracle_weights(prob: Problem, experts=None):
     if experts is None:
         experts = np.arange(w.E)
     experts = np.asarray(experts)
+    if w.codebook == wl.MXFP4:
+        wgu = oracle.dequantize_mxfp4(prob.pg[experts], prob.ag[experts], (len(experts), 2 * w.I, w.H))
+        wd = oracle.dequantize_mxfp4(prob.pd[experts], prob.ad[experts], (len(experts), w.H, w.I))
+        return wgu, wd
     wgu = oracle.dequantize(prob.pg[experts], prob.ag[experts], (len(experts), 2 * w.I, w.H), w.codebook)
     wd = oracle.dequantize(prob.pd[experts], prob.ad[experts], (len(experts), w.H, w.I), w.codebook)
     return wgu, wd

@@ -110,6 +110,16 @@ def test_host_side_validation(lib):
     assert b(4, gl=16) == lib.E4B_ERR_INVALID_ARG                      # grad_logits needs router_logits
     assert b(4, logits=16, gw=None, gl=16) == lib.E4B_ERR_INVALID_ARG  # ... and grad_topk_w
     assert b(4) == lib.E4B_ERR_WORKSPACE                               # valid request, no workspace
+    # MXFP4: blocksize 32 with that codebook only; the scale arrays replace absmax
+    mxd = lib.make_desc(8, 256, 512, 2, codebook=lib.MXFP4, blocksize=32)
+    assert lib.e4b_moe_workspace_size(mxd, 64) > 0
+    assert lib.e4b_moe_workspace_size(lib.make_desc(8, 256, 512, 2, codebook=lib.MXFP4), 64) == 0   # blocksize 64
+    assert lib.e4b_moe_workspace_size(lib.make_desc(8, 256, 512, 2, blocksize=32), 64) == 0         # NF4 at 32
+    assert f(mxd, 4, 16, 16, 1 << 40) == lib.E4B_ERR_INVALID_ARG      # scales missing
+    assert lib.e4b_mxfp4_scale_stride(2880) == 96 and lib.e4b_mxfp4_scale_stride(512) == 16
+    assert L.e4b_quantize_mxfp4(nullp, 1, 2, 48, nullp, nullp, nullp) == lib.E4B_ERR_BLOCKSIZE
+    assert L.e4b_quantize_mxfp4(nullp, 1, 2, 64, nullp, nullp, nullp) == lib.E4B_ERR_INVALID_ARG
+    assert L.e4b_dequantize_mxfp4(nullp, nullp, 1, 2, 64, 7, nullp, nullp) == lib.E4B_ERR_INVALID_ARG
     # LoRA: rank a multiple of 8 up to 64, finite scale, all four adapters present
     for bad in (lib.make_desc(8, 256, 512, 2, lora_rank=12), lib.make_desc(8, 256, 512, 2, lora_rank=72),
                 lib.make_desc(8, 256, 512, 2, lora_rank=-8),
