@@ -25,6 +25,7 @@ value = tokens of all ranks / max-over-ranks device time.
 from __future__ import annotations
 
 import argparse
+import dataclasses
 import hashlib
 import json
 import os
@@ -52,6 +53,8 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-aux", action="store_true", help="skip the secondary legs")
+    ap.add_argument("--codebook", default="native", choices=["native", "mxfp4"],
+                    help="variant leg: the workload's own 4-bit codebook or native MXFP4 storage")
     ap.add_argument("--leg", default="step", choices=["step", "decode", "codec", "variant", "router", "lora"],
                     help="step: the benchmark line; decode / codec / variant / router: only that secondary leg "
                          "(for profiling); decode runs the Qwen3-shaped layer (or --workload) at --tokens "
@@ -68,7 +71,7 @@ def headline_workload(args):
 def workload_desc(w) -> str:
     rt = "zipf-skewed routing, " if w.router == "zipf" else ""
     return (f"{w.name}-shaped E={w.E} H={w.H} I={w.I} top{w.k} {'renorm' if w.renorm else 'no-renorm'} T={w.T}/GPU, "
-            f"{'fp4' if w.codebook else 'nf4'} blocksize 64, {rt}fwd (routed from logits, g/u saved) + dgrad")
+            f"{('nf4', 'fp4', 'mxfp4')[w.codebook]} blocksize 64, {rt}fwd (routed from logits, g/u saved) + dgrad")
 
 
 def bench_config(w, world):
@@ -230,8 +233,10 @@ class Layer:
         self.logits_h = wl.router_logits(w, self.x_h)
         self.go_h = wl.grad_output(w)
         gu, dn = wl.weights(w, device=dev)
-        self.pg, self.ag = e4b.e4b_quantize_nf4(gu, codebook=w.codebook)
-        self.pd, self.ad = e4b.e4b_quantize_nf4(dn, codebook=w.codebook)
+        self.mx = w.codebook == wl.MXFP4   # native MXFP4: packed codes + E8M0 scale bytes
+        quant = e4b.e4b_quantize_mxfp4 if self.mx else (lambda t: e4b.e4b_quantize_nf4(t, codebook=w.codebook))
+        self.pg, self.ag = quant(gu)
+        self.pd, self.ad = quant(dn)
         del gu, dn
         self.bgu = self.bd = None
         if biases:
@@ -249,9 +254,13 @@ class Layer:
             self.lora = tuple((torch.randn(a, b, c, device=dev, generator=g) * v ** 0.5).to(torch.bfloat16)
                               for a, b, c, v in shapes)
             self.lora_grads = tuple(torch.empty(t.shape, dtype=torch.float32, device=dev) for t in self.lora)
-        self.experts = e4b.make_experts(self.pg, self.pd, self.ag, self.ad, self.bgu, self.bd, lora=self.lora)
-        self.desc = e4b.make_desc(w.E, w.H, w.I, w.k, w.renorm, w.codebook, 64, path, act, 1.702, 7.0,
-                                  lora_rank=lora_rank, lora_scale=2.0)
+        if self.mx:
+            self.experts = e4b.make_experts(self.pg, self.pd, None, None, self.bgu, self.bd, lora=self.lora,
+                                            gate_up_scales=self.ag, down_scales=self.ad)
+        else:
+            self.experts = e4b.make_experts(self.pg, self.pd, self.ag, self.ad, self.bgu, self.bd, lora=self.lora)
+        self.desc = e4b.make_desc(w.E, w.H, w.I, w.k, w.renorm, w.codebook, 32 if self.mx else 64, path, act, 1.702,
+                                  7.0, lora_rank=lora_rank, lora_scale=2.0)
         T, P = w.T, w.P
         self.x = self.x_h.to(dev)
         self.logits = self.logits_h.to(dev)
@@ -421,7 +430,7 @@ def decode_leg(w, dev, reps=20):
     if e4b.e4b_device_status() != e4b.E4B_OK:
         raise RuntimeError("device status not ok after the decode leg")
     return {"workload": f"{w.name}-shaped E={w.E} H={w.H} I={w.I} top{w.k} T={w.T} "
-                        f"{'fp4' if w.codebook else 'nf4'}", "us_per_forward": st,
+                        f"{('nf4', 'fp4', 'mxfp4')[w.codebook]}", "us_per_forward": st,
             "experts_touched": touched, "bytes_per_forward": nbytes, "weight_stream_gbs": gbs,
             "roofline": {"bound": "hbm", "achieved": gbs, "peak": hbm, "unit": "GB/s", "frac": gbs / hbm},
             "layer_copies": copies, "touched_bytes_all_copies": nbytes * copies,
@@ -584,7 +593,7 @@ def codec_leg(w, dev, reps=10):
         gbs = n * bpe / (us * 1e-6) / 1e9
         res[name] = {"elements": n, "us": us, "achieved": gbs, "peak": hbm, "unit": "GB/s", "frac": gbs / hbm,
                      "bytes_per_element": bpe}
-    res["workload"] = f"{w.name}-shaped gate_up stack [{w.E},{2 * w.I},{w.H}] {'fp4' if w.codebook else 'nf4'}"
+    res["workload"] = f"{w.name}-shaped gate_up stack [{w.E},{2 * w.I},{w.H}] {('nf4', 'fp4', 'mxfp4')[w.codebook]}"
     del gu, out
     torch.cuda.empty_cache()
     return res
@@ -609,6 +618,14 @@ def reconstruction_leg(w, dev):
             den += float(stack.double().pow(2).sum())
             del p, a, d
         res[f"{name}_rel_rmse"] = (num / den) ** 0.5
+    num = den = 0.0
+    for stack in (gu, dn):   # native MXFP4 (32-element blocks, E8M0 scales)
+        p, sc = e4b.e4b_quantize_mxfp4(stack)
+        d = e4b.e4b_dequantize_mxfp4(p, sc, tuple(stack.shape))
+        num += float((stack - d.float()).double().pow(2).sum())
+        den += float(stack.double().pow(2).sum())
+        del p, sc, d
+    res["mxfp4_rel_rmse"] = (num / den) ** 0.5
     del gu, dn
     torch.cuda.empty_cache()
     return res
@@ -849,6 +866,8 @@ def run_e4b(args, w):
         aux["codec"] = codec_leg(wl.OLMOE, dev)
         aux["reconstruction_nf4_vs_fp4"] = reconstruction_leg(wl.GPTOSS, dev)
         aux["gptoss_variant"] = variant_leg(wl.GPTOSS.with_tokens(2048), dev, flush)
+        aux["gptoss_variant_mxfp4"] = variant_leg(dataclasses.replace(wl.GPTOSS.with_tokens(2048),
+                                                                      codebook=wl.MXFP4), dev, flush)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -901,7 +920,10 @@ def main():
             print(json.dumps({"router_fused": router_fused_leg(layer, flush, steps=max(args.steps, 3)),
                               "router_backward": router_leg(layer, flush, steps=max(args.steps, 3))}), flush=True)
         elif args.leg == "variant":
-            print(json.dumps(variant_leg(wl.GPTOSS.with_tokens(2048), dev, flush, steps=max(args.steps, 3))),
+            vw = wl.GPTOSS.with_tokens(2048)
+            if args.codebook == "mxfp4":
+                vw = dataclasses.replace(vw, codebook=wl.MXFP4)
+            print(json.dumps(variant_leg(vw, dev, flush, steps=max(args.steps, 3))),
                   flush=True)
         else:
             print(json.dumps(codec_leg(wl.OLMOE, dev, reps=max(args.steps, 3))), flush=True)
