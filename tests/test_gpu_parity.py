@@ -214,10 +214,28 @@ def test_forward_and_dgrad_medium(e4b, w):
     _check_status(e4b)
 
 
+def _tile_edge_tokens(idx, E, k, tile_rows=256):
+    """Tokens owning the first and the last grouped row of every expert's first and
+    last m-tile (from the oracle's permutation): each expert's first and last tile
+    then has checked rows."""
+    counts, offsets, perm = oracle.permute(idx, E)
+    toks = set()
+    for e in range(E):
+        lo, hi = int(offsets[e]), int(offsets[e + 1])
+        if hi == lo:
+            continue
+        last0 = lo + (hi - 1 - lo) // tile_rows * tile_rows   # first row of the last m-tile
+        for row in (lo, min(lo + tile_rows, hi) - 1, last0, hi - 1):
+            toks.add(int(perm[row]) // k)
+    return np.array(sorted(toks), np.int64)
+
+
 @pytest.mark.parametrize("wname,T", [("olmoe", 4096), ("qwen3", 8192), ("mixtral", 16384), ("gptoss", 2048)])
 def test_forward_and_dgrad_full_size_sampled(e4b, wname, T):
     """Full-size layer in the launch configuration the benchmark uses; routing,
-    offsets and permutation checked on every token, y and grad_x on sampled tokens."""
+    offsets and permutation checked on every token, y and grad_x on sampled tokens:
+    random ones plus the owners of the first and last rows of every expert's first
+    and last m-tile."""
     w = wl.ALL[wname].with_tokens(T)
     prob = pb.build(w)
     r = _run_forward(e4b, prob, path=e4b.PATH_GROUPED)
@@ -226,7 +244,7 @@ def test_forward_and_dgrad_full_size_sampled(e4b, wname, T):
     gx = e4b.e4b_moe_backward_dgrad(r["d"], r["experts"], r["x"], r["idx"], r["wts"], go, saved_gu=r["gu"])
     torch.cuda.synchronize()
     _check_status(e4b)
-    toks = _sample_tokens(T, 12 if wname == "mixtral" else 24, seed=T)
+    toks = np.union1d(_sample_tokens(T, 12 if wname == "mixtral" else 24, seed=T), _tile_edge_tokens(oi, w.E, w.k))
     yref, gref = pb.oracle_forward_dgrad(prob, oi, ow, toks)
     pb.assert_close_rel_max(r["y"].float().cpu().numpy()[toks], yref, TOL, "forward")
     pb.assert_close_rel_max(gx.float().cpu().numpy()[toks], gref, TOL, "dgrad")
