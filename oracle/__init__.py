@@ -16,6 +16,12 @@ Parity status of each function (what pins it is in ``tests/test_oracle_pins.py``
   route / permute        pinned (brute-force sort, softmax ratio closed form, bijection)
   forward                pinned (fp64 dense all-experts reference; E=1 dense SwiGLU MLP)
   dgrad                  pinned (central finite differences; adjoint identity)
+  int8 / fp8 quantize / dequantize
+                         pinned (fp8 values vs torch's float8_e4m3fn decoding, int8 map
+                         structure from its definition, exact reproduction, tie rule,
+                         idempotence, round-trip bound, the support matrix's error
+                         ordering int8 < fp8 < nf4 < fp4); parity with bitsandbytes'
+                         own tables unpinned (not on the pages)
   MXFP4 quantize / dequantize
                          pinned (exact reproduction of scaled E2M1 values, the scale
                          exponent on hand-picked maxima and its clamp, ties to even,
@@ -38,6 +44,7 @@ _lock = threading.Lock()
 _lib = None
 
 NF4, FP4 = 0, 1
+INT8, FP8 = 3, 4      # 8-bit blockwise codebooks (one byte per element)
 
 
 def build(force: bool = False) -> str:
@@ -63,6 +70,9 @@ def _L():
             lib.e4bo_dequantize_f32.argtypes = [P, P, i64, i32, i32, P]
             lib.e4bo_dequantize_bf16.argtypes = [P, P, i64, i32, i32, P]
             lib.e4bo_quantize_mxfp4.argtypes = [P, i64, i64, i64, P, P]
+            lib.e4bo_quantize8.argtypes = [P, i64, i64, i64, i32, P, P]
+            lib.e4bo_dequantize8.argtypes = [P, P, i64, i32, i32, P]
+            lib.e4bo_codebook8.argtypes = [i32, P]
             lib.e4bo_dequantize_mxfp4.argtypes = [P, P, i64, i64, i64, i32, P]
             lib.e4bo_mxfp4_scale_stride.argtypes = [i64]
             lib.e4bo_mxfp4_scale_stride.restype = i64
@@ -150,6 +160,38 @@ def dequantize(packed: np.ndarray, absmax: np.ndarray, shape, cb: int = NF4,
         return out.reshape(shape)
     bits = np.zeros(n, np.uint16)
     _check("e4bo_dequantize_bf16", _L().e4bo_dequantize_bf16(_p(packed), _p(absmax), n, blocksize, cb, _p(bits)))
+    bits = bits.reshape(shape)
+    return bits if out_dtype == "bf16_bits" else bf16_bits_to_f32(bits)
+
+
+def codebook8(cb: int) -> np.ndarray:
+    """The 256 values of an 8-bit codebook (INT8 or FP8), indexed by code (NaN
+    for the FP8 NaN patterns)."""
+    out = np.zeros(256, np.float32)
+    _L().e4bo_codebook8(cb, _p(out))
+    return out
+
+
+def quantize8(w: np.ndarray, cb: int):
+    """w: fp32 [E, out, in] -> (codes uint8 [E, out*in], absmax fp32 [E, out*in/64])."""
+    w = np.ascontiguousarray(w, np.float32)
+    E, o, i = w.shape
+    codes = np.zeros((E, o * i), np.uint8)
+    absmax = np.zeros((E, o * i // 64), np.float32)
+    _check("e4bo_quantize8", _L().e4bo_quantize8(_p(w), E, o, i, cb, _p(codes), _p(absmax)))
+    return codes, absmax
+
+
+def dequantize8(codes: np.ndarray, absmax: np.ndarray, shape, cb: int, out_dtype: str = "bf16") -> np.ndarray:
+    codes = np.ascontiguousarray(codes, np.uint8)
+    absmax = np.ascontiguousarray(absmax, np.float32)
+    n = int(np.prod(shape))
+    if out_dtype == "f32":
+        out = np.zeros(n, np.float32)
+        _check("e4bo_dequantize8", _L().e4bo_dequantize8(_p(codes), _p(absmax), n, cb, 0, _p(out)))
+        return out.reshape(shape)
+    bits = np.zeros(n, np.uint16)
+    _check("e4bo_dequantize8", _L().e4bo_dequantize8(_p(codes), _p(absmax), n, cb, 1, _p(bits)))
     bits = bits.reshape(shape)
     return bits if out_dtype == "bf16_bits" else bf16_bits_to_f32(bits)
 

@@ -188,6 +188,110 @@ int e4bo_dequantize_bf16(const uint8_t *packed, const float *absmax, int64_t n,
     return ORC_OK;
 }
 
+/* ---- 8-bit blockwise modes ([P1] "Storage modes: the support matrix") -----
+ * int8 is a "blockwise dynamic map" and fp8 a "bnb e4m3 codebook"; the pages
+ * print neither table.  Readings taken, both normalised to max 1 and used like
+ * the 4-bit codebooks (64-element blocks, fp32 absmax, nearest value with an
+ * exact tie going to the smaller value, one byte per element):
+ *   int8: the dynamic tree quantization of Dettmers et al. (2022, "8-bit
+ *     optimizers via block-wise quantization"): bit 7 the sign; in the 7-bit tail
+ *     the number E of leading zeros is a decimal exponent, the first 1 bit an
+ *     indicator, and the F = 6 - E bits after it a linear fraction j on
+ *     [0.1, 1]: |value| = 10^-E (0.1 + 0.9 (j + 1/2) / 2^F), the centres of 2^F
+ *     equal bins.  Tail 0 is 0 (sign clear) or +1 (sign set: the absmax element);
+ *   fp8: the E4M3 values (OCP 8-bit floating point: bias 7, subnormals, 448 the
+ *     largest, S.1111.111 NaN) divided by 448; the code is the E4M3 bit pattern
+ *     (the two NaNs and -0 are never produced).
+ * With these, the reconstruction error ordering of the support matrix holds:
+ * int8 < fp8 < nf4 < fp4. */
+
+static float int8_value(int code) {
+    const int s = code >> 7, t = code & 127;
+    if (t == 0) return s ? 1.0f : 0.0f;
+    int E = 0;
+    while (!(t & (64 >> E))) ++E;              /* leading zeros of the 7-bit tail */
+    const int F = 6 - E, j = t & ((1 << F) - 1);
+    const double v = pow(10.0, -E) * (0.1 + 0.9 * (j + 0.5) / (double)(1 << F));
+    return (float)(s ? -v : v);
+}
+
+static float fp8_value(int code) {   /* NaN patterns give NaN, never produced */
+    const int s = code >> 7, e = (code >> 3) & 15, m = code & 7;
+    if (e == 15 && m == 7) return NAN;
+    const double mag = (e == 0) ? (m / 8.0) * pow(2.0, -6) : (1.0 + m / 8.0) * pow(2.0, e - 7);
+    const float v = (float)(mag / 448.0);
+    return s ? -v : v;
+}
+
+/* codebook 3 = int8, 4 = fp8: value of a byte code */
+float e4bo_code_value8(int cb, int q) { return cb == 3 ? int8_value(q & 255) : fp8_value(q & 255); }
+
+/* The distinct values in ascending order with their codes (fp8: NaNs and -0
+ * dropped). */
+static int sorted_codebook8(int cb, float *vals, int *codes) {
+    int n = 0;
+    for (int q = 0; q < 256; ++q) {
+        const float v = e4bo_code_value8(cb, q);
+        if (v != v) continue;
+        if (cb == 4 && q == 0x80) continue;
+        vals[n] = v;
+        codes[n] = q;
+        ++n;
+    }
+    for (int i = 1; i < n; ++i)   /* insertion sort by value */
+        for (int k = i; k > 0 && vals[k - 1] > vals[k]; --k) {
+            float tv = vals[k]; vals[k] = vals[k - 1]; vals[k - 1] = tv;
+            int tc = codes[k]; codes[k] = codes[k - 1]; codes[k - 1] = tc;
+        }
+    return n;
+}
+
+void e4bo_codebook8(int cb, float *out256) {
+    for (int q = 0; q < 256; ++q) out256[q] = e4bo_code_value8(cb, q);
+}
+
+/* w fp32 [E, out, in] -> codes [E, out*in] (one byte per element), absmax
+ * [E, out*in/64]; the quantization rule of e4bo_quantize with the 8-bit table. */
+int e4bo_quantize8(const float *w, int64_t E, int64_t out, int64_t in, int cb, uint8_t *codes, float *absmax) {
+    if (!w || !codes || !absmax || E < 0 || out < 0 || in < 0 || (cb != 3 && cb != 4)) return ORC_ERR_ARG;
+    if (in % 64) return ORC_ERR_BLOCKSIZE;
+    float vals[256], mid[255];
+    int cds[256];
+    const int nv = sorted_codebook8(cb, vals, cds);
+    for (int i = 0; i + 1 < nv; ++i) mid[i] = (vals[i] + vals[i + 1]) * 0.5f;
+    int zero_code = 0;
+    for (int i = 0; i < nv; ++i)
+        if (vals[i] == 0.0f) zero_code = cds[i];
+    const int64_t nblocks = E * out * in / 64;
+#pragma omp parallel for schedule(static)
+    for (int64_t b = 0; b < nblocks; ++b) {
+        const float *src = w + b * 64;
+        float a = 0.0f;
+        for (int i = 0; i < 64; ++i) a = fmaxf(a, fabsf(src[i]));
+        absmax[b] = a;
+        for (int i = 0; i < 64; ++i) {
+            if (a == 0.0f) { codes[b * 64 + i] = (uint8_t)zero_code; continue; }
+            const float n = src[i] / a;
+            int r = 0;
+            for (int m = 0; m < nv - 1; ++m) r += (mid[m] < n) ? 1 : 0;
+            codes[b * 64 + i] = (uint8_t)cds[r];
+        }
+    }
+    return ORC_OK;
+}
+
+/* value = code value * absmax in fp32, then bf16 (bf16 != 0) or fp32 */
+int e4bo_dequantize8(const uint8_t *codes, const float *absmax, int64_t n, int cb, int bf16, void *dst) {
+    if (!codes || !absmax || !dst || n < 0 || n % 64 || (cb != 3 && cb != 4)) return ORC_ERR_ARG;
+#pragma omp parallel for schedule(static)
+    for (int64_t i = 0; i < n; ++i) {
+        const float v = e4bo_code_value8(cb, codes[i]) * absmax[i / 64];
+        if (bf16) ((uint16_t *)dst)[i] = e4bo_f32_to_bf16(v);
+        else ((float *)dst)[i] = v;
+    }
+    return ORC_OK;
+}
+
 /* ---- MXFP4 ([P2] "Scope": the gpt-oss experts ship MXFP4 weights) --------
  * The pages name the format only; the reading taken is the OCP Microscaling
  * Formats (MX) v1.0 specification: blocks of 32 consecutive elements of a row
