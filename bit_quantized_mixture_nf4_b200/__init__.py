@@ -19,7 +19,7 @@ LIB_PATH = os.path.join(_HERE, "libe4b.so")
 
 E4B_OK, E4B_ERR_INVALID_ARG, E4B_ERR_BLOCKSIZE, E4B_ERR_UNSUPPORTED, E4B_ERR_WORKSPACE, E4B_ERR_CUDA, \
     E4B_ERR_TIMEOUT = range(7)
-NF4, FP4, MXFP4 = 0, 1, 2
+NF4, FP4, MXFP4, INT8, FP8, BF16_WEIGHTS = 0, 1, 2, 3, 4, 5   # storage formats (e4b_codebook)
 F32, BF16 = 0, 1
 PATH_AUTO, PATH_GROUPED, PATH_DECODE = 0, 1, 2
 ACT_SWIGLU, ACT_CLAMPED_GLU = 0, 1
@@ -188,13 +188,14 @@ def e4b_device_status(stream=None) -> int:
 
 def e4b_quantize_nf4(w: torch.Tensor, blocksize: int = 64, codebook: int = NF4, packed=None, absmax=None,
                      stream=None):
-    """w: fp32 [E, out, in] on the GPU -> (packed uint8 [E, out*in/2], absmax fp32 [E, out*in/64])."""
+    """w: fp32 [E, out, in] on the GPU -> (packed uint8 [E, out*in/2] (the 8-bit
+    codebooks INT8 / FP8: [E, out*in], one byte per element), absmax fp32 [E, out*in/64])."""
     _cuda(w, "w", torch.float32)
     if w.dim() != 3:
         raise ValueError("w must be a 3-D [E, out, in] stack")
     E, o, i = w.shape
     if packed is None:
-        packed = torch.empty(E, o * i // 2, dtype=torch.uint8, device=w.device)
+        packed = torch.empty(E, o * i // (1 if codebook in (INT8, FP8) else 2), dtype=torch.uint8, device=w.device)
     if absmax is None:
         absmax = torch.empty(E, o * i // max(blocksize, 1), dtype=torch.float32, device=w.device)
     _check("e4b_quantize_nf4", _load().e4b_quantize_nf4(_ptr(w), E, o, i, blocksize, codebook, _ptr(packed), _ptr(absmax),

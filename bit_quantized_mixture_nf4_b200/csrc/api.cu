@@ -99,7 +99,7 @@ uint32_t* device_status_ptr() {
 // ------------------------------------------------------------ workspace layout
 struct WsLayout {
     size_t chunk_counts, chunk_base, counts, offsets, tile_prefix, sched, perm, inv_perm, a_perm, h, gu, dgu, dec, ones,
-        dw_part, lz_gu, lz_d, lv_d, lv_gu, x_perm, lbt_gu, lbt_d, total;
+        dw_part, lz_gu, lz_d, lv_d, lv_gu, x_perm, lbt_gu, lbt_d, wbf16, total;
 };
 
 static size_t align_up(size_t v) { return (v + 255) & ~size_t(255); }
@@ -138,6 +138,8 @@ static WsLayout layout_for(const e4b_moe_desc* d, int64_t T) {
         L.lbt_gu = take((size_t)d->E * d->lora_rank * 2 * d->I * 2);   // B_gu as [E, r, 2I]
         L.lbt_d = take((size_t)d->E * d->lora_rank * d->H * 2);        // B_d as [E, r, H]
     }
+    if (d->codebook == E4B_CODEBOOK_INT8 || d->codebook == E4B_CODEBOOK_FP8)   // one stack dequantized to bf16
+        L.wbf16 = take((size_t)d->E * std::max(2 * (int64_t)d->I * d->H, (int64_t)d->H * d->I) * 2);
     L.total = off;
     return L;
 }
@@ -145,11 +147,10 @@ static WsLayout layout_for(const e4b_moe_desc* d, int64_t T) {
 static e4b_status check_desc(const e4b_moe_desc* d) {
     if (!d) return E4B_ERR_INVALID_ARG;
     if (d->blocksize != (d->codebook == E4B_CODEBOOK_MXFP4 ? 32 : 64)) return E4B_ERR_BLOCKSIZE;
+    if (d->codebook < E4B_CODEBOOK_NF4 || d->codebook > E4B_CODEBOOK_BF16) return E4B_ERR_INVALID_ARG;
     if (d->E < 1 || d->E > 256 || d->H <= 0 || d->I <= 0) return E4B_ERR_INVALID_ARG;
     if (d->H % 64 || d->I % 64) return E4B_ERR_BLOCKSIZE;
     if (d->top_k < 1 || d->top_k > 8 || d->top_k > d->E) return E4B_ERR_INVALID_ARG;
-    if (d->codebook != E4B_CODEBOOK_NF4 && d->codebook != E4B_CODEBOOK_FP4 && d->codebook != E4B_CODEBOOK_MXFP4)
-        return E4B_ERR_INVALID_ARG;
     if (d->path < E4B_PATH_AUTO || d->path > E4B_PATH_DECODE) return E4B_ERR_INVALID_ARG;
     if (d->activation != E4B_ACT_SWIGLU && d->activation != E4B_ACT_CLAMPED_GLU) return E4B_ERR_INVALID_ARG;
     if (d->activation == E4B_ACT_CLAMPED_GLU && (!std::isfinite(d->glu_alpha) || !(d->glu_limit > 0.0f)))
@@ -162,7 +163,8 @@ static e4b_status check_desc(const e4b_moe_desc* d) {
 static e4b_status check_experts(const e4b_moe_desc* d, const e4b_experts* w) {
     if (!w || !w->gate_up || !w->down) return E4B_ERR_INVALID_ARG;
     if (d->codebook == E4B_CODEBOOK_MXFP4 ? (!w->gate_up_scales || !w->down_scales)
-                                          : (!w->gate_up_absmax || !w->down_absmax))
+        : d->codebook == E4B_CODEBOOK_BF16 ? false
+                                           : (!w->gate_up_absmax || !w->down_absmax))
         return E4B_ERR_INVALID_ARG;
     if (d->lora_rank > 0 && (!w->lora_A_gu || !w->lora_B_gu || !w->lora_A_d || !w->lora_B_d))
         return E4B_ERR_INVALID_ARG;
@@ -185,6 +187,27 @@ static GemmParams base_params(const e4b_moe_desc* d, uint8_t* ws, const WsLayout
     p.status = device_status_ptr();
     (void)P;
     return p;
+}
+
+// The grouped GEMMs' weight format: the 4-bit codebooks and MXFP4 are decoded in the
+// dequantizing warps; the 8-bit codebooks are first dequantized to bf16 (one stack
+// at a time, into ws.wbf16), and those and bf16 passthrough stacks are copied as is.
+static int gemm_codebook(const e4b_moe_desc* d) { return d->codebook <= E4B_CODEBOOK_MXFP4 ? d->codebook : 3; }
+
+// bf16 weights of one stack (gate_up when up, else down) for the GEMM, or null for
+// the decoded formats.
+static e4b_status stack_bf16(const e4b_moe_desc* d, const e4b_experts* w, bool up, uint8_t* ws, const WsLayout& L,
+                             cudaStream_t st, const __nv_bfloat16** out) {
+    *out = nullptr;
+    if (d->codebook == E4B_CODEBOOK_BF16) {
+        *out = static_cast<const __nv_bfloat16*>(static_cast<const void*>(up ? w->gate_up : w->down));
+    } else if (d->codebook == E4B_CODEBOOK_INT8 || d->codebook == E4B_CODEBOOK_FP8) {
+        const int64_t n = (int64_t)d->E * (up ? 2 * (int64_t)d->I * d->H : (int64_t)d->H * d->I);
+        E4B_CUDA_TRY(launch_dequantize8(up ? w->gate_up : w->down, up ? w->gate_up_absmax : w->down_absmax, n,
+                                        d->codebook, 1, ws + L.wbf16, st));
+        *out = reinterpret_cast<const __nv_bfloat16*>(ws + L.wbf16);
+    }
+    return E4B_OK;
 }
 
 // MXFP4 stacks: the scale bytes of the stored matrix (cols = its row length).
@@ -237,7 +260,8 @@ static e4b_status run_gateup(const e4b_moe_desc* d, const e4b_experts* w, uint8_
     p.bias = w->gate_up_bias;
     p.lora_r = d->lora_rank;
     p.lora_b = bf(w->lora_B_gu);
-    E4B_CUDA_TRY(launch_grouped_gemm(EPI_GATEUP, d->codebook, a, P, w->gate_up, p.b_rows_total, d->H / 2, p,
+    if ((s = stack_bf16(d, w, true, ws, L, st, &p.bf16_b)) != E4B_OK) return s;
+    E4B_CUDA_TRY(launch_grouped_gemm(EPI_GATEUP, gemm_codebook(d), a, P, w->gate_up, p.b_rows_total, d->H / 2, p,
                                      max_m_tiles(P, d->E), st, d->lora_rank > 0 ? ws + L.lz_gu : nullptr));
     return E4B_OK;
 }
@@ -264,7 +288,8 @@ static e4b_status run_down(const e4b_moe_desc* d, const e4b_experts* w, uint8_t*
     p.ld_out = d->H;
     p.lora_r = d->lora_rank;
     p.lora_b = bf(w->lora_B_d);
-    E4B_CUDA_TRY(launch_grouped_gemm(EPI_DOWN, d->codebook, h, P, w->down, p.b_rows_total, d->I / 2, p,
+    if ((s = stack_bf16(d, w, false, ws, L, st, &p.bf16_b)) != E4B_OK) return s;
+    E4B_CUDA_TRY(launch_grouped_gemm(EPI_DOWN, gemm_codebook(d), h, P, w->down, p.b_rows_total, d->I / 2, p,
                                      max_m_tiles(P, d->E), st, d->lora_rank > 0 ? ws + L.lz_d : nullptr));
     return E4B_OK;
 }
@@ -342,11 +367,13 @@ e4b_status e4b_quantize_nf4(const float* w, int64_t E, int64_t out, int64_t in, 
     if (blocksize != 64) return E4B_ERR_BLOCKSIZE;
     if (E < 0 || out < 0 || in < 0) return E4B_ERR_INVALID_ARG;
     if (in % 64) return E4B_ERR_BLOCKSIZE;
-    if (cb != E4B_CODEBOOK_NF4 && cb != E4B_CODEBOOK_FP4) return E4B_ERR_INVALID_ARG;
+    const bool eight = cb == E4B_CODEBOOK_INT8 || cb == E4B_CODEBOOK_FP8;
+    if (cb != E4B_CODEBOOK_NF4 && cb != E4B_CODEBOOK_FP4 && !eight) return E4B_ERR_INVALID_ARG;
     const int64_t n = E * out * in;
     if (n == 0) return E4B_OK;
     if (!w || !packed || !absmax) return E4B_ERR_INVALID_ARG;
-    E4B_CUDA_TRY(launch_quantize(w, n / 64, cb, packed, absmax, static_cast<cudaStream_t>(stream)));
+    if (eight) E4B_CUDA_TRY(launch_quantize8(w, n / 64, cb, packed, absmax, static_cast<cudaStream_t>(stream)));
+    else E4B_CUDA_TRY(launch_quantize(w, n / 64, cb, packed, absmax, static_cast<cudaStream_t>(stream)));
     return E4B_OK;
 }
 
@@ -379,13 +406,18 @@ e4b_status e4b_dequantize_nf4(const uint8_t* packed, const float* absmax, int64_
     if (blocksize != 64) return E4B_ERR_BLOCKSIZE;
     if (E < 0 || out < 0 || in < 0) return E4B_ERR_INVALID_ARG;
     if (in % 64) return E4B_ERR_BLOCKSIZE;
-    if (cb != E4B_CODEBOOK_NF4 && cb != E4B_CODEBOOK_FP4) return E4B_ERR_INVALID_ARG;
+    const bool eight = cb == E4B_CODEBOOK_INT8 || cb == E4B_CODEBOOK_FP8;
+    if (cb != E4B_CODEBOOK_NF4 && cb != E4B_CODEBOOK_FP4 && !eight) return E4B_ERR_INVALID_ARG;
     if (out_dtype != E4B_F32 && out_dtype != E4B_BF16) return E4B_ERR_INVALID_ARG;
     const int64_t n = E * out * in;
     if (n == 0) return E4B_OK;
     if (!packed || !absmax || !w_out) return E4B_ERR_INVALID_ARG;
-    E4B_CUDA_TRY(launch_dequantize(packed, absmax, n, cb, out_dtype == E4B_BF16, w_out,
-                                   static_cast<cudaStream_t>(stream)));
+    if (eight)
+        E4B_CUDA_TRY(launch_dequantize8(packed, absmax, n, cb, out_dtype == E4B_BF16, w_out,
+                                        static_cast<cudaStream_t>(stream)));
+    else
+        E4B_CUDA_TRY(launch_dequantize(packed, absmax, n, cb, out_dtype == E4B_BF16, w_out,
+                                       static_cast<cudaStream_t>(stream)));
     return E4B_OK;
 }
 
@@ -409,7 +441,7 @@ e4b_status e4b_moe_forward(const e4b_moe_desc* d, const e4b_experts* w, const vo
     const bool want_grouped_outputs = saved_gu || saved_h || offsets_out || perm_out;
     // the decode kernels implement SwiGLU without biases
     const bool plain_experts = d->activation == E4B_ACT_SWIGLU && !w->gate_up_bias && !w->down_bias &&
-                               d->lora_rank == 0 && d->codebook != E4B_CODEBOOK_MXFP4;
+                               d->lora_rank == 0 && d->codebook <= E4B_CODEBOOK_FP4;
     const bool dec_ok = !want_grouped_outputs && plain_experts && decode_supported(d->E, d->H, d->I, T, d->top_k);
     const bool decode = (d->path == E4B_PATH_DECODE) || (d->path == E4B_PATH_AUTO && dec_ok);
     if (d->path == E4B_PATH_DECODE && !dec_ok) return E4B_ERR_UNSUPPORTED;
@@ -530,8 +562,9 @@ e4b_status e4b_moe_backward(const e4b_moe_desc* d, const e4b_experts* w, const v
         p.h_in = h;
         p.dw_part = dw_part;
     }
-    E4B_CUDA_TRY(launch_grouped_gemm(EPI_DGRAD_DOWN, d->codebook, a_perm, P, w->down, p.b_rows_total, d->I / 2, p,
-                                     max_m_tiles(P, d->E), st, lora ? ws + L.lv_d : nullptr));
+    if ((s = stack_bf16(d, w, false, ws, L, st, &p.bf16_b)) != E4B_OK) return s;
+    E4B_CUDA_TRY(launch_grouped_gemm(EPI_DGRAD_DOWN, gemm_codebook(d), a_perm, P, w->down, p.b_rows_total, d->I / 2,
+                                     p, max_m_tiles(P, d->E), st, lora ? ws + L.lv_d : nullptr));
     if (grad_topk_w)
         E4B_CUDA_TRY(launch_router_grad_parts(bf(grad_out), dw_part, dw_tiles(d), w->down_bias, inv_perm, topk_idx,
                                               topk_w, router_logits, T, d->E, d->top_k, d->H, d->renormalize,
@@ -573,8 +606,9 @@ e4b_status e4b_moe_backward(const e4b_moe_desc* d, const e4b_experts* w, const v
     q.ld_out = d->H;
     q.lora_r = d->lora_rank;
     q.lora_b = bf(w->lora_A_gu);
-    E4B_CUDA_TRY(launch_grouped_gemm(EPI_DGRAD_GATEUP, d->codebook, dgu, P, w->gate_up, q.b_rows_total, d->H / 2, q,
-                                     max_m_tiles(P, d->E), st, lora ? ws + L.lv_gu : nullptr));
+    if ((s = stack_bf16(d, w, true, ws, L, st, &q.bf16_b)) != E4B_OK) return s;
+    E4B_CUDA_TRY(launch_grouped_gemm(EPI_DGRAD_GATEUP, gemm_codebook(d), dgu, P, w->gate_up, q.b_rows_total, d->H / 2,
+                                     q, max_m_tiles(P, d->E), st, lora ? ws + L.lv_gu : nullptr));
     E4B_CUDA_TRY(launch_combine(a_perm, inv_perm, d->top_k, T, d->H, static_cast<__nv_bfloat16*>(grad_x), st));
     return E4B_OK;
 }

@@ -46,6 +46,10 @@ struct GemmParams {
     // MXFP4 weights (codebook 2): the E8M0 scale bytes [rows, mx_stride] replace absmax
     const uint8_t* mx_scales;
     int64_t mx_stride;
+    // bf16 weights (GEMM codebook 3: the 8-bit modes after their dequantization, or
+    // bf16 passthrough): [b_rows_total, stored cols] row-major; copied into the operand
+    // ring by the dequantizing warps
+    const __nv_bfloat16* bf16_b;
 };
 
 // launch bookkeeping
@@ -64,6 +68,11 @@ cudaError_t launch_quantize(const float* w, int64_t nblocks, int codebook, uint8
                             cudaStream_t st);
 cudaError_t launch_dequantize(const uint8_t* packed, const float* absmax, int64_t n, int codebook, int out_bf16,
                               void* out, cudaStream_t st);
+// 8-bit blockwise codebooks (3 int8, 4 fp8): one code byte per element, fp32 absmax per 64
+cudaError_t launch_quantize8(const float* w, int64_t nblocks, int codebook, uint8_t* codes, float* absmax,
+                             cudaStream_t st);
+cudaError_t launch_dequantize8(const uint8_t* codes, const float* absmax, int64_t n, int codebook, int out_bf16,
+                               void* out, cudaStream_t st);
 // MXFP4 (32-element blocks, E8M0 scales [rows, S], S = mxfp4_scale_stride(in) bytes per row)
 int64_t mxfp4_scale_stride(int64_t in);
 cudaError_t launch_quantize_mxfp4(const float* w, int64_t rows, int64_t in, uint8_t* packed, uint8_t* scales,
@@ -91,6 +100,7 @@ cudaError_t launch_combine(const __nv_bfloat16* rows, const int32_t* inv_perm, i
 
 // grouped_gemm.cu
 int gemm_tile_rows();
+// codebook: 0 NF4, 1 FP4, 2 MXFP4 (packed + E8M0 scales), 3 bf16 weights in p.bf16_b.
 // lora_a: the thin A operand of the LoRA k-stage, [a_rows, 64] bf16 (rank padded with
 // zeros), when p.lora_r > 0; otherwise null.
 cudaError_t launch_grouped_gemm(int epi, int codebook, const void* a, int64_t a_rows, const uint8_t* packed,

@@ -345,7 +345,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_con
                 ok = __shfl_sync(0xffffffffu, ok, 0);
                 if (!ok) break;
                 const uint32_t rb = smem_u32(&ctl->raw_full[s]);
-                if (ks == nk) {   // the LoRA stage brings no packed weights: the same 1 + 32 arrivals
+                if (CB == 3 || ks == nk) {   // bf16 weights or the LoRA stage: no packed bytes, the same 1 + 32 arrivals
                     if (lane == 0) mbar_arrive(rb);
                     mbar_arrive(rb);
                     continue;
@@ -439,9 +439,10 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_con
             const int rs = it % RSTAGES;
             const uint32_t rr = it / RSTAGES;
             if (!mbar_wait(smem_u32(&ctl->raw_full[rs]), rr & 1, abort_flag, p.status)) break;
-            if (cur_ks == nk) {
-                // LoRA stage: the adapter tile in bf16 straight from global memory, in the
-                // same shared-memory layout as a dequantized tile
+            if (CB == 3 || cur_ks == nk) {
+                // bf16 weights (CB 3) or the LoRA stage: the tile in bf16 straight from global
+                // memory, in the same shared-memory layout as a dequantized tile
+                const bool lora_stage = cur_ks == nk;
                 __syncwarp();
                 if (lane == 0) mbar_arrive(smem_u32(&ctl->raw_empty[rs]));
                 if (!wait(&ctl->empty[s], (r & 1) ^ 1)) break;
@@ -452,19 +453,27 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_con
                     const int b = tg + TPG * i;
                     const __nv_bfloat16* src = nullptr;   // 64 consecutive bf16 of the tile row b, or null
                     int nvalid = 0;                        // of which the first nvalid are in range
-                    if (kMajorB) {   // row b of this CTA's half; the adapter's r values, zeros after
+                    if (kMajorB) {   // row b of this CTA's half
                         const int n = (int)rank * C::N_CTA + b;
                         const int row = kmajor_row<EPI>(p, ti.nt, n);
                         const bool in = (EPI == EPI_GATEUP) ? (ti.nt * 128 + (n & 127) < p.up_offset)
                                                             : (row < p.b_rows_per_expert);
-                        if (in) {
+                        if (in && lora_stage) {   // the adapter's r values, zeros after
                             src = p.lora_b + ((int64_t)ti.e * p.b_rows_per_expert + row) * p.lora_r;
                             nvalid = p.lora_r;
+                        } else if (in) {          // 64 weights of the row at this k-stage
+                            src = p.bf16_b + ((int64_t)ti.e * p.b_rows_per_expert + row) * p.K + cur_ks * BK;
+                            nvalid = 64;
                         }
-                    } else {         // k-row q = b & 63 (the rank index), columns of block b >> 6
+                    } else {         // k-row q = b & 63, columns of block b >> 6
                         const int q = b & 63, col = ti.nt * BN + (int)rank * C::N_CTA + (b >> 6) * 64;
-                        if (q < p.lora_r && col < p.N) {
-                            src = p.lora_b + ((int64_t)ti.e * p.lora_r + q) * p.N + col;
+                        if (lora_stage) {   // q is the rank index
+                            if (q < p.lora_r && col < p.N) {
+                                src = p.lora_b + ((int64_t)ti.e * p.lora_r + q) * p.N + col;
+                                nvalid = min(64, p.N - col);
+                            }
+                        } else if (col < p.N) {   // stored row ks * 64 + q of the expert
+                            src = p.bf16_b + ((int64_t)ti.e * p.b_rows_per_expert + cur_ks * BK + q) * p.N + col;
                             nvalid = min(64, p.N - col);
                         }
                     }
@@ -515,10 +524,10 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_con
                 if (CB == 2) {
                     const uint32_t sc = __float_as_uint(a_cur[i]);
                     const int sel = kMajorB ? 2 * (cur_ks & 1) : 2 * (b >> 6);
-                    tb = make_table<CB>(mx_scale((sc >> (8 * sel)) & 0xFFu));
-                    tb1 = make_table<CB>(mx_scale((sc >> (8 * sel + 8)) & 0xFFu));
+                    tb = make_table<2>(mx_scale((sc >> (8 * sel)) & 0xFFu));
+                    tb1 = make_table<2>(mx_scale((sc >> (8 * sel + 8)) & 0xFFu));
                 } else {
-                    tb = make_table<CB>(a_cur[i]);
+                    tb = make_table<(CB < 3 ? CB : 0)>(a_cur[i]);   // CB 3 never reaches this path
                 }
                 const uint32_t words[8] = {pk[i][0].x, pk[i][0].y, pk[i][0].z, pk[i][0].w,
                                            pk[i][1].x, pk[i][1].y, pk[i][1].z, pk[i][1].w};
@@ -1006,10 +1015,12 @@ cudaError_t launch_grouped_gemm(int epi, int codebook, const void* a, int64_t a_
 if (epi == EPI_DGRAD_DOWN && p.dw_part && !p.h_in) return cudaErrorInvalidValue;
     if (codebook == 2 && (!p.mx_scales || p.mx_stride < (p.b_blocks_per_row * 2 + 15) / 16 * 16))
         return cudaErrorInvalidValue;
+    if (codebook == 3 && !p.bf16_b) return cudaErrorInvalidValue;
     switch (codebook) {
         case 0: return launch_cb<0>(epi, ma, mr, mo, mg, ml, p, grid, st);
         case 1: return launch_cb<1>(epi, ma, mr, mo, mg, ml, p, grid, st);
-        default: return launch_cb<2>(epi, ma, mr, mo, mg, ml, p, grid, st);
+        case 2: return launch_cb<2>(epi, ma, mr, mo, mg, ml, p, grid, st);
+        default: return launch_cb<3>(epi, ma, mr, mo, mg, ml, p, grid, st);
     }
 }
 

@@ -6,6 +6,11 @@
 // exact tie goes to the smaller value), two codes per byte with the first
 // element in the high nibble.  Dequantize follows _dequantize_expert: code value
 // times absmax in fp32, optionally rounded to bf16 (nearest-even).
+#include <cmath>
+#include <limits>
+#include <mutex>
+#include <utility>
+
 #include "e4b_internal.h"
 
 namespace e4b {
@@ -272,6 +277,196 @@ cudaError_t launch_dequantize_mxfp4(const uint8_t* packed, const uint8_t* scales
     timing_begin(KK_DEQUANT, st);
     if (out_bf16) dequantize_kernel<2, true><<<grid, 256, 0, st>>>(packed, nullptr, nchunks, out, scales, nb, S);
     else dequantize_kernel<2, false><<<grid, 256, 0, st>>>(packed, nullptr, nchunks, out, scales, nb, S);
+    timing_end(KK_DEQUANT, st);
+    count_launch();
+    return cudaGetLastError();
+}
+
+}  // namespace e4b
+
+namespace e4b {
+
+// ------------------------------------------------------- 8-bit blockwise modes
+// int8: the dynamic tree map (Dettmers et al. 2022, block-wise 8-bit
+// quantization): bit 7 the sign; in the 7-bit tail, E leading zeros give the
+// decimal exponent 10^-E, then an indicator bit, then F = 6 - E bits of a linear
+// fraction on [0.1, 1] at bin centres; tail 0 is 0, or +1 with the sign set.
+// fp8: the E4M3 values (bias 7, subnormals, S.1111.111 NaN) divided by 448.  Both
+// normalised to max 1 and used with 64-element blocks and fp32 absmax like the
+// 4-bit codebooks ("experts4bit-qlora" 0.4.0, "Storage modes: the support
+// matrix": int8 a blockwise dynamic map, fp8 an e4m3 codebook).
+static float code8_value(int cb, int q) {
+    if (cb == 3) {
+        static const double kPow10[7] = {1.0, 0.1, 0.01, 0.001, 0.0001, 0.00001, 0.000001};
+        const int s = q >> 7, t = q & 127;
+        if (t == 0) return s ? 1.0f : 0.0f;
+        int E = 0;
+        while (!(t & (64 >> E))) ++E;
+        const int F = 6 - E, j = t & ((1 << F) - 1);
+        const double v = kPow10[E] * (0.1 + 0.9 * (j + 0.5) / (double)(1 << F));
+        return (float)(s ? -v : v);
+    }
+    const int s = q >> 7, e = (q >> 3) & 15, m = q & 7;
+    if (e == 15 && m == 7) return std::numeric_limits<float>::quiet_NaN();
+    const double mag = (e == 0) ? (m / 8.0) * std::ldexp(1.0, -6) : (1.0 + m / 8.0) * std::ldexp(1.0, e - 7);
+    const float v = (float)(mag / 448.0);
+    return s ? -v : v;
+}
+
+// Per codebook: the value of every code, the sorted distinct values' midpoints
+// (+inf padded) and the code of each sorted value.
+struct Table8 {
+    float value[256];
+    float mid[256];
+    uint8_t code[256];
+    int n;
+};
+static __constant__ Table8 c_t8[2];   // [0] int8, [1] fp8
+
+static Table8 make_table8(int cb) {
+    Table8 t{};
+    float v[256];
+    int c[256], n = 0;
+    for (int q = 0; q < 256; ++q) {
+        t.value[q] = code8_value(cb, q);
+        if (t.value[q] != t.value[q] || (cb == 4 && q == 0x80)) continue;   // NaN and -0 never produced
+        v[n] = t.value[q];
+        c[n] = q;
+        ++n;
+    }
+    for (int i = 1; i < n; ++i)
+        for (int k = i; k > 0 && v[k - 1] > v[k]; --k) {
+            std::swap(v[k], v[k - 1]);
+            std::swap(c[k], c[k - 1]);
+        }
+    for (int i = 0; i < 256; ++i) {
+        t.mid[i] = i + 1 < n ? (v[i] + v[i + 1]) * 0.5f : std::numeric_limits<float>::infinity();
+        t.code[i] = (uint8_t)(i < n ? c[i] : 0);
+    }
+    t.n = n;
+    return t;
+}
+
+static cudaError_t ensure_tables8() {
+    static std::mutex mu;
+    static bool done[64] = {};
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+    std::lock_guard<std::mutex> lock(mu);
+    if (done[dev]) return cudaSuccess;
+    Table8 t[2] = {make_table8(3), make_table8(4)};
+    e = cudaMemcpyToSymbol(c_t8, t, sizeof(t));
+    if (e == cudaSuccess) done[dev] = true;
+    return e;
+}
+
+// One thread per 64-element block: n = w / absmax (IEEE division), code of the
+// sorted value r = the number of midpoints strictly below n (an exact tie goes to
+// the smaller value), found by an 8-step binary search in shared memory.
+template <int T8>
+__global__ void __launch_bounds__(256) quantize8_kernel(const float* __restrict__ w, int64_t nblocks,
+                                                        uint8_t* __restrict__ codes, float* __restrict__ absmax) {
+    __shared__ float mid[256];
+    __shared__ uint8_t cds[256];
+    mid[threadIdx.x] = c_t8[T8].mid[threadIdx.x];
+    cds[threadIdx.x] = c_t8[T8].code[threadIdx.x];
+    __syncthreads();
+    uint8_t zero_code = 0;
+    for (int i = 0; i < 256; ++i)
+        if (c_t8[T8].value[i] == 0.0f && !(T8 == 1 && i == 0x80)) { zero_code = (uint8_t)i; break; }
+    for (int64_t b = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; b < nblocks; b += (int64_t)gridDim.x * blockDim.x) {
+        const float4* src = reinterpret_cast<const float4*>(w + b * 64);
+        float a = 0.0f;
+        for (int k = 0; k < 16; ++k) {
+            const float4 f = __ldg(src + k);
+            a = fmaxf(a, fmaxf(fmaxf(fabsf(f.x), fabsf(f.y)), fmaxf(fabsf(f.z), fabsf(f.w))));
+        }
+        absmax[b] = a;
+        uint32_t* dst = reinterpret_cast<uint32_t*>(codes + b * 64);
+        for (int k = 0; k < 16; ++k) {
+            const float4 f = __ldcs(src + k);
+            const float x[4] = {f.x, f.y, f.z, f.w};
+            uint32_t word = 0;
+#pragma unroll
+            for (int t = 0; t < 4; ++t) {
+                uint32_t code = zero_code;
+                if (a != 0.0f) {
+                    const float n = __fdiv_rn(x[t], a);
+                    int r = 0;   // midpoints below n: the largest r with mid[r - 1] < n
+#pragma unroll
+                    for (int step = 128; step >= 1; step >>= 1)
+                        if (mid[r + step - 1] < n) r += step;
+                    code = cds[r];
+                }
+                word |= code << (8 * t);
+            }
+            dst[k] = word;
+        }
+    }
+}
+
+// value = code value * absmax (fp32), then bf16 nearest-even or fp32; one thread
+// per 16 codes.
+template <int T8, bool BF16>
+__global__ void __launch_bounds__(256) dequantize8_kernel(const uint8_t* __restrict__ codes,
+                                                          const float* __restrict__ absmax, int64_t nchunks,
+                                                          void* __restrict__ out) {
+    __shared__ float val[256];
+    val[threadIdx.x] = c_t8[T8].value[threadIdx.x];
+    __syncthreads();
+    for (int64_t c = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; c < nchunks; c += (int64_t)gridDim.x * blockDim.x) {
+        const uint4 q = __ldcs(reinterpret_cast<const uint4*>(codes) + c);
+        const float a = __ldg(absmax + c / 4);
+        const uint32_t w[4] = {q.x, q.y, q.z, q.w};
+        float f[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) f[i] = __fmul_rn(val[(w[i >> 2] >> (8 * (i & 3))) & 0xFFu], a);
+        if (BF16) {
+            uint32_t o[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) o[i] = pack_bf16x2(f[2 * i], f[2 * i + 1]);
+            uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(out) + c * 16);
+            __stcs(dst, make_uint4(o[0], o[1], o[2], o[3]));
+            __stcs(dst + 1, make_uint4(o[4], o[5], o[6], o[7]));
+        } else {
+            float4* dst = reinterpret_cast<float4*>(static_cast<float*>(out) + c * 16);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) __stcs(dst + i, make_float4(f[4 * i], f[4 * i + 1], f[4 * i + 2], f[4 * i + 3]));
+        }
+    }
+}
+
+cudaError_t launch_quantize8(const float* w, int64_t nblocks, int codebook, uint8_t* codes, float* absmax,
+                             cudaStream_t st) {
+    if (nblocks == 0) return cudaSuccess;
+    cudaError_t e = ensure_tables8();
+    if (e != cudaSuccess) return e;
+    const int grid = grid_for(nblocks, 256);
+    timing_begin(KK_QUANT, st);
+    if (codebook == 3) quantize8_kernel<0><<<grid, 256, 0, st>>>(w, nblocks, codes, absmax);
+    else quantize8_kernel<1><<<grid, 256, 0, st>>>(w, nblocks, codes, absmax);
+    timing_end(KK_QUANT, st);
+    count_launch();
+    return cudaGetLastError();
+}
+
+cudaError_t launch_dequantize8(const uint8_t* codes, const float* absmax, int64_t n, int codebook, int out_bf16,
+                               void* out, cudaStream_t st) {
+    const int64_t nchunks = n / 16;
+    if (nchunks == 0) return cudaSuccess;
+    cudaError_t e = ensure_tables8();
+    if (e != cudaSuccess) return e;
+    const int grid = grid_for(nchunks, 256);
+    timing_begin(KK_DEQUANT, st);
+    if (codebook == 3) {
+        if (out_bf16) dequantize8_kernel<0, true><<<grid, 256, 0, st>>>(codes, absmax, nchunks, out);
+        else dequantize8_kernel<0, false><<<grid, 256, 0, st>>>(codes, absmax, nchunks, out);
+    } else {
+        if (out_bf16) dequantize8_kernel<1, true><<<grid, 256, 0, st>>>(codes, absmax, nchunks, out);
+        else dequantize8_kernel<1, false><<<grid, 256, 0, st>>>(codes, absmax, nchunks, out);
+    }
     timing_end(KK_DEQUANT, st);
     count_launch();
     return cudaGetLastError();

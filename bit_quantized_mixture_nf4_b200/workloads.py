@@ -18,7 +18,7 @@ import math
 
 import torch
 
-NF4, FP4, MXFP4 = 0, 1, 2   # MXFP4: the gpt-oss experts' native storage (32-element E8M0 blocks)
+NF4, FP4, MXFP4, INT8, FP8, BF16_WEIGHTS = 0, 1, 2, 3, 4, 5   # storage formats (e4b_codebook)
 
 
 @dataclasses.dataclass(frozen=True)

@@ -67,7 +67,19 @@ typedef enum {
  * {0, .5, 1, 1.5, 2, 3, 4, 6}), packed like the 4-bit stacks; scales uint8
  * [E, out, S] with S = e4b_mxfp4_scale_stride(in) (in/32 rounded up to a multiple
  * of 16, padding bytes 0).  The descriptor's blocksize is 32 for MXFP4. */
-typedef enum { E4B_CODEBOOK_NF4 = 0, E4B_CODEBOOK_FP4 = 1, E4B_CODEBOOK_MXFP4 = 2 } e4b_codebook;
+/* INT8 / FP8: the 8-bit blockwise modes ([P1] "Storage modes: the support
+ * matrix"): 64-element blocks with an fp32 absmax and ONE code byte per element
+ * (packed stacks [E, out*in]); int8 is the dynamic tree map (bit 7 the sign; in
+ * the 7-bit tail, E leading zeros give 10^-E, then an indicator bit and 6 - E
+ * fraction bits on [0.1, 1] at bin centres; tail 0 is 0, or +1 with the sign set),
+ * fp8 the E4M3 values divided by 448.  The grouped GEMMs take them as bf16,
+ * dequantized one stack at a time into the workspace.
+ * BF16: passthrough, the stacks given as bf16 [E, out, in] in gate_up / down (no
+ * absmax). */
+typedef enum {
+    E4B_CODEBOOK_NF4 = 0, E4B_CODEBOOK_FP4 = 1, E4B_CODEBOOK_MXFP4 = 2,
+    E4B_CODEBOOK_INT8 = 3, E4B_CODEBOOK_FP8 = 4, E4B_CODEBOOK_BF16 = 5
+} e4b_codebook;
 typedef enum { E4B_F32 = 0, E4B_BF16 = 1 } e4b_dtype;
 typedef enum { E4B_PATH_AUTO = 0, E4B_PATH_GROUPED = 1, E4B_PATH_DECODE = 2 } e4b_path;
 /* The experts' gated activation of the pre-activations g (gate rows) and u (up rows):
@@ -142,7 +154,8 @@ typedef struct {
  * max|w| (stored as is, fp32); each element is divided by absmax (IEEE fp32
  * division) and takes the code of the nearest codebook value, an exact tie
  * going to the smaller value; an all-zero block stores absmax 0 and the zero
- * code.  Writes packed [E, out*in/2] and absmax [E, out*in/64].
+ * code.  Writes packed [E, out*in/2] and absmax [E, out*in/64]; for the 8-bit
+ * codebooks (INT8, FP8) packed holds one byte per element, [E, out*in].
  * Errors: E4B_ERR_BLOCKSIZE if blocksize != 64 or in % 64 != 0;
  * E4B_ERR_INVALID_ARG for null pointers, negative sizes or an unknown codebook.
  * Non-finite inputs are outside the contract. */

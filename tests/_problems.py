@@ -48,6 +48,13 @@ def build(w: wl.Workload) -> Problem:
     if w.codebook == wl.MXFP4:   # packed codes + E8M0 scale bytes (in ag / ad)
         pg, ag = oracle.quantize_mxfp4(gu)
         pd, ad = oracle.quantize_mxfp4(dn)
+    elif w.codebook in (wl.INT8, wl.FP8):   # one code byte per element
+        pg, ag = oracle.quantize8(gu, w.codebook)
+        pd, ad = oracle.quantize8(dn, w.codebook)
+    elif w.codebook == wl.BF16_WEIGHTS:   # passthrough: the bf16 bits of the weights, no absmax
+        pg = torch.from_numpy(gu).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint8)
+        pd = torch.from_numpy(dn).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint8)
+        ag = ad = np.zeros((w.E, 1), np.float32)
     else:
         pg, ag = oracle.quantize(gu, w.codebook)
         pd, ad = oracle.quantize(dn, w.codebook)
@@ -68,6 +75,13 @@ def oracle_weights(prob: Problem, experts=None):
         wgu = oracle.dequantize_mxfp4(prob.pg[experts], prob.ag[experts], (len(experts), 2 * w.I, w.H))
         wd = oracle.dequantize_mxfp4(prob.pd[experts], prob.ad[experts], (len(experts), w.H, w.I))
         return wgu, wd
+    if w.codebook in (wl.INT8, wl.FP8):
+        wgu = oracle.dequantize8(prob.pg[experts], prob.ag[experts], (len(experts), 2 * w.I, w.H), w.codebook)
+        wd = oracle.dequantize8(prob.pd[experts], prob.ad[experts], (len(experts), w.H, w.I), w.codebook)
+        return wgu, wd
+    if w.codebook == wl.BF16_WEIGHTS:
+        bits = lambda a, shape: oracle.bf16_bits_to_f32(np.ascontiguousarray(a).view(np.uint16).reshape(shape))
+        return (bits(prob.pg[experts], (len(experts), 2 * w.I, w.H)), bits(prob.pd[experts], (len(experts), w.H, w.I)))
     wgu = oracle.dequantize(prob.pg[experts], prob.ag[experts], (len(experts), 2 * w.I, w.H), w.codebook)
     wd = oracle.dequantize(prob.pd[experts], prob.ad[experts], (len(experts), w.H, w.I), w.codebook)
     return wgu, wd

@@ -120,6 +120,18 @@ def test_host_side_validation(lib):
     assert L.e4b_quantize_mxfp4(nullp, 1, 2, 48, nullp, nullp, nullp) == lib.E4B_ERR_BLOCKSIZE
     assert L.e4b_quantize_mxfp4(nullp, 1, 2, 64, nullp, nullp, nullp) == lib.E4B_ERR_INVALID_ARG
     assert L.e4b_dequantize_mxfp4(nullp, nullp, 1, 2, 64, 7, nullp, nullp) == lib.E4B_ERR_INVALID_ARG
+    # 8-bit and bf16 storage: codebooks 3..5 at blocksize 64; anything past 5 is refused
+    for cb in (lib.INT8, lib.FP8, lib.BF16_WEIGHTS):
+        assert lib.e4b_moe_workspace_size(lib.make_desc(8, 256, 512, 2, codebook=cb), 64) > 0
+    assert lib.e4b_moe_workspace_size(lib.make_desc(8, 256, 512, 2, codebook=6), 64) == 0
+    # the 8-bit modes hold one stack dequantized to bf16 in the workspace
+    assert (lib.e4b_moe_workspace_size(lib.make_desc(8, 256, 512, 2, codebook=lib.INT8), 64)
+            >= lib.e4b_moe_workspace_size(d, 64) + 8 * 2 * 512 * 256 * 2)
+    bfx = lib.e4b_experts(16, 16, None, None)   # bf16 passthrough needs no absmax
+    bfd = lib.make_desc(8, 256, 512, 2, codebook=lib.BF16_WEIGHTS)
+    assert L.e4b_moe_forward(ctypes.byref(bfd), ctypes.byref(bfx), 16, 4, None, 16, 16, 16, None, None, None, None,
+                             16, 10, None) == lib.E4B_ERR_WORKSPACE
+    assert L.e4b_quantize_nf4(nullp, 1, 2, 64, 64, lib.BF16_WEIGHTS, nullp, nullp, nullp) == lib.E4B_ERR_INVALID_ARG
     # LoRA: rank a multiple of 8 up to 64, finite scale, all four adapters present
     for bad in (lib.make_desc(8, 256, 512, 2, lora_rank=12), lib.make_desc(8, 256, 512, 2, lora_rank=72),
                 lib.make_desc(8, 256, 512, 2, lora_rank=-8),
