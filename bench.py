@@ -55,7 +55,8 @@ def parse():
     ap.add_argument("--no-aux", action="store_true", help="skip the secondary legs")
     ap.add_argument("--codebook", default="native", choices=["native", "mxfp4"],
                     help="variant leg: the workload's own 4-bit codebook or native MXFP4 storage")
-    ap.add_argument("--leg", default="step", choices=["step", "decode", "codec", "variant", "router", "lora"],
+    ap.add_argument("--leg", default="step",
+                    choices=["step", "decode", "codec", "variant", "router", "lora", "storage"],
                     help="step: the benchmark line; decode / codec / variant / router: only that secondary leg "
                          "(for profiling); decode runs the Qwen3-shaped layer (or --workload) at --tokens "
                          "(default 1); router runs the routing-gradient legs on --workload")
@@ -71,7 +72,7 @@ def headline_workload(args):
 def workload_desc(w) -> str:
     rt = "zipf-skewed routing, " if w.router == "zipf" else ""
     return (f"{w.name}-shaped E={w.E} H={w.H} I={w.I} top{w.k} {'renorm' if w.renorm else 'no-renorm'} T={w.T}/GPU, "
-            f"{('nf4', 'fp4', 'mxfp4')[w.codebook]} blocksize 64, {rt}fwd (routed from logits, g/u saved) + dgrad")
+            f"{('nf4', 'fp4', 'mxfp4', 'int8', 'fp8', 'bf16')[w.codebook]} blocksize 64, {rt}fwd (routed from logits, g/u saved) + dgrad")
 
 
 def bench_config(w, world):
@@ -234,7 +235,12 @@ class Layer:
         self.go_h = wl.grad_output(w)
         gu, dn = wl.weights(w, device=dev)
         self.mx = w.codebook == wl.MXFP4   # native MXFP4: packed codes + E8M0 scale bytes
-        quant = e4b.e4b_quantize_mxfp4 if self.mx else (lambda t: e4b.e4b_quantize_nf4(t, codebook=w.codebook))
+        if self.mx:
+            quant = e4b.e4b_quantize_mxfp4
+        elif w.codebook == wl.BF16_WEIGHTS:   # passthrough: the bf16 stacks themselves, no absmax
+            quant = lambda t: (t.to(torch.bfloat16).view(torch.uint8).reshape(t.shape[0], -1), None)
+        else:
+            quant = lambda t: e4b.e4b_quantize_nf4(t, codebook=w.codebook)
         self.pg, self.ag = quant(gu)
         self.pd, self.ad = quant(dn)
         del gu, dn
@@ -430,7 +436,7 @@ def decode_leg(w, dev, reps=20):
     if e4b.e4b_device_status() != e4b.E4B_OK:
         raise RuntimeError("device status not ok after the decode leg")
     return {"workload": f"{w.name}-shaped E={w.E} H={w.H} I={w.I} top{w.k} T={w.T} "
-                        f"{('nf4', 'fp4', 'mxfp4')[w.codebook]}", "us_per_forward": st,
+                        f"{('nf4', 'fp4', 'mxfp4', 'int8', 'fp8', 'bf16')[w.codebook]}", "us_per_forward": st,
             "experts_touched": touched, "bytes_per_forward": nbytes, "weight_stream_gbs": gbs,
             "roofline": {"bound": "hbm", "achieved": gbs, "peak": hbm, "unit": "GB/s", "frac": gbs / hbm},
             "layer_copies": copies, "touched_bytes_all_copies": nbytes * copies,
@@ -525,6 +531,27 @@ def router_fused_leg(layer, flush, steps=10):
                     "row and 256-column tile, a per-token kernel sums them and runs the softmax backward"}
 
 
+def storage_leg(w, dev, flush, steps=10):
+    """The fwd+dgrad step of workload w in every storage format: the 4-bit
+    codebooks NF4 / FP4, native MXFP4, the 8-bit blockwise int8 / fp8 (dequantized
+    to bf16 one stack at a time before each GEMM) and bf16 passthrough."""
+    import torch
+    from bit_quantized_mixture_nf4_b200 import workloads as wl
+    _, bf16, _, src = peaks()
+    out = {"workload": workload_desc(w)}
+    for name, cb in (("nf4", wl.NF4), ("fp4", wl.FP4), ("mxfp4", wl.MXFP4), ("int8", wl.INT8), ("fp8", wl.FP8),
+                     ("bf16", wl.BF16_WEIGHTS)):
+        layer = Layer(dataclasses.replace(w, codebook=cb), dev)
+        ms, _, _ = timed_steps(layer, steps, 3, flush, torch.cuda.current_stream(), kinds=())
+        del layer
+        torch.cuda.empty_cache()
+        st = step_stats(ms)
+        tf = 12 * w.H * w.I * w.P / (st["median"] / 1e3) / 1e12
+        out[name] = {"step_ms": st, "tokens_per_s": w.T / (st["median"] / 1e3), "frac": tf / bf16}
+    out["peak_kind"] = f"{src} bf16 dense (burst)"
+    return out
+
+
 def lora_leg(w, dev, flush, rank=16, steps=10):
     """The training step with per-expert LoRA adapters of rank r on both stacks:
     forward (saving g/u and h) + the one-pass backward with the input gradient and
@@ -593,7 +620,7 @@ def codec_leg(w, dev, reps=10):
         gbs = n * bpe / (us * 1e-6) / 1e9
         res[name] = {"elements": n, "us": us, "achieved": gbs, "peak": hbm, "unit": "GB/s", "frac": gbs / hbm,
                      "bytes_per_element": bpe}
-    res["workload"] = f"{w.name}-shaped gate_up stack [{w.E},{2 * w.I},{w.H}] {('nf4', 'fp4', 'mxfp4')[w.codebook]}"
+    res["workload"] = f"{w.name}-shaped gate_up stack [{w.E},{2 * w.I},{w.H}] {('nf4', 'fp4', 'mxfp4', 'int8', 'fp8', 'bf16')[w.codebook]}"
     del gu, out
     torch.cuda.empty_cache()
     return res
@@ -859,6 +886,7 @@ def run_e4b(args, w):
                 legs[f"{v.name}_T{v.T}"] = step_leg(v, dev, flush)
         aux["large_layers"] = legs
         aux["lora"] = lora_leg(wl.OLMOE, dev, flush)
+        aux["storage_formats"] = storage_leg(wl.OLMOE, dev, flush)
         aux["decode"] = [decode_leg(v, dev) for v in (wl.QWEN3.with_tokens(1), wl.QWEN3.with_tokens(2),
                                                       wl.QWEN3.with_tokens(4), wl.QWEN3.with_tokens(8),
                                                       wl.GPTOSS.with_tokens(1))]
@@ -911,6 +939,9 @@ def main():
             tokens = args.tokens if 0 < args.tokens <= 8 else 1
             base = wl.QWEN3 if args.workload == "mixtral" else wl.ALL[args.workload]   # decode: Qwen3 by default
             print(json.dumps(decode_leg(base.with_tokens(tokens), dev, reps=max(args.steps, 3))), flush=True)
+        elif args.leg == "storage":
+            w = headline_workload(args) if args.workload != "mixtral" else wl.OLMOE
+            print(json.dumps(storage_leg(w, dev, flush, steps=max(args.steps, 3))), flush=True)
         elif args.leg == "lora":
             w = headline_workload(args)
             print(json.dumps(lora_leg(w, dev, flush, steps=max(args.steps, 3))), flush=True)
