@@ -72,7 +72,7 @@ def headline_workload(args):
 def workload_desc(w) -> str:
     rt = "zipf-skewed routing, " if w.router == "zipf" else ""
     return (f"{w.name}-shaped E={w.E} H={w.H} I={w.I} top{w.k} {'renorm' if w.renorm else 'no-renorm'} T={w.T}/GPU, "
-            f"{('nf4', 'fp4', 'mxfp4', 'int8', 'fp8', 'bf16')[w.codebook]} blocksize 64, {rt}fwd (routed from logits, g/u saved) + dgrad")
+            f"{('nf4', 'fp4', 'mxfp4', 'int8', 'fp8', 'bf16')[w.codebook]} blocksize {32 if w.codebook == 2 else 64}, {rt}fwd (routed from logits, g/u saved) + dgrad")
 
 
 def bench_config(w, world):
