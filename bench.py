@@ -342,17 +342,28 @@ def timed_steps(layer, steps, warmup, flush, stream, clk=None, kinds=tuple(GEMM_
     return ms, kernels, launches
 
 
-def gemm_roofline(w, kernels, bf16, peak_kind):
-    """The dominant grouped GEMM (largest total time) against the dense-bf16 peak."""
+def gemm_roofline(w, kernels, bf16, peak_kind, bf16_burst=None):
+    """The dominant grouped GEMM (largest total time) against the dense-bf16 peak `bf16`
+    (the burst figure, or the sustained one for kernels timed inside a long step loop;
+    bf16_burst given: the fraction of the burst figure is reported beside it)."""
     dom = max((k for k in GEMM_FLOPS if k in kernels), key=lambda k: kernels[k]["avg_ms"] * kernels[k]["launches"])
     flops = GEMM_FLOPS[dom] * w.H * w.I * w.P
     achieved = flops / (kernels[dom]["avg_ms"] / 1e3) / 1e12
-    per_kernel = {k: {"avg_ms": v["avg_ms"], "tflops": GEMM_FLOPS[k] * w.H * w.I * w.P / (v["avg_ms"] / 1e3) / 1e12,
-                      "frac": GEMM_FLOPS[k] * w.H * w.I * w.P / (v["avg_ms"] / 1e3) / 1e12 / bf16}
-                  for k, v in kernels.items() if k in GEMM_FLOPS}
-    return {"kernel": dom, "bound": "tensor", "achieved": achieved, "peak": bf16, "unit": "TFLOP/s",
+
+    def entry(k, v):
+        tf = GEMM_FLOPS[k] * w.H * w.I * w.P / (v["avg_ms"] / 1e3) / 1e12
+        e = {"avg_ms": v["avg_ms"], "tflops": tf, "frac": tf / bf16}
+        if bf16_burst:
+            e["frac_of_burst"] = tf / bf16_burst
+        return e
+
+    per_kernel = {k: entry(k, v) for k, v in kernels.items() if k in GEMM_FLOPS}
+    roof = {"kernel": dom, "bound": "tensor", "achieved": achieved, "peak": bf16, "unit": "TFLOP/s",
             "frac": achieved / bf16, "peak_kind": peak_kind, "flops_per_launch": flops,
-            "avg_launch_ms": kernels[dom]["avg_ms"]}, per_kernel
+            "avg_launch_ms": kernels[dom]["avg_ms"]}
+    if bf16_burst:
+        roof["frac_of_burst"] = achieved / bf16_burst
+    return roof, per_kernel
 
 
 # ------------------------------------------------------------------ secondary legs
@@ -852,7 +863,13 @@ def run_e4b(args, w):
     total_ms = max_over_ranks(sum(step_ms), dev)
     ms_per_step = total_ms / args.steps
     value = job_throughput(w.T, world, ms_per_step)
-    roof, per_kernel = gemm_roofline(w, kernels, bf16_burst, f"{peak_src} bf16 dense (burst)")
+    # The GEMMs are timed inside the step loop.  A loop that runs for a quarter of a
+    # second or more runs under the board's power cap, so the sustained dense-bf16
+    # figure is the denominator there; a short loop uses the burst figure.
+    long_loop = total_ms >= 250.0 and bf16_sus is not None
+    peak, peak_kind = ((bf16_sus, f"{peak_src} bf16 dense (sustained): timed inside a {total_ms / 1e3:.2f} s step loop")
+                       if long_loop else (bf16_burst, f"{peak_src} bf16 dense (burst)"))
+    roof, per_kernel = gemm_roofline(w, kernels, peak, peak_kind, bf16_burst)
     roof["traffic"] = recorded_traffic(roof["kernel"], f"{w.name}_T{w.T}")
     step_tf = 12 * w.H * w.I * w.P / (ms_per_step / 1e3) / 1e12
 
@@ -910,10 +927,9 @@ def run_e4b(args, w):
             "config": bench_config(w, world),
             "step_ms": step_stats(step_ms),
             "roofline": roof,
-            "step_roofline": {"bound": "tensor", "achieved": step_tf, "peak": bf16_burst, "unit": "TFLOP/s",
-                              "frac": step_tf / bf16_burst, "flops_per_step": 12 * w.H * w.I * w.P,
-                              "peak_kind": f"{peak_src} bf16 dense (burst)",
-                              "vs_sustained_peak": step_tf / bf16_sus if bf16_sus else None},
+            "step_roofline": {"bound": "tensor", "achieved": step_tf, "peak": peak, "unit": "TFLOP/s",
+                              "frac": step_tf / peak, "flops_per_step": 12 * w.H * w.I * w.P,
+                              "peak_kind": peak_kind, "frac_of_burst": step_tf / bf16_burst},
             "kernels": per_kernel,
             "small_kernels": {"timed": "separate 3-step pass, every launch bracketed by events", **small_kernels},
             "clocks": clk.summary(),

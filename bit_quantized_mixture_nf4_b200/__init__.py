@@ -15,10 +15,15 @@ import os
 import torch
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_HERE, "libe4b.so")
+# E4B_DEBUG=1 loads the debug-check build (device-side bounds and schedule checks)
+DEBUG = os.environ.get("E4B_DEBUG", "0") not in ("", "0")
+LIB_PATH = os.path.join(_HERE, "libe4b_debug.so" if DEBUG else "libe4b.so")
 
 E4B_OK, E4B_ERR_INVALID_ARG, E4B_ERR_BLOCKSIZE, E4B_ERR_UNSUPPORTED, E4B_ERR_WORKSPACE, E4B_ERR_CUDA, \
-    E4B_ERR_TIMEOUT = range(7)
+    E4B_ERR_TIMEOUT, E4B_ERR_DEBUG_CHECK = range(8)
+# debug-check sites (bits 8..15 of e4b_last_status_word)
+SITE_GEMM_TILE, SITE_GEMM_PERM, SITE_GATHER_PERM, SITE_COMBINE_INV, SITE_ROUTER_INV, SITE_OFFSETS, SITE_COUNTS, \
+    SITE_TILE_PREFIX, SITE_SCHEDULE, SITE_PERM, SITE_INV_PERM = range(1, 12)
 NF4, FP4, MXFP4, INT8, FP8, BF16_WEIGHTS = 0, 1, 2, 3, 4, 5   # storage formats (e4b_codebook)
 F32, BF16 = 0, 1
 PATH_AUTO, PATH_GROUPED, PATH_DECODE = 0, 1, 2
@@ -29,7 +34,8 @@ EXPORTS = ("e4b_quantize_nf4", "e4b_dequantize_nf4", "e4b_quantize_mxfp4", "e4b_
            "e4b_moe_backward", "e4b_moe_backward_dgrad", "e4b_moe_backward_router", "e4b_device_status", "e4b_status_string",
            "e4b_launch_count", "e4b_timing_enable", "e4b_timing_enable_kinds", "e4b_timing_reset", "e4b_timing_get",
            "e4b_moe_forward_noalloc", "e4b_watchdog_selftest", "e4b_pipe_arena_size", "e4b_pipe_create",
-           "e4b_pipe_submit", "e4b_pipe_join", "e4b_pipe_sync", "e4b_pipe_destroy")
+           "e4b_pipe_submit", "e4b_pipe_join", "e4b_pipe_sync", "e4b_pipe_destroy", "e4b_last_status_word",
+           "e4b_debug_checks", "e4b_debug_validate_schedule")
 # kernel kinds of e4b_timing_get
 KERNEL_KINDS = ("quantize", "dequantize", "route", "group", "gather", "combine", "gemm_gateup", "gemm_down",
                 "gemm_dgrad_down", "gemm_dgrad_gateup", "decode_gateup", "decode_down")
@@ -68,7 +74,8 @@ def _load():
     if _lib is not None:
         return _lib
     if not os.path.exists(LIB_PATH):
-        raise ImportError(f"libe4b.so not built at {LIB_PATH}; run python -m bit_quantized_mixture_nf4_b200.build")
+        raise ImportError(f"{os.path.basename(LIB_PATH)} not built at {LIB_PATH}; run "
+                          f"python -m bit_quantized_mixture_nf4_b200.build --all")
     lib = ctypes.CDLL(LIB_PATH)
     P, i64, i32, sz = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_size_t
     lib.e4b_quantize_nf4.argtypes = [P, i64, i64, i64, i32, i32, P, P, P]
@@ -90,6 +97,12 @@ def _load():
     lib.e4b_moe_backward_router.argtypes = [ctypes.POINTER(e4b_moe_desc), ctypes.POINTER(e4b_experts), P, i64, P, P,
                                             P, P, P, P, P, sz, P]
     lib.e4b_device_status.argtypes = [P]
+    lib.e4b_last_status_word.argtypes = []
+    lib.e4b_last_status_word.restype = ctypes.c_uint32
+    lib.e4b_debug_checks.argtypes = []
+    lib.e4b_debug_checks.restype = ctypes.c_int
+    lib.e4b_debug_validate_schedule.argtypes = [P, i64, i32, i32, P, P, P, P, i64, P, P, P]
+    lib.e4b_debug_validate_schedule.restype = ctypes.c_int
     lib.e4b_watchdog_selftest.argtypes = [P]
     lib.e4b_status_string.argtypes = [i32]
     lib.e4b_status_string.restype = ctypes.c_char_p
@@ -184,6 +197,30 @@ def e4b_timing_get(kind) -> tuple:
 
 def e4b_device_status(stream=None) -> int:
     return int(_load().e4b_device_status(_stream(stream)))
+
+
+def e4b_last_status_word() -> int:
+    """Raw status word of the last e4b_device_status call (bits 8..15: debug-check site)."""
+    return int(_load().e4b_last_status_word())
+
+
+def e4b_debug_checks() -> bool:
+    """True when the loaded library is the debug-check build."""
+    return bool(_load().e4b_debug_checks())
+
+
+def e4b_debug_validate_schedule(topk_idx, E: int, tile_rows: int, counts, offsets, tile_prefix, sched, perm, inv_perm,
+                                stream=None) -> int:
+    """Checks a grouping schedule on the device; returns the status (E4B_OK or
+    E4B_ERR_DEBUG_CHECK, the failing site then in e4b_last_status_word() >> 8)."""
+    for t, n in ((topk_idx, "topk_idx"), (counts, "counts"), (offsets, "offsets"), (tile_prefix, "tile_prefix"),
+                 (sched, "sched"), (perm, "perm"), (inv_perm, "inv_perm")):
+        _cuda(t, n, torch.int32)
+    if sched.dim() != 2 or sched.shape[1] != 4:
+        raise ValueError("sched must be [n, 4] int32")
+    return int(_load().e4b_debug_validate_schedule(_ptr(topk_idx), topk_idx.numel(), E, tile_rows, _ptr(counts),
+                                                   _ptr(offsets), _ptr(tile_prefix), _ptr(sched), sched.shape[0],
+                                                   _ptr(perm), _ptr(inv_perm), _stream(stream)))
 
 
 def e4b_quantize_nf4(w: torch.Tensor, blocksize: int = 64, codebook: int = NF4, packed=None, absmax=None,

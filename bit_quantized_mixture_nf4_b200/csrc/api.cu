@@ -7,6 +7,8 @@
 #include <utility>
 #include <vector>
 
+#include <nvtx3/nvToolsExt.h>
+
 #include "../../include/e4b.h"
 #include "e4b_internal.h"
 #include "lora.h"
@@ -35,14 +37,29 @@ static cudaEvent_t new_event() {
     return e;
 }
 
+// NVTX: every kernel kind's launches sit inside a host range named for the kind
+// ("e4b.gemm_gateup", ...), and every entry point inside one named for itself, so a
+// profiler can select them (ncu --nvtx --nvtx-include).  Without an attached tool
+// the ranges cost a call through a no-op function pointer.
+static const char* const kKindRange[KK_COUNT] = {
+    "e4b.quantize", "e4b.dequantize", "e4b.route", "e4b.group", "e4b.gather", "e4b.combine",
+    "e4b.gemm_gateup", "e4b.gemm_down", "e4b.gemm_dgrad_down", "e4b.gemm_dgrad_gateup",
+    "e4b.decode_gateup", "e4b.decode_down"};
+static_assert(KK_COUNT == 12, "one range name per kernel kind");
+
 void timing_begin(int kind, cudaStream_t st) {
+    nvtxRangePushA(kKindRange[kind]);
     std::lock_guard<std::mutex> lock(g_timing.mu);
     if (!g_timing.on || !((g_timing.mask >> kind) & 1u)) return;
     g_timing.open[kind] = new_event();
     cudaEventRecord(g_timing.open[kind], st);
 }
 
+NvtxScope::NvtxScope(const char* name) { nvtxRangePushA(name); }
+NvtxScope::~NvtxScope() { nvtxRangePop(); }
+
 void timing_end(int kind, cudaStream_t st) {
+    nvtxRangePop();
     std::lock_guard<std::mutex> lock(g_timing.mu);
     if (!g_timing.on || !g_timing.open[kind]) return;
     cudaEvent_t e = new_event();
@@ -118,7 +135,7 @@ static WsLayout layout_for(const e4b_moe_desc* d, int64_t T) {
     L.chunk_base = take((size_t)nch * d->E * 4);
     L.counts = take((size_t)d->E * 4);
     L.offsets = take((size_t)(d->E + 1) * 4);
-    L.tile_prefix = take((size_t)(d->E + 1) * 4);
+    L.tile_prefix = take((size_t)(d->E + 2) * 4);   // [E] all m-tiles, [E+1] the big ones
     L.sched = take(((size_t)(P + gemm_tile_rows() - 1) / gemm_tile_rows() + d->E) * 16);
     L.perm = take((size_t)P * 4);
     L.inv_perm = take((size_t)P * 4);
@@ -219,6 +236,27 @@ static void set_mx(const e4b_moe_desc* d, const uint8_t* scales, int64_t cols, G
 
 static int max_m_tiles(int64_t P, int E) { return (int)((P + gemm_tile_rows() - 1) / gemm_tile_rows()) + E; }
 
+// Pairs grouped by expert into the workspace (counts, offsets, m-tile schedule, perm,
+// inv_perm); debug builds then check the schedule's consistency.
+static cudaError_t group_pairs(const e4b_moe_desc* d, const int32_t* topk_idx, int64_t P, uint8_t* ws,
+                               const WsLayout& L, cudaStream_t st) {
+    cudaError_t e = launch_group(topk_idx, P, d->E, gemm_tile_rows(), reinterpret_cast<int32_t*>(ws + L.chunk_counts),
+                                 reinterpret_cast<int32_t*>(ws + L.chunk_base), reinterpret_cast<int32_t*>(ws + L.counts),
+                                 reinterpret_cast<int32_t*>(ws + L.offsets), reinterpret_cast<int32_t*>(ws + L.tile_prefix),
+                                 reinterpret_cast<int4*>(ws + L.sched), reinterpret_cast<int32_t*>(ws + L.perm),
+                                 reinterpret_cast<int32_t*>(ws + L.inv_perm), st);
+#if E4B_DEBUG_CHECKS
+    if (e == cudaSuccess && P > 0)
+        e = launch_validate_schedule(topk_idx, P, d->E, gemm_tile_rows(), reinterpret_cast<const int32_t*>(ws + L.counts),
+                                     reinterpret_cast<const int32_t*>(ws + L.offsets),
+                                     reinterpret_cast<const int32_t*>(ws + L.tile_prefix),
+                                     reinterpret_cast<const int4*>(ws + L.sched), max_m_tiles(P, d->E),
+                                     reinterpret_cast<const int32_t*>(ws + L.perm),
+                                     reinterpret_cast<const int32_t*>(ws + L.inv_perm), st);
+#endif
+    return e;
+}
+
 static const __nv_bfloat16* bf(const void* p) { return static_cast<const __nv_bfloat16*>(p); }
 
 // The thin LoRA operand out [P, 64] = s * in [P, K] M_e^T (M an A adapter [E, r, K]
@@ -309,6 +347,7 @@ const char* e4b_status_string(e4b_status s) {
         case E4B_ERR_WORKSPACE: return "workspace missing or too small";
         case E4B_ERR_CUDA: return "CUDA error";
         case E4B_ERR_TIMEOUT: return "device wait timed out";
+        case E4B_ERR_DEBUG_CHECK: return "debug-build check failed";
     }
     return "unknown status";
 }
@@ -348,22 +387,45 @@ e4b_status e4b_timing_get(int kind, double* total_ms, uint64_t* launches) {
     return E4B_OK;
 }
 
+static std::atomic<uint32_t> g_last_status_word{0};
+
 e4b_status e4b_device_status(void* stream) {
     if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return E4B_ERR_CUDA;
     uint32_t* ptr = device_status_ptr();
     if (!ptr) return E4B_ERR_CUDA;
     uint32_t v = 0;
     if (cudaMemcpy(&v, ptr, 4, cudaMemcpyDeviceToHost) != cudaSuccess) return E4B_ERR_CUDA;
+    g_last_status_word.store(v);
     if (v) {
         const uint32_t zero = 0;
         if (cudaMemcpy(ptr, &zero, 4, cudaMemcpyHostToDevice) != cudaSuccess) return E4B_ERR_CUDA;
-        return E4B_ERR_TIMEOUT;
+        return (v & kStatusTimeout) ? E4B_ERR_TIMEOUT : E4B_ERR_DEBUG_CHECK;
     }
     return E4B_OK;
 }
 
+uint32_t e4b_last_status_word(void) { return g_last_status_word.load(); }
+
+int e4b_debug_checks(void) { return E4B_DEBUG_CHECKS; }
+
+e4b_status e4b_debug_validate_schedule(const int32_t* topk_idx, int64_t P, int E, int tile_rows, const int32_t* counts,
+                                       const int32_t* offsets, const int32_t* tile_prefix, const int32_t* sched,
+                                       int64_t n_sched, const int32_t* perm, const int32_t* inv_perm, void* stream) {
+    NvtxScope nvtx_scope("e4b_debug_validate_schedule");
+    if (!topk_idx || !counts || !offsets || !tile_prefix || !sched || !perm || !inv_perm || P <= 0 || E <= 0 ||
+        E > 256 || tile_rows <= 0 || n_sched < 0 || P > INT32_MAX)
+        return E4B_ERR_INVALID_ARG;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const e4b_status prior = e4b_device_status(stream);   // an earlier kernel's error comes first
+    if (prior != E4B_OK) return prior;
+    E4B_CUDA_TRY(launch_validate_schedule(topk_idx, P, E, tile_rows, counts, offsets, tile_prefix,
+                                          reinterpret_cast<const int4*>(sched), n_sched, perm, inv_perm, st));
+    return e4b_device_status(stream);
+}
+
 e4b_status e4b_quantize_nf4(const float* w, int64_t E, int64_t out, int64_t in, int blocksize, e4b_codebook cb,
                             uint8_t* packed, float* absmax, void* stream) {
+    NvtxScope nvtx_scope("e4b_quantize_nf4");
     if (blocksize != 64) return E4B_ERR_BLOCKSIZE;
     if (E < 0 || out < 0 || in < 0) return E4B_ERR_INVALID_ARG;
     if (in % 64) return E4B_ERR_BLOCKSIZE;
@@ -381,6 +443,7 @@ int64_t e4b_mxfp4_scale_stride(int64_t in) { return in < 0 ? 0 : mxfp4_scale_str
 
 e4b_status e4b_quantize_mxfp4(const float* w, int64_t E, int64_t out, int64_t in, uint8_t* packed, uint8_t* scales,
                               void* stream) {
+    NvtxScope nvtx_scope("e4b_quantize_mxfp4");
     if (E < 0 || out < 0 || in < 0) return E4B_ERR_INVALID_ARG;
     if (in % 32) return E4B_ERR_BLOCKSIZE;
     if (E * out * in == 0) return E4B_OK;
@@ -391,6 +454,7 @@ e4b_status e4b_quantize_mxfp4(const float* w, int64_t E, int64_t out, int64_t in
 
 e4b_status e4b_dequantize_mxfp4(const uint8_t* packed, const uint8_t* scales, int64_t E, int64_t out, int64_t in,
                                 e4b_dtype out_dtype, void* w_out, void* stream) {
+    NvtxScope nvtx_scope("e4b_dequantize_mxfp4");
     if (E < 0 || out < 0 || in < 0) return E4B_ERR_INVALID_ARG;
     if (in % 32) return E4B_ERR_BLOCKSIZE;
     if (out_dtype != E4B_F32 && out_dtype != E4B_BF16) return E4B_ERR_INVALID_ARG;
@@ -403,6 +467,7 @@ e4b_status e4b_dequantize_mxfp4(const uint8_t* packed, const uint8_t* scales, in
 
 e4b_status e4b_dequantize_nf4(const uint8_t* packed, const float* absmax, int64_t E, int64_t out, int64_t in,
                               int blocksize, e4b_codebook cb, e4b_dtype out_dtype, void* w_out, void* stream) {
+    NvtxScope nvtx_scope("e4b_dequantize_nf4");
     if (blocksize != 64) return E4B_ERR_BLOCKSIZE;
     if (E < 0 || out < 0 || in < 0) return E4B_ERR_INVALID_ARG;
     if (in % 64) return E4B_ERR_BLOCKSIZE;
@@ -430,6 +495,7 @@ e4b_status e4b_moe_forward(const e4b_moe_desc* d, const e4b_experts* w, const vo
                            const float* router_logits, int32_t* topk_idx, float* topk_w, void* y, void* saved_gu,
                            void* saved_h, int32_t* offsets_out, int32_t* perm_out, void* workspace, size_t ws_bytes,
                            void* stream) {
+    NvtxScope nvtx_scope("e4b_moe_forward");
     e4b_status s = check_desc(d);
     if (s != E4B_OK) return s;
     if ((s = check_experts(d, w)) != E4B_OK) return s;
@@ -461,11 +527,7 @@ e4b_status e4b_moe_forward(const e4b_moe_desc* d, const e4b_experts* w, const vo
 
     int32_t* offsets = reinterpret_cast<int32_t*>(ws + L.offsets);
     int32_t* perm = reinterpret_cast<int32_t*>(ws + L.perm);
-    E4B_CUDA_TRY(launch_group(topk_idx, P, d->E, gemm_tile_rows(), reinterpret_cast<int32_t*>(ws + L.chunk_counts),
-                              reinterpret_cast<int32_t*>(ws + L.chunk_base), reinterpret_cast<int32_t*>(ws + L.counts),
-                              offsets, reinterpret_cast<int32_t*>(ws + L.tile_prefix),
-                              reinterpret_cast<int4*>(ws + L.sched), perm, reinterpret_cast<int32_t*>(ws + L.inv_perm),
-                              st));
+    E4B_CUDA_TRY(group_pairs(d, topk_idx, P, ws, L, st));
     E4B_CUDA_TRY(launch_gather_rows(static_cast<const __nv_bfloat16*>(x), perm, offsets + d->E, d->top_k, P, d->H,
                                     reinterpret_cast<__nv_bfloat16*>(ws + L.a_perm), st));
     // h goes straight to the caller's saved_h when asked for (the down GEMM reads it there)
@@ -486,6 +548,7 @@ e4b_status e4b_moe_backward(const e4b_moe_desc* d, const e4b_experts* w, const v
                             const void* grad_out, const void* saved_gu, const void* saved_h, void* grad_x,
                             float* grad_topk_w, float* grad_logits, const e4b_lora_grads* lora_grads,
                             void* workspace, size_t ws_bytes, void* stream) {
+    NvtxScope nvtx_scope("e4b_moe_backward");
     e4b_status s = check_desc(d);
     if (s != E4B_OK) return s;
     if ((s = check_experts(d, w)) != E4B_OK) return s;
@@ -508,11 +571,7 @@ e4b_status e4b_moe_backward(const e4b_moe_desc* d, const e4b_experts* w, const v
     int32_t* perm = reinterpret_cast<int32_t*>(ws + L.perm);
     const int32_t* inv_perm = reinterpret_cast<const int32_t*>(ws + L.inv_perm);
     const int32_t* offsets = reinterpret_cast<const int32_t*>(ws + L.offsets);
-    E4B_CUDA_TRY(launch_group(topk_idx, P, d->E, gemm_tile_rows(), reinterpret_cast<int32_t*>(ws + L.chunk_counts),
-                              reinterpret_cast<int32_t*>(ws + L.chunk_base), reinterpret_cast<int32_t*>(ws + L.counts),
-                              reinterpret_cast<int32_t*>(ws + L.offsets), reinterpret_cast<int32_t*>(ws + L.tile_prefix),
-                              reinterpret_cast<int4*>(ws + L.sched), perm, reinterpret_cast<int32_t*>(ws + L.inv_perm),
-                              st));
+    E4B_CUDA_TRY(group_pairs(d, topk_idx, P, ws, L, st));
     __nv_bfloat16* a_perm = reinterpret_cast<__nv_bfloat16*>(ws + L.a_perm);
     const int32_t* nrows = offsets + d->E;
     const __nv_bfloat16* gu = static_cast<const __nv_bfloat16*>(saved_gu);
@@ -617,6 +676,7 @@ e4b_status e4b_moe_backward_dgrad(const e4b_moe_desc* d, const e4b_experts* w, c
                                   const int32_t* topk_idx, const float* topk_w, const void* grad_out,
                                   const void* saved_gu, void* grad_x, void* workspace, size_t ws_bytes,
                                   void* stream) {
+    NvtxScope nvtx_scope("e4b_moe_backward_dgrad");
     if (T > 0 && !grad_x) return E4B_ERR_INVALID_ARG;
     return e4b_moe_backward(d, w, x, T, nullptr, topk_idx, topk_w, grad_out, saved_gu, nullptr, grad_x, nullptr,
                             nullptr, nullptr, workspace, ws_bytes, stream);
@@ -626,6 +686,7 @@ e4b_status e4b_moe_backward_router(const e4b_moe_desc* d, const e4b_experts* w, 
                                    const float* router_logits, const int32_t* topk_idx, const float* topk_w,
                                    const void* grad_out, float* grad_topk_w, float* grad_logits, void* workspace,
                                    size_t ws_bytes, void* stream) {
+    NvtxScope nvtx_scope("e4b_moe_backward_router");
     e4b_status s = check_desc(d);
     if (s != E4B_OK) return s;
     if ((s = check_experts(d, w)) != E4B_OK) return s;
@@ -641,11 +702,7 @@ e4b_status e4b_moe_backward_router(const e4b_moe_desc* d, const e4b_experts* w, 
     // h recomputed through the grouped gate_up GEMM, then the unweighted expert
     // outputs Y (the down GEMM with unit weights), one grouped row per pair
     int32_t* perm = reinterpret_cast<int32_t*>(ws + L.perm);
-    E4B_CUDA_TRY(launch_group(topk_idx, P, d->E, gemm_tile_rows(), reinterpret_cast<int32_t*>(ws + L.chunk_counts),
-                              reinterpret_cast<int32_t*>(ws + L.chunk_base), reinterpret_cast<int32_t*>(ws + L.counts),
-                              reinterpret_cast<int32_t*>(ws + L.offsets), reinterpret_cast<int32_t*>(ws + L.tile_prefix),
-                              reinterpret_cast<int4*>(ws + L.sched), perm, reinterpret_cast<int32_t*>(ws + L.inv_perm),
-                              st));
+    E4B_CUDA_TRY(group_pairs(d, topk_idx, P, ws, L, st));
     const int32_t* nrows = reinterpret_cast<const int32_t*>(ws + L.offsets) + d->E;
     __nv_bfloat16* a_perm = reinterpret_cast<__nv_bfloat16*>(ws + L.a_perm);
     E4B_CUDA_TRY(launch_gather_rows(static_cast<const __nv_bfloat16*>(x), perm, nrows, d->top_k, P, d->H, a_perm, st));

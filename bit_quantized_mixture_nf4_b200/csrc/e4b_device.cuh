@@ -13,8 +13,43 @@
 
 namespace e4b {
 
-// Device status word bits (read and cleared by e4b_device_status).
-enum : uint32_t { kStatusTimeout = 1u };
+// Device status word (read and cleared by e4b_device_status): bit 0 a bounded wait
+// timed out; bit 1 a debug-build bounds check failed, with the first failing
+// check's site in bits 8..15.
+enum : uint32_t { kStatusTimeout = 1u, kStatusDebugCheck = 2u };
+
+// Debug-build bounds checks (E4B_DEBUG_CHECKS=1): a check that fails records its
+// site and the kernel skips the access it guarded (nothing traps).  The sites:
+enum : uint32_t {
+    kSiteGemmTile = 1,       // grouped GEMM: an m-tile entry outside the experts or the grouped rows
+    kSiteGemmPerm = 2,       // grouped GEMM epilogue: a grouped row's pair id outside [0, rows)
+    kSiteGatherPerm = 3,     // row gather: a pair id outside [0, P)
+    kSiteCombineInv = 4,     // combine: an inverse-permutation entry outside [-1, P)
+    kSiteRouterInv = 5,      // routing gradient: an inverse-permutation entry outside [-1, P)
+    kSiteOffsets = 6,        // schedule: expert offsets not ascending from 0, or past P
+    kSiteCounts = 7,         // schedule: counts[e] != offsets[e+1] - offsets[e]
+    kSiteTilePrefix = 8,     // schedule: m-tile total != sum of ceil(counts / tile rows)
+    kSiteSchedule = 9,       // schedule: an m-tile entry outside its expert's rows
+    kSitePerm = 10,          // schedule: perm[r] outside [0, P), or of another expert
+    kSiteInvPerm = 11,       // schedule: inv_perm not the inverse of perm
+};
+#ifndef E4B_DEBUG_CHECKS
+#define E4B_DEBUG_CHECKS 0
+#endif
+
+// Records a failed check: sets bit 1 and, if no site is recorded yet, this site.
+// A compare-and-swap loop with a bound (it only repeats while other threads change
+// the word).
+__device__ __forceinline__ void debug_fail(uint32_t* status, uint32_t site) {
+    uint32_t cur = *reinterpret_cast<volatile uint32_t*>(status);
+    for (int i = 0; i < 64; ++i) {
+        const uint32_t nv = cur | kStatusDebugCheck | ((cur & 0xFF00u) ? 0u : ((site & 0xFFu) << 8));
+        const uint32_t prev = atomicCAS(status, cur, nv);
+        if (prev == cur) return;
+        cur = prev;
+    }
+    atomicOr(status, kStatusDebugCheck);
+}
 
 // ----------------------------------------------------------------- codebooks
 // NF4: the 16 NormalFloat values (QLoRA appendix, the "standard" table the

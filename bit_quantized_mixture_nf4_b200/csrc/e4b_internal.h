@@ -16,8 +16,9 @@ enum Epi { EPI_GATEUP = 0, EPI_DOWN = 1, EPI_DGRAD_DOWN = 2, EPI_DGRAD_GATEUP = 
 
 struct GemmParams {
     int E, K, N, n_tiles;
-    const int* tile_prefix;   // [E+1] prefix of ceil(M_e / tile_rows); [E] = total m-tiles
-    const int4* sched;        // per m-tile: (expert, first row, rows, 0)
+    const int* tile_prefix;   // the grouping's m-tile counts: [E] = all m-tiles, [E+1] = big ones
+    const int4* sched;        // per m-tile: (expert, first row, rows, 0); the big tiles first, then
+                              // the tails of at most half a tile (the single-SM instance's)
     const int* perm;          // [P] pair id of each grouped row
     const float* topk_w;      // [P] routing weight by pair id
     const float* absmax;      // absmax of the weight stack
@@ -50,6 +51,8 @@ struct GemmParams {
     // bf16 passthrough): [b_rows_total, stored cols] row-major; copied into the operand
     // ring by the dequantizing warps
     const __nv_bfloat16* bf16_b;
+    int64_t a_rows;           // rows of A and of the per-row arrays (set by launch_grouped_gemm;
+                              // the debug-build bounds checks compare against it)
 };
 
 // launch bookkeeping
@@ -58,9 +61,17 @@ void count_launch();
 // with CUDA events on its stream.
 enum KernelKind { KK_QUANT = 0, KK_DEQUANT, KK_ROUTE, KK_GROUP, KK_GATHER, KK_COMBINE, KK_GEMM_GATEUP, KK_GEMM_DOWN,
                   KK_GEMM_DGRAD_DOWN, KK_GEMM_DGRAD_GATEUP, KK_DECODE_GATEUP, KK_DECODE_DOWN, KK_COUNT };
+// Also opens / closes the kind's NVTX range (api.cu).
 void timing_begin(int kind, cudaStream_t st);
 void timing_end(int kind, cudaStream_t st);
 int num_sms();
+// NVTX range over an entry point's host scope (api.cu)
+struct NvtxScope {
+    explicit NvtxScope(const char* name);
+    ~NvtxScope();
+    NvtxScope(const NvtxScope&) = delete;
+    NvtxScope& operator=(const NvtxScope&) = delete;
+};
 uint32_t* device_status_ptr();
 
 // quant.cu
@@ -85,11 +96,19 @@ constexpr int kChunkPairs = 256;   // pairs per grouping block (one per thread o
 cudaError_t launch_route(const float* logits, int64_t T, int E, int k, int renorm, int32_t* idx, float* w,
                          cudaStream_t st);
 // counts/offsets/tile_prefix/perm from topk_idx; chunk scratch: [nchunks * E] ints x2
-// sched: [ceil(P/tile_rows) + E] m-tile entries (expert, first row, rows, 0)
+// sched: [ceil(P/tile_rows) + E] m-tile entries (expert, first row, rows, 0): the big
+// m-tiles (full ones and tails above tile_rows / 2), experts ascending, then the tails
+// of at most tile_rows / 2 rows; tile_prefix [E+2]: [E] = all m-tiles, [E+1] = big ones
 // inv_perm[pair] = grouped row of the pair, -1 for a pair of an out-of-range expert
 cudaError_t launch_group(const int32_t* idx, int64_t P, int E, int tile_rows, int32_t* chunk_counts,
                          int32_t* chunk_base, int32_t* counts, int32_t* offsets, int32_t* tile_prefix,
                          int4* sched, int32_t* perm, int32_t* inv_perm, cudaStream_t st);
+// Consistency checks of a grouping schedule (sched has n_sched entries); a violated
+// property records its site in the device status word.  Debug builds run it after
+// every grouping.
+cudaError_t launch_validate_schedule(const int32_t* idx, int64_t P, int E, int tile_rows, const int32_t* counts,
+                                     const int32_t* offsets, const int32_t* tile_prefix, const int4* sched,
+                                     int64_t n_sched, const int32_t* perm, const int32_t* inv_perm, cudaStream_t st);
 // nrows: device pointer to the number of grouped rows (offsets[E])
 cudaError_t launch_gather_rows(const __nv_bfloat16* src, const int32_t* perm, const int32_t* nrows, int k,
                                int64_t P, int H, __nv_bfloat16* dst, cudaStream_t st);

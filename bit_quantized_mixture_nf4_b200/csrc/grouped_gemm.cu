@@ -61,16 +61,22 @@ struct Cfg {
     static constexpr int B_BYTES = N_CTA * BK * 2;
     static constexpr int RAW_BYTES = N_CTA * BK / 2;
     static constexpr int ASTAGES = (CTAS == 2) ? 6 : 4;    // A (activation) ring: TMA latency under load
-    static constexpr int STAGES = (CTAS == 2) ? 4 : 2;     // dequantized-B ring
+    static constexpr int STAGES = (CTAS == 2) ? 4 : 3;     // dequantized-B ring
     // packed-weight ring, prefetched far ahead (the input gradient's down^T GEMM gives two
-    // stages to the epilogue buffers that bring in the saved SwiGLU derivatives)
-    static constexpr int RSTAGES = (CTAS == 2) ? (EPI == EPI_DGRAD_DOWN ? 6 : 8) : 6;
+    // stages to the epilogue buffers that bring in the saved SwiGLU derivatives).  The
+    // single-SM tiles (twice the B columns per SM) have room for 3: one per dequantizing
+    // group, so each group reuses its own slot.
+    static constexpr int RSTAGES = (CTAS == 2) ? (EPI == EPI_DGRAD_DOWN ? 6 : 8) : 3;
     static constexpr int AM_BYTES = N_CTA * 4;             // the stage's absmax values, one per block
     static constexpr int RAW_STAGE = RAW_BYTES + AM_BYTES;
     // dequantizing warps: 6 warps (none on the MMA thread's scheduler), 3 groups of 2
     // taking every third k-stage; a thread owns N_CTA / 64 blocks of 64 elements
     static constexpr int DEQ_GROUPS = 3, DEQ_GROUP_WARPS = 2;
     static constexpr int BLK_PER_THREAD = N_CTA / (32 * DEQ_GROUP_WARPS);
+    // A group's next stage reuses a ring slot whose previous use is at most one barrier
+    // phase old only if each ring has a slot per group: with fewer, a parity wait could
+    // pass on a phase two behind while another group's stage is still in use.
+    static_assert(STAGES >= DEQ_GROUPS && RSTAGES >= DEQ_GROUPS, "ring slots per dequantizing group");
     // epilogue staging: per epilogue warp three 32 x 32 bf16 buffers (2 KB each); four (two
     // pairs of saved-derivative chunks, loaded and stored in place) for the down^T GEMM
     static constexpr int STAGE_BUF = 2048, STAGE_BUFS = (EPI == EPI_DGRAD_DOWN) ? 4 : 3;
@@ -82,6 +88,15 @@ static_assert(Cfg<2, EPI_GATEUP>::RINGS_BYTES % 1024 == 0 && Cfg<2, EPI_DGRAD_DO
               "staging buffers stay 1024-byte aligned");
 static_assert(Cfg<2, EPI_GATEUP>::SMEM_BYTES <= 232448 && Cfg<2, EPI_DGRAD_DOWN>::SMEM_BYTES <= 232448,
               "shared memory per block");
+static_assert(Cfg<1, EPI_GATEUP>::RINGS_BYTES % 1024 == 0 && Cfg<1, EPI_DGRAD_DOWN>::RINGS_BYTES % 1024 == 0,
+              "staging buffers stay 1024-byte aligned (single-SM tiles)");
+static_assert(Cfg<1, EPI_GATEUP>::SMEM_BYTES <= 232448 && Cfg<1, EPI_DGRAD_DOWN>::SMEM_BYTES <= 232448,
+              "shared memory per block (single-SM tiles)");
+
+// Programmatic dependent launch: the pair launch lets the single-SM launch after it
+// start early; the single-SM launch waits for the pair launch before it completes.
+__device__ __forceinline__ void pdl_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;"); }
+__device__ __forceinline__ void pdl_wait_primary() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 
 // TMA tensor store of a 32 x 32 bf16 box from shared memory, and its bulk-group
 // bookkeeping (issued and awaited by one thread).
@@ -116,10 +131,19 @@ struct TileInfo {
     int e, row0, rows, nt;
 };
 
-// One load: the m-tile schedule written by the grouping scan.
-__device__ __forceinline__ TileInfo decode_tile(const GemmParams& p, int tile) {
+// One load: the m-tile schedule written by the grouping scan (sched: this instance's
+// part of it; max_rows: its tile height).  Debug builds check the entry; a bad one
+// becomes an empty tile of expert 0 (every role of the CTA decodes the same entry, so
+// they all skip it alike).
+__device__ __forceinline__ TileInfo decode_tile(const GemmParams& p, const int4* sched, int tile, int max_rows) {
     const int mt = tile / p.n_tiles;
-    const int4 v = __ldg(p.sched + mt);
+    const int4 v = __ldg(sched + mt);
+#if E4B_DEBUG_CHECKS
+    if (v.x < 0 || v.x >= p.E || v.z < 1 || v.z > max_rows || v.y < 0 || (int64_t)v.y + v.z > p.a_rows) {
+        debug_fail(p.status, kSiteGemmTile);
+        return TileInfo{0, 0, 0, tile - mt * p.n_tiles};
+    }
+#endif
     return TileInfo{v.x, v.y, v.z, tile - mt * p.n_tiles};
 }
 
@@ -154,8 +178,8 @@ __device__ __forceinline__ int64_t absmax_index(const GemmParams& p, const TileI
 // MXFP4: byte offset, in p.mx_scales, of the 4 scale bytes the raw warp copies for
 // block b at k-stage 0 (-1 outside the stack).  K-major: row b's bytes for 32-blocks
 // 0..3 (k-stage ks reads bytes 2ks, 2ks+1 of the group starting at 4 (ks / 2));
-// MN-major: k-row (b & 63)'s bytes for the 4 32-column groups of this CTA's 128
-// columns (n-block b >> 6 takes bytes 2 (b >> 6), +1).
+// MN-major: k-row (b & 63)'s bytes for the 32-column groups 4 j .. 4 j + 3 of this
+// CTA's columns, j = (b >> 6) / 2 (n-block b >> 6 takes bytes 2 ((b >> 6) & 1), +1).
 template <int EPI, int CTAS>
 __device__ __forceinline__ int64_t mx_offset(const GemmParams& p, const TileInfo& ti, int b, int rank) {
     if (absmax_index<EPI, CTAS>(p, ti, 0, b, rank) < 0) return -1;
@@ -164,7 +188,7 @@ __device__ __forceinline__ int64_t mx_offset(const GemmParams& p, const TileInfo
         return row * p.mx_stride;
     }
     const int64_t row = (int64_t)ti.e * p.b_rows_per_expert + (b & 63);
-    return row * p.mx_stride + (ti.nt * BN + rank * Cfg<CTAS>::N_CTA) / 32;
+    return row * p.mx_stride + (ti.nt * BN + rank * Cfg<CTAS>::N_CTA) / 32 + 4 * ((b >> 6) >> 1);
 }
 
 // This row's part of the routing-weight gradient over one 32-column chunk:
@@ -260,7 +284,12 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_con
         else mbar_arrive(smem_u32(bar));
     };
 
-    const int total_tiles = __ldg(p.tile_prefix + p.E) * p.n_tiles;
+    // This instance's m-tiles: the big ones (cta_group::2 pairs) or the small tails
+    // (single SMs), which follow the big ones in the schedule.
+    const int n_big = __ldg(p.tile_prefix + p.E + 1);
+    const int4* sched = p.sched + (CTAS == 2 ? 0 : n_big);
+    const int total_tiles = (CTAS == 2 ? n_big : __ldg(p.tile_prefix + p.E) - n_big) * p.n_tiles;
+    if (CTAS == 2) pdl_launch_dependents();   // the single-SM launch that follows may start as SMs free up
     const int nk = p.K / BK;              // k-stages of the quantized weights
     const int nkt = nk + (p.lora_r > 0);  // plus the LoRA stage (the last one of a tile)
 
@@ -273,21 +302,21 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_con
             const int a_off = 128 * (int)rank;
             int pf_tile = cluster_id, pf_ks = 0;
             TileInfo pf_ti{};
-            if (pf_tile < total_tiles) pf_ti = decode_tile(p, pf_tile);
+            if (pf_tile < total_tiles) pf_ti = decode_tile(p, sched, pf_tile, C::TILE_M);
             auto prefetch_next = [&]() {
                 if (pf_tile >= total_tiles) return;
                 if (pf_ks < nk) tma_prefetch_l2_2d(&tmap_a, pf_ks * BK, pf_ti.row0 + a_off);
                 if (++pf_ks == nkt) {
                     pf_ks = 0;
                     pf_tile += nclusters;
-                    if (pf_tile < total_tiles) pf_ti = decode_tile(p, pf_tile);
+                    if (pf_tile < total_tiles) pf_ti = decode_tile(p, sched, pf_tile, C::TILE_M);
                 }
             };
             for (int i = 0; i < APF; ++i) prefetch_next();
             uint32_t it = 0;
             bool ok = true;
             for (int tile = cluster_id; tile < total_tiles && ok; tile += nclusters) {
-                const TileInfo ti = decode_tile(p, tile);
+                const TileInfo ti = decode_tile(p, sched, tile, C::TILE_M);
                 for (int ks = 0; ks < nkt; ++ks, ++it) {
                     prefetch_next();
                     const int s = it % ASTAGES;
@@ -316,7 +345,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_con
         constexpr int PER_LANE = C::N_CTA / 32;   // absmax values this lane copies per stage
         uint32_t it = 0;
         for (int tile = cluster_id; tile < total_tiles; tile += nclusters) {
-            const TileInfo ti = decode_tile(p, tile);
+            const TileInfo ti = decode_tile(p, sched, tile, C::TILE_M);
             const int ebase = ti.e * p.b_rows_per_expert;
             // per-tile source of each of this lane's absmax values at k-stage 0, and the
             // step per k-stage (K-major: next block of the row; MN-major: 64 rows down)
@@ -446,7 +475,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_con
                 __syncwarp();
                 if (lane == 0) mbar_arrive(smem_u32(&ctl->raw_empty[rs]));
                 if (!wait(&ctl->empty[s], (r & 1) ^ 1)) break;
-                const TileInfo ti = decode_tile(p, cur_tile);
+                const TileInfo ti = decode_tile(p, sched, cur_tile, C::TILE_M);
                 uint8_t* dst_tile = sB + s * C::B_BYTES;
 #pragma unroll
                 for (int i = 0; i < NB; ++i) {
@@ -523,7 +552,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_con
                 BlockTable tb, tb1;
                 if (CB == 2) {
                     const uint32_t sc = __float_as_uint(a_cur[i]);
-                    const int sel = kMajorB ? 2 * (cur_ks & 1) : 2 * (b >> 6);
+                    const int sel = kMajorB ? 2 * (cur_ks & 1) : 2 * ((b >> 6) & 1);
                     tb = make_table<2>(mx_scale((sc >> (8 * sel)) & 0xFFu));
                     tb1 = make_table<2>(mx_scale((sc >> (8 * sel + 8)) & 0xFFu));
                 } else {
@@ -593,7 +622,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_con
         };
         uint32_t lt = 0;
         for (int tile = cluster_id; tile < total_tiles; tile += nclusters, ++lt) {
-            const TileInfo ti = decode_tile(p, tile);
+            const TileInfo ti = decode_tile(p, sched, tile, C::TILE_M);
             const uint32_t ab = lt & 1, ar = lt >> 1;
             const int rtile = 128 * (int)rank + rloc;
             const int wrow0 = 128 * (int)rank + 32 * warp;   // this warp's first row in the tile
@@ -604,7 +633,14 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_con
             const int srow = ti.row0 + wrow0;                 // first row of the warp's TMA boxes
             // everything that does not depend on the accumulator is fetched before waiting for it
             float wgt = 1.0f;
-            if ((EPI == EPI_DOWN || EPI == EPI_DGRAD_DOWN) && valid) wgt = __ldg(p.topk_w + __ldg(p.perm + row));
+            if ((EPI == EPI_DOWN || EPI == EPI_DGRAD_DOWN) && valid) {
+                const int pid = __ldg(p.perm + row);
+#if E4B_DEBUG_CHECKS
+                if (pid < 0 || pid >= p.a_rows) debug_fail(p.status, kSiteGemmPerm);
+                else
+#endif
+                    wgt = __ldg(p.topk_w + pid);
+            }
             float dwdot = 0.0f;   // EPI_DGRAD_DOWN, XACT: <grad_out W_d, h> over the tile's columns
             uint4 gq[4], uq[4];   // EPI_DGRAD_DOWN: saved dh/dg, dh/du of the current 32-column chunk
             auto load_gu = [&](int q, uint4 (&g4)[4], uint4 (&u4)[4]) {
@@ -647,15 +683,12 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_con
                                 u[j] += __shfl_sync(0xffffffffu, bul, j);
                             }
                         }
-                        // h = act(g, u) and the two derivatives the input gradient needs, in
-                        // place: u <- dh/dg, g <- dh/du, so few registers stay live.
-                        //   SwiGLU: h = silu(g) u, dh/dg = u s (1 + g (1 - s)), dh/du = silu(g),
-                        //           s = sigmoid(g)
-                        //   clamped GLU: g' = min(g, L), u' = clamp(u, -L, L), s = sigmoid(a g'),
-                        //           h = (u' + 1) g' s, dh/dg = [g <= L] (u' + 1) s (1 + a g' (1 - s)),
-                        //           dh/du = [-L <= u <= L] g' s
-                        uint32_t hv[16];
-                        if (!XACT || p.act == 0) {
+                        if (!XACT) {
+                            // h = silu(g) u and the two derivatives the input gradient needs, in place:
+                            // u <- dh/dg = u s (1 + g (1 - s)), g <- dh/du = silu(g), s = sigmoid(g).
+                            // (This plain instance needs no spill in the in-place form; the extended
+                            // instance below packs its outputs as it goes, which spills least there.)
+                            uint32_t hv[16];
 #pragma unroll
                             for (int i = 0; i < 16; ++i) {
                                 float hh[2];
@@ -671,55 +704,88 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_con
                                 }
                                 hv[i] = pack_bf16x2(hh[0], hh[1]);
                             }
+                            auto pack32 = [&](const float (&f)[32], uint32_t (&o)[16]) {
+#pragma unroll
+                                for (int i = 0; i < 16; ++i) o[i] = pack_bf16x2(f[2 * i], f[2 * i + 1]);
+                            };
+                            if (bulk) {
+                                stage_store(hv, &tmap_out, f0, srow);
+                                if (p.gu) {
+                                    uint32_t pk[16];
+                                    pack32(u, pk);
+                                    stage_store(pk, &tmap_gu, f0, srow);
+                                    pack32(g, pk);
+                                    stage_store(pk, &tmap_gu, I + f0, srow);
+                                }
+                            } else if (valid) {
+                                uint4* dst = reinterpret_cast<uint4*>(p.out_bf16 + (int64_t)row * p.ld_out + f0);
+#pragma unroll
+                                for (int i = 0; i < 4; ++i) dst[i] = make_uint4(hv[4 * i], hv[4 * i + 1], hv[4 * i + 2], hv[4 * i + 3]);
+                                if (p.gu) {
+                                    uint32_t pk[16];
+                                    pack32(u, pk);
+                                    uint4* dg = reinterpret_cast<uint4*>(p.gu + (int64_t)row * 2 * I + f0);
+#pragma unroll
+                                    for (int i = 0; i < 4; ++i) dg[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
+                                    pack32(g, pk);
+                                    uint4* du = reinterpret_cast<uint4*>(p.gu + (int64_t)row * 2 * I + I + f0);
+#pragma unroll
+                                    for (int i = 0; i < 4; ++i) du[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
+                                }
+                            }
                         } else {
-                            const float al = p.alpha, L = p.limit;
+                            // Extended instance: h = act(g, u) and the two derivatives, each packed to
+                            // bf16 pairs as soon as its column pair is done.
+                            //   SwiGLU: as above
+                            //   clamped GLU: g' = min(g, L), u' = clamp(u, -L, L), s = sigmoid(a g'),
+                            //     h = (u' + 1) g' s, dh/dg = [g <= L] (u' + 1) s (1 + a g' (1 - s)),
+                            //     dh/du = [-L <= u <= L] g' s
+                            uint32_t hv[16], pdg[16], pdu[16];
+                            const bool clamped = p.act != 0;
+                            const float al = clamped ? p.alpha : 1.0f, L = p.limit;
 #pragma unroll
                             for (int i = 0; i < 16; ++i) {
-                                float hh[2];
+                                float hh[2], dg[2], du[2];
 #pragma unroll
                                 for (int h = 0; h < 2; ++h) {
                                     const int j = 2 * i + h;
                                     const float gg = g[j], uu = u[j];
-                                    const float gc = fminf(gg, L), uc = fminf(fmaxf(uu, -L), L);
-                                    const float sg = __fdividef(1.0f, 1.0f + __expf(-al * gc));
-                                    const float gs = gc * sg;
-                                    hh[h] = (uc + 1.0f) * gs;
-                                    u[j] = (gg <= L) ? (uc + 1.0f) * sg * (1.0f + al * gc * (1.0f - sg)) : 0.0f;
-                                    g[j] = (uu >= -L && uu <= L) ? gs : 0.0f;
+                                    if (!clamped) {
+                                        const float sg = __fdividef(1.0f, 1.0f + __expf(-gg));
+                                        const float sl = gg * sg;
+                                        hh[h] = sl * uu;
+                                        dg[h] = uu * sg * (1.0f + gg * (1.0f - sg));
+                                        du[h] = sl;
+                                    } else {
+                                        const float gc = fminf(gg, L), uc = fminf(fmaxf(uu, -L), L);
+                                        const float sg = __fdividef(1.0f, 1.0f + __expf(-al * gc));
+                                        const float gs = gc * sg;
+                                        hh[h] = (uc + 1.0f) * gs;
+                                        dg[h] = (gg <= L) ? (uc + 1.0f) * sg * (1.0f + al * gc * (1.0f - sg)) : 0.0f;
+                                        du[h] = (uu >= -L && uu <= L) ? gs : 0.0f;
+                                    }
                                 }
                                 hv[i] = pack_bf16x2(hh[0], hh[1]);
+                                pdg[i] = pack_bf16x2(dg[0], dg[1]);
+                                pdu[i] = pack_bf16x2(du[0], du[1]);
                             }
-                        }
-                        auto pack32 = [&](const float (&f)[32], uint32_t (&o)[16]) {
+                            if (bulk) {
+                                stage_store(hv, &tmap_out, f0, srow);
+                                if (p.gu) {
+                                    stage_store(pdg, &tmap_gu, f0, srow);
+                                    stage_store(pdu, &tmap_gu, I + f0, srow);
+                                }
+                            } else if (valid) {
+                                auto put = [&](__nv_bfloat16* base, const uint32_t (&v)[16]) {
+                                    uint4* dst = reinterpret_cast<uint4*>(base);
 #pragma unroll
-                            for (int i = 0; i < 16; ++i) o[i] = pack_bf16x2(f[2 * i], f[2 * i + 1]);
-                        };
-                        if (bulk) {
-                            stage_store(hv, &tmap_out, f0, srow);
-                            if (p.gu) {
-                                uint32_t pk[16];
-                                pack32(u, pk);
-                                stage_store(pk, &tmap_gu, f0, srow);
-                                pack32(g, pk);
-                                stage_store(pk, &tmap_gu, I + f0, srow);
-                            }
-                        } else if (valid) {
-                            uint4* dst = reinterpret_cast<uint4*>(p.out_bf16 + (int64_t)row * p.ld_out + f0);
-#pragma unroll
-                            for (int i = 0; i < 4; ++i)
-                                dst[i] = make_uint4(hv[4 * i], hv[4 * i + 1], hv[4 * i + 2], hv[4 * i + 3]);
-                            if (p.gu) {
-                                uint32_t pk[16];
-                                pack32(u, pk);
-                                uint4* dg = reinterpret_cast<uint4*>(p.gu + (int64_t)row * 2 * I + f0);
-#pragma unroll
-                                for (int i = 0; i < 4; ++i)
-                                    dg[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
-                                pack32(g, pk);
-                                uint4* du = reinterpret_cast<uint4*>(p.gu + (int64_t)row * 2 * I + I + f0);
-#pragma unroll
-                                for (int i = 0; i < 4; ++i)
-                                    du[i] = make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
+                                    for (int i = 0; i < 4; ++i) dst[i] = make_uint4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+                                };
+                                put(p.out_bf16 + (int64_t)row * p.ld_out + f0, hv);
+                                if (p.gu) {
+                                    put(p.gu + (int64_t)row * 2 * I + f0, pdg);
+                                    put(p.gu + (int64_t)row * 2 * I + I + f0, pdu);
+                                }
                             }
                         }
                     }
@@ -774,10 +840,11 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_con
             } else {
 #pragma unroll 1
                 for (int q = 0; q < BN / 32; ++q) {
+                    // the partial tile's rows (this path): the chunk's saved derivatives are
+                    // loaded with it, not one chunk ahead, which keeps 32 registers free
+                    if (EPI == EPI_DGRAD_DOWN && q > 0) load_gu(q, gq, uq);
                     float v[32];
                     tmem_load32(tbase + 32 * q, v);
-                    uint4 gn[4], un[4];
-                    if (EPI == EPI_DGRAD_DOWN && q + 1 < BN / 32) load_gu(q + 1, gn, un);   // next chunk in flight
                     const int c0 = ti.nt * BN + 32 * q;
                     if (any && c0 < p.N) {
                         if (EPI == EPI_DOWN || EPI == EPI_DGRAD_GATEUP) {
@@ -834,13 +901,6 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_con
                             }
                         }
                     }
-                    if (EPI == EPI_DGRAD_DOWN && q + 1 < BN / 32) {
-#pragma unroll
-                        for (int i = 0; i < 4; ++i) {
-                            gq[i] = gn[i];
-                            uq[i] = un[i];
-                        }
-                    }
                 }
                 if (EPI == EPI_DGRAD_DOWN && XACT && valid) p.dw_part[(int64_t)row * p.n_tiles + ti.nt] = dwdot;
             }
@@ -863,6 +923,10 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_con
         if (CTAS == 2) tmem_dealloc_pair(tmem_base, TMEM_COLS);
         else tmem_dealloc(tmem_base, TMEM_COLS);
     }
+    // The single-SM launch may run beside the pair launch before it (programmatic
+    // dependent launch; they write disjoint rows): it completes only after that one
+    // has, so whatever follows in the stream sees both.
+    if (CTAS == 1) pdl_wait_primary();
 }
 
 // ------------------------------------------------------------------ host side
@@ -907,16 +971,16 @@ static bool make_map_2d(CUtensorMap* m, CUtensorMapDataType dt, const void* base
               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// CTAs per tile of the grouped GEMMs (2: cta_group::2 pairs on two SMs).
-constexpr int kCtas = 2;
-int gemm_tile_rows() { return Cfg<kCtas>::TILE_M; }
+// Rows of a big tile (a cta_group::2 pair on two SMs); tails of at most half of it
+// run as single-SM tiles.
+int gemm_tile_rows() { return Cfg<2>::TILE_M; }
 
-template <int EPI, int CB, bool XACT = false>
+template <int EPI, int CB, int CTAS, bool XACT = false>
 static cudaError_t launch_one(const CUtensorMap& ma, const CUtensorMap& mr, const CUtensorMap& mo,
-                              const CUtensorMap& mg, const CUtensorMap& ml, const GemmParams& p, int grid,
+                              const CUtensorMap& mg, const CUtensorMap& ml, const GemmParams& p, int grid, bool pdl,
                               cudaStream_t st) {
-    using C = Cfg<kCtas, EPI>;
-    auto kern = grouped_gemm_kernel<EPI, CB, kCtas, XACT>;
+    using C = Cfg<CTAS, EPI>;
+    auto kern = grouped_gemm_kernel<EPI, CB, CTAS, XACT>;
     // The shared-memory limit is a per-device function attribute: set it once per
     // device and instantiation, under a lock.
     {
@@ -938,16 +1002,16 @@ static cudaError_t launch_one(const CUtensorMap& ma, const CUtensorMap& mr, cons
     cfg.blockDim = dim3(GEMM_THREADS);
     cfg.dynamicSmemBytes = C::SMEM_BYTES;
     cfg.stream = st;
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = kCtas;
+    attr[0].val.clusterDim.x = CTAS;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    timing_begin(KK_GEMM_GATEUP + EPI, st);
+    cfg.numAttrs = pdl ? 2 : 1;
     cudaError_t e = cudaLaunchKernelEx(&cfg, kern, ma, mr, mo, mg, ml, p);
-    timing_end(KK_GEMM_GATEUP + EPI, st);
     count_launch();
     if (e != cudaSuccess) return e;
     return cudaGetLastError();
@@ -955,25 +1019,30 @@ static cudaError_t launch_one(const CUtensorMap& ma, const CUtensorMap& mr, cons
 
 // The instance for the epilogue kind and codebook: the extended epilogue (XACT) for the
 // gate_up variant (clamped GLU or biases) and for the routing-gradient dot products.
-template <int CB>
+template <int CB, int CTAS>
 static cudaError_t launch_cb(int epi, const CUtensorMap& ma, const CUtensorMap& mr, const CUtensorMap& mo,
-                             const CUtensorMap& mg, const CUtensorMap& ml, const GemmParams& p, int grid,
+                             const CUtensorMap& mg, const CUtensorMap& ml, const GemmParams& p, int grid, bool pdl,
                              cudaStream_t st) {
     if (epi == EPI_GATEUP && (p.act != 0 || p.bias != nullptr))
-        return launch_one<EPI_GATEUP, CB, true>(ma, mr, mo, mg, ml, p, grid, st);
-    if (epi == EPI_DGRAD_DOWN && p.dw_part) return launch_one<EPI_DGRAD_DOWN, CB, true>(ma, mr, mo, mg, ml, p, grid, st);
+        return launch_one<EPI_GATEUP, CB, CTAS, true>(ma, mr, mo, mg, ml, p, grid, pdl, st);
+    if (epi == EPI_DGRAD_DOWN && p.dw_part)
+        return launch_one<EPI_DGRAD_DOWN, CB, CTAS, true>(ma, mr, mo, mg, ml, p, grid, pdl, st);
     switch (epi) {
-        case EPI_GATEUP: return launch_one<EPI_GATEUP, CB>(ma, mr, mo, mg, ml, p, grid, st);
-        case EPI_DOWN: return launch_one<EPI_DOWN, CB>(ma, mr, mo, mg, ml, p, grid, st);
-        case EPI_DGRAD_DOWN: return launch_one<EPI_DGRAD_DOWN, CB>(ma, mr, mo, mg, ml, p, grid, st);
-        default: return launch_one<EPI_DGRAD_GATEUP, CB>(ma, mr, mo, mg, ml, p, grid, st);
+        case EPI_GATEUP: return launch_one<EPI_GATEUP, CB, CTAS>(ma, mr, mo, mg, ml, p, grid, pdl, st);
+        case EPI_DOWN: return launch_one<EPI_DOWN, CB, CTAS>(ma, mr, mo, mg, ml, p, grid, pdl, st);
+        case EPI_DGRAD_DOWN: return launch_one<EPI_DGRAD_DOWN, CB, CTAS>(ma, mr, mo, mg, ml, p, grid, pdl, st);
+        default: return launch_one<EPI_DGRAD_GATEUP, CB, CTAS>(ma, mr, mo, mg, ml, p, grid, pdl, st);
     }
 }
 
-cudaError_t launch_grouped_gemm(int epi, int codebook, const void* a, int64_t a_rows, const uint8_t* packed,
-                                int64_t packed_rows_total, int packed_row_bytes, GemmParams p, int max_m_tiles,
-                                cudaStream_t st, const void* lora_a) {
-    using C = Cfg<kCtas>;
+// One configuration: CTAS = 2 runs the big m-tiles (cta_group::2 pairs, 256 rows),
+// CTAS = 1 the small tails (one SM, 128 rows, the whole 256-column B tile dequantized
+// there).  max_tiles bounds the tiles the launch can find in its part of the schedule.
+template <int CTAS>
+static cudaError_t launch_cfg(int epi, int codebook, const void* a, int64_t a_rows, const uint8_t* packed,
+                              int64_t packed_rows_total, int packed_row_bytes, const GemmParams& p, int64_t max_tiles,
+                              bool pdl, cudaStream_t st, const void* lora_a) {
+    using C = Cfg<CTAS>;
     CUtensorMap ma, mr;
     if (!make_map_2d(&ma, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a, (uint64_t)p.K, (uint64_t)a_rows, (uint64_t)p.K * 2, 64,
                      128, CU_TENSOR_MAP_SWIZZLE_128B))
@@ -1001,27 +1070,43 @@ cudaError_t launch_grouped_gemm(int epi, int codebook, const void* a, int64_t a_
         !make_map_2d(&mg, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, p.gu, (uint64_t)n_feat * 2, (uint64_t)a_rows,
                      (uint64_t)n_feat * 4, 32, 32, CU_TENSOR_MAP_SWIZZLE_64B))
         return cudaErrorInvalidValue;
-    // the LoRA stage's thin A operand [rows, 64] bf16: one 64-deep box per tile row block
+    // the LoRA stage's thin A operand [rows, 64] bf16: one 64-deep box per 128 tile rows
     CUtensorMap ml = ma;
-    if (p.lora_r > 0) {
-        if (!lora_a || !p.lora_b || p.lora_r % 8 || p.lora_r > 64 ||
-            !make_map_2d(&ml, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, lora_a, 64, (uint64_t)a_rows, 128, 64, 128,
-                         CU_TENSOR_MAP_SWIZZLE_128B))
-            return cudaErrorInvalidValue;
-    }
-    const int64_t tiles = (int64_t)max_m_tiles * p.n_tiles;
-    const int grid = (int)std::min<int64_t>(tiles * kCtas, (num_sms() / kCtas) * kCtas);
+    if (p.lora_r > 0 &&
+        !make_map_2d(&ml, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, lora_a, 64, (uint64_t)a_rows, 128, 64, 128,
+                     CU_TENSOR_MAP_SWIZZLE_128B))
+        return cudaErrorInvalidValue;
+    const int grid = (int)std::min<int64_t>(max_tiles * CTAS, (num_sms() / CTAS) * CTAS);
     if (grid <= 0) return cudaSuccess;
-if (epi == EPI_DGRAD_DOWN && p.dw_part && !p.h_in) return cudaErrorInvalidValue;
+    switch (codebook) {
+        case 0: return launch_cb<0, CTAS>(epi, ma, mr, mo, mg, ml, p, grid, pdl, st);
+        case 1: return launch_cb<1, CTAS>(epi, ma, mr, mo, mg, ml, p, grid, pdl, st);
+        case 2: return launch_cb<2, CTAS>(epi, ma, mr, mo, mg, ml, p, grid, pdl, st);
+        default: return launch_cb<3, CTAS>(epi, ma, mr, mo, mg, ml, p, grid, pdl, st);
+    }
+}
+
+cudaError_t launch_grouped_gemm(int epi, int codebook, const void* a, int64_t a_rows, const uint8_t* packed,
+                                int64_t packed_rows_total, int packed_row_bytes, GemmParams p, int max_m_tiles,
+                                cudaStream_t st, const void* lora_a) {
+    p.a_rows = a_rows;
+    if (p.lora_r > 0 && (!lora_a || !p.lora_b || p.lora_r % 8 || p.lora_r > 64)) return cudaErrorInvalidValue;
+    if (epi == EPI_DGRAD_DOWN && p.dw_part && !p.h_in) return cudaErrorInvalidValue;
     if (codebook == 2 && (!p.mx_scales || p.mx_stride < (p.b_blocks_per_row * 2 + 15) / 16 * 16))
         return cudaErrorInvalidValue;
     if (codebook == 3 && !p.bf16_b) return cudaErrorInvalidValue;
-    switch (codebook) {
-        case 0: return launch_cb<0>(epi, ma, mr, mo, mg, ml, p, grid, st);
-        case 1: return launch_cb<1>(epi, ma, mr, mo, mg, ml, p, grid, st);
-        case 2: return launch_cb<2>(epi, ma, mr, mo, mg, ml, p, grid, st);
-        default: return launch_cb<3>(epi, ma, mr, mo, mg, ml, p, grid, st);
-    }
+    if (max_m_tiles <= 0) return cudaSuccess;
+    // The big m-tiles on cta_group::2 pairs, then the small tails (at most one per
+    // expert) on single SMs, launched to start as the pairs' SMs free up.  One timing
+    // bracket covers both launches.
+    timing_begin(KK_GEMM_GATEUP + epi, st);
+    cudaError_t e = launch_cfg<2>(epi, codebook, a, a_rows, packed, packed_rows_total, packed_row_bytes, p,
+                                  (int64_t)max_m_tiles * p.n_tiles, false, st, lora_a);
+    if (e == cudaSuccess)
+        e = launch_cfg<1>(epi, codebook, a, a_rows, packed, packed_rows_total, packed_row_bytes, p,
+                          (int64_t)std::min(p.E, max_m_tiles) * p.n_tiles, true, st, lora_a);
+    timing_end(KK_GEMM_GATEUP + epi, st);
+    return e;
 }
 
 }  // namespace e4b

@@ -55,6 +55,7 @@ void* noalloc_scratch(e4b_status* st) {
 extern "C" e4b_status e4b_moe_forward_noalloc(const e4b_moe_desc* d, const e4b_experts* w, const void* x, int64_t T,
                                               const float* router_logits, int32_t* topk_idx, float* topk_w, void* y,
                                               void* stream) {
+    e4b::NvtxScope nvtx_scope("e4b_moe_forward_noalloc");
     // Size check first, on the host: nothing is touched for a request that does not fit.
     const size_t need = e4b_moe_workspace_size(d, T);
     if (T > 0 && need > kNoAllocScratchBytes) return E4B_ERR_WORKSPACE;

@@ -21,6 +21,8 @@
 
 #include <new>
 
+#include <nvtx3/nvToolsExt.h>
+
 #include "../../include/e4b.h"
 
 struct e4b_pipe {
@@ -45,6 +47,13 @@ struct e4b_pipe {
 };
 
 namespace {
+
+// NVTX range over a submission's host scope (the library's other entry points open
+// their own inside it)
+struct PipeRange {
+    explicit PipeRange(const char* name) { nvtxRangePushA(name); }
+    ~PipeRange() { nvtxRangePop(); }
+};
 
 size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
 
@@ -139,6 +148,7 @@ e4b_status e4b_pipe_create(const e4b_moe_desc* d, const e4b_experts* w, int64_t 
 
 e4b_status e4b_pipe_submit(e4b_pipe* p, int64_t T, const void* x_host, const float* logits_host,
                            const void* grad_out_host, void* y_host, void* grad_x_host) {
+    PipeRange nvtx_scope("e4b_pipe_submit");
     if (!p || T < 0 || T > p->T_max) return E4B_ERR_INVALID_ARG;
     if (T == 0) return E4B_OK;
     if (!x_host || !logits_host || !grad_out_host || !y_host || !grad_x_host) return E4B_ERR_INVALID_ARG;

@@ -80,7 +80,13 @@ __global__ void __launch_bounds__(1024) scan_kernel(const int32_t* __restrict__ 
                                                     int tile_rows, int32_t* __restrict__ chunk_base,
                                                     int32_t* __restrict__ counts, int32_t* __restrict__ offsets,
                                                     int32_t* __restrict__ tile_prefix, int4* __restrict__ sched) {
-    __shared__ int s_tot[256], s_off[256], s_toff[256];
+    // An expert's rows make full m-tiles of tile_rows, then a tail.  A tail of more
+    // than half a tile is one more big tile; a tail of at most half a tile is a small
+    // tile, run by the single-SM instance of the grouped GEMMs.  The schedule lists
+    // all big tiles first (experts ascending), then the small ones:
+    // tile_prefix[E] = all m-tiles, tile_prefix[E + 1] = big m-tiles.
+    __shared__ int s_tot[256], s_off[256], s_toff[256], s_soff[257];
+    const int half = tile_rows / 2;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
     chain_release();
     chain_wait();
@@ -92,23 +98,30 @@ __global__ void __launch_bounds__(1024) scan_kernel(const int32_t* __restrict__ 
         if (lane == 0) s_tot[e] = sum;
     }
     __syncthreads();
-    if (warp == 0) {   // exclusive scans of the row counts and m-tile counts over experts
-        int run = 0, trun = 0;
+    if (warp == 0) {   // exclusive scans of the row counts, big m-tiles and small tails over experts
+        int run = 0, trun = 0, srun = 0;
         for (int e0 = 0; e0 < E; e0 += 32) {
             const int e = e0 + lane;
             const int v = e < E ? s_tot[e] : 0;
-            const int tv = (v + tile_rows - 1) / tile_rows;
+            const int rem = v % tile_rows;
+            const int tv = v / tile_rows + (rem > half ? 1 : 0);
+            const int sv = (rem > 0 && rem <= half) ? 1 : 0;
             const int x = warp_inclusive_scan(v, lane), tx = warp_inclusive_scan(tv, lane);
+            const int sx = warp_inclusive_scan(sv, lane);
             if (e < E) {
                 s_off[e] = run + x - v;
                 s_toff[e] = trun + tx - tv;
+                s_soff[e] = srun + sx - sv;
             }
             run += __shfl_sync(0xffffffffu, x, 31);
             trun += __shfl_sync(0xffffffffu, tx, 31);
+            srun += __shfl_sync(0xffffffffu, sx, 31);
         }
         if (lane == 0) {
             offsets[E] = run;
-            tile_prefix[E] = trun;
+            tile_prefix[E] = trun + srun;
+            tile_prefix[E + 1] = trun;
+            s_soff[E] = trun;   // first small entry
         }
     }
     __syncthreads();
@@ -129,10 +142,13 @@ __global__ void __launch_bounds__(1024) scan_kernel(const int32_t* __restrict__ 
             offsets[e] = off;
             tile_prefix[e] = toff;
         }
-        // m-tile schedule: (expert, first row, rows) of every m-tile, experts ascending
-        const int nt = (tot + tile_rows - 1) / tile_rows;
+        // m-tile schedule: (expert, first row, rows) of every m-tile
+        const int rem = tot % tile_rows, full = tot / tile_rows;
+        const int nt = full + (rem > half ? 1 : 0);
         for (int m = lane; m < nt; m += 32)
             sched[toff + m] = make_int4(e, off + m * tile_rows, min(tile_rows, tot - m * tile_rows), 0);
+        if (lane == 0 && rem > 0 && rem <= half)
+            sched[s_soff[E] + s_soff[e]] = make_int4(e, off + full * tile_rows, rem, 0);
     }
 }
 
@@ -191,15 +207,23 @@ __global__ void __launch_bounds__(256) scatter_kernel(const int32_t* __restrict_
 __global__ void __launch_bounds__(256) gather_rows_kernel(const __nv_bfloat16* __restrict__ src,
                                                           const int32_t* __restrict__ perm,
                                                           const int32_t* __restrict__ nrows, int k, int64_t P,
-                                                          int H, __nv_bfloat16* __restrict__ dst) {
+                                                          int H, __nv_bfloat16* __restrict__ dst,
+                                                          uint32_t* __restrict__ status) {
     const int lane = threadIdx.x & 31;
     chain_release();
     chain_wait();
-    P = min(P, (int64_t)__ldcg(nrows));   // rows that belong to a valid expert
+    const int64_t n = min(P, (int64_t)__ldcg(nrows));   // rows that belong to a valid expert
     const int64_t wstride = (int64_t)gridDim.x * blockDim.x / 32;
     const int vec = H / 8;
-    for (int64_t r = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) / 32; r < P; r += wstride) {
-        const int64_t t = __ldcg(perm + r) / k;
+    for (int64_t r = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) / 32; r < n; r += wstride) {
+        const int64_t pid = __ldcg(perm + r);
+#if E4B_DEBUG_CHECKS
+        if (pid < 0 || pid >= P) {
+            if (lane == 0) debug_fail(status, kSiteGatherPerm);
+            continue;
+        }
+#endif
+        const int64_t t = pid / k;
         const uint4* s = reinterpret_cast<const uint4*>(src + t * H);
         uint4* d = reinterpret_cast<uint4*>(dst + r * H);
 #pragma unroll 1
@@ -222,7 +246,8 @@ __global__ void __launch_bounds__(256) gather_rows_kernel(const __nv_bfloat16* _
 // are skipped.
 __global__ void __launch_bounds__(256) combine_kernel(const __nv_bfloat16* __restrict__ rows,
                                                       const int32_t* __restrict__ inv_perm, int k, int64_t T,
-                                                      int H, __nv_bfloat16* __restrict__ y) {
+                                                      int H, __nv_bfloat16* __restrict__ y,
+                                                      uint32_t* __restrict__ status) {
     const int h8 = H / 8;
     const int64_t n = T * h8;
     const int64_t stride = (int64_t)gridDim.x * blockDim.x;
@@ -236,6 +261,12 @@ __global__ void __launch_bounds__(256) combine_kernel(const __nv_bfloat16* __res
             v[j] = make_uint4(0u, 0u, 0u, 0u);
             if (j < k) {
                 const int r = __ldg(inv_perm + t * k + j);
+#if E4B_DEBUG_CHECKS
+                if (r < -1 || r >= T * k) {
+                    debug_fail(status, kSiteCombineInv);
+                    continue;
+                }
+#endif
                 if (r >= 0) v[j] = __ldcs(reinterpret_cast<const uint4*>(rows + (int64_t)r * H) + c);
             }
         }
@@ -251,6 +282,74 @@ __global__ void __launch_bounds__(256) combine_kernel(const __nv_bfloat16* __res
         }
         reinterpret_cast<uint4*>(y)[i] = make_uint4(pack_bf16x2(acc[0], acc[1]), pack_bf16x2(acc[2], acc[3]),
                                                     pack_bf16x2(acc[4], acc[5]), pack_bf16x2(acc[6], acc[7]));
+    }
+}
+
+// Consistency checks of a grouping schedule (the output of the three grouping
+// kernels): expert offsets and counts, the m-tile total and entries, and perm /
+// inv_perm as inverse maps that respect the experts.  A violated property records
+// its site in the status word (debug_fail).  Every value read from the schedule is
+// range-checked before it is used as an index, so a corrupt schedule is reported,
+// never followed.
+__global__ void __launch_bounds__(256) validate_schedule_kernel(const int32_t* __restrict__ idx, int64_t P, int E,
+                                                                int tile_rows, const int32_t* __restrict__ counts,
+                                                                const int32_t* __restrict__ offsets,
+                                                                const int32_t* __restrict__ tile_prefix,
+                                                                const int4* __restrict__ sched, int64_t n_sched,
+                                                                const int32_t* __restrict__ perm,
+                                                                const int32_t* __restrict__ inv_perm,
+                                                                uint32_t* __restrict__ status) {
+    __shared__ unsigned long long s_tiles;
+    if (blockIdx.x == 0) {   // per-expert properties
+        if (threadIdx.x == 0) {
+            s_tiles = 0ull;
+            if (offsets[0] != 0) debug_fail(status, kSiteOffsets);
+        }
+        __syncthreads();
+        for (int e = threadIdx.x; e < E; e += blockDim.x) {
+            const int64_t a = offsets[e], b = offsets[e + 1];
+            if (b < a || b > P) debug_fail(status, kSiteOffsets);
+            if (counts[e] != b - a) debug_fail(status, kSiteCounts);
+            if (b > a) atomicAdd(&s_tiles, (unsigned long long)((b - a + tile_rows - 1) / tile_rows));
+        }
+        __syncthreads();
+        if (threadIdx.x == 0 && (int64_t)s_tiles != (int64_t)tile_prefix[E]) debug_fail(status, kSiteTilePrefix);
+    }
+    const int64_t n = min(max((int64_t)offsets[E], (int64_t)0), P);   // grouped rows
+    int64_t nt = tile_prefix[E];
+    if (nt < 0 || nt > n_sched) {
+        if (blockIdx.x == 0 && threadIdx.x == 0) debug_fail(status, kSiteTilePrefix);
+        nt = nt < 0 ? 0 : n_sched;
+    }
+    const int64_t i0 = (int64_t)blockIdx.x * blockDim.x + threadIdx.x, stride = (int64_t)gridDim.x * blockDim.x;
+    for (int64_t m = i0; m < nt; m += stride) {   // m-tile entries
+        const int4 v = sched[m];
+        if (v.x < 0 || v.x >= E) {
+            debug_fail(status, kSiteSchedule);
+            continue;
+        }
+        const int64_t a = offsets[v.x], b = offsets[v.x + 1];
+        if (v.y < a || v.z < 1 || v.z > tile_rows || (int64_t)v.y + v.z > b || (v.y - a) % tile_rows != 0)
+            debug_fail(status, kSiteSchedule);
+    }
+    for (int64_t r = i0; r < n; r += stride) {   // grouped row -> pair of the row's expert
+        const int64_t pid = perm[r];
+        if (pid < 0 || pid >= P) {
+            debug_fail(status, kSitePerm);
+            continue;
+        }
+        const int e = idx[pid];
+        if (e < 0 || e >= E || r < offsets[e] || r >= offsets[e + 1]) debug_fail(status, kSitePerm);
+        if (inv_perm[pid] != r) debug_fail(status, kSiteInvPerm);
+    }
+    for (int64_t pid = i0; pid < P; pid += stride) {   // pair -> its grouped row, -1 for a dropped pair
+        const int64_t r = inv_perm[pid];
+        const int e = idx[pid];
+        if (e >= 0 && e < E) {
+            if (r < 0 || r >= n || perm[r] != pid) debug_fail(status, kSiteInvPerm);
+        } else if (r != -1) {
+            debug_fail(status, kSiteInvPerm);
+        }
     }
 }
 
@@ -311,7 +410,8 @@ cudaError_t launch_gather_rows(const __nv_bfloat16* src, const int32_t* perm, co
     if (P == 0) return cudaSuccess;
     timing_begin(KK_GATHER, st);
     const cudaError_t err =
-        launch_chained(gather_rows_kernel, capped_grid((P * 32 + 255) / 256), 256, st, src, perm, nrows, k, P, H, dst);
+        launch_chained(gather_rows_kernel, capped_grid((P * 32 + 255) / 256), 256, st, src, perm, nrows, k, P, H, dst,
+                       device_status_ptr());
     timing_end(KK_GATHER, st);
     count_launch();
     return err;
@@ -322,8 +422,20 @@ cudaError_t launch_combine(const __nv_bfloat16* rows, const int32_t* inv_perm, i
     const int64_t n = T * (H / 8);
     if (n == 0) return cudaSuccess;
     timing_begin(KK_COMBINE, st);
-    combine_kernel<<<capped_grid((n + 255) / 256), 256, 0, st>>>(rows, inv_perm, k, T, H, y);
+    combine_kernel<<<capped_grid((n + 255) / 256), 256, 0, st>>>(rows, inv_perm, k, T, H, y, device_status_ptr());
     timing_end(KK_COMBINE, st);
+    count_launch();
+    return cudaGetLastError();
+}
+
+cudaError_t launch_validate_schedule(const int32_t* idx, int64_t P, int E, int tile_rows, const int32_t* counts,
+                                     const int32_t* offsets, const int32_t* tile_prefix, const int4* sched,
+                                     int64_t n_sched, const int32_t* perm, const int32_t* inv_perm, cudaStream_t st) {
+    uint32_t* status = device_status_ptr();
+    if (!status) return cudaErrorUnknown;
+    const int grid = capped_grid((std::max<int64_t>(std::max<int64_t>(P, n_sched), E) + 255) / 256);
+    validate_schedule_kernel<<<grid, 256, 0, st>>>(idx, P, E, tile_rows, counts, offsets, tile_prefix, sched, n_sched,
+                                                   perm, inv_perm, status);
     count_launch();
     return cudaGetLastError();
 }

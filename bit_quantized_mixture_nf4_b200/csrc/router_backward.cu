@@ -35,7 +35,7 @@ __global__ void __launch_bounds__(256) router_grad_kernel(const __nv_bfloat16* _
                                                           const float* __restrict__ wts,
                                                           const float* __restrict__ logits, int64_t T, int E,
                                                           int k, int H, int renorm, float* __restrict__ dw_out,
-                                                          float* __restrict__ dl_out) {
+                                                          float* __restrict__ dl_out, uint32_t* __restrict__ status) {
     const int lane = threadIdx.x & 31;
     const int64_t t = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
     if (t >= T) return;
@@ -48,10 +48,16 @@ __global__ void __launch_bounds__(256) router_grad_kernel(const __nv_bfloat16* _
         if (j >= k) continue;
         const int64_t p = t * k + j;
         const int e = __ldg(idx + p);
-        const bool valid = e >= 0 && e < E;
+        bool valid = e >= 0 && e < E;
         float acc = 0.0f;
+        const int64_t r = valid ? __ldg(inv_perm + p) : -1;
+#if E4B_DEBUG_CHECKS
+        if (valid && (r < 0 || r >= T * k)) {   // a routed pair has a grouped row
+            if (lane == 0) debug_fail(status, kSiteRouterInv);
+            valid = false;
+        }
+#endif
         if (valid) {
-            const int64_t r = __ldg(inv_perm + p);
             const uint4* g4 = reinterpret_cast<const uint4*>(grad_out + t * H);
             if (FROM_PARTS) {
                 for (int c = lane; c < n_parts; c += 32) acc += __ldcs(parts + r * n_parts + c);
@@ -153,7 +159,8 @@ cudaError_t launch_router_grad(const __nv_bfloat16* grad_out, const __nv_bfloat1
     if (T == 0) return cudaSuccess;
     const int64_t grid = (T * 32 + 255) / 256;
     router_grad_kernel<false><<<(unsigned)grid, 256, 0, st>>>(grad_out, Y, nullptr, 0, nullptr, inv_perm, idx, wts,
-                                                              logits, T, E, k, H, renorm, dw, dlogits);
+                                                              logits, T, E, k, H, renorm, dw, dlogits,
+                                                              device_status_ptr());
     count_launch();
     return cudaGetLastError();
 }
@@ -165,7 +172,8 @@ cudaError_t launch_router_grad_parts(const __nv_bfloat16* grad_out, const float*
     if (T == 0) return cudaSuccess;
     const int64_t grid = (T * 32 + 255) / 256;
     router_grad_kernel<true><<<(unsigned)grid, 256, 0, st>>>(grad_out, nullptr, parts, n_parts, down_bias, inv_perm,
-                                                             idx, wts, logits, T, E, k, H, renorm, dw, dlogits);
+                                                             idx, wts, logits, T, E, k, H, renorm, dw, dlogits,
+                                                             device_status_ptr());
     count_launch();
     return cudaGetLastError();
 }

@@ -57,7 +57,8 @@ typedef enum {
     E4B_ERR_UNSUPPORTED = 3,   /* valid request outside what the kernels implement       */
     E4B_ERR_WORKSPACE = 4,     /* workspace NULL or smaller than e4b_moe_workspace_size  */
     E4B_ERR_CUDA = 5,          /* a CUDA runtime call or launch failed                    */
-    E4B_ERR_TIMEOUT = 6        /* a device-side wait hit its time limit                   */
+    E4B_ERR_TIMEOUT = 6,       /* a device-side wait hit its time limit                   */
+    E4B_ERR_DEBUG_CHECK = 7    /* a debug-build bounds or consistency check failed        */
 } e4b_status;
 
 /* NF4 / FP4: 64-element blocks with an fp32 absmax (the 4-bit stacks above).
@@ -371,8 +372,45 @@ E4B_API void e4b_pipe_destroy(e4b_pipe *p);
 
 /* Synchronizes `stream`, then reads and clears the library's device status
  * word: E4B_OK, or E4B_ERR_TIMEOUT if a kernel gave up on a wait since the last
- * call.  E4B_ERR_CUDA if the synchronization itself fails. */
+ * call, or else E4B_ERR_DEBUG_CHECK if a check of the debug build failed.
+ * E4B_ERR_CUDA if the synchronization itself fails. */
 E4B_API e4b_status e4b_device_status(void *stream);
+
+/* The raw status word the last e4b_device_status call read (0 when it returned
+ * E4B_OK): bit 0 timeout, bit 1 debug check, bits 8..15 the first failing check's
+ * site.  Sites: 1 grouped-GEMM m-tile entry, 2 grouped-GEMM pair id, 3 row-gather
+ * pair id, 4 combine inverse-permutation entry, 5 routing-gradient
+ * inverse-permutation entry, 6 expert offsets, 7 expert counts, 8 m-tile total,
+ * 9 m-tile entry against its expert's rows, 10 perm entry, 11 inv_perm entry. */
+E4B_API uint32_t e4b_last_status_word(void);
+
+/* 1 in the debug build (libe4b_debug.so, compiled with E4B_DEBUG_CHECKS=1), else 0.
+ * The debug build checks, on the device, every m-tile entry and pair id the
+ * grouped GEMMs use, the pair ids of the row gather, the inverse-permutation
+ * entries of the combine and the routing gradient, and, after every grouping, the
+ * whole schedule (e4b_debug_validate_schedule).  A failed check records its site
+ * in the status word and skips the access it guards; nothing traps.  This is the
+ * stand-in for a memory checker on the expert layer's pages' "fails loudly"
+ * contract (bitsandbytes PR #1965, "Correctness & coverage").  Release builds
+ * compile the checks out. */
+E4B_API int e4b_debug_checks(void);
+
+/* Diagnostic, in every build: checks a grouping schedule on the device.  Given the
+ * routing topk_idx [P] (P = T * top_k pairs), E experts and the m-tile height
+ * tile_rows, the schedule is counts [E], offsets [E+1] (expert e owns the grouped
+ * rows [offsets[e], offsets[e+1])), tile_prefix [E+1] (tile_prefix[E] = number of
+ * m-tiles), sched [n_sched][4] int32 m-tile entries (expert, first row, rows, 0),
+ * perm [P] (pair id of each grouped row) and inv_perm [P] (grouped row of each pair,
+ * -1 for a pair whose expert is outside [0, E)).  All pointers are device memory
+ * the caller owns.  Every value read is range-checked before it serves as an index.
+ * Returns E4B_OK for a consistent schedule; E4B_ERR_DEBUG_CHECK otherwise, with the
+ * first failing property in e4b_last_status_word (sites 6-11); an earlier kernel's
+ * pending error is returned first.  E4B_ERR_INVALID_ARG for null pointers, P <= 0,
+ * E outside 1..256, tile_rows <= 0 or n_sched < 0.  Synchronizes `stream`. */
+E4B_API e4b_status e4b_debug_validate_schedule(const int32_t *topk_idx, int64_t P, int E, int tile_rows,
+                                               const int32_t *counts, const int32_t *offsets,
+                                               const int32_t *tile_prefix, const int32_t *sched, int64_t n_sched,
+                                               const int32_t *perm, const int32_t *inv_perm, void *stream);
 
 /* Diagnostic: launches one kernel whose single thread waits, through the same
  * bounded mbarrier wait every pipelined kernel uses, on a barrier nothing

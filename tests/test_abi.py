@@ -37,9 +37,35 @@ def test_library_exports_every_declared_symbol(lib):
     assert set(declared_functions()) == set(lib.EXPORTS)
 
 
+def test_debug_build_exports_the_same_symbols_and_says_so(lib):
+    """The debug-check build (E4B_DEBUG_CHECKS=1) has the same ABI; e4b_debug_checks
+    (a host-only query) tells the two apart."""
+    path = e4b_build.build(debug=True)
+    dbg = ctypes.CDLL(path)
+    for n in declared_functions():
+        assert hasattr(dbg, n), n
+    dbg.e4b_debug_checks.restype = ctypes.c_int
+    rel = ctypes.CDLL(e4b_build.LIB)
+    rel.e4b_debug_checks.restype = ctypes.c_int
+    assert dbg.e4b_debug_checks() == 1
+    assert rel.e4b_debug_checks() == 0
+
+
 def test_status_strings(lib):
-    for s in range(7):
+    for s in range(8):
         assert lib.e4b_status_string(s)
+    assert lib.e4b_status_string(lib.E4B_ERR_DEBUG_CHECK) != lib.e4b_status_string(99)
+
+
+def test_validate_schedule_rejects_bad_arguments_on_the_host(lib):
+    L = lib.lib
+    f = lambda P, E, tr, n: L.e4b_debug_validate_schedule(16, P, E, tr, 16, 16, 16, 16, n, 16, 16, None)
+    assert f(0, 4, 256, 1) == lib.E4B_ERR_INVALID_ARG
+    assert f(8, 0, 256, 1) == lib.E4B_ERR_INVALID_ARG
+    assert f(8, 257, 256, 1) == lib.E4B_ERR_INVALID_ARG
+    assert f(8, 4, 0, 1) == lib.E4B_ERR_INVALID_ARG
+    assert f(8, 4, 256, -1) == lib.E4B_ERR_INVALID_ARG
+    assert L.e4b_debug_validate_schedule(None, 8, 4, 256, 16, 16, 16, 16, 1, 16, 16, None) == lib.E4B_ERR_INVALID_ARG
 
 
 def test_host_side_validation(lib):
