@@ -135,7 +135,7 @@ static WsLayout layout_for(const e4b_moe_desc* d, int64_t T) {
     L.chunk_base = take((size_t)nch * d->E * 4);
     L.counts = take((size_t)d->E * 4);
     L.offsets = take((size_t)(d->E + 1) * 4);
-    L.tile_prefix = take((size_t)(d->E + 2) * 4);   // [E] all m-tiles, [E+1] the big ones
+    L.tile_prefix = take((size_t)(d->E + 1) * 4);
     L.sched = take(((size_t)(P + gemm_tile_rows() - 1) / gemm_tile_rows() + d->E) * 16);
     L.perm = take((size_t)P * 4);
     L.inv_perm = take((size_t)P * 4);

@@ -16,9 +16,8 @@ enum Epi { EPI_GATEUP = 0, EPI_DOWN = 1, EPI_DGRAD_DOWN = 2, EPI_DGRAD_GATEUP = 
 
 struct GemmParams {
     int E, K, N, n_tiles;
-    const int* tile_prefix;   // the grouping's m-tile counts: [E] = all m-tiles, [E+1] = big ones
-    const int4* sched;        // per m-tile: (expert, first row, rows, 0); the big tiles first, then
-                              // the tails of at most half a tile (the single-SM instance's)
+    const int* tile_prefix;   // [E+1] prefix of ceil(M_e / tile_rows); [E] = total m-tiles
+    const int4* sched;        // per m-tile: (expert, first row, rows, 0)
     const int* perm;          // [P] pair id of each grouped row
     const float* topk_w;      // [P] routing weight by pair id
     const float* absmax;      // absmax of the weight stack
@@ -96,9 +95,7 @@ constexpr int kChunkPairs = 256;   // pairs per grouping block (one per thread o
 cudaError_t launch_route(const float* logits, int64_t T, int E, int k, int renorm, int32_t* idx, float* w,
                          cudaStream_t st);
 // counts/offsets/tile_prefix/perm from topk_idx; chunk scratch: [nchunks * E] ints x2
-// sched: [ceil(P/tile_rows) + E] m-tile entries (expert, first row, rows, 0): the big
-// m-tiles (full ones and tails above tile_rows / 2), experts ascending, then the tails
-// of at most tile_rows / 2 rows; tile_prefix [E+2]: [E] = all m-tiles, [E+1] = big ones
+// sched: [ceil(P/tile_rows) + E] m-tile entries (expert, first row, rows, 0)
 // inv_perm[pair] = grouped row of the pair, -1 for a pair of an out-of-range expert
 cudaError_t launch_group(const int32_t* idx, int64_t P, int E, int tile_rows, int32_t* chunk_counts,
                          int32_t* chunk_base, int32_t* counts, int32_t* offsets, int32_t* tile_prefix,

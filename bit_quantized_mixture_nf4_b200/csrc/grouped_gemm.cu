@@ -93,17 +93,27 @@ static_assert(Cfg<1, EPI_GATEUP>::RINGS_BYTES % 1024 == 0 && Cfg<1, EPI_DGRAD_DO
 static_assert(Cfg<1, EPI_GATEUP>::SMEM_BYTES <= 232448 && Cfg<1, EPI_DGRAD_DOWN>::SMEM_BYTES <= 232448,
               "shared memory per block (single-SM tiles)");
 
-// Programmatic dependent launch: the pair launch lets the single-SM launch after it
-// start early; the single-SM launch waits for the pair launch before it completes.
-__device__ __forceinline__ void pdl_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;"); }
-__device__ __forceinline__ void pdl_wait_primary() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
-
 // TMA tensor store of a 32 x 32 bf16 box from shared memory, and its bulk-group
 // bookkeeping (issued and awaited by one thread).
+// The outputs stream through L2 once (the next kernel reads them from HBM at these
+// sizes), so the stores carry an evict-first policy: they do not push out the weight
+// columns and activation rows the neighbouring tiles are still reading.
+constexpr bool kStoreEvictFirst = true;
+__device__ __forceinline__ uint64_t l2_evict_first_policy() {
+    uint64_t pol;
+    asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
+    return pol;
+}
 __device__ __forceinline__ void tma_store_2d(const CUtensorMap* m, uint32_t src, int x, int y) {
-    asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];"
-                 ::"l"(reinterpret_cast<uint64_t>(m)), "r"(src), "r"(x), "r"(y)
-                 : "memory");
+    if (kStoreEvictFirst) {
+        asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group.L2::cache_hint [%0, {%2, %3}], [%1], %4;"
+                     ::"l"(reinterpret_cast<uint64_t>(m)), "r"(src), "r"(x), "r"(y), "l"(l2_evict_first_policy())
+                     : "memory");
+    } else {
+        asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];"
+                     ::"l"(reinterpret_cast<uint64_t>(m)), "r"(src), "r"(x), "r"(y)
+                     : "memory");
+    }
 }
 __device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
 template <int N>
@@ -131,20 +141,51 @@ struct TileInfo {
     int e, row0, rows, nt;
 };
 
-// One load: the m-tile schedule written by the grouping scan (sched: this instance's
-// part of it; max_rows: its tile height).  Debug builds check the entry; a bad one
-// becomes an empty tile of expert 0 (every role of the CTA decodes the same entry, so
-// they all skip it alike).
+// Tile order.  Tiles are numbered expert by expert.  Inside an expert, its n-tiles
+// go in groups of kTileGroup; inside a group, the expert's m-tiles are the outer
+// loop and the group's n-tiles the inner one.  The tiles that run at the same time
+// on neighbouring clusters then share one group of weight columns (re-read from L2
+// by every m-tile of the expert) and a few m-tiles of activation rows, instead of
+// sweeping all of the expert's weights once per m-tile.  16 measured best on the
+// Mixtral shape (HBM reads of the gate_up GEMM 4.3 -> 1.8 GB per launch; 8 re-reads
+// the long activation rows of the K = 14336 and 28672 GEMMs); where an expert has
+// at most 16 n-tiles this is the plain (m-tile, n-tile) order.
+constexpr int kTileGroup = 16;
+
+// Tile -> (m-tile entry of the grouping scan's schedule, n-tile); one schedule load.
+// max_rows: the tile height.  Debug builds check the entry; a bad one becomes an
+// empty tile of expert 0 (every role of the CTA decodes the same entry, so they all
+// skip it alike).
 __device__ __forceinline__ TileInfo decode_tile(const GemmParams& p, const int4* sched, int tile, int max_rows) {
-    const int mt = tile / p.n_tiles;
-    const int4 v = __ldg(sched + mt);
+    const int n = p.n_tiles;
+    const int mt_tile = tile / n;   // m-tile that the plain (m, n) order would give: locates the expert
+    int lo = 0, hi = p.E;           // the last expert whose first m-tile is at or before mt_tile
+    while (hi - lo > 1) {
+        const int mid = (lo + hi) >> 1;
+        if (__ldg(p.tile_prefix + mid) <= mt_tile) lo = mid;
+        else hi = mid;
+    }
+    const int m0 = __ldg(p.tile_prefix + lo), me = __ldg(p.tile_prefix + lo + 1) - m0;
+    const int l = tile - m0 * n;    // the tile's index inside its expert: [0, me * n)
+    const int g = min(kTileGroup, n), full = n / g;
+    int m, nt;
+    if (l < full * g * me) {
+        const int grp = l / (g * me), r = l - grp * g * me;
+        m = r / g;
+        nt = grp * g + (r - m * g);
+    } else {                        // the last, narrower group
+        const int gw = n - full * g, r = l - full * g * me;
+        m = r / gw;
+        nt = full * g + (r - m * gw);
+    }
+    const int4 v = __ldg(sched + m0 + m);
 #if E4B_DEBUG_CHECKS
     if (v.x < 0 || v.x >= p.E || v.z < 1 || v.z > max_rows || v.y < 0 || (int64_t)v.y + v.z > p.a_rows) {
         debug_fail(p.status, kSiteGemmTile);
-        return TileInfo{0, 0, 0, tile - mt * p.n_tiles};
+        return TileInfo{0, 0, 0, nt};
     }
 #endif
-    return TileInfo{v.x, v.y, v.z, tile - mt * p.n_tiles};
+    return TileInfo{v.x, v.y, v.z, nt};
 }
 
 // Stored weight row (within one expert) feeding B column `n` (0..255) of tile nt (K-major mode).
@@ -284,12 +325,8 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_con
         else mbar_arrive(smem_u32(bar));
     };
 
-    // This instance's m-tiles: the big ones (cta_group::2 pairs) or the small tails
-    // (single SMs), which follow the big ones in the schedule.
-    const int n_big = __ldg(p.tile_prefix + p.E + 1);
-    const int4* sched = p.sched + (CTAS == 2 ? 0 : n_big);
-    const int total_tiles = (CTAS == 2 ? n_big : __ldg(p.tile_prefix + p.E) - n_big) * p.n_tiles;
-    if (CTAS == 2) pdl_launch_dependents();   // the single-SM launch that follows may start as SMs free up
+    const int4* sched = p.sched;
+    const int total_tiles = __ldg(p.tile_prefix + p.E) * p.n_tiles;
     const int nk = p.K / BK;              // k-stages of the quantized weights
     const int nkt = nk + (p.lora_r > 0);  // plus the LoRA stage (the last one of a tile)
 
@@ -477,6 +514,40 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_con
                 if (!wait(&ctl->empty[s], (r & 1) ^ 1)) break;
                 const TileInfo ti = decode_tile(p, sched, cur_tile, C::TILE_M);
                 uint8_t* dst_tile = sB + s * C::B_BYTES;
+                if (CB == 3 && !lora_stage) {
+                    // bf16 weights: the group's first warp loads this CTA's part of the tile by
+                    // TMA (tmap_raw maps the bf16 stack, 128B-swizzled: the operand layout),
+                    // completing on the first CTA's barrier; the other warps only arrive.
+                    // Rows or columns outside the stack read as zero; those of a neighbouring
+                    // expert only feed output columns that are never stored.
+                    if (lane == 0) {
+                        if (tg == 0) {
+                            const uint32_t bar = smem_u32(&ctl->b_full[s]);
+                            if (leader) mbar_arrive_expect_tx(bar, CTAS * C::B_BYTES);
+                            else mbar_arrive_cluster(mapa_shared(bar, 0));
+                            const int ebase = ti.e * p.b_rows_per_expert;
+                            auto load = [&](uint32_t dst, int x, int y) {
+                                if (CTAS == 2) tma_load_2d_pair(dst, &tmap_raw, mapa_shared(bar, 0), x, y);
+                                else tma_load_2d(dst, &tmap_raw, bar, x, y);
+                            };
+                            if (kMajorB) {   // boxes of 128 stored rows x 64 k
+#pragma unroll
+                                for (int h = 0; h < C::N_CTA / 128; ++h)
+                                    load(smem_u32(dst_tile) + h * 16384, cur_ks * BK,
+                                         ebase + kmajor_row<EPI>(p, ti.nt, (int)rank * C::N_CTA + 128 * h));
+                            } else {         // boxes of 64 k-rows x 64 stored columns
+#pragma unroll
+                                for (int j = 0; j < C::N_CTA / 64; ++j)
+                                    load(smem_u32(dst_tile) + j * 8192, ti.nt * BN + (int)rank * C::N_CTA + 64 * j,
+                                         ebase + cur_ks * BK);
+                            }
+                        } else {
+                            arrive_leader(&ctl->b_full[s]);
+                        }
+                    }
+                    it += C::DEQ_GROUPS;
+                    continue;
+                }
 #pragma unroll
                 for (int i = 0; i < NB; ++i) {
                     const int b = tg + TPG * i;
@@ -923,10 +994,6 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_con
         if (CTAS == 2) tmem_dealloc_pair(tmem_base, TMEM_COLS);
         else tmem_dealloc(tmem_base, TMEM_COLS);
     }
-    // The single-SM launch may run beside the pair launch before it (programmatic
-    // dependent launch; they write disjoint rows): it completes only after that one
-    // has, so whatever follows in the stream sees both.
-    if (CTAS == 1) pdl_wait_primary();
 }
 
 // ------------------------------------------------------------------ host side
@@ -971,13 +1038,14 @@ static bool make_map_2d(CUtensorMap* m, CUtensorMapDataType dt, const void* base
               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// Rows of a big tile (a cta_group::2 pair on two SMs); tails of at most half of it
-// run as single-SM tiles.
-int gemm_tile_rows() { return Cfg<2>::TILE_M; }
+// CTAs per tile of the grouped GEMMs (2: cta_group::2 pairs on two SMs; the kernel
+// template also has a single-SM configuration, CTAS = 1, which is not launched).
+constexpr int kCtas = 2;
+int gemm_tile_rows() { return Cfg<kCtas>::TILE_M; }
 
 template <int EPI, int CB, int CTAS, bool XACT = false>
 static cudaError_t launch_one(const CUtensorMap& ma, const CUtensorMap& mr, const CUtensorMap& mo,
-                              const CUtensorMap& mg, const CUtensorMap& ml, const GemmParams& p, int grid, bool pdl,
+                              const CUtensorMap& mg, const CUtensorMap& ml, const GemmParams& p, int grid,
                               cudaStream_t st) {
     using C = Cfg<CTAS, EPI>;
     auto kern = grouped_gemm_kernel<EPI, CB, CTAS, XACT>;
@@ -1002,15 +1070,13 @@ static cudaError_t launch_one(const CUtensorMap& ma, const CUtensorMap& mr, cons
     cfg.blockDim = dim3(GEMM_THREADS);
     cfg.dynamicSmemBytes = C::SMEM_BYTES;
     cfg.stream = st;
-    cudaLaunchAttribute attr[2];
+    cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeClusterDimension;
     attr[0].val.clusterDim.x = CTAS;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
-    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = pdl ? 2 : 1;
+    cfg.numAttrs = 1;
     cudaError_t e = cudaLaunchKernelEx(&cfg, kern, ma, mr, mo, mg, ml, p);
     count_launch();
     if (e != cudaSuccess) return e;
@@ -1021,27 +1087,26 @@ static cudaError_t launch_one(const CUtensorMap& ma, const CUtensorMap& mr, cons
 // gate_up variant (clamped GLU or biases) and for the routing-gradient dot products.
 template <int CB, int CTAS>
 static cudaError_t launch_cb(int epi, const CUtensorMap& ma, const CUtensorMap& mr, const CUtensorMap& mo,
-                             const CUtensorMap& mg, const CUtensorMap& ml, const GemmParams& p, int grid, bool pdl,
+                             const CUtensorMap& mg, const CUtensorMap& ml, const GemmParams& p, int grid,
                              cudaStream_t st) {
     if (epi == EPI_GATEUP && (p.act != 0 || p.bias != nullptr))
-        return launch_one<EPI_GATEUP, CB, CTAS, true>(ma, mr, mo, mg, ml, p, grid, pdl, st);
+        return launch_one<EPI_GATEUP, CB, CTAS, true>(ma, mr, mo, mg, ml, p, grid, st);
     if (epi == EPI_DGRAD_DOWN && p.dw_part)
-        return launch_one<EPI_DGRAD_DOWN, CB, CTAS, true>(ma, mr, mo, mg, ml, p, grid, pdl, st);
+        return launch_one<EPI_DGRAD_DOWN, CB, CTAS, true>(ma, mr, mo, mg, ml, p, grid, st);
     switch (epi) {
-        case EPI_GATEUP: return launch_one<EPI_GATEUP, CB, CTAS>(ma, mr, mo, mg, ml, p, grid, pdl, st);
-        case EPI_DOWN: return launch_one<EPI_DOWN, CB, CTAS>(ma, mr, mo, mg, ml, p, grid, pdl, st);
-        case EPI_DGRAD_DOWN: return launch_one<EPI_DGRAD_DOWN, CB, CTAS>(ma, mr, mo, mg, ml, p, grid, pdl, st);
-        default: return launch_one<EPI_DGRAD_GATEUP, CB, CTAS>(ma, mr, mo, mg, ml, p, grid, pdl, st);
+        case EPI_GATEUP: return launch_one<EPI_GATEUP, CB, CTAS>(ma, mr, mo, mg, ml, p, grid, st);
+        case EPI_DOWN: return launch_one<EPI_DOWN, CB, CTAS>(ma, mr, mo, mg, ml, p, grid, st);
+        case EPI_DGRAD_DOWN: return launch_one<EPI_DGRAD_DOWN, CB, CTAS>(ma, mr, mo, mg, ml, p, grid, st);
+        default: return launch_one<EPI_DGRAD_GATEUP, CB, CTAS>(ma, mr, mo, mg, ml, p, grid, st);
     }
 }
 
-// One configuration: CTAS = 2 runs the big m-tiles (cta_group::2 pairs, 256 rows),
-// CTAS = 1 the small tails (one SM, 128 rows, the whole 256-column B tile dequantized
-// there).  max_tiles bounds the tiles the launch can find in its part of the schedule.
+// One launch of configuration CTAS over the whole m-tile schedule (max_tiles bounds
+// the tiles it can find there).
 template <int CTAS>
 static cudaError_t launch_cfg(int epi, int codebook, const void* a, int64_t a_rows, const uint8_t* packed,
                               int64_t packed_rows_total, int packed_row_bytes, const GemmParams& p, int64_t max_tiles,
-                              bool pdl, cudaStream_t st, const void* lora_a) {
+                              cudaStream_t st, const void* lora_a) {
     using C = Cfg<CTAS>;
     CUtensorMap ma, mr;
     if (!make_map_2d(&ma, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a, (uint64_t)p.K, (uint64_t)a_rows, (uint64_t)p.K * 2, 64,
@@ -1051,12 +1116,21 @@ static cudaError_t launch_cfg(int epi, int codebook, const void* a, int64_t a_ro
     // K-major: boxes of 128 rows x 32 bytes; MN-major: 64 k-rows x (N_CTA/2) bytes, swizzled so the
     // dequantizing threads read it without bank conflicts.
     const uint32_t mn_row = C::N_CTA / 2;
-    if (!make_map_2d(&mr, CU_TENSOR_MAP_DATA_TYPE_UINT8, packed, (uint64_t)packed_row_bytes,
-                     (uint64_t)packed_rows_total, (uint64_t)packed_row_bytes, kmaj ? BK / 2 : mn_row,
-                     kmaj ? 128 : BK,
-                     kmaj ? CU_TENSOR_MAP_SWIZZLE_NONE
-                          : (mn_row == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B)))
+    if (codebook == 3) {
+        // bf16 weights [b_rows_total, cols] (cols = K when K-major, N when MN-major): boxes
+        // of 64 columns (128 B, 128B swizzle: the UMMA operand layout) x 128 rows (K-major)
+        // or x 64 k-rows (MN-major)
+        const uint64_t cols = kmaj ? (uint64_t)p.K : (uint64_t)p.N;
+        if (!make_map_2d(&mr, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, p.bf16_b, cols, (uint64_t)p.b_rows_total, cols * 2,
+                         64, kmaj ? 128 : BK, CU_TENSOR_MAP_SWIZZLE_128B))
+            return cudaErrorInvalidValue;
+    } else if (!make_map_2d(&mr, CU_TENSOR_MAP_DATA_TYPE_UINT8, packed, (uint64_t)packed_row_bytes,
+                            (uint64_t)packed_rows_total, (uint64_t)packed_row_bytes, kmaj ? BK / 2 : mn_row,
+                            kmaj ? 128 : BK,
+                            kmaj ? CU_TENSOR_MAP_SWIZZLE_NONE
+                                 : (mn_row == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B))) {
         return cudaErrorInvalidValue;
+    }
     // epilogue outputs: 32 x 32 boxes, 64B-swizzled, of the [rows, ld_out] output (h, the
     // input-gradient halves or the per-pair rows) and of the saved derivatives [rows, 2I]
     CUtensorMap mo, mg;
@@ -1079,10 +1153,10 @@ static cudaError_t launch_cfg(int epi, int codebook, const void* a, int64_t a_ro
     const int grid = (int)std::min<int64_t>(max_tiles * CTAS, (num_sms() / CTAS) * CTAS);
     if (grid <= 0) return cudaSuccess;
     switch (codebook) {
-        case 0: return launch_cb<0, CTAS>(epi, ma, mr, mo, mg, ml, p, grid, pdl, st);
-        case 1: return launch_cb<1, CTAS>(epi, ma, mr, mo, mg, ml, p, grid, pdl, st);
-        case 2: return launch_cb<2, CTAS>(epi, ma, mr, mo, mg, ml, p, grid, pdl, st);
-        default: return launch_cb<3, CTAS>(epi, ma, mr, mo, mg, ml, p, grid, pdl, st);
+        case 0: return launch_cb<0, CTAS>(epi, ma, mr, mo, mg, ml, p, grid, st);
+        case 1: return launch_cb<1, CTAS>(epi, ma, mr, mo, mg, ml, p, grid, st);
+        case 2: return launch_cb<2, CTAS>(epi, ma, mr, mo, mg, ml, p, grid, st);
+        default: return launch_cb<3, CTAS>(epi, ma, mr, mo, mg, ml, p, grid, st);
     }
 }
 
@@ -1096,15 +1170,9 @@ cudaError_t launch_grouped_gemm(int epi, int codebook, const void* a, int64_t a_
         return cudaErrorInvalidValue;
     if (codebook == 3 && !p.bf16_b) return cudaErrorInvalidValue;
     if (max_m_tiles <= 0) return cudaSuccess;
-    // The big m-tiles on cta_group::2 pairs, then the small tails (at most one per
-    // expert) on single SMs, launched to start as the pairs' SMs free up.  One timing
-    // bracket covers both launches.
     timing_begin(KK_GEMM_GATEUP + epi, st);
-    cudaError_t e = launch_cfg<2>(epi, codebook, a, a_rows, packed, packed_rows_total, packed_row_bytes, p,
-                                  (int64_t)max_m_tiles * p.n_tiles, false, st, lora_a);
-    if (e == cudaSuccess)
-        e = launch_cfg<1>(epi, codebook, a, a_rows, packed, packed_rows_total, packed_row_bytes, p,
-                          (int64_t)std::min(p.E, max_m_tiles) * p.n_tiles, true, st, lora_a);
+    const cudaError_t e = launch_cfg<kCtas>(epi, codebook, a, a_rows, packed, packed_rows_total, packed_row_bytes, p,
+                                            (int64_t)max_m_tiles * p.n_tiles, st, lora_a);
     timing_end(KK_GEMM_GATEUP + epi, st);
     return e;
 }

@@ -80,13 +80,7 @@ __global__ void __launch_bounds__(1024) scan_kernel(const int32_t* __restrict__ 
                                                     int tile_rows, int32_t* __restrict__ chunk_base,
                                                     int32_t* __restrict__ counts, int32_t* __restrict__ offsets,
                                                     int32_t* __restrict__ tile_prefix, int4* __restrict__ sched) {
-    // An expert's rows make full m-tiles of tile_rows, then a tail.  A tail of more
-    // than half a tile is one more big tile; a tail of at most half a tile is a small
-    // tile, run by the single-SM instance of the grouped GEMMs.  The schedule lists
-    // all big tiles first (experts ascending), then the small ones:
-    // tile_prefix[E] = all m-tiles, tile_prefix[E + 1] = big m-tiles.
-    __shared__ int s_tot[256], s_off[256], s_toff[256], s_soff[257];
-    const int half = tile_rows / 2;
+    __shared__ int s_tot[256], s_off[256], s_toff[256];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
     chain_release();
     chain_wait();
@@ -98,30 +92,23 @@ __global__ void __launch_bounds__(1024) scan_kernel(const int32_t* __restrict__ 
         if (lane == 0) s_tot[e] = sum;
     }
     __syncthreads();
-    if (warp == 0) {   // exclusive scans of the row counts, big m-tiles and small tails over experts
-        int run = 0, trun = 0, srun = 0;
+    if (warp == 0) {   // exclusive scans of the row counts and m-tile counts over experts
+        int run = 0, trun = 0;
         for (int e0 = 0; e0 < E; e0 += 32) {
             const int e = e0 + lane;
             const int v = e < E ? s_tot[e] : 0;
-            const int rem = v % tile_rows;
-            const int tv = v / tile_rows + (rem > half ? 1 : 0);
-            const int sv = (rem > 0 && rem <= half) ? 1 : 0;
+            const int tv = (v + tile_rows - 1) / tile_rows;
             const int x = warp_inclusive_scan(v, lane), tx = warp_inclusive_scan(tv, lane);
-            const int sx = warp_inclusive_scan(sv, lane);
             if (e < E) {
                 s_off[e] = run + x - v;
                 s_toff[e] = trun + tx - tv;
-                s_soff[e] = srun + sx - sv;
             }
             run += __shfl_sync(0xffffffffu, x, 31);
             trun += __shfl_sync(0xffffffffu, tx, 31);
-            srun += __shfl_sync(0xffffffffu, sx, 31);
         }
         if (lane == 0) {
             offsets[E] = run;
-            tile_prefix[E] = trun + srun;
-            tile_prefix[E + 1] = trun;
-            s_soff[E] = trun;   // first small entry
+            tile_prefix[E] = trun;
         }
     }
     __syncthreads();
@@ -142,13 +129,10 @@ __global__ void __launch_bounds__(1024) scan_kernel(const int32_t* __restrict__ 
             offsets[e] = off;
             tile_prefix[e] = toff;
         }
-        // m-tile schedule: (expert, first row, rows) of every m-tile
-        const int rem = tot % tile_rows, full = tot / tile_rows;
-        const int nt = full + (rem > half ? 1 : 0);
+        // m-tile schedule: (expert, first row, rows) of every m-tile, experts ascending
+        const int nt = (tot + tile_rows - 1) / tile_rows;
         for (int m = lane; m < nt; m += 32)
             sched[toff + m] = make_int4(e, off + m * tile_rows, min(tile_rows, tot - m * tile_rows), 0);
-        if (lane == 0 && rem > 0 && rem <= half)
-            sched[s_soff[E] + s_soff[e]] = make_int4(e, off + full * tile_rows, rem, 0);
     }
 }
 
