@@ -44,18 +44,23 @@ __device__ __forceinline__ void cp16z(uint32_t dst, const void* src, uint32_t sr
 }
 __device__ __forceinline__ void cp_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
 __device__ __forceinline__ void cp_wait1() { asm volatile("cp.async.wait_group 1;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
 
-constexpr int THIN_ROWS = 256, THIN_SA = 72;   // rows per CTA (8 warps x 32); smem row stride (bf16)
-constexpr int THIN_SMEM = 2 * (THIN_ROWS + 64) * THIN_SA * 2;
+constexpr int THIN_ROWS = 128, THIN_SA = 72;   // rows per CTA (8 warps x 16); smem row stride (bf16)
+constexpr int THIN_STAGES = 4;                 // K chunks in the cp.async ring (3 in flight)
+constexpr int THIN_SMEM = THIN_STAGES * (THIN_ROWS + 64) * THIN_SA * 2;
 constexpr int GR_P = 32, GR_A = 128, GR_SU = GR_A + 8, GR_SV = 72;   // rows per chunk, columns per CTA
 
 }  // namespace
 
-// out[row, q] = s * sum_k in[row, k] * M_e(q, k) for the rows of one m-tile (one
-// expert, up to 256 rows), q < r; columns r..63 of out are zero.  M_e(q, k) =
-// m[e][q][k] (Q_MAJOR, an A adapter [E, r, K]) or m[e][k][q] (a B adapter
-// [E, K, r]).  K in chunks of 64, double-buffered: the rows' chunk and M_e's
-// chunk as [q][k] in shared memory; warp w owns rows 32w..32w+31 (two m16 tiles).
+// out[row, q] = s * sum_k in[row, k] * M_e(q, k) for the rows of half an m-tile
+// (one expert, up to 128 of the m-tile's up to 256 rows; block 2 mt + h takes half h
+// of m-tile mt), q < r; columns r..63 of out are zero.  M_e(q, k) = m[e][q][k]
+// (Q_MAJOR, an A adapter [E, r, K]) or m[e][k][q] (a B adapter [E, K, r]).  K in
+// chunks of 64 through a 4-deep cp.async ring (three chunks in flight: the kernel
+// streams its rows from HBM once), the rows' chunk and M_e's chunk as [q][k] in
+// shared memory; warp w owns rows 16w..16w+15 (one m16 tile).
 template <bool Q_MAJOR>
 __global__ void __launch_bounds__(256) lora_thin_kernel(const __nv_bfloat16* __restrict__ in, int K,
                                                         const __nv_bfloat16* __restrict__ m, int r, float s,
@@ -63,13 +68,14 @@ __global__ void __launch_bounds__(256) lora_thin_kernel(const __nv_bfloat16* __r
                                                         const int* __restrict__ tile_prefix, int E,
                                                         __nv_bfloat16* __restrict__ out) {
     extern __shared__ __align__(16) uint8_t sm[];
-    const int mt = blockIdx.x;
+    const int mt = blockIdx.x >> 1, half = blockIdx.x & 1;
     if (mt >= __ldg(tile_prefix + E)) return;
     const int4 tl = __ldg(sched + mt);   // (expert, first row, rows, 0)
-    const int e = tl.x, row0 = tl.y, rows = tl.z;
+    const int e = tl.x, row0 = tl.y + THIN_ROWS * half, rows = min(tl.z - THIN_ROWS * half, THIN_ROWS);
+    if (rows <= 0) return;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    __nv_bfloat16* sA = reinterpret_cast<__nv_bfloat16*>(sm);                 // [2][256][72]
-    __nv_bfloat16* sM = sA + 2 * THIN_ROWS * THIN_SA;                         // [2][64][72]
+    __nv_bfloat16* sA = reinterpret_cast<__nv_bfloat16*>(sm);                 // [STAGES][128][72]
+    __nv_bfloat16* sM = sA + THIN_STAGES * THIN_ROWS * THIN_SA;               // [STAGES][64][72]
     const __nv_bfloat16* me = m + (int64_t)e * r * K;
     const int nch = K / 64;
     auto stage = [&](int c, int b) {
@@ -100,51 +106,48 @@ __global__ void __launch_bounds__(256) lora_thin_kernel(const __nv_bfloat16* __r
         }
         cp_commit();
     };
-    float acc[2][8][4];
+    float acc[8][4];
 #pragma unroll
-    for (int i = 0; i < 2; ++i)
-#pragma unroll
-        for (int j = 0; j < 8; ++j) acc[i][j][0] = acc[i][j][1] = acc[i][j][2] = acc[i][j][3] = 0.0f;
+    for (int j = 0; j < 8; ++j) acc[j][0] = acc[j][1] = acc[j][2] = acc[j][3] = 0.0f;
     const int nt_n = r / 8;
-    stage(0, 0);
-    for (int c = 0; c < nch; ++c) {
-        if (c + 1 < nch) stage(c + 1, (c + 1) & 1);
+#pragma unroll
+    for (int c = 0; c < THIN_STAGES - 1; ++c) {   // prologue: chunks 0 .. STAGES-2 in flight
+        if (c < nch) stage(c, c);
         else cp_commit();
-        cp_wait1();
-        __syncthreads();
-        const __nv_bfloat16* a = sA + (c & 1) * THIN_ROWS * THIN_SA;
-        const __nv_bfloat16* mm = sM + (c & 1) * 64 * THIN_SA;
+    }
+    for (int c = 0; c < nch; ++c) {
+        const int cn = c + THIN_STAGES - 1;
+        if (cn < nch) stage(cn, cn % THIN_STAGES);   // its slot was read in iteration c - 1
+        else cp_commit();
+        cp_wait<THIN_STAGES - 1>();                   // chunk c has landed (this thread's part)
+        __syncthreads();                              // ... and everyone's
+        const __nv_bfloat16* a = sA + (c % THIN_STAGES) * THIN_ROWS * THIN_SA;
+        const __nv_bfloat16* mm = sM + (c % THIN_STAGES) * 64 * THIN_SA;
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk) {
-            uint32_t af[2][4];
-#pragma unroll
-            for (int t = 0; t < 2; ++t)
-                ldsm_x4(af[t], smem_u32(a + (32 * warp + 16 * t + (lane & 15)) * THIN_SA + kk * 16 + (lane >> 4) * 8));
+            uint32_t af[4];
+            ldsm_x4(af, smem_u32(a + (16 * warp + (lane & 15)) * THIN_SA + kk * 16 + (lane >> 4) * 8));
 #pragma unroll
             for (int nt = 0; nt < 8; ++nt) {
                 if (nt >= nt_n) break;
                 uint32_t b0, b1;
                 ldsm_x2(b0, b1, smem_u32(mm + (8 * nt + (lane & 7)) * THIN_SA + kk * 16 + ((lane >> 3) & 1) * 8));
-                mma16816(acc[0][nt], af[0], b0, b1);
-                mma16816(acc[1][nt], af[1], b0, b1);
+                mma16816(acc[nt], af, b0, b1);
             }
         }
-        __syncthreads();
+        __syncthreads();                              // slot c % STAGES is free for chunk c + STAGES
     }
     const int g = lane >> 2, c2 = (lane & 3) * 2;
 #pragma unroll
-    for (int t = 0; t < 2; ++t) {
+    for (int h = 0; h < 2; ++h) {
+        const int rr = 16 * warp + g + 8 * h;
+        if (rr >= rows) continue;
+        uint32_t* o = reinterpret_cast<uint32_t*>(out + (int64_t)(row0 + rr) * 64);
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {
-            const int rr = 32 * warp + 16 * t + g + 8 * h;
-            if (rr >= rows) continue;
-            uint32_t* o = reinterpret_cast<uint32_t*>(out + (int64_t)(row0 + rr) * 64);
-#pragma unroll
-            for (int nt = 0; nt < 8; ++nt) {
-                const float v0 = nt < nt_n ? s * acc[t][nt][2 * h] : 0.0f;
-                const float v1 = nt < nt_n ? s * acc[t][nt][2 * h + 1] : 0.0f;
-                o[(8 * nt + c2) >> 1] = pack_bf16x2(v0, v1);
-            }
+        for (int nt = 0; nt < 8; ++nt) {
+            const float v0 = nt < nt_n ? s * acc[nt][2 * h] : 0.0f;
+            const float v1 = nt < nt_n ? s * acc[nt][2 * h + 1] : 0.0f;
+            o[(8 * nt + c2) >> 1] = pack_bf16x2(v0, v1);
         }
     }
 }
@@ -287,9 +290,9 @@ cudaError_t launch_lora_thin(const __nv_bfloat16* in, int K, const __nv_bfloat16
         }
     }
     if (m_q_major)
-        lora_thin_kernel<true><<<max_m_tiles, 256, THIN_SMEM, st>>>(in, K, m, r, s, sched, tile_prefix, E, out);
+        lora_thin_kernel<true><<<2 * max_m_tiles, 256, THIN_SMEM, st>>>(in, K, m, r, s, sched, tile_prefix, E, out);
     else
-        lora_thin_kernel<false><<<max_m_tiles, 256, THIN_SMEM, st>>>(in, K, m, r, s, sched, tile_prefix, E, out);
+        lora_thin_kernel<false><<<2 * max_m_tiles, 256, THIN_SMEM, st>>>(in, K, m, r, s, sched, tile_prefix, E, out);
     count_launch();
     return cudaGetLastError();
 }
