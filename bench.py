@@ -342,6 +342,16 @@ def timed_steps(layer, steps, warmup, flush, stream, clk=None, kinds=tuple(GEMM_
     return ms, kernels, launches
 
 
+def roofline_peak(loop_ms, burst, sustained, source):
+    """(peak TFLOP/s, description) for GEMMs timed inside a step loop of loop_ms.  A
+    loop that runs for a quarter of a second or more runs under the board's power cap,
+    so the sustained dense-bf16 figure is the denominator there; a short loop (or no
+    sustained figure) uses the burst one."""
+    if sustained is not None and loop_ms >= 250.0:
+        return sustained, f"{source} bf16 dense (sustained): timed inside a {loop_ms / 1e3:.2f} s step loop"
+    return burst, f"{source} bf16 dense (burst)"
+
+
 def gemm_roofline(w, kernels, bf16, peak_kind, bf16_burst=None):
     """The dominant grouped GEMM (largest total time) against the dense-bf16 peak `bf16`
     (the burst figure, or the sustained one for kernels timed inside a long step loop;
@@ -863,12 +873,7 @@ def run_e4b(args, w):
     total_ms = max_over_ranks(sum(step_ms), dev)
     ms_per_step = total_ms / args.steps
     value = job_throughput(w.T, world, ms_per_step)
-    # The GEMMs are timed inside the step loop.  A loop that runs for a quarter of a
-    # second or more runs under the board's power cap, so the sustained dense-bf16
-    # figure is the denominator there; a short loop uses the burst figure.
-    long_loop = total_ms >= 250.0 and bf16_sus is not None
-    peak, peak_kind = ((bf16_sus, f"{peak_src} bf16 dense (sustained): timed inside a {total_ms / 1e3:.2f} s step loop")
-                       if long_loop else (bf16_burst, f"{peak_src} bf16 dense (burst)"))
+    peak, peak_kind = roofline_peak(total_ms, bf16_burst, bf16_sus, peak_src)
     roof, per_kernel = gemm_roofline(w, kernels, peak, peak_kind, bf16_burst)
     roof["traffic"] = recorded_traffic(roof["kernel"], f"{w.name}_T{w.T}")
     step_tf = 12 * w.H * w.I * w.P / (ms_per_step / 1e3) / 1e12
